@@ -1,0 +1,181 @@
+/*
+ * pa_oracle.c -- plain fp64 CPU oracle for paged decode attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, loads or
+ * calls this file; only the test-suite, the smoke check and the CPU-baseline
+ * leg of the benchmark do.  It shares no code, header or constant with the
+ * CUDA path.
+ *
+ * What it computes (sources are the three web pages the method is taken from):
+ *
+ *   - Cache layout and address of one key/value row.  The pseudocode kernel on
+ *     "KV Cache memory optimisation and PagedAttention" (yunthe.com), section
+ *     "PagedAttention注意力计算流程", reads element (head h, token in physical
+ *     block pb at offset off) at  h*head_dim + (pb*block_size + off)*num_heads*head_dim,
+ *     i.e. a cache laid out as [num_blocks, block_size, num_heads, head_dim].
+ *   - Logical -> physical mapping.  Same pseudocode, and "vLLM source first look:
+ *     PagedAttention memory design" (trdm.cn), section 二, BlockTable.get_physical_block
+ *     and get_offset: logical block i // block_size, offset i % block_size, physical
+ *     block = block_table[logical block].
+ *   - The attention itself.  The pseudocode computes score = dot(q, k) * scale and
+ *     elides "softmax and weighted sum"; the oracle writes out textbook softmax
+ *     attention over the gathered, contiguous K/V rows.
+ *   - Sliding window.  "KV Cache optimisation strategies in deployment"
+ *     (yunthe.com), section "Sliding Window Attention控制长序列显存": only the most
+ *     recent W tokens take part.  Reading: tokens [max(0, ctx - W), ctx), the current
+ *     token included; window <= 0 means full attention.
+ *   - INT8 cache.  Same page, section "量化压缩KV Cache的INT8与FP8方案", names an
+ *     INT8 KV cache but not its scheme.  Reading: one fp16 scale per (token, head)
+ *     row, value = int8 code * scale, both converted to fp64 exactly.
+ *
+ * Steps, in the order the pages give them, per (sequence s, head h):
+ *   1. lo = window > 0 ? max(0, ctx - window) : 0.
+ *   2. Gather K and V rows of logical tokens lo..ctx-1 through the block table into
+ *      contiguous fp64 arrays Kc[n][D], Vc[n][D]  (n = ctx - lo).
+ *   3. score_i = scale * sum_d q[d] * Kc[i][d].
+ *   4. m = max_i score_i;  p_i = exp(score_i - m) / sum_j exp(score_j - m).
+ *   5. out[d] = sum_i p_i * Vc[i][d].
+ *   ctx == 0 (nothing to attend): out = 0.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { ORC_F32 = 0, ORC_F16 = 1, ORC_BF16 = 2, ORC_I8 = 3 };
+
+enum {
+  ORC_OK = 0,
+  ORC_BAD_ARG = 1,
+  ORC_BAD_TABLE = 2,   /* a block-table entry outside [0, num_blocks) */
+  ORC_BAD_CONTEXT = 3, /* context_len < 0 or > max_blocks_per_seq * block_size */
+  ORC_NO_MEMORY = 4
+};
+
+/* IEEE-754 binary16 -> double, exactly (every binary16 value is a double). */
+double orc_f16_to_f64(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int exponent = (h >> 10) & 0x1f;
+  int mantissa = h & 0x3ff;
+  double v;
+  if (exponent == 0) {
+    v = ldexp((double)mantissa, -24); /* subnormal: mantissa * 2^-24 */
+  } else if (exponent == 31) {
+    v = mantissa ? NAN : INFINITY;
+  } else {
+    v = ldexp((double)(mantissa | 0x400), exponent - 25); /* 1.m * 2^(e-15) */
+  }
+  return sign ? -v : v;
+}
+
+/* bfloat16 is the upper half of an IEEE binary32; widen, then convert exactly. */
+double orc_bf16_to_f64(uint16_t b) {
+  uint32_t bits = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &bits, sizeof f);
+  return (double)f;
+}
+
+static double load_value(const void* base, int dtype, size_t index) {
+  switch (dtype) {
+    case ORC_F32: return (double)((const float*)base)[index];
+    case ORC_F16: return orc_f16_to_f64(((const uint16_t*)base)[index]);
+    case ORC_BF16: return orc_bf16_to_f64(((const uint16_t*)base)[index]);
+    case ORC_I8: return (double)((const int8_t*)base)[index];
+    default: return NAN;
+  }
+}
+
+/*
+ * Paged decode attention, one query token per sequence.
+ *
+ *   out          [S, H, D] fp64, written
+ *   q            [S, H, D] in q_dtype (F32 / F16 / BF16)
+ *   k_cache,     [NB, bs, H, D] in cache_dtype (F32 / F16 / BF16 / I8)
+ *   v_cache
+ *   k_scale,     [NB, bs, H] binary16 bit patterns; required for I8, ignored otherwise
+ *   v_scale
+ *   block_tables [S, MB] int32; only entries of blocks that hold attended tokens are read
+ *   context_lens [S] int32
+ */
+int orc_paged_decode(double* out, const void* q, int q_dtype, const void* k_cache,
+                     const void* v_cache, int cache_dtype, const uint16_t* k_scale,
+                     const uint16_t* v_scale, const int32_t* block_tables,
+                     const int32_t* context_lens, int S, int H, int D, int bs, int MB, int NB,
+                     double scale, int window) {
+  if (S < 0 || H <= 0 || D <= 0 || bs <= 0 || MB <= 0 || NB <= 0) return ORC_BAD_ARG;
+  if (cache_dtype == ORC_I8 && (!k_scale || !v_scale)) return ORC_BAD_ARG;
+
+  int max_ctx = MB * bs;
+  double* Kc = (double*)malloc(sizeof(double) * (size_t)max_ctx * D);
+  double* Vc = (double*)malloc(sizeof(double) * (size_t)max_ctx * D);
+  double* score = (double*)malloc(sizeof(double) * (size_t)max_ctx);
+  double* qv = (double*)malloc(sizeof(double) * (size_t)D);
+  if (!Kc || !Vc || !score || !qv) {
+    free(Kc); free(Vc); free(score); free(qv);
+    return ORC_NO_MEMORY;
+  }
+  int status = ORC_OK;
+
+  for (int s = 0; s < S && status == ORC_OK; ++s) {
+    int ctx = context_lens[s];
+    if (ctx < 0 || ctx > max_ctx) { status = ORC_BAD_CONTEXT; break; }
+    int lo = 0;
+    if (window > 0 && ctx > window) lo = ctx - window;
+    int n = ctx - lo;
+
+    for (int h = 0; h < H && status == ORC_OK; ++h) {
+      double* o = out + ((size_t)s * H + h) * D;
+      if (n == 0) {
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        continue;
+      }
+
+      /* step 2: gather through the block table */
+      for (int i = lo; i < ctx; ++i) {
+        int logical_block = i / bs;
+        int offset = i % bs;
+        int32_t pb = block_tables[(size_t)s * MB + logical_block];
+        if (pb < 0 || pb >= NB) { status = ORC_BAD_TABLE; break; }
+        size_t row = ((size_t)pb * bs + offset) * H + h; /* (pb*bs+off)*H + h */
+        double ks = 1.0, vs = 1.0;
+        if (cache_dtype == ORC_I8) {
+          ks = orc_f16_to_f64(k_scale[row]);
+          vs = orc_f16_to_f64(v_scale[row]);
+        }
+        for (int d = 0; d < D; ++d) {
+          Kc[(size_t)(i - lo) * D + d] = load_value(k_cache, cache_dtype, row * D + d) * ks;
+          Vc[(size_t)(i - lo) * D + d] = load_value(v_cache, cache_dtype, row * D + d) * vs;
+        }
+      }
+      if (status != ORC_OK) break;
+
+      for (int d = 0; d < D; ++d) qv[d] = load_value(q, q_dtype, ((size_t)s * H + h) * D + d);
+
+      /* step 3: scaled dot products */
+      for (int i = 0; i < n; ++i) {
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += qv[d] * Kc[(size_t)i * D + d];
+        score[i] = scale * dot;
+      }
+
+      /* step 4: textbook softmax */
+      double m = score[0];
+      for (int i = 1; i < n; ++i) if (score[i] > m) m = score[i];
+      double z = 0.0;
+      for (int i = 0; i < n; ++i) { score[i] = exp(score[i] - m); z += score[i]; }
+      for (int i = 0; i < n; ++i) score[i] /= z;
+
+      /* step 5: probability-weighted sum of the value rows */
+      for (int d = 0; d < D; ++d) {
+        double acc = 0.0;
+        for (int i = 0; i < n; ++i) acc += score[i] * Vc[(size_t)i * D + d];
+        o[d] = acc;
+      }
+    }
+  }
+
+  free(Kc); free(Vc); free(score); free(qv);
+  return status;
+}

@@ -1,0 +1,106 @@
+"""Pins of the oracle's INT8 quantiser and cache-maintenance definitions (CPU only).
+
+Quantiser (reading of "KV Cache optimisation strategies in deployment" (yunthe.com),
+section "量化压缩KV Cache的INT8与FP8方案", which names INT8 without a scheme): brute
+force over every finite fp16 value checks the dequantisation error bound, the code
+range, symmetry, that the row maximum maps to +-127, and ties-to-even on exact halves.
+Cache operations: the page's flat address h*D + (pb*bs + off)*H*D ("KV Cache memory
+optimisation and PagedAttention" (yunthe.com), section "PagedAttention注意力计算流程").
+"""
+import numpy as np
+import pytest
+
+from oracle import cache_ops, quant
+
+
+def _all_finite_f16():
+    v = np.arange(65536, dtype=np.uint16).view(np.float16)
+    return v[np.isfinite(v)]
+
+
+def test_every_fp16_value_dequantises_within_half_a_step():
+    x = _all_finite_f16()
+    # rows [x, m]: m = 1.0 sets the scale unless |x| is larger
+    rows = np.stack([x, np.full_like(x, 1.0)], axis=1)
+    codes, scale = quant.quantize_rows(rows)
+    deq = quant.dequantize_rows(codes, scale)
+    s = scale.astype(np.float64)
+    assert np.all(np.abs(codes.astype(np.int32)) <= 127)
+    err = np.abs(deq - rows.astype(np.float64))
+    # |x / s| <= 127 * (1 + 2^-11) so rounding to the nearest code is within s/2 (+ the fp32 division)
+    assert np.all(err <= s[:, None] * (0.5 + 1e-3))
+
+
+def test_row_maximum_maps_to_127():
+    rng = np.random.default_rng(0)
+    rows = rng.standard_normal((4096, 128)).astype(np.float16)
+    codes, scale = quant.quantize_rows(rows)
+    amax_idx = np.argmax(np.abs(rows.astype(np.float32)), axis=1)
+    top = np.abs(codes[np.arange(4096), amax_idx].astype(np.int32))
+    assert np.all(top == 127)
+    assert np.all(scale > 0)
+
+
+def test_quantiser_is_odd_symmetric():
+    rng = np.random.default_rng(1)
+    rows = rng.standard_normal((512, 64)).astype(np.float16)
+    c1, s1 = quant.quantize_rows(rows)
+    c2, s2 = quant.quantize_rows(-rows)
+    assert np.array_equal(s1, s2)
+    assert np.array_equal(c1.astype(np.int32), -c2.astype(np.int32))
+
+
+def test_exact_halves_round_to_even():
+    s = 2.0 ** -7                       # 127 * s is exact in fp16, amax / 127 = s exactly
+    row = np.array([127 * s, 2.5 * s, 3.5 * s, -2.5 * s, 0.5 * s, 1.5 * s, 0.0, -0.5 * s], np.float16)
+    codes, scale = quant.quantize_rows(row[None, :])
+    assert float(scale[0]) == s
+    assert codes[0].tolist() == [127, 2, 4, -2, 0, 2, 0, 0]
+
+
+def test_zero_row_has_zero_scale_and_codes():
+    codes, scale = quant.quantize_rows(np.zeros((3, 16), np.float16))
+    assert np.all(scale == 0) and np.all(codes == 0)
+
+
+def test_tiny_row_whose_scale_underflows_stores_zeros():
+    row = np.array([[2.0 ** -24, 0.0]], np.float16)  # amax / 127 rounds to 0 in fp16
+    codes, scale = quant.quantize_rows(row)
+    assert scale[0] == 0 and np.all(codes == 0)
+
+
+def test_reshape_and_cache_follows_the_pages_flat_address():
+    rng = np.random.default_rng(2)
+    NB, bs, H, D, T = 5, 4, 3, 8, 7
+    kc = np.zeros((NB, bs, H, D), np.float32)
+    vc = np.zeros((NB, bs, H, D), np.float32)
+    k = rng.standard_normal((T, H, D)).astype(np.float32)
+    v = rng.standard_normal((T, H, D)).astype(np.float32)
+    slots = np.array([0, 19, 5, -1, 7, 12, 3])
+    cache_ops.reshape_and_cache(k, v, kc, vc, slots)
+    flat_k, flat_v = kc.reshape(-1), vc.reshape(-1)
+    for t, slot in enumerate(slots):
+        if slot < 0:
+            continue
+        pb, off = slot // bs, slot % bs
+        for h in range(H):
+            addr = h * D + (pb * bs + off) * H * D   # the page's address expression
+            assert np.array_equal(flat_k[addr: addr + D], k[t, h])
+            assert np.array_equal(flat_v[addr: addr + D], v[t, h])
+    written = {int(s) for s in slots if s >= 0}
+    untouched = [s for s in range(NB * bs) if s not in written]
+    assert np.all(kc.reshape(NB * bs, -1)[untouched] == 0)
+
+
+def test_copy_blocks_duplicates_whole_blocks_and_nothing_else():
+    rng = np.random.default_rng(3)
+    NB, bs, H, D = 6, 4, 2, 8
+    kc = rng.standard_normal((NB, bs, H, D)).astype(np.float32)
+    vc = rng.standard_normal((NB, bs, H, D)).astype(np.float32)
+    k0, v0 = kc.copy(), vc.copy()
+    pairs = np.array([[1, 4], [2, 5]])
+    cache_ops.copy_blocks(kc, vc, pairs)
+    assert np.array_equal(kc[4], k0[1]) and np.array_equal(kc[5], k0[2])
+    assert np.array_equal(vc[4], v0[1]) and np.array_equal(vc[5], v0[2])
+    for b in (0, 1, 2, 3):
+        assert np.array_equal(kc[b], k0[b]) and np.array_equal(vc[b], v0[b])
