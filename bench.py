@@ -1,0 +1,362 @@
+"""Benchmark: paged decode attention on B200, one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--seed S]
+
+Workload: one Llama-2-70B attention layer decode step -- 32 sequences x 64 heads x 128
+dims, block_size 16, contexts uniform in [1, 2048], pool = blocks needed + 10 %, shuffled
+free list, fp16, synthetic N(0, 1) data.  A step is the whole hot path: write each
+sequence's newest K/V row into its slot (reshape_and_cache; no copy-on-write occurs in
+this workload, so copy_blocks has nothing to do), then paged decode attention (partition
++ merge kernels).  With N GPUs every rank runs its own batch (seed + rank): weak
+scaling, no collective on the data path; the timing is the max over ranks.
+
+Metric: algorithmic KV bytes (every attended K and V row read once) / step time, in GB/s;
+also tokens/s per layer (= sequences / step time) and % of the measured HBM copy peak.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+from paged_kv_cache_384_b200 import accounting  # noqa: E402
+
+PRESET = "llama70b_fp16"
+METRIC = "paged decode attention KV GB/s (% of B200 HBM peak) and tokens/s per layer"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------------------
+# helpers shared with the multi-rank tests
+# ---------------------------------------------------------------------------------------
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank decodes its own batch (weak scaling)."""
+    return seed + 1000 * rank
+
+
+def reduce_max(value: float, dist=None) -> float:
+    """Max over ranks of a per-rank time (identity without a process group)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(bytes_per_rank_step, steps: int, max_seconds: float) -> float:
+    """Aggregate GB/s: bytes of every rank over the slowest rank's time."""
+    return sum(bytes_per_rank_step) * steps / max_seconds / 1e9
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_traffic(kernel_source: str):
+    """ncu DRAM bytes per launch of the partition kernel, if captured for this exact source."""
+    path = os.path.join(ROOT, "profiles", "decode_partition_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    with open(kernel_source, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    if rec.get("source_sha256") != sha or rec.get("workload") != PRESET:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock / throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=10)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        rows = []
+        for line in getattr(self, "lines", []):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), max=float(f[2]), power=float(f[3]),
+                                 hw=f[5], hwt=f[6], swt=f[7], pcap=f[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["max"] for r in rows),
+                "samples": len(rows), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------------------
+# workload
+# ---------------------------------------------------------------------------------------
+def build(seed: int, device):
+    import paged_kv_cache_384_b200 as pa
+    w = synth.build_workload(PRESET, seed, pa.BlockManager)
+    ctx = w.context_lens.tolist()
+    slots = pa.slot_mapping(w.block_tables, range(w.num_seqs), [c - 1 for c in ctx], w.block_size)
+    host = dict(q=w.q, k_new=w.k_new, v_new=w.v_new, slots=slots, block_tables=w.block_tables,
+                context_lens=w.context_lens)
+    dev = {k: v.to(device) for k, v in host.items()}
+    dev["k_cache"] = w.k_cache.to(device)
+    dev["v_cache"] = w.v_cache.to(device)
+    dev["out"] = torch.empty_like(dev["q"])
+    dev["ws"] = pa.alloc_workspace(w.num_seqs, w.num_heads, w.head_dim, device)
+    dev["pairs"] = w.copy_pairs.to(device)
+    kv_bytes = accounting.decode_kv_bytes(ctx, w.num_heads, w.head_dim, w.cache_dtype, w.window)
+    return w, host, dev, kv_bytes
+
+
+def step(pa, w, d, stream):
+    """One pass of the hot path: append the newest rows, copy-on-write copies, decode."""
+    pa.reshape_and_cache(d["k_new"], d["v_new"], d["k_cache"], d["v_cache"], d["slots"], stream=stream)
+    if d["pairs"].shape[0]:
+        pa.copy_blocks(d["k_cache"], d["v_cache"], d["pairs"], stream=stream)
+    pa.paged_attention_decode(d["out"], d["q"], d["k_cache"], d["v_cache"], d["block_tables"],
+                              d["context_lens"], w.scale, w.window, workspace=d["ws"], stream=stream)
+
+
+def launches_per_step(d) -> int:
+    return 1 + (1 if d["pairs"].shape[0] else 0) + 2
+
+
+# ---------------------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------------------
+def cpu_oracle_rate(w, seqs, repeats=1):
+    """Time the fp64 oracle (single-threaded C) on the given sequences of the workload."""
+    import oracle  # the CPU-baseline leg is the one place the benchmark runs the oracle
+    sel = list(seqs)
+    kv = accounting.decode_kv_bytes([int(w.context_lens[s]) for s in sel], w.num_heads, w.head_dim,
+                                    w.cache_dtype, w.window)
+    t0 = time.perf_counter()
+    for _ in range(repeats):
+        oracle.paged_decode(w.q[sel], w.k_cache, w.v_cache, w.block_tables[sel], w.context_lens[sel],
+                            w.scale, w.window)
+    dt = (time.perf_counter() - t0) / repeats
+    return kv / dt / 1e9, dt, kv
+
+
+def run_reference(args):
+    """The oracle as it stands on the host cores, same workload/metric; rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import paged_kv_cache_384_b200 as pa  # only for the block manager that lays out the batch
+    w = synth.build_workload(PRESET, args.seed, pa.BlockManager)
+    sample = list(range(0, w.num_seqs, 4))          # 8 of the 32 sequences per step
+    for _ in range(args.warmup):
+        cpu_oracle_rate(w, sample)
+    times, kv = [], 0
+    for _ in range(args.steps):
+        _, dt, kv = cpu_oracle_rate(w, sample)
+        times.append(dt)
+    t = sum(times) / len(times)
+    value = kv / t / 1e9
+    desc = f"sequences 0,4,...,28 (8 of 32) of the {PRESET} batch per step, fp64 C oracle"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * t, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": PRESET, "num_seqs": len(sample), "num_heads": w.num_heads, "head_dim": w.head_dim,
+                   "block_size": w.block_size, "context": "uniform [1, 2048]", "seed": args.seed},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import paged_kv_cache_384_b200 as pa
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w, host, d, kv_bytes = build(rank_seed(args.seed, rank), device)
+    stream = torch.cuda.current_stream(device)
+    peak, peak_kind = measured_peak()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize(device)
+
+    # ---- warm-up, then the timed region: K steps between two events ----
+    for _ in range(args.warmup):
+        step(pa, w, d, stream)
+    barrier()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    props = torch.cuda.get_device_properties(device)
+    smi_id = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+    with ClockSampler(smi_id) as clocks:
+        start.record(stream)
+        for _ in range(args.steps):
+            step(pa, w, d, stream)
+        end.record(stream)
+        barrier()
+    sec = start.elapsed_time(end) / 1e3
+    sec_max = reduce_max(sec, dist)
+    all_bytes = [kv_bytes] * world if dist is None else None
+    if dist is not None:
+        t = torch.tensor([float(kv_bytes)], dtype=torch.float64, device=device)
+        gathered = [torch.zeros_like(t) for _ in range(world)]
+        dist.all_gather(gathered, t)
+        all_bytes = [float(x.item()) for x in gathered]
+    value = whole_job_gbs(all_bytes, args.steps, sec_max)
+    ms_step = 1e3 * sec_max / args.steps
+    tokens_per_s = world * w.num_seqs * args.steps / sec_max
+    device_errors = pa.device_error(clear=True)
+    pa.device_error(clear=True)
+
+    # ---- roofline: the partition kernel alone (library events around it) ----
+    pa.profile_enable(True)
+    pa.profile_read(reset=True)
+    for _ in range(args.steps):
+        step(pa, w, d, stream)
+    part_ms, merge_ms, calls = pa.profile_read(reset=True)
+    pa.profile_enable(False)
+    part_avg = part_ms / max(calls, 1)
+    merge_avg = merge_ms / max(calls, 1)
+    achieved = kv_bytes / (part_avg / 1e3) / 1e9
+    traffic = kernel_traffic(os.path.join(ROOT, "paged_kv_cache_384_b200", "csrc", "pa_decode.cu"))
+
+    # ---- end to end through the public API with host buffers ----
+    pin = {k: v.pin_memory() for k, v in host.items()}
+    out_host = torch.empty(d["out"].shape, dtype=d["out"].dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for k, v in pin.items():
+            d[k].copy_(v, non_blocking=True)
+        step(pa, w, d, stream)
+        out_host.copy_(d["out"], non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_sec = reduce_max(e0.elapsed_time(e1) / 1e3, dist)
+    e2e_value = whole_job_gbs(all_bytes, args.steps, e2e_sec)
+
+    # ---- CPU baseline: the oracle on this batch, rank 0 at N = 1 only ----
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        rate, dt, _ = cpu_oracle_rate(w, range(w.num_seqs))
+        cpu = {"value": round(rate, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"the full {PRESET} batch (32 sequences) once, fp64 C oracle, {dt:.1f} s"}
+
+    if dist is not None:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": PRESET, "num_seqs": w.num_seqs, "num_heads": w.num_heads, "head_dim": w.head_dim,
+                   "block_size": w.block_size, "num_blocks": w.num_blocks, "context": "uniform [1, 2048]",
+                   "kv_bytes_per_step_per_gpu": kv_bytes, "seed": args.seed,
+                   "l2": "inputs larger than L2 (KV per step >> 126 MB), no flush", "parallelism": f"replicas x{world}"},
+        "tokens_per_s_per_layer": round(tokens_per_s, 1),
+        "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_kind,
+                     "kernel": "decode_partition_kernel<half,half,128,16>", "partition_ms": round(part_avg, 4),
+                     "merge_ms": round(merge_avg, 4)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step(d) * args.steps,
+        "clocks": clocks.summary(),
+        "device_errors": device_errors,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)  # timing rule: at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

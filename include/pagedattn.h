@@ -1,0 +1,245 @@
+/*
+ * pagedattn.h -- C ABI of libpagedattn.so: paged decode attention on NVIDIA B200 (sm_100a).
+ *
+ * The method (sources: three web pages on PagedAttention):
+ *   "KV Cache memory optimisation and PagedAttention" (yunthe.com)              [page A]
+ *   "KV Cache optimisation strategies in deployment" (yunthe.com)               [page B]
+ *   "vLLM source first look: PagedAttention memory design" (trdm.cn)             [page C]
+ *
+ * The KV cache is cut into fixed-size physical blocks of block_size tokens (page A,
+ * section "PagedAttention分页内存管理原理").  A sequence finds token i through its block
+ * table: logical block i / block_size, offset i % block_size (page C, section 二,
+ * BlockTable.get_physical_block / get_offset).  Cache layout, from the pseudocode
+ * kernel's address h*D + (pb*bs + off)*H*D (page A, section "PagedAttention注意力计算流程"):
+ *
+ *     k_cache, v_cache : [num_blocks, block_size, num_heads, head_dim]   (row-major)
+ *     k_scale, v_scale : [num_blocks, block_size, num_heads] fp16        (INT8 cache only)
+ *
+ * A *slot* is pb*block_size + off: one token row of num_heads*head_dim values.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller (cudaMalloc or any
+ *     allocator); the library never allocates, frees or keeps them.  Tensors are dense,
+ *     row-major, and their base addresses must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is enqueued
+ *     asynchronously; the call returns once it is launched.
+ *   - Arguments are validated on the host before anything is launched; a non-PA_OK
+ *     status means nothing was enqueued.  pa_last_error() then gives a message.
+ *   - Device-side checks never fault: a block-table entry outside [0, num_blocks), a
+ *     context length above max_blocks_per_seq*block_size, a slot or copy pair outside
+ *     the pool is skipped or clamped and recorded in a device error word, read with
+ *     pa_device_error().  Results of such a call are unspecified.
+ *   - No call aborts, throws across the ABI or spins without a bound.
+ */
+#ifndef PAGEDATTN_H_
+#define PAGEDATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_dtype {
+  PA_F32 = 0,  /* IEEE binary32 */
+  PA_F16 = 1,  /* IEEE binary16 */
+  PA_BF16 = 2, /* bfloat16 */
+  PA_I8 = 3    /* signed 8-bit code with a per-(token, head) fp16 scale */
+} pa_dtype;
+
+typedef enum pa_status {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,   /* a pointer, size, alignment or dtype is not acceptable */
+  PA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. head_dim 96) */
+  PA_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed (message has the CUDA error) */
+  PA_ERR_OUT_OF_BLOCKS = 4, /* block manager: fewer free blocks than requested */
+  PA_ERR_BAD_BLOCK = 5      /* block manager: id out of range, or reference count would go negative */
+} pa_status;
+
+/* Bits of the device error word (pa_device_error). */
+#define PA_DEVERR_TABLE 0x1u   /* block-table entry outside [0, num_blocks): block 0 read instead */
+#define PA_DEVERR_CONTEXT 0x2u /* context_len < 0 or > max_blocks_per_seq*block_size: clamped */
+#define PA_DEVERR_SLOT 0x4u    /* reshape_and_cache slot >= num_blocks*block_size: token skipped */
+#define PA_DEVERR_PAIR 0x8u    /* copy_blocks pair index outside [0, num_blocks): pair skipped */
+#define PA_DEVERR_TIMEOUT 0x10u /* a bounded pipeline wait gave up (a library bug; results invalid) */
+
+/* Message for the last non-PA_OK status returned on the calling thread ("" if none). */
+const char* pa_last_error(void);
+
+/* Library version string. */
+const char* pa_version(void);
+
+/*
+ * Read (and if clear != 0, reset) the device error word of the current device.
+ * Synchronises the device first.  *flags receives an OR of PA_DEVERR_* bits.
+ */
+pa_status pa_device_error(uint32_t* flags, int clear);
+
+/* ------------------------------------------------------------------------------------ */
+/* Decode attention                                                                     */
+/* ------------------------------------------------------------------------------------ */
+
+/*
+ * Bytes of scratch workspace paged_attention_decode needs on the CURRENT device for a
+ * batch of num_seqs sequences x num_heads heads of size head_dim (any block_size,
+ * dtype or context length).  Returns 0 for invalid sizes or when no device is present.
+ */
+size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim);
+
+/*
+ * Paged decode attention: one query token per sequence attends over its cached keys
+ * and values.  Source: page A, section "PagedAttention注意力计算流程" (score =
+ * dot(q, k) * scale through the block table; softmax and the probability-weighted
+ * sum of values), page C, section 三 (walk the cache block by block), page B,
+ * section "Sliding Window Attention控制长序列显存" (window).
+ *
+ * For sequence s, head h, with ctx = context_lens[s] and lo = window > 0 ?
+ * max(0, ctx - window) : 0, the attended tokens are i in [lo, ctx):
+ *     k_i  = k_cache[block_tables[s][i / block_size], i % block_size, h, :]
+ *     p    = softmax_i(scale * <q[s,h,:], k_i>)
+ *     out[s,h,:] = sum_i p_i * v_i                      (ctx == 0: zeros)
+ * An INT8 cache holds codes c with k = c * k_scale[slot, h] (likewise v).
+ *
+ *   out            [num_seqs, num_heads, head_dim]        io_dtype, written
+ *   q              [num_seqs, num_heads, head_dim]        io_dtype
+ *   k_cache,
+ *   v_cache        [num_blocks, block_size, num_heads, head_dim]   cache_dtype
+ *   k_scale,
+ *   v_scale        [num_blocks, block_size, num_heads] fp16; required iff cache_dtype == PA_I8
+ *   block_tables   [num_seqs, max_blocks_per_seq] int32; only entries of blocks that hold
+ *                  attended tokens are read (others may hold anything, e.g. -1)
+ *   context_lens   [num_seqs] int32, 0 <= ctx <= max_blocks_per_seq*block_size
+ *   head_dim       64 or 128;  block_size 1..32;  num_heads >= 1 (multiple of 8 for PA_I8)
+ *   scale          softmax scale (typically 1/sqrt(head_dim))
+ *   window         0 = full attention, W > 0 = the last W tokens only
+ *   io_dtype       PA_F32, PA_F16 or PA_BF16; cache_dtype == io_dtype, or PA_I8 with
+ *                  io_dtype PA_F16 / PA_BF16
+ *   workspace      device scratch of >= pa_decode_workspace_bytes(...) bytes; contents
+ *                  need no initialisation and are clobbered.  Two calls that may run
+ *                  concurrently need distinct workspaces.
+ *
+ * Two kernels are enqueued (partition pass, then merge of split partitions).
+ * Accumulation is fp32; out is rounded to io_dtype (round to nearest even).
+ */
+pa_status paged_attention_decode(void* out, const void* q, const void* k_cache,
+                                 const void* v_cache, const void* k_scale, const void* v_scale,
+                                 const int32_t* block_tables, const int32_t* context_lens,
+                                 int num_seqs, int num_heads, int head_dim, int block_size,
+                                 int num_blocks, int max_blocks_per_seq, float scale, int window,
+                                 pa_dtype io_dtype, pa_dtype cache_dtype, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------ */
+/* Cache maintenance                                                                    */
+/* ------------------------------------------------------------------------------------ */
+
+/*
+ * Write each new token's key/value rows into its slot.  Source: the cache grows by one
+ * row per generated token (page C, section 一) into blocks allocated on demand (page A,
+ * section "vLLM调度器与PagedAttention协同工作").
+ *
+ *   k, v           [num_tokens, num_heads, head_dim] rows of `dtype`; consecutive tokens
+ *                  k_token_stride / v_token_stride ELEMENTS apart (>= num_heads*head_dim,
+ *                  so rows of a fused QKV tensor can be passed directly)
+ *   k_cache,
+ *   v_cache        [num_blocks, block_size, num_heads, head_dim] of `dtype`
+ *   slot_mapping   [num_tokens] int64: token t goes to slot slot_mapping[t]
+ *                  (= block*block_size + offset); a negative slot skips the token
+ *   dtype          PA_F32 / PA_F16 / PA_BF16 / PA_I8 (codes are copied as they are)
+ *   k_scale_src,   [num_tokens, num_heads] fp16 scales of the new rows, and
+ *   v_scale_src    k_scale_cache, v_scale_cache [num_blocks, block_size, num_heads] fp16:
+ *   k_scale_cache, required iff dtype == PA_I8, NULL otherwise
+ *   v_scale_cache
+ * Bit-exact copy.  Slots must be distinct (otherwise which token lands is unspecified).
+ */
+pa_status reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache,
+                            const int64_t* slot_mapping, int num_tokens, int num_heads,
+                            int head_dim, int block_size, int num_blocks, int64_t k_token_stride,
+                            int64_t v_token_stride, pa_dtype dtype, const void* k_scale_src,
+                            const void* v_scale_src, void* k_scale_cache, void* v_scale_cache,
+                            void* stream);
+
+/*
+ * Copy whole physical blocks for copy-on-write.  Source: page C, section 二,
+ * BlockManager.copy_on_write (the new block receives a copy of the old block's KV
+ * data) and section 四 (the copy is a latency cost of forking).
+ *
+ *   k_cache, v_cache    pools of num_blocks blocks, block_bytes bytes each
+ *                       (block_size*num_heads*head_dim*element size)
+ *   src_dst_pairs       [num_pairs, 2] int64 device array of (src, dst) block ids
+ *   k_scale_cache,      optional (both or neither) pools of scale_block_bytes bytes per
+ *   v_scale_cache       block (INT8 cache: block_size*num_heads*2)
+ * Destinations must be distinct and no destination may also be a source (otherwise the
+ * result is unspecified).  Bit-exact copy.
+ */
+pa_status copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs, int num_pairs,
+                      int num_blocks, size_t block_bytes, void* k_scale_cache, void* v_scale_cache,
+                      size_t scale_block_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------ */
+/* Host-side block manager (free list + reference counts)                               */
+/* ------------------------------------------------------------------------------------ */
+
+/*
+ * Physical-block allocator of page C, section 二 (BlockManager): a free list popped
+ * from its end, one reference count per block, copy-on-write.  Host memory only; not
+ * thread-safe (one manager per thread, or external locking).
+ */
+typedef struct pa_block_manager pa_block_manager;
+
+/* free_order: optional permutation of 0..num_blocks-1 giving the initial free list
+ * (the last entry is allocated first); NULL means 0..num_blocks-1.  NULL on bad input. */
+pa_block_manager* pa_bm_create(int num_blocks, int block_size, const int32_t* free_order);
+void pa_bm_destroy(pa_block_manager* bm);
+
+/* Take n blocks (reference count 1 each) into out_ids[n].  PA_ERR_OUT_OF_BLOCKS if fewer
+ * than n are free (nothing allocated). */
+pa_status pa_bm_allocate(pa_block_manager* bm, int n, int32_t* out_ids);
+
+/* Drop one reference of each listed block; a block whose count reaches 0 returns to the
+ * end of the free list.  PA_ERR_BAD_BLOCK (and no change at all) if any id is out of
+ * range or would drop below zero (double free). */
+pa_status pa_bm_free(pa_block_manager* bm, const int32_t* ids, int n);
+
+/* Add one reference to each listed, allocated block (a sequence forks and shares it). */
+pa_status pa_bm_share(pa_block_manager* bm, const int32_t* ids, int n);
+
+/* Copy-on-write: a block referenced at most once is returned unchanged; otherwise a new
+ * block is allocated (count 1), the old block loses one reference, and the new id is
+ * returned -- the caller then copies the data with copy_blocks. */
+pa_status pa_bm_copy_on_write(pa_block_manager* bm, int32_t block_id, int32_t* out_id);
+
+int pa_bm_num_free(const pa_block_manager* bm);
+int pa_bm_ref_count(const pa_block_manager* bm, int32_t block_id); /* -1 if out of range */
+double pa_bm_usage_ratio(const pa_block_manager* bm);             /* 1 - free/num_blocks */
+/* Copy the free list (bottom to top) into out[cap]; *n receives its length. */
+pa_status pa_bm_free_list(const pa_block_manager* bm, int32_t* out, int cap, int* n);
+
+/*
+ * Slot of token position pos of a sequence (host arrays): for each of n entries,
+ *   out[i] = block_tables[seq[i]*max_blocks_per_seq + pos[i]/block_size]*block_size
+ *            + pos[i] % block_size
+ * (page A, pseudocode kernel: physical_offset = physical_block*block_size + offset).
+ * PA_ERR_INVALID_ARG if a position falls outside the table or hits a negative entry.
+ */
+pa_status pa_slot_mapping_host(const int32_t* block_tables, int num_seqs, int max_blocks_per_seq,
+                               int block_size, const int32_t* seq, const int32_t* pos, int n,
+                               int64_t* out);
+
+/* ------------------------------------------------------------------------------------ */
+/* Profiling hooks                                                                      */
+/* ------------------------------------------------------------------------------------ */
+
+/* When enabled, paged_attention_decode records CUDA events around each of its two
+ * kernels on the launch stream (a few hundred ns of host time per call). */
+pa_status pa_profile_enable(int on);
+/* Synchronise the recorded events and return the summed device time of the partition
+ * and merge kernels over *calls calls since the last reset (reset != 0 clears). */
+pa_status pa_profile_read(double* partition_ms, double* merge_ms, int* calls, int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H_ */

@@ -1,0 +1,261 @@
+"""paged_kv_cache_384_b200 -- paged decode attention for NVIDIA B200 (sm_100a).
+
+Thin Python binding over ``libpagedattn.so`` (C ABI in ``include/pagedattn.h``).  PyTorch
+only supplies device memory and the current CUDA stream; every step of the computation
+runs in the library's CUDA kernels.  Functions take torch tensors, check that shapes,
+dtypes and devices agree, and pass raw pointers.
+
+    decode_workspace_bytes(num_seqs, num_heads, head_dim)
+    paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, ...)
+    reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, ...)
+    copy_blocks(k_cache, v_cache, src_dst_pairs, ...)
+    BlockManager(num_blocks, block_size, free_order=None)
+    slot_mapping(block_tables, seq_ids, positions, block_size)
+    device_error(clear=True)
+
+Cache layout: [num_blocks, block_size, num_heads, head_dim]; INT8 scales [num_blocks,
+block_size, num_heads] fp16.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import torch
+
+from . import _lib
+
+_L = _lib.load()
+
+PA_F32, PA_F16, PA_BF16, PA_I8 = 0, 1, 2, 3
+_DTYPE = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16, torch.int8: PA_I8}
+_STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_CUDA",
+           4: "PA_ERR_OUT_OF_BLOCKS", 5: "PA_ERR_BAD_BLOCK"}
+DEVERR = {"table": 0x1, "context": 0x2, "slot": 0x4, "pair": 0x8, "timeout": 0x10}
+
+LIB_PATH = _lib.LIB_PATH
+
+
+class PagedAttnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+def _check(status: int):
+    if status != 0:
+        raise PagedAttnError(status, _L.pa_last_error().decode())
+
+
+def version() -> str:
+    return _L.pa_version().decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dense(name, t):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+# ---------------------------------------------------------------------------------------
+# Decode attention
+# ---------------------------------------------------------------------------------------
+def decode_workspace_bytes(num_seqs: int, num_heads: int, head_dim: int) -> int:
+    """Scratch bytes paged_attention_decode needs on the current device."""
+    n = _L.pa_decode_workspace_bytes(num_seqs, num_heads, head_dim)
+    if n == 0 and num_seqs >= 0:
+        raise PagedAttnError(1, "no workspace size (invalid sizes or no CUDA device)")
+    return n
+
+
+def alloc_workspace(num_seqs: int, num_heads: int, head_dim: int, device=None) -> torch.Tensor:
+    """A workspace tensor (uint8) of the size paged_attention_decode needs."""
+    return torch.empty(decode_workspace_bytes(num_seqs, num_heads, head_dim), dtype=torch.uint8,
+                       device=device or "cuda")
+
+
+def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, window=0,
+                           k_scale=None, v_scale=None, workspace=None, stream=None):
+    """out[s,h,:] = softmax(scale * q[s,h] . K_s^T) V_s over the paged cache (fp32 accumulate).
+
+    q, out [S,H,D] fp32/fp16/bf16; k_cache, v_cache [NB,bs,H,D] of q's dtype, or int8 with
+    k_scale, v_scale [NB,bs,H] fp16; block_tables int32 [S,MB]; context_lens int32 [S].
+    window > 0 attends only the last ``window`` tokens.  ``workspace`` defaults to a fresh
+    allocation (pass one to keep allocation off the hot path).
+    """
+    S, H, D = q.shape
+    NB, bs, Hc, Dc = k_cache.shape
+    if out.shape != q.shape or out.dtype != q.dtype or (Hc, Dc) != (H, D) or v_cache.shape != k_cache.shape:
+        raise ValueError("shape/dtype mismatch between out, q and the caches")
+    if k_cache.dtype != v_cache.dtype:
+        raise ValueError("k_cache and v_cache must share a dtype")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise ValueError("block_tables and context_lens must be int32")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.shape != (S,):
+        raise ValueError("block_tables must be [S, MB] and context_lens [S]")
+    for name, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
+                    ("block_tables", block_tables), ("context_lens", context_lens)):
+        _dense(name, t)
+    if k_cache.dtype == torch.int8:
+        if k_scale is None or v_scale is None or k_scale.dtype != torch.float16 or \
+                k_scale.shape != (NB, bs, H) or v_scale.shape != (NB, bs, H):
+            raise ValueError("an int8 cache needs fp16 k_scale/v_scale of shape [NB, bs, H]")
+        _dense("k_scale", k_scale), _dense("v_scale", v_scale)
+    if workspace is None:
+        workspace = alloc_workspace(S, H, D, q.device)
+    _check(_L.paged_attention_decode(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
+        _ptr(block_tables), _ptr(context_lens), S, H, D, bs, NB, block_tables.shape[1],
+        float(scale), int(window), _DTYPE[q.dtype], _DTYPE[k_cache.dtype], _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
+
+
+# ---------------------------------------------------------------------------------------
+# Cache maintenance
+# ---------------------------------------------------------------------------------------
+def reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, k_scale=None, v_scale=None,
+                      k_scale_cache=None, v_scale_cache=None, stream=None):
+    """Write token t's rows k[t], v[t] ([T,H,D], token stride may exceed H*D) into slot
+    slot_mapping[t] (int64; negative = skip).  int8 caches also take per-(token, head)
+    fp16 scales [T,H] and the scale caches [NB,bs,H]."""
+    T, H, D = k.shape
+    NB, bs, Hc, Dc = k_cache.shape
+    if v.shape != k.shape or (Hc, Dc) != (H, D) or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch between k/v and the caches")
+    if k.dtype != k_cache.dtype or v.dtype != k_cache.dtype or v_cache.dtype != k_cache.dtype:
+        raise ValueError("k, v and the caches must share a dtype")
+    if slot_mapping.dtype != torch.int64 or slot_mapping.shape != (T,):
+        raise ValueError("slot_mapping must be int64 [T]")
+    for name, t in (("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+        if t.stride(2) != 1 or t.stride(1) != D:
+            raise ValueError(f"{name} rows must be dense [H, D] blocks")
+    _dense("k_cache", k_cache), _dense("v_cache", v_cache), _dense("slot_mapping", slot_mapping)
+    _check(_L.reshape_and_cache(
+        _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), T, H, D, bs, NB,
+        k.stride(0), v.stride(0), _DTYPE[k.dtype], _ptr(k_scale), _ptr(v_scale),
+        _ptr(k_scale_cache), _ptr(v_scale_cache), _stream(stream)))
+
+
+def copy_blocks(k_cache, v_cache, src_dst_pairs, k_scale_cache=None, v_scale_cache=None, stream=None):
+    """k_cache[dst] = k_cache[src] (and v, and the scale pools) for each (src, dst) pair."""
+    NB = k_cache.shape[0]
+    if v_cache.shape != k_cache.shape or v_cache.dtype != k_cache.dtype:
+        raise ValueError("k_cache and v_cache must match")
+    if src_dst_pairs.dtype != torch.int64 or src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2:
+        raise ValueError("src_dst_pairs must be int64 [N, 2]")
+    _dense("k_cache", k_cache), _dense("v_cache", v_cache), _dense("src_dst_pairs", src_dst_pairs)
+    block_bytes = k_cache[0].numel() * k_cache.element_size()
+    sbytes = 0 if k_scale_cache is None else k_scale_cache[0].numel() * k_scale_cache.element_size()
+    _check(_L.copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(src_dst_pairs), src_dst_pairs.shape[0], NB,
+                          block_bytes, _ptr(k_scale_cache), _ptr(v_scale_cache), sbytes, _stream(stream)))
+
+
+# ---------------------------------------------------------------------------------------
+# Host-side helpers
+# ---------------------------------------------------------------------------------------
+def slot_mapping(block_tables, seq_ids, positions, block_size: int) -> torch.Tensor:
+    """int64 slots of (sequence, position) pairs through host block tables (C helper)."""
+    bt = np.ascontiguousarray(torch.as_tensor(block_tables).cpu().numpy(), dtype=np.int32)
+    sq = np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int32).reshape(-1))
+    ps = np.ascontiguousarray(np.asarray(positions, dtype=np.int32).reshape(-1))
+    if sq.shape != ps.shape:
+        raise ValueError("seq_ids and positions must have the same length")
+    out = np.empty(sq.shape, np.int64)
+    _check(_L.pa_slot_mapping_host(bt.ctypes.data, bt.shape[0], bt.shape[1], block_size,
+                                   sq.ctypes.data, ps.ctypes.data, sq.size, out.ctypes.data))
+    return torch.from_numpy(out)
+
+
+def device_error(clear: bool = True) -> int:
+    """OR of PA_DEVERR_* bits raised by kernels on the current device (synchronises)."""
+    flags = ctypes.c_uint32(0)
+    _check(_L.pa_device_error(ctypes.byref(flags), int(clear)))
+    return flags.value
+
+
+def profile_enable(on: bool = True):
+    _check(_L.pa_profile_enable(int(on)))
+
+
+def profile_read(reset: bool = True):
+    """(partition_ms_total, merge_ms_total, calls) recorded since the last reset."""
+    a, b, n = ctypes.c_double(), ctypes.c_double(), ctypes.c_int()
+    _check(_L.pa_profile_read(ctypes.byref(a), ctypes.byref(b), ctypes.byref(n), int(reset)))
+    return a.value, b.value, n.value
+
+
+class BlockManager:
+    """Physical-block allocator (free list popped from its end + reference counts), native.
+
+    ``allocate(n)`` raises RuntimeError when fewer than n blocks are free; ``free(ids)``
+    raises RuntimeError (changing nothing) on a double free; ``copy_on_write(id)`` returns
+    the id unchanged when it is referenced at most once, else a fresh block.
+    """
+
+    def __init__(self, num_blocks: int, block_size: int, free_order=None):
+        order = None
+        if free_order is not None:
+            order = np.ascontiguousarray(np.asarray(free_order, dtype=np.int32))
+        self._h = _L.pa_bm_create(num_blocks, block_size, None if order is None else order.ctypes.data)
+        if not self._h:
+            raise ValueError(_L.pa_last_error().decode())
+        self.num_blocks, self.block_size = num_blocks, block_size
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h and _L is not None:
+            _L.pa_bm_destroy(h)
+        self._h = None
+
+    @staticmethod
+    def _raise(st):
+        if st in (4, 5):
+            raise RuntimeError(_L.pa_last_error().decode())
+        _check(st)
+
+    def allocate(self, num_blocks: int = 1):
+        out = np.empty(max(num_blocks, 0), np.int32)
+        self._raise(_L.pa_bm_allocate(self._h, num_blocks, out.ctypes.data))
+        return out.tolist()
+
+    def free(self, block_ids):
+        ids = np.ascontiguousarray(np.asarray(list(block_ids), dtype=np.int32))
+        self._raise(_L.pa_bm_free(self._h, ids.ctypes.data, ids.size))
+
+    def share(self, block_ids):
+        ids = np.ascontiguousarray(np.asarray(list(block_ids), dtype=np.int32))
+        self._raise(_L.pa_bm_share(self._h, ids.ctypes.data, ids.size))
+
+    def copy_on_write(self, block_id: int) -> int:
+        out = ctypes.c_int32()
+        self._raise(_L.pa_bm_copy_on_write(self._h, int(block_id), ctypes.byref(out)))
+        return out.value
+
+    def usage_ratio(self) -> float:
+        return _L.pa_bm_usage_ratio(self._h)
+
+    def ref_count(self, block_id: int) -> int:
+        return _L.pa_bm_ref_count(self._h, int(block_id))
+
+    @property
+    def free_blocks(self):
+        n = ctypes.c_int()
+        _check(_L.pa_bm_free_list(self._h, None, 0, ctypes.byref(n)))
+        out = np.empty(n.value, np.int32)
+        _check(_L.pa_bm_free_list(self._h, out.ctypes.data, n.value, ctypes.byref(n)))
+        return out.tolist()

@@ -1,0 +1,50 @@
+"""Byte and waste accounting for paged KV caches (host arithmetic on sizes only).
+
+* Per-token KV bytes: 2 (K and V) x layers x heads x head_dim x element bytes
+  ("KV Cache memory optimisation and PagedAttention" (yunthe.com), section
+  "大模型推理KV Cache内存消耗模型").
+* Waste of a contiguous reservation vs. a paged allocation ("vLLM source first look:
+  PagedAttention memory design" (trdm.cn), section 一, flowchart; block-size-16 waste claim
+  in "KV Cache memory optimisation and PagedAttention", section "vLLM调度器与PagedAttention协同工作").
+* Algorithmic bytes of one decode call: every attended token's K and V row for every head
+  is read exactly once (plus the fp16 scales of an INT8 cache).  This is the numerator of
+  the KV GB/s metric.
+"""
+from __future__ import annotations
+
+from typing import Iterable
+
+ELEM_BYTES = {"fp32": 4, "fp16": 2, "bf16": 2, "int8": 1}
+
+
+def kv_bytes_per_token(layers: int, num_heads: int, head_dim: int, dtype_size: int) -> int:
+    return 2 * layers * num_heads * head_dim * dtype_size
+
+
+def contiguous_waste_fraction(used_tokens: int, reserved_tokens: int) -> float:
+    """Share of a contiguous max-length reservation left unused."""
+    return 1.0 - used_tokens / reserved_tokens
+
+
+def paged_waste_fraction(used_tokens: int, block_size: int) -> float:
+    """Share of the allocated blocks left unused when blocks are taken on demand."""
+    if used_tokens <= 0:
+        return 0.0
+    allocated = -(-used_tokens // block_size) * block_size
+    return (allocated - used_tokens) / allocated
+
+
+def attended_tokens(context_len: int, window: int = 0) -> int:
+    """Tokens one decode step reads: the whole context, or its last ``window`` tokens."""
+    return min(context_len, window) if window > 0 else context_len
+
+
+def decode_kv_bytes(context_lens: Iterable[int], num_heads: int, head_dim: int, cache_dtype: str,
+                    window: int = 0) -> int:
+    """Algorithmic K+V bytes of one decode call over a batch (scales included for int8)."""
+    e = ELEM_BYTES[cache_dtype]
+    tokens = sum(attended_tokens(int(c), window) for c in context_lens)
+    total = tokens * num_heads * head_dim * 2 * e
+    if cache_dtype == "int8":
+        total += tokens * num_heads * 2 * 2  # one fp16 scale per (token, head) for K and for V
+    return total

@@ -1,0 +1,194 @@
+// pa_cache_ops.cu -- reshape_and_cache and copy_blocks for sm_100a.
+//
+// Both are pure data movement and HBM-bound.  Each thread moves 16-byte vectors; a CTA
+// covers a contiguous byte range so every warp issues fully coalesced 512-byte
+// transactions.  Slot and pair indices are bounds-checked on the device: an index outside
+// the pool skips the copy and sets a bit in the device error word instead of faulting.
+#include "pa_device.cuh"
+#include "pa_host.h"
+
+namespace pa {
+
+static __device__ unsigned int g_cache_error;
+
+__device__ __forceinline__ void cache_error(unsigned int bits) { atomicOr(&g_cache_error, bits); }
+
+// ---------------------------------------------------------------------------------------
+// reshape_and_cache: token t's row of H*D elements (row_bytes) goes to slot slot_mapping[t]
+// ("vLLM source first look: PagedAttention memory design" (trdm.cn), section 一: the cache
+// gains one row per generated token).  Grid: (vector chunks of a row, tokens).
+// ---------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+reshape_and_cache_kernel(const uint8_t* __restrict__ k, const uint8_t* __restrict__ v, uint8_t* __restrict__ kc,
+                         uint8_t* __restrict__ vc, const int64_t* __restrict__ slots, long long row_bytes,
+                         long long k_stride_bytes, long long v_stride_bytes, long long num_slots,
+                         const uint16_t* __restrict__ ks_src, const uint16_t* __restrict__ vs_src,
+                         uint16_t* __restrict__ ks_cache, uint16_t* __restrict__ vs_cache, int H) {
+  const int t = blockIdx.y;
+  const long long slot = __ldg(slots + t);
+  if (slot < 0) return;  // padding token
+  if (slot >= num_slots) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) cache_error(PA_DEVERR_SLOT);
+    return;
+  }
+  const long long nvec = row_bytes / 16;
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < nvec) {
+    const uint4 kv = __ldg(reinterpret_cast<const uint4*>(k + t * k_stride_bytes) + i);
+    const uint4 vv = __ldg(reinterpret_cast<const uint4*>(v + t * v_stride_bytes) + i);
+    reinterpret_cast<uint4*>(kc + slot * row_bytes)[i] = kv;
+    reinterpret_cast<uint4*>(vc + slot * row_bytes)[i] = vv;
+  }
+  if (ks_src && blockIdx.x == 0) {
+    for (int h = threadIdx.x; h < H; h += blockDim.x) {
+      ks_cache[slot * H + h] = ks_src[static_cast<long long>(t) * H + h];
+      vs_cache[slot * H + h] = vs_src[static_cast<long long>(t) * H + h];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// copy_blocks: pool block dst <- pool block src for each (src, dst) pair ("vLLM source first
+// look: PagedAttention memory design" (trdm.cn), section 二, BlockManager.copy_on_write).
+// Grid: (chunks of a block, pairs, 2 or 4 pools).  VEC = 16 moves uint4; VEC = 1 moves bytes.
+// ---------------------------------------------------------------------------------------
+template <int VEC>
+__global__ void __launch_bounds__(256)
+copy_blocks_kernel(uint8_t* k, uint8_t* v, uint8_t* ks, uint8_t* vs, const int64_t* __restrict__ pairs,
+                   long long block_bytes, long long scale_block_bytes, long long num_blocks) {
+  const int pool = blockIdx.z;  // 0: K, 1: V, 2: K scales, 3: V scales
+  const long long src = __ldg(pairs + 2 * blockIdx.y), dst = __ldg(pairs + 2 * blockIdx.y + 1);
+  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && pool == 0) cache_error(PA_DEVERR_PAIR);
+    return;
+  }
+  uint8_t* base = pool == 0 ? k : pool == 1 ? v : pool == 2 ? ks : vs;
+  const long long bytes = pool < 2 ? block_bytes : scale_block_bytes;
+  const uint8_t* from = base + src * bytes;
+  uint8_t* to = base + dst * bytes;
+  if (VEC == 16 && pool < 2) {
+    constexpr int kPerThread = 4;  // 4 independent 16-byte loads in flight per thread
+    const long long nvec = bytes / 16;
+    const long long first = (static_cast<long long>(blockIdx.x) * blockDim.x * kPerThread) + threadIdx.x;
+    uint4 tmp[kPerThread];
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+      const long long i = first + static_cast<long long>(u) * blockDim.x;
+      if (i < nvec) tmp[u] = reinterpret_cast<const uint4*>(from)[i];
+    }
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+      const long long i = first + static_cast<long long>(u) * blockDim.x;
+      if (i < nvec) reinterpret_cast<uint4*>(to)[i] = tmp[u];
+    }
+  } else {
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < bytes; i += stride)
+      to[i] = from[i];
+  }
+}
+
+namespace {
+
+cudaError_t read_cache_error(uint32_t* flags, int clear) {
+  unsigned int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_cache_error, sizeof v);
+  if (e != cudaSuccess) return e;
+  *flags = v;
+  if (clear && v) {
+    const unsigned int z = 0;
+    e = cudaMemcpyToSymbol(g_cache_error, &z, sizeof z);
+  }
+  return e;
+}
+
+struct RegisterCache {
+  RegisterCache() { register_device_error_reader(read_cache_error); }
+} g_register_cache;
+
+size_t elem_size(pa_dtype t) { return t == PA_F32 ? 4 : (t == PA_I8 ? 1 : 2); }
+
+}  // namespace
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" pa_status reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache,
+                                       const int64_t* slot_mapping, int num_tokens, int num_heads, int head_dim,
+                                       int block_size, int num_blocks, int64_t k_token_stride, int64_t v_token_stride,
+                                       pa_dtype dtype, const void* k_scale_src, const void* v_scale_src,
+                                       void* k_scale_cache, void* v_scale_cache, void* stream) {
+  if (num_tokens < 0 || num_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: sizes must be positive (num_tokens >= 0)");
+  if (dtype != PA_F32 && dtype != PA_F16 && dtype != PA_BF16 && dtype != PA_I8)
+    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: unknown dtype %d", static_cast<int>(dtype));
+  const long long row_elems = static_cast<long long>(num_heads) * head_dim;
+  const size_t e = elem_size(dtype);
+  const long long row_bytes = row_elems * static_cast<long long>(e);
+  if (row_bytes % 16) return fail(PA_ERR_UNSUPPORTED, "reshape_and_cache: a token row (%lld bytes) must be a multiple of 16 bytes", row_bytes);
+  if (k_token_stride < row_elems || v_token_stride < row_elems)
+    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: token strides must be >= num_heads*head_dim");
+  if ((k_token_stride * static_cast<long long>(e)) % 16 || (v_token_stride * static_cast<long long>(e)) % 16)
+    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: token strides must be multiples of 16 bytes");
+  const bool int8 = dtype == PA_I8;
+  if (int8 != (k_scale_src && v_scale_src && k_scale_cache && v_scale_cache) ||
+      (!int8 && (k_scale_src || v_scale_src || k_scale_cache || v_scale_cache)))
+    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: the four scale pointers are required for PA_I8 and must be NULL otherwise");
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !k_cache || !v_cache || !slot_mapping) return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: NULL pointer");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      reinterpret_cast<uintptr_t>(slot_mapping) % 8)
+    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: k, v and caches must be 16-byte aligned, slot_mapping 8-byte aligned");
+  if (int8 && ((reinterpret_cast<uintptr_t>(k_scale_src) | reinterpret_cast<uintptr_t>(v_scale_src) |
+                reinterpret_cast<uintptr_t>(k_scale_cache) | reinterpret_cast<uintptr_t>(v_scale_cache)) & 1))
+    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: scale pointers must be 2-byte aligned");
+  if (num_tokens > 65535) return fail(PA_ERR_UNSUPPORTED, "reshape_and_cache: at most 65535 tokens per call");
+
+  const long long nvec = row_bytes / 16;
+  const int threads = 256;
+  dim3 grid(static_cast<unsigned>((nvec + threads - 1) / threads), static_cast<unsigned>(num_tokens));
+  reshape_and_cache_kernel<<<grid, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(k), static_cast<const uint8_t*>(v), static_cast<uint8_t*>(k_cache),
+      static_cast<uint8_t*>(v_cache), slot_mapping, row_bytes, k_token_stride * static_cast<long long>(e),
+      v_token_stride * static_cast<long long>(e), static_cast<long long>(num_blocks) * block_size,
+      static_cast<const uint16_t*>(k_scale_src), static_cast<const uint16_t*>(v_scale_src),
+      static_cast<uint16_t*>(k_scale_cache), static_cast<uint16_t*>(v_scale_cache), num_heads);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return cuda_fail(err, "launching reshape_and_cache");
+  return PA_OK;
+}
+
+extern "C" pa_status copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs, int num_pairs,
+                                 int num_blocks, size_t block_bytes, void* k_scale_cache, void* v_scale_cache,
+                                 size_t scale_block_bytes, void* stream) {
+  if (num_pairs < 0 || num_blocks <= 0 || block_bytes == 0)
+    return fail(PA_ERR_INVALID_ARG, "copy_blocks: num_pairs >= 0, num_blocks > 0 and block_bytes > 0 required");
+  const bool scales = k_scale_cache || v_scale_cache;
+  if (scales && (!k_scale_cache || !v_scale_cache || scale_block_bytes == 0))
+    return fail(PA_ERR_INVALID_ARG, "copy_blocks: pass both scale pools with scale_block_bytes > 0, or neither");
+  if (num_pairs == 0) return PA_OK;
+  if (!k_cache || !v_cache || !src_dst_pairs) return fail(PA_ERR_INVALID_ARG, "copy_blocks: NULL pointer");
+  if (reinterpret_cast<uintptr_t>(src_dst_pairs) % 8) return fail(PA_ERR_INVALID_ARG, "copy_blocks: pairs must be 8-byte aligned");
+  if (num_pairs > 65535) return fail(PA_ERR_UNSUPPORTED, "copy_blocks: at most 65535 pairs per call");
+
+  const bool vec_ok = block_bytes % 16 == 0 && aligned16(k_cache) && aligned16(v_cache);
+  const int threads = 256;
+  const long long per_cta = vec_ok ? 16LL * threads * 4 : threads * 64LL;
+  const long long longest = static_cast<long long>(block_bytes > scale_block_bytes ? block_bytes : scale_block_bytes);
+  dim3 grid(static_cast<unsigned>((longest + per_cta - 1) / per_cta), static_cast<unsigned>(num_pairs), scales ? 4u : 2u);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (vec_ok) {
+    copy_blocks_kernel<16><<<grid, threads, 0, s>>>(
+        static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache), static_cast<uint8_t*>(k_scale_cache),
+        static_cast<uint8_t*>(v_scale_cache), src_dst_pairs, static_cast<long long>(block_bytes),
+        static_cast<long long>(scale_block_bytes), num_blocks);
+  } else {
+    copy_blocks_kernel<1><<<grid, threads, 0, s>>>(
+        static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache), static_cast<uint8_t*>(k_scale_cache),
+        static_cast<uint8_t*>(v_scale_cache), src_dst_pairs, static_cast<long long>(block_bytes),
+        static_cast<long long>(scale_block_bytes), num_blocks);
+  }
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return cuda_fail(err, "launching copy_blocks");
+  return PA_OK;
+}

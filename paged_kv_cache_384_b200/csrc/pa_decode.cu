@@ -1,0 +1,769 @@
+// pa_decode.cu -- paged decode attention for sm_100a.
+//
+// Method: one query token per sequence attends over its cached K/V, which live in
+// fixed-size physical blocks found through a per-sequence block table ("KV Cache memory
+// optimisation and PagedAttention" (yunthe.com), section "PagedAttention注意力计算流程";
+// "vLLM source first look: PagedAttention memory design" (trdm.cn), section 三: walk the
+// cache block by block so each block's rows are read contiguously).
+//
+// B200 design (the pages' pseudocode -- one thread per token, one CTA per (head, seq) --
+// is prior art only):
+//   * Work unit = one physical block x a group of HG heads ("tile").  All tiles of all
+//     sequences form one stream ordered (sequence, head group, block); a persistent grid
+//     of C CTAs (a small multiple of the SM count) takes equal contiguous slices of it, so
+//     ragged context lengths cost no load imbalance.  A slice that ends inside a
+//     (sequence, head group) "segment" leaves a partial softmax state (m, l, acc) in the
+//     workspace; a second kernel merges the partials of split segments.
+//   * Inside a CTA, one producer warp walks the slice, reads block-table entries 32 at a
+//     time, and issues one 3-D TMA load per tile for K and one for V ([bs, HG, D] boxes of
+//     the [NB*bs, H, D] cache) into an NS-stage shared-memory ring guarded by mbarriers.
+//     HG consumer warps (one per head) compute the scores with 16-byte shared loads and
+//     warp-shuffle dot products, keep an online softmax (running max / sum, base 2), and
+//     accumulate the probability-weighted V rows in fp32.
+//   * HBM-bound: ~1 FMA per byte of fp16 K/V, far below the FP32 pipes' limit; tensor cores
+//     have nothing dense to do with a single query row per head.
+#include <cfloat>
+#include <cstdio>
+#include <type_traits>
+
+#include "pa_device.cuh"
+#include "pa_host.h"
+
+namespace pa {
+
+static __device__ unsigned int g_decode_error;
+
+__device__ __forceinline__ void decode_error(unsigned int bits) { atomicOr(&g_decode_error, bits); }
+
+constexpr int kMaxCtasPerSm = 4;    // persistent-grid CTAs per SM (upper bound)
+constexpr int kMaxHeadGroup = 8;    // heads per CTA (upper bound)
+constexpr int kMaxThreads = 32 * (kMaxHeadGroup + 1);
+constexpr int kBarrierBytes = 128;  // mbarriers at the front of dynamic smem (<= 8 stages)
+
+struct DecodeParams {
+  void* out;
+  const void* q;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  long long* ws_prefix;  // [S + 1] per-sequence tile prefix (written by CTA 0)
+  float* ws_ml;          // [nslot][HG][2] partial (max, sum)
+  float* ws_acc;         // [nslot][HG][D] partial accumulators
+  int S, H, bs, MB, NB, window;
+  int HG, G, num_ctas, nstage;
+  float qscale;          // softmax scale * log2(e): scores are kept in base 2
+  uint32_t stage_bytes;  // bytes per pipeline stage
+  uint32_t v_off, ks_off, vs_off;  // offsets of the V tile and the INT8 scale tiles in a stage
+  uint32_t tx_bytes;     // TMA transaction bytes per stage
+};
+
+// Attended span of one sequence: tokens [lo, ctx), blocks first_lb .. first_lb + nb - 1.
+struct Span {
+  int ctx, lo, first_lb, nb;
+};
+
+__device__ __forceinline__ Span seq_span(const DecodeParams& p, int s, bool report) {
+  int ctx = __ldg(p.context_lens + s);
+  const int cap = p.MB * p.bs;
+  if (ctx < 0 || ctx > cap) {
+    if (report) decode_error(PA_DEVERR_CONTEXT);
+    ctx = ctx < 0 ? 0 : cap;
+  }
+  Span r;
+  r.ctx = ctx;
+  r.lo = (p.window > 0 && ctx > p.window) ? ctx - p.window : 0;
+  r.first_lb = r.lo / p.bs;
+  r.nb = ctx > 0 ? (ctx - 1) / p.bs - r.first_lb + 1 : 0;
+  return r;
+}
+
+// Position in the tile stream: sequence s, head group g, tile j of the segment.
+struct Cursor {
+  int s, g, j;
+  Span sp;
+};
+
+__device__ __forceinline__ void advance(Cursor& c, const DecodeParams& p) {
+  if (++c.j < c.sp.nb) return;
+  c.j = 0;
+  if (++c.g < p.G) return;
+  c.g = 0;
+  for (++c.s; c.s < p.S; ++c.s) {
+    c.sp = seq_span(p, c.s, false);
+    if (c.sp.nb > 0) return;
+  }
+}
+
+// Slice [t0, t0 + count) of the T-tile stream owned by CTA c of C (equal split, the
+// first T % C CTAs take one extra tile).
+__device__ __forceinline__ void cta_slice(long long T, int C, int c, long long* t0, long long* count) {
+  const long long base = T / C, rem = T % C;
+  *t0 = c * base + (c < rem ? c : rem);
+  *count = base + (c < rem ? 1 : 0);
+}
+
+// CTA owning tile t (inverse of cta_slice).
+__device__ __forceinline__ int cta_of(long long t, long long T, int C) {
+  const long long base = T / C, rem = T % C;
+  const long long big = rem * (base + 1);
+  return static_cast<int>(t < big ? t / (base + 1) : rem + (t - big) / base);
+}
+
+// Load n consecutive elements of type IO as floats (n * sizeof(IO) is a multiple of 16).
+template <typename IO, int N>
+__device__ __forceinline__ void load_floats(const IO* src, float* dst) {
+  constexpr int EVIO = Elem<IO>::kEV;
+  static_assert(N % EVIO == 0, "vector multiple");
+#pragma unroll
+  for (int i = 0; i < N / EVIO; ++i) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + i);
+    Elem<IO>::to_float(v, dst + i * EVIO);
+  }
+}
+
+template <typename IO, int N>
+__device__ __forceinline__ void store_floats(IO* dst, const float* src) {
+  static_assert((N * sizeof(IO)) % 16 == 0, "vector multiple");
+  IO tmp[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i) tmp[i] = float_to<IO>(src[i]);
+#pragma unroll
+  for (int i = 0; i < static_cast<int>(N * sizeof(IO) / 16); ++i)
+    reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(tmp)[i];
+}
+
+// ---------------------------------------------------------------------------------------
+// Partition kernel.
+//   IO: q/out type; CT: cache element type; D: head_dim; BS: block_size if fixed, 0 = runtime.
+// ---------------------------------------------------------------------------------------
+template <typename IO, typename CT, int D, int BS>
+__global__ void __launch_bounds__(kMaxThreads)
+decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                        const __grid_constant__ CUtensorMap tmKs, const __grid_constant__ CUtensorMap tmVs,
+                        const DecodeParams p) {
+  constexpr bool kInt8 = std::is_same<CT, int8_t>::value;
+  constexpr int E = Elem<CT>::kBytes;  // bytes per cache element
+  constexpr int EV = Elem<CT>::kEV;    // cache elements per 16-byte vector (dims per lane)
+  constexpr int LPR = D / EV;          // lanes covering one token row of one head
+  constexpr int RPP = 32 / LPR;        // token rows per warp-wide pass
+  constexpr int MAXP = BS > 0 ? (BS + RPP - 1) / RPP : (32 + RPP - 1) / RPP;
+  static_assert(LPR >= 1 && LPR <= 32 && 32 % LPR == 0, "lane mapping");
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ long long s_chunk[kMaxThreads];
+  __shared__ long long s_total;
+  __shared__ int s_first_seq;
+  __shared__ long long s_first_prefix;
+
+  const int bs = BS > 0 ? BS : p.bs;
+  const int HG = p.HG, G = p.G, NS = p.nstage;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nthr = blockDim.x;
+
+  // ---- 1. Plan: tiles per sequence, their prefix sum, and this CTA's slice. -----------
+  const int chunk = (p.S + nthr - 1) / nthr;
+  const int s_lo = min(p.S, threadIdx.x * chunk), s_hi = min(p.S, s_lo + chunk);
+  long long mine = 0;
+  for (int s = s_lo; s < s_hi; ++s) mine += seq_span(p, s, blockIdx.x == 0).nb;
+  s_chunk[threadIdx.x] = mine;
+  if (threadIdx.x == 0) s_first_seq = -1;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long run = 0;
+    for (int i = 0; i < nthr; ++i) {
+      const long long v = s_chunk[i];
+      s_chunk[i] = run;
+      run += v;
+    }
+    s_total = run;
+  }
+  __syncthreads();
+  const long long per_group = s_total;  // tiles of one head group over all sequences
+  const long long T = per_group * G;
+  const long long my_prefix = s_chunk[threadIdx.x];
+  if (blockIdx.x == 0) {  // publish the per-sequence prefix for the merge kernel
+    long long r = my_prefix;
+    for (int s = s_lo; s < s_hi; ++s) {
+      p.ws_prefix[s] = r;
+      r += seq_span(p, s, false).nb;
+    }
+    if (threadIdx.x == 0) p.ws_prefix[p.S] = per_group;
+  }
+  long long t0, count;
+  cta_slice(T, p.num_ctas, blockIdx.x, &t0, &count);
+  if (count == 0) return;  // uniform across the CTA; no barrier in use yet
+
+  // Sequence holding t0: sequence s starts at tile G * prefix(s).
+  if (t0 >= G * my_prefix && t0 < G * (my_prefix + mine)) {
+    long long r = my_prefix;
+    for (int s = s_lo; s < s_hi; ++s) {
+      const int nb = seq_span(p, s, false).nb;
+      if (t0 < G * (r + nb)) {
+        s_first_seq = s;
+        s_first_prefix = r;
+        break;
+      }
+      r += nb;
+    }
+  }
+
+  // ---- 2. Pipeline barriers. --------------------------------------------------------
+  const uint32_t bar_base = smem_u32(smem);
+  const uint32_t stage_base = (bar_base + kBarrierBytes + 127u) & ~127u;  // TMA wants 128-B aligned tiles
+  auto full_bar = [&](int st) { return bar_base + 8u * st; };
+  auto empty_bar = [&](int st) { return bar_base + 8u * (NS + st); };
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < NS; ++st) {
+      mbar_init(full_bar(st), 1);
+      mbar_init(empty_bar(st), HG);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (s_first_seq < 0) {  // cannot happen when count > 0; never index with it
+    if (threadIdx.x == 0) decode_error(PA_DEVERR_TIMEOUT);
+    return;
+  }
+
+  Cursor start;
+  start.s = s_first_seq;
+  start.sp = seq_span(p, start.s, false);
+  {
+    const long long rem = t0 - G * s_first_prefix;
+    start.g = static_cast<int>(rem / start.sp.nb);
+    start.j = static_cast<int>(rem % start.sp.nb);
+  }
+  const int n = static_cast<int>(count);
+
+  if (warp == HG) {
+    // ---- 3. Producer warp: block-table lookups + TMA issue. --------------------------
+    const uint64_t policy = l2_policy_evict_first();
+    if (lane == 0) {
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      if (kInt8) {
+        prefetch_tensormap(&tmKs);
+        prefetch_tensormap(&tmVs);
+      }
+    }
+    Cursor c = start;
+    int tab_seq = -1, tab_base = 0;
+    int32_t tab = 0;
+    int issued = 0;
+    bool ok = true;
+    for (; issued < n; ++issued) {
+      const int lb = c.sp.first_lb + c.j;  // logical block index
+      if (c.s != tab_seq || lb - tab_base >= 32 || lb < tab_base) {
+        tab_seq = c.s;
+        tab_base = lb;
+        const int idx = tab_base + lane;
+        tab = idx < c.sp.first_lb + c.sp.nb ? __ldg(p.block_tables + static_cast<size_t>(c.s) * p.MB + idx) : 0;
+      }
+      int pb = __shfl_sync(0xffffffffu, tab, lb - tab_base);
+      if (pb < 0 || pb >= p.NB) {
+        if (lane == 0) decode_error(PA_DEVERR_TABLE);
+        pb = 0;
+      }
+      const int st = issued % NS;
+      if (lane == 0) {
+        if (issued >= NS && !mbar_wait_bounded(empty_bar(st), ((issued / NS) - 1) & 1)) {
+          decode_error(PA_DEVERR_TIMEOUT);
+          ok = false;
+        }
+        if (ok) {
+          const uint32_t dst = stage_base + st * p.stage_bytes;
+          const int head0 = c.g * HG, row0 = pb * bs;
+          mbar_arrive_expect_tx(full_bar(st), p.tx_bytes);
+          tma_load_3d(dst, &tmK, full_bar(st), 0, head0, row0, policy);
+          tma_load_3d(dst + p.v_off, &tmV, full_bar(st), 0, head0, row0, policy);
+          if (kInt8) {
+            const int hx = head0 & ~7;  // 16-byte aligned x for the fp16 scale rows
+            tma_load_2d(dst + p.ks_off, &tmKs, full_bar(st), hx, row0, policy);
+            tma_load_2d(dst + p.vs_off, &tmVs, full_bar(st), hx, row0, policy);
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      advance(c, p);
+    }
+    // Never leave the CTA with copies in flight: wait (bounded) for the last stages.
+    if (lane == 0) {
+      for (int k = issued - NS < 0 ? 0 : issued - NS; k < issued; ++k)
+        if (!mbar_wait_bounded(full_bar(k % NS), (k / NS) & 1)) decode_error(PA_DEVERR_TIMEOUT);
+    }
+    return;
+  }
+
+  // ---- 4. Consumer warps: warp w owns head g*HG + w of every tile. ---------------------
+  const int w = warp;
+  const int r = lane / LPR;  // token row within a pass
+  const int v = lane % LPR;  // 16-byte vector within the row: dims [v*EV, v*EV + EV)
+  Cursor c = start;
+  bool seg_from_start = (c.j == 0);
+  float qf[EV], acc[EV];
+  float m = -FLT_MAX, l = 0.f;  // running max (base 2) and sum; -FLT_MAX keeps exp2 finite
+  auto load_q = [&](const Cursor& cc) {
+    const int h = cc.g * HG + w;
+    const IO* qrow = reinterpret_cast<const IO*>(p.q) + (static_cast<size_t>(cc.s) * p.H + h) * D + v * EV;
+    load_floats<IO, EV>(qrow, qf);
+#pragma unroll
+    for (int e = 0; e < EV; ++e) qf[e] *= p.qscale;
+  };
+  load_q(c);
+#pragma unroll
+  for (int e = 0; e < EV; ++e) acc[e] = 0.f;
+
+  for (int it = 0; it < n; ++it) {
+    const int st = it % NS;
+    if (!mbar_wait_bounded(full_bar(st), (it / NS) & 1)) {
+      if (lane == 0) decode_error(PA_DEVERR_TIMEOUT);
+      break;
+    }
+    const uint32_t kt = stage_base + st * p.stage_bytes;
+    const uint32_t vt = kt + p.v_off;
+    const int tok0 = (c.sp.first_lb + c.j) * bs;  // logical index of the tile's first row
+    const int hs = c.g * HG - ((c.g * HG) & ~7) + w;  // head column in the INT8 scale tile
+
+    // Scores of this lane's rows (tokens pi*RPP + r), base-2 scaled.
+    float sc[MAXP];
+    float tile_max = -FLT_MAX;
+#pragma unroll
+    for (int pi = 0; pi < MAXP; ++pi) {
+      sc[pi] = -INFINITY;
+      if (BS > 0 || pi * RPP < bs) {  // warp-uniform
+        const int t = pi * RPP + r;
+        float part = 0.f;
+        if (t < bs) {
+          float kf[EV];
+          Elem<CT>::to_float(ld_shared_v4(kt + ((t * HG + w) * D + v * EV) * E), kf);
+#pragma unroll
+          for (int e = 0; e < EV; ++e) part = fmaf(qf[e], kf[e], part);
+        }
+#pragma unroll
+        for (int off = LPR / 2; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+        const int tok = tok0 + t;
+        if (t < bs && tok >= c.sp.lo && tok < c.sp.ctx) {
+          if (kInt8) part *= __half2float(__ushort_as_half(ld_shared_u16(kt + p.ks_off + (t * 8 + hs) * 2)));
+          sc[pi] = part;
+          tile_max = fmaxf(tile_max, part);
+        }
+      }
+    }
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1) tile_max = fmaxf(tile_max, __shfl_xor_sync(0xffffffffu, tile_max, off));
+
+    // Online softmax update, then the probability-weighted V rows.
+    const float m_new = fmaxf(m, tile_max);
+    const float alpha = exp2f(m - m_new);
+    m = m_new;
+    l *= alpha;
+#pragma unroll
+    for (int e = 0; e < EV; ++e) acc[e] *= alpha;
+#pragma unroll
+    for (int pi = 0; pi < MAXP; ++pi) {
+      if (BS > 0 || pi * RPP < bs) {
+        const int t = pi * RPP + r;
+        if (sc[pi] != -INFINITY) {  // attended row (rows outside [lo, ctx) may hold garbage)
+          const float pr = exp2f(sc[pi] - m);
+          l += pr;
+          float vf[EV];
+          Elem<CT>::to_float(ld_shared_v4(vt + ((t * HG + w) * D + v * EV) * E), vf);
+          float pv = pr;
+          if (kInt8) pv *= __half2float(__ushort_as_half(ld_shared_u16(kt + p.vs_off + (t * 8 + hs) * 2)));
+#pragma unroll
+          for (int e = 0; e < EV; ++e) acc[e] = fmaf(pv, vf[e], acc[e]);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty_bar(st));
+
+    const bool seg_last = (c.j == c.sp.nb - 1);
+    if (seg_last || it == n - 1) {
+      // Combine the RPP row groups of the warp.
+      float lt = l;
+#pragma unroll
+      for (int off = LPR; off < 32; off <<= 1) {
+        lt += __shfl_xor_sync(0xffffffffu, lt, off);
+#pragma unroll
+        for (int e = 0; e < EV; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+      }
+      const int h = c.g * HG + w;
+      if (seg_from_start && seg_last) {  // whole segment in this CTA: final output
+        if (r == 0) {
+          const float inv = 1.f / lt;
+          float o[EV];
+#pragma unroll
+          for (int e = 0; e < EV; ++e) o[e] = acc[e] * inv;
+          IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(c.s) * p.H + h) * D + v * EV;
+          store_floats<IO, EV>(orow, o);
+        }
+      } else {  // partial state for the merge kernel
+        const long long slot = blockIdx.x + static_cast<long long>(c.s) * G + c.g;
+        if (r == 0) {
+          float4* dst = reinterpret_cast<float4*>(p.ws_acc + (slot * HG + w) * D + v * EV);
+#pragma unroll
+          for (int i = 0; i < EV / 4; ++i) dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+        }
+        if (lane == 0) {
+          p.ws_ml[(slot * HG + w) * 2 + 0] = m;
+          p.ws_ml[(slot * HG + w) * 2 + 1] = lt;
+        }
+      }
+      m = -FLT_MAX;
+      l = 0.f;
+#pragma unroll
+      for (int e = 0; e < EV; ++e) acc[e] = 0.f;
+    }
+    if (it + 1 < n) {
+      advance(c, p);
+      if (c.j == 0) {  // a new segment starts
+        seg_from_start = true;
+        load_q(c);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Merge kernel: one CTA per sequence; a warp per head combines the partial states of a
+// segment split across CTAs:  M = max m_k,  out = sum_k 2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k.
+// Segments of empty sequences get zeros; segments held by one CTA were already written.
+// ---------------------------------------------------------------------------------------
+template <typename IO, int D>
+__global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p) {
+  constexpr int DL = D / 32;  // dims per lane
+  const int s = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long per_group = p.ws_prefix[p.S];
+  const long long pre = p.ws_prefix[s];
+  const long long nb = p.ws_prefix[s + 1] - pre;
+  const long long T = per_group * p.G;
+  for (int h = warp; h < p.H; h += blockDim.x >> 5) {
+    IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(s) * p.H + h) * D + lane * DL;
+    float o[DL];
+    if (nb == 0) {
+#pragma unroll
+      for (int e = 0; e < DL; ++e) o[e] = 0.f;
+#pragma unroll
+      for (int e = 0; e < DL; ++e) orow[e] = float_to<IO>(o[e]);
+      continue;
+    }
+    const int g = h / p.HG, w = h % p.HG;
+    const long long a = p.G * pre + g * nb;
+    const int c0 = cta_of(a, T, p.num_ctas), c1 = cta_of(a + nb - 1, T, p.num_ctas);
+    if (c0 == c1) continue;
+    const long long seg = static_cast<long long>(s) * p.G + g;
+    float M = -FLT_MAX;
+    for (int k = c0; k <= c1; ++k) M = fmaxf(M, p.ws_ml[((k + seg) * p.HG + w) * 2]);
+    float L = 0.f;
+#pragma unroll
+    for (int e = 0; e < DL; ++e) o[e] = 0.f;
+    for (int k = c0; k <= c1; ++k) {
+      const long long slot = k + seg;
+      const float f = exp2f(p.ws_ml[(slot * p.HG + w) * 2] - M);
+      L += f * p.ws_ml[(slot * p.HG + w) * 2 + 1];
+      const float* src = p.ws_acc + (slot * p.HG + w) * D + lane * DL;
+#pragma unroll
+      for (int e = 0; e < DL; ++e) o[e] = fmaf(f, src[e], o[e]);
+    }
+    const float inv = 1.f / L;
+#pragma unroll
+    for (int e = 0; e < DL; ++e) orow[e] = float_to<IO>(o[e] * inv);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------------------
+namespace {
+
+cudaError_t read_decode_error(uint32_t* flags, int clear) {
+  unsigned int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_decode_error, sizeof v);
+  if (e != cudaSuccess) return e;
+  *flags = v;
+  if (clear && v) {
+    const unsigned int z = 0;
+    e = cudaMemcpyToSymbol(g_decode_error, &z, sizeof z);
+  }
+  return e;
+}
+
+struct RegisterDecode {
+  RegisterDecode() { register_device_error_reader(read_decode_error); }
+} g_register_decode;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+pa_status get_encoder(EncodeTiledFn* out) {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !ptr)
+      return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  *out = fn;
+  return PA_OK;
+}
+
+pa_status encode(EncodeTiledFn fn, CUtensorMap* map, CUtensorMapDataType type, int rank, const void* base,
+                 const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box) {
+  const cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = fn(map, type, rank, const_cast<void*>(base), dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+  return PA_OK;
+}
+
+size_t elem_bytes(pa_dtype t) { return t == PA_F32 ? 4 : (t == PA_I8 ? 1 : 2); }
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Workspace layout for `rows` = (partial slots x heads per slot) rows.
+struct WsLayout {
+  size_t prefix_off, ml_off, acc_off, total;
+};
+WsLayout ws_layout(int S, int D, long long rows) {
+  WsLayout l;
+  l.prefix_off = 0;
+  l.ml_off = align256(sizeof(long long) * (static_cast<size_t>(S) + 1));
+  l.acc_off = l.ml_off + align256(sizeof(float) * 2 * static_cast<size_t>(rows));
+  l.total = l.acc_off + align256(sizeof(float) * static_cast<size_t>(D) * rows);
+  return l;
+}
+
+// Heads per CTA: the largest power of two dividing H with K+V tiles of one stage <= 32 KiB.
+int pick_head_group(int H, int bs, int D, size_t e) {
+  int hg = kMaxHeadGroup;
+  while (hg > 1 && (H % hg != 0 || 2 * static_cast<size_t>(bs) * hg * D * e > 32768)) hg >>= 1;
+  return hg;
+}
+
+struct KernelInfo {
+  const void* fn = nullptr;
+  int smem_configured = 0;
+};
+
+template <typename IO, typename CT, int D>
+const void* partition_kernel_for(int bs) {
+  switch (bs) {
+    case 8: return reinterpret_cast<const void*>(&decode_partition_kernel<IO, CT, D, 8>);
+    case 16: return reinterpret_cast<const void*>(&decode_partition_kernel<IO, CT, D, 16>);
+    case 32: return reinterpret_cast<const void*>(&decode_partition_kernel<IO, CT, D, 32>);
+    default: return reinterpret_cast<const void*>(&decode_partition_kernel<IO, CT, D, 0>);
+  }
+}
+
+template <typename IO, typename CT>
+const void* partition_kernel_for(int D, int bs) {
+  return D == 64 ? partition_kernel_for<IO, CT, 64>(bs) : partition_kernel_for<IO, CT, 128>(bs);
+}
+
+const void* select_partition(pa_dtype io, pa_dtype cache, int D, int bs) {
+  if (cache == PA_I8) {
+    return io == PA_F16 ? partition_kernel_for<__half, int8_t>(D, bs)
+                        : partition_kernel_for<__nv_bfloat16, int8_t>(D, bs);
+  }
+  switch (io) {
+    case PA_F32: return partition_kernel_for<float, float>(D, bs);
+    case PA_F16: return partition_kernel_for<__half, __half>(D, bs);
+    default: return partition_kernel_for<__nv_bfloat16, __nv_bfloat16>(D, bs);
+  }
+}
+
+const void* select_merge(pa_dtype io, int D) {
+  switch (io) {
+    case PA_F32: return D == 64 ? reinterpret_cast<const void*>(&decode_merge_kernel<float, 64>)
+                                : reinterpret_cast<const void*>(&decode_merge_kernel<float, 128>);
+    case PA_F16: return D == 64 ? reinterpret_cast<const void*>(&decode_merge_kernel<__half, 64>)
+                                : reinterpret_cast<const void*>(&decode_merge_kernel<__half, 128>);
+    default: return D == 64 ? reinterpret_cast<const void*>(&decode_merge_kernel<__nv_bfloat16, 64>)
+                            : reinterpret_cast<const void*>(&decode_merge_kernel<__nv_bfloat16, 128>);
+  }
+}
+
+// Occupancy of a kernel at a given dynamic smem size, cached.
+pa_status occupancy(const void* fn, int threads, size_t smem, int* occ) {
+  struct Entry { const void* fn; int threads; size_t smem; int occ; };
+  static Entry cache[64];
+  static int used = 0;
+  for (int i = 0; i < used; ++i)
+    if (cache[i].fn == fn && cache[i].threads == threads && cache[i].smem == smem) {
+      *occ = cache[i].occ;
+      return PA_OK;
+    }
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(MaxDynamicSharedMemorySize)");
+  int o = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, fn, threads, smem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+  if (used < 64) cache[used++] = Entry{fn, threads, smem, o};
+  *occ = o;
+  return PA_OK;
+}
+
+bool valid_pair(pa_dtype io, pa_dtype cache) {
+  if (io == PA_F32) return cache == PA_F32;
+  if (io == PA_F16) return cache == PA_F16 || cache == PA_I8;
+  if (io == PA_BF16) return cache == PA_BF16 || cache == PA_I8;
+  return false;
+}
+
+}  // namespace
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim) {
+  if (num_seqs < 0 || num_heads <= 0 || (head_dim != 64 && head_dim != 128)) return 0;
+  int dev = 0, sms = 0;
+  if (current_device(&dev, &sms) != PA_OK) return 0;
+  const long long rows = static_cast<long long>(sms) * kMaxCtasPerSm * kMaxHeadGroup +
+                         static_cast<long long>(num_seqs) * num_heads;
+  return ws_layout(num_seqs, head_dim, rows).total;
+}
+
+extern "C" pa_status paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                            const void* k_scale, const void* v_scale, const int32_t* block_tables,
+                                            const int32_t* context_lens, int num_seqs, int num_heads, int head_dim,
+                                            int block_size, int num_blocks, int max_blocks_per_seq, float scale,
+                                            int window, pa_dtype io_dtype, pa_dtype cache_dtype, void* workspace,
+                                            size_t workspace_bytes, void* stream) {
+  // ---- host validation (no CUDA call before this block passes) ----
+  if (num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "num_seqs < 0");
+  if (num_heads <= 0 || num_heads > 4096) return fail(PA_ERR_INVALID_ARG, "num_heads must be in [1, 4096]");
+  if (head_dim != 64 && head_dim != 128) return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", head_dim);
+  if (block_size < 1 || block_size > 32) return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 1..32)", block_size);
+  if (num_blocks <= 0 || max_blocks_per_seq <= 0) return fail(PA_ERR_INVALID_ARG, "num_blocks and max_blocks_per_seq must be positive");
+  if (static_cast<long long>(num_blocks) * block_size > 0x7fffffffLL ||
+      static_cast<long long>(max_blocks_per_seq) * block_size > 0x7fffffffLL)
+    return fail(PA_ERR_INVALID_ARG, "num_blocks*block_size and max_blocks_per_seq*block_size must fit in int32");
+  if (window < 0) return fail(PA_ERR_INVALID_ARG, "window must be >= 0 (0 = full attention)");
+  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
+  if (!valid_pair(io_dtype, cache_dtype))
+    return fail(PA_ERR_INVALID_ARG, "dtype pair (io %d, cache %d) not supported: cache must equal io, or be PA_I8 with fp16/bf16 io",
+                static_cast<int>(io_dtype), static_cast<int>(cache_dtype));
+  const bool int8 = cache_dtype == PA_I8;
+  if (int8 && (num_heads % 8 != 0)) return fail(PA_ERR_UNSUPPORTED, "an INT8 cache needs num_heads to be a multiple of 8");
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !workspace)
+    return fail(PA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (int8 && (!k_scale || !v_scale)) return fail(PA_ERR_INVALID_ARG, "INT8 cache needs k_scale and v_scale");
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (int8 && (!aligned16(k_scale) || !aligned16(v_scale))) || !aligned16(workspace))
+    return fail(PA_ERR_INVALID_ARG, "tensor base addresses must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(block_tables) % 4 || reinterpret_cast<uintptr_t>(context_lens) % 4)
+    return fail(PA_ERR_INVALID_ARG, "block_tables / context_lens must be 4-byte aligned");
+
+  // ---- launch configuration ----
+  int dev = 0, sms = 0;
+  pa_status st = current_device(&dev, &sms);
+  if (st != PA_OK) return st;
+  const size_t need = pa_decode_workspace_bytes(num_seqs, num_heads, head_dim);
+  if (workspace_bytes < need)
+    return fail(PA_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+
+  const size_t e = elem_bytes(cache_dtype);
+  const int HG = pick_head_group(num_heads, block_size, head_dim, e);
+  const int G = num_heads / HG;
+  const uint32_t kv_tile = static_cast<uint32_t>(block_size) * HG * head_dim * e;
+  const uint32_t kv_tile_al = (kv_tile + 127u) & ~127u;
+  const uint32_t sc_tile = int8 ? static_cast<uint32_t>(block_size) * 8 * 2 : 0;
+  const uint32_t sc_tile_al = (sc_tile + 127u) & ~127u;
+  const uint32_t stage_bytes = 2 * kv_tile_al + 2 * sc_tile_al;
+  int nstage = static_cast<int>((96 * 1024) / stage_bytes);
+  nstage = nstage < 2 ? 2 : (nstage > 8 ? 8 : nstage);
+  const size_t smem = kBarrierBytes + 128 + static_cast<size_t>(nstage) * stage_bytes;
+  const int threads = 32 * (HG + 1);
+
+  const void* part_fn = select_partition(io_dtype, cache_dtype, head_dim, block_size);
+  const void* merge_fn = select_merge(io_dtype, head_dim);
+  int occ = 0;
+  st = occupancy(part_fn, threads, smem, &occ);
+  if (st != PA_OK) return st;
+  if (occ <= 0) return fail(PA_ERR_CUDA, "partition kernel cannot be resident (smem %zu)", smem);
+  const int C = sms * (occ < kMaxCtasPerSm ? occ : kMaxCtasPerSm);
+
+  const long long rows = static_cast<long long>(C) * HG + static_cast<long long>(num_seqs) * num_heads;
+  const WsLayout lay = ws_layout(num_seqs, head_dim, rows);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  // ---- tensor maps ----
+  EncodeTiledFn enc = nullptr;
+  st = get_encoder(&enc);
+  if (st != PA_OK) return st;
+  const CUtensorMapDataType ttype = cache_dtype == PA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                  : cache_dtype == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                  : cache_dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                           : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  CUtensorMap tmK, tmV, tmKs, tmVs;
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_heads),
+                                static_cast<cuuint64_t>(num_blocks) * block_size};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * e, static_cast<cuuint64_t>(num_heads) * head_dim * e};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(head_dim), static_cast<cuuint32_t>(HG),
+                               static_cast<cuuint32_t>(block_size)};
+    if ((st = encode(enc, &tmK, ttype, 3, k_cache, dims, strides, box)) != PA_OK) return st;
+    if ((st = encode(enc, &tmV, ttype, 3, v_cache, dims, strides, box)) != PA_OK) return st;
+  }
+  if (int8) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(num_heads), static_cast<cuuint64_t>(num_blocks) * block_size};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(num_heads) * 2};
+    const cuuint32_t box[2] = {8, static_cast<cuuint32_t>(block_size)};
+    if ((st = encode(enc, &tmKs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, k_scale, dims, strides, box)) != PA_OK) return st;
+    if ((st = encode(enc, &tmVs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, v_scale, dims, strides, box)) != PA_OK) return st;
+  } else {
+    tmKs = tmK;
+    tmVs = tmV;
+  }
+
+  DecodeParams prm;
+  prm.out = out;
+  prm.q = q;
+  prm.block_tables = block_tables;
+  prm.context_lens = context_lens;
+  prm.ws_prefix = reinterpret_cast<long long*>(ws + lay.prefix_off);
+  prm.ws_ml = reinterpret_cast<float*>(ws + lay.ml_off);
+  prm.ws_acc = reinterpret_cast<float*>(ws + lay.acc_off);
+  prm.S = num_seqs;
+  prm.H = num_heads;
+  prm.bs = block_size;
+  prm.MB = max_blocks_per_seq;
+  prm.NB = num_blocks;
+  prm.window = window;
+  prm.HG = HG;
+  prm.G = G;
+  prm.num_ctas = C;
+  prm.nstage = nstage;
+  prm.qscale = scale * 1.4426950408889634f;  // log2(e): exp(x) = 2^(x log2 e)
+  prm.stage_bytes = stage_bytes;
+  prm.v_off = kv_tile_al;
+  prm.ks_off = 2 * kv_tile_al;
+  prm.vs_off = 2 * kv_tile_al + sc_tile_al;
+  prm.tx_bytes = 2 * kv_tile + 2 * sc_tile;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaEvent_t ev[3];
+  profiling_next_events(ev);
+  if (ev[0]) cudaEventRecord(ev[0], s);
+
+  {
+    void* args[] = {&tmK, &tmV, &tmKs, &tmVs, &prm};
+    cudaError_t err = cudaLaunchKernel(part_fn, dim3(C), dim3(threads), args, smem, s);
+    if (err != cudaSuccess) return cuda_fail(err, "launching the decode partition kernel");
+  }
+  if (ev[1]) cudaEventRecord(ev[1], s);
+  {
+    void* args[] = {&prm};
+    cudaError_t err = cudaLaunchKernel(merge_fn, dim3(num_seqs), dim3(128), args, 0, s);
+    if (err != cudaSuccess) return cuda_fail(err, "launching the decode merge kernel");
+  }
+  if (ev[2]) cudaEventRecord(ev[2], s);
+  return PA_OK;
+}

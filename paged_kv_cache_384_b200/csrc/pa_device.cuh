@@ -1,0 +1,202 @@
+// pa_device.cuh -- device-side building blocks shared by the sm_100a kernels:
+// element traits, 16-byte vector conversion, mbarrier + TMA wrappers (inline PTX) and the
+// device error word.  Internal header; not part of the C ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/pagedattn.h"
+
+namespace pa {
+
+// ---------------------------------------------------------------------------------------
+// Device error word (OR of PA_DEVERR_* bits), one per device per process.
+// ---------------------------------------------------------------------------------------
+extern __device__ unsigned int g_device_error;
+
+__device__ __forceinline__ void raise_device_error(unsigned int bits) {
+  atomicOr(&g_device_error, bits);
+}
+
+// ---------------------------------------------------------------------------------------
+// Element traits.  A 16-byte vector holds EV elements; `to_float` widens EV elements of a
+// vector held as 4 x uint32.
+// ---------------------------------------------------------------------------------------
+template <typename T> struct Elem;
+
+template <> struct Elem<float> {
+  static constexpr int kBytes = 4;
+  static constexpr int kEV = 4;
+  static __device__ __forceinline__ void to_float(const uint4& v, float* f) {
+    f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+  }
+  static __device__ __forceinline__ float from_float_store(float x) { return x; }
+};
+
+template <> struct Elem<__half> {
+  static constexpr int kBytes = 2;
+  static constexpr int kEV = 8;
+  static __device__ __forceinline__ void to_float(const uint4& v, float* f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __half2 h = *reinterpret_cast<const __half2*>(&w[i]);
+      float2 p = __half22float2(h);
+      f[2 * i] = p.x; f[2 * i + 1] = p.y;
+    }
+  }
+};
+
+template <> struct Elem<__nv_bfloat16> {
+  static constexpr int kBytes = 2;
+  static constexpr int kEV = 8;
+  // bf16 is the upper half of a binary32: widening is a shift / mask, exact.
+  static __device__ __forceinline__ void to_float(const uint4& v, float* f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+};
+
+template <> struct Elem<int8_t> {
+  static constexpr int kBytes = 1;
+  static constexpr int kEV = 16;
+  // Exact int8 -> fp32 without the (quarter-rate) integer-convert pipe: flip the sign bit
+  // so the byte reads as c + 128 in [0, 255], splice it under the exponent of 2^23
+  // (0x4B000000 | b is the float 2^23 + b), then subtract 2^23 + 128.  One byte-permute
+  // and one FADD per element, both exact.
+  static __device__ __forceinline__ void to_float(const uint4& v, float* f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t u = w[i] ^ 0x80808080u;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const uint32_t bits = __byte_perm(u, 0x4B000000u, 0x7440u | b);
+        f[4 * i + b] = __uint_as_float(bits) - 8388736.0f;
+      }
+    }
+  }
+};
+
+template <typename T> __device__ __forceinline__ T float_to(float x);
+template <> __device__ __forceinline__ float float_to<float>(float x) { return x; }
+template <> __device__ __forceinline__ __half float_to<__half>(float x) { return __float2half_rn(x); }
+template <> __device__ __forceinline__ __nv_bfloat16 float_to<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// ---------------------------------------------------------------------------------------
+// Shared-memory addresses, mbarrier and TMA (cp.async.bulk.tensor) wrappers.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Every wait is bounded.  try_wait already suspends the thread for a hardware-chosen
+// interval per attempt, so this limit ends a wait that can never complete (a library
+// bug) after well under a minute; the caller then records PA_DEVERR_TIMEOUT and unwinds.
+constexpr uint32_t kWaitLimit = 1u << 22;
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// 3-D tiled TMA load global -> shared, completion counted on `bar` (transaction bytes).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int x, int y, int z, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+// 2-D tiled TMA load global -> shared.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int x, int y, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// L2 policy for data read exactly once (the K/V stream): evict first.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint16_t ld_shared_u16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+
+// Programmatic dependent launch: wait for the preceding kernel's memory, and let the next
+// kernel of the stream start its prologue early.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_launch_next() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+}  // namespace pa
