@@ -48,7 +48,7 @@ SIGNATURES = {
 def load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_384_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python paged_kv_cache_384_b200/build.py` "
             "(there is no CPU fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in SIGNATURES.items():

@@ -1,6 +1,6 @@
 """Build ``libpagedattn.so`` in-tree from ``csrc/`` with nvcc for sm_100a.
 
-    python -m paged_kv_cache_384_b200.build [--force]
+    python paged_kv_cache_384_b200/build.py [--force]
 
 Sources compile in parallel to objects under ``_build/``; the library links the CUDA
 runtime statically, so it depends only on the driver at run time.  ptxas resource usage
