@@ -130,6 +130,35 @@ pa_status paged_attention_decode(void* out, const void* q, const void* k_cache,
                                  pa_dtype io_dtype, pa_dtype cache_dtype, void* workspace,
                                  size_t workspace_bytes, void* stream);
 
+/*
+ * paged_attention_decode for callers that cannot allocate device memory.  No counterpart
+ * on the pages: it exists for callers with no device allocator of their own -- e.g. a
+ * plugin inside a host framework that owns all device memory and passes only the op's
+ * tensors, or a latency-critical loop that cannot afford cudaMalloc's implicit device
+ * synchronisation.
+ *
+ * Same arguments and results as paged_attention_decode, minus the workspace.  The
+ * scratch is a fixed 16 MiB array inside the library's device memory, present on every
+ * GPU that loads the library until the process exits; this call allocates nothing.
+ *   - Batches whose pa_decode_workspace_bytes() exceeds 16 MiB are rejected with
+ *     PA_ERR_INVALID_ARG (nothing is launched).
+ *   - The first call on a device looks up the array's device address (once per device,
+ *     with that device current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array: calls that may overlap on the GPU
+ *     (different streams, no ordering between them) race and corrupt each other's
+ *     results.  Calls ordered on one stream are fine.
+ *   - The array keeps the last call's contents; the kernels overwrite every part of it
+ *     that they read, so nothing has to be cleared between calls.
+ */
+pa_status paged_attention_decode_static_scratch(void* out, const void* q, const void* k_cache,
+                                                const void* v_cache, const void* k_scale,
+                                                const void* v_scale, const int32_t* block_tables,
+                                                const int32_t* context_lens, int num_seqs,
+                                                int num_heads, int head_dim, int block_size,
+                                                int num_blocks, int max_blocks_per_seq, float scale,
+                                                int window, pa_dtype io_dtype, pa_dtype cache_dtype,
+                                                void* stream);
+
 /* ------------------------------------------------------------------------------------ */
 /* Cache maintenance                                                                    */
 /* ------------------------------------------------------------------------------------ */

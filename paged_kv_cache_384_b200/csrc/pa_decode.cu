@@ -24,6 +24,7 @@
 //     have nothing dense to do with a single query row per head.
 #include <cfloat>
 #include <cstdio>
+#include <mutex>
 #include <type_traits>
 
 #include "pa_device.cuh"
@@ -766,4 +767,66 @@ extern "C" pa_status paged_attention_decode(void* out, const void* q, const void
   }
   if (ev[2]) cudaEventRecord(ev[2], s);
   return PA_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// Decode without a caller-provided workspace.
+//
+// Some callers cannot call cudaMalloc: a plugin living inside a host framework that owns
+// every byte of device memory and hands out nothing but the tensors of the op, or a
+// latency-critical loop where cudaMalloc's implicit device synchronisation is not
+// acceptable.  For them the split-softmax scratch lives in a fixed array in the library's
+// own device memory (kStaticScratchBytes on every GPU that loads the library, held until
+// the process exits).  The array's host-side name is only a stand-in for it, so its device
+// address is looked up once per device with cudaGetSymbolAddress (on the first call on
+// that device, which must therefore come before any stream capture) and that address is
+// handed to paged_attention_decode.
+// ---------------------------------------------------------------------------------------
+namespace pa {
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+pa_status static_scratch_address(void** out) {
+  static std::mutex m;
+  static void* addr[256] = {nullptr};
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 256) return fail(PA_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(m);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static decode scratch)");
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return PA_OK;
+}
+
+}  // namespace
+}  // namespace pa
+
+extern "C" pa_status paged_attention_decode_static_scratch(
+    void* out, const void* q, const void* k_cache, const void* v_cache, const void* k_scale, const void* v_scale,
+    const int32_t* block_tables, const int32_t* context_lens, int num_seqs, int num_heads, int head_dim,
+    int block_size, int num_blocks, int max_blocks_per_seq, float scale, int window, pa_dtype io_dtype,
+    pa_dtype cache_dtype, void* stream) {
+  if (num_seqs == 0) return PA_OK;
+  const size_t need = pa_decode_workspace_bytes(num_seqs, num_heads, head_dim);
+  if (need == 0)
+    return fail(PA_ERR_INVALID_ARG, "paged_attention_decode_static_scratch: invalid sizes or no CUDA device");
+  if (need > kStaticScratchBytes)
+    return fail(PA_ERR_INVALID_ARG,
+                "paged_attention_decode_static_scratch: %d sequences x %d heads x %d dims need %zu bytes of "
+                "scratch, above the built-in %zu; use paged_attention_decode with a workspace",
+                num_seqs, num_heads, head_dim, need, kStaticScratchBytes);
+  void* scratch = nullptr;
+  pa_status st = static_scratch_address(&scratch);
+  if (st != PA_OK) return st;
+  return paged_attention_decode(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, num_seqs,
+                                num_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, scale, window,
+                                io_dtype, cache_dtype, scratch, kStaticScratchBytes, stream);
 }
