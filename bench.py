@@ -87,48 +87,73 @@ def kernel_traffic(kernel_source: str):
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock / throttle reasons while the timed region runs."""
+    """nvidia-smi samples (every 100 ms) of SM clock, power and throttle reasons.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    ``mark()`` is called when the timed region starts; ``summary()`` keeps only samples
+    taken after it (the timed region plus, when it is shorter than a second, an untimed
+    soak of the same steps that follows it, so that there is something to sample).
+    """
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
-        self.idx = device_index
+    def __init__(self, device_id: str):
+        self.idx = device_id
         self.proc = None
+        self.lines = []
+        self.t_mark = None
 
     def __enter__(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="pa_clocks_", suffix=".csv")
+        os.close(fd)
         try:
+            # -f: nvidia-smi writes each sample line itself (a pipe would buffer them away)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "100", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
         except OSError:
             self.proc = None
         return self
 
+    def mark(self):
+        import datetime
+        self.t_mark = datetime.datetime.now()
+
     def __exit__(self, *exc):
-        self.lines = []
         if self.proc is not None:
-            self.proc.terminate()
+            time.sleep(0.15)
+            self.proc.send_signal(2)
             try:
-                out, _ = self.proc.communicate(timeout=10)
+                self.proc.wait(timeout=10)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+                self.proc.wait()
+        try:
+            with open(self.path) as f:
+                self.lines = [l for l in f.read().splitlines() if l.strip()]
+            os.unlink(self.path)
+        except OSError:
+            self.lines = []
         return False
 
     def summary(self):
+        import datetime
         rows = []
-        for line in getattr(self, "lines", []):
+        for line in self.lines:
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
             try:
-                rows.append(dict(sm=float(f[1]), max=float(f[2]), power=float(f[3]),
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f")
+                rows.append(dict(ts=ts, sm=float(f[1]), max=float(f[2]), power=float(f[3]),
                                  hw=f[5], hwt=f[6], swt=f[7], pcap=f[8]))
             except ValueError:
                 continue
+        if self.t_mark is not None:
+            rows = [r for r in rows if r["ts"] >= self.t_mark]
         if not rows:
             return None
         reasons = set()
@@ -138,7 +163,8 @@ class ClockSampler:
                 if r[key].lower() == "active":
                     reasons.add(name)
         return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["max"] for r in rows),
-                "samples": len(rows), "reasons": sorted(reasons)}
+                "samples": len(rows), "power_w_median": statistics.median(r["power"] for r in rows),
+                "reasons": sorted(reasons)}
 
 
 # ---------------------------------------------------------------------------------------
@@ -168,6 +194,79 @@ def step(pa, w, d, stream):
         pa.copy_blocks(d["k_cache"], d["v_cache"], d["pairs"], stream=stream)
     pa.paged_attention_decode(d["out"], d["q"], d["k_cache"], d["v_cache"], d["block_tables"],
                               d["context_lens"], w.scale, w.window, workspace=d["ws"], stream=stream)
+
+
+class PackedInputs:
+    """A step's per-request inputs packed into one pinned host buffer and one device
+    buffer (256-byte aligned fields), so they cross PCIe in a single copy."""
+
+    def __init__(self, host: dict, device):
+        self.layout, off = {}, 0
+        for k, t in host.items():
+            n = t.numel() * t.element_size()
+            self.layout[k] = (off, t.dtype, tuple(t.shape))
+            off = (off + n + 255) // 256 * 256
+        self.nbytes = off
+        self.h = torch.zeros(off, dtype=torch.uint8).pin_memory()
+        for k, t in host.items():
+            o, _, _ = self.layout[k]
+            n = t.numel() * t.element_size()
+            self.h[o:o + n].copy_(t.contiguous().view(-1).view(torch.uint8))
+        self.d = torch.empty(off, dtype=torch.uint8, device=device)
+
+    def views(self):
+        out = {}
+        for k, (o, dt, shape) in self.layout.items():
+            n = math.prod(shape) * torch.empty((), dtype=dt).element_size()
+            out[k] = self.d[o:o + n].view(dt).view(shape)
+        return out
+
+
+def run_e2e(pa, w, d, host, args, device, stream, barrier):
+    """Steps through the public API with inputs in pinned host memory and the result read
+    back every step.  Two input/output buffer sets and a copy stream pipeline the
+    transfers: the inputs of step i+1 cross PCIe while step i computes."""
+    sets = [PackedInputs(host, device) for _ in range(2)]
+    outs_h = [torch.empty(d["out"].shape, dtype=d["out"].dtype).pin_memory() for _ in range(2)]
+    outs_d = [torch.empty_like(d["out"]) for _ in range(2)]
+    copy = torch.cuda.Stream(device)
+    h2d = sets[0].nbytes
+    d2h = outs_h[0].numel() * outs_h[0].element_size()
+    dd = [dict(d, **s.views()) for s in sets]
+    for i in range(2):
+        dd[i]["out"] = outs_d[i]
+
+    def run(n):
+        ready = [torch.cuda.Event() for _ in range(2)]     # inputs of set i on the device
+        done = [torch.cuda.Event() for _ in range(2)]      # step on set i finished
+        copy.wait_stream(stream)                           # no transfer starts before the timer
+        with torch.cuda.stream(copy):
+            sets[0].d.copy_(sets[0].h, non_blocking=True)
+            ready[0].record(copy)
+        for i in range(n):
+            b = i % 2
+            stream.wait_event(ready[b])
+            step(pa, w, dd[b], stream)
+            done[b].record(stream)
+            with torch.cuda.stream(copy):
+                if i + 1 < n:                               # prefetch the next step's inputs
+                    nb = (i + 1) % 2
+                    if i >= 1:
+                        copy.wait_event(done[nb])
+                    sets[nb].d.copy_(sets[nb].h, non_blocking=True)
+                    ready[nb].record(copy)
+                copy.wait_event(done[b])
+                outs_h[b].copy_(outs_d[b], non_blocking=True)  # read the result back
+        stream.wait_stream(copy)
+
+    run(args.warmup)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    run(args.steps)
+    e1.record(stream)
+    barrier()
+    return e0.elapsed_time(e1) / 1e3, h2d, d2h
 
 
 def launches_per_step(d) -> int:
@@ -252,12 +351,17 @@ def run_ours(args):
     props = torch.cuda.get_device_properties(device)
     smi_id = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
     with ClockSampler(smi_id) as clocks:
+        clocks.mark()
         start.record(stream)
         for _ in range(args.steps):
             step(pa, w, d, stream)
         end.record(stream)
         barrier()
-    sec = start.elapsed_time(end) / 1e3
+        sec = start.elapsed_time(end) / 1e3
+        soak = max(0, int((1.0 - sec) / max(sec / args.steps, 1e-6)))  # same steps, untimed
+        for _ in range(soak):
+            step(pa, w, d, stream)
+        torch.cuda.synchronize(device)
     sec_max = reduce_max(sec, dist)
     all_bytes = [kv_bytes] * world if dist is None else None
     if dist is not None:
@@ -284,27 +388,8 @@ def run_ours(args):
     traffic = kernel_traffic(os.path.join(ROOT, "paged_kv_cache_384_b200", "csrc", "pa_decode.cu"))
 
     # ---- end to end through the public API with host buffers ----
-    pin = {k: v.pin_memory() for k, v in host.items()}
-    out_host = torch.empty(d["out"].shape, dtype=d["out"].dtype).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in pin.values())
-    d2h = out_host.numel() * out_host.element_size()
-
-    def e2e_step():
-        for k, v in pin.items():
-            d[k].copy_(v, non_blocking=True)
-        step(pa, w, d, stream)
-        out_host.copy_(d["out"], non_blocking=True)
-
-    for _ in range(args.warmup):
-        e2e_step()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    barrier()
-    e2e_sec = reduce_max(e0.elapsed_time(e1) / 1e3, dist)
+    e2e_sec, h2d, d2h = run_e2e(pa, w, d, host, args, device, stream, barrier)
+    e2e_sec = reduce_max(e2e_sec, dist)
     e2e_value = whole_job_gbs(all_bytes, args.steps, e2e_sec)
 
     # ---- CPU baseline: the oracle on this batch, rank 0 at N = 1 only ----
@@ -346,7 +431,7 @@ def run_ours(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)

@@ -24,6 +24,8 @@ reshape_and_cache_kernel(const uint8_t* __restrict__ k, const uint8_t* __restric
                          long long k_stride_bytes, long long v_stride_bytes, long long num_slots,
                          const uint16_t* __restrict__ ks_src, const uint16_t* __restrict__ vs_src,
                          uint16_t* __restrict__ ks_cache, uint16_t* __restrict__ vs_cache, int H) {
+  grid_dependency_launch_next();
+  grid_dependency_wait();  // launched as a programmatic dependent: inputs may come from the previous kernel
   const int t = blockIdx.y;
   const long long slot = __ldg(slots + t);
   if (slot < 0) return;  // padding token
@@ -56,6 +58,8 @@ template <int VEC>
 __global__ void __launch_bounds__(256)
 copy_blocks_kernel(uint8_t* k, uint8_t* v, uint8_t* ks, uint8_t* vs, const int64_t* __restrict__ pairs,
                    long long block_bytes, long long scale_block_bytes, long long num_blocks) {
+  grid_dependency_launch_next();
+  grid_dependency_wait();
   const int pool = blockIdx.z;  // 0: K, 1: V, 2: K scales, 3: V scales
   const long long src = __ldg(pairs + 2 * blockIdx.y), dst = __ldg(pairs + 2 * blockIdx.y + 1);
   if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
@@ -147,13 +151,21 @@ extern "C" pa_status reshape_and_cache(const void* k, const void* v, void* k_cac
   const long long nvec = row_bytes / 16;
   const int threads = 256;
   dim3 grid(static_cast<unsigned>((nvec + threads - 1) / threads), static_cast<unsigned>(num_tokens));
-  reshape_and_cache_kernel<<<grid, threads, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint8_t*>(k), static_cast<const uint8_t*>(v), static_cast<uint8_t*>(k_cache),
-      static_cast<uint8_t*>(v_cache), slot_mapping, row_bytes, k_token_stride * static_cast<long long>(e),
-      v_token_stride * static_cast<long long>(e), static_cast<long long>(num_blocks) * block_size,
-      static_cast<const uint16_t*>(k_scale_src), static_cast<const uint16_t*>(v_scale_src),
-      static_cast<uint16_t*>(k_scale_cache), static_cast<uint16_t*>(v_scale_cache), num_heads);
-  cudaError_t err = cudaGetLastError();
+  const uint8_t* kp = static_cast<const uint8_t*>(k);
+  const uint8_t* vp = static_cast<const uint8_t*>(v);
+  uint8_t* kcp = static_cast<uint8_t*>(k_cache);
+  uint8_t* vcp = static_cast<uint8_t*>(v_cache);
+  long long kst = k_token_stride * static_cast<long long>(e), vst = v_token_stride * static_cast<long long>(e);
+  long long nslots = static_cast<long long>(num_blocks) * block_size;
+  const uint16_t* kss = static_cast<const uint16_t*>(k_scale_src);
+  const uint16_t* vss = static_cast<const uint16_t*>(v_scale_src);
+  uint16_t* ksc = static_cast<uint16_t*>(k_scale_cache);
+  uint16_t* vsc = static_cast<uint16_t*>(v_scale_cache);
+  int H = num_heads;
+  long long rb = row_bytes;
+  void* args[] = {&kp, &vp, &kcp, &vcp, &slot_mapping, &rb, &kst, &vst, &nslots, &kss, &vss, &ksc, &vsc, &H};
+  cudaError_t err = launch_dependent(reinterpret_cast<const void*>(&reshape_and_cache_kernel), grid, dim3(threads), 0,
+                                     static_cast<cudaStream_t>(stream), args);
   if (err != cudaSuccess) return cuda_fail(err, "launching reshape_and_cache");
   return PA_OK;
 }
@@ -177,18 +189,16 @@ extern "C" pa_status copy_blocks(void* k_cache, void* v_cache, const int64_t* sr
   const long long longest = static_cast<long long>(block_bytes > scale_block_bytes ? block_bytes : scale_block_bytes);
   dim3 grid(static_cast<unsigned>((longest + per_cta - 1) / per_cta), static_cast<unsigned>(num_pairs), scales ? 4u : 2u);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (vec_ok) {
-    copy_blocks_kernel<16><<<grid, threads, 0, s>>>(
-        static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache), static_cast<uint8_t*>(k_scale_cache),
-        static_cast<uint8_t*>(v_scale_cache), src_dst_pairs, static_cast<long long>(block_bytes),
-        static_cast<long long>(scale_block_bytes), num_blocks);
-  } else {
-    copy_blocks_kernel<1><<<grid, threads, 0, s>>>(
-        static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache), static_cast<uint8_t*>(k_scale_cache),
-        static_cast<uint8_t*>(v_scale_cache), src_dst_pairs, static_cast<long long>(block_bytes),
-        static_cast<long long>(scale_block_bytes), num_blocks);
-  }
-  cudaError_t err = cudaGetLastError();
+  uint8_t* kp = static_cast<uint8_t*>(k_cache);
+  uint8_t* vp = static_cast<uint8_t*>(v_cache);
+  uint8_t* ksp = static_cast<uint8_t*>(k_scale_cache);
+  uint8_t* vsp = static_cast<uint8_t*>(v_scale_cache);
+  long long bb = static_cast<long long>(block_bytes), sb = static_cast<long long>(scale_block_bytes);
+  long long nb = num_blocks;
+  void* args[] = {&kp, &vp, &ksp, &vsp, &src_dst_pairs, &bb, &sb, &nb};
+  const void* fn = vec_ok ? reinterpret_cast<const void*>(&copy_blocks_kernel<16>)
+                          : reinterpret_cast<const void*>(&copy_blocks_kernel<1>);
+  cudaError_t err = launch_dependent(fn, grid, dim3(threads), 0, s, args);
   if (err != cudaSuccess) return cuda_fail(err, "launching copy_blocks");
   return PA_OK;
 }

@@ -160,6 +160,11 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nthr = blockDim.x;
 
+  // Programmatic dependent launch: let the merge kernel get resident now, and wait for
+  // the previous kernel of the stream (e.g. the cache write) before reading anything.
+  grid_dependency_launch_next();
+  grid_dependency_wait();
+
   // ---- 1. Plan: tiles per sequence, their prefix sum, and this CTA's slice. -----------
   const int chunk = (p.S + nthr - 1) / nthr;
   const int s_lo = min(p.S, threadIdx.x * chunk), s_hi = min(p.S, s_lo + chunk);
@@ -427,51 +432,60 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
 }
 
 // ---------------------------------------------------------------------------------------
-// Merge kernel: one CTA per sequence; a warp per head combines the partial states of a
-// segment split across CTAs:  M = max m_k,  out = sum_k 2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k.
-// Segments of empty sequences get zeros; segments held by one CTA were already written.
+// Merge kernel: one warp per (sequence, head) combines the partial states of a segment that
+// was split across CTAs:  M = max_k m_k,  out = sum_k 2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k.
+// Sequences with nothing to attend get zeros; segments held by one CTA were written by it.
+// Launched as a programmatic dependent of the partition kernel: the grid is resident while
+// the partition kernel runs and proceeds the moment its results are visible.
 // ---------------------------------------------------------------------------------------
+constexpr int kMergeWarps = 8;
+
 template <typename IO, int D>
-__global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const DecodeParams p) {
   constexpr int DL = D / 32;  // dims per lane
-  const int s = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  grid_dependency_wait();
+  const int lane = threadIdx.x & 31;
+  const long long item = static_cast<long long>(blockIdx.x) * kMergeWarps + (threadIdx.x >> 5);
+  if (item >= static_cast<long long>(p.S) * p.H) return;
+  const int s = static_cast<int>(item / p.H), h = static_cast<int>(item % p.H);
   const long long per_group = p.ws_prefix[p.S];
   const long long pre = p.ws_prefix[s];
   const long long nb = p.ws_prefix[s + 1] - pre;
-  const long long T = per_group * p.G;
-  for (int h = warp; h < p.H; h += blockDim.x >> 5) {
-    IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(s) * p.H + h) * D + lane * DL;
-    float o[DL];
-    if (nb == 0) {
+  IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(s) * p.H + h) * D + lane * DL;
+  float o[DL];
 #pragma unroll
-      for (int e = 0; e < DL; ++e) o[e] = 0.f;
+  for (int e = 0; e < DL; ++e) o[e] = 0.f;
+  if (nb == 0) {
 #pragma unroll
-      for (int e = 0; e < DL; ++e) orow[e] = float_to<IO>(o[e]);
-      continue;
-    }
-    const int g = h / p.HG, w = h % p.HG;
-    const long long a = p.G * pre + g * nb;
-    const int c0 = cta_of(a, T, p.num_ctas), c1 = cta_of(a + nb - 1, T, p.num_ctas);
-    if (c0 == c1) continue;
-    const long long seg = static_cast<long long>(s) * p.G + g;
-    float M = -FLT_MAX;
-    for (int k = c0; k <= c1; ++k) M = fmaxf(M, p.ws_ml[((k + seg) * p.HG + w) * 2]);
-    float L = 0.f;
-#pragma unroll
-    for (int e = 0; e < DL; ++e) o[e] = 0.f;
-    for (int k = c0; k <= c1; ++k) {
-      const long long slot = k + seg;
-      const float f = exp2f(p.ws_ml[(slot * p.HG + w) * 2] - M);
-      L += f * p.ws_ml[(slot * p.HG + w) * 2 + 1];
-      const float* src = p.ws_acc + (slot * p.HG + w) * D + lane * DL;
-#pragma unroll
-      for (int e = 0; e < DL; ++e) o[e] = fmaf(f, src[e], o[e]);
-    }
-    const float inv = 1.f / L;
-#pragma unroll
-    for (int e = 0; e < DL; ++e) orow[e] = float_to<IO>(o[e] * inv);
+    for (int e = 0; e < DL; ++e) orow[e] = float_to<IO>(0.f);
+    return;
   }
+  const long long T = per_group * p.G;
+  const int g = h / p.HG, w = h % p.HG;
+  const long long a = p.G * pre + g * nb;
+  const int c0 = cta_of(a, T, p.num_ctas), c1 = cta_of(a + nb - 1, T, p.num_ctas);
+  if (c0 == c1) return;
+  const long long seg = static_cast<long long>(s) * p.G + g;
+  const float2* ml = reinterpret_cast<const float2*>(p.ws_ml);
+  // Global max over the partials, 32 partials per round (one per lane).
+  float M = -FLT_MAX;
+  for (int k = c0 + lane; k <= c1; k += 32) M = fmaxf(M, ml[(k + seg) * p.HG + w].x);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  float L = 0.f;
+#pragma unroll 4
+  for (int k = c0; k <= c1; ++k) {
+    const long long row = (k + seg) * p.HG + w;
+    const float2 st = ml[row];
+    const float f = exp2f(st.x - M);
+    L = fmaf(f, st.y, L);
+    const float* src = p.ws_acc + row * D + lane * DL;
+#pragma unroll
+    for (int e = 0; e < DL; ++e) o[e] = fmaf(f, src[e], o[e]);
+  }
+  const float inv = 1.f / L;
+#pragma unroll
+  for (int e = 0; e < DL; ++e) orow[e] = float_to<IO>(o[e] * inv);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -756,13 +770,15 @@ extern "C" pa_status paged_attention_decode(void* out, const void* q, const void
 
   {
     void* args[] = {&tmK, &tmV, &tmKs, &tmVs, &prm};
-    cudaError_t err = cudaLaunchKernel(part_fn, dim3(C), dim3(threads), args, smem, s);
+    cudaError_t err = launch_dependent(part_fn, dim3(C), dim3(threads), smem, s, args);
     if (err != cudaSuccess) return cuda_fail(err, "launching the decode partition kernel");
   }
   if (ev[1]) cudaEventRecord(ev[1], s);
   {
     void* args[] = {&prm};
-    cudaError_t err = cudaLaunchKernel(merge_fn, dim3(num_seqs), dim3(128), args, 0, s);
+    const long long items = static_cast<long long>(num_seqs) * num_heads;
+    const unsigned grid = static_cast<unsigned>((items + kMergeWarps - 1) / kMergeWarps);
+    cudaError_t err = launch_dependent(merge_fn, dim3(grid), dim3(32 * kMergeWarps), 0, s, args);
     if (err != cudaSuccess) return cuda_fail(err, "launching the decode merge kernel");
   }
   if (ev[2]) cudaEventRecord(ev[2], s);

@@ -23,6 +23,12 @@ pa_status current_device(int* device, int* sm_count);
 using DeviceErrorReader = cudaError_t (*)(uint32_t* flags, int clear);
 void register_device_error_reader(DeviceErrorReader reader);
 
+// Launch `fn` as a programmatic dependent of the previous kernel on `stream`: it may be
+// scheduled before that kernel finishes; the kernel itself must execute
+// griddepcontrol.wait before touching memory the previous kernel may write.
+cudaError_t launch_dependent(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             void** args);
+
 // Profiling hooks used by paged_attention_decode.
 bool profiling_enabled();
 // Returns three events (before partition, between kernels, after merge) to record, or
