@@ -34,6 +34,9 @@ import synth  # noqa: E402
 from paged_kv_cache_384_b200 import accounting  # noqa: E402
 
 PRESET = "llama70b_fp16"
+CONTEXT_DESC = {"llama70b_fp16": "uniform [1, 2048]",
+                "chat_prefix_bf16": "2000 shared + lognormal(median 300, sigma 1) tail, 64 copy-on-write forks",
+                "sliding_window_fp16": "32768 each, window 4096"}
 METRIC = "paged decode attention KV GB/s (% of B200 HBM peak) and tokens/s per layer"
 FALLBACK_HBM_GBS = 6650.0
 
@@ -170,12 +173,14 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------------
 # workload
 # ---------------------------------------------------------------------------------------
-def build(seed: int, device):
+def build(seed: int, device, workload: str = PRESET, block_size=None):
     import paged_kv_cache_384_b200 as pa
-    w = synth.build_workload(PRESET, seed, pa.BlockManager)
+    over = {} if block_size is None else {"block_size": block_size}
+    big = workload == "sliding_window_fp16"          # 8.6 GB of cache: draw values on the GPU
+    w = synth.build_workload(workload, seed, pa.BlockManager, device=device if big else "cpu", **over)
     ctx = w.context_lens.tolist()
     slots = pa.slot_mapping(w.block_tables, range(w.num_seqs), [c - 1 for c in ctx], w.block_size)
-    host = dict(q=w.q, k_new=w.k_new, v_new=w.v_new, slots=slots, block_tables=w.block_tables,
+    host = dict(q=w.q.cpu(), k_new=w.k_new.cpu(), v_new=w.v_new.cpu(), slots=slots, block_tables=w.block_tables,
                 context_lens=w.context_lens)
     dev = {k: v.to(device) for k, v in host.items()}
     dev["k_cache"] = w.k_cache.to(device)
@@ -334,7 +339,9 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    w, host, d, kv_bytes = build(rank_seed(args.seed, rank), device)
+    if args.workload == "llama70b_int8":
+        raise SystemExit("the int8 workload needs a quantised cache; see --workload choices")
+    w, host, d, kv_bytes = build(rank_seed(args.seed, rank), device, args.workload, args.block_size)
     stream = torch.cuda.current_stream(device)
     peak, peak_kind = measured_peak()
 
@@ -394,7 +401,7 @@ def run_ours(args):
 
     # ---- CPU baseline: the oracle on this batch, rank 0 at N = 1 only ----
     cpu = None
-    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+    if world == 1 and rank == 0 and not args.no_cpu_baseline and args.workload == PRESET:
         rate, dt, _ = cpu_oracle_rate(w, range(w.num_seqs))
         cpu = {"value": round(rate, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                "sample": f"the full {PRESET} batch (32 sequences) once, fp64 C oracle, {dt:.1f} s"}
@@ -407,16 +414,18 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": {"workload": PRESET, "num_seqs": w.num_seqs, "num_heads": w.num_heads, "head_dim": w.head_dim,
-                   "block_size": w.block_size, "num_blocks": w.num_blocks, "context": "uniform [1, 2048]",
+        "vs_baseline": None, "dtype": {"fp16": "f16", "bf16": "bf16", "fp32": "f32", "int8": "i8"}[w.cache_dtype],
+        "data": "synthetic",
+        "config": {"workload": args.workload, "num_seqs": w.num_seqs, "num_heads": w.num_heads, "head_dim": w.head_dim,
+                   "block_size": w.block_size, "num_blocks": w.num_blocks, "window": w.window,
+                   "context": CONTEXT_DESC.get(args.workload, ""),
                    "kv_bytes_per_step_per_gpu": kv_bytes, "seed": args.seed,
                    "l2": "inputs larger than L2 (KV per step >> 126 MB), no flush", "parallelism": f"replicas x{world}"},
         "tokens_per_s_per_layer": round(tokens_per_s, 1),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_kind,
-                     "kernel": "decode_partition_kernel<half,half,128,16>", "partition_ms": round(part_avg, 4),
+                     "kernel": "decode_partition_kernel", "partition_ms": round(part_avg, 4),
                      "merge_ms": round(merge_avg, 4)},
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -436,6 +445,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=PRESET, choices=["llama70b_fp16", "chat_prefix_bf16", "sliding_window_fp16"],
+                    help="secondary workloads are for study; the metric is quoted on the default")
+    ap.add_argument("--block-size", type=int, default=None)
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)  # timing rule: at least 3 untimed warm-up steps
     if args.impl == "reference":
