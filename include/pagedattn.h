@@ -13,7 +13,7 @@
  * kernel's address h*D + (pb*bs + off)*H*D (page A, section "PagedAttention注意力计算流程"):
  *
  *     k_cache, v_cache : [num_blocks, block_size, num_heads, head_dim]   (row-major)
- *     k_scale, v_scale : [num_blocks, block_size, num_heads] fp16        (INT8 cache only)
+ *     k_scale, v_scale : [num_blocks, block_size, num_heads] fp16        (INT8 / FP8 caches only)
  *
  * A *slot* is pb*block_size + off: one token row of num_heads*head_dim values.
  *
@@ -45,7 +45,8 @@ typedef enum pa_dtype {
   PA_F32 = 0,  /* IEEE binary32 */
   PA_F16 = 1,  /* IEEE binary16 */
   PA_BF16 = 2, /* bfloat16 */
-  PA_I8 = 3    /* signed 8-bit code with a per-(token, head) fp16 scale */
+  PA_I8 = 3,   /* signed 8-bit code with a per-(token, head) fp16 scale */
+  PA_FP8_E4M3 = 4 /* OCP FP8 E4M3 code with a per-(token, head) fp16 scale */
 } pa_dtype;
 
 typedef enum pa_status {
@@ -99,21 +100,21 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim);
  *     k_i  = k_cache[block_tables[s][i / block_size], i % block_size, h, :]
  *     p    = softmax_i(scale * <q[s,h,:], k_i>)
  *     out[s,h,:] = sum_i p_i * v_i                      (ctx == 0: zeros)
- * An INT8 cache holds codes c with k = c * k_scale[slot, h] (likewise v).
+ * An INT8 or FP8 (E4M3) cache holds codes c with k = value(c) * k_scale[slot, h] (likewise v).
  *
  *   out            [num_seqs, num_heads, head_dim]        io_dtype, written
  *   q              [num_seqs, num_heads, head_dim]        io_dtype
  *   k_cache,
  *   v_cache        [num_blocks, block_size, num_heads, head_dim]   cache_dtype
  *   k_scale,
- *   v_scale        [num_blocks, block_size, num_heads] fp16; required iff cache_dtype == PA_I8
+ *   v_scale        [num_blocks, block_size, num_heads] fp16; required iff cache_dtype is PA_I8 or PA_FP8_E4M3
  *   block_tables   [num_seqs, max_blocks_per_seq] int32; only entries of blocks that hold
  *                  attended tokens are read (others may hold anything, e.g. -1)
  *   context_lens   [num_seqs] int32, 0 <= ctx <= max_blocks_per_seq*block_size
- *   head_dim       64 or 128;  block_size 1..32;  num_heads >= 1 (multiple of 8 for PA_I8)
+ *   head_dim       64 or 128;  block_size 1..32;  num_heads >= 1 (multiple of 8 for 8-bit caches)
  *   scale          softmax scale (typically 1/sqrt(head_dim))
  *   window         0 = full attention, W > 0 = the last W tokens only
- *   io_dtype       PA_F32, PA_F16 or PA_BF16; cache_dtype == io_dtype, or PA_I8 with
+ *   io_dtype       PA_F32, PA_F16 or PA_BF16; cache_dtype == io_dtype, or PA_I8 / PA_FP8_E4M3 with
  *                  io_dtype PA_F16 / PA_BF16
  *   workspace      device scratch of >= pa_decode_workspace_bytes(...) bytes; contents
  *                  need no initialisation and are clobbered.  Two calls that may run
@@ -175,10 +176,10 @@ pa_status paged_attention_decode_static_scratch(void* out, const void* q, const 
  *   v_cache        [num_blocks, block_size, num_heads, head_dim] of `dtype`
  *   slot_mapping   [num_tokens] int64: token t goes to slot slot_mapping[t]
  *                  (= block*block_size + offset); a negative slot skips the token
- *   dtype          PA_F32 / PA_F16 / PA_BF16 / PA_I8 (codes are copied as they are)
+ *   dtype          PA_F32 / PA_F16 / PA_BF16 / PA_I8 / PA_FP8_E4M3 (codes are copied as they are)
  *   k_scale_src,   [num_tokens, num_heads] fp16 scales of the new rows, and
  *   v_scale_src    k_scale_cache, v_scale_cache [num_blocks, block_size, num_heads] fp16:
- *   k_scale_cache, required iff dtype == PA_I8, NULL otherwise
+ *   k_scale_cache, required iff dtype is PA_I8 or PA_FP8_E4M3, NULL otherwise
  *   v_scale_cache
  * Bit-exact copy.  Slots must be distinct (otherwise which token lands is unspecified).
  */
@@ -205,6 +206,33 @@ pa_status reshape_and_cache(const void* k, const void* v, void* k_cache, void* v
 pa_status copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs, int num_pairs,
                       int num_blocks, size_t block_bytes, void* k_scale_cache, void* v_scale_cache,
                       size_t scale_block_bytes, void* stream);
+
+/*
+ * Quantise-on-write: like reshape_and_cache, but the new rows arrive in fp16 / bf16 and
+ * are stored as 8-bit codes with one fp16 scale per (token, head) row.  Source: page B,
+ * section "量化压缩KV Cache的INT8与FP8方案" (an INT8 KV cache halves the memory; FP8 --
+ * printed "E4M1", read as E4M3 -- is the alternative); the scheme is this library's:
+ *   PA_I8:        scale = max_d |x_d| / 127 (fp32, then rounded to fp16),
+ *                 code  = clamp(rint(x_d / scale), -127, 127)      (fp32 division, ties to even)
+ *   PA_FP8_E4M3:  scale = max_d |x_d| / 448 (fp32, then rounded to fp16),
+ *                 code  = E4M3(x_d / scale)       (fp32 division, nearest even, saturating)
+ *   a row whose fp16 scale is 0 stores scale 0 and zero codes.
+ *
+ *   k, v           [num_tokens, num_heads, head_dim] of src_dtype (PA_F16 or PA_BF16),
+ *                  token strides in elements as in reshape_and_cache
+ *   k_cache,       [num_blocks, block_size, num_heads, head_dim] of cache_dtype
+ *   v_cache        (PA_I8 or PA_FP8_E4M3)
+ *   k_scale_cache, [num_blocks, block_size, num_heads] fp16
+ *   v_scale_cache
+ *   slot_mapping   [num_tokens] int64 (negative = skip)
+ *   head_dim       64 or 128
+ * Results are bit-exact with the definition above (IEEE fp32 division, RNE roundings).
+ */
+pa_status reshape_and_cache_quant(const void* k, const void* v, pa_dtype src_dtype, void* k_cache,
+                                  void* v_cache, void* k_scale_cache, void* v_scale_cache,
+                                  pa_dtype cache_dtype, const int64_t* slot_mapping, int num_tokens,
+                                  int num_heads, int head_dim, int block_size, int num_blocks,
+                                  int64_t k_token_stride, int64_t v_token_stride, void* stream);
 
 /* ------------------------------------------------------------------------------------ */
 /* Host-side block manager (free list + reference counts)                               */

@@ -24,7 +24,7 @@ import numpy as np
 from . import block_manager, cache_ops, quant  # noqa: F401
 from .build import LIB, build
 
-F32, F16, BF16, I8 = 0, 1, 2, 3
+F32, F16, BF16, I8, FP8 = 0, 1, 2, 3, 4
 _STATUS = {1: "bad argument", 2: "block-table entry out of range",
            3: "context length out of range", 4: "out of memory"}
 
@@ -46,6 +46,8 @@ def _load():
         lib.orc_f16_to_f64.argtypes = [ctypes.c_uint16]
         lib.orc_bf16_to_f64.restype = ctypes.c_double
         lib.orc_bf16_to_f64.argtypes = [ctypes.c_uint16]
+        lib.orc_e4m3_to_f64.restype = ctypes.c_double
+        lib.orc_e4m3_to_f64.argtypes = [ctypes.c_uint8]
         _lib = lib
     return _lib
 
@@ -64,6 +66,8 @@ def _raw(x):
                 return x.view(torch.int16).numpy(), BF16
             if x.dtype == torch.int8:
                 return x.numpy(), I8
+            if x.dtype == torch.float8_e4m3fn:
+                return x.view(torch.uint8).numpy(), FP8
             raise TypeError(f"unsupported tensor dtype {x.dtype}")
     except ImportError:  # pragma: no cover
         pass
@@ -99,7 +103,7 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, window=
     """Decode attention of one query token per sequence over a paged KV cache.
 
     q [S,H,D]; k_cache/v_cache [NB,bs,H,D]; block_tables [S,MB] int; context_lens [S];
-    k_scale/v_scale [NB,bs,H] fp16 for an int8 cache.  Returns fp64 numpy [S,H,D].
+    k_scale/v_scale [NB,bs,H] fp16 for an int8 or fp8 (torch.float8_e4m3fn) cache.  Returns fp64 numpy [S,H,D].
     """
     lib = _load()
     qa, qd = _raw(q)
@@ -117,10 +121,10 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, window=
     if bt.size == 0:
         bt = np.zeros((S, 1), np.int32)
     ks = vs = None
-    if kd == I8:
+    if kd in (I8, FP8):
         ks, vs = _u16(k_scale), _u16(v_scale)
         if ks.shape != (NB, bs, H) or vs.shape != (NB, bs, H):
-            raise ValueError("int8 cache needs k_scale/v_scale of shape [NB, bs, H]")
+            raise ValueError("an int8/fp8 cache needs k_scale/v_scale of shape [NB, bs, H]")
     out = np.zeros((S, H, D), np.float64)
     st = lib.orc_paged_decode(
         out.ctypes.data, qa.ctypes.data, qd, ka.ctypes.data, va.ctypes.data, kd,
@@ -137,3 +141,7 @@ def f16_to_f64(bits: int) -> float:
 
 def bf16_to_f64(bits: int) -> float:
     return _load().orc_bf16_to_f64(bits)
+
+
+def e4m3_to_f64(bits: int) -> float:
+    return _load().orc_e4m3_to_f64(bits)

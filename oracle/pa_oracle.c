@@ -26,7 +26,9 @@
  *     token included; window <= 0 means full attention.
  *   - INT8 cache.  Same page, section "量化压缩KV Cache的INT8与FP8方案", names an
  *     INT8 KV cache but not its scheme.  Reading: one fp16 scale per (token, head)
- *     row, value = int8 code * scale, both converted to fp64 exactly.
+ *     row, value = int8 code * scale, both converted to fp64 exactly.  The same
+ *     section names FP8 ("E4M1", read as E4M3): the same per-row fp16 scale with an
+ *     OCP FP8 E4M3 code, value = e4m3 value * scale, exact in fp64.
  *
  * Steps, in the order the pages give them, per (sequence s, head h):
  *   1. lo = window > 0 ? max(0, ctx - window) : 0.
@@ -43,7 +45,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { ORC_F32 = 0, ORC_F16 = 1, ORC_BF16 = 2, ORC_I8 = 3 };
+enum { ORC_F32 = 0, ORC_F16 = 1, ORC_BF16 = 2, ORC_I8 = 3, ORC_FP8 = 4 };
 
 enum {
   ORC_OK = 0,
@@ -77,12 +79,26 @@ double orc_bf16_to_f64(uint16_t b) {
   return (double)f;
 }
 
+/* FP8 E4M3 (the OCP "fn" variant: no infinities, S.1111.111 is NaN) -> double, exactly:
+ * exponent field 0 is subnormal, m * 2^-9; otherwise (1 + m/8) * 2^(e - 7). */
+double orc_e4m3_to_f64(uint8_t c) {
+  int sign = (c >> 7) & 1;
+  int exponent = (c >> 3) & 0xf;
+  int mantissa = c & 0x7;
+  double v;
+  if (exponent == 15 && mantissa == 7) return NAN;
+  if (exponent == 0) v = ldexp((double)mantissa, -9);
+  else v = ldexp((double)(8 + mantissa), exponent - 10);
+  return sign ? -v : v;
+}
+
 static double load_value(const void* base, int dtype, size_t index) {
   switch (dtype) {
     case ORC_F32: return (double)((const float*)base)[index];
     case ORC_F16: return orc_f16_to_f64(((const uint16_t*)base)[index]);
     case ORC_BF16: return orc_bf16_to_f64(((const uint16_t*)base)[index]);
     case ORC_I8: return (double)((const int8_t*)base)[index];
+    case ORC_FP8: return orc_e4m3_to_f64(((const uint8_t*)base)[index]);
     default: return NAN;
   }
 }
@@ -94,7 +110,7 @@ static double load_value(const void* base, int dtype, size_t index) {
  *   q            [S, H, D] in q_dtype (F32 / F16 / BF16)
  *   k_cache,     [NB, bs, H, D] in cache_dtype (F32 / F16 / BF16 / I8)
  *   v_cache
- *   k_scale,     [NB, bs, H] binary16 bit patterns; required for I8, ignored otherwise
+ *   k_scale,     [NB, bs, H] binary16 bit patterns; required for I8 and FP8, ignored otherwise
  *   v_scale
  *   block_tables [S, MB] int32; only entries of blocks that hold attended tokens are read
  *   context_lens [S] int32
@@ -105,7 +121,7 @@ int orc_paged_decode(double* out, const void* q, int q_dtype, const void* k_cach
                      const int32_t* context_lens, int S, int H, int D, int bs, int MB, int NB,
                      double scale, int window) {
   if (S < 0 || H <= 0 || D <= 0 || bs <= 0 || MB <= 0 || NB <= 0) return ORC_BAD_ARG;
-  if (cache_dtype == ORC_I8 && (!k_scale || !v_scale)) return ORC_BAD_ARG;
+  if ((cache_dtype == ORC_I8 || cache_dtype == ORC_FP8) && (!k_scale || !v_scale)) return ORC_BAD_ARG;
 
   int max_ctx = MB * bs;
   double* Kc = (double*)malloc(sizeof(double) * (size_t)max_ctx * D);
@@ -140,7 +156,7 @@ int orc_paged_decode(double* out, const void* q, int q_dtype, const void* k_cach
         if (pb < 0 || pb >= NB) { status = ORC_BAD_TABLE; break; }
         size_t row = ((size_t)pb * bs + offset) * H + h; /* (pb*bs+off)*H + h */
         double ks = 1.0, vs = 1.0;
-        if (cache_dtype == ORC_I8) {
+        if (cache_dtype == ORC_I8 || cache_dtype == ORC_FP8) {
           ks = orc_f16_to_f64(k_scale[row]);
           vs = orc_f16_to_f64(v_scale[row]);
         }

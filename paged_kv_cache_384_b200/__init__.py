@@ -27,8 +27,10 @@ from . import _lib
 
 _L = _lib.load()
 
-PA_F32, PA_F16, PA_BF16, PA_I8 = 0, 1, 2, 3
-_DTYPE = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16, torch.int8: PA_I8}
+PA_F32, PA_F16, PA_BF16, PA_I8, PA_FP8_E4M3 = 0, 1, 2, 3, 4
+_DTYPE = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16, torch.int8: PA_I8,
+          torch.float8_e4m3fn: PA_FP8_E4M3}
+_SCALED = (torch.int8, torch.float8_e4m3fn)
 _STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_CUDA",
            4: "PA_ERR_OUT_OF_BLOCKS", 5: "PA_ERR_BAD_BLOCK"}
 DEVERR = {"table": 0x1, "context": 0x2, "slot": 0x4, "pair": 0x8, "timeout": 0x10}
@@ -90,7 +92,8 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
                            k_scale=None, v_scale=None, workspace=None, stream=None):
     """out[s,h,:] = softmax(scale * q[s,h] . K_s^T) V_s over the paged cache (fp32 accumulate).
 
-    q, out [S,H,D] fp32/fp16/bf16; k_cache, v_cache [NB,bs,H,D] of q's dtype, or int8 with
+    q, out [S,H,D] fp32/fp16/bf16; k_cache, v_cache [NB,bs,H,D] of q's dtype, or int8 /
+    float8_e4m3fn with
     k_scale, v_scale [NB,bs,H] fp16; block_tables int32 [S,MB]; context_lens int32 [S].
     window > 0 attends only the last ``window`` tokens.  ``workspace`` defaults to a fresh
     allocation (pass one to keep allocation off the hot path).
@@ -108,10 +111,10 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
     for name, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
                     ("block_tables", block_tables), ("context_lens", context_lens)):
         _dense(name, t)
-    if k_cache.dtype == torch.int8:
+    if k_cache.dtype in _SCALED:
         if k_scale is None or v_scale is None or k_scale.dtype != torch.float16 or \
                 k_scale.shape != (NB, bs, H) or v_scale.shape != (NB, bs, H):
-            raise ValueError("an int8 cache needs fp16 k_scale/v_scale of shape [NB, bs, H]")
+            raise ValueError("an int8 / fp8 cache needs fp16 k_scale/v_scale of shape [NB, bs, H]")
         _dense("k_scale", k_scale), _dense("v_scale", v_scale)
     if workspace is None:
         workspace = alloc_workspace(S, H, D, q.device)
@@ -149,6 +152,36 @@ def reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, k_scale=None, v_scal
         _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), T, H, D, bs, NB,
         k.stride(0), v.stride(0), _DTYPE[k.dtype], _ptr(k_scale), _ptr(v_scale),
         _ptr(k_scale_cache), _ptr(v_scale_cache), _stream(stream)))
+
+
+def reshape_and_cache_quant(k, v, k_cache, v_cache, k_scale_cache, v_scale_cache, slot_mapping, stream=None):
+    """Quantise token rows k[t], v[t] ([T,H,D] fp16/bf16) to the int8 or float8_e4m3fn cache
+    with one fp16 scale per (token, head), writing slot slot_mapping[t] (negative = skip)."""
+    T, H, D = k.shape
+    NB, bs, Hc, Dc = k_cache.shape
+    if v.shape != k.shape or (Hc, Dc) != (H, D) or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch between k/v and the caches")
+    if k.dtype not in (torch.float16, torch.bfloat16) or v.dtype != k.dtype:
+        raise ValueError("k and v must be fp16 or bf16")
+    if k_cache.dtype not in _SCALED or v_cache.dtype != k_cache.dtype:
+        raise ValueError("the caches must be int8 or float8_e4m3fn")
+    if k_scale_cache.shape != (NB, bs, H) or v_scale_cache.shape != (NB, bs, H) or \
+            k_scale_cache.dtype != torch.float16 or v_scale_cache.dtype != torch.float16:
+        raise ValueError("scale caches must be fp16 [NB, bs, H]")
+    if slot_mapping.dtype != torch.int64 or slot_mapping.shape != (T,):
+        raise ValueError("slot_mapping must be int64 [T]")
+    for name, t in (("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+        if t.stride(2) != 1 or t.stride(1) != D:
+            raise ValueError(f"{name} rows must be dense [H, D] blocks")
+    for name, t in (("k_cache", k_cache), ("v_cache", v_cache), ("k_scale_cache", k_scale_cache),
+                    ("v_scale_cache", v_scale_cache), ("slot_mapping", slot_mapping)):
+        _dense(name, t)
+    _check(_L.reshape_and_cache_quant(
+        _ptr(k), _ptr(v), _DTYPE[k.dtype], _ptr(k_cache), _ptr(v_cache), _ptr(k_scale_cache),
+        _ptr(v_scale_cache), _DTYPE[k_cache.dtype], _ptr(slot_mapping), T, H, D, bs, NB,
+        k.stride(0), v.stride(0), _stream(stream)))
 
 
 def copy_blocks(k_cache, v_cache, src_dst_pairs, k_scale_cache=None, v_scale_cache=None, stream=None):

@@ -30,6 +30,9 @@ SIGNATURES = {
     "reshape_and_cache": (c_int, [
         c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
         c_int64, c_int64, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "reshape_and_cache_quant": (c_int, [
+        c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_int, c_int,
+        c_int, c_int, c_int, c_int64, c_int64, c_void_p]),
     "copy_blocks": (c_int, [
         c_void_p, c_void_p, c_void_p, c_int, c_int, c_size_t, c_void_p, c_void_p, c_size_t, c_void_p]),
     "pa_bm_create": (c_void_p, [c_int, c_int, c_void_p]),

@@ -110,7 +110,7 @@ struct RegisterCache {
   RegisterCache() { register_device_error_reader(read_cache_error); }
 } g_register_cache;
 
-size_t elem_size(pa_dtype t) { return t == PA_F32 ? 4 : (t == PA_I8 ? 1 : 2); }
+size_t elem_size(pa_dtype t) { return t == PA_F32 ? 4 : ((t == PA_I8 || t == PA_FP8_E4M3) ? 1 : 2); }
 
 }  // namespace
 }  // namespace pa
@@ -124,7 +124,7 @@ extern "C" pa_status reshape_and_cache(const void* k, const void* v, void* k_cac
                                        void* k_scale_cache, void* v_scale_cache, void* stream) {
   if (num_tokens < 0 || num_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
     return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: sizes must be positive (num_tokens >= 0)");
-  if (dtype != PA_F32 && dtype != PA_F16 && dtype != PA_BF16 && dtype != PA_I8)
+  if (dtype != PA_F32 && dtype != PA_F16 && dtype != PA_BF16 && dtype != PA_I8 && dtype != PA_FP8_E4M3)
     return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: unknown dtype %d", static_cast<int>(dtype));
   const long long row_elems = static_cast<long long>(num_heads) * head_dim;
   const size_t e = elem_size(dtype);
@@ -134,10 +134,10 @@ extern "C" pa_status reshape_and_cache(const void* k, const void* v, void* k_cac
     return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: token strides must be >= num_heads*head_dim");
   if ((k_token_stride * static_cast<long long>(e)) % 16 || (v_token_stride * static_cast<long long>(e)) % 16)
     return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: token strides must be multiples of 16 bytes");
-  const bool int8 = dtype == PA_I8;
+  const bool int8 = dtype == PA_I8 || dtype == PA_FP8_E4M3;  // 8-bit codes travel with their scales
   if (int8 != (k_scale_src && v_scale_src && k_scale_cache && v_scale_cache) ||
       (!int8 && (k_scale_src || v_scale_src || k_scale_cache || v_scale_cache)))
-    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: the four scale pointers are required for PA_I8 and must be NULL otherwise");
+    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: the four scale pointers are required for PA_I8 / PA_FP8_E4M3 and must be NULL otherwise");
   if (num_tokens == 0) return PA_OK;
   if (!k || !v || !k_cache || !v_cache || !slot_mapping) return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: NULL pointer");
   if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
@@ -200,5 +200,130 @@ extern "C" pa_status copy_blocks(void* k_cache, void* v_cache, const int64_t* sr
                           : reinterpret_cast<const void*>(&copy_blocks_kernel<1>);
   cudaError_t err = launch_dependent(fn, grid, dim3(threads), 0, s, args);
   if (err != cudaSuccess) return cuda_fail(err, "launching copy_blocks");
+  return PA_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// Quantise-on-write ("KV Cache optimisation strategies in deployment" (yunthe.com),
+// section "量化压缩KV Cache的INT8与FP8方案": an 8-bit KV cache; the per-(token, head) scheme
+// is this library's).  One warp per (token, head, K-or-V) row: the row's max |x| by a warp
+// reduction, scale = fp16(max / QMAX) with an IEEE fp32 division, then every element's code
+// from an IEEE fp32 division by the fp16 scale, rounded to nearest even.
+// ---------------------------------------------------------------------------------------
+namespace pa {
+
+template <typename CODE> struct Code;
+template <> struct Code<int8_t> {
+  static constexpr float kMax = 127.f;
+  static __device__ __forceinline__ uint8_t encode(float r) {
+    const float c = fminf(fmaxf(rintf(r), -127.f), 127.f);
+    return static_cast<uint8_t>(static_cast<int8_t>(c));
+  }
+};
+template <> struct Code<__nv_fp8_e4m3> {
+  static constexpr float kMax = 448.f;
+  static __device__ __forceinline__ uint8_t encode(float r) {
+    return static_cast<uint8_t>(__nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E4M3));
+  }
+};
+
+template <typename SRC, typename CODE, int D>
+__global__ void __launch_bounds__(256)
+reshape_and_cache_quant_kernel(const SRC* __restrict__ k, const SRC* __restrict__ v, uint8_t* __restrict__ kc,
+                               uint8_t* __restrict__ vc, __half* __restrict__ ks, __half* __restrict__ vs,
+                               const int64_t* __restrict__ slots, int T, int H, long long k_stride,
+                               long long v_stride, long long num_slots) {
+  constexpr int PER = D / 32;  // elements per lane: 2 or 4
+  grid_dependency_launch_next();
+  grid_dependency_wait();
+  const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= 2LL * T * H) return;
+  const int which = static_cast<int>(row & 1);  // 0: K, 1: V
+  const long long th = row >> 1;
+  const int t = static_cast<int>(th / H), h = static_cast<int>(th % H);
+  const long long slot = __ldg(slots + t);
+  if (slot < 0) return;
+  if (slot >= num_slots) {
+    if (lane == 0 && which == 0 && h == 0) cache_error(PA_DEVERR_SLOT);
+    return;
+  }
+  const SRC* src = (which ? v + t * v_stride : k + t * k_stride) + static_cast<long long>(h) * D + lane * PER;
+  float x[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) x[i] = static_cast<float>(src[i]);
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) amax = fmaxf(amax, fabsf(x[i]));
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const __half scale = __float2half_rn(__fdiv_rn(amax, Code<CODE>::kMax));
+  const float s = __half2float(scale);
+  uint8_t c[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) c[i] = s > 0.f ? Code<CODE>::encode(__fdiv_rn(x[i], s)) : 0;
+  uint8_t* dst = (which ? vc : kc) + (slot * H + h) * D + lane * PER;
+  if (PER == 4) {
+    *reinterpret_cast<uint32_t*>(dst) = c[0] | (c[1] << 8) | (c[2] << 16) | (static_cast<uint32_t>(c[3]) << 24);
+  } else {
+    *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(c[0] | (c[1] << 8));
+  }
+  if (lane == 0) (which ? vs : ks)[slot * H + h] = scale;
+}
+
+template <typename SRC, typename CODE>
+const void* quant_kernel_for(int D) {
+  return D == 64 ? reinterpret_cast<const void*>(&reshape_and_cache_quant_kernel<SRC, CODE, 64>)
+                 : reinterpret_cast<const void*>(&reshape_and_cache_quant_kernel<SRC, CODE, 128>);
+}
+
+}  // namespace pa
+
+extern "C" pa_status reshape_and_cache_quant(const void* k, const void* v, pa_dtype src_dtype, void* k_cache,
+                                             void* v_cache, void* k_scale_cache, void* v_scale_cache,
+                                             pa_dtype cache_dtype, const int64_t* slot_mapping, int num_tokens,
+                                             int num_heads, int head_dim, int block_size, int num_blocks,
+                                             int64_t k_token_stride, int64_t v_token_stride, void* stream) {
+  if (num_tokens < 0 || num_heads <= 0 || block_size <= 0 || num_blocks <= 0)
+    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache_quant: sizes must be positive (num_tokens >= 0)");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(PA_ERR_UNSUPPORTED, "reshape_and_cache_quant: head_dim %d (supported: 64, 128)", head_dim);
+  if (src_dtype != PA_F16 && src_dtype != PA_BF16)
+    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache_quant: src_dtype must be PA_F16 or PA_BF16");
+  if (cache_dtype != PA_I8 && cache_dtype != PA_FP8_E4M3)
+    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache_quant: cache_dtype must be PA_I8 or PA_FP8_E4M3");
+  const long long row_elems = static_cast<long long>(num_heads) * head_dim;
+  if (k_token_stride < row_elems || v_token_stride < row_elems)
+    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache_quant: token strides must be >= num_heads*head_dim");
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !k_cache || !v_cache || !k_scale_cache || !v_scale_cache || !slot_mapping)
+    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache_quant: NULL pointer");
+  if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) % 8 ||
+      (reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) % 4 ||
+      (reinterpret_cast<uintptr_t>(k_scale_cache) | reinterpret_cast<uintptr_t>(v_scale_cache)) % 2 ||
+      reinterpret_cast<uintptr_t>(slot_mapping) % 8 || (k_token_stride * 2) % 8 || (v_token_stride * 2) % 8)
+    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache_quant: misaligned pointer or stride");
+  const long long rows = 2LL * num_tokens * num_heads;
+  const int threads = 256;
+  const long long blocks = (rows + (threads / 32) - 1) / (threads / 32);
+  if (blocks > 0x7fffffffLL) return fail(PA_ERR_UNSUPPORTED, "reshape_and_cache_quant: too many rows");
+  const void* fn;
+  if (src_dtype == PA_F16)
+    fn = cache_dtype == PA_I8 ? quant_kernel_for<__half, int8_t>(head_dim) : quant_kernel_for<__half, __nv_fp8_e4m3>(head_dim);
+  else
+    fn = cache_dtype == PA_I8 ? quant_kernel_for<__nv_bfloat16, int8_t>(head_dim)
+                              : quant_kernel_for<__nv_bfloat16, __nv_fp8_e4m3>(head_dim);
+  const void* kp = k;
+  const void* vp = v;
+  void* kcp = k_cache;
+  void* vcp = v_cache;
+  void* ksp = k_scale_cache;
+  void* vsp = v_scale_cache;
+  int T = num_tokens, H = num_heads;
+  long long kst = k_token_stride, vst = v_token_stride, nslots = static_cast<long long>(num_blocks) * block_size;
+  void* args[] = {&kp, &vp, &kcp, &vcp, &ksp, &vsp, &slot_mapping, &T, &H, &kst, &vst, &nslots};
+  cudaError_t err = launch_dependent(fn, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0,
+                                     static_cast<cudaStream_t>(stream), args);
+  if (err != cudaSuccess) return cuda_fail(err, "launching reshape_and_cache_quant");
   return PA_OK;
 }

@@ -50,6 +50,7 @@ struct DecodeParams {
   float* ws_ml;          // [nslot][HG][2] partial (max, sum)
   float* ws_acc;         // [nslot][HG][D] partial accumulators
   int S, H, bs, MB, NB, window;
+  int tt, tpb;           // rows per tile (a divisor of bs) and tiles per physical block
   int HG, G, num_ctas, nstage;
   float qscale;          // softmax scale * log2(e): scores are kept in base 2
   uint32_t stage_bytes;  // bytes per pipeline stage
@@ -57,9 +58,10 @@ struct DecodeParams {
   uint32_t tx_bytes;     // TMA transaction bytes per stage
 };
 
-// Attended span of one sequence: tokens [lo, ctx), blocks first_lb .. first_lb + nb - 1.
+// Attended span of one sequence: tokens [lo, ctx), tiles first_t .. first_t + nb - 1.  Tile ti
+// holds the tt rows of logical block ti / tpb starting at row (ti % tpb) * tt.
 struct Span {
-  int ctx, lo, first_lb, nb;
+  int ctx, lo, first_t, nb;
 };
 
 __device__ __forceinline__ Span seq_span(const DecodeParams& p, int s, bool report) {
@@ -72,8 +74,8 @@ __device__ __forceinline__ Span seq_span(const DecodeParams& p, int s, bool repo
   Span r;
   r.ctx = ctx;
   r.lo = (p.window > 0 && ctx > p.window) ? ctx - p.window : 0;
-  r.first_lb = r.lo / p.bs;
-  r.nb = ctx > 0 ? (ctx - 1) / p.bs - r.first_lb + 1 : 0;
+  r.first_t = r.lo / p.tt;
+  r.nb = ctx > 0 ? (ctx - 1) / p.tt - r.first_t + 1 : 0;
   return r;
 }
 
@@ -134,19 +136,19 @@ __device__ __forceinline__ void store_floats(IO* dst, const float* src) {
 
 // ---------------------------------------------------------------------------------------
 // Partition kernel.
-//   IO: q/out type; CT: cache element type; D: head_dim; BS: block_size if fixed, 0 = runtime.
+//   IO: q/out type; CT: cache element type; D: head_dim; TT: rows per tile if fixed, 0 = runtime.
 // ---------------------------------------------------------------------------------------
-template <typename IO, typename CT, int D, int BS>
+template <typename IO, typename CT, int D, int TT>
 __global__ void __launch_bounds__(kMaxThreads)
 decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ CUtensorMap tmKs, const __grid_constant__ CUtensorMap tmVs,
                         const DecodeParams p) {
-  constexpr bool kInt8 = std::is_same<CT, int8_t>::value;
+  constexpr bool kInt8 = std::is_same<CT, int8_t>::value || std::is_same<CT, __nv_fp8_e4m3>::value;  // scaled 8-bit codes
   constexpr int E = Elem<CT>::kBytes;  // bytes per cache element
   constexpr int EV = Elem<CT>::kEV;    // cache elements per 16-byte vector (dims per lane)
   constexpr int LPR = D / EV;          // lanes covering one token row of one head
   constexpr int RPP = 32 / LPR;        // token rows per warp-wide pass
-  constexpr int MAXP = BS > 0 ? (BS + RPP - 1) / RPP : (32 + RPP - 1) / RPP;
+  constexpr int MAXP = TT > 0 ? (TT + RPP - 1) / RPP : (32 + RPP - 1) / RPP;
   static_assert(LPR >= 1 && LPR <= 32 && 32 % LPR == 0, "lane mapping");
 
   extern __shared__ __align__(128) uint8_t smem[];
@@ -155,7 +157,7 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   __shared__ int s_first_seq;
   __shared__ long long s_first_prefix;
 
-  const int bs = BS > 0 ? BS : p.bs;
+  const int tt = TT > 0 ? TT : p.tt;
   const int HG = p.HG, G = p.G, NS = p.nstage;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nthr = blockDim.x;
@@ -257,12 +259,14 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
     int issued = 0;
     bool ok = true;
     for (; issued < n; ++issued) {
-      const int lb = c.sp.first_lb + c.j;  // logical block index
+      const int ti = c.sp.first_t + c.j;  // tile index within the sequence
+      const int lb = ti / p.tpb;          // logical block index
       if (c.s != tab_seq || lb - tab_base >= 32 || lb < tab_base) {
         tab_seq = c.s;
         tab_base = lb;
         const int idx = tab_base + lane;
-        tab = idx < c.sp.first_lb + c.sp.nb ? __ldg(p.block_tables + static_cast<size_t>(c.s) * p.MB + idx) : 0;
+        const int lb_end = (c.sp.first_t + c.sp.nb - 1) / p.tpb + 1;
+        tab = idx < lb_end ? __ldg(p.block_tables + static_cast<size_t>(c.s) * p.MB + idx) : 0;
       }
       int pb = __shfl_sync(0xffffffffu, tab, lb - tab_base);
       if (pb < 0 || pb >= p.NB) {
@@ -277,7 +281,7 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
         }
         if (ok) {
           const uint32_t dst = stage_base + st * p.stage_bytes;
-          const int head0 = c.g * HG, row0 = pb * bs;
+          const int head0 = c.g * HG, row0 = pb * p.bs + (ti % p.tpb) * tt;
           mbar_arrive_expect_tx(full_bar(st), p.tx_bytes);
           tma_load_3d(dst, &tmK, full_bar(st), 0, head0, row0, policy);
           tma_load_3d(dst + p.v_off, &tmV, full_bar(st), 0, head0, row0, policy);
@@ -327,7 +331,7 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
     }
     const uint32_t kt = stage_base + st * p.stage_bytes;
     const uint32_t vt = kt + p.v_off;
-    const int tok0 = (c.sp.first_lb + c.j) * bs;  // logical index of the tile's first row
+    const int tok0 = (c.sp.first_t + c.j) * tt;  // logical index of the tile's first row
     const int hs = c.g * HG - ((c.g * HG) & ~7) + w;  // head column in the INT8 scale tile
 
     // Scores of this lane's rows (tokens pi*RPP + r), base-2 scaled.
@@ -336,10 +340,10 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
 #pragma unroll
     for (int pi = 0; pi < MAXP; ++pi) {
       sc[pi] = -INFINITY;
-      if (BS > 0 || pi * RPP < bs) {  // warp-uniform
+      if (TT > 0 || pi * RPP < tt) {  // warp-uniform
         const int t = pi * RPP + r;
         float part = 0.f;
-        if (t < bs) {
+        if (t < tt) {
           float kf[EV];
           Elem<CT>::to_float(ld_shared_v4(kt + ((t * HG + w) * D + v * EV) * E), kf);
 #pragma unroll
@@ -348,7 +352,7 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
 #pragma unroll
         for (int off = LPR / 2; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
         const int tok = tok0 + t;
-        if (t < bs && tok >= c.sp.lo && tok < c.sp.ctx) {
+        if (t < tt && tok >= c.sp.lo && tok < c.sp.ctx) {
           if (kInt8) part *= __half2float(__ushort_as_half(ld_shared_u16(kt + p.ks_off + (t * 8 + hs) * 2)));
           sc[pi] = part;
           tile_max = fmaxf(tile_max, part);
@@ -367,7 +371,7 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
     for (int e = 0; e < EV; ++e) acc[e] *= alpha;
 #pragma unroll
     for (int pi = 0; pi < MAXP; ++pi) {
-      if (BS > 0 || pi * RPP < bs) {
+      if (TT > 0 || pi * RPP < tt) {
         const int t = pi * RPP + r;
         if (sc[pi] != -INFINITY) {  // attended row (rows outside [lo, ctx) may hold garbage)
           const float pr = exp2f(sc[pi] - m);
@@ -536,7 +540,7 @@ pa_status encode(EncodeTiledFn fn, CUtensorMap* map, CUtensorMapDataType type, i
   return PA_OK;
 }
 
-size_t elem_bytes(pa_dtype t) { return t == PA_F32 ? 4 : (t == PA_I8 ? 1 : 2); }
+size_t elem_bytes(pa_dtype t) { return t == PA_F32 ? 4 : ((t == PA_I8 || t == PA_FP8_E4M3) ? 1 : 2); }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -554,9 +558,9 @@ WsLayout ws_layout(int S, int D, long long rows) {
 }
 
 // Heads per CTA: the largest power of two dividing H with K+V tiles of one stage <= 32 KiB.
-int pick_head_group(int H, int bs, int D, size_t e) {
+int pick_head_group(int H, int tt, int D, size_t e) {
   int hg = kMaxHeadGroup;
-  while (hg > 1 && (H % hg != 0 || 2 * static_cast<size_t>(bs) * hg * D * e > 32768)) hg >>= 1;
+  while (hg > 1 && (H % hg != 0 || 2 * static_cast<size_t>(tt) * hg * D * e > 32768)) hg >>= 1;
   return hg;
 }
 
@@ -566,11 +570,10 @@ struct KernelInfo {
 };
 
 template <typename IO, typename CT, int D>
-const void* partition_kernel_for(int bs) {
-  switch (bs) {
+const void* partition_kernel_for(int tt) {
+  switch (tt) {
     case 8: return reinterpret_cast<const void*>(&decode_partition_kernel<IO, CT, D, 8>);
     case 16: return reinterpret_cast<const void*>(&decode_partition_kernel<IO, CT, D, 16>);
-    case 32: return reinterpret_cast<const void*>(&decode_partition_kernel<IO, CT, D, 32>);
     default: return reinterpret_cast<const void*>(&decode_partition_kernel<IO, CT, D, 0>);
   }
 }
@@ -584,6 +587,10 @@ const void* select_partition(pa_dtype io, pa_dtype cache, int D, int bs) {
   if (cache == PA_I8) {
     return io == PA_F16 ? partition_kernel_for<__half, int8_t>(D, bs)
                         : partition_kernel_for<__nv_bfloat16, int8_t>(D, bs);
+  }
+  if (cache == PA_FP8_E4M3) {
+    return io == PA_F16 ? partition_kernel_for<__half, __nv_fp8_e4m3>(D, bs)
+                        : partition_kernel_for<__nv_bfloat16, __nv_fp8_e4m3>(D, bs);
   }
   switch (io) {
     case PA_F32: return partition_kernel_for<float, float>(D, bs);
@@ -625,8 +632,8 @@ pa_status occupancy(const void* fn, int threads, size_t smem, int* occ) {
 
 bool valid_pair(pa_dtype io, pa_dtype cache) {
   if (io == PA_F32) return cache == PA_F32;
-  if (io == PA_F16) return cache == PA_F16 || cache == PA_I8;
-  if (io == PA_BF16) return cache == PA_BF16 || cache == PA_I8;
+  if (io == PA_F16) return cache == PA_F16 || cache == PA_I8 || cache == PA_FP8_E4M3;
+  if (io == PA_BF16) return cache == PA_BF16 || cache == PA_I8 || cache == PA_FP8_E4M3;
   return false;
 }
 
@@ -662,14 +669,14 @@ extern "C" pa_status paged_attention_decode(void* out, const void* q, const void
   if (window < 0) return fail(PA_ERR_INVALID_ARG, "window must be >= 0 (0 = full attention)");
   if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
   if (!valid_pair(io_dtype, cache_dtype))
-    return fail(PA_ERR_INVALID_ARG, "dtype pair (io %d, cache %d) not supported: cache must equal io, or be PA_I8 with fp16/bf16 io",
+    return fail(PA_ERR_INVALID_ARG, "dtype pair (io %d, cache %d) not supported: cache must equal io, or be PA_I8 / PA_FP8_E4M3 with fp16/bf16 io",
                 static_cast<int>(io_dtype), static_cast<int>(cache_dtype));
-  const bool int8 = cache_dtype == PA_I8;
-  if (int8 && (num_heads % 8 != 0)) return fail(PA_ERR_UNSUPPORTED, "an INT8 cache needs num_heads to be a multiple of 8");
+  const bool int8 = cache_dtype == PA_I8 || cache_dtype == PA_FP8_E4M3;  // scaled 8-bit cache
+  if (int8 && (num_heads % 8 != 0)) return fail(PA_ERR_UNSUPPORTED, "an INT8 or FP8 cache needs num_heads to be a multiple of 8");
   if (num_seqs == 0) return PA_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !workspace)
     return fail(PA_ERR_INVALID_ARG, "a required pointer is NULL");
-  if (int8 && (!k_scale || !v_scale)) return fail(PA_ERR_INVALID_ARG, "INT8 cache needs k_scale and v_scale");
+  if (int8 && (!k_scale || !v_scale)) return fail(PA_ERR_INVALID_ARG, "INT8 and FP8 caches need k_scale and v_scale");
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
       (int8 && (!aligned16(k_scale) || !aligned16(v_scale))) || !aligned16(workspace))
     return fail(PA_ERR_INVALID_ARG, "tensor base addresses must be 16-byte aligned");
@@ -684,12 +691,20 @@ extern "C" pa_status paged_attention_decode(void* out, const void* q, const void
   if (workspace_bytes < need)
     return fail(PA_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
 
+  // Rows per tile: the largest divisor of block_size in [8, 16] (the whole block if none),
+  // so 32-token blocks stream as two 16-row tiles and keep four heads per CTA.
+  int tt = block_size;
+  for (int d = 16; d >= 8; --d)
+    if (block_size % d == 0) {
+      tt = d;
+      break;
+    }
   const size_t e = elem_bytes(cache_dtype);
-  const int HG = pick_head_group(num_heads, block_size, head_dim, e);
+  const int HG = pick_head_group(num_heads, tt, head_dim, e);
   const int G = num_heads / HG;
-  const uint32_t kv_tile = static_cast<uint32_t>(block_size) * HG * head_dim * e;
+  const uint32_t kv_tile = static_cast<uint32_t>(tt) * HG * head_dim * e;
   const uint32_t kv_tile_al = (kv_tile + 127u) & ~127u;
-  const uint32_t sc_tile = int8 ? static_cast<uint32_t>(block_size) * 8 * 2 : 0;
+  const uint32_t sc_tile = int8 ? static_cast<uint32_t>(tt) * 8 * 2 : 0;
   const uint32_t sc_tile_al = (sc_tile + 127u) & ~127u;
   const uint32_t stage_bytes = 2 * kv_tile_al + 2 * sc_tile_al;
   int nstage = static_cast<int>((96 * 1024) / stage_bytes);
@@ -697,7 +712,7 @@ extern "C" pa_status paged_attention_decode(void* out, const void* q, const void
   const size_t smem = kBarrierBytes + 128 + static_cast<size_t>(nstage) * stage_bytes;
   const int threads = 32 * (HG + 1);
 
-  const void* part_fn = select_partition(io_dtype, cache_dtype, head_dim, block_size);
+  const void* part_fn = select_partition(io_dtype, cache_dtype, head_dim, tt);
   const void* merge_fn = select_merge(io_dtype, head_dim);
   int occ = 0;
   st = occupancy(part_fn, threads, smem, &occ);
@@ -723,14 +738,14 @@ extern "C" pa_status paged_attention_decode(void* out, const void* q, const void
                                 static_cast<cuuint64_t>(num_blocks) * block_size};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * e, static_cast<cuuint64_t>(num_heads) * head_dim * e};
     const cuuint32_t box[3] = {static_cast<cuuint32_t>(head_dim), static_cast<cuuint32_t>(HG),
-                               static_cast<cuuint32_t>(block_size)};
+                               static_cast<cuuint32_t>(tt)};
     if ((st = encode(enc, &tmK, ttype, 3, k_cache, dims, strides, box)) != PA_OK) return st;
     if ((st = encode(enc, &tmV, ttype, 3, v_cache, dims, strides, box)) != PA_OK) return st;
   }
   if (int8) {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(num_heads), static_cast<cuuint64_t>(num_blocks) * block_size};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(num_heads) * 2};
-    const cuuint32_t box[2] = {8, static_cast<cuuint32_t>(block_size)};
+    const cuuint32_t box[2] = {8, static_cast<cuuint32_t>(tt)};
     if ((st = encode(enc, &tmKs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, k_scale, dims, strides, box)) != PA_OK) return st;
     if ((st = encode(enc, &tmVs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, v_scale, dims, strides, box)) != PA_OK) return st;
   } else {
@@ -749,6 +764,8 @@ extern "C" pa_status paged_attention_decode(void* out, const void* q, const void
   prm.S = num_seqs;
   prm.H = num_heads;
   prm.bs = block_size;
+  prm.tt = tt;
+  prm.tpb = block_size / tt;
   prm.MB = max_blocks_per_seq;
   prm.NB = num_blocks;
   prm.window = window;

@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -82,6 +83,27 @@ template <> struct Elem<int8_t> {
       for (int b = 0; b < 4; ++b) {
         const uint32_t bits = __byte_perm(u, 0x4B000000u, 0x7440u | b);
         f[4 * i + b] = __uint_as_float(bits) - 8388736.0f;
+      }
+    }
+  }
+};
+
+// OCP FP8 E4M3 codes: the hardware converts pairs to fp16 exactly (every E4M3 value is an
+// fp16 value), then fp16 -> fp32 is exact too.
+template <> struct Elem<__nv_fp8_e4m3> {
+  static constexpr int kBytes = 1;
+  static constexpr int kEV = 16;
+  static __device__ __forceinline__ void to_float(const uint4& v, float* f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int hw = 0; hw < 2; ++hw) {
+        const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>(w[i] >> (16 * hw));
+        const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+        const float2 p = __half22float2(*reinterpret_cast<const __half2*>(&h));
+        f[4 * i + 2 * hw] = p.x;
+        f[4 * i + 2 * hw + 1] = p.y;
       }
     }
   }

@@ -8,7 +8,7 @@ Tolerances (fp32 accumulation on the GPU, fp64 in the oracle):
     the midpoint of two adjacent I/O values that the fp32 result rounded to the other one
     (|gpu - oracle_fp64| <= half an I/O ulp + 1e-5 relative).  Such cases are counted and
     must stay rare.  For bf16 one ulp at |o| >= 0.5 already exceeds 2e-3, hence the rule.
-  * INT8 cache: the same against the oracle on the dequantised values, with 1e-2.
+  * INT8 and FP8 caches: the same against the oracle on the dequantised values, with 1e-2.
 """
 import numpy as np
 import torch
@@ -91,3 +91,9 @@ def oracle_decode(q, k_cache, v_cache, block_tables, context_lens, scale, window
 def assert_no_device_error():
     flags = pa.device_error(clear=True)
     assert flags == 0, f"device error flags 0x{flags:x}"
+
+
+def quantize_cache_fp8(cache_f16: torch.Tensor):
+    """Oracle FP8 (E4M3) quantiser on a [NB, bs, H, D] fp16 cache -> (float8 codes, fp16 scales)."""
+    codes, scale = oracle.quant.quantize_rows_fp8(cache_f16.cpu().numpy())
+    return torch.from_numpy(codes).view(torch.float8_e4m3fn), torch.from_numpy(scale)

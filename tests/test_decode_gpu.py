@@ -19,7 +19,7 @@ import paged_kv_cache_384_b200 as pa
 import synth
 from oracle.block_manager import BlockManager as OracleBM
 from oracle.block_manager import BlockTable
-from parity import TOL, GpuCase, assert_no_device_error, compare, oracle_decode, quantize_cache
+from parity import TOL, GpuCase, assert_no_device_error, compare, oracle_decode, quantize_cache, quantize_cache_fp8
 
 pytestmark = pytest.mark.gpu
 
@@ -37,7 +37,7 @@ def _poison_unattended(k, v, tables, ctx, bs, window=0):
         lo = max(0, c - window) if window > 0 else 0
         for i in range(lo, c):
             live[t[i // bs], i % bs] = True
-    if k.dtype == torch.int8:
+    if k.dtype in (torch.int8, torch.float8_e4m3fn):  # 8-bit codes: the NaN goes into the scales
         return live
     k[~live] = float("nan")
     v[~live] = float("nan")
@@ -57,19 +57,19 @@ def _small_case(seed, S, H, D, bs, ctx, dtype, window=0, device="cuda"):
     for s, t in enumerate(tables):
         if t:
             bt[s, : len(t)] = torch.tensor(t, dtype=torch.int32)
-    io = "fp16" if dtype.startswith("int8") and dtype != "int8-bf16" else dtype
-    if dtype == "int8-bf16":
-        io = "bf16"
+    eight_bit = dtype.startswith("int8") or dtype.startswith("fp8")
+    io = ("bf16" if dtype.endswith("-bf16") else "fp16") if eight_bit else dtype
     tdt = {"fp32": torch.float32, "fp16": torch.float16, "bf16": torch.bfloat16}[io]
     q = torch.randn(S, H, D, generator=g).to(tdt)
-    src = torch.float16 if dtype.startswith("int8") else tdt
+    src = torch.float16 if eight_bit else tdt
     k = torch.randn(NB, bs, H, D, generator=g).to(src)
     v = torch.randn(NB, bs, H, D, generator=g).to(src)
     scale = 1.0 / math.sqrt(D)
     ks = vs = None
-    if dtype.startswith("int8"):
-        k, ks = quantize_cache(k)
-        v, vs = quantize_cache(v)
+    if eight_bit:
+        quantize = quantize_cache if dtype.startswith("int8") else quantize_cache_fp8
+        k, ks = quantize(k)
+        v, vs = quantize(v)
         live = _poison_unattended(k, v, tables, ctx, bs, window)
         ks[~live] = float("nan")
         vs[~live] = float("nan")
@@ -211,12 +211,12 @@ def test_sliding_window_32k_fp16(cuda_device, bs):
 # ---------------------------------------------------------------------------------------
 # Edge cases
 # ---------------------------------------------------------------------------------------
-DTYPES = ["fp32", "fp16", "bf16", "int8", "int8-bf16"]
+DTYPES = ["fp32", "fp16", "bf16", "int8", "int8-bf16", "fp8", "fp8-bf16"]
 
 
 @pytest.mark.parametrize("dtype", DTYPES)
 @pytest.mark.parametrize("D", [64, 128])
-@pytest.mark.parametrize("bs", [1, 5, 8, 16, 32])
+@pytest.mark.parametrize("bs", [1, 5, 8, 12, 16, 24, 32])
 def test_dtype_headdim_blocksize_grid(cuda_device, dtype, D, bs):
     ctx = [0, 1, bs, bs + 1, 2 * bs - 1, 97, 300, 5]
     case, ref, io = _small_case(100 + bs + D, len(ctx), 8, D, bs, ctx, dtype)

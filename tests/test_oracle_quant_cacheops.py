@@ -104,3 +104,51 @@ def test_copy_blocks_duplicates_whole_blocks_and_nothing_else():
     assert np.array_equal(vc[4], v0[1]) and np.array_equal(vc[5], v0[2])
     for b in (0, 1, 2, 3):
         assert np.array_equal(kc[b], k0[b]) and np.array_equal(vc[b], v0[b])
+
+
+# ---------------------------------------------------------------------------------------
+# FP8 (E4M3) quantiser
+# ---------------------------------------------------------------------------------------
+def test_e4m3_code_points_match_torch_and_the_c_decoder():
+    import oracle
+    import torch
+    mine = quant.e4m3_values()
+    lib = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    c = np.array([oracle.e4m3_to_f64(i) for i in range(256)])
+    for other in (lib, c):
+        assert np.array_equal(np.isnan(mine), np.isnan(other))
+        assert np.array_equal(mine[~np.isnan(mine)], other[~np.isnan(other)])
+    assert np.nanmax(mine) == 448.0
+
+
+def test_e4m3_rounding_matches_torch_on_a_dense_sweep():
+    import torch
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.standard_normal(300000).astype(np.float32) * np.float32(40),
+                        (rng.random(100000).astype(np.float32) - np.float32(0.5)) * np.float32(0.03),
+                        np.float32([2 ** -10, -2 ** -10, 3 * 2 ** -10, 448, -448, 2 ** -6, 0.0, -0.0])])
+    x = x[np.abs(x) <= 448]
+    mine = quant.e4m3_round(x)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn)
+    assert np.array_equal(quant.e4m3_encode(mine), ref.view(torch.uint8).numpy())
+
+
+def test_fp8_quantiser_properties_on_every_fp16_value():
+    x = _all_finite_f16()
+    rows = np.stack([x, np.full_like(x, 1.0)], axis=1)
+    codes, scale = quant.quantize_rows_fp8(rows)
+    deq = quant.dequantize_rows_fp8(codes, scale)
+    s = scale.astype(np.float64)[:, None]
+    ratio = rows.astype(np.float64) / s
+    # E4M3 has 3 mantissa bits: relative error <= 2^-4 for normal values, absolute <= 2^-10 * s below
+    err = np.abs(deq - rows.astype(np.float64))
+    bound = np.maximum(np.abs(rows.astype(np.float64)) * 2.0 ** -4, 2.0 ** -10 * s) * (1 + 1e-3)
+    assert np.all(err <= bound + 1e-3 * s * 2.0 ** -9)
+    top = np.argmax(np.abs(rows.astype(np.float32)), axis=1)
+    assert np.all(np.abs(quant.e4m3_values()[codes[np.arange(len(x)), top]]) == 448.0)
+    assert np.all(np.isfinite(ratio))
+
+
+def test_fp8_zero_row():
+    codes, scale = quant.quantize_rows_fp8(np.zeros((2, 8), np.float16))
+    assert np.all(codes == 0) and np.all(scale == 0)
