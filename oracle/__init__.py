@@ -36,12 +36,12 @@ def _load():
     if _lib is None:
         build()
         lib = ctypes.CDLL(LIB)
-        lib.orc_paged_decode.restype = ctypes.c_int
-        lib.orc_paged_decode.argtypes = [
+        lib.orc_paged_decode_gqa.restype = ctypes.c_int
+        lib.orc_paged_decode_gqa.argtypes = [
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
             ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-            ctypes.c_double, ctypes.c_int]
+            ctypes.c_int, ctypes.c_double, ctypes.c_int]
         lib.orc_f16_to_f64.restype = ctypes.c_double
         lib.orc_f16_to_f64.argtypes = [ctypes.c_uint16]
         lib.orc_bf16_to_f64.restype = ctypes.c_double
@@ -102,7 +102,8 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, window=
                  k_scale=None, v_scale=None):
     """Decode attention of one query token per sequence over a paged KV cache.
 
-    q [S,H,D]; k_cache/v_cache [NB,bs,H,D]; block_tables [S,MB] int; context_lens [S];
+    q [S,Hq,D]; k_cache/v_cache [NB,bs,Hkv,D] with Hq a multiple of Hkv (grouped-query:
+    query head h reads cached head h // (Hq // Hkv)); block_tables [S,MB] int; context_lens [S];
     k_scale/v_scale [NB,bs,H] fp16 for an int8 or fp8 (torch.float8_e4m3fn) cache.  Returns fp64 numpy [S,H,D].
     """
     lib = _load()
@@ -113,7 +114,7 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, window=
         raise TypeError("k_cache and v_cache must share a dtype")
     S, H, D = qa.shape
     NB, bs, Hc, Dc = ka.shape
-    if (Hc, Dc) != (H, D) or va.shape != ka.shape:
+    if Dc != D or H % Hc != 0 or va.shape != ka.shape:
         raise ValueError("cache shape does not match q")
     bt = _i32(block_tables).reshape(S, -1)
     cl = _i32(context_lens).reshape(S)
@@ -123,13 +124,13 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, window=
     ks = vs = None
     if kd in (I8, FP8):
         ks, vs = _u16(k_scale), _u16(v_scale)
-        if ks.shape != (NB, bs, H) or vs.shape != (NB, bs, H):
+        if ks.shape != (NB, bs, Hc) or vs.shape != (NB, bs, Hc):
             raise ValueError("an int8/fp8 cache needs k_scale/v_scale of shape [NB, bs, H]")
     out = np.zeros((S, H, D), np.float64)
-    st = lib.orc_paged_decode(
+    st = lib.orc_paged_decode_gqa(
         out.ctypes.data, qa.ctypes.data, qd, ka.ctypes.data, va.ctypes.data, kd,
         ks.ctypes.data if ks is not None else None, vs.ctypes.data if vs is not None else None,
-        bt.ctypes.data, cl.ctypes.data, S, H, D, bs, MB, NB, float(scale), int(window))
+        bt.ctypes.data, cl.ctypes.data, S, H, Hc, D, bs, MB, NB, float(scale), int(window))
     if st != 0:
         raise ValueError(f"oracle: {_STATUS.get(st, st)}")
     return out

@@ -104,23 +104,27 @@ static double load_value(const void* base, int dtype, size_t index) {
 }
 
 /*
- * Paged decode attention, one query token per sequence.
+ * Paged decode attention, one query token per sequence.  Grouped-query attention (not on
+ * the pages; the usual definition): query head h reads key/value head h / (Hq / Hkv), so
+ * consecutive query heads share a cached head; Hq == Hkv is the pages' multi-head case.
  *
- *   out          [S, H, D] fp64, written
- *   q            [S, H, D] in q_dtype (F32 / F16 / BF16)
- *   k_cache,     [NB, bs, H, D] in cache_dtype (F32 / F16 / BF16 / I8)
+ *   out          [S, Hq, D] fp64, written
+ *   q            [S, Hq, D] in q_dtype (F32 / F16 / BF16)
+ *   k_cache,     [NB, bs, Hkv, D] in cache_dtype (F32 / F16 / BF16 / I8 / FP8)
  *   v_cache
- *   k_scale,     [NB, bs, H] binary16 bit patterns; required for I8 and FP8, ignored otherwise
+ *   k_scale,     [NB, bs, Hkv] binary16 bit patterns; required for I8 and FP8, ignored otherwise
  *   v_scale
  *   block_tables [S, MB] int32; only entries of blocks that hold attended tokens are read
  *   context_lens [S] int32
  */
-int orc_paged_decode(double* out, const void* q, int q_dtype, const void* k_cache,
-                     const void* v_cache, int cache_dtype, const uint16_t* k_scale,
-                     const uint16_t* v_scale, const int32_t* block_tables,
-                     const int32_t* context_lens, int S, int H, int D, int bs, int MB, int NB,
-                     double scale, int window) {
-  if (S < 0 || H <= 0 || D <= 0 || bs <= 0 || MB <= 0 || NB <= 0) return ORC_BAD_ARG;
+int orc_paged_decode_gqa(double* out, const void* q, int q_dtype, const void* k_cache,
+                         const void* v_cache, int cache_dtype, const uint16_t* k_scale,
+                         const uint16_t* v_scale, const int32_t* block_tables,
+                         const int32_t* context_lens, int S, int Hq, int Hkv, int D, int bs, int MB,
+                         int NB, double scale, int window) {
+  if (S < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || D <= 0 || bs <= 0 || MB <= 0 || NB <= 0)
+    return ORC_BAD_ARG;
+  const int group = Hq / Hkv; /* query heads sharing one key/value head */
   if ((cache_dtype == ORC_I8 || cache_dtype == ORC_FP8) && (!k_scale || !v_scale)) return ORC_BAD_ARG;
 
   int max_ctx = MB * bs;
@@ -141,8 +145,8 @@ int orc_paged_decode(double* out, const void* q, int q_dtype, const void* k_cach
     if (window > 0 && ctx > window) lo = ctx - window;
     int n = ctx - lo;
 
-    for (int h = 0; h < H && status == ORC_OK; ++h) {
-      double* o = out + ((size_t)s * H + h) * D;
+    for (int h = 0; h < Hq && status == ORC_OK; ++h) {
+      double* o = out + ((size_t)s * Hq + h) * D;
       if (n == 0) {
         for (int d = 0; d < D; ++d) o[d] = 0.0;
         continue;
@@ -154,7 +158,7 @@ int orc_paged_decode(double* out, const void* q, int q_dtype, const void* k_cach
         int offset = i % bs;
         int32_t pb = block_tables[(size_t)s * MB + logical_block];
         if (pb < 0 || pb >= NB) { status = ORC_BAD_TABLE; break; }
-        size_t row = ((size_t)pb * bs + offset) * H + h; /* (pb*bs+off)*H + h */
+        size_t row = ((size_t)pb * bs + offset) * Hkv + h / group; /* (pb*bs+off)*Hkv + kv head */
         double ks = 1.0, vs = 1.0;
         if (cache_dtype == ORC_I8 || cache_dtype == ORC_FP8) {
           ks = orc_f16_to_f64(k_scale[row]);
@@ -167,7 +171,7 @@ int orc_paged_decode(double* out, const void* q, int q_dtype, const void* k_cach
       }
       if (status != ORC_OK) break;
 
-      for (int d = 0; d < D; ++d) qv[d] = load_value(q, q_dtype, ((size_t)s * H + h) * D + d);
+      for (int d = 0; d < D; ++d) qv[d] = load_value(q, q_dtype, ((size_t)s * Hq + h) * D + d);
 
       /* step 3: scaled dot products */
       for (int i = 0; i < n; ++i) {
@@ -194,4 +198,14 @@ int orc_paged_decode(double* out, const void* q, int q_dtype, const void* k_cach
 
   free(Kc); free(Vc); free(score); free(qv);
   return status;
+}
+
+/* Multi-head decode: every query head has its own cached key/value head. */
+int orc_paged_decode(double* out, const void* q, int q_dtype, const void* k_cache,
+                     const void* v_cache, int cache_dtype, const uint16_t* k_scale,
+                     const uint16_t* v_scale, const int32_t* block_tables,
+                     const int32_t* context_lens, int S, int H, int D, int bs, int MB, int NB,
+                     double scale, int window) {
+  return orc_paged_decode_gqa(out, q, q_dtype, k_cache, v_cache, cache_dtype, k_scale, v_scale,
+                              block_tables, context_lens, S, H, H, D, bs, MB, NB, scale, window);
 }

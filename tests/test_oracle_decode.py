@@ -242,3 +242,44 @@ def test_out_of_range_table_entry_is_an_error():
         oracle.paged_decode(q, kc, kc, [[0, 5]], [6], 0.3)
     with pytest.raises(ValueError, match="context"):
         oracle.paged_decode(q, kc, kc, [[0, 1]], [9], 0.3)
+
+
+# ---------------------------------------------------------------------------------------
+# Grouped-query attention (query head h reads cached head h // (Hq // Hkv))
+# ---------------------------------------------------------------------------------------
+@pytest.mark.parametrize("hq,hkv", [(8, 2), (8, 1), (6, 3), (4, 4)])
+def test_gqa_equals_multi_head_on_a_repeated_cache(hq, hkv):
+    rng = np.random.default_rng(hq * 10 + hkv)
+    S, D, bs = 3, 8, 8
+    ctx = [5, 17, 30]
+    NB = sum(-(-c // bs) for c in ctx) + 2
+    q = rng.standard_normal((S, hq, D)).astype(np.float32)
+    kc = rng.standard_normal((NB, bs, hkv, D)).astype(np.float32)
+    vc = rng.standard_normal((NB, bs, hkv, D)).astype(np.float32)
+    bt = rng.permutation(NB)[: sum(-(-c // bs) for c in ctx)]
+    tables, k = [], 0
+    for c in ctx:
+        n = -(-c // bs)
+        tables.append(list(bt[k:k + n]) + [-1] * (4 - n))
+        k += n
+    bt = np.array(tables, np.int32)
+    g = hq // hkv
+    gqa = oracle.paged_decode(_as_f32_tensor(q), _as_f32_tensor(kc), _as_f32_tensor(vc), bt, ctx, 0.3)
+    kx = torch.from_numpy(kc).repeat_interleave(g, dim=2)   # library expansion of the shared heads
+    vx = torch.from_numpy(vc).repeat_interleave(g, dim=2)
+    mha = oracle.paged_decode(_as_f32_tensor(q), kx, vx, bt, ctx, 0.3)
+    assert np.array_equal(gqa, mha)
+
+
+def test_gqa_dense_case_matches_library_attention():
+    rng = np.random.default_rng(11)
+    hq, hkv, D, n = 8, 2, 16, 29
+    q = rng.standard_normal((1, hq, D)).astype(np.float32)
+    K = rng.standard_normal((1, n, hkv, D)).astype(np.float32)
+    V = rng.standard_normal((1, n, hkv, D)).astype(np.float32)
+    out = oracle.paged_decode(_as_f32_tensor(q), _as_f32_tensor(K), _as_f32_tensor(V), [[0]], [n], 0.25)
+    qt = torch.from_numpy(q[0]).double()[None, :, None, :]                  # [1, Hq, 1, D]
+    kt = torch.from_numpy(K[0]).double().permute(1, 0, 2)[None]             # [1, Hkv, n, D]
+    vt = torch.from_numpy(V[0]).double().permute(1, 0, 2)[None]
+    ref = F.scaled_dot_product_attention(qt, kt, vt, scale=0.25, enable_gqa=True)[0, :, 0, :].numpy()
+    np.testing.assert_allclose(out[0], ref, rtol=0, atol=1e-12)
