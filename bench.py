@@ -36,7 +36,8 @@ from paged_kv_cache_384_b200 import accounting  # noqa: E402
 PRESET = "llama70b_fp16"
 CONTEXT_DESC = {"llama70b_fp16": "uniform [1, 2048]",
                 "chat_prefix_bf16": "2000 shared + lognormal(median 300, sigma 1) tail, 64 copy-on-write forks",
-                "sliding_window_fp16": "32768 each, window 4096"}
+                "sliding_window_fp16": "32768 each, window 4096",
+                "llama70b_gqa_fp16": "uniform [1, 2048], 64 query heads over 8 cached heads"}
 METRIC = "paged decode attention KV GB/s (% of B200 HBM peak) and tokens/s per layer"
 FALLBACK_HBM_GBS = 6650.0
 
@@ -188,7 +189,7 @@ def build(seed: int, device, workload: str = PRESET, block_size=None):
     dev["out"] = torch.empty_like(dev["q"])
     dev["ws"] = pa.alloc_workspace(w.num_seqs, w.num_heads, w.head_dim, device)
     dev["pairs"] = w.copy_pairs.to(device)
-    kv_bytes = accounting.decode_kv_bytes(ctx, w.num_heads, w.head_dim, w.cache_dtype, w.window)
+    kv_bytes = accounting.decode_kv_bytes(ctx, w.num_kv_heads, w.head_dim, w.cache_dtype, w.window)
     return w, host, dev, kv_bytes
 
 
@@ -445,7 +446,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default=PRESET, choices=["llama70b_fp16", "chat_prefix_bf16", "sliding_window_fp16"],
+    ap.add_argument("--workload", default=PRESET, choices=["llama70b_fp16", "chat_prefix_bf16", "sliding_window_fp16",
+                                                           "llama70b_gqa_fp16"],
                     help="secondary workloads are for study; the metric is quoted on the default")
     ap.add_argument("--block-size", type=int, default=None)
     args = ap.parse_args(argv)

@@ -132,6 +132,27 @@ pa_status paged_attention_decode(void* out, const void* q, const void* k_cache,
                                  size_t workspace_bytes, void* stream);
 
 /*
+ * Grouped-query (and multi-query) paged decode: num_q_heads query heads share
+ * num_kv_heads cached heads, query head h reading cached head h / (num_q_heads /
+ * num_kv_heads).  Not on the pages (which size Llama-2-70B with 64 cached heads); the
+ * usual grouped-query definition.  Arguments as paged_attention_decode, except
+ *   q, out         [num_seqs, num_q_heads, head_dim]
+ *   k_cache,
+ *   v_cache        [num_blocks, block_size, num_kv_heads, head_dim]
+ *   k_scale, v_scale [num_blocks, block_size, num_kv_heads] (8-bit caches)
+ *   num_q_heads    a multiple of num_kv_heads
+ * and the workspace is sized by pa_decode_workspace_bytes(num_seqs, num_q_heads, head_dim).
+ * paged_attention_decode(..., num_heads, ...) is this call with both head counts equal.
+ */
+pa_status paged_attention_decode_gqa(void* out, const void* q, const void* k_cache,
+                                     const void* v_cache, const void* k_scale, const void* v_scale,
+                                     const int32_t* block_tables, const int32_t* context_lens,
+                                     int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                     int block_size, int num_blocks, int max_blocks_per_seq,
+                                     float scale, int window, pa_dtype io_dtype, pa_dtype cache_dtype,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * paged_attention_decode for callers that cannot allocate device memory.  No counterpart
  * on the pages: it exists for callers with no device allocator of their own -- e.g. a
  * plugin inside a host framework that owns all device memory and passes only the op's

@@ -92,15 +92,15 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
                            k_scale=None, v_scale=None, workspace=None, stream=None):
     """out[s,h,:] = softmax(scale * q[s,h] . K_s^T) V_s over the paged cache (fp32 accumulate).
 
-    q, out [S,H,D] fp32/fp16/bf16; k_cache, v_cache [NB,bs,H,D] of q's dtype, or int8 /
-    float8_e4m3fn with
-    k_scale, v_scale [NB,bs,H] fp16; block_tables int32 [S,MB]; context_lens int32 [S].
-    window > 0 attends only the last ``window`` tokens.  ``workspace`` defaults to a fresh
-    allocation (pass one to keep allocation off the hot path).
+    q, out [S,Hq,D] fp32/fp16/bf16; k_cache, v_cache [NB,bs,Hkv,D] of q's dtype, or int8 /
+    float8_e4m3fn with k_scale, v_scale [NB,bs,Hkv] fp16; Hq a multiple of Hkv (grouped-query
+    when Hkv < Hq: query head h reads cached head h // (Hq // Hkv)); block_tables int32
+    [S,MB]; context_lens int32 [S].  window > 0 attends only the last ``window`` tokens.
+    ``workspace`` defaults to a fresh allocation (pass one to keep allocation off the hot path).
     """
     S, H, D = q.shape
     NB, bs, Hc, Dc = k_cache.shape
-    if out.shape != q.shape or out.dtype != q.dtype or (Hc, Dc) != (H, D) or v_cache.shape != k_cache.shape:
+    if out.shape != q.shape or out.dtype != q.dtype or Dc != D or H % Hc != 0 or v_cache.shape != k_cache.shape:
         raise ValueError("shape/dtype mismatch between out, q and the caches")
     if k_cache.dtype != v_cache.dtype:
         raise ValueError("k_cache and v_cache must share a dtype")
@@ -113,14 +113,14 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
         _dense(name, t)
     if k_cache.dtype in _SCALED:
         if k_scale is None or v_scale is None or k_scale.dtype != torch.float16 or \
-                k_scale.shape != (NB, bs, H) or v_scale.shape != (NB, bs, H):
-            raise ValueError("an int8 / fp8 cache needs fp16 k_scale/v_scale of shape [NB, bs, H]")
+                k_scale.shape != (NB, bs, Hc) or v_scale.shape != (NB, bs, Hc):
+            raise ValueError("an int8 / fp8 cache needs fp16 k_scale/v_scale of shape [NB, bs, Hkv]")
         _dense("k_scale", k_scale), _dense("v_scale", v_scale)
     if workspace is None:
         workspace = alloc_workspace(S, H, D, q.device)
-    _check(_L.paged_attention_decode(
+    _check(_L.paged_attention_decode_gqa(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
-        _ptr(block_tables), _ptr(context_lens), S, H, D, bs, NB, block_tables.shape[1],
+        _ptr(block_tables), _ptr(context_lens), S, H, Hc, D, bs, NB, block_tables.shape[1],
         float(scale), int(window), _DTYPE[q.dtype], _DTYPE[k_cache.dtype], _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
     return out

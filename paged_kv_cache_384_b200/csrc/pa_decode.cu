@@ -26,6 +26,7 @@
 #include <cstdio>
 #include <mutex>
 #include <type_traits>
+#include <vector>
 
 #include "pa_device.cuh"
 #include "pa_host.h"
@@ -47,11 +48,12 @@ struct DecodeParams {
   const int32_t* block_tables;
   const int32_t* context_lens;
   long long* ws_prefix;  // [S + 1] per-sequence tile prefix (written by CTA 0)
-  float* ws_ml;          // [nslot][HG][2] partial (max, sum)
-  float* ws_acc;         // [nslot][HG][D] partial accumulators
+  float* ws_ml;          // [nslot][QW][2] partial (max, sum) per query head of the tile
+  float* ws_acc;         // [nslot][QW][D] partial accumulators
   int S, H, bs, MB, NB, window;
   int tt, tpb;           // rows per tile (a divisor of bs) and tiles per physical block
-  int HG, G, num_ctas, nstage;
+  int HG, G, num_ctas, nstage;   // cached heads per tile, head groups, grid size, ring depth
+  int Hq, GQ, QW;        // query heads, query heads per cached head, query heads per tile
   float qscale;          // softmax scale * log2(e): scores are kept in base 2
   uint32_t stage_bytes;  // bytes per pipeline stage
   uint32_t v_off, ks_off, vs_off;  // offsets of the V tile and the INT8 scale tiles in a stage
@@ -158,7 +160,7 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   __shared__ long long s_first_prefix;
 
   const int tt = TT > 0 ? TT : p.tt;
-  const int HG = p.HG, G = p.G, NS = p.nstage;
+  const int HG = p.HG, G = p.G, NS = p.nstage, QW = p.QW;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nthr = blockDim.x;
 
@@ -222,7 +224,7 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   if (threadIdx.x == 0) {
     for (int st = 0; st < NS; ++st) {
       mbar_init(full_bar(st), 1);
-      mbar_init(empty_bar(st), HG);
+      mbar_init(empty_bar(st), QW);
     }
     fence_barrier_init();
   }
@@ -242,7 +244,7 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   }
   const int n = static_cast<int>(count);
 
-  if (warp == HG) {
+  if (warp == QW) {
     // ---- 3. Producer warp: block-table lookups + TMA issue. --------------------------
     const uint64_t policy = l2_policy_evict_first();
     if (lane == 0) {
@@ -304,8 +306,10 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
     return;
   }
 
-  // ---- 4. Consumer warps: warp w owns head g*HG + w of every tile. ---------------------
+  // ---- 4. Consumer warps: warp w owns query head g*QW + w of every tile, which reads ------
+  //         cached head g*HG + w/GQ (grouped-query; GQ = 1 is multi-head attention).
   const int w = warp;
+  const int kw = w / p.GQ;  // cached head of this warp within the tile
   const int r = lane / LPR;  // token row within a pass
   const int v = lane % LPR;  // 16-byte vector within the row: dims [v*EV, v*EV + EV)
   Cursor c = start;
@@ -313,8 +317,8 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   float qf[EV], acc[EV];
   float m = -FLT_MAX, l = 0.f;  // running max (base 2) and sum; -FLT_MAX keeps exp2 finite
   auto load_q = [&](const Cursor& cc) {
-    const int h = cc.g * HG + w;
-    const IO* qrow = reinterpret_cast<const IO*>(p.q) + (static_cast<size_t>(cc.s) * p.H + h) * D + v * EV;
+    const int h = cc.g * QW + w;
+    const IO* qrow = reinterpret_cast<const IO*>(p.q) + (static_cast<size_t>(cc.s) * p.Hq + h) * D + v * EV;
     load_floats<IO, EV>(qrow, qf);
 #pragma unroll
     for (int e = 0; e < EV; ++e) qf[e] *= p.qscale;
@@ -332,7 +336,7 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
     const uint32_t kt = stage_base + st * p.stage_bytes;
     const uint32_t vt = kt + p.v_off;
     const int tok0 = (c.sp.first_t + c.j) * tt;  // logical index of the tile's first row
-    const int hs = c.g * HG - ((c.g * HG) & ~7) + w;  // head column in the INT8 scale tile
+    const int hs = c.g * HG - ((c.g * HG) & ~7) + kw;  // head column in the 8-bit scale tile
 
     // Scores of this lane's rows (tokens pi*RPP + r), base-2 scaled.
     float sc[MAXP];
@@ -345,7 +349,7 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
         float part = 0.f;
         if (t < tt) {
           float kf[EV];
-          Elem<CT>::to_float(ld_shared_v4(kt + ((t * HG + w) * D + v * EV) * E), kf);
+          Elem<CT>::to_float(ld_shared_v4(kt + ((t * HG + kw) * D + v * EV) * E), kf);
 #pragma unroll
           for (int e = 0; e < EV; ++e) part = fmaf(qf[e], kf[e], part);
         }
@@ -377,7 +381,7 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
           const float pr = exp2f(sc[pi] - m);
           l += pr;
           float vf[EV];
-          Elem<CT>::to_float(ld_shared_v4(vt + ((t * HG + w) * D + v * EV) * E), vf);
+          Elem<CT>::to_float(ld_shared_v4(vt + ((t * HG + kw) * D + v * EV) * E), vf);
           float pv = pr;
           if (kInt8) pv *= __half2float(__ushort_as_half(ld_shared_u16(kt + p.vs_off + (t * 8 + hs) * 2)));
 #pragma unroll
@@ -398,26 +402,26 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
 #pragma unroll
         for (int e = 0; e < EV; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
       }
-      const int h = c.g * HG + w;
+      const int h = c.g * QW + w;
       if (seg_from_start && seg_last) {  // whole segment in this CTA: final output
         if (r == 0) {
           const float inv = 1.f / lt;
           float o[EV];
 #pragma unroll
           for (int e = 0; e < EV; ++e) o[e] = acc[e] * inv;
-          IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(c.s) * p.H + h) * D + v * EV;
+          IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(c.s) * p.Hq + h) * D + v * EV;
           store_floats<IO, EV>(orow, o);
         }
       } else {  // partial state for the merge kernel
         const long long slot = blockIdx.x + static_cast<long long>(c.s) * G + c.g;
         if (r == 0) {
-          float4* dst = reinterpret_cast<float4*>(p.ws_acc + (slot * HG + w) * D + v * EV);
+          float4* dst = reinterpret_cast<float4*>(p.ws_acc + (slot * QW + w) * D + v * EV);
 #pragma unroll
           for (int i = 0; i < EV / 4; ++i) dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
         }
         if (lane == 0) {
-          p.ws_ml[(slot * HG + w) * 2 + 0] = m;
-          p.ws_ml[(slot * HG + w) * 2 + 1] = lt;
+          p.ws_ml[(slot * QW + w) * 2 + 0] = m;
+          p.ws_ml[(slot * QW + w) * 2 + 1] = lt;
         }
       }
       m = -FLT_MAX;
@@ -450,12 +454,12 @@ __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const De
   grid_dependency_wait();
   const int lane = threadIdx.x & 31;
   const long long item = static_cast<long long>(blockIdx.x) * kMergeWarps + (threadIdx.x >> 5);
-  if (item >= static_cast<long long>(p.S) * p.H) return;
-  const int s = static_cast<int>(item / p.H), h = static_cast<int>(item % p.H);
+  if (item >= static_cast<long long>(p.S) * p.Hq) return;
+  const int s = static_cast<int>(item / p.Hq), h = static_cast<int>(item % p.Hq);
   const long long per_group = p.ws_prefix[p.S];
   const long long pre = p.ws_prefix[s];
   const long long nb = p.ws_prefix[s + 1] - pre;
-  IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(s) * p.H + h) * D + lane * DL;
+  IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(s) * p.Hq + h) * D + lane * DL;
   float o[DL];
 #pragma unroll
   for (int e = 0; e < DL; ++e) o[e] = 0.f;
@@ -465,7 +469,7 @@ __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const De
     return;
   }
   const long long T = per_group * p.G;
-  const int g = h / p.HG, w = h % p.HG;
+  const int g = h / p.QW, w = h % p.QW;
   const long long a = p.G * pre + g * nb;
   const int c0 = cta_of(a, T, p.num_ctas), c1 = cta_of(a + nb - 1, T, p.num_ctas);
   if (c0 == c1) return;
@@ -473,13 +477,13 @@ __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const De
   const float2* ml = reinterpret_cast<const float2*>(p.ws_ml);
   // Global max over the partials, 32 partials per round (one per lane).
   float M = -FLT_MAX;
-  for (int k = c0 + lane; k <= c1; k += 32) M = fmaxf(M, ml[(k + seg) * p.HG + w].x);
+  for (int k = c0 + lane; k <= c1; k += 32) M = fmaxf(M, ml[(k + seg) * p.QW + w].x);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   float L = 0.f;
 #pragma unroll 4
   for (int k = c0; k <= c1; ++k) {
-    const long long row = (k + seg) * p.HG + w;
+    const long long row = (k + seg) * p.QW + w;
     const float2 st = ml[row];
     const float f = exp2f(st.x - M);
     L = fmaf(f, st.y, L);
@@ -557,9 +561,10 @@ WsLayout ws_layout(int S, int D, long long rows) {
   return l;
 }
 
-// Heads per CTA: the largest power of two dividing H with K+V tiles of one stage <= 32 KiB.
-int pick_head_group(int H, int tt, int D, size_t e) {
-  int hg = kMaxHeadGroup;
+// Cached heads per CTA: the largest power of two <= cap dividing H with K+V tiles of one
+// stage <= 32 KiB.
+int pick_head_group(int H, int tt, int D, size_t e, int cap) {
+  int hg = cap;
   while (hg > 1 && (H % hg != 0 || 2 * static_cast<size_t>(tt) * hg * D * e > 32768)) hg >>= 1;
   return hg;
 }
@@ -610,22 +615,35 @@ const void* select_merge(pa_dtype io, int D) {
   }
 }
 
-// Occupancy of a kernel at a given dynamic smem size, cached.
+// Make `fn` launchable with `smem` bytes of dynamic shared memory and return its occupancy.
+// The per-kernel dynamic-smem limit is a global attribute of the function: it is only ever
+// raised (lowering it for a small ring would break a later launch with a larger one).  The
+// occupancy answers are cached per (kernel, block size, smem).  Thread-safe.
 pa_status occupancy(const void* fn, int threads, size_t smem, int* occ) {
   struct Entry { const void* fn; int threads; size_t smem; int occ; };
-  static Entry cache[64];
-  static int used = 0;
-  for (int i = 0; i < used; ++i)
-    if (cache[i].fn == fn && cache[i].threads == threads && cache[i].smem == smem) {
-      *occ = cache[i].occ;
+  struct Limit { const void* fn; size_t smem; };
+  static std::mutex m;
+  static std::vector<Entry> cache;
+  static std::vector<Limit> limits;
+  std::lock_guard<std::mutex> lock(m);
+  for (const Entry& en : cache)
+    if (en.fn == fn && en.threads == threads && en.smem == smem) {
+      *occ = en.occ;
       return PA_OK;
     }
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(MaxDynamicSharedMemorySize)");
+  Limit* lim = nullptr;
+  for (Limit& l : limits)
+    if (l.fn == fn) lim = &l;
+  if (!lim || lim->smem < smem) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(MaxDynamicSharedMemorySize)");
+    if (lim) lim->smem = smem;
+    else limits.push_back(Limit{fn, smem});
+  }
   int o = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, fn, threads, smem);
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, fn, threads, smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
-  if (used < 64) cache[used++] = Entry{fn, threads, smem, o};
+  cache.push_back(Entry{fn, threads, smem, o});
   *occ = o;
   return PA_OK;
 }
@@ -651,15 +669,23 @@ extern "C" size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int hea
   return ws_layout(num_seqs, head_dim, rows).total;
 }
 
-extern "C" pa_status paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+namespace pa {
+namespace {
+pa_status decode_launch(void* out, const void* q, const void* k_cache, const void* v_cache,
                                             const void* k_scale, const void* v_scale, const int32_t* block_tables,
-                                            const int32_t* context_lens, int num_seqs, int num_heads, int head_dim,
+                                            const int32_t* context_lens, int num_seqs, int num_q_heads, int num_heads, int head_dim,
                                             int block_size, int num_blocks, int max_blocks_per_seq, float scale,
                                             int window, pa_dtype io_dtype, pa_dtype cache_dtype, void* workspace,
                                             size_t workspace_bytes, void* stream) {
   // ---- host validation (no CUDA call before this block passes) ----
   if (num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "num_seqs < 0");
-  if (num_heads <= 0 || num_heads > 4096) return fail(PA_ERR_INVALID_ARG, "num_heads must be in [1, 4096]");
+  if (num_heads <= 0 || num_heads > 4096 || num_q_heads <= 0 || num_q_heads > 4096)
+    return fail(PA_ERR_INVALID_ARG, "head counts must be in [1, 4096]");
+  if (num_q_heads % num_heads != 0)
+    return fail(PA_ERR_INVALID_ARG, "num_q_heads (%d) must be a multiple of num_kv_heads (%d)", num_q_heads, num_heads);
+  const int GQ = num_q_heads / num_heads;  // query heads per cached head
+  if (GQ > kMaxHeadGroup)
+    return fail(PA_ERR_UNSUPPORTED, "%d query heads per cached head (supported: up to %d)", GQ, kMaxHeadGroup);
   if (head_dim != 64 && head_dim != 128) return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", head_dim);
   if (block_size < 1 || block_size > 32) return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 1..32)", block_size);
   if (num_blocks <= 0 || max_blocks_per_seq <= 0) return fail(PA_ERR_INVALID_ARG, "num_blocks and max_blocks_per_seq must be positive");
@@ -687,7 +713,7 @@ extern "C" pa_status paged_attention_decode(void* out, const void* q, const void
   int dev = 0, sms = 0;
   pa_status st = current_device(&dev, &sms);
   if (st != PA_OK) return st;
-  const size_t need = pa_decode_workspace_bytes(num_seqs, num_heads, head_dim);
+  const size_t need = pa_decode_workspace_bytes(num_seqs, num_q_heads, head_dim);
   if (workspace_bytes < need)
     return fail(PA_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
 
@@ -700,7 +726,8 @@ extern "C" pa_status paged_attention_decode(void* out, const void* q, const void
       break;
     }
   const size_t e = elem_bytes(cache_dtype);
-  const int HG = pick_head_group(num_heads, tt, head_dim, e);
+  const int HG = pick_head_group(num_heads, tt, head_dim, e, kMaxHeadGroup / GQ);
+  const int QW = HG * GQ;  // consumer warps: one per query head of the tile
   const int G = num_heads / HG;
   const uint32_t kv_tile = static_cast<uint32_t>(tt) * HG * head_dim * e;
   const uint32_t kv_tile_al = (kv_tile + 127u) & ~127u;
@@ -710,7 +737,7 @@ extern "C" pa_status paged_attention_decode(void* out, const void* q, const void
   int nstage = static_cast<int>((96 * 1024) / stage_bytes);
   nstage = nstage < 2 ? 2 : (nstage > 8 ? 8 : nstage);
   const size_t smem = kBarrierBytes + 128 + static_cast<size_t>(nstage) * stage_bytes;
-  const int threads = 32 * (HG + 1);
+  const int threads = 32 * (QW + 1);
 
   const void* part_fn = select_partition(io_dtype, cache_dtype, head_dim, tt);
   const void* merge_fn = select_merge(io_dtype, head_dim);
@@ -720,7 +747,7 @@ extern "C" pa_status paged_attention_decode(void* out, const void* q, const void
   if (occ <= 0) return fail(PA_ERR_CUDA, "partition kernel cannot be resident (smem %zu)", smem);
   const int C = sms * (occ < kMaxCtasPerSm ? occ : kMaxCtasPerSm);
 
-  const long long rows = static_cast<long long>(C) * HG + static_cast<long long>(num_seqs) * num_heads;
+  const long long rows = static_cast<long long>(C) * QW + static_cast<long long>(num_seqs) * num_q_heads;
   const WsLayout lay = ws_layout(num_seqs, head_dim, rows);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
 
@@ -770,6 +797,9 @@ extern "C" pa_status paged_attention_decode(void* out, const void* q, const void
   prm.NB = num_blocks;
   prm.window = window;
   prm.HG = HG;
+  prm.Hq = num_q_heads;
+  prm.GQ = GQ;
+  prm.QW = QW;
   prm.G = G;
   prm.num_ctas = C;
   prm.nstage = nstage;
@@ -793,13 +823,38 @@ extern "C" pa_status paged_attention_decode(void* out, const void* q, const void
   if (ev[1]) cudaEventRecord(ev[1], s);
   {
     void* args[] = {&prm};
-    const long long items = static_cast<long long>(num_seqs) * num_heads;
+    const long long items = static_cast<long long>(num_seqs) * num_q_heads;
     const unsigned grid = static_cast<unsigned>((items + kMergeWarps - 1) / kMergeWarps);
     cudaError_t err = launch_dependent(merge_fn, dim3(grid), dim3(32 * kMergeWarps), 0, s, args);
     if (err != cudaSuccess) return cuda_fail(err, "launching the decode merge kernel");
   }
   if (ev[2]) cudaEventRecord(ev[2], s);
   return PA_OK;
+}
+}  // namespace
+}  // namespace pa
+
+extern "C" pa_status paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                            const void* k_scale, const void* v_scale, const int32_t* block_tables,
+                                            const int32_t* context_lens, int num_seqs, int num_heads, int head_dim,
+                                            int block_size, int num_blocks, int max_blocks_per_seq, float scale,
+                                            int window, pa_dtype io_dtype, pa_dtype cache_dtype, void* workspace,
+                                            size_t workspace_bytes, void* stream) {
+  return decode_launch(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, num_seqs, num_heads,
+                       num_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, scale, window, io_dtype,
+                       cache_dtype, workspace, workspace_bytes, stream);
+}
+
+extern "C" pa_status paged_attention_decode_gqa(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                                const void* k_scale, const void* v_scale, const int32_t* block_tables,
+                                                const int32_t* context_lens, int num_seqs, int num_q_heads,
+                                                int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                                int max_blocks_per_seq, float scale, int window, pa_dtype io_dtype,
+                                                pa_dtype cache_dtype, void* workspace, size_t workspace_bytes,
+                                                void* stream) {
+  return decode_launch(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, num_seqs,
+                       num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, scale, window,
+                       io_dtype, cache_dtype, workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------------------

@@ -26,7 +26,7 @@ _DT = {"fp32": torch.float32, "fp16": torch.float16, "bf16": torch.bfloat16}
 class Workload:
     name: str
     num_seqs: int
-    num_heads: int
+    num_heads: int                  # query heads
     head_dim: int
     block_size: int
     num_blocks: int
@@ -44,6 +44,7 @@ class Workload:
     copy_pairs: torch.Tensor        # int64 [N, 2] (src, dst) copy-on-write block copies
     tables: List[List[int]] = field(default_factory=list)
     notes: dict = field(default_factory=dict)
+    num_kv_heads: int = 0           # cached heads (== num_heads unless grouped-query)
 
     @property
     def max_blocks_per_seq(self) -> int:
@@ -150,15 +151,16 @@ def _build_prefix_shared(name, seed, bm_factory, device, p) -> Workload:
 
 def _finish(name, seed, device, p, ctx, nb, tables, bm, pairs) -> Workload:
     S, H, D, bs = p["num_seqs"], p["num_heads"], p["head_dim"], p["block_size"]
+    Hkv = p.get("num_kv_heads", H)
     gdev = _generator(seed, device)
     dt = p["dtype"]
     q = _values(gdev, (S, H, D), dt, device)
     if dt == "int8":
         q = q.to(torch.float16)
-    kc = _values(gdev, (nb, bs, H, D), dt, device)
-    vc = _values(gdev, (nb, bs, H, D), dt, device)
-    kn = _values(gdev, (S, H, D), dt, device)
-    vn = _values(gdev, (S, H, D), dt, device)
+    kc = _values(gdev, (nb, bs, Hkv, D), dt, device)
+    vc = _values(gdev, (nb, bs, Hkv, D), dt, device)
+    kn = _values(gdev, (S, Hkv, D), dt, device)
+    vn = _values(gdev, (S, Hkv, D), dt, device)
     mb = p.get("max_blocks_per_seq")
     return Workload(
         name=name, num_seqs=S, num_heads=H, head_dim=D, block_size=bs, num_blocks=nb,
@@ -167,7 +169,7 @@ def _finish(name, seed, device, p, ctx, nb, tables, bm, pairs) -> Workload:
         context_lens=torch.tensor(ctx, dtype=torch.int32),
         block_tables=_pack_tables(tables, mb), q=q, k_cache=kc, v_cache=vc, k_new=kn, v_new=vn,
         copy_pairs=torch.tensor(pairs, dtype=torch.int64).reshape(-1, 2),
-        tables=[list(t) for t in tables], notes={"seed": seed, "allocator": bm})
+        tables=[list(t) for t in tables], notes={"seed": seed, "allocator": bm}, num_kv_heads=Hkv)
 
 
 _BUILDERS = {"independent": _build_independent, "prefix": _build_prefix_shared}
@@ -183,6 +185,10 @@ PRESETS = {
     # Same shapes, INT8 cache (values are the fp16 source; the consumer quantises).
     "llama70b_int8": dict(kind="independent", num_seqs=32, num_heads=64, head_dim=128,
                           block_size=16, ctx_range=(1, 2048), slack=1.1, dtype="int8"),
+    # The real Llama-2-70B attention layer is grouped-query (64 query heads share 8 cached
+    # heads); 256 sequences keep the per-step KV stream above 1 GB like the layer above.
+    "llama70b_gqa_fp16": dict(kind="independent", num_seqs=256, num_heads=64, num_kv_heads=8, head_dim=128,
+                              block_size=16, ctx_range=(1, 2048), slack=1.1, dtype="fp16"),
     # High-concurrency chat: 256 sequences share a 2000-token prompt, lognormal tails
     # (median 300, sigma 1.0, cap 2048); 64 sequences fork the last shared block.
     "chat_prefix_bf16": dict(kind="prefix", num_seqs=256, num_heads=32, head_dim=128, block_size=16,

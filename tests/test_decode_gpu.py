@@ -303,3 +303,12 @@ def test_workspace_too_small_is_rejected(cuda_device):
     with pytest.raises(pa.PagedAttnError, match="workspace"):
         pa.paged_attention_decode(out, case.q, case.k_cache, case.v_cache, case.block_tables,
                                   case.context_lens, case.scale, workspace=case.workspace[:64])
+
+
+def test_alternating_ring_sizes_on_one_kernel(cuda_device):
+    """One kernel instantiation launched with a large, then a small, then the large
+    shared-memory ring again (a regression test for the per-kernel smem limit)."""
+    big, ref_big, io = _small_case(21, 3, 64, 128, 16, [40, 300, 17], "fp16")
+    small, ref_small, _ = _small_case(22, 3, 1, 128, 16, [40, 300, 17], "fp16")
+    for case, ref in ((big, ref_big), (small, ref_small), (big, ref_big)):
+        _check(case, ref, io)

@@ -133,3 +133,13 @@ def test_cache_ops_host_validation(L):
 def test_workspace_query_rejects_bad_sizes(L):
     assert L.pa_decode_workspace_bytes(1, 4, 96) == 0
     assert L.pa_decode_workspace_bytes(-1, 4, 64) == 0
+
+
+def test_gqa_host_validation(L):
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    def call(hq, hkv, io=1, cache=1):
+        return L.paged_attention_decode_gqa(P(16), P(16), P(16), P(16), None, None, P(16), P(16), 1, hq, hkv, 128,
+                                            16, 4, 2, 0.1, 0, io, cache, P(16), 1 << 20, None)
+    assert call(6, 4) == 1              # query heads not a multiple of cached heads
+    assert call(8, 0) == 1
+    assert call(64, 8, 3, 3) == 1       # int8 queries are not a thing

@@ -1,0 +1,111 @@
+"""Grouped-query / multi-query paged decode on the GPU against the fp64 oracle.
+
+query head h reads cached head h // (Hq // Hkv).  Covers group sizes 1..8 on every cache
+dtype, block sizes 8/16/32, windows, NaN-poisoned unattended rows, and the real Llama-2-70B
+layer shape (64 query heads over 8 cached heads) at 256 sequences on sampled outputs.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_384_b200 as pa
+import synth
+from oracle.block_manager import BlockManager as OracleBM
+from parity import TOL, GpuCase, assert_no_device_error, compare, oracle_decode, quantize_cache, quantize_cache_fp8
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(seed, hq, hkv, D, bs, ctx, dtype, window=0):
+    g = torch.Generator().manual_seed(seed)
+    S = len(ctx)
+    NB = sum(-(-c // bs) for c in ctx) + 4
+    bm = OracleBM(NB, bs, torch.randperm(NB, generator=g).tolist())
+    tables = [bm.allocate(-(-c // bs)) if c else [] for c in ctx]
+    MB = max(1, max(len(t) for t in tables))
+    bt = torch.tensor([t + [-1] * (MB - len(t)) for t in tables], dtype=torch.int32)
+    eight = dtype in ("int8", "fp8")
+    io = torch.float16 if eight else {"fp32": torch.float32, "fp16": torch.float16, "bf16": torch.bfloat16}[dtype]
+    q = torch.randn(S, hq, D, generator=g).to(io)
+    k = torch.randn(NB, bs, hkv, D, generator=g).to(torch.float16 if eight else io)
+    v = torch.randn(NB, bs, hkv, D, generator=g).to(torch.float16 if eight else io)
+    live = torch.zeros(NB, bs, dtype=torch.bool)
+    for t, c in zip(tables, ctx):
+        for i in range(max(0, c - window) if window else 0, c):
+            live[t[i // bs], i % bs] = True
+    ks = vs = None
+    if eight:
+        quant = quantize_cache if dtype == "int8" else quantize_cache_fp8
+        k, ks = quant(k)
+        v, vs = quant(v)
+        ks[~live] = float("nan")
+        vs[~live] = float("nan")
+    else:
+        k[~live] = float("nan")
+        v[~live] = float("nan")
+    scale = 1 / math.sqrt(D)
+    ref = oracle_decode(q, k, v, bt, ctx, scale, window, ks, vs)
+    ioname = {torch.float32: "fp32", torch.float16: "fp16", torch.bfloat16: "bf16"}[io]
+    return GpuCase(q, k, v, bt, ctx, scale, window, ks, vs), ref, ioname
+
+
+def _run(case, ref, io, tol):
+    out = case.decode()
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    return compare(out, ref, io, tol)
+
+
+@pytest.mark.parametrize("hq,hkv", [(2, 1), (8, 1), (8, 2), (6, 2), (12, 4), (24, 8)])
+@pytest.mark.parametrize("dtype", ["fp32", "fp16", "bf16"])
+def test_group_sizes(cuda_device, hq, hkv, dtype):
+    ctx = [0, 1, 16, 17, 250, 1100, 33]
+    case, ref, io = _case(hq * 7 + hkv, hq, hkv, 128, 16, ctx, dtype)
+    _run(case, ref, io, TOL[io])
+
+
+@pytest.mark.parametrize("dtype", ["int8", "fp8"])
+@pytest.mark.parametrize("hq", [16, 64])
+def test_eight_bit_caches(cuda_device, dtype, hq):
+    ctx = [5, 300, 64, 1500]
+    case, ref, io = _case(hq, hq, 8, 128, 16, ctx, dtype)
+    _run(case, ref, io, TOL["int8"])
+
+
+@pytest.mark.parametrize("bs", [8, 32])
+@pytest.mark.parametrize("D", [64, 128])
+def test_block_sizes_and_head_dims(cuda_device, bs, D):
+    ctx = [3, 64, 65, 900]
+    case, ref, io = _case(bs + D, 16, 2, D, bs, ctx, "bf16")
+    _run(case, ref, io, TOL[io])
+
+
+@pytest.mark.parametrize("window", [1, 100, 4096])
+def test_window(cuda_device, window):
+    ctx = [1, 99, 100, 101, 3000]
+    case, ref, io = _case(window, 32, 4, 128, 16, ctx, "fp16", window=window)
+    _run(case, ref, io, TOL[io])
+
+
+def test_llama70b_gqa_layer_sampled(cuda_device):
+    """64 query heads over 8 cached heads, 256 sequences of U[1, 2048] tokens."""
+    w = synth.build_workload("llama70b_gqa_fp16", 0, OracleBM)
+    case = GpuCase(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale)
+    out = case.decode()
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    sample = torch.randperm(w.num_seqs, generator=torch.Generator().manual_seed(5))[:20].tolist()
+    sample += [int(torch.argmax(w.context_lens)), int(torch.argmin(w.context_lens))]
+    ref = oracle_decode(w.q[sample], w.k_cache, w.v_cache, w.block_tables[sample], w.context_lens[sample], w.scale)
+    compare(out[sample], ref, "fp16", TOL["fp16"])
+
+
+def test_head_count_mismatch_is_rejected(cuda_device):
+    q = torch.zeros(1, 6, 128, dtype=torch.float16, device="cuda")
+    kc = torch.zeros(4, 16, 4, 128, dtype=torch.float16, device="cuda")
+    bt = torch.zeros(1, 1, dtype=torch.int32, device="cuda")
+    cl = torch.ones(1, dtype=torch.int32, device="cuda")
+    with pytest.raises(ValueError):
+        pa.paged_attention_decode(torch.empty_like(q), q, kc, kc, bt, cl, 0.1)
