@@ -153,6 +153,17 @@ pa_status paged_attention_decode_gqa(void* out, const void* q, const void* k_cac
                                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Process-wide switch (default 1): let grouped-query decode run on the tensor cores when
+ * the call qualifies -- fp16 or bf16 cache equal to io_dtype, head_dim 128, block_size a
+ * multiple of 8 dividing 128, and 4..16 query heads per cached head.  Then each 128-token
+ * tile of one cached head is two tcgen05 MMAs (scores K.q^T and the weighted sum
+ * V^T.p^T, fp32 accumulators in tensor memory) instead of CUDA-core dot products.  0 forces
+ * the CUDA-core kernel (same results within rounding).  Not thread-safe against concurrent
+ * decode calls; set it once at start-up.
+ */
+pa_status pa_decode_use_tensor_cores(int enable);
+
+/*
  * paged_attention_decode for callers that cannot allocate device memory.  No counterpart
  * on the pages: it exists for callers with no device allocator of their own -- e.g. a
  * plugin inside a host framework that owns all device memory and passes only the op's

@@ -221,6 +221,11 @@ def device_error(clear: bool = True) -> int:
     return flags.value
 
 
+def use_tensor_cores(enable: bool = True):
+    """Let grouped-query decode use the tcgen05 kernel where it qualifies (default on)."""
+    _check(_L.pa_decode_use_tensor_cores(int(enable)))
+
+
 def profile_enable(on: bool = True):
     _check(_L.pa_profile_enable(int(on)))
 

@@ -51,6 +51,7 @@ SIGNATURES = {
     "pa_bm_free_list": (c_int, [c_void_p, c_void_p, c_int, P(c_int)]),
     "pa_slot_mapping_host": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_int, c_void_p]),
     "pa_profile_enable": (c_int, [c_int]),
+    "pa_decode_use_tensor_cores": (c_int, [c_int]),
     "pa_profile_read": (c_int, [P(c_double), P(c_double), P(c_int), c_int]),
 }
 

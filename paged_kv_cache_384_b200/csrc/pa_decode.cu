@@ -28,113 +28,11 @@
 #include <type_traits>
 #include <vector>
 
+#include "pa_decode_shared.cuh"
 #include "pa_device.cuh"
 #include "pa_host.h"
 
 namespace pa {
-
-static __device__ unsigned int g_decode_error;
-
-__device__ __forceinline__ void decode_error(unsigned int bits) { atomicOr(&g_decode_error, bits); }
-
-constexpr int kMaxCtasPerSm = 4;    // persistent-grid CTAs per SM (upper bound)
-constexpr int kMaxHeadGroup = 8;    // heads per CTA (upper bound)
-constexpr int kMaxThreads = 32 * (kMaxHeadGroup + 1);
-constexpr int kBarrierBytes = 128;  // mbarriers at the front of dynamic smem (<= 8 stages)
-
-struct DecodeParams {
-  void* out;
-  const void* q;
-  const int32_t* block_tables;
-  const int32_t* context_lens;
-  long long* ws_prefix;  // [S + 1] per-sequence tile prefix (written by CTA 0)
-  float* ws_ml;          // [nslot][QW][2] partial (max, sum) per query head of the tile
-  float* ws_acc;         // [nslot][QW][D] partial accumulators
-  int S, H, bs, MB, NB, window;
-  int tt, tpb;           // rows per tile (a divisor of bs) and tiles per physical block
-  int HG, G, num_ctas, nstage;   // cached heads per tile, head groups, grid size, ring depth
-  int Hq, GQ, QW;        // query heads, query heads per cached head, query heads per tile
-  float qscale;          // softmax scale * log2(e): scores are kept in base 2
-  uint32_t stage_bytes;  // bytes per pipeline stage
-  uint32_t v_off, ks_off, vs_off;  // offsets of the V tile and the INT8 scale tiles in a stage
-  uint32_t tx_bytes;     // TMA transaction bytes per stage
-};
-
-// Attended span of one sequence: tokens [lo, ctx), tiles first_t .. first_t + nb - 1.  Tile ti
-// holds the tt rows of logical block ti / tpb starting at row (ti % tpb) * tt.
-struct Span {
-  int ctx, lo, first_t, nb;
-};
-
-__device__ __forceinline__ Span seq_span(const DecodeParams& p, int s, bool report) {
-  int ctx = __ldg(p.context_lens + s);
-  const int cap = p.MB * p.bs;
-  if (ctx < 0 || ctx > cap) {
-    if (report) decode_error(PA_DEVERR_CONTEXT);
-    ctx = ctx < 0 ? 0 : cap;
-  }
-  Span r;
-  r.ctx = ctx;
-  r.lo = (p.window > 0 && ctx > p.window) ? ctx - p.window : 0;
-  r.first_t = r.lo / p.tt;
-  r.nb = ctx > 0 ? (ctx - 1) / p.tt - r.first_t + 1 : 0;
-  return r;
-}
-
-// Position in the tile stream: sequence s, head group g, tile j of the segment.
-struct Cursor {
-  int s, g, j;
-  Span sp;
-};
-
-__device__ __forceinline__ void advance(Cursor& c, const DecodeParams& p) {
-  if (++c.j < c.sp.nb) return;
-  c.j = 0;
-  if (++c.g < p.G) return;
-  c.g = 0;
-  for (++c.s; c.s < p.S; ++c.s) {
-    c.sp = seq_span(p, c.s, false);
-    if (c.sp.nb > 0) return;
-  }
-}
-
-// Slice [t0, t0 + count) of the T-tile stream owned by CTA c of C (equal split, the
-// first T % C CTAs take one extra tile).
-__device__ __forceinline__ void cta_slice(long long T, int C, int c, long long* t0, long long* count) {
-  const long long base = T / C, rem = T % C;
-  *t0 = c * base + (c < rem ? c : rem);
-  *count = base + (c < rem ? 1 : 0);
-}
-
-// CTA owning tile t (inverse of cta_slice).
-__device__ __forceinline__ int cta_of(long long t, long long T, int C) {
-  const long long base = T / C, rem = T % C;
-  const long long big = rem * (base + 1);
-  return static_cast<int>(t < big ? t / (base + 1) : rem + (t - big) / base);
-}
-
-// Load n consecutive elements of type IO as floats (n * sizeof(IO) is a multiple of 16).
-template <typename IO, int N>
-__device__ __forceinline__ void load_floats(const IO* src, float* dst) {
-  constexpr int EVIO = Elem<IO>::kEV;
-  static_assert(N % EVIO == 0, "vector multiple");
-#pragma unroll
-  for (int i = 0; i < N / EVIO; ++i) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + i);
-    Elem<IO>::to_float(v, dst + i * EVIO);
-  }
-}
-
-template <typename IO, int N>
-__device__ __forceinline__ void store_floats(IO* dst, const float* src) {
-  static_assert((N * sizeof(IO)) % 16 == 0, "vector multiple");
-  IO tmp[N];
-#pragma unroll
-  for (int i = 0; i < N; ++i) tmp[i] = float_to<IO>(src[i]);
-#pragma unroll
-  for (int i = 0; i < static_cast<int>(N * sizeof(IO) / 16); ++i)
-    reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(tmp)[i];
-}
 
 // ---------------------------------------------------------------------------------------
 // Partition kernel.
@@ -154,67 +52,22 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   static_assert(LPR >= 1 && LPR <= 32 && 32 % LPR == 0, "lane mapping");
 
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ long long s_chunk[kMaxThreads];
-  __shared__ long long s_total;
-  __shared__ int s_first_seq;
-  __shared__ long long s_first_prefix;
 
   const int tt = TT > 0 ? TT : p.tt;
   const int HG = p.HG, G = p.G, NS = p.nstage, QW = p.QW;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nthr = blockDim.x;
 
   // Programmatic dependent launch: let the merge kernel get resident now, and wait for
   // the previous kernel of the stream (e.g. the cache write) before reading anything.
   grid_dependency_launch_next();
   grid_dependency_wait();
 
-  // ---- 1. Plan: tiles per sequence, their prefix sum, and this CTA's slice. -----------
-  const int chunk = (p.S + nthr - 1) / nthr;
-  const int s_lo = min(p.S, threadIdx.x * chunk), s_hi = min(p.S, s_lo + chunk);
-  long long mine = 0;
-  for (int s = s_lo; s < s_hi; ++s) mine += seq_span(p, s, blockIdx.x == 0).nb;
-  s_chunk[threadIdx.x] = mine;
-  if (threadIdx.x == 0) s_first_seq = -1;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    long long run = 0;
-    for (int i = 0; i < nthr; ++i) {
-      const long long v = s_chunk[i];
-      s_chunk[i] = run;
-      run += v;
-    }
-    s_total = run;
-  }
-  __syncthreads();
-  const long long per_group = s_total;  // tiles of one head group over all sequences
-  const long long T = per_group * G;
-  const long long my_prefix = s_chunk[threadIdx.x];
-  if (blockIdx.x == 0) {  // publish the per-sequence prefix for the merge kernel
-    long long r = my_prefix;
-    for (int s = s_lo; s < s_hi; ++s) {
-      p.ws_prefix[s] = r;
-      r += seq_span(p, s, false).nb;
-    }
-    if (threadIdx.x == 0) p.ws_prefix[p.S] = per_group;
-  }
-  long long t0, count;
-  cta_slice(T, p.num_ctas, blockIdx.x, &t0, &count);
+  // ---- 1. Plan: this CTA's slice of the tile stream. ------------------------------------
+  __shared__ PlanScratch plan;
+  Cursor start;
+  long long t0 = 0;
+  const long long count = plan_slice(p, plan, &t0, &start);
   if (count == 0) return;  // uniform across the CTA; no barrier in use yet
-
-  // Sequence holding t0: sequence s starts at tile G * prefix(s).
-  if (t0 >= G * my_prefix && t0 < G * (my_prefix + mine)) {
-    long long r = my_prefix;
-    for (int s = s_lo; s < s_hi; ++s) {
-      const int nb = seq_span(p, s, false).nb;
-      if (t0 < G * (r + nb)) {
-        s_first_seq = s;
-        s_first_prefix = r;
-        break;
-      }
-      r += nb;
-    }
-  }
 
   // ---- 2. Pipeline barriers. --------------------------------------------------------
   const uint32_t bar_base = smem_u32(smem);
@@ -229,19 +82,7 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
     fence_barrier_init();
   }
   __syncthreads();
-  if (s_first_seq < 0) {  // cannot happen when count > 0; never index with it
-    if (threadIdx.x == 0) decode_error(PA_DEVERR_TIMEOUT);
-    return;
-  }
 
-  Cursor start;
-  start.s = s_first_seq;
-  start.sp = seq_span(p, start.s, false);
-  {
-    const long long rem = t0 - G * s_first_prefix;
-    start.g = static_cast<int>(rem / start.sp.nb);
-    start.j = static_cast<int>(rem % start.sp.nb);
-  }
   const int n = static_cast<int>(count);
 
   if (warp == QW) {
@@ -536,10 +377,11 @@ pa_status get_encoder(EncodeTiledFn* out) {
 }
 
 pa_status encode(EncodeTiledFn fn, CUtensorMap* map, CUtensorMapDataType type, int rank, const void* base,
-                 const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box) {
+                 const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
+                 CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE) {
   const cuuint32_t estride[3] = {1, 1, 1};
   CUresult r = fn(map, type, rank, const_cast<void*>(base), dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
   return PA_OK;
 }
@@ -671,6 +513,83 @@ extern "C" size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int hea
 
 namespace pa {
 namespace {
+
+bool g_tensor_cores = true;  // pa_decode_use_tensor_cores()
+
+// Grouped-query decode on the tensor cores: one CTA per SM, 128-token tiles of one cached
+// head (pa_decode_tc.cu), then the shared merge kernel.
+pa_status decode_launch_tc(void* out, const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, const int32_t* context_lens, int num_seqs, int num_q_heads,
+                           int num_kv_heads, int block_size, int num_blocks, int max_blocks_per_seq, float scale,
+                           int window, pa_dtype io_dtype, void* workspace, int sms, cudaStream_t s) {
+  const int head_dim = 128;
+  const int GQ = num_q_heads / num_kv_heads;
+  const int C = sms;
+  const long long rows = static_cast<long long>(C) * GQ + static_cast<long long>(num_seqs) * num_q_heads;
+  const WsLayout lay = ws_layout(num_seqs, head_dim, rows);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  EncodeTiledFn enc = nullptr;
+  pa_status st = get_encoder(&enc);
+  if (st != PA_OK) return st;
+  const CUtensorMapDataType ttype = io_dtype == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUtensorMap tmK, tmV, tmQ;
+  {
+    // [NB*bs rows][Hkv][128]: boxes of one block's rows x one head x 64 dims, 128-byte swizzle
+    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(num_kv_heads),
+                                static_cast<cuuint64_t>(num_blocks) * block_size};
+    const cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(num_kv_heads) * 256};
+    const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(block_size)};
+    if ((st = encode(enc, &tmK, ttype, 3, k_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != PA_OK) return st;
+    if ((st = encode(enc, &tmV, ttype, 3, v_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != PA_OK) return st;
+  }
+  {
+    // q as [S*Hq rows][128]: the GQ rows of one head group x 64 dims
+    const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(num_seqs) * num_q_heads};
+    const cuuint64_t strides[1] = {256};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(GQ)};
+    if ((st = encode(enc, &tmQ, ttype, 2, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != PA_OK) return st;
+  }
+  DecodeParams prm = {};
+  prm.out = out;
+  prm.q = q;
+  prm.block_tables = block_tables;
+  prm.context_lens = context_lens;
+  prm.ws_prefix = reinterpret_cast<long long*>(ws + lay.prefix_off);
+  prm.ws_ml = reinterpret_cast<float*>(ws + lay.ml_off);
+  prm.ws_acc = reinterpret_cast<float*>(ws + lay.acc_off);
+  prm.S = num_seqs;
+  prm.H = num_kv_heads;
+  prm.bs = block_size;
+  prm.MB = max_blocks_per_seq;
+  prm.NB = num_blocks;
+  prm.window = window;
+  prm.tt = tc_decode_tile_tokens();
+  prm.tpb = 1;
+  prm.HG = 1;
+  prm.G = num_kv_heads;
+  prm.num_ctas = C;
+  prm.nstage = 0;
+  prm.Hq = num_q_heads;
+  prm.GQ = GQ;
+  prm.QW = GQ;
+  prm.qscale = scale * 1.4426950408889634f;
+
+  cudaEvent_t ev[3];
+  profiling_next_events(ev);
+  if (ev[0]) cudaEventRecord(ev[0], s);
+  if ((st = tc_decode_launch(tmK, tmV, tmQ, prm, io_dtype, C, s)) != PA_OK) return st;
+  if (ev[1]) cudaEventRecord(ev[1], s);
+  {
+    void* args[] = {&prm};
+    const long long items = static_cast<long long>(num_seqs) * num_q_heads;
+    const unsigned grid = static_cast<unsigned>((items + kMergeWarps - 1) / kMergeWarps);
+    cudaError_t err = launch_dependent(select_merge(io_dtype, head_dim), dim3(grid), dim3(32 * kMergeWarps), 0, s, args);
+    if (err != cudaSuccess) return cuda_fail(err, "launching the decode merge kernel");
+  }
+  if (ev[2]) cudaEventRecord(ev[2], s);
+  return PA_OK;
+}
+
 pa_status decode_launch(void* out, const void* q, const void* k_cache, const void* v_cache,
                                             const void* k_scale, const void* v_scale, const int32_t* block_tables,
                                             const int32_t* context_lens, int num_seqs, int num_q_heads, int num_heads, int head_dim,
@@ -684,8 +603,12 @@ pa_status decode_launch(void* out, const void* q, const void* k_cache, const voi
   if (num_q_heads % num_heads != 0)
     return fail(PA_ERR_INVALID_ARG, "num_q_heads (%d) must be a multiple of num_kv_heads (%d)", num_q_heads, num_heads);
   const int GQ = num_q_heads / num_heads;  // query heads per cached head
-  if (GQ > kMaxHeadGroup)
-    return fail(PA_ERR_UNSUPPORTED, "%d query heads per cached head (supported: up to %d)", GQ, kMaxHeadGroup);
+  const bool use_tc = g_tensor_cores && tc_decode_eligible(io_dtype, cache_dtype, head_dim, block_size, GQ);
+  if (GQ > kMaxHeadGroup && !use_tc)
+    return fail(PA_ERR_UNSUPPORTED,
+                "%d query heads per cached head: up to %d on the CUDA-core kernel; more need the tensor-core "
+                "kernel (fp16/bf16 cache, head_dim 128, block_size a multiple of 8 dividing 128, up to 16)",
+                GQ, kMaxHeadGroup);
   if (head_dim != 64 && head_dim != 128) return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", head_dim);
   if (block_size < 1 || block_size > 32) return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 1..32)", block_size);
   if (num_blocks <= 0 || max_blocks_per_seq <= 0) return fail(PA_ERR_INVALID_ARG, "num_blocks and max_blocks_per_seq must be positive");
@@ -716,6 +639,10 @@ pa_status decode_launch(void* out, const void* q, const void* k_cache, const voi
   const size_t need = pa_decode_workspace_bytes(num_seqs, num_q_heads, head_dim);
   if (workspace_bytes < need)
     return fail(PA_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+  if (use_tc)
+    return decode_launch_tc(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_q_heads, num_heads,
+                            block_size, num_blocks, max_blocks_per_seq, scale, window, io_dtype, workspace, sms,
+                            static_cast<cudaStream_t>(stream));
 
   // Rows per tile: the largest divisor of block_size in [8, 16] (the whole block if none),
   // so 32-token blocks stream as two 16-row tiles and keep four heads per CTA.
@@ -917,4 +844,9 @@ extern "C" pa_status paged_attention_decode_static_scratch(
   return paged_attention_decode(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, num_seqs,
                                 num_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, scale, window,
                                 io_dtype, cache_dtype, scratch, kStaticScratchBytes, stream);
+}
+
+extern "C" pa_status pa_decode_use_tensor_cores(int enable) {
+  g_tensor_cores = enable != 0;
+  return PA_OK;
 }

@@ -1,0 +1,444 @@
+// pa_decode_tc.cu -- grouped-query paged decode on the 5th-generation tensor cores (sm_100a).
+//
+// With GQ query heads sharing one cached head, every cached K/V byte feeds GQ dot products
+// and GQ weighted sums.  At 8 query heads per cached head that is more FP32 FMA work per
+// HBM byte than the CUDA cores can retire at full bandwidth, so here the two contractions
+// of a 128-token tile run as tcgen05 MMAs with fp32 accumulators in tensor memory (TMEM):
+//
+//   S^T[128 tok x 16]  = K[128 tok x 128 d] . Q^T[128 d x 16 heads]     (K-major A, K-major B)
+//   O^T[128 d   x 16]  = V^T[128 d x 128 tok] . P^T[128 tok x 16 heads] (MN-major A and B)
+//
+// (query heads padded to N = 16; M = 128 puts one token, then one head dim, on each TMEM lane).
+// The pages fix only the cache layout and the block-table walk ("KV Cache memory
+// optimisation and PagedAttention" (yunthe.com), section "PagedAttention注意力计算流程";
+// "vLLM source first look: PagedAttention memory design" (trdm.cn), section 三); the
+// grouped-query tile is this library's design.
+//
+// Roles (one CTA per SM, 6 warps):
+//   warp 0      TMA producer: per tile, the q rows of the head group and, block by block,
+//               the 64-dim halves of each attended K and V block (128-byte swizzle) into a
+//               3-stage ring; block-table entries are loaded by the warp's lanes in parallel.
+//   warp 1      TMEM owner and MMA issuer (one lane): score MMA of tile i+1 is issued before
+//               the value MMA of tile i, so it overlaps the softmax of tile i.
+//   warps 2..5  softmax (thread = token row of S^T) and accumulation (thread = head dim row
+//               of O^T): online softmax in base 2, probabilities written as the B operand of
+//               the value MMA, V rows of unattended tokens zeroed, running output rescaled in
+//               registers.  Segment ends write the output or a partial (m, l, acc) exactly
+//               like the CUDA-core kernel, so the same merge kernel finishes split segments.
+// Every wait is bounded; a wait that gives up sets an abort flag that ends all the others.
+#include <cfloat>
+#include <mutex>
+#include <type_traits>
+
+#include "pa_decode_shared.cuh"
+#include "pa_device.cuh"
+#include "pa_host.h"
+
+namespace pa {
+namespace {
+
+constexpr int kTokens = 128;                    // tile rows (MMA M of the score product)
+constexpr int kDim = 128;                       // head_dim
+constexpr int kHeadsN = 16;                     // query heads per cached head, padded (MMA N)
+constexpr int kHalf = kTokens * 128;            // one 64-dim half of a tile: 128 rows x 128 B
+constexpr int kQHalf = kHeadsN * 128;           // one 64-dim half of the q rows: 16 rows x 128 B
+constexpr int kStageBytes = 4 * kHalf + 2 * kQHalf;  // K lo, K hi, V lo, V hi, Q lo, Q hi
+constexpr int kStages = 3;
+constexpr int kPBytes = kTokens * kHeadsN * 2;  // one probability operand, 128 tokens x 16 heads
+constexpr int kPBuffers = 4;                    // 2 tiles in flight x (hi, lo) parts
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 64;              // S0 [0,16)  S1 [16,32)  O0 [32,48)  O1 [48,64)
+constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + kPBuffers * kPBytes;
+
+struct TcShared {
+  uint64_t full[kStages], empty[kStages];       // TMA ring
+  uint64_t s_full[2], s_empty[2];               // score accumulators in TMEM
+  uint64_t p_full[2], o_full[2];                // probabilities written / value MMA done
+  uint32_t tmem_base;
+  int abort;
+  float red[2][4][kHeadsN];                     // per-tile maxima across the softmax warps (by tile parity)
+  float red_l[4][kHeadsN];                      // softmax denominators at segment ends
+};
+
+__device__ __forceinline__ uint32_t bits16(__half x) { return __half_as_ushort(x); }
+__device__ __forceinline__ uint32_t bits16(__nv_bfloat16 x) { return __bfloat16_as_ushort(x); }
+
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+  }
+  *abort = 1;
+  decode_error(PA_DEVERR_TIMEOUT);
+  return false;
+}
+
+// Row r of a probability operand P^T (MN-major, 32-byte swizzle): 16 heads = 32 B, the two
+// 16-byte chunks trade places on rows 4..7 of every 8.
+__device__ __forceinline__ void store_p_row(uint32_t buf, int r, const uint32_t* w) {
+  const uint32_t row = buf + r * 32;
+  const uint32_t sw = (r >> 2) & 1;
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + 16 * sw), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+               "r"(w[3]) : "memory");
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + 16 * (sw ^ 1)), "r"(w[4]), "r"(w[5]), "r"(w[6]),
+               "r"(w[7]) : "memory");
+}
+
+// IO: fp16 or bf16 cache and queries.  NH: query heads a thread tracks (8 or 16 >= GQ).
+// bf16 probabilities are split into hi + lo bf16 parts and the value MMA runs on both, so
+// the weights keep ~16 significant bits (one bf16 part alone keeps 8).
+template <typename IO, int NH>
+__global__ void __launch_bounds__(kThreads, 1)
+decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const __grid_constant__ CUtensorMap tmQ, const DecodeParams p) {
+  constexpr bool kSplit = std::is_same<IO, __nv_bfloat16>::value;
+  constexpr uint32_t kFmt = kSplit ? 1u : 0u;
+  constexpr uint32_t kIdescS = mma_idesc_f16(kFmt, 0, 0, kTokens, kHeadsN);  // K-major A and B
+  constexpr uint32_t kIdescO = mma_idesc_f16(kFmt, 1, 1, kDim, kHeadsN);     // MN-major A and B
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ TcShared sh;
+  __shared__ PlanScratch plan;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int GQ = p.GQ;
+
+  grid_dependency_launch_next();
+  grid_dependency_wait();
+
+  Cursor start;
+  long long t0 = 0;
+  const long long count = plan_slice(p, plan, &t0, &start);
+  if (count == 0) return;
+  const int n = static_cast<int>(count);
+
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;  // swizzle atoms are 1024-B aligned
+  auto stage = [&](int st) { return base + st * kStageBytes; };
+  auto pbuf = [&](int b, int part) { return base + kStages * kStageBytes + (2 * b + part) * kPBytes; };
+  const uint32_t full0 = smem_u32(&sh.full[0]), empty0 = smem_u32(&sh.empty[0]);
+  const uint32_t s_full0 = smem_u32(&sh.s_full[0]), s_empty0 = smem_u32(&sh.s_empty[0]);
+  const uint32_t p_full0 = smem_u32(&sh.p_full[0]), o_full0 = smem_u32(&sh.o_full[0]);
+  volatile int* abort = &sh.abort;
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(full0 + 8 * st, 1);
+      mbar_init(empty0 + 8 * st, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(s_full0 + 8 * b, 1);
+      mbar_init(s_empty0 + 8 * b, 128);
+      mbar_init(p_full0 + 8 * b, 128);
+      mbar_init(o_full0 + 8 * b, 1);
+    }
+    sh.abort = 0;
+    fence_barrier_init();
+  }
+  // The q rows of a head group fill rows 0..GQ-1 of each stage's 16-row q block; rows
+  // GQ..15 stay zero (padding of the MMA N dimension).
+  for (int i = threadIdx.x; i < kStages * 2 * kQHalf / 16; i += kThreads) {
+    const int st = i / (2 * kQHalf / 16), off = (i % (2 * kQHalf / 16)) * 16;
+    uint8_t* ptr = smem_raw + (stage(st) - smem_u32(smem_raw)) + 4 * kHalf + off;
+    *reinterpret_cast<uint4*>(ptr) = make_uint4(0, 0, 0, 0);
+  }
+  fence_proxy_async_shared();
+  if (warp == 1) tmem_alloc(smem_u32(&sh.tmem_base), kTmemCols);
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = sh.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer --
+    const uint64_t policy = l2_policy_evict_first();
+    if (lane == 0) {
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      prefetch_tensormap(&tmQ);
+    }
+    const int bs = p.bs;
+    const int bpt = kTokens / bs;  // blocks per tile
+    Cursor c = start;
+    int issued = 0;
+    for (; issued < n; ++issued) {
+      const int st = issued % kStages;
+      const int tok0 = (c.sp.first_t + c.j) * kTokens;
+      const int lb_first = tok0 / bs;
+      const int lb_lo = max(lb_first, c.sp.lo / bs), lb_hi = min(lb_first + bpt - 1, (c.sp.ctx - 1) / bs);
+      const int nload = lb_hi - lb_lo + 1;
+      int pb = lane < nload ? __ldg(p.block_tables + static_cast<size_t>(c.s) * p.MB + lb_lo + lane) : 0;
+      if (lane < nload && (pb < 0 || pb >= p.NB)) {
+        decode_error(PA_DEVERR_TABLE);
+        pb = 0;
+      }
+      bool ok = true;
+      if (lane == 0) {
+        if (issued >= kStages) ok = wait_or_abort(empty0 + 8 * st, ((issued / kStages) - 1) & 1, abort);
+        if (ok) {
+          const uint32_t bar = full0 + 8 * st;
+          mbar_arrive_expect_tx(bar, 2u * GQ * 128u + static_cast<uint32_t>(nload) * 4u * bs * 128u);
+          const uint32_t sb = stage(st);
+          const int qrow = c.s * p.Hq + c.g * GQ;
+          tma_load_2d(sb + 4 * kHalf, &tmQ, bar, 0, qrow, policy);
+          tma_load_2d(sb + 4 * kHalf + kQHalf, &tmQ, bar, 64, qrow, policy);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      for (int i = 0; i < nload; ++i) {
+        const int b = __shfl_sync(0xffffffffu, pb, i);
+        if (lane == 0) {
+          const uint32_t bar = full0 + 8 * st;
+          const uint32_t row = static_cast<uint32_t>(lb_lo + i - lb_first) * bs * 128u;
+          const uint32_t sb = stage(st);
+          tma_load_3d(sb + row, &tmK, bar, 0, c.g, b * bs, policy);
+          tma_load_3d(sb + kHalf + row, &tmK, bar, 64, c.g, b * bs, policy);
+          tma_load_3d(sb + 2 * kHalf + row, &tmV, bar, 0, c.g, b * bs, policy);
+          tma_load_3d(sb + 3 * kHalf + row, &tmV, bar, 64, c.g, b * bs, policy);
+        }
+      }
+      advance(c, p);
+    }
+    if (lane == 0)  // never leave with copies in flight
+      for (int k = issued - kStages < 0 ? 0 : issued - kStages; k < issued; ++k)
+        wait_or_abort(full0 + 8 * (k % kStages), (k / kStages) & 1, abort);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      auto score_mma = [&](int i) -> bool {  // S^T[i % 2] = K . Q^T
+        const int st = i % kStages, b = i % 2;
+        if (!wait_or_abort(full0 + 8 * st, (i / kStages) & 1, abort)) return false;
+        if (i >= 2 && !wait_or_abort(s_empty0 + 8 * b, ((i / 2) - 1) & 1, abort)) return false;
+        tc_fence_after_sync();
+        const uint32_t sb = stage(st);
+#pragma unroll
+        for (int kk = 0; kk < kDim / 16; ++kk) {
+          const uint32_t koff = (kk / 4) * kHalf + (kk % 4) * 32;   // 16 dims = 32 B inside a swizzled row
+          const uint32_t qoff = 4 * kHalf + (kk / 4) * kQHalf + (kk % 4) * 32;
+          const uint64_t a = smem_desc(sb + koff, 16, 1024, kSwizzle128B);
+          const uint64_t bdesc = smem_desc(sb + qoff, 16, 1024, kSwizzle128B);
+          tc_mma_f16(tmem + b * kHeadsN, a, bdesc, kIdescS, kk > 0);
+        }
+        tc_commit(s_full0 + 8 * b);
+        return true;
+      };
+      bool ok = score_mma(0);
+      for (int i = 0; ok && i < n; ++i) {
+        const int b = i % 2;
+        if (i + 1 < n && !score_mma(i + 1)) break;
+        if (!wait_or_abort(p_full0 + 8 * b, (i / 2) & 1, abort)) break;
+        tc_fence_after_sync();
+        const uint32_t sb = stage(i % kStages);
+        const uint32_t o_tmem = tmem + 2 * kHeadsN + b * kHeadsN;
+#pragma unroll
+        for (int part = 0; part < (kSplit ? 2 : 1); ++part) {
+#pragma unroll
+          for (int kk = 0; kk < kTokens / 16; ++kk) {  // 16 tokens per MMA: two 8-row swizzle atoms
+            const uint64_t a = smem_desc(sb + 2 * kHalf + kk * 2048, kHalf, 1024, kSwizzle128B);
+            const uint64_t bdesc = smem_desc(pbuf(b, part) + kk * 512, kPBytes, 256, kSwizzle32B);
+            tc_mma_f16(o_tmem, a, bdesc, kIdescO, part > 0 || kk > 0);
+          }
+        }
+        tc_commit(o_full0 + 8 * b);
+        tc_commit(empty0 + 8 * (i % kStages));
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------- softmax + accumulation warps --
+    const int q4 = warp & 3;              // TMEM lane quarter this warp may access
+    const int r = 32 * q4 + lane;         // token row (softmax) and head-dim row (accumulate)
+    const uint32_t lane_addr = static_cast<uint32_t>(32 * q4) << 16;
+    float m[NH], l[NH], acc[NH], alpha_prev[NH];
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      m[h] = -FLT_MAX;
+      l[h] = 0.f;
+      acc[h] = 0.f;
+      alpha_prev[h] = 1.f;
+    }
+    // Fold the value product of tile t into the running output (thread = head dim r).
+    auto accumulate = [&](int t, const float* alpha) -> bool {
+      if (!wait_or_abort(o_full0 + 8 * (t % 2), (t / 2) & 1, abort)) return false;
+      tc_fence_after_sync();
+      float o[NH];
+      tmem_load<NH>(tmem + lane_addr + 2 * kHeadsN + (t % 2) * kHeadsN, o);
+      tc_fence_before_sync();
+#pragma unroll
+      for (int h = 0; h < NH; ++h) acc[h] = acc[h] * alpha[h] + o[h];
+      return true;
+    };
+    Cursor c = start;
+    bool seg_from_start = (c.j == 0);
+    bool pending = false;  // the value product of the previous tile is not folded in yet
+    for (int i = 0; i < n; ++i) {
+      const int b = i % 2, st = i % kStages;
+      if (!wait_or_abort(s_full0 + 8 * b, (i / 2) & 1, abort)) break;
+      tc_fence_after_sync();
+      float sc[NH];
+      tmem_load<NH>(tmem + lane_addr + b * kHeadsN, sc);
+      tc_fence_before_sync();
+      mbar_arrive(s_empty0 + 8 * b);
+
+      const int tok = (c.sp.first_t + c.j) * kTokens + r;
+      const bool valid = tok >= c.sp.lo && tok < c.sp.ctx;
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        sc[h] = (valid && h < GQ) ? sc[h] * p.qscale : -INFINITY;
+        float x = sc[h];
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
+        if (lane == 0) sh.red[b][q4][h] = x;
+      }
+      named_barrier_sync(1, 128);
+      float alpha[NH];
+      uint32_t w_hi[8], w_lo[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) w_hi[k] = w_lo[k] = 0;
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        const float t = fmaxf(fmaxf(sh.red[b][0][h], sh.red[b][1][h]), fmaxf(sh.red[b][2][h], sh.red[b][3][h]));
+        const float m_new = fmaxf(m[h], t);
+        alpha[h] = exp2f(m[h] - m_new);
+        m[h] = m_new;
+        const float pr = sc[h] == -INFINITY ? 0.f : exp2f(sc[h] - m_new);
+        const IO hi = float_to<IO>(pr);
+        w_hi[h / 2] |= bits16(hi) << (16 * (h & 1));
+        if (kSplit) {
+          const IO lo = float_to<IO>(pr - static_cast<float>(hi));
+          w_lo[h / 2] |= bits16(lo) << (16 * (h & 1));
+          l[h] = l[h] * alpha[h] + pr;
+        } else {
+          l[h] = l[h] * alpha[h] + static_cast<float>(hi);  // the rounded weight the MMA uses
+        }
+      }
+      store_p_row(pbuf(b, 0), r, w_hi);
+      if (kSplit) store_p_row(pbuf(b, 1), r, w_lo);
+      if (!valid) {  // unattended rows may hold anything (NaN): give the value MMA zeros
+        const uint32_t v0 = stage(st) + 2 * kHalf + r * 128;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(v0 + 16 * k), "r"(0) : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(v0 + kHalf + 16 * k), "r"(0) : "memory");
+        }
+      }
+      fence_proxy_async_shared();
+      mbar_arrive(p_full0 + 8 * b);
+
+      // Overlap: the value MMA of tile i runs while the previous tile is folded in.
+      if (pending && !accumulate(i - 1, alpha_prev)) break;
+      pending = false;
+      const bool seg_last = (c.j == c.sp.nb - 1);
+      if (!(seg_last || i == n - 1)) {
+        pending = true;
+#pragma unroll
+        for (int h = 0; h < NH; ++h) alpha_prev[h] = alpha[h];
+      } else {
+        if (!accumulate(i, alpha)) break;
+        // Softmax denominators: every thread holds the sums of its own token rows.
+        float lt[NH];
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+          float x = l[h];
+#pragma unroll
+          for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+          lt[h] = x;
+        }
+        if (lane == 0)
+#pragma unroll
+          for (int h = 0; h < NH; ++h) sh.red_l[q4][h] = lt[h];
+        named_barrier_sync(1, 128);
+#pragma unroll
+        for (int h = 0; h < NH; ++h) lt[h] = sh.red_l[0][h] + sh.red_l[1][h] + sh.red_l[2][h] + sh.red_l[3][h];
+        named_barrier_sync(1, 128);  // sh.red_l is free again
+        const int h0 = c.g * GQ;
+        if (seg_from_start && seg_last) {
+          IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(c.s) * p.Hq + h0) * kDim + r;
+#pragma unroll
+          for (int h = 0; h < NH; ++h)
+            if (h < GQ) orow[static_cast<size_t>(h) * kDim] = float_to<IO>(acc[h] / lt[h]);
+        } else {
+          const long long slot = blockIdx.x + static_cast<long long>(c.s) * p.G + c.g;
+#pragma unroll
+          for (int h = 0; h < NH; ++h) {
+            if (h >= GQ) continue;
+            p.ws_acc[(slot * GQ + h) * kDim + r] = acc[h];
+            if (r == 0) {
+              p.ws_ml[(slot * GQ + h) * 2 + 0] = m[h];
+              p.ws_ml[(slot * GQ + h) * 2 + 1] = lt[h];
+            }
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+          m[h] = -FLT_MAX;
+          l[h] = 0.f;
+          acc[h] = 0.f;
+        }
+      }
+      if (i + 1 < n) {
+        advance(c, p);
+        if (c.j == 0) seg_from_start = true;
+      }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+cudaError_t read_tc_error(uint32_t* flags, int clear) {
+  unsigned int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_decode_error, sizeof v);
+  if (e != cudaSuccess) return e;
+  *flags = v;
+  if (clear && v) {
+    const unsigned int z = 0;
+    e = cudaMemcpyToSymbol(g_decode_error, &z, sizeof z);
+  }
+  return e;
+}
+
+struct RegisterTc {
+  RegisterTc() { register_device_error_reader(read_tc_error); }
+} g_register_tc;
+
+}  // namespace
+
+bool tc_decode_eligible(pa_dtype io, pa_dtype cache, int head_dim, int block_size, int group) {
+  return (io == PA_F16 || io == PA_BF16) && cache == io && head_dim == kDim && block_size >= 8 &&
+         block_size <= kTokens && block_size % 8 == 0 && kTokens % block_size == 0 && group >= 4 &&
+         group <= kHeadsN;
+}
+
+size_t tc_decode_smem_bytes() { return kSmemBytes; }
+
+int tc_decode_tile_tokens() { return kTokens; }
+
+pa_status tc_decode_launch(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
+                           const DecodeParams& prm, pa_dtype io, int grid, cudaStream_t stream) {
+  const bool small = prm.GQ <= 8;
+  const void* fn = io == PA_BF16
+                       ? (small ? reinterpret_cast<const void*>(&decode_gqa_tc_kernel<__nv_bfloat16, 8>)
+                                : reinterpret_cast<const void*>(&decode_gqa_tc_kernel<__nv_bfloat16, 16>))
+                       : (small ? reinterpret_cast<const void*>(&decode_gqa_tc_kernel<__half, 8>)
+                                : reinterpret_cast<const void*>(&decode_gqa_tc_kernel<__half, 16>));
+  static std::once_flag once[4];
+  cudaError_t attr_err = cudaSuccess;
+  std::call_once(once[(io == PA_BF16 ? 2 : 0) + (small ? 1 : 0)], [&] {
+    attr_err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(tensor-core decode)");
+  CUtensorMap k = tmK, v = tmV, q = tmQ;
+  DecodeParams p = prm;
+  void* args[] = {&k, &v, &q, &p};
+  cudaError_t err = launch_dependent(fn, dim3(grid), dim3(kThreads), kSmemBytes, stream, args);
+  if (err != cudaSuccess) return cuda_fail(err, "launching the tensor-core decode kernel");
+  return PA_OK;
+}
+
+}  // namespace pa

@@ -1,6 +1,6 @@
-// pa_device.cuh -- device-side building blocks shared by the sm_100a kernels:
-// element traits, 16-byte vector conversion, mbarrier + TMA wrappers (inline PTX) and the
-// device error word.  Internal header; not part of the C ABI.
+// pa_device.cuh -- device-side building blocks shared by the sm_100a kernels: element
+// traits, 16-byte vector conversion, mbarrier / TMA / tcgen05 wrappers (inline PTX).
+// Internal header; not part of the C ABI.
 #pragma once
 
 #include <cuda.h>
@@ -13,15 +13,6 @@
 #include "../../include/pagedattn.h"
 
 namespace pa {
-
-// ---------------------------------------------------------------------------------------
-// Device error word (OR of PA_DEVERR_* bits), one per device per process.
-// ---------------------------------------------------------------------------------------
-extern __device__ unsigned int g_device_error;
-
-__device__ __forceinline__ void raise_device_error(unsigned int bits) {
-  atomicOr(&g_device_error, bits);
-}
 
 // ---------------------------------------------------------------------------------------
 // Element traits.  A 16-byte vector holds EV elements; `to_float` widens EV elements of a
@@ -221,4 +212,89 @@ __device__ __forceinline__ void grid_dependency_launch_next() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+}  // namespace pa
+
+namespace pa {
+// ---------------------------------------------------------------------------------------
+// tcgen05 (5th-generation tensor core) wrappers: TMEM allocation, MMA issue and commit,
+// TMEM -> register loads, and the ordering fences between them and thread barriers.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before_sync() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after_sync() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D[tmem] (+)= A[smem desc] x B[smem desc], kind::f16 (fp16 or bf16 in, fp32 accumulate).
+__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on an mbarrier once every tcgen05 operation issued so far by this thread is done.
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+// 8 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_load8(uint32_t taddr, float* v) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 16 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_load16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <int N> __device__ __forceinline__ void tmem_load(uint32_t taddr, float* v);
+template <> __device__ __forceinline__ void tmem_load<8>(uint32_t taddr, float* v) { tmem_load8(taddr, v); }
+template <> __device__ __forceinline__ void tmem_load<16>(uint32_t taddr, float* v) { tmem_load16(taddr, v); }
+
+// Shared-memory matrix descriptor of a tcgen05 operand (start address, leading / stride
+// byte offsets, swizzle mode; version 1, base offset 0: swizzle atoms are aligned).
+enum SmemSwizzle : uint64_t { kSwizzleNone = 0, kSwizzle128B = 2, kSwizzle32B = 6 };
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                              SmemSwizzle swz) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3FFF) | (static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFF) << 16) |
+         (static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFF) << 32) | (1ull << 46) | (static_cast<uint64_t>(swz) << 61);
+}
+// Instruction descriptor, kind::f16: fp32 accumulator, A/B both fp16 (fmt 0) or bf16 (fmt 1),
+// A/B major (0 = K, 1 = MN), shape M x N.
+__host__ __device__ constexpr uint32_t mma_idesc_f16(uint32_t fmt, uint32_t a_mn, uint32_t b_mn, uint32_t M,
+                                                     uint32_t N) {
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | (a_mn << 15) | (b_mn << 16) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 }  // namespace pa

@@ -109,3 +109,28 @@ def test_head_count_mismatch_is_rejected(cuda_device):
     cl = torch.ones(1, dtype=torch.int32, device="cuda")
     with pytest.raises(ValueError):
         pa.paged_attention_decode(torch.empty_like(q), q, kc, kc, bt, cl, 0.1)
+
+
+@pytest.mark.parametrize("hq,hkv", [(16, 4), (64, 8), (32, 2)])
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_tensor_core_path(cuda_device, hq, hkv, dtype, bs):
+    """Groups of 4..16 query heads on fp16/bf16 caches run as tcgen05 MMAs; the result must
+    match the oracle, and the CUDA-core kernel where it applies (groups up to 8)."""
+    ctx = [0, 1, 127, 128, 129, 300, 2048, 5, 700]
+    case, ref, io = _case(hq + hkv + bs, hq, hkv, 128, bs, ctx, dtype)
+    tc = _run(case, ref, io, TOL[io])
+    if hq // hkv <= 8:
+        pa.use_tensor_cores(False)
+        try:
+            _run(case, ref, io, TOL[io])
+        finally:
+            pa.use_tensor_cores(True)
+
+
+def test_tensor_core_path_windows_and_long_contexts(cuda_device):
+    ctx = [1, 4095, 4096, 4097, 9000, 20000]
+    case, ref, io = _case(77, 64, 8, 128, 16, ctx, "bf16", window=4096)
+    _run(case, ref, io, TOL[io])
+    case, ref, io = _case(78, 32, 4, 128, 16, [32768], "fp16")
+    _run(case, ref, io, TOL[io])
