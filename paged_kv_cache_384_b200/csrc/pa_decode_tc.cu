@@ -18,8 +18,9 @@
 //   warp 0      TMA producer: per tile, the q rows of the head group and, block by block,
 //               the 64-dim halves of each attended K and V block (128-byte swizzle) into a
 //               3-stage ring; block-table entries are loaded by the warp's lanes in parallel.
-//   warp 1      TMEM owner and MMA issuer (one lane): score MMA of tile i+1 is issued before
-//               the value MMA of tile i, so it overlaps the softmax of tile i.
+//   warp 1      TMEM owner and MMA issuer (one lane): polls for ready work and issues the score
+//               MMA of the next landed tile or the value MMA of the oldest softmaxed tile,
+//               whichever is ready, so stages are released without waiting on later tiles.
 //   warps 2..5  softmax (thread = token row of S^T) and accumulation (thread = head dim row
 //               of O^T): online softmax in base 2, probabilities written as the B operand of
 //               the value MMA, V rows of unattended tokens zeroed, running output rescaled in
@@ -158,6 +159,17 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     }
     const int bs = p.bs;
     const int bpt = kTokens / bs;  // blocks per tile
+    // Block-table entries travel in 32-entry windows held one per lane, starting at a tile
+    // boundary.  The window after the current one is loaded in the background, and the
+    // first window of the sequence is kept for its other head groups, so the TMA issue
+    // rarely waits for a table load.
+    auto fetch = [&](int s, int from, int lim) -> int {
+      const int idx = from + lane;
+      return idx < lim ? __ldg(p.block_tables + static_cast<size_t>(s) * p.MB + idx) : 0;
+    };
+    int win_seq = -1, win_base = 0, win = 0;     // window in use
+    int pre_seq = -1, pre_base = 0, pre = 0;     // next window, in flight
+    int fst_seq = -1, fst_base = 0, fst = 0;     // first window of the sequence
     Cursor c = start;
     int issued = 0;
     for (; issued < n; ++issued) {
@@ -166,7 +178,20 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       const int lb_first = tok0 / bs;
       const int lb_lo = max(lb_first, c.sp.lo / bs), lb_hi = min(lb_first + bpt - 1, (c.sp.ctx - 1) / bs);
       const int nload = lb_hi - lb_lo + 1;
-      int pb = lane < nload ? __ldg(p.block_tables + static_cast<size_t>(c.s) * p.MB + lb_lo + lane) : 0;
+      const int lim = (c.sp.ctx - 1) / bs + 1;  // blocks of this sequence
+      if (!(c.s == win_seq && lb_lo >= win_base && lb_hi < win_base + 32)) {
+        if (c.s == pre_seq && lb_lo >= pre_base && lb_hi < pre_base + 32) {
+          win_seq = pre_seq, win_base = pre_base, win = pre;
+        } else if (c.s == fst_seq && lb_lo >= fst_base && lb_hi < fst_base + 32) {
+          win_seq = fst_seq, win_base = fst_base, win = fst;
+        } else {
+          win_seq = c.s, win_base = lb_first, win = fetch(c.s, lb_first, lim);
+        }
+        if (c.s != fst_seq && c.j == 0) fst_seq = win_seq, fst_base = win_base, fst = win;
+        pre_seq = c.s, pre_base = win_base + 32;
+        pre = pre_base < lim ? fetch(c.s, pre_base, lim) : 0;
+      }
+      int pb = __shfl_sync(0xffffffffu, win, (lb_lo - win_base + lane) & 31);
       if (lane < nload && (pb < 0 || pb >= p.NB)) {
         decode_error(PA_DEVERR_TABLE);
         pb = 0;
@@ -204,43 +229,60 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         wait_or_abort(full0 + 8 * (k % kStages), (k / kStages) & 1, abort);
   } else if (warp == 1) {
     // ------------------------------------------------------------------- MMA issuer --
+    // One lane polls both kinds of work and issues whichever is ready: the score MMA of
+    // the next tile whose K/V/q landed, or the value MMA of the oldest tile whose
+    // probabilities are written.  Neither waits behind the other, so a stage is released
+    // as soon as its value MMA is done.
     if (lane == 0) {
-      auto score_mma = [&](int i) -> bool {  // S^T[i % 2] = K . Q^T
-        const int st = i % kStages, b = i % 2;
-        if (!wait_or_abort(full0 + 8 * st, (i / kStages) & 1, abort)) return false;
-        if (i >= 2 && !wait_or_abort(s_empty0 + 8 * b, ((i / 2) - 1) & 1, abort)) return false;
-        tc_fence_after_sync();
-        const uint32_t sb = stage(st);
+      int s_next = 0, o_next = 0;
+      uint32_t idle = 0;
+      while (o_next < n) {
+        bool progressed = false;
+        if (s_next < n) {
+          const int st = s_next % kStages, b = s_next % 2;
+          if (mbar_try_wait(full0 + 8 * st, (s_next / kStages) & 1) &&
+              (s_next < 2 || mbar_try_wait(s_empty0 + 8 * b, ((s_next / 2) - 1) & 1))) {
+            tc_fence_after_sync();
+            const uint32_t sb = stage(st);
 #pragma unroll
-        for (int kk = 0; kk < kDim / 16; ++kk) {
-          const uint32_t koff = (kk / 4) * kHalf + (kk % 4) * 32;   // 16 dims = 32 B inside a swizzled row
-          const uint32_t qoff = 4 * kHalf + (kk / 4) * kQHalf + (kk % 4) * 32;
-          const uint64_t a = smem_desc(sb + koff, 16, 1024, kSwizzle128B);
-          const uint64_t bdesc = smem_desc(sb + qoff, 16, 1024, kSwizzle128B);
-          tc_mma_f16(tmem + b * kHeadsN, a, bdesc, kIdescS, kk > 0);
-        }
-        tc_commit(s_full0 + 8 * b);
-        return true;
-      };
-      bool ok = score_mma(0);
-      for (int i = 0; ok && i < n; ++i) {
-        const int b = i % 2;
-        if (i + 1 < n && !score_mma(i + 1)) break;
-        if (!wait_or_abort(p_full0 + 8 * b, (i / 2) & 1, abort)) break;
-        tc_fence_after_sync();
-        const uint32_t sb = stage(i % kStages);
-        const uint32_t o_tmem = tmem + 2 * kHeadsN + b * kHeadsN;
-#pragma unroll
-        for (int part = 0; part < (kSplit ? 2 : 1); ++part) {
-#pragma unroll
-          for (int kk = 0; kk < kTokens / 16; ++kk) {  // 16 tokens per MMA: two 8-row swizzle atoms
-            const uint64_t a = smem_desc(sb + 2 * kHalf + kk * 2048, kHalf, 1024, kSwizzle128B);
-            const uint64_t bdesc = smem_desc(pbuf(b, part) + kk * 512, kPBytes, 256, kSwizzle32B);
-            tc_mma_f16(o_tmem, a, bdesc, kIdescO, part > 0 || kk > 0);
+            for (int kk = 0; kk < kDim / 16; ++kk) {  // S^T[b] = K . Q^T, 16 dims per MMA
+              const uint32_t koff = (kk / 4) * kHalf + (kk % 4) * 32;  // 32 B steps inside a swizzled row
+              const uint32_t qoff = 4 * kHalf + (kk / 4) * kQHalf + (kk % 4) * 32;
+              tc_mma_f16(tmem + b * kHeadsN, smem_desc(sb + koff, 16, 1024, kSwizzle128B),
+                         smem_desc(sb + qoff, 16, 1024, kSwizzle128B), kIdescS, kk > 0);
+            }
+            tc_commit(s_full0 + 8 * b);
+            ++s_next;
+            progressed = true;
           }
         }
-        tc_commit(o_full0 + 8 * b);
-        tc_commit(empty0 + 8 * (i % kStages));
+        if (o_next < s_next) {
+          const int b = o_next % 2;
+          if (mbar_try_wait(p_full0 + 8 * b, (o_next / 2) & 1)) {
+            tc_fence_after_sync();
+            const uint32_t sb = stage(o_next % kStages);
+            const uint32_t o_tmem = tmem + 2 * kHeadsN + b * kHeadsN;
+#pragma unroll
+            for (int part = 0; part < (kSplit ? 2 : 1); ++part) {
+#pragma unroll
+              for (int kk = 0; kk < kTokens / 16; ++kk) {  // O^T[b] = V^T . P^T, 16 tokens per MMA
+                tc_mma_f16(o_tmem, smem_desc(sb + 2 * kHalf + kk * 2048, kHalf, 1024, kSwizzle128B),
+                           smem_desc(pbuf(b, part) + kk * 512, kPBytes, 256, kSwizzle32B), kIdescO, part > 0 || kk > 0);
+              }
+            }
+            tc_commit(o_full0 + 8 * b);
+            tc_commit(empty0 + 8 * (o_next % kStages));
+            ++o_next;
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          idle = 0;
+        } else if (*abort || ++idle > 4 * kWaitLimit) {
+          if (!*abort) decode_error(PA_DEVERR_TIMEOUT);
+          *abort = 1;
+          break;
+        }
       }
     }
     __syncwarp();
