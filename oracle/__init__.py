@@ -8,6 +8,8 @@ package imports nothing from it.
 Contents
   * ``paged_decode``    -- textbook softmax attention over K/V gathered through the
                            block table, fp64 (``pa_oracle.c``).
+  * ``paged_prefill``   -- the same for several causal query tokens per sequence
+                           (prefill / chunked prefill), fp64 (``pa_oracle.c``).
   * ``quant``           -- INT8 per-(token, head) quantiser (fp32 decisions).
   * ``cache_ops``       -- reshape_and_cache / copy_blocks placement definitions.
   * ``block_manager``   -- BlockTable / BlockManager allocator model.
@@ -42,6 +44,12 @@ def _load():
             ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_double, ctypes.c_int]
+        lib.orc_paged_prefill.restype = ctypes.c_int
+        lib.orc_paged_prefill.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int]
         lib.orc_f16_to_f64.restype = ctypes.c_double
         lib.orc_f16_to_f64.argtypes = [ctypes.c_uint16]
         lib.orc_bf16_to_f64.restype = ctypes.c_double
@@ -131,6 +139,49 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, window=
         out.ctypes.data, qa.ctypes.data, qd, ka.ctypes.data, va.ctypes.data, kd,
         ks.ctypes.data if ks is not None else None, vs.ctypes.data if vs is not None else None,
         bt.ctypes.data, cl.ctypes.data, S, H, Hc, D, bs, MB, NB, float(scale), int(window))
+    if st != 0:
+        raise ValueError(f"oracle: {_STATUS.get(st, st)}")
+    return out
+
+
+def paged_prefill(q, k_cache, v_cache, block_tables, cu_q, context_lens, scale, window=0,
+                  k_scale=None, v_scale=None):
+    """Causal attention of each sequence's newest q_len tokens over a paged KV cache.
+
+    q [T,Hq,D] packs the sequences' query tokens (sequence s owns rows cu_q[s]..cu_q[s+1]-1);
+    the chunk's own K/V are already in the cache, so query i of sequence s sits at position
+    context_lens[s] - q_len + i and attends up to itself (the last ``window`` tokens if
+    window > 0).  Other arguments as for ``paged_decode``.  Returns fp64 numpy [T,Hq,D].
+    """
+    lib = _load()
+    qa, qd = _raw(q)
+    ka, kd = _raw(k_cache)
+    va, vd = _raw(v_cache)
+    if kd != vd:
+        raise TypeError("k_cache and v_cache must share a dtype")
+    T, H, D = qa.shape
+    NB, bs, Hc, Dc = ka.shape
+    if Dc != D or H % Hc != 0 or va.shape != ka.shape:
+        raise ValueError("cache shape does not match q")
+    cu = _i32(cu_q).reshape(-1)
+    S = cu.size - 1
+    if S < 0 or (S > 0 and cu[-1] != T):
+        raise ValueError("cu_q must have S+1 entries ending at the number of query rows")
+    bt = _i32(block_tables).reshape(S, -1)
+    cl = _i32(context_lens).reshape(S)
+    MB = bt.shape[1] if bt.size else 1
+    if bt.size == 0:
+        bt = np.zeros((max(S, 1), 1), np.int32)
+    ks = vs = None
+    if kd in (I8, FP8):
+        ks, vs = _u16(k_scale), _u16(v_scale)
+        if ks.shape != (NB, bs, Hc) or vs.shape != (NB, bs, Hc):
+            raise ValueError("an int8/fp8 cache needs k_scale/v_scale of shape [NB, bs, H]")
+    out = np.zeros((T, H, D), np.float64)
+    st = lib.orc_paged_prefill(
+        out.ctypes.data, qa.ctypes.data, qd, ka.ctypes.data, va.ctypes.data, kd,
+        ks.ctypes.data if ks is not None else None, vs.ctypes.data if vs is not None else None,
+        bt.ctypes.data, cu.ctypes.data, cl.ctypes.data, S, H, Hc, D, bs, MB, NB, float(scale), int(window))
     if st != 0:
         raise ValueError(f"oracle: {_STATUS.get(st, st)}")
     return out

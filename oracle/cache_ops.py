@@ -54,3 +54,23 @@ def copy_blocks(k_cache, v_cache, pairs, k_scale_cache=None, v_scale_cache=None)
             k_scale_cache[dst] = k_scale_cache[src].copy()
             v_scale_cache[dst] = v_scale_cache[src].copy()
     return k_cache, v_cache
+
+
+def swap_blocks(src_k, src_v, dst_k, dst_v, pairs, src_scales=None, dst_scales=None):
+    """Move whole blocks between two pools: dst[d] = src[s] for each (s, d) pair.
+
+    "KV Cache memory optimisation and PagedAttention" (yunthe.com), section
+    "vLLM调度器与PagedAttention协同工作", item 3: when GPU memory runs short a preempted
+    request's KV blocks are moved out to CPU memory (swap-out) and brought back later
+    (swap-in); section "vLLM部署配置与PagedAttention参数调优" sizes that CPU pool
+    (swap_space).  The operation is a block copy between two pools that may differ in
+    size; the scale pools ((k, v) tuples, [NB, bs, H]) follow their blocks.
+    Pairs apply in order.  Updates the destination pools in place and returns them.
+    """
+    for s, d in np.asarray(pairs).reshape(-1, 2).tolist():
+        dst_k[d] = src_k[s]
+        dst_v[d] = src_v[s]
+        if src_scales is not None:
+            dst_scales[0][d] = src_scales[0][s]
+            dst_scales[1][d] = src_scales[1][s]
+    return dst_k, dst_v

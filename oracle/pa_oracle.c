@@ -209,3 +209,100 @@ int orc_paged_decode(double* out, const void* q, int q_dtype, const void* k_cach
   return orc_paged_decode_gqa(out, q, q_dtype, k_cache, v_cache, cache_dtype, k_scale, v_scale,
                               block_tables, context_lens, S, H, H, D, bs, MB, NB, scale, window);
 }
+
+/*
+ * Paged prefill / chunked-prefill attention: several new query tokens per sequence, each
+ * attending causally to the cache.  The pages motivate it (the prompt stage writes many
+ * tokens' K/V at once: "vLLM source first look: PagedAttention memory design" (trdm.cn),
+ * section 四; long single-sequence contexts such as document summarisation: "KV Cache
+ * memory optimisation and PagedAttention" (yunthe.com), section
+ * "PagedAttention在不同推理场景下的适用性") but print no formula; this is the usual causal
+ * attention, read with the same cache layout, block table, window and GQA rules as decode.
+ *
+ * Readings.  The chunk's K/V rows are already in the cache (written before attention, as
+ * for decode), so sequence s holds context_lens[s] tokens and its q_len newest ones are the
+ * queries: query i sits at position p = ctx - q_len + i and attends tokens [lo, p], with
+ * lo = max(0, p + 1 - window) for window > 0 (the last `window` tokens up to and
+ * including itself) and 0 otherwise.  q_len == 1 is exactly decode.
+ *
+ *   out          [T, Hq, D] fp64, T = cu_q[S]; row t = cu_q[s] + i
+ *   q            [T, Hq, D] in q_dtype
+ *   cu_q         [S + 1] int32, cu_q[0] = 0, non-decreasing; q_len = cu_q[s+1] - cu_q[s]
+ *   other arguments as for orc_paged_decode_gqa; q_len <= context_lens[s] is required.
+ */
+int orc_paged_prefill(double* out, const void* q, int q_dtype, const void* k_cache,
+                      const void* v_cache, int cache_dtype, const uint16_t* k_scale,
+                      const uint16_t* v_scale, const int32_t* block_tables, const int32_t* cu_q,
+                      const int32_t* context_lens, int S, int Hq, int Hkv, int D, int bs, int MB,
+                      int NB, double scale, int window) {
+  if (S < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || D <= 0 || bs <= 0 || MB <= 0 || NB <= 0)
+    return ORC_BAD_ARG;
+  if ((cache_dtype == ORC_I8 || cache_dtype == ORC_FP8) && (!k_scale || !v_scale)) return ORC_BAD_ARG;
+  if (S > 0 && cu_q[0] != 0) return ORC_BAD_ARG;
+  const int group = Hq / Hkv;
+  const int max_ctx = MB * bs;
+  double* Kc = (double*)malloc(sizeof(double) * (size_t)max_ctx * D);
+  double* Vc = (double*)malloc(sizeof(double) * (size_t)max_ctx * D);
+  double* score = (double*)malloc(sizeof(double) * (size_t)max_ctx);
+  double* qv = (double*)malloc(sizeof(double) * (size_t)D);
+  if (!Kc || !Vc || !score || !qv) {
+    free(Kc); free(Vc); free(score); free(qv);
+    return ORC_NO_MEMORY;
+  }
+  int status = ORC_OK;
+
+  for (int s = 0; s < S && status == ORC_OK; ++s) {
+    const int ctx = context_lens[s];
+    const int q_len = cu_q[s + 1] - cu_q[s];
+    if (ctx < 0 || ctx > max_ctx) { status = ORC_BAD_CONTEXT; break; }
+    if (q_len < 0 || q_len > ctx) { status = ORC_BAD_ARG; break; }
+    if (q_len == 0) continue;
+
+    for (int kh = 0; kh < Hkv && status == ORC_OK; ++kh) {
+      /* gather every cached token of this key/value head through the block table */
+      for (int i = 0; i < ctx; ++i) {
+        int32_t pb = block_tables[(size_t)s * MB + i / bs];
+        if (pb < 0 || pb >= NB) { status = ORC_BAD_TABLE; break; }
+        size_t row = ((size_t)pb * bs + i % bs) * Hkv + kh;
+        double ks = 1.0, vs = 1.0;
+        if (cache_dtype == ORC_I8 || cache_dtype == ORC_FP8) {
+          ks = orc_f16_to_f64(k_scale[row]);
+          vs = orc_f16_to_f64(v_scale[row]);
+        }
+        for (int d = 0; d < D; ++d) {
+          Kc[(size_t)i * D + d] = load_value(k_cache, cache_dtype, row * D + d) * ks;
+          Vc[(size_t)i * D + d] = load_value(v_cache, cache_dtype, row * D + d) * vs;
+        }
+      }
+      if (status != ORC_OK) break;
+
+      for (int h = kh * group; h < (kh + 1) * group; ++h) {
+        for (int i = 0; i < q_len; ++i) {
+          const size_t t = (size_t)cu_q[s] + i;
+          const int p = ctx - q_len + i;
+          const int lo = (window > 0 && p + 1 > window) ? p + 1 - window : 0;
+          const int n = p + 1 - lo;
+          double* o = out + (t * Hq + h) * D;
+          for (int d = 0; d < D; ++d) qv[d] = load_value(q, q_dtype, (t * Hq + h) * D + d);
+          for (int j = 0; j < n; ++j) {
+            double dot = 0.0;
+            for (int d = 0; d < D; ++d) dot += qv[d] * Kc[(size_t)(lo + j) * D + d];
+            score[j] = scale * dot;
+          }
+          double m = score[0];
+          for (int j = 1; j < n; ++j) if (score[j] > m) m = score[j];
+          double z = 0.0;
+          for (int j = 0; j < n; ++j) { score[j] = exp(score[j] - m); z += score[j]; }
+          for (int j = 0; j < n; ++j) score[j] /= z;
+          for (int d = 0; d < D; ++d) {
+            double acc = 0.0;
+            for (int j = 0; j < n; ++j) acc += score[j] * Vc[(size_t)(lo + j) * D + d];
+            o[d] = acc;
+          }
+        }
+      }
+    }
+  }
+  free(Kc); free(Vc); free(score); free(qv);
+  return status;
+}

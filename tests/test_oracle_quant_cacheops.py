@@ -106,6 +106,49 @@ def test_copy_blocks_duplicates_whole_blocks_and_nothing_else():
         assert np.array_equal(kc[b], k0[b]) and np.array_equal(vc[b], v0[b])
 
 
+
+def _memmove_swap(src, dst, pairs):
+    """Byte model of a block swap written with raw memmove on flat buffers."""
+    import ctypes
+    src_b, dst_b = src.view(np.uint8).reshape(-1), dst.view(np.uint8).reshape(-1)
+    blk = src[0].nbytes
+    for s, d in pairs:
+        ctypes.memmove(dst_b.ctypes.data + d * blk, src_b.ctypes.data + s * blk, blk)
+
+
+def test_swap_blocks_matches_a_memmove_model_between_pools_of_different_sizes():
+    rng = np.random.default_rng(5)
+    bs, H, D = 4, 3, 8
+    gk = rng.integers(0, 256, (9, bs, H, D), dtype=np.uint8)
+    gv = rng.integers(0, 256, (9, bs, H, D), dtype=np.uint8)
+    gks = rng.integers(0, 1 << 16, (9, bs, H), dtype=np.uint16)
+    gvs = rng.integers(0, 1 << 16, (9, bs, H), dtype=np.uint16)
+    hk, hv = np.zeros((5, bs, H, D), np.uint8), np.zeros((5, bs, H, D), np.uint8)
+    hks, hvs = np.zeros((5, bs, H), np.uint16), np.zeros((5, bs, H), np.uint16)
+    pairs = [(7, 0), (2, 4), (8, 1)]
+    want = [x.copy() for x in (hk, hv, hks, hvs)]
+    for s_, w in zip((gk, gv, gks, gvs), want):
+        _memmove_swap(s_, w, pairs)
+    cache_ops.swap_blocks(gk, gv, hk, hv, np.array(pairs), (gks, gvs), (hks, hvs))
+    for got, w in zip((hk, hv, hks, hvs), want):
+        assert np.array_equal(got, w)
+    assert not hk[2].any() and not hk[3].any()  # blocks not named by a pair stay as they were
+
+
+def test_swap_out_then_in_restores_blocks_at_their_new_ids():
+    rng = np.random.default_rng(6)
+    g = rng.standard_normal((2, 8, 2, 2, 4)).astype(np.float32)
+    gk, gv = g[0].copy(), g[1].copy()
+    hk, hv = np.full((4, 2, 2, 4), np.nan, np.float32), np.full((4, 2, 2, 4), np.nan, np.float32)
+    out_pairs = np.array([[1, 3], [6, 0]])
+    cache_ops.swap_blocks(gk, gv, hk, hv, out_pairs)
+    gk[[1, 6]] = 0  # the GPU blocks are reused by someone else meanwhile
+    back = np.array([[3, 5], [0, 2]])  # swap-in lands in other free GPU blocks
+    cache_ops.swap_blocks(hk, hv, gk, gv, back)
+    assert np.array_equal(gk[5], g[0][1]) and np.array_equal(gk[2], g[0][6])
+    assert np.array_equal(gv[5], g[1][1]) and np.array_equal(gv[2], g[1][6])
+
+
 # ---------------------------------------------------------------------------------------
 # FP8 (E4M3) quantiser
 # ---------------------------------------------------------------------------------------
