@@ -208,18 +208,18 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
           tma_load_2d(sb + 4 * kHalf + kQHalf, &tmQ, bar, 64, qrow, policy);
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ok = __shfl_sync(0xffffffffu, ok, 0);  // also orders lane 0's expect_tx before any copy
       if (!ok) break;
-      for (int i = 0; i < nload; ++i) {
-        const int b = __shfl_sync(0xffffffffu, pb, i);
-        if (lane == 0) {
-          const uint32_t bar = full0 + 8 * st;
-          const uint32_t row = static_cast<uint32_t>(lb_lo + i - lb_first) * bs * 128u;
-          const uint32_t sb = stage(st);
-          tma_load_3d(sb + row, &tmK, bar, 0, c.g, b * bs, policy);
-          tma_load_3d(sb + kHalf + row, &tmK, bar, 64, c.g, b * bs, policy);
-          tma_load_3d(sb + 2 * kHalf + row, &tmV, bar, 0, c.g, b * bs, policy);
-          tma_load_3d(sb + 3 * kHalf + row, &tmV, bar, 64, c.g, b * bs, policy);
+      // The tile's copies (4 per block: K and V, two 64-dim halves each) are issued by the
+      // warp's lanes together, one copy per lane, rather than one after another.
+      for (int base_copy = 0; base_copy < 4 * nload; base_copy += 32) {
+        const int cp = base_copy + lane;
+        const int b = __shfl_sync(0xffffffffu, pb, (cp >> 2) & 31);
+        if (cp < 4 * nload) {
+          const int part = cp & 3;  // 0: K lo, 1: K hi, 2: V lo, 3: V hi
+          const uint32_t row = static_cast<uint32_t>(lb_lo + (cp >> 2) - lb_first) * bs * 128u;
+          tma_load_3d(stage(st) + part * kHalf + row, part < 2 ? &tmK : &tmV, full0 + 8 * st, (part & 1) * 64, c.g,
+                      b * bs, policy);
         }
       }
       advance(c, p);
