@@ -438,6 +438,216 @@ def run_ours(args):
     return 0
 
 
+def run_swap(args):
+    """Preemption swap of the Llama-2-70B layer batch: the blocks of the last 8 of the 32
+    sequences move to a page-locked host pool (swap-out) and back (swap-in), one
+    swap_blocks launch per direction.  The host-link ceiling is measured live: one copy
+    of the same bytes per direction between contiguous pinned and device buffers."""
+    import paged_kv_cache_384_b200 as pa
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(device)
+    w = synth.build_workload(PRESET, args.seed, pa.BlockManager)
+    gk, gv = w.k_cache.to(device), w.v_cache.to(device)
+    ctx = w.context_lens.tolist()
+    victims = range(w.num_seqs - 8, w.num_seqs)
+    blocks = [int(w.block_tables[s, j]) for s in victims for j in range(-(-ctx[s] // w.block_size))]
+    n = len(blocks)
+    hk = torch.empty((n,) + tuple(gk.shape[1:]), dtype=gk.dtype).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    out_pairs = torch.tensor([[b, i] for i, b in enumerate(blocks)], dtype=torch.int64)
+    in_pairs = out_pairs.flip(1).contiguous()
+    d_out, d_in = out_pairs.to(device), in_pairs.to(device)
+    block_bytes = gk[0].numel() * gk.element_size()
+    bytes_step = 2 * 2 * n * block_bytes                    # K and V, out and back in
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        pa.swap_blocks(gk, gv, hk, hv, d_out, stream=stream)
+        pa.swap_blocks(hk, hv, gk, gv, d_in, stream=stream)
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1) / 1e3 / reps
+
+    # host-link ceiling: contiguous copies of the same bytes, one per direction
+    flat_d = torch.empty(n * block_bytes * 2, dtype=torch.uint8, device=device)
+    flat_h = torch.empty(n * block_bytes * 2, dtype=torch.uint8).pin_memory()
+
+    def link():
+        flat_h.copy_(flat_d, non_blocking=True)
+        flat_d.copy_(flat_h, non_blocking=True)
+    link_gbs = bytes_step / timed(link, 5) / 1e9
+
+    # the per-block alternative: one copy-engine transfer per block and pool
+    def per_block():
+        for s_, t_ in out_pairs.tolist():
+            hk[t_].copy_(gk[s_], non_blocking=True)
+            hv[t_].copy_(gv[s_], non_blocking=True)
+        for s_, t_ in in_pairs.tolist():
+            gk[t_].copy_(hk[s_], non_blocking=True)
+            gv[t_].copy_(hv[s_], non_blocking=True)
+    per_block_gbs = bytes_step / timed(per_block, 2) / 1e9
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    props = torch.cuda.get_device_properties(device)
+    smi_id = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+    with ClockSampler(smi_id) as clocks:
+        clocks.mark()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+    sec = e0.elapsed_time(e1) / 1e3
+    value = bytes_step * args.steps / sec / 1e9
+
+    # end to end: pairs handed over in pinned host memory each step (read by the kernel)
+    h_out, h_in = out_pairs.pin_memory(), in_pairs.pin_memory()
+
+    def e2e_step():
+        pa.swap_blocks(gk, gv, hk, hv, h_out, stream=stream)
+        pa.swap_blocks(hk, hv, gk, gv, h_in, stream=stream)
+    e2e_sec = timed(e2e_step, args.steps)
+    ok = torch.equal(gk[blocks[0]], hk[0].to(device)) and pa.device_error(clear=True) == 0
+    line = {
+        "metric": "KV block swap GB/s (GPU <-> page-locked host pool, out + in)", "value": round(value, 2),
+        "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * sec / args.steps, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": "swap_llama70b_fp16", "preempted_seqs": 8, "blocks_swapped": n,
+                   "block_bytes": block_bytes, "bytes_per_step": bytes_step, "seed": args.seed,
+                   "l2": "inputs larger than L2, no flush"},
+        "roofline": {"bound": "host_link", "achieved": round(value, 2), "peak": round(link_gbs, 2), "unit": "GB/s",
+                     "frac": round(value / link_gbs, 4), "traffic": None,
+                     "peak_source": "measured live: one contiguous pinned copy per direction, same bytes"},
+        "per_block_copy_engine_gbs": round(per_block_gbs, 2),
+        "cpu_baseline": None,
+        "e2e": {"value": round(bytes_step / e2e_sec / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": bytes_step // 2 + 2 * out_pairs.numel() * 8,
+                "d2h_bytes_per_step": bytes_step // 2},
+        "gpu_launches": 2 * args.steps, "clocks": clocks.summary(), "verified": bool(ok),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+PREFILL = {  # name: (prompts, prompt/chunk tokens, cached tokens before the chunk, q heads, kv heads)
+    "prefill_llama70b_fp16": (4, 2048, 0, 64, 64),
+    "prefill_llama70b_gqa_fp16": (4, 2048, 0, 64, 8),
+    "chunked_prefill_llama70b_fp16": (8, 512, 1536, 64, 64),
+}
+
+
+def run_prefill(args):
+    """Prompt processing of one Llama-2-70B attention layer: each sequence's new tokens
+    are written into the paged cache (reshape_and_cache) and attend causally to it
+    (paged_attention_prefill).  The prompt batch holds 8192 tokens (the engine's
+    max_num_batched_tokens on the deployment page).  Metric: attention FLOP/s, where a
+    query row that attends n tokens costs 4 * n * head_dim FLOPs (QK^T and PV)."""
+    import paged_kv_cache_384_b200 as pa
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(device)
+    S, qn, cached, Hq, Hkv = PREFILL[args.workload]
+    D, bs = 128, args.block_size or 16
+    ctx = qn + cached
+    nblk = -(-ctx // bs)
+    g = torch.Generator(device=device).manual_seed(args.seed)
+    NB = int(math.ceil(1.1 * S * nblk))
+    perm = torch.randperm(NB, generator=g, device=device)
+    bt = perm[: S * nblk].view(S, nblk).to(torch.int32).contiguous()
+    kc = torch.randn(NB, bs, Hkv, D, generator=g, device=device, dtype=torch.float16)
+    vc = torch.randn(NB, bs, Hkv, D, generator=g, device=device, dtype=torch.float16)
+    T = S * qn
+    q = torch.randn(T, Hq, D, generator=g, device=device, dtype=torch.float16)
+    k_new = torch.randn(T, Hkv, D, generator=g, device=device, dtype=torch.float16)
+    v_new = torch.randn(T, Hkv, D, generator=g, device=device, dtype=torch.float16)
+    pos = torch.arange(cached, ctx, device=device).repeat(S)
+    seq = torch.arange(S, device=device).repeat_interleave(qn)
+    slots = (bt[seq, pos // bs].long() * bs + pos % bs).contiguous()
+    cu = torch.arange(0, T + 1, qn, dtype=torch.int32, device=device)
+    cl = torch.full((S,), ctx, dtype=torch.int32, device=device)
+    out = torch.empty_like(q)
+    scale = 1 / math.sqrt(D)
+    stream = torch.cuda.current_stream(device)
+    attended = sum(p + 1 for p in range(cached, ctx))  # causal, no window: position p sees p + 1 tokens
+    flops = 4.0 * D * Hq * S * attended
+
+    def attn():
+        pa.paged_attention_prefill(out, q, kc, vc, bt, cu, cl, qn, scale, stream=stream)
+
+    def step():
+        pa.reshape_and_cache(k_new, v_new, kc, vc, slots, stream=stream)
+        attn()
+
+    def timed(fn, reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1) / 1e3 / reps
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    props = torch.cuda.get_device_properties(device)
+    smi_id = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+    with ClockSampler(smi_id) as clocks:
+        clocks.mark()
+        sec = timed(step, args.steps)
+        attn_sec = timed(attn, args.steps)
+    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    peak = float(peaks["bf16_tflops"])  # fp16 and bf16 run at the same tensor rate
+    # end to end: q and the new K/V rows from pinned host memory, the output read back
+    hq, hk, hv = q.cpu().pin_memory(), k_new.cpu().pin_memory(), v_new.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k_new.copy_(hk, non_blocking=True)
+        v_new.copy_(hv, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+    e2e_step()
+    torch.cuda.synchronize(device)
+    e2e_sec = timed(e2e_step, max(3, args.steps // 4))
+    nbytes = lambda t: t.numel() * t.element_size()
+    errs = pa.device_error(clear=True)
+    line = {
+        "metric": "paged prefill attention TFLOP/s (causal, 4*n*head_dim FLOPs per query row)",
+        "value": round(flops / sec / 1e12, 2), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * sec, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": args.workload, "prompts": S, "new_tokens_per_seq": qn, "cached_before": cached,
+                   "num_q_heads": Hq, "num_kv_heads": Hkv, "head_dim": D, "block_size": bs, "seed": args.seed,
+                   "step": "reshape_and_cache of the new K/V rows + paged_attention_prefill",
+                   "l2": "K/V and q per step larger than L2, no flush"},
+        "tokens_per_s": round(T / sec, 1),
+        "roofline": {"bound": "tensor", "achieved": round(flops / attn_sec / 1e12, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(flops / attn_sec / 1e12 / peak, 4), "traffic": None,
+                     "peak_source": "measured (cuBLAS bf16 burst)", "kernel": "prefill_tc_kernel",
+                     "kernel_ms": round(1e3 * attn_sec, 4)},
+        "cpu_baseline": None,
+        "e2e": {"value": round(flops / e2e_sec / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": nbytes(q) + nbytes(k_new) + nbytes(v_new), "d2h_bytes_per_step": nbytes(out)},
+        "gpu_launches": 2 * args.steps, "clocks": clocks.summary(), "device_errors": errs,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -447,13 +657,17 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=PRESET, choices=["llama70b_fp16", "chat_prefix_bf16", "sliding_window_fp16",
-                                                           "llama70b_gqa_fp16"],
+                                                           "llama70b_gqa_fp16", "swap_llama70b_fp16", *PREFILL],
                     help="secondary workloads are for study; the metric is quoted on the default")
     ap.add_argument("--block-size", type=int, default=None)
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)  # timing rule: at least 3 untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "swap_llama70b_fp16":
+        return run_swap(args)
+    if args.workload in PREFILL:
+        return run_prefill(args)
     return run_ours(args)
 
 

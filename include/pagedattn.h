@@ -19,7 +19,8 @@
  *
  * Conventions for every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller (cudaMalloc or any
- *     allocator); the library never allocates, frees or keeps them.  Tensors are dense,
+ *     allocator; swap_blocks also takes mapped page-locked host memory); the library
+ *     never allocates, frees or keeps them.  Tensors are dense,
  *     row-major, and their base addresses must be 16-byte aligned.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is enqueued
  *     asynchronously; the call returns once it is launched.
@@ -62,7 +63,7 @@ typedef enum pa_status {
 #define PA_DEVERR_TABLE 0x1u   /* block-table entry outside [0, num_blocks): block 0 read instead */
 #define PA_DEVERR_CONTEXT 0x2u /* context_len < 0 or > max_blocks_per_seq*block_size: clamped */
 #define PA_DEVERR_SLOT 0x4u    /* reshape_and_cache slot >= num_blocks*block_size: token skipped */
-#define PA_DEVERR_PAIR 0x8u    /* copy_blocks pair index outside [0, num_blocks): pair skipped */
+#define PA_DEVERR_PAIR 0x8u    /* copy_blocks / swap_blocks pair outside its pool: pair skipped */
 #define PA_DEVERR_TIMEOUT 0x10u /* a bounded pipeline wait gave up (a library bug; results invalid) */
 
 /* Message for the last non-PA_OK status returned on the calling thread ("" if none). */
@@ -223,6 +224,41 @@ pa_status reshape_and_cache(const void* k, const void* v, void* k_cache, void* v
                             void* stream);
 
 /*
+ * Paged prefill / chunked-prefill attention: several new query tokens per sequence, each
+ * attending causally to the paged cache.  The pages motivate it (page C, section 四: the
+ * prompt stage writes many tokens' K/V at once; page A, section
+ * "PagedAttention在不同推理场景下的适用性": long single-sequence contexts) but give no
+ * formula; this is the usual causal attention with the cache layout, block-table walk and
+ * window rule of paged_attention_decode:
+ *   the chunk's own K/V rows are already in the cache (reshape_and_cache first), so
+ *   sequence s holds context_lens[s] tokens and its q_len newest are the queries; query i
+ *   sits at position p = ctx - q_len + i and attends tokens [lo, p], lo = max(0, p + 1 -
+ *   window) for window > 0, else 0.  q_len == 1 is decode.
+ *
+ *   out, q         [num_q_tokens, num_q_heads, 128] in dtype (PA_F16 or PA_BF16); the rows of
+ *                  sequence s are cu_q_lens[s] .. cu_q_lens[s+1]-1
+ *   k_cache,       [num_blocks, block_size, num_kv_heads, 128] in dtype
+ *   v_cache
+ *   block_tables   [num_seqs, max_blocks_per_seq] int32
+ *   cu_q_lens      [num_seqs + 1] int32 device array, cu_q_lens[0] = 0, non-decreasing
+ *   context_lens   [num_seqs] int32 device array, q_len <= context_len <= max_blocks_per_seq*block_size
+ *   max_q_len      an upper bound of every q_len (sizes the grid; a larger q_len is an error)
+ *   num_q_heads    a multiple of num_kv_heads with 1, 2, 4, 8 or 16 query heads per cached head
+ *   block_size     8, 16, 32, 64 or 128
+ * Tensor cores (tcgen05), fp32 accumulation; bf16 probabilities keep ~16 bits (hi + lo
+ * parts).  A sequence whose q_len exceeds max_q_len or its context, whose rows run
+ * past num_q_tokens, or whose context exceeds the table, is skipped and sets
+ * PA_DEVERR_CONTEXT; a table entry outside
+ * [0, num_blocks) reads block 0 and sets PA_DEVERR_TABLE.  Needs no workspace.
+ */
+pa_status paged_attention_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                  const int32_t* block_tables, const int32_t* cu_q_lens,
+                                  const int32_t* context_lens, int num_seqs, int num_q_tokens,
+                                  int max_q_len, int num_q_heads, int num_kv_heads, int head_dim,
+                                  int block_size, int num_blocks, int max_blocks_per_seq,
+                                  float scale, int window, pa_dtype dtype, void* stream);
+
+/*
  * Copy whole physical blocks for copy-on-write.  Source: page C, section 二,
  * BlockManager.copy_on_write (the new block receives a copy of the old block's KV
  * data) and section 四 (the copy is a latency cost of forking).
@@ -265,6 +301,37 @@ pa_status reshape_and_cache_quant(const void* k, const void* v, pa_dtype src_dty
                                   pa_dtype cache_dtype, const int64_t* slot_mapping, int num_tokens,
                                   int num_heads, int head_dim, int block_size, int num_blocks,
                                   int64_t k_token_stride, int64_t v_token_stride, void* stream);
+
+/*
+ * Swap whole blocks between two pools that live in different address spaces: the GPU
+ * pool and a page-locked host pool ("swap space").  Source: page A, section
+ * "vLLM调度器与PagedAttention协同工作", item 3 (preemption: under memory pressure a
+ * low-priority request's KV blocks move out to CPU memory, freeing GPU blocks, and move
+ * back when room returns) and section "vLLM部署配置与PagedAttention参数调优" (swap_space,
+ * the size of the CPU pool in GB).  Swap-out is (GPU pool -> host pool), swap-in the
+ * reverse; one call moves every listed block in ONE kernel launch whose threads read and
+ * write the host pool directly over the host link (no staging copy, no per-block call).
+ *
+ *   src_k, src_v          source pools, num_src_blocks blocks of block_bytes bytes each
+ *   dst_k, dst_v          destination pools, num_dst_blocks blocks of block_bytes bytes
+ *   src_dst_pairs         [num_pairs, 2] int64 of (source block id, destination block id)
+ *   src_k_scale, ...      optional (all four or none) scale pools, scale_block_bytes per
+ *                         block (8-bit caches: block_size*num_heads*2)
+ * Every pool and the pair array may each be device memory (any allocator) or page-locked
+ * host memory mapped into the device's address space (cudaHostAlloc, or cudaHostRegister
+ * with the mapped flag; torch's pin_memory qualifies).  Pageable host memory is rejected
+ * with PA_ERR_INVALID_ARG.  Pools passed as host pointers are translated to their device
+ * addresses by the library.  Destinations must be distinct and, when source and
+ * destination are the same pool, no destination may also be a source.  A pair outside
+ * either pool is skipped and sets PA_DEVERR_PAIR.  Bit-exact copy.  The copy is ordered
+ * on `stream` like a kernel: host code must synchronise the stream before it reads a
+ * host destination or reuses a host source.
+ */
+pa_status swap_blocks(const void* src_k, const void* src_v, void* dst_k, void* dst_v,
+                      const int64_t* src_dst_pairs, int num_pairs, int num_src_blocks,
+                      int num_dst_blocks, size_t block_bytes, const void* src_k_scale,
+                      const void* src_v_scale, void* dst_k_scale, void* dst_v_scale,
+                      size_t scale_block_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------ */
 /* Host-side block manager (free list + reference counts)                               */

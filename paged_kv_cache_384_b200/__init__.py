@@ -129,6 +129,35 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
 # ---------------------------------------------------------------------------------------
 # Cache maintenance
 # ---------------------------------------------------------------------------------------
+def paged_attention_prefill(out, q, k_cache, v_cache, block_tables, cu_q_lens, context_lens, max_q_len: int,
+                            scale: float, window: int = 0, stream=None):
+    """Causal attention of each sequence's newest q_len tokens over the paged cache.
+
+    q/out [T, Hq, 128] (fp16 or bf16) pack the sequences' query rows (sequence s owns rows
+    cu_q_lens[s]..cu_q_lens[s+1]-1, int32 [S+1] on the GPU); the chunk's K/V must already
+    be in the cache, so query i of sequence s is at position context_lens[s] - q_len + i.
+    ``max_q_len`` bounds every q_len (host-known, sizes the grid).
+    """
+    if q.dim() != 3 or out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("q and out must be [T, Hq, D] of one dtype")
+    if k_cache.dim() != 4 or v_cache.shape != k_cache.shape or k_cache.dtype != q.dtype:
+        raise ValueError("caches must be [NB, bs, Hkv, D] in q's dtype")
+    if cu_q_lens.dtype != torch.int32 or context_lens.dtype != torch.int32 or block_tables.dtype != torch.int32:
+        raise ValueError("cu_q_lens, context_lens and block_tables must be int32")
+    for name, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
+                    ("block_tables", block_tables), ("cu_q_lens", cu_q_lens), ("context_lens", context_lens)):
+        _dense(name, t)
+    T, Hq, D = q.shape
+    NB, bs, Hkv, _ = k_cache.shape
+    S = context_lens.shape[0]
+    if cu_q_lens.shape[0] != S + 1:
+        raise ValueError("cu_q_lens must have num_seqs + 1 entries")
+    _check(_L.paged_attention_prefill(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                      _ptr(cu_q_lens), _ptr(context_lens), S, T, int(max_q_len), Hq, Hkv, D, bs,
+                                      NB, block_tables.shape[1], float(scale), int(window), _DTYPE[q.dtype],
+                                      _stream(stream)))
+
+
 def reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, k_scale=None, v_scale=None,
                       k_scale_cache=None, v_scale_cache=None, stream=None):
     """Write token t's rows k[t], v[t] ([T,H,D], token stride may exceed H*D) into slot
@@ -196,6 +225,42 @@ def copy_blocks(k_cache, v_cache, src_dst_pairs, k_scale_cache=None, v_scale_cac
     sbytes = 0 if k_scale_cache is None else k_scale_cache[0].numel() * k_scale_cache.element_size()
     _check(_L.copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(src_dst_pairs), src_dst_pairs.shape[0], NB,
                           block_bytes, _ptr(k_scale_cache), _ptr(v_scale_cache), sbytes, _stream(stream)))
+
+
+def swap_blocks(src_k, src_v, dst_k, dst_v, src_dst_pairs, src_scales=None, dst_scales=None, stream=None):
+    """dst_k[d] = src_k[s] (and v, and the scale pools) for each (s, d) pair, across pools.
+
+    One pool side is normally the GPU cache and the other a page-locked host pool
+    (``torch.empty(..., pin_memory=True)``): swap-out is GPU -> host, swap-in host -> GPU.
+    ``src_dst_pairs`` (int64 [N, 2]) may sit on the GPU or in pinned host memory.  The
+    scale pools are given as (k_scale, v_scale) tuples, both sides or neither.  Ordered
+    on ``stream``: synchronise it before reading a host destination.
+    """
+    if src_k.shape[1:] != dst_k.shape[1:] or src_k.dtype != dst_k.dtype:
+        raise ValueError("source and destination pools must have the same block shape and dtype")
+    for a, b in ((src_k, src_v), (dst_k, dst_v)):
+        if a.shape != b.shape or a.dtype != b.dtype:
+            raise ValueError("K and V pools must match")
+    if src_dst_pairs.dtype != torch.int64 or src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2:
+        raise ValueError("src_dst_pairs must be int64 [N, 2]")
+    if (src_scales is None) != (dst_scales is None):
+        raise ValueError("pass scale pools for both sides or neither")
+    for name, t in (("src_k", src_k), ("src_v", src_v), ("dst_k", dst_k), ("dst_v", dst_v),
+                    ("src_dst_pairs", src_dst_pairs)) + tuple(
+                        (f"scale pool {i}", t) for i, t in enumerate((src_scales or ()) + (dst_scales or ()))):
+        if not (t.is_cuda or t.is_pinned()):
+            raise ValueError(f"{name} must be a CUDA tensor or page-locked host memory (pin_memory=True)")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    block_bytes = src_k[0].numel() * src_k.element_size()
+    sk = sv = dk = dv = None
+    sbytes = 0
+    if src_scales is not None:
+        (sk, sv), (dk, dv) = src_scales, dst_scales
+        sbytes = sk[0].numel() * sk.element_size()
+    _check(_L.swap_blocks(_ptr(src_k), _ptr(src_v), _ptr(dst_k), _ptr(dst_v), _ptr(src_dst_pairs),
+                          src_dst_pairs.shape[0], src_k.shape[0], dst_k.shape[0], block_bytes,
+                          _ptr(sk), _ptr(sv), _ptr(dk), _ptr(dv), sbytes, _stream(stream)))
 
 
 # ---------------------------------------------------------------------------------------

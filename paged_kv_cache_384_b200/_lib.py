@@ -31,6 +31,9 @@ SIGNATURES = {
     "paged_attention_decode_static_scratch": (c_int, [
         c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
         c_int, c_int, c_int, c_int, c_int, c_int, c_float, c_int, c_int, c_int, c_void_p]),
+    "paged_attention_prefill": (c_int, [
+        c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int,
+        c_int, c_int, c_int, c_int, c_int, c_float, c_int, c_int, c_void_p]),
     "reshape_and_cache": (c_int, [
         c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
         c_int64, c_int64, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
@@ -39,6 +42,9 @@ SIGNATURES = {
         c_int, c_int, c_int, c_int64, c_int64, c_void_p]),
     "copy_blocks": (c_int, [
         c_void_p, c_void_p, c_void_p, c_int, c_int, c_size_t, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "swap_blocks": (c_int, [
+        c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_size_t,
+        c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "pa_bm_create": (c_void_p, [c_int, c_int, c_void_p]),
     "pa_bm_destroy": (None, [c_void_p]),
     "pa_bm_allocate": (c_int, [c_void_p, c_int, c_void_p]),

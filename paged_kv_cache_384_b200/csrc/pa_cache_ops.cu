@@ -1,4 +1,4 @@
-// pa_cache_ops.cu -- reshape_and_cache and copy_blocks for sm_100a.
+// pa_cache_ops.cu -- reshape_and_cache, copy_blocks and swap_blocks for sm_100a.
 //
 // Both are pure data movement and HBM-bound.  Each thread moves 16-byte vectors; a CTA
 // covers a contiguous byte range so every warp issues fully coalesced 512-byte
@@ -50,26 +50,36 @@ reshape_and_cache_kernel(const uint8_t* __restrict__ k, const uint8_t* __restric
 }
 
 // ---------------------------------------------------------------------------------------
-// copy_blocks: pool block dst <- pool block src for each (src, dst) pair ("vLLM source first
-// look: PagedAttention memory design" (trdm.cn), section 二, BlockManager.copy_on_write).
+// Whole-block copies, dst pool block d <- src pool block s for each (s, d) pair.
+//  * copy_blocks: source and destination are the same GPU pool ("vLLM source first look:
+//    PagedAttention memory design" (trdm.cn), section 二, BlockManager.copy_on_write).
+//  * swap_blocks: one pool is page-locked host memory mapped into the device address
+//    space ("KV Cache memory optimisation and PagedAttention" (yunthe.com), section
+//    "vLLM调度器与PagedAttention协同工作", item 3: preempted requests' blocks move to CPU
+//    memory and back).  The threads read or write the host pool directly; the many
+//    16-byte requests in flight across the grid keep the host link busy.
 // Grid: (chunks of a block, pairs, 2 or 4 pools).  VEC = 16 moves uint4; VEC = 1 moves bytes.
 // ---------------------------------------------------------------------------------------
+struct BlockPools {
+  const uint8_t* src[4];  // K, V, K scales, V scales
+  uint8_t* dst[4];
+};
+
 template <int VEC>
 __global__ void __launch_bounds__(256)
-copy_blocks_kernel(uint8_t* k, uint8_t* v, uint8_t* ks, uint8_t* vs, const int64_t* __restrict__ pairs,
-                   long long block_bytes, long long scale_block_bytes, long long num_blocks) {
+block_copy_kernel(BlockPools pools, const int64_t* pairs, long long block_bytes, long long scale_block_bytes,
+                  long long num_src, long long num_dst) {
   grid_dependency_launch_next();
   grid_dependency_wait();
-  const int pool = blockIdx.z;  // 0: K, 1: V, 2: K scales, 3: V scales
-  const long long src = __ldg(pairs + 2 * blockIdx.y), dst = __ldg(pairs + 2 * blockIdx.y + 1);
-  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+  const int pool = blockIdx.z;
+  const long long src = pairs[2 * blockIdx.y], dst = pairs[2 * blockIdx.y + 1];
+  if (src < 0 || src >= num_src || dst < 0 || dst >= num_dst) {
     if (threadIdx.x == 0 && blockIdx.x == 0 && pool == 0) cache_error(PA_DEVERR_PAIR);
     return;
   }
-  uint8_t* base = pool == 0 ? k : pool == 1 ? v : pool == 2 ? ks : vs;
   const long long bytes = pool < 2 ? block_bytes : scale_block_bytes;
-  const uint8_t* from = base + src * bytes;
-  uint8_t* to = base + dst * bytes;
+  const uint8_t* from = pools.src[pool] + src * bytes;
+  uint8_t* to = pools.dst[pool] + dst * bytes;
   if (VEC == 16 && pool < 2) {
     constexpr int kPerThread = 4;  // 4 independent 16-byte loads in flight per thread
     const long long nvec = bytes / 16;
@@ -111,6 +121,50 @@ struct RegisterCache {
 } g_register_cache;
 
 size_t elem_size(pa_dtype t) { return t == PA_F32 ? 4 : ((t == PA_I8 || t == PA_FP8_E4M3) ? 1 : 2); }
+
+}  // namespace
+}  // namespace pa
+
+namespace pa {
+namespace {
+
+cudaError_t launch_block_copy(const BlockPools& pools, const int64_t* pairs, int num_pairs, size_t block_bytes,
+                              size_t scale_block_bytes, long long num_src, long long num_dst, bool scales,
+                              cudaStream_t s) {
+  const bool vec_ok = block_bytes % 16 == 0 && aligned16(pools.src[0]) && aligned16(pools.src[1]) &&
+                      aligned16(pools.dst[0]) && aligned16(pools.dst[1]);
+  const int threads = 256;
+  const long long per_cta = vec_ok ? 16LL * threads * 4 : threads * 64LL;
+  const long long longest = static_cast<long long>(block_bytes > scale_block_bytes ? block_bytes : scale_block_bytes);
+  dim3 grid(static_cast<unsigned>((longest + per_cta - 1) / per_cta), static_cast<unsigned>(num_pairs), scales ? 4u : 2u);
+  BlockPools p = pools;
+  long long bb = static_cast<long long>(block_bytes), sb = static_cast<long long>(scale_block_bytes);
+  void* args[] = {&p, &pairs, &bb, &sb, &num_src, &num_dst};
+  const void* fn = vec_ok ? reinterpret_cast<const void*>(&block_copy_kernel<16>)
+                          : reinterpret_cast<const void*>(&block_copy_kernel<1>);
+  return launch_dependent(fn, grid, dim3(threads), 0, s, args);
+}
+
+// The address under which the device reaches `p`: device memory as it is, page-locked host
+// memory through its mapping.  Pageable host memory has no such address.
+pa_status device_view(const void* p, const char* what, const void** out) {
+  cudaPointerAttributes a;
+  const cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return cuda_fail(e, what);
+  }
+  if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) {
+    *out = p;
+    return PA_OK;
+  }
+  if (a.type == cudaMemoryTypeHost && a.devicePointer) {
+    *out = a.devicePointer;
+    return PA_OK;
+  }
+  return fail(PA_ERR_INVALID_ARG, "swap_blocks: %s is pageable (or unmapped) host memory; use page-locked, mapped memory",
+              what);
+}
 
 }  // namespace
 }  // namespace pa
@@ -183,23 +237,47 @@ extern "C" pa_status copy_blocks(void* k_cache, void* v_cache, const int64_t* sr
   if (reinterpret_cast<uintptr_t>(src_dst_pairs) % 8) return fail(PA_ERR_INVALID_ARG, "copy_blocks: pairs must be 8-byte aligned");
   if (num_pairs > 65535) return fail(PA_ERR_UNSUPPORTED, "copy_blocks: at most 65535 pairs per call");
 
-  const bool vec_ok = block_bytes % 16 == 0 && aligned16(k_cache) && aligned16(v_cache);
-  const int threads = 256;
-  const long long per_cta = vec_ok ? 16LL * threads * 4 : threads * 64LL;
-  const long long longest = static_cast<long long>(block_bytes > scale_block_bytes ? block_bytes : scale_block_bytes);
-  dim3 grid(static_cast<unsigned>((longest + per_cta - 1) / per_cta), static_cast<unsigned>(num_pairs), scales ? 4u : 2u);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* kp = static_cast<uint8_t*>(k_cache);
-  uint8_t* vp = static_cast<uint8_t*>(v_cache);
-  uint8_t* ksp = static_cast<uint8_t*>(k_scale_cache);
-  uint8_t* vsp = static_cast<uint8_t*>(v_scale_cache);
-  long long bb = static_cast<long long>(block_bytes), sb = static_cast<long long>(scale_block_bytes);
-  long long nb = num_blocks;
-  void* args[] = {&kp, &vp, &ksp, &vsp, &src_dst_pairs, &bb, &sb, &nb};
-  const void* fn = vec_ok ? reinterpret_cast<const void*>(&copy_blocks_kernel<16>)
-                          : reinterpret_cast<const void*>(&copy_blocks_kernel<1>);
-  cudaError_t err = launch_dependent(fn, grid, dim3(threads), 0, s, args);
+  BlockPools pools{{static_cast<const uint8_t*>(k_cache), static_cast<const uint8_t*>(v_cache),
+                    static_cast<const uint8_t*>(k_scale_cache), static_cast<const uint8_t*>(v_scale_cache)},
+                   {static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache),
+                    static_cast<uint8_t*>(k_scale_cache), static_cast<uint8_t*>(v_scale_cache)}};
+  cudaError_t err = launch_block_copy(pools, src_dst_pairs, num_pairs, block_bytes, scale_block_bytes, num_blocks,
+                                      num_blocks, scales, static_cast<cudaStream_t>(stream));
   if (err != cudaSuccess) return cuda_fail(err, "launching copy_blocks");
+  return PA_OK;
+}
+
+extern "C" pa_status swap_blocks(const void* src_k, const void* src_v, void* dst_k, void* dst_v,
+                                 const int64_t* src_dst_pairs, int num_pairs, int num_src_blocks, int num_dst_blocks,
+                                 size_t block_bytes, const void* src_k_scale, const void* src_v_scale,
+                                 void* dst_k_scale, void* dst_v_scale, size_t scale_block_bytes, void* stream) {
+  if (num_pairs < 0 || num_src_blocks <= 0 || num_dst_blocks <= 0 || block_bytes == 0)
+    return fail(PA_ERR_INVALID_ARG, "swap_blocks: num_pairs >= 0, pool sizes > 0 and block_bytes > 0 required");
+  const int nscale = !!src_k_scale + !!src_v_scale + !!dst_k_scale + !!dst_v_scale;
+  if (nscale != 0 && (nscale != 4 || scale_block_bytes == 0))
+    return fail(PA_ERR_INVALID_ARG, "swap_blocks: pass all four scale pools with scale_block_bytes > 0, or none");
+  if (num_pairs == 0) return PA_OK;
+  if (!src_k || !src_v || !dst_k || !dst_v || !src_dst_pairs) return fail(PA_ERR_INVALID_ARG, "swap_blocks: NULL pointer");
+  if (reinterpret_cast<uintptr_t>(src_dst_pairs) % 8) return fail(PA_ERR_INVALID_ARG, "swap_blocks: pairs must be 8-byte aligned");
+  if (num_pairs > 65535) return fail(PA_ERR_UNSUPPORTED, "swap_blocks: at most 65535 pairs per call");
+
+  const void* in[9] = {src_k, src_v, src_k_scale, src_v_scale, dst_k, dst_v, dst_k_scale, dst_v_scale, src_dst_pairs};
+  static const char* const names[9] = {"src_k", "src_v", "src_k_scale", "src_v_scale", "dst_k",
+                                       "dst_v", "dst_k_scale", "dst_v_scale", "src_dst_pairs"};
+  const void* dev[9] = {};
+  for (int i = 0; i < 9; ++i) {
+    if (!in[i]) continue;
+    const pa_status st = device_view(in[i], names[i], &dev[i]);
+    if (st != PA_OK) return st;
+  }
+  BlockPools pools{{static_cast<const uint8_t*>(dev[0]), static_cast<const uint8_t*>(dev[1]),
+                    static_cast<const uint8_t*>(dev[2]), static_cast<const uint8_t*>(dev[3])},
+                   {static_cast<uint8_t*>(const_cast<void*>(dev[4])), static_cast<uint8_t*>(const_cast<void*>(dev[5])),
+                    static_cast<uint8_t*>(const_cast<void*>(dev[6])), static_cast<uint8_t*>(const_cast<void*>(dev[7]))}};
+  cudaError_t err = launch_block_copy(pools, static_cast<const int64_t*>(dev[8]), num_pairs, block_bytes,
+                                      scale_block_bytes, num_src_blocks, num_dst_blocks, nscale != 0,
+                                      static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "launching swap_blocks");
   return PA_OK;
 }
 

@@ -31,6 +31,7 @@
 #include "pa_decode_shared.cuh"
 #include "pa_device.cuh"
 #include "pa_host.h"
+#include "pa_tmap.h"
 
 namespace pa {
 
@@ -357,34 +358,6 @@ cudaError_t read_decode_error(uint32_t* flags, int clear) {
 struct RegisterDecode {
   RegisterDecode() { register_device_error_reader(read_decode_error); }
 } g_register_decode;
-
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-pa_status get_encoder(EncodeTiledFn* out) {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q);
-    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !ptr)
-      return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-    fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  *out = fn;
-  return PA_OK;
-}
-
-pa_status encode(EncodeTiledFn fn, CUtensorMap* map, CUtensorMapDataType type, int rank, const void* base,
-                 const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
-                 CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE) {
-  const cuuint32_t estride[3] = {1, 1, 1};
-  CUresult r = fn(map, type, rank, const_cast<void*>(base), dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
-  return PA_OK;
-}
 
 size_t elem_bytes(pa_dtype t) { return t == PA_F32 ? 4 : ((t == PA_I8 || t == PA_FP8_E4M3) ? 1 : 2); }
 

@@ -1,0 +1,180 @@
+"""GPU paged prefill / chunked-prefill attention (tcgen05) through the C ABI against the
+fp64 oracle: whole prompts, chunks behind cached context and single tokens in one batch,
+fp16 and bf16, 1 to 16 query heads per cached head, every block size, sliding windows,
+several query and KV tiles with ragged tails, chunked = one-shot, empty sequences, and
+out-of-range inputs reported (not faulted).  Pool rows no sequence owns hold NaN, so a
+read outside the attended tokens shows up as a non-finite output."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_384_b200 as pa
+from parity import TOL, assert_no_device_error, compare
+
+pytestmark = pytest.mark.gpu
+
+DT = {"fp16": torch.float16, "bf16": torch.bfloat16}
+
+
+def paged_case(seed, ctx, qlen, Hq, Hkv, bs, io, D=128, extra=5):
+    """A shuffled pool holding each sequence's ctx tokens; q rows for its newest qlen tokens."""
+    g = torch.Generator().manual_seed(seed)
+    S = len(ctx)
+    nblk = [-(-c // bs) for c in ctx]
+    NB = sum(nblk) + extra
+    perm = torch.randperm(NB, generator=g).tolist()
+    kc = torch.full((NB, bs, Hkv, D), float("nan"), dtype=DT[io])
+    vc = torch.full((NB, bs, Hkv, D), float("nan"), dtype=DT[io])
+    MB = max(1, max(nblk))
+    bt = torch.full((S, MB), -1, dtype=torch.int32)
+    k = 0
+    for s in range(S):
+        K = torch.randn(ctx[s], Hkv, D, generator=g).to(DT[io])
+        V = torch.randn(ctx[s], Hkv, D, generator=g).to(DT[io])
+        for lb in range(nblk[s]):
+            pb = perm[k]
+            k += 1
+            bt[s, lb] = pb
+            lo, hi = lb * bs, min(ctx[s], (lb + 1) * bs)
+            kc[pb, : hi - lo] = K[lo:hi]
+            vc[pb, : hi - lo] = V[lo:hi]
+    q = torch.randn(sum(qlen), Hq, D, generator=g).to(DT[io])
+    cu = torch.tensor([0] + list(np.cumsum(qlen)), dtype=torch.int32)
+    return q, kc, vc, bt, cu, torch.tensor(ctx, dtype=torch.int32)
+
+
+def run_gpu(q, kc, vc, bt, cu, ctx, scale, window=0, max_q_len=None):
+    out = torch.empty_like(q, device="cuda")
+    mq = int((cu[1:] - cu[:-1]).max()) if max_q_len is None else max_q_len
+    pa.paged_attention_prefill(out, q.cuda(), kc.cuda(), vc.cuda(), bt.cuda(), cu.cuda(), ctx.cuda(), mq, scale,
+                               window)
+    torch.cuda.synchronize()
+    return out
+
+
+def check(seed, ctx, qlen, Hq, Hkv, bs, io, window=0):
+    q, kc, vc, bt, cu, cl = paged_case(seed, ctx, qlen, Hq, Hkv, bs, io)
+    scale = 1 / math.sqrt(128)
+    out = run_gpu(q, kc, vc, bt, cu, cl, scale, window)
+    assert_no_device_error()
+    ref = oracle.paged_prefill(q, kc, vc, bt, cu, cl, scale, window)
+    return compare(out, ref, io, TOL[io])
+
+
+@pytest.mark.parametrize("io", ["fp16", "bf16"])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 2), (16, 2), (8, 1)])
+def test_prefill_mixed_batch(cuda_device, io, Hq, Hkv):
+    # a whole prompt, a chunk behind cached context, a single token, a prompt of one block
+    check(1, [37, 300, 129, 16], [37, 90, 1, 16], Hq, Hkv, 16, io)
+
+
+@pytest.mark.parametrize("bs", [8, 16, 32, 64, 128])
+def test_prefill_block_sizes(cuda_device, bs):
+    check(2, [130, 77, 256], [130, 40, 129], 4, 2, bs, "fp16")
+
+
+@pytest.mark.parametrize("window", [1, 17, 128, 300, 5000])
+def test_prefill_sliding_window(cuda_device, window):
+    check(3, [400, 260, 45], [400, 70, 45], 8, 2, 16, "fp16", window)
+    check(4, [333], [200], 2, 2, 32, "bf16", window)
+
+
+def test_prefill_sixteen_query_heads_per_cached_head(cuda_device):
+    check(5, [200, 57], [200, 57], 32, 2, 16, "bf16")
+
+
+@pytest.mark.parametrize("io", ["fp16", "bf16"])
+def test_prefill_long_prompt_many_tiles(cuda_device, io):
+    # 9 query tiles x 8 KV tiles per head, ragged in both
+    check(6, [1000], [1000], 2, 2, 16, io)
+
+
+def test_chunked_prefill_equals_one_shot(cuda_device):
+    n = 700
+    q, kc, vc, bt, cu, cl = paged_case(7, [n], [n], 8, 8, 16, "fp16")
+    scale = 0.09
+    whole = run_gpu(q, kc, vc, bt, cu, cl, scale)
+    pieces = []
+    for a, b in ((0, 130), (130, 131), (131, 512), (512, 700)):
+        pieces.append(run_gpu(q[a:b].contiguous(), kc, vc, bt, torch.tensor([0, b - a], dtype=torch.int32),
+                              torch.tensor([b], dtype=torch.int32), scale))
+    chunked = torch.cat(pieces)
+    ref = oracle.paged_prefill(q, kc, vc, bt, cu, cl, scale)
+    compare(chunked, ref, "fp16", TOL["fp16"])
+    compare(whole, ref, "fp16", TOL["fp16"])
+    assert (chunked.float() - whole.float()).abs().max().item() <= 2e-3
+
+
+def test_prefill_empty_sequences_and_loose_max_q_len(cuda_device):
+    q, kc, vc, bt, cu, cl = paged_case(8, [50, 20, 90], [0, 20, 0], 4, 4, 16, "bf16")
+    out = run_gpu(q, kc, vc, bt, cu, cl, 0.1, max_q_len=300)
+    assert_no_device_error()
+    ref = oracle.paged_prefill(q, kc, vc, bt, cu, cl, 0.1)
+    compare(out, ref, "bf16", TOL["bf16"])
+
+
+def test_prefill_single_tokens_match_decode(cuda_device):
+    ctx = [1, 15, 16, 33, 700]
+    q, kc, vc, bt, cu, cl = paged_case(9, ctx, [1] * 5, 16, 2, 16, "fp16")
+    pre = run_gpu(q, kc, vc, bt, cu, cl, 0.2)
+    dec = torch.empty_like(q, device="cuda")
+    pa.paged_attention_decode(dec, q.cuda(), kc.cuda(), vc.cuda(), bt.cuda(), cl.cuda(), 0.2)
+    torch.cuda.synchronize()
+    assert (pre.float() - dec.float()).abs().max().item() <= 2e-3
+    compare(pre, oracle.paged_prefill(q, kc, vc, bt, cu, cl, 0.2), "fp16", TOL["fp16"])
+
+
+def test_prefill_reports_bad_lengths_and_table_entries(cuda_device):
+    q, kc, vc, bt, cu, cl = paged_case(10, [40, 40], [40, 40], 2, 2, 16, "fp16")
+    bad_cl = cl.clone()
+    bad_cl[1] = 30                                      # fewer cached tokens than queries
+    run_gpu(q, kc, vc, bt, cu, bad_cl, 0.1)
+    assert pa.device_error() & pa.DEVERR["context"]
+    run_gpu(q, kc, vc, bt, cu, cl, 0.1, max_q_len=20)   # q_len above the promised bound
+    assert pa.device_error() & pa.DEVERR["context"]
+    bad_bt = bt.clone()
+    bad_bt[0, 1] = kc.shape[0] + 3                      # a block id outside the pool
+    run_gpu(q, kc, vc, bad_bt, cu, cl, 0.1)
+    assert pa.device_error() & pa.DEVERR["table"]
+    assert_no_device_error()
+
+
+def test_prefill_host_validation(cuda_device):
+    q, kc, vc, bt, cu, cl = paged_case(11, [20], [20], 6, 2, 16, "fp16")   # 3 heads per cached head
+    with pytest.raises(pa.PagedAttnError):
+        run_gpu(q, kc, vc, bt, cu, cl, 0.1)
+    q, kc, vc, bt, cu, cl = paged_case(12, [20], [20], 2, 2, 16, "fp16", D=64)
+    with pytest.raises(pa.PagedAttnError):
+        run_gpu(q, kc, vc, bt, cu, cl, 0.1)
+
+
+def test_prefill_llama70b_prompt_batch_sampled(cuda_device):
+    """4 prompts x 2048 tokens (8192 query rows), 64 heads, bs 16, fp16: the prefill
+    workload's shape.  The oracle checks the first and last 48 query rows of every prompt
+    on 4 heads (its causal semantics make a prefix or a suffix a problem of its own)."""
+    S, n, H, bs = 4, 2048, 64, 16
+    g = torch.Generator().manual_seed(13)
+    NB = S * n // bs + 16
+    perm = torch.randperm(NB, generator=g)
+    bt = perm[: S * n // bs].view(S, n // bs).to(torch.int32).contiguous()
+    kc = torch.randn(NB, bs, H, 128, generator=g, dtype=torch.float16)
+    vc = torch.randn(NB, bs, H, 128, generator=g, dtype=torch.float16)
+    q = torch.randn(S * n, H, 128, generator=g, dtype=torch.float16)
+    cu = torch.arange(0, S * n + 1, n, dtype=torch.int32)
+    cl = torch.full((S,), n, dtype=torch.int32)
+    scale = 1 / math.sqrt(128)
+    out = run_gpu(q, kc, vc, bt, cu, cl, scale).cpu()
+    assert_no_device_error()
+    heads = [0, 21, 42, 63]
+    ks, vs = kc[:, :, heads].contiguous(), vc[:, :, heads].contiguous()
+    k = 48
+    for s in range(S):
+        rows = q[s * n:(s + 1) * n][:, heads]
+        one = torch.tensor([0, k], dtype=torch.int32)
+        first = oracle.paged_prefill(rows[:k].contiguous(), ks, vs, bt[s:s + 1], one, [k], scale)
+        last = oracle.paged_prefill(rows[-k:].contiguous(), ks, vs, bt[s:s + 1], one, [n], scale)
+        compare(out[s * n:s * n + k][:, heads], first, "fp16", TOL["fp16"])
+        compare(out[(s + 1) * n - k:(s + 1) * n][:, heads], last, "fp16", TOL["fp16"])
