@@ -229,10 +229,10 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         wait_or_abort(full0 + 8 * (k % kStages), (k / kStages) & 1, abort);
   } else if (warp == 1) {
     // ------------------------------------------------------------------- MMA issuer --
-    // One lane polls both kinds of work and issues whichever is ready: the score MMA of
-    // the next tile whose K/V/q landed, or the value MMA of the oldest tile whose
-    // probabilities are written.  Neither waits behind the other, so a stage is released
-    // as soon as its value MMA is done.
+    // One lane polls both kinds of work (non-blocking probes) and issues whichever is
+    // ready: the score MMA of the next tile whose K/V/q landed, or the value MMA of the
+    // oldest tile whose probabilities are written.  Neither waits behind the other, so a
+    // stage is released as soon as its value MMA is done.
     if (lane == 0) {
       int s_next = 0, o_next = 0;
       uint32_t idle = 0;
@@ -240,8 +240,8 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         bool progressed = false;
         if (s_next < n) {
           const int st = s_next % kStages, b = s_next % 2;
-          if (mbar_try_wait(full0 + 8 * st, (s_next / kStages) & 1) &&
-              (s_next < 2 || mbar_try_wait(s_empty0 + 8 * b, ((s_next / 2) - 1) & 1))) {
+          if (mbar_test_wait(full0 + 8 * st, (s_next / kStages) & 1) &&
+              (s_next < 2 || mbar_test_wait(s_empty0 + 8 * b, ((s_next / 2) - 1) & 1))) {
             tc_fence_after_sync();
             const uint32_t sb = stage(st);
 #pragma unroll
@@ -258,7 +258,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         }
         if (o_next < s_next) {
           const int b = o_next % 2;
-          if (mbar_try_wait(p_full0 + 8 * b, (o_next / 2) & 1)) {
+          if (mbar_test_wait(p_full0 + 8 * b, (o_next / 2) & 1)) {
             tc_fence_after_sync();
             const uint32_t sb = stage(o_next % kStages);
             const uint32_t o_tmem = tmem + 2 * kHeadsN + b * kHeadsN;
@@ -278,7 +278,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         }
         if (progressed) {
           idle = 0;
-        } else if (*abort || ++idle > 4 * kWaitLimit) {
+        } else if (*abort || ++idle > 16 * kWaitLimit) {
           if (!*abort) decode_error(PA_DEVERR_TIMEOUT);
           *abort = 1;
           break;

@@ -18,16 +18,16 @@
 //   S[128 rows x 128 kv]  = Q[128 x 128 d] . K^T          (K-major A and B; fp32 in TMEM)
 //   O[128 rows x 128 d]  += P[128 x 128 kv] . V           (K-major A, MN-major B; fp32 in TMEM)
 //
-// Roles (one CTA per SM, 6 warps):
+// Roles (one CTA per SM, 10 warps):
 //   warp 0      TMA producer: the q rows once, then per tile the attended blocks' K and V
 //               (64-dim halves, 128-byte swizzle) into separate 2-deep K and V rings; block
 //               ids for the next tile are fetched while the current one is issued.
 //   warp 1      TMEM owner and MMA issuer (one lane), polling: score MMA of the next tile
 //               whose K landed, value MMA of the tile whose probabilities are written.
-//   warps 2..5  softmax, thread = query row = TMEM lane: scale, causal/window mask, online
-//               softmax in base 2 with a lazily moved reference maximum (O in TMEM is
-//               rescaled only when a row's maximum grows by more than 2^8), probabilities
-//               to shared memory as the A operand, final O / l to the output.
+//   warps 2..9  softmax, two warps per query row (TMEM lane), 64 columns each: scale,
+//               causal/window mask, online softmax in base 2 with a lazily moved reference
+//               maximum (O in TMEM is rescaled only when a row's maximum grows by more than
+//               2^8), probabilities to shared memory as the A operand, final O / l out.
 // bf16 probabilities are split into hi + lo bf16 parts (two value MMAs) so the weights keep
 // ~16 significant bits.  Every wait is bounded; one that gives up raises PA_DEVERR_TIMEOUT
 // and an abort flag that ends the others.
@@ -53,14 +53,22 @@ constexpr int kDim = 128;                 // head_dim
 constexpr int kHalf = 128 * 128;          // one 64-element half of a 128-row operand: 16 KiB
 constexpr int kOpBytes = 2 * kHalf;       // a whole 128 x 128 operand (Q, K, V or P)
 constexpr int kRing = 2;                  // depth of the K ring and of the V ring
-constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 512;       // S0 [0,128)  S1 [128,256)  O [256,384)
+constexpr int kSoftmaxThreads = 256;   // 8 warps: two per TMEM lane quarter, 64 columns each
+constexpr int kThreads = 64 + kSoftmaxThreads;
+constexpr uint32_t kTmemCols = 512;       // S0 [0,128)  S1 [128,256)  O [256,384)  exchange [384,390)
 constexpr uint32_t kColO = 256;
+constexpr uint32_t kColX = 384;           // per-row partial maxima (by tile parity and half), then sums
 constexpr float kRescaleThreshold = 8.f;  // log2 units: probabilities stay below 2^8
 
+// Probability buffers: fp16 keeps two (tile j+1 is written while the value MMA of tile j
+// reads the other); bf16 needs hi + lo parts, which leave room for one.
+template <bool SPLIT>
+constexpr int p_buffers() {
+  return SPLIT ? 1 : 2;
+}
 template <bool SPLIT>
 constexpr size_t smem_bytes() {
-  return 1024 + kOpBytes + 2 * kRing * kOpBytes + (SPLIT ? 2 : 1) * kOpBytes;
+  return 1024 + kOpBytes + 2 * kRing * kOpBytes + 2 * kOpBytes;
 }
 
 struct PrefillParams {
@@ -76,7 +84,8 @@ struct PfShared {
   uint64_t q_full;
   uint64_t k_full[kRing], k_empty[kRing], v_full[kRing], v_empty[kRing];
   uint64_t s_full[2], s_empty[2];
-  uint64_t p_full, o_full, mma_done;
+  uint64_t p_full[2], o_full[2];  // by tile parity: probabilities written / value MMA done
+  uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
 };
@@ -91,12 +100,26 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
   return false;
 }
 
-__device__ __forceinline__ uint32_t pack2(__half a, __half b) {
-  return static_cast<uint32_t>(__half_as_ushort(a)) | (static_cast<uint32_t>(__half_as_ushort(b)) << 16);
-}
-__device__ __forceinline__ uint32_t pack2(__nv_bfloat16 a, __nv_bfloat16 b) {
-  return static_cast<uint32_t>(__bfloat16_as_ushort(a)) | (static_cast<uint32_t>(__bfloat16_as_ushort(b)) << 16);
-}
+// Two weights rounded to IO by one packed conversion, with their values back in fp32.
+template <typename IO> struct Pair;
+template <> struct Pair<__half> {
+  __half2 v;
+  uint32_t bits;
+  __device__ __forceinline__ Pair(float a, float b) : v(__floats2half2_rn(a, b)) {
+    bits = *reinterpret_cast<const uint32_t*>(&v);
+  }
+  __device__ __forceinline__ float lo_f() const { return __low2float(v); }
+  __device__ __forceinline__ float hi_f() const { return __high2float(v); }
+};
+template <> struct Pair<__nv_bfloat16> {
+  __nv_bfloat162 v;
+  uint32_t bits;
+  __device__ __forceinline__ Pair(float a, float b) : v(__floats2bfloat162_rn(a, b)) {
+    bits = *reinterpret_cast<const uint32_t*>(&v);
+  }
+  __device__ __forceinline__ float lo_f() const { return __uint_as_float(bits << 16); }
+  __device__ __forceinline__ float hi_f() const { return __uint_as_float(bits & 0xFFFF0000u); }
+};
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
@@ -153,12 +176,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   const uint32_t sQ = base;
   auto sK = [&](int st) { return base + kOpBytes + st * kOpBytes; };
   auto sV = [&](int st) { return base + (1 + kRing) * kOpBytes + st * kOpBytes; };
-  const uint32_t sP = base + (1 + 2 * kRing) * kOpBytes;  // hi part; the lo part follows (bf16)
+  constexpr int kPBuf = p_buffers<kSplit>();
+  // probability buffer i (fp16), or the hi (i = 0) and lo (i = 1) parts of the one bf16 buffer
+  auto sP = [&](int i) { return base + (1 + 2 * kRing) * kOpBytes + i * kOpBytes; };
   const uint32_t q_full = smem_u32(&sh.q_full);
   const uint32_t k_full0 = smem_u32(&sh.k_full[0]), k_empty0 = smem_u32(&sh.k_empty[0]);
   const uint32_t v_full0 = smem_u32(&sh.v_full[0]), v_empty0 = smem_u32(&sh.v_empty[0]);
   const uint32_t s_full0 = smem_u32(&sh.s_full[0]), s_empty0 = smem_u32(&sh.s_empty[0]);
-  const uint32_t p_full = smem_u32(&sh.p_full), o_full = smem_u32(&sh.o_full);
+  const uint32_t p_full0 = smem_u32(&sh.p_full[0]), o_full0 = smem_u32(&sh.o_full[0]);
   const uint32_t mma_done = smem_u32(&sh.mma_done);
   volatile int* abort = &sh.abort;
 
@@ -172,10 +197,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full0 + 8 * b, 1);
-      mbar_init(s_empty0 + 8 * b, 128);
+      mbar_init(s_empty0 + 8 * b, kSoftmaxThreads);
+      mbar_init(p_full0 + 8 * b, kSoftmaxThreads);
+      mbar_init(o_full0 + 8 * b, 1);
     }
-    mbar_init(p_full, 128);
-    mbar_init(o_full, 1);
     mbar_init(mma_done, 1);
     sh.abort = 0;
     fence_barrier_init();
@@ -188,6 +213,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer --
+    // Polls both rings and issues whichever load has a free slot, K first (the score MMA
+    // needs it earlier): a V slot waiting on a slow value MMA does not hold back K.
     const uint64_t keep = l2_policy_evict_last();    // K/V tiles are shared by the sequence's q tiles
     const uint64_t once = l2_policy_evict_first();   // q rows are read once
     if (lane == 0) {
@@ -199,65 +226,103 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       tma_load_3d(sQ + kHalf, &tmQ, q_full, 64, kh * p.GQ, q_start + i0, once);
     }
     const int32_t* table = p.block_tables + static_cast<size_t>(s) * p.MB;
-    TileBlocks tb = tile_blocks(j_lo, bs, kv_lo, p_max);
-    int pb_next = lane <= tb.hi - tb.lo ? __ldg(table + tb.lo + lane) : 0;
-    int k_issued = 0, v_issued = 0;
-    for (int j = 0; j < n; ++j) {
-      const TileBlocks cur = tb;
-      int pb = pb_next;
-      if (j + 1 < n) {  // next tile's block ids, in flight while this tile is issued
-        tb = tile_blocks(j_lo + j + 1, bs, kv_lo, p_max);
-        pb_next = lane <= tb.hi - tb.lo ? __ldg(table + tb.lo + lane) : 0;
+    auto entries = [&](int j) {  // lane l: block id of the tile's l-th attended block
+      const TileBlocks t = tile_blocks(j_lo + j, bs, kv_lo, p_max);
+      return lane <= t.hi - t.lo ? __ldg(table + t.lo + lane) : 0;
+    };
+    int k_next = 0, v_next = 0;
+    int pb_k = entries(0), pb_v = pb_k;  // entries of tiles k_next and v_next, fetched ahead
+    uint32_t idle = 0;
+    while (v_next < n) {
+      int which = -1;
+      if (lane == 0) {
+        if (k_next < n && (k_next < kRing || mbar_test_wait(k_empty0 + 8 * (k_next % kRing), ((k_next / kRing) - 1) & 1)))
+          which = 0;
+        else if (v_next < k_next &&
+                 (v_next < kRing || mbar_test_wait(v_empty0 + 8 * (v_next % kRing), ((v_next / kRing) - 1) & 1)))
+          which = 1;
       }
+      which = __shfl_sync(0xffffffffu, which, 0);
+      if (which < 0) {
+        if (*abort || ++idle > 4 * kWaitLimit) {
+          if (!*abort) prefill_error(PA_DEVERR_TIMEOUT);
+          *abort = 1;
+          break;
+        }
+        continue;
+      }
+      idle = 0;
+      const int j = which ? v_next : k_next;
+      int pb = which ? pb_v : pb_k;
+      const TileBlocks cur = tile_blocks(j_lo + j, bs, kv_lo, p_max);
       const int nload = cur.hi - cur.lo + 1;
       if (lane < nload && (pb < 0 || pb >= p.NB)) {
-        prefill_error(PA_DEVERR_TABLE);
+        if (which == 0) prefill_error(PA_DEVERR_TABLE);
         pb = 0;
       }
       const int st = j % kRing;
-      const uint32_t bytes = static_cast<uint32_t>(nload) * 2u * bs * 128u;
-      // K of tile j, then V of tile j; each copy is one 64-dim half of one block, one per lane.
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t full = (which ? v_full0 : k_full0) + 8 * st;
-        const uint32_t empty = (which ? v_empty0 : k_empty0) + 8 * st;
-        bool ok = true;
-        if (lane == 0) {
-          if (j >= kRing) ok = wait_or_abort(empty, ((j / kRing) - 1) & 1, abort);
-          if (ok) mbar_arrive_expect_tx(full, bytes);
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
-        const int cp = lane;  // 2 * nload <= 32 copies
-        const int b = __shfl_sync(0xffffffffu, pb, (cp >> 1) & 31);
-        if (cp < 2 * nload) {
-          const uint32_t row = static_cast<uint32_t>(cur.lo + (cp >> 1) - cur.first) * bs * 128u;
-          const uint32_t dst = (which ? sV(st) : sK(st)) + (cp & 1) * kHalf + row;
-          tma_load_3d(dst, which ? &tmV : &tmK, full, (cp & 1) * 64, kh, b * bs, keep);
-        }
-        if (which) ++v_issued; else ++k_issued;
+      const uint32_t full = (which ? v_full0 : k_full0) + 8 * st;
+      if (lane == 0) mbar_arrive_expect_tx(full, static_cast<uint32_t>(nload) * 2u * bs * 128u);
+      __syncwarp();
+      // each copy is one 64-dim half of one block, one copy per lane (2 * nload <= 32)
+      const int b = __shfl_sync(0xffffffffu, pb, (lane >> 1) & 31);
+      if (lane < 2 * nload) {
+        const uint32_t row = static_cast<uint32_t>(cur.lo + (lane >> 1) - cur.first) * bs * 128u;
+        const uint32_t dst = (which ? sV(st) : sK(st)) + (lane & 1) * kHalf + row;
+        tma_load_3d(dst, which ? &tmV : &tmK, full, (lane & 1) * 64, kh, b * bs, keep);
       }
-      if (v_issued != j + 1) break;
+      if (which) {
+        ++v_next;
+        if (v_next < n) pb_v = entries(v_next);
+      } else {
+        ++k_next;
+        if (k_next < n) pb_k = entries(k_next);
+      }
     }
     if (lane == 0) {  // never leave with copies in flight
       mbar_wait_bounded(q_full, 0);
-      for (int k = k_issued - kRing < 0 ? 0 : k_issued - kRing; k < k_issued; ++k)
+      for (int k = k_next - kRing < 0 ? 0 : k_next - kRing; k < k_next; ++k)
         mbar_wait_bounded(k_full0 + 8 * (k % kRing), (k / kRing) & 1);
-      for (int k = v_issued - kRing < 0 ? 0 : v_issued - kRing; k < v_issued; ++k)
+      for (int k = v_next - kRing < 0 ? 0 : v_next - kRing; k < v_next; ++k)
         mbar_wait_bounded(v_full0 + 8 * (k % kRing), (k / kRing) & 1);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------- MMA issuer --
+    // Polls without blocking; the value MMA goes first when both are ready, since the
+    // softmax warps wait on it.
     if (lane == 0) {
       int s_next = 0, o_next = 0;
       uint32_t idle = 0;
       bool ok = wait_or_abort(q_full, 0, abort);
       while (ok && o_next < n) {
         bool progressed = false;
+        if (o_next < s_next) {
+          const int st = o_next % kRing, b = o_next % 2;
+          if (mbar_test_wait(p_full0 + 8 * b, (o_next / 2) & 1) &&
+              mbar_test_wait(v_full0 + 8 * st, (o_next / kRing) & 1)) {
+            tc_fence_after_sync();
+            const int pbuf = o_next % kPBuf;
+#pragma unroll
+            for (int part = 0; part < (kSplit ? 2 : 1); ++part) {
+#pragma unroll
+              for (int kk = 0; kk < kKv / 16; ++kk) {  // O += P . V, 16 kv tokens per MMA
+                tc_mma_f16(tmem + kColO,
+                           smem_desc(sP(pbuf + part) + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024, kSwizzle128B),
+                           smem_desc(sV(st) + kk * 2048, kHalf, 1024, kSwizzle128B), kIdescO,
+                           o_next > 0 || part > 0 || kk > 0);
+              }
+            }
+            tc_commit(o_full0 + 8 * b);
+            tc_commit(v_empty0 + 8 * st);
+            ++o_next;
+            progressed = true;
+          }
+        }
         if (s_next < n) {
           const int st = s_next % kRing, b = s_next % 2;
-          if (mbar_try_wait(k_full0 + 8 * st, (s_next / kRing) & 1) &&
-              (s_next < 2 || mbar_try_wait(s_empty0 + 8 * b, ((s_next / 2) - 1) & 1))) {
+          if (mbar_test_wait(k_full0 + 8 * st, (s_next / kRing) & 1) &&
+              (s_next < 2 || mbar_test_wait(s_empty0 + 8 * b, ((s_next / 2) - 1) & 1))) {
             tc_fence_after_sync();
 #pragma unroll
             for (int kk = 0; kk < kDim / 16; ++kk) {  // S[b] = Q . K^T, 16 dims per MMA
@@ -271,29 +336,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
             progressed = true;
           }
         }
-        if (o_next < s_next) {
-          const int st = o_next % kRing;
-          if (mbar_try_wait(p_full, o_next & 1) && mbar_try_wait(v_full0 + 8 * st, (o_next / kRing) & 1)) {
-            tc_fence_after_sync();
-#pragma unroll
-            for (int part = 0; part < (kSplit ? 2 : 1); ++part) {
-#pragma unroll
-              for (int kk = 0; kk < kKv / 16; ++kk) {  // O += P . V, 16 kv tokens per MMA
-                tc_mma_f16(tmem + kColO,
-                           smem_desc(sP + part * kOpBytes + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024, kSwizzle128B),
-                           smem_desc(sV(st) + kk * 2048, kHalf, 1024, kSwizzle128B), kIdescO,
-                           o_next > 0 || part > 0 || kk > 0);
-              }
-            }
-            tc_commit(o_full);
-            tc_commit(v_empty0 + 8 * st);
-            ++o_next;
-            progressed = true;
-          }
-        }
         if (progressed) {
           idle = 0;
-        } else if (*abort || ++idle > 4 * kWaitLimit) {
+        } else if (*abort || ++idle > 16 * kWaitLimit) {
           if (!*abort) prefill_error(PA_DEVERR_TIMEOUT);
           *abort = 1;
           break;
@@ -305,119 +350,156 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     __syncwarp();
   } else {
     // ------------------------------------------------------------- softmax warps --
+    // Warps 2..9.  A warp may only touch the TMEM lane quarter (warp % 4); the two warps of
+    // a quarter share its 32 query rows and split the columns: half 0 takes kv tokens
+    // 0..63 of a tile (and head dims 0..63 of O), half 1 the rest.  They combine row
+    // maxima every tile through spare TMEM columns of their own lanes (shared memory is
+    // all taken by the operands), with a 64-thread named barrier per quarter.
     const int q4 = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int r = 32 * q4 + lane;  // query row = TMEM lane
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q4) << 16;
+    const uint32_t pair_bar = 1 + q4;
     const int tl = r >> p.gq_shift, g = r & (p.GQ - 1);
     const bool row_valid = tl < ntok;
     const int pos = p_min + tl;
     const int lo_row = p.window > 0 ? max(0, pos - p.window + 1) : 0;
     float m_run = -FLT_MAX, l = 0.f;
-    bool done = false;
+    // Bounded wait for the value MMA of tile t, agreed by the whole warp.
+    auto wait_pv = [&](int t) {
+      return __all_sync(0xffffffffu, wait_or_abort(o_full0 + 8 * (t % 2), (t / 2) & 1, abort));
+    };
+    // The two warps of a quarter meet at a named barrier every tile, so neither may leave
+    // the loop early: after an abort a warp keeps stepping through the barriers with `ok`
+    // false and does no other work.
+    bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int b = j % 2, st = j % kRing;
-      if (!__all_sync(0xffffffffu, wait_or_abort(s_full0 + 8 * b, (j / 2) & 1, abort))) break;
-      tc_fence_after_sync();
-      float sc[kKv];
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) tmem_load32(tmem + lane_addr + b * kKv + 32 * c4, sc + 32 * c4);
-      tc_fence_before_sync();
-      mbar_arrive(s_empty0 + 8 * b);
-
+      ok = ok && __all_sync(0xffffffffu, wait_or_abort(s_full0 + 8 * b, (j / 2) & 1, abort));
       const int kv0 = (j_lo + j) * kKv;
-      const int c_lo = lo_row - kv0, c_hi = row_valid ? pos - kv0 : -1;
-      float mt = -INFINITY;
+      const int c0 = 64 * half;  // this warp's first column
+      float sc[64];
+      float mraw = -INFINITY;
+      if (ok) {
+        tc_fence_after_sync();
+        tmem_load64(tmem + lane_addr + b * kKv + c0, sc);
+        tc_fence_before_sync();
+        mbar_arrive(s_empty0 + 8 * b);
+        // Interior tiles (every row attends every column) skip the mask.
+        const bool interior =
+            ntok == p.tq && kv0 + kKv - 1 <= p_min && (p.window <= 0 || kv0 >= p_max - p.window + 1);
+        if (!interior) {
+          const int c_lo = lo_row - kv0 - c0, c_hi = row_valid ? pos - kv0 - c0 : -1;
 #pragma unroll
-      for (int c = 0; c < kKv; ++c) {
-        sc[c] = (c >= c_lo && c <= c_hi) ? sc[c] * p.qscale : -INFINITY;
-        mt = fmaxf(mt, sc[c]);
+          for (int c = 0; c < 64; ++c) sc[c] = (c >= c_lo && c <= c_hi) ? sc[c] : -INFINITY;
+        }
+        float mx[8];  // eight independent chains instead of one 64-long one
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = sc[k];
+#pragma unroll
+        for (int c = 8; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], sc[c]);
+        mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       }
+      tmem_store1(tmem + lane_addr + kColX + 2 * b + half, mraw);
+      tc_fence_before_sync();
+      named_barrier_sync(pair_bar, 64);
+      tc_fence_after_sync();
+      mraw = fmaxf(mraw, tmem_load1(tmem + lane_addr + kColX + 2 * b + (half ^ 1)));
+      if (!ok) continue;
+      const float mt = mraw * p.qscale;  // scores in base-2 units (qscale > 0 keeps the order)
       float alpha = 1.f;
       bool rescale = false;
       if (mt > m_run + kRescaleThreshold) {  // move the reference maximum
-        alpha = exp2f(m_run - mt);
+        alpha = ex2_ftz(m_run - mt);
         rescale = l > 0.f;                   // O holds earlier contributions of this row
         l *= alpha;
         m_run = mt;
       }
-      // The previous value MMA must be done before P is overwritten or O rescaled.
-      if (j > 0 && !__all_sync(0xffffffffu, wait_or_abort(o_full, (j - 1) & 1, abort))) break;
-      if (__any_sync(0xffffffffu, rescale)) {
+      // O may be rescaled only after the previous value MMA; the probability buffer of
+      // tile j is free once the value MMA that last read it (tile j - kPBuf) is done.
+      const bool any_rescale = __any_sync(0xffffffffu, rescale);
+      if (any_rescale && !wait_pv(j - 1)) ok = false;
+      if (ok && !any_rescale && j >= kPBuf && !wait_pv(j - kPBuf)) ok = false;
+      if (!ok) continue;
+      if (any_rescale) {
         tc_fence_after_sync();
         const float a = rescale ? alpha : 1.f;
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
+        for (int c4 = 0; c4 < 2; ++c4) {  // this warp's 64 columns of O
           float o[32];
-          tmem_load32(tmem + lane_addr + kColO + 32 * c4, o);
+          tmem_load32(tmem + lane_addr + kColO + 64 * half + 32 * c4, o);
 #pragma unroll
           for (int k = 0; k < 32; ++k) o[k] *= a;
-          tmem_store32(tmem + lane_addr + kColO + 32 * c4, o);
+          tmem_store32(tmem + lane_addr + kColO + 64 * half + 32 * c4, o);
         }
       }
       // V rows of tokens outside the loaded blocks or past the context may hold anything
-      // (NaN); their weights are 0, so give the value MMA zeros there (thread r: kv row r).
+      // (NaN); their weights are 0, so give the value MMA zeros there (kv row r; half 0
+      // clears its 64-dim lo half, half 1 the hi half).
       const TileBlocks tb = tile_blocks(j_lo + j, bs, kv_lo, p_max);
       const int clean_lo = tb.lo * bs - kv0, clean_hi = min(ctx, (tb.hi + 1) * bs) - kv0;
       if (clean_lo > 0 || clean_hi < kKv) {
-        if (!__all_sync(0xffffffffu, wait_or_abort(v_full0 + 8 * st, (j / kRing) & 1, abort))) break;
+        if (!__all_sync(0xffffffffu, wait_or_abort(v_full0 + 8 * st, (j / kRing) & 1, abort))) {
+          ok = false;
+          continue;
+        }
         if (r < clean_lo || r >= clean_hi) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            st_shared_v4(sV(st) + r * 128 + 16 * k, 0, 0, 0, 0);
-            st_shared_v4(sV(st) + kHalf + r * 128 + 16 * k, 0, 0, 0, 0);
-          }
+          for (int k = 0; k < 8; ++k) st_shared_v4(sV(st) + half * kHalf + r * 128 + 16 * k, 0, 0, 0, 0);
         }
       }
-      // Probabilities, written as row r of the K-major, 128-byte-swizzled A operand.
-      float ls = 0.f;
-      const uint32_t prow = (r >> 3) * 1024 + (r & 7) * 128;
+      // Probabilities, written as row r of this warp's 64-token half of the K-major,
+      // 128-byte-swizzled A operand.  exp2(s * qscale - m) is one FFMA and one MUFU op;
+      // two weights are rounded and packed by one conversion.
+      float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const float neg_m = -m_run;
+      const uint32_t pdst = sP(kSplit ? 0 : j % kPBuf) + half * kHalf + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int c = 0; c < 8; ++c) {
+        uint32_t w_hi[4], w_lo[4];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t w_hi[4], w_lo[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float x0 = exp2f(sc[64 * h + 8 * c + 2 * e] - m_run);
-            const float x1 = exp2f(sc[64 * h + 8 * c + 2 * e + 1] - m_run);
-            const IO h0 = float_to<IO>(x0), h1 = float_to<IO>(x1);
-            w_hi[e] = pack2(h0, h1);
-            if (kSplit) {
-              w_lo[e] = pack2(float_to<IO>(x0 - static_cast<float>(h0)), float_to<IO>(x1 - static_cast<float>(h1)));
-              ls += x0 + x1;
-            } else {
-              ls += static_cast<float>(h0) + static_cast<float>(h1);  // the rounded weights the MMA uses
-            }
+        for (int e = 0; e < 4; ++e) {
+          const int k = 8 * c + 2 * e;
+          const float x0 = ex2_ftz(fmaf(sc[k], p.qscale, neg_m));
+          const float x1 = ex2_ftz(fmaf(sc[k + 1], p.qscale, neg_m));
+          const Pair<IO> hi(x0, x1);
+          w_hi[e] = hi.bits;
+          if (kSplit) {
+            w_lo[e] = Pair<IO>(x0 - hi.lo_f(), x1 - hi.hi_f()).bits;
+            ls[(c & 1) * 4 + e] += x0 + x1;
+          } else {
+            ls[(c & 1) * 4 + e] += hi.lo_f() + hi.hi_f();  // the rounded weights the MMA uses
           }
-          const uint32_t addr = sP + h * kHalf + prow + ((c ^ (r & 7)) << 4);
-          st_shared_v4(addr, w_hi[0], w_hi[1], w_hi[2], w_hi[3]);
-          if (kSplit) st_shared_v4(addr + kOpBytes, w_lo[0], w_lo[1], w_lo[2], w_lo[3]);
         }
+        const uint32_t addr = pdst + ((c ^ (r & 7)) << 4);
+        st_shared_v4(addr, w_hi[0], w_hi[1], w_hi[2], w_hi[3]);
+        if (kSplit) st_shared_v4(addr + kOpBytes, w_lo[0], w_lo[1], w_lo[2], w_lo[3]);
       }
-      l += ls;
+      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       fence_proxy_async_shared();
       tc_fence_before_sync();
-      mbar_arrive(p_full);
-      if (j == n - 1) done = true;
+      mbar_arrive(p_full0 + 8 * b);
     }
-    if (done && __all_sync(0xffffffffu, wait_or_abort(o_full, (n - 1) & 1, abort))) {
+    // Softmax denominators: the two halves of a row add their partial sums.
+    tmem_store1(tmem + lane_addr + kColX + 4 + half, l);
+    tc_fence_before_sync();
+    named_barrier_sync(pair_bar, 64);
+    tc_fence_after_sync();
+    l += tmem_load1(tmem + lane_addr + kColX + 4 + (half ^ 1));
+    if (ok && wait_pv(n - 1)) {
       tc_fence_after_sync();
       const float inv = row_valid ? 1.f / l : 0.f;
       IO* orow = reinterpret_cast<IO*>(p.out) +
-                 (static_cast<size_t>(q_start + i0 + tl) * p.Hq + static_cast<size_t>(kh) * p.GQ + g) * kDim;
+                 (static_cast<size_t>(q_start + i0 + tl) * p.Hq + static_cast<size_t>(kh) * p.GQ + g) * kDim + 64 * half;
+      float o[64];
+      tmem_load64(tmem + lane_addr + kColO + 64 * half, o);
+      if (row_valid) {
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        float o[32];
-        tmem_load32(tmem + lane_addr + kColO + 32 * c4, o);
-        if (row_valid) {
+        for (int v = 0; v < 8; ++v) {
+          uint32_t w[4];
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              w[e] = pack2(float_to<IO>(o[8 * v + 2 * e] * inv), float_to<IO>(o[8 * v + 2 * e + 1] * inv));
-            *reinterpret_cast<uint4*>(orow + 32 * c4 + 8 * v) = make_uint4(w[0], w[1], w[2], w[3]);
-          }
+          for (int e = 0; e < 4; ++e) w[e] = Pair<IO>(o[8 * v + 2 * e] * inv, o[8 * v + 2 * e + 1] * inv).bits;
+          *reinterpret_cast<uint4*>(orow + 8 * v) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
     }
