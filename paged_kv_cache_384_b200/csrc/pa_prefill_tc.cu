@@ -15,19 +15,23 @@
 // times the GQ query heads that share the cached head (row = token * GQ + head).  Per
 // 128-token KV tile:
 //
-//   S[128 rows x 128 kv]  = Q[128 x 128 d] . K^T          (K-major A and B; fp32 in TMEM)
-//   O[128 rows x 128 d]  += P[128 x 128 kv] . V           (K-major A, MN-major B; fp32 in TMEM)
+//   S[128 rows x 128 kv]  = Q[128 x 128 d] . K^T          (K-major A and B in shared memory)
+//   O_h[128 rows x 128 d] += P[:, 64h..] . V[64h.., :]   (A = P in TMEM over S, MN-major V)
+//
+// with fp32 accumulators in TMEM.  Keeping P in tensor memory leaves shared memory to the
+// q rows and 3-deep K and V rings.
 //
 // Roles (one CTA per SM, 10 warps):
 //   warp 0      TMA producer: the q rows once, then per tile the attended blocks' K and V
-//               (64-dim halves, 128-byte swizzle) into separate 2-deep K and V rings; block
+//               (64-dim halves, 128-byte swizzle) into separate 3-deep K and V rings; block
 //               ids for the next tile are fetched while the current one is issued.
 //   warp 1      TMEM owner and MMA issuer (one lane), polling: score MMA of the next tile
 //               whose K landed, value MMA of the tile whose probabilities are written.
-//   warps 2..9  softmax, two warps per query row (TMEM lane), 64 columns each: scale,
-//               causal/window mask, online softmax in base 2 with a lazily moved reference
-//               maximum (O in TMEM is rescaled only when a row's maximum grows by more than
-//               2^8), probabilities to shared memory as the A operand, final O / l out.
+//   warps 2..9  softmax, two warps per query row (TMEM lane), each with its own half of
+//               every tile's kv tokens and its own accumulator O_h: scale, causal/window
+//               mask, online softmax in base 2 with a lazily moved reference maximum (O_h is
+//               rescaled only when the half's maximum grows by more than 2^8), probabilities
+//               into TMEM as the A operand; the halves are merged at the end.
 // bf16 probabilities are split into hi + lo bf16 parts (two value MMAs) so the weights keep
 // ~16 significant bits.  Every wait is bounded; one that gives up raises PA_DEVERR_TIMEOUT
 // and an abort flag that ends the others.
@@ -52,24 +56,18 @@ constexpr int kKv = 128;                  // kv tokens per tile
 constexpr int kDim = 128;                 // head_dim
 constexpr int kHalf = 128 * 128;          // one 64-element half of a 128-row operand: 16 KiB
 constexpr int kOpBytes = 2 * kHalf;       // a whole 128 x 128 operand (Q, K, V or P)
-constexpr int kRing = 2;                  // depth of the K ring and of the V ring
+constexpr int kRing = 3;                  // depth of the K ring and of the V ring
 constexpr int kSoftmaxThreads = 256;   // 8 warps: two per TMEM lane quarter, 64 columns each
 constexpr int kThreads = 64 + kSoftmaxThreads;
-constexpr uint32_t kTmemCols = 512;       // S0 [0,128)  S1 [128,256)  O [256,384)  exchange [384,390)
+constexpr uint32_t kTmemCols = 512;       // S0 [0,128)  S1 [128,256)  O_0 [256,384)  O_1 [384,512)
+// Each softmax half h owns the 64 score columns [64h, 64h+64) of an S buffer and writes its
+// probabilities over them: hi weights in the first 32 columns (two 16-bit weights per
+// column), the lo parts of bf16 weights in the next 32.  Half h accumulates O_h over its
+// own kv tokens with its own running maximum; the halves are combined once at the end.
 constexpr uint32_t kColO = 256;
-constexpr uint32_t kColX = 384;           // per-row partial maxima (by tile parity and half), then sums
 constexpr float kRescaleThreshold = 8.f;  // log2 units: probabilities stay below 2^8
 
-// Probability buffers: fp16 keeps two (tile j+1 is written while the value MMA of tile j
-// reads the other); bf16 needs hi + lo parts, which leave room for one.
-template <bool SPLIT>
-constexpr int p_buffers() {
-  return SPLIT ? 1 : 2;
-}
-template <bool SPLIT>
-constexpr size_t smem_bytes() {
-  return 1024 + kOpBytes + 2 * kRing * kOpBytes + 2 * kOpBytes;
-}
+constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(1 + 2 * kRing) * kOpBytes;  // Q, K ring, V ring
 
 struct PrefillParams {
   void* out;
@@ -83,7 +81,7 @@ struct PrefillParams {
 struct PfShared {
   uint64_t q_full;
   uint64_t k_full[kRing], k_empty[kRing], v_full[kRing], v_empty[kRing];
-  uint64_t s_full[2], s_empty[2];
+  uint64_t s_full[2];
   uint64_t p_full[2], o_full[2];  // by tile parity: probabilities written / value MMA done
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -137,6 +135,36 @@ __device__ __forceinline__ TileBlocks tile_blocks(int jt, int bs, int kv_lo, int
   return t;
 }
 
+// Block-table entries of one sequence, 32 at a time, one per lane: the window in use and
+// the next one, whose load is in flight while the current one serves.
+struct TableWindow {
+  const int32_t* table;
+  int lim, base, cur, next;
+  __device__ __forceinline__ int fetch(int from, int lane) const {
+    return from + lane < lim ? __ldg(table + from + lane) : 0;
+  }
+  __device__ __forceinline__ void init(const int32_t* t, int limit, int first, int lane) {
+    table = t;
+    lim = limit;
+    base = first;
+    cur = fetch(first, lane);
+    next = fetch(first + 32, lane);
+  }
+  // Lane l (< count <= 16) gets the entry of block lo + l; lo never decreases.
+  __device__ __forceinline__ int get(int lo, int count, int lane) {
+    while (lo >= base + 32) {
+      base += 32;
+      cur = next;
+      next = fetch(base + 32, lane);
+    }
+    const int idx = lo - base + lane;
+    const int a = __shfl_sync(0xffffffffu, cur, idx & 31);
+    if (lo - base + count <= 32) return a;  // uniform: the tile lies in the current window
+    const int b = __shfl_sync(0xffffffffu, next, idx & 31);
+    return idx < 32 ? a : b;
+  }
+};
+
 template <typename IO>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -176,13 +204,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   const uint32_t sQ = base;
   auto sK = [&](int st) { return base + kOpBytes + st * kOpBytes; };
   auto sV = [&](int st) { return base + (1 + kRing) * kOpBytes + st * kOpBytes; };
-  constexpr int kPBuf = p_buffers<kSplit>();
-  // probability buffer i (fp16), or the hi (i = 0) and lo (i = 1) parts of the one bf16 buffer
-  auto sP = [&](int i) { return base + (1 + 2 * kRing) * kOpBytes + i * kOpBytes; };
   const uint32_t q_full = smem_u32(&sh.q_full);
   const uint32_t k_full0 = smem_u32(&sh.k_full[0]), k_empty0 = smem_u32(&sh.k_empty[0]);
   const uint32_t v_full0 = smem_u32(&sh.v_full[0]), v_empty0 = smem_u32(&sh.v_empty[0]);
-  const uint32_t s_full0 = smem_u32(&sh.s_full[0]), s_empty0 = smem_u32(&sh.s_empty[0]);
+  const uint32_t s_full0 = smem_u32(&sh.s_full[0]);
   const uint32_t p_full0 = smem_u32(&sh.p_full[0]), o_full0 = smem_u32(&sh.o_full[0]);
   const uint32_t mma_done = smem_u32(&sh.mma_done);
   volatile int* abort = &sh.abort;
@@ -197,7 +222,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full0 + 8 * b, 1);
-      mbar_init(s_empty0 + 8 * b, kSoftmaxThreads);
       mbar_init(p_full0 + 8 * b, kSoftmaxThreads);
       mbar_init(o_full0 + 8 * b, 1);
     }
@@ -213,8 +237,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer --
-    // Polls both rings and issues whichever load has a free slot, K first (the score MMA
-    // needs it earlier): a V slot waiting on a slow value MMA does not hold back K.
+    // Polls both rings and issues whichever load has a free slot: V of the oldest tile
+    // whose K is out first (the value MMA is on the softmax warps' path), else the next K.
+    // K and V each walk the block table through their own prefetched windows.
     const uint64_t keep = l2_policy_evict_last();    // K/V tiles are shared by the sequence's q tiles
     const uint64_t once = l2_policy_evict_first();   // q rows are read once
     if (lane == 0) {
@@ -226,21 +251,19 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       tma_load_3d(sQ + kHalf, &tmQ, q_full, 64, kh * p.GQ, q_start + i0, once);
     }
     const int32_t* table = p.block_tables + static_cast<size_t>(s) * p.MB;
-    auto entries = [&](int j) {  // lane l: block id of the tile's l-th attended block
-      const TileBlocks t = tile_blocks(j_lo + j, bs, kv_lo, p_max);
-      return lane <= t.hi - t.lo ? __ldg(table + t.lo + lane) : 0;
-    };
+    const int first_block = tile_blocks(j_lo, bs, kv_lo, p_max).lo;
+    TableWindow win_k, win_v;
+    win_k.init(table, p_max / bs + 1, first_block, lane);
+    win_v.init(table, p_max / bs + 1, first_block, lane);
     int k_next = 0, v_next = 0;
-    int pb_k = entries(0), pb_v = pb_k;  // entries of tiles k_next and v_next, fetched ahead
     uint32_t idle = 0;
     while (v_next < n) {
       int which = -1;
       if (lane == 0) {
-        if (k_next < n && (k_next < kRing || mbar_test_wait(k_empty0 + 8 * (k_next % kRing), ((k_next / kRing) - 1) & 1)))
-          which = 0;
-        else if (v_next < k_next &&
-                 (v_next < kRing || mbar_test_wait(v_empty0 + 8 * (v_next % kRing), ((v_next / kRing) - 1) & 1)))
+        if (v_next < k_next && (v_next < kRing || mbar_test_wait(v_empty0 + 8 * (v_next % kRing), ((v_next / kRing) - 1) & 1)))
           which = 1;
+        else if (k_next < n && (k_next < kRing || mbar_test_wait(k_empty0 + 8 * (k_next % kRing), ((k_next / kRing) - 1) & 1)))
+          which = 0;
       }
       which = __shfl_sync(0xffffffffu, which, 0);
       if (which < 0) {
@@ -253,9 +276,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       }
       idle = 0;
       const int j = which ? v_next : k_next;
-      int pb = which ? pb_v : pb_k;
       const TileBlocks cur = tile_blocks(j_lo + j, bs, kv_lo, p_max);
       const int nload = cur.hi - cur.lo + 1;
+      int pb = which ? win_v.get(cur.lo, nload, lane) : win_k.get(cur.lo, nload, lane);
       if (lane < nload && (pb < 0 || pb >= p.NB)) {
         if (which == 0) prefill_error(PA_DEVERR_TABLE);
         pb = 0;
@@ -271,13 +294,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         const uint32_t dst = (which ? sV(st) : sK(st)) + (lane & 1) * kHalf + row;
         tma_load_3d(dst, which ? &tmV : &tmK, full, (lane & 1) * 64, kh, b * bs, keep);
       }
-      if (which) {
-        ++v_next;
-        if (v_next < n) pb_v = entries(v_next);
-      } else {
-        ++k_next;
-        if (k_next < n) pb_k = entries(k_next);
-      }
+      if (which) ++v_next; else ++k_next;
     }
     if (lane == 0) {  // never leave with copies in flight
       mbar_wait_bounded(q_full, 0);
@@ -290,7 +307,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   } else if (warp == 1) {
     // ------------------------------------------------------------------- MMA issuer --
     // Polls without blocking; the value MMA goes first when both are ready, since the
-    // softmax warps wait on it.
+    // softmax warps wait on it and the next score MMA reuses its probabilities' columns.
     if (lane == 0) {
       int s_next = 0, o_next = 0;
       uint32_t idle = 0;
@@ -302,15 +319,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
           if (mbar_test_wait(p_full0 + 8 * b, (o_next / 2) & 1) &&
               mbar_test_wait(v_full0 + 8 * st, (o_next / kRing) & 1)) {
             tc_fence_after_sync();
-            const int pbuf = o_next % kPBuf;
 #pragma unroll
             for (int part = 0; part < (kSplit ? 2 : 1); ++part) {
 #pragma unroll
-              for (int kk = 0; kk < kKv / 16; ++kk) {  // O += P . V, 16 kv tokens per MMA
-                tc_mma_f16(tmem + kColO,
-                           smem_desc(sP(pbuf + part) + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024, kSwizzle128B),
-                           smem_desc(sV(st) + kk * 2048, kHalf, 1024, kSwizzle128B), kIdescO,
-                           o_next > 0 || part > 0 || kk > 0);
+              for (int kk = 0; kk < kKv / 16; ++kk) {  // O_h += P_h . V_h, 16 kv tokens per MMA
+                const int h = kk / 4;                    // softmax half owning these tokens
+                tc_mma_f16_ts(tmem + kColO + 128 * h, tmem + b * kKv + 64 * h + 32 * part + (kk % 4) * 8,
+                              smem_desc(sV(st) + kk * 2048, kHalf, 1024, kSwizzle128B), kIdescO,
+                              o_next > 0 || part > 0 || (kk % 4) > 0);
               }
             }
             tc_commit(o_full0 + 8 * b);
@@ -321,8 +337,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         }
         if (s_next < n) {
           const int st = s_next % kRing, b = s_next % 2;
-          if (mbar_test_wait(k_full0 + 8 * st, (s_next / kRing) & 1) &&
-              (s_next < 2 || mbar_test_wait(s_empty0 + 8 * b, ((s_next / 2) - 1) & 1))) {
+          // S(j) lands on P(j - 2): the value MMA that reads P(j - 2) must be issued first
+          // (MMAs of one thread run in order).
+          if (o_next >= s_next - 1 && mbar_test_wait(k_full0 + 8 * st, (s_next / kRing) & 1)) {
             tc_fence_after_sync();
 #pragma unroll
             for (int kk = 0; kk < kDim / 16; ++kk) {  // S[b] = Q . K^T, 16 dims per MMA
@@ -351,15 +368,15 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   } else {
     // ------------------------------------------------------------- softmax warps --
     // Warps 2..9.  A warp may only touch the TMEM lane quarter (warp % 4); the two warps of
-    // a quarter share its 32 query rows and split the columns: half 0 takes kv tokens
-    // 0..63 of a tile (and head dims 0..63 of O), half 1 the rest.  They combine row
-    // maxima every tile through spare TMEM columns of their own lanes (shared memory is
-    // all taken by the operands), with a 64-thread named barrier per quarter.
+    // a quarter share its 32 query rows and split each tile's kv tokens: half h takes
+    // tokens [64h, 64h + 64).  Each half runs its own online softmax (maximum, sum and
+    // output accumulator O_h), so the halves never wait for each other within the loop;
+    // they are combined once at the end.
     const int q4 = warp & 3;
     const int half = (warp - 2) >> 2;
     const int r = 32 * q4 + lane;  // query row = TMEM lane
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q4) << 16;
-    const uint32_t pair_bar = 1 + q4;
+    const uint32_t o_col = tmem + lane_addr + kColO + 128 * half;
     const int tl = r >> p.gq_shift, g = r & (p.GQ - 1);
     const bool row_valid = tl < ntok;
     const int pos = p_min + tl;
@@ -369,68 +386,58 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     auto wait_pv = [&](int t) {
       return __all_sync(0xffffffffu, wait_or_abort(o_full0 + 8 * (t % 2), (t / 2) & 1, abort));
     };
-    // The two warps of a quarter meet at a named barrier every tile, so neither may leave
-    // the loop early: after an abort a warp keeps stepping through the barriers with `ok`
-    // false and does no other work.
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
+    for (int j = 0; j < n && ok; ++j) {
       const int b = j % 2, st = j % kRing;
-      ok = ok && __all_sync(0xffffffffu, wait_or_abort(s_full0 + 8 * b, (j / 2) & 1, abort));
+      if (!__all_sync(0xffffffffu, wait_or_abort(s_full0 + 8 * b, (j / 2) & 1, abort))) {
+        ok = false;
+        break;
+      }
       const int kv0 = (j_lo + j) * kKv;
       const int c0 = 64 * half;  // this warp's first column
+      const uint32_t s_col = tmem + lane_addr + b * kKv + c0;
       float sc[64];
-      float mraw = -INFINITY;
-      if (ok) {
-        tc_fence_after_sync();
-        tmem_load64(tmem + lane_addr + b * kKv + c0, sc);
-        tc_fence_before_sync();
-        mbar_arrive(s_empty0 + 8 * b);
-        // Interior tiles (every row attends every column) skip the mask.
-        const bool interior =
-            ntok == p.tq && kv0 + kKv - 1 <= p_min && (p.window <= 0 || kv0 >= p_max - p.window + 1);
-        if (!interior) {
-          const int c_lo = lo_row - kv0 - c0, c_hi = row_valid ? pos - kv0 - c0 : -1;
-#pragma unroll
-          for (int c = 0; c < 64; ++c) sc[c] = (c >= c_lo && c <= c_hi) ? sc[c] : -INFINITY;
-        }
-        float mx[8];  // eight independent chains instead of one 64-long one
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = sc[k];
-#pragma unroll
-        for (int c = 8; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], sc[c]);
-        mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      }
-      tmem_store1(tmem + lane_addr + kColX + 2 * b + half, mraw);
-      tc_fence_before_sync();
-      named_barrier_sync(pair_bar, 64);
       tc_fence_after_sync();
-      mraw = fmaxf(mraw, tmem_load1(tmem + lane_addr + kColX + 2 * b + (half ^ 1)));
-      if (!ok) continue;
+      tmem_load64(s_col, sc);
+      // Interior tiles (every row attends every column) skip the mask.
+      const bool interior =
+          ntok == p.tq && kv0 + kKv - 1 <= p_min && (p.window <= 0 || kv0 >= p_max - p.window + 1);
+      if (!interior) {
+        const int c_lo = lo_row - kv0 - c0, c_hi = row_valid ? pos - kv0 - c0 : -1;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) sc[c] = (c >= c_lo && c <= c_hi) ? sc[c] : -INFINITY;
+      }
+      float mx[8];  // eight independent chains instead of one 64-long one
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx[k] = sc[k];
+#pragma unroll
+      for (int c = 8; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], sc[c]);
+      const float mraw =
+          fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float mt = mraw * p.qscale;  // scores in base-2 units (qscale > 0 keeps the order)
       float alpha = 1.f;
       bool rescale = false;
       if (mt > m_run + kRescaleThreshold) {  // move the reference maximum
         alpha = ex2_ftz(m_run - mt);
-        rescale = l > 0.f;                   // O holds earlier contributions of this row
+        rescale = l > 0.f;                   // O_h holds earlier contributions of this row
         l *= alpha;
         m_run = mt;
       }
-      // O may be rescaled only after the previous value MMA; the probability buffer of
-      // tile j is free once the value MMA that last read it (tile j - kPBuf) is done.
-      const bool any_rescale = __any_sync(0xffffffffu, rescale);
-      if (any_rescale && !wait_pv(j - 1)) ok = false;
-      if (ok && !any_rescale && j >= kPBuf && !wait_pv(j - kPBuf)) ok = false;
-      if (!ok) continue;
-      if (any_rescale) {
+      // O_h may be rescaled only after the previous value MMA.
+      if (__any_sync(0xffffffffu, rescale)) {
+        if (!wait_pv(j - 1)) {
+          ok = false;
+          break;
+        }
         tc_fence_after_sync();
         const float a = rescale ? alpha : 1.f;
 #pragma unroll
-        for (int c4 = 0; c4 < 2; ++c4) {  // this warp's 64 columns of O
+        for (int c4 = 0; c4 < 4; ++c4) {
           float o[32];
-          tmem_load32(tmem + lane_addr + kColO + 64 * half + 32 * c4, o);
+          tmem_load32(o_col + 32 * c4, o);
 #pragma unroll
           for (int k = 0; k < 32; ++k) o[k] *= a;
-          tmem_store32(tmem + lane_addr + kColO + 64 * half + 32 * c4, o);
+          tmem_store32(o_col + 32 * c4, o);
         }
       }
       // V rows of tokens outside the loaded blocks or past the context may hold anything
@@ -441,64 +448,73 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       if (clean_lo > 0 || clean_hi < kKv) {
         if (!__all_sync(0xffffffffu, wait_or_abort(v_full0 + 8 * st, (j / kRing) & 1, abort))) {
           ok = false;
-          continue;
+          break;
         }
         if (r < clean_lo || r >= clean_hi) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) st_shared_v4(sV(st) + half * kHalf + r * 128 + 16 * k, 0, 0, 0, 0);
         }
       }
-      // Probabilities, written as row r of this warp's 64-token half of the K-major,
-      // 128-byte-swizzled A operand.  exp2(s * qscale - m) is one FFMA and one MUFU op;
-      // two weights are rounded and packed by one conversion.
+      // Probabilities of this half's 64 tokens, written over its own score columns as the
+      // A operand of the value MMA.  exp2(s * qscale - m) is one FFMA and one MUFU op; two
+      // weights are rounded and packed by one conversion.  The denominator sums the
+      // unrounded weights (fp16 rounding errors of the packed weights average out).
       float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       const float neg_m = -m_run;
-      const uint32_t pdst = sP(kSplit ? 0 : j % kPBuf) + half * kHalf + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t w_hi[4], w_lo[4];
+      for (int q = 0; q < 2; ++q) {  // two stores of 16 columns (32 tokens) each
+        uint32_t w_hi[16], w_lo[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int k = 8 * c + 2 * e;
-          const float x0 = ex2_ftz(fmaf(sc[k], p.qscale, neg_m));
-          const float x1 = ex2_ftz(fmaf(sc[k + 1], p.qscale, neg_m));
+        for (int k = 0; k < 16; ++k) {
+          const int c = 32 * q + 2 * k;
+          const float x0 = ex2_ftz(fmaf(sc[c], p.qscale, neg_m));
+          const float x1 = ex2_ftz(fmaf(sc[c + 1], p.qscale, neg_m));
           const Pair<IO> hi(x0, x1);
-          w_hi[e] = hi.bits;
-          if (kSplit) {
-            w_lo[e] = Pair<IO>(x0 - hi.lo_f(), x1 - hi.hi_f()).bits;
-            ls[(c & 1) * 4 + e] += x0 + x1;
-          } else {
-            ls[(c & 1) * 4 + e] += hi.lo_f() + hi.hi_f();  // the rounded weights the MMA uses
-          }
+          w_hi[k] = hi.bits;
+          if (kSplit) w_lo[k] = Pair<IO>(x0 - hi.lo_f(), x1 - hi.hi_f()).bits;
+          ls[k & 7] += x0 + x1;
         }
-        const uint32_t addr = pdst + ((c ^ (r & 7)) << 4);
-        st_shared_v4(addr, w_hi[0], w_hi[1], w_hi[2], w_hi[3]);
-        if (kSplit) st_shared_v4(addr + kOpBytes, w_lo[0], w_lo[1], w_lo[2], w_lo[3]);
+        tmem_store16_bits(s_col + 16 * q, w_hi);
+        if (kSplit) tmem_store16_bits(s_col + 32 + 16 * q, w_lo);
       }
+      tmem_wait_store();
       l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-      fence_proxy_async_shared();
+      fence_proxy_async_shared();  // zeroed V rows (if any) are read by the tensor core
       tc_fence_before_sync();
       mbar_arrive(p_full0 + 8 * b);
     }
-    // Softmax denominators: the two halves of a row add their partial sums.
-    tmem_store1(tmem + lane_addr + kColX + 4 + half, l);
-    tc_fence_before_sync();
-    named_barrier_sync(pair_bar, 64);
+    // Combine the halves: both must reach this barrier (neither returns early).  The S
+    // buffers are free once the last value MMA is done, so (m, l) travel through them.
+    const bool fin = ok && wait_pv(n - 1);
     tc_fence_after_sync();
-    l += tmem_load1(tmem + lane_addr + kColX + 4 + (half ^ 1));
-    if (ok && wait_pv(n - 1)) {
-      tc_fence_after_sync();
-      const float inv = row_valid ? 1.f / l : 0.f;
+    tmem_store1(tmem + lane_addr + 2 * half, m_run);
+    tmem_store1(tmem + lane_addr + 2 * half + 1, l);
+    tc_fence_before_sync();
+    named_barrier_sync(1 + q4, 64);
+    tc_fence_after_sync();
+    const float m_o = tmem_load1(tmem + lane_addr + 2 * (half ^ 1));
+    const float l_o = tmem_load1(tmem + lane_addr + 2 * (half ^ 1) + 1);
+    if (fin) {
+      const float m_all = fmaxf(m_run, m_o);
+      const float a_me = ex2_ftz(m_run - m_all), a_o = ex2_ftz(m_o - m_all);
+      const float l_all = l * a_me + l_o * a_o;
+      const float inv = row_valid ? 1.f / l_all : 0.f;
+      // this warp writes head dims [64 half, 64 half + 64): O_0 and O_1 there, weighted
+      const float w0 = (half == 0 ? a_me : a_o) * inv, w1 = (half == 0 ? a_o : a_me) * inv;
       IO* orow = reinterpret_cast<IO*>(p.out) +
                  (static_cast<size_t>(q_start + i0 + tl) * p.Hq + static_cast<size_t>(kh) * p.GQ + g) * kDim + 64 * half;
-      float o[64];
-      tmem_load64(tmem + lane_addr + kColO + 64 * half, o);
+      float o0[64], o1[64];
+      tmem_load64(tmem + lane_addr + kColO + 64 * half, o0);
+      tmem_load64(tmem + lane_addr + kColO + 128 + 64 * half, o1);
       if (row_valid) {
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
           uint32_t w[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) w[e] = Pair<IO>(o[8 * v + 2 * e] * inv, o[8 * v + 2 * e + 1] * inv).bits;
+          for (int e = 0; e < 4; ++e) {
+            const int c = 8 * v + 2 * e;
+            w[e] = Pair<IO>(o0[c] * w0 + o1[c] * w1, o0[c + 1] * w0 + o1[c + 1] * w1).bits;
+          }
           *reinterpret_cast<uint4*>(orow + 8 * v) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
@@ -608,7 +624,7 @@ extern "C" pa_status paged_attention_prefill(void* out, const void* q, const voi
   const bool bf16 = dtype == PA_BF16;
   const void* fn = bf16 ? reinterpret_cast<const void*>(&prefill_tc_kernel<__nv_bfloat16>)
                         : reinterpret_cast<const void*>(&prefill_tc_kernel<__half>);
-  const size_t smem = bf16 ? smem_bytes<true>() : smem_bytes<false>();
+  const size_t smem = kSmemBytes;
   static std::once_flag once[2];
   cudaError_t attr_err = cudaSuccess;
   std::call_once(once[bf16 ? 1 : 0], [&] {
