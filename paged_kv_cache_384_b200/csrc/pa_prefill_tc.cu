@@ -58,7 +58,7 @@ constexpr int kHalf = 128 * 128;          // one 64-element half of a 128-row op
 constexpr int kOpBytes = 2 * kHalf;       // a whole 128 x 128 operand (Q, K, V or P)
 constexpr int kRing = 3;                  // depth of the K ring and of the V ring
 constexpr int kSoftmaxThreads = 256;   // 8 warps: two per TMEM lane quarter, 64 columns each
-constexpr int kThreads = 64 + kSoftmaxThreads;
+constexpr int kThreads = 96 + kSoftmaxThreads;  // + K producer, MMA issuer, V producer
 constexpr uint32_t kTmemCols = 512;       // S0 [0,128)  S1 [128,256)  O_0 [256,384)  O_1 [384,512)
 // Each softmax half h owns the 64 score columns [64h, 64h+64) of an S buffer and writes its
 // probabilities over them: hi weights in the first 32 columns (two 16-bit weights per
@@ -235,73 +235,53 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   tc_fence_after_sync();
   const uint32_t tmem = sh.tmem_base;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer --
-    // Polls both rings and issues whichever load has a free slot: V of the oldest tile
-    // whose K is out first (the value MMA is on the softmax warps' path), else the next K.
-    // K and V each walk the block table through their own prefetched windows.
+  if (warp == 0 || warp == 10) {
+    // ------------------------------------------------------------------ TMA producers --
+    // Warp 0 loads the q rows and then K, warp 10 loads V, each into its own ring and each
+    // walking the block table through its own prefetched window, so neither tensor's
+    // copies wait behind the other's.  One copy is one 64-dim half of one block.
+    const bool is_v = warp == 10;
     const uint64_t keep = l2_policy_evict_last();    // K/V tiles are shared by the sequence's q tiles
-    const uint64_t once = l2_policy_evict_first();   // q rows are read once
-    if (lane == 0) {
+    if (!is_v && lane == 0) {
       prefetch_tensormap(&tmK);
-      prefetch_tensormap(&tmV);
       prefetch_tensormap(&tmQ);
       mbar_arrive_expect_tx(q_full, kOpBytes);
+      const uint64_t once = l2_policy_evict_first();  // q rows are read once
       tma_load_3d(sQ, &tmQ, q_full, 0, kh * p.GQ, q_start + i0, once);
       tma_load_3d(sQ + kHalf, &tmQ, q_full, 64, kh * p.GQ, q_start + i0, once);
     }
+    if (is_v && lane == 0) prefetch_tensormap(&tmV);
+    const CUtensorMap* map = is_v ? &tmV : &tmK;
+    const uint32_t full0 = is_v ? v_full0 : k_full0, empty0 = is_v ? v_empty0 : k_empty0;
     const int32_t* table = p.block_tables + static_cast<size_t>(s) * p.MB;
-    const int first_block = tile_blocks(j_lo, bs, kv_lo, p_max).lo;
-    TableWindow win_k, win_v;
-    win_k.init(table, p_max / bs + 1, first_block, lane);
-    win_v.init(table, p_max / bs + 1, first_block, lane);
-    int k_next = 0, v_next = 0;
-    uint32_t idle = 0;
-    while (v_next < n) {
-      int which = -1;
-      if (lane == 0) {
-        if (v_next < k_next && (v_next < kRing || mbar_test_wait(v_empty0 + 8 * (v_next % kRing), ((v_next / kRing) - 1) & 1)))
-          which = 1;
-        else if (k_next < n && (k_next < kRing || mbar_test_wait(k_empty0 + 8 * (k_next % kRing), ((k_next / kRing) - 1) & 1)))
-          which = 0;
-      }
-      which = __shfl_sync(0xffffffffu, which, 0);
-      if (which < 0) {
-        if (*abort || ++idle > 4 * kWaitLimit) {
-          if (!*abort) prefill_error(PA_DEVERR_TIMEOUT);
-          *abort = 1;
-          break;
-        }
-        continue;
-      }
-      idle = 0;
-      const int j = which ? v_next : k_next;
-      const TileBlocks cur = tile_blocks(j_lo + j, bs, kv_lo, p_max);
+    TableWindow win;
+    win.init(table, p_max / bs + 1, tile_blocks(j_lo, bs, kv_lo, p_max).lo, lane);
+    int next = 0;
+    for (; next < n; ++next) {
+      const int st = next % kRing;
+      bool ok = true;
+      if (lane == 0 && next >= kRing) ok = wait_or_abort(empty0 + 8 * st, ((next / kRing) - 1) & 1, abort);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      const TileBlocks cur = tile_blocks(j_lo + next, bs, kv_lo, p_max);
       const int nload = cur.hi - cur.lo + 1;
-      int pb = which ? win_v.get(cur.lo, nload, lane) : win_k.get(cur.lo, nload, lane);
+      int pb = win.get(cur.lo, nload, lane);
       if (lane < nload && (pb < 0 || pb >= p.NB)) {
-        if (which == 0) prefill_error(PA_DEVERR_TABLE);
+        if (!is_v) prefill_error(PA_DEVERR_TABLE);
         pb = 0;
       }
-      const int st = j % kRing;
-      const uint32_t full = (which ? v_full0 : k_full0) + 8 * st;
-      if (lane == 0) mbar_arrive_expect_tx(full, static_cast<uint32_t>(nload) * 2u * bs * 128u);
+      if (lane == 0) mbar_arrive_expect_tx(full0 + 8 * st, static_cast<uint32_t>(nload) * 2u * bs * 128u);
       __syncwarp();
-      // each copy is one 64-dim half of one block, one copy per lane (2 * nload <= 32)
       const int b = __shfl_sync(0xffffffffu, pb, (lane >> 1) & 31);
-      if (lane < 2 * nload) {
+      if (lane < 2 * nload) {  // 2 * nload <= 32 copies, one per lane
         const uint32_t row = static_cast<uint32_t>(cur.lo + (lane >> 1) - cur.first) * bs * 128u;
-        const uint32_t dst = (which ? sV(st) : sK(st)) + (lane & 1) * kHalf + row;
-        tma_load_3d(dst, which ? &tmV : &tmK, full, (lane & 1) * 64, kh, b * bs, keep);
+        const uint32_t dst = (is_v ? sV(st) : sK(st)) + (lane & 1) * kHalf + row;
+        tma_load_3d(dst, map, full0 + 8 * st, (lane & 1) * 64, kh, b * bs, keep);
       }
-      if (which) ++v_next; else ++k_next;
     }
     if (lane == 0) {  // never leave with copies in flight
-      mbar_wait_bounded(q_full, 0);
-      for (int k = k_next - kRing < 0 ? 0 : k_next - kRing; k < k_next; ++k)
-        mbar_wait_bounded(k_full0 + 8 * (k % kRing), (k / kRing) & 1);
-      for (int k = v_next - kRing < 0 ? 0 : v_next - kRing; k < v_next; ++k)
-        mbar_wait_bounded(v_full0 + 8 * (k % kRing), (k / kRing) & 1);
+      if (!is_v) mbar_wait_bounded(q_full, 0);
+      for (int k = next - kRing < 0 ? 0 : next - kRing; k < next; ++k)
+        mbar_wait_bounded(full0 + 8 * (k % kRing), (k / kRing) & 1);
     }
     __syncwarp();
   } else if (warp == 1) {
