@@ -14,10 +14,11 @@
 // "vLLM source first look: PagedAttention memory design" (trdm.cn), section 三); the
 // grouped-query tile is this library's design.
 //
-// Roles (one CTA per SM, 6 warps):
-//   warp 0      TMA producer: per tile, the q rows of the head group and, block by block,
-//               the 64-dim halves of each attended K and V block (128-byte swizzle) into a
-//               3-stage ring; block-table entries are loaded by the warp's lanes in parallel.
+// Roles (one CTA per SM, 9 warps):
+//   warps 0,6-8 TMA producers, one per part of a tile (K or V, 64-dim half, 128-byte
+//               swizzle): each issues its part of every attended block into a 3-stage ring
+//               (warp 0 also the q rows of the head group); block-table entries are loaded
+//               by the lanes in parallel.
 //   warp 1      TMEM owner and MMA issuer (one lane): polls for ready work and issues the score
 //               MMA of the next landed tile or the value MMA of the oldest softmaxed tile,
 //               whichever is ready, so stages are released without waiting on later tiles.
@@ -47,7 +48,7 @@ constexpr int kStageBytes = 4 * kHalf + 2 * kQHalf;  // K lo, K hi, V lo, V hi, 
 constexpr int kStages = 3;
 constexpr int kPBytes = kTokens * kHeadsN * 2;  // one probability operand, 128 tokens x 16 heads
 constexpr int kPBuffers = 4;                    // 2 tiles in flight x (hi, lo) parts
-constexpr int kThreads = 192;
+constexpr int kThreads = 288;  // TMA warps 0 and 6..8, MMA warp 1, softmax warps 2..5
 constexpr uint32_t kTmemCols = 64;              // S0 [0,16)  S1 [16,32)  O0 [32,48)  O1 [48,64)
 constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + kPBuffers * kPBytes;
 
@@ -123,7 +124,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < kStages; ++st) {
-      mbar_init(full0 + 8 * st, 1);
+      mbar_init(full0 + 8 * st, 4);  // one arrival per TMA warp
       mbar_init(empty0 + 8 * st, 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -149,13 +150,17 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
   tc_fence_after_sync();
   const uint32_t tmem = sh.tmem_base;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer --
+  if (warp == 0 || warp >= 6) {
+    // ------------------------------------------------------------------ TMA producers --
+    // Four warps, one per (K or V) x (64-dim half) part of a tile: a warp issues its copies
+    // one after another, so four warps issue a tile four times as fast as one.  Warp 0
+    // also loads the q rows.  Every warp walks the same tile stream and block table.
+    const int part = warp == 0 ? 0 : warp - 5;  // 0: K lo, 1: K hi, 2: V lo, 3: V hi
+    const CUtensorMap* map = part < 2 ? &tmK : &tmV;
     const uint64_t policy = l2_policy_evict_first();
     if (lane == 0) {
-      prefetch_tensormap(&tmK);
-      prefetch_tensormap(&tmV);
-      prefetch_tensormap(&tmQ);
+      prefetch_tensormap(map);
+      if (part == 0) prefetch_tensormap(&tmQ);
     }
     const int bs = p.bs;
     const int bpt = kTokens / bs;  // blocks per tile
@@ -193,7 +198,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       }
       int pb = __shfl_sync(0xffffffffu, win, (lb_lo - win_base + lane) & 31);
       if (lane < nload && (pb < 0 || pb >= p.NB)) {
-        decode_error(PA_DEVERR_TABLE);
+        if (part == 0) decode_error(PA_DEVERR_TABLE);
         pb = 0;
       }
       bool ok = true;
@@ -201,26 +206,20 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         if (issued >= kStages) ok = wait_or_abort(empty0 + 8 * st, ((issued / kStages) - 1) & 1, abort);
         if (ok) {
           const uint32_t bar = full0 + 8 * st;
-          mbar_arrive_expect_tx(bar, 2u * GQ * 128u + static_cast<uint32_t>(nload) * 4u * bs * 128u);
-          const uint32_t sb = stage(st);
-          const int qrow = c.s * p.Hq + c.g * GQ;
-          tma_load_2d(sb + 4 * kHalf, &tmQ, bar, 0, qrow, policy);
-          tma_load_2d(sb + 4 * kHalf + kQHalf, &tmQ, bar, 64, qrow, policy);
+          mbar_arrive_expect_tx(bar, (part == 0 ? 2u * GQ * 128u : 0u) + static_cast<uint32_t>(nload) * bs * 128u);
+          if (part == 0) {
+            const uint32_t sb = stage(st);
+            const int qrow = c.s * p.Hq + c.g * GQ;
+            tma_load_2d(sb + 4 * kHalf, &tmQ, bar, 0, qrow, policy);
+            tma_load_2d(sb + 4 * kHalf + kQHalf, &tmQ, bar, 64, qrow, policy);
+          }
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);  // also orders lane 0's expect_tx before any copy
       if (!ok) break;
-      // The tile's copies (4 per block: K and V, two 64-dim halves each) are issued by the
-      // warp's lanes together, one copy per lane, rather than one after another.
-      for (int base_copy = 0; base_copy < 4 * nload; base_copy += 32) {
-        const int cp = base_copy + lane;
-        const int b = __shfl_sync(0xffffffffu, pb, (cp >> 2) & 31);
-        if (cp < 4 * nload) {
-          const int part = cp & 3;  // 0: K lo, 1: K hi, 2: V lo, 3: V hi
-          const uint32_t row = static_cast<uint32_t>(lb_lo + (cp >> 2) - lb_first) * bs * 128u;
-          tma_load_3d(stage(st) + part * kHalf + row, part < 2 ? &tmK : &tmV, full0 + 8 * st, (part & 1) * 64, c.g,
-                      b * bs, policy);
-        }
+      if (lane < nload) {  // this warp's part of each attended block, one copy per lane
+        const uint32_t row = static_cast<uint32_t>(lb_lo + lane - lb_first) * bs * 128u;
+        tma_load_3d(stage(st) + part * kHalf + row, map, full0 + 8 * st, (part & 1) * 64, c.g, pb * bs, policy);
       }
       advance(c, p);
     }
@@ -288,6 +287,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     __syncwarp();
   } else {
     // ------------------------------------------------- softmax + accumulation warps --
+    // (warps 2..5)
     const int q4 = warp & 3;              // TMEM lane quarter this warp may access
     const int r = 32 * q4 + lane;         // token row (softmax) and head-dim row (accumulate)
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q4) << 16;
