@@ -75,17 +75,20 @@ struct PrefillParams {
   const int32_t* cu_q;
   const int32_t* context_lens;
   int S, T, Hq, Hkv, GQ, gq_shift, tq, bs, MB, NB, window, max_q_len;
+  int qtiles;    // query tiles of the longest sequence: ceil(max_q_len / tq)
+  int units;     // S * Hkv * qtiles work units, walked by a persistent grid
   float qscale;  // scale * log2(e)
 };
 
 struct PfShared {
-  uint64_t q_full;
+  uint64_t q_full, q_empty, o_free;  // q rows landed / read by the last score MMA; O read out
   uint64_t k_full[kRing], k_empty[kRing], v_full[kRing], v_empty[kRing];
   uint64_t s_full[2];
   uint64_t p_full[2], o_full[2];  // by tile parity: probabilities written / value MMA done
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
+  float xch[2][kRows];  // the two softmax halves of a row combine (m, l) through here
 };
 
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort) {
@@ -135,6 +138,44 @@ __device__ __forceinline__ TileBlocks tile_blocks(int jt, int bs, int kv_lo, int
   return t;
 }
 
+// One unit of work: 128 query rows (query tile qt of sequence s, cached head kh).  Units
+// are numbered with the query tile fastest (heaviest first), so the CTAs working at the
+// same time share the K/V tiles of a few (sequence, head) pairs in L2.  The persistent
+// grid deals them out in rounds of gridDim.x, in alternate directions (CTA c takes the
+// c-th unit of even rounds and the c-th from the end of odd ones), which evens out the
+// causal tiles' unequal costs.
+__device__ __forceinline__ int unit_of(int k) {  // k-th unit of this CTA
+  const int G = gridDim.x;
+  return k * G + ((k & 1) ? G - 1 - static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x));
+}
+struct Unit {
+  int s, kh, q_start, i0, ntok, ctx, p_min, p_max, kv_lo, j_lo, n;
+};
+__device__ __forceinline__ bool unit_at(const PrefillParams& p, int u, Unit* w) {
+  const int qt = p.qtiles - 1 - u % p.qtiles;
+  const int g = u / p.qtiles;
+  w->kh = g % p.Hkv;
+  w->s = g / p.Hkv;
+  const int q_start = __ldg(p.cu_q + w->s);
+  const int q_len = __ldg(p.cu_q + w->s + 1) - q_start;
+  const int ctx = __ldg(p.context_lens + w->s);
+  if (q_start < 0 || q_len < 0 || q_start + q_len > p.T || q_len > ctx || ctx > p.MB * p.bs || q_len > p.max_q_len) {
+    if (threadIdx.x == 0) prefill_error(PA_DEVERR_CONTEXT);
+    return false;
+  }
+  w->i0 = qt * p.tq;
+  if (w->i0 >= q_len) return false;
+  w->q_start = q_start;
+  w->ctx = ctx;
+  w->ntok = min(p.tq, q_len - w->i0);
+  w->p_min = ctx - q_len + w->i0;  // positions of the unit's first and last query
+  w->p_max = w->p_min + w->ntok - 1;
+  w->kv_lo = p.window > 0 ? max(0, w->p_min - p.window + 1) : 0;
+  w->j_lo = w->kv_lo / kKv;
+  w->n = w->p_max / kKv - w->j_lo + 1;  // KV tiles
+  return true;
+}
+
 // Block-table entries of one sequence, 32 at a time, one per lane: the window in use and
 // the next one, whose load is in flight while the current one serves.
 struct TableWindow {
@@ -180,31 +221,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 
   grid_dependency_launch_next();
   grid_dependency_wait();
-
-  // ---- this CTA's work: query tile qt (heaviest first) of sequence s, cached head kh ----
-  const int s = blockIdx.z, kh = blockIdx.y;
-  const int qt = static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x);
-  const int q_start = __ldg(p.cu_q + s);
-  const int q_len = __ldg(p.cu_q + s + 1) - q_start;
-  const int ctx = __ldg(p.context_lens + s);
-  if (q_start < 0 || q_len < 0 || q_start + q_len > p.T || q_len > ctx || ctx > p.MB * p.bs || q_len > p.max_q_len) {
-    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) prefill_error(PA_DEVERR_CONTEXT);
-    return;
-  }
-  const int i0 = qt * p.tq;
-  if (i0 >= q_len) return;
-  const int ntok = min(p.tq, q_len - i0);
-  const int p_min = ctx - q_len + i0, p_max = p_min + ntok - 1;  // positions of the first / last query
-  const int kv_lo = p.window > 0 ? max(0, p_min - p.window + 1) : 0;
-  const int j_lo = kv_lo / kKv;
-  const int n = p_max / kKv - j_lo + 1;  // KV tiles
   const int bs = p.bs;
 
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;  // swizzle atoms are 1024-B aligned
   const uint32_t sQ = base;
   auto sK = [&](int st) { return base + kOpBytes + st * kOpBytes; };
   auto sV = [&](int st) { return base + (1 + kRing) * kOpBytes + st * kOpBytes; };
-  const uint32_t q_full = smem_u32(&sh.q_full);
+  const uint32_t q_full = smem_u32(&sh.q_full), q_empty = smem_u32(&sh.q_empty), o_free = smem_u32(&sh.o_free);
   const uint32_t k_full0 = smem_u32(&sh.k_full[0]), k_empty0 = smem_u32(&sh.k_empty[0]);
   const uint32_t v_full0 = smem_u32(&sh.v_full[0]), v_empty0 = smem_u32(&sh.v_empty[0]);
   const uint32_t s_full0 = smem_u32(&sh.s_full[0]);
@@ -214,6 +237,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    mbar_init(o_free, kSoftmaxThreads);
     for (int st = 0; st < kRing; ++st) {
       mbar_init(k_full0 + 8 * st, 2);  // one arrival per producer warp of the tensor
       mbar_init(k_empty0 + 8 * st, 1);
@@ -235,70 +260,111 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   tc_fence_after_sync();
   const uint32_t tmem = sh.tmem_base;
 
+  // Every role walks the same units in the same order; tile counters (ring slots and
+  // barrier parities) and unit counters run on across units.
   if (warp == 0 || warp >= 10) {
     // ------------------------------------------------------------------ TMA producers --
     // Four warps: (K, V) x (64-dim half).  A warp issues its copies one per lane, and a
     // warp's copies go out one after another, so splitting them over four warps issues a
-    // tile four times as fast.  Warp 0 also loads the q rows.  Each warp walks the block
-    // table through its own prefetched window.
-    const int pi = warp == 0 ? 0 : warp - 9;  // 0..3
+    // tile four times as fast.  The V-hi warp also loads each unit's q rows once the last
+    // score MMA of the previous unit has read them.  Each warp walks the block table
+    // through its own prefetched window.
+    const int pi = warp == 0 ? 0 : warp - 9;  // 0: K lo, 1: V lo, 2: K hi, 3: V hi
     const bool is_v = pi & 1;
     const int dh = pi >> 1;                   // 64-dim half this warp copies
     const uint64_t keep = l2_policy_evict_last();    // K/V tiles are shared by the sequence's q tiles
-    if (pi == 0 && lane == 0) {
-      prefetch_tensormap(&tmQ);
-      mbar_arrive_expect_tx(q_full, kOpBytes);
-      const uint64_t once = l2_policy_evict_first();  // q rows are read once
-      tma_load_3d(sQ, &tmQ, q_full, 0, kh * p.GQ, q_start + i0, once);
-      tma_load_3d(sQ + kHalf, &tmQ, q_full, 64, kh * p.GQ, q_start + i0, once);
-    }
+    const uint64_t once = l2_policy_evict_first();   // q rows are read once
     const CUtensorMap* map = is_v ? &tmV : &tmK;
-    if (lane == 0) prefetch_tensormap(map);
+    if (lane == 0) {
+      prefetch_tensormap(map);
+      if (pi == 3) prefetch_tensormap(&tmQ);
+    }
     const uint32_t full0 = is_v ? v_full0 : k_full0, empty0 = is_v ? v_empty0 : k_empty0;
-    const int32_t* table = p.block_tables + static_cast<size_t>(s) * p.MB;
-    TableWindow win;
-    win.init(table, p_max / bs + 1, tile_blocks(j_lo, bs, kv_lo, p_max).lo, lane);
-    int next = 0;
-    for (; next < n; ++next) {
-      const int st = next % kRing;
-      bool ok = true;
-      if (lane == 0 && next >= kRing) ok = wait_or_abort(empty0 + 8 * st, ((next / kRing) - 1) & 1, abort);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      const TileBlocks cur = tile_blocks(j_lo + next, bs, kv_lo, p_max);
-      const int nload = cur.hi - cur.lo + 1;
-      int pb = win.get(cur.lo, nload, lane);
-      if (lane < nload && (pb < 0 || pb >= p.NB)) {
-        if (pi == 0) prefill_error(PA_DEVERR_TABLE);
-        pb = 0;
+    int gt = 0, uq = 0;
+    bool ok = true;
+    for (int k = 0, u = unit_of(0); u < p.units && ok; u = unit_of(++k)) {
+      Unit w;
+      if (!unit_at(p, u, &w)) continue;
+      if (pi == 3) {
+        if (lane == 0) {
+          ok = uq == 0 || wait_or_abort(q_empty, (uq - 1) & 1, abort);
+          if (ok) {
+            mbar_arrive_expect_tx(q_full, kOpBytes);
+            tma_load_3d(sQ, &tmQ, q_full, 0, w.kh * p.GQ, w.q_start + w.i0, once);
+            tma_load_3d(sQ + kHalf, &tmQ, q_full, 64, w.kh * p.GQ, w.q_start + w.i0, once);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
       }
-      if (lane == 0) mbar_arrive_expect_tx(full0 + 8 * st, static_cast<uint32_t>(nload) * bs * 128u);
-      __syncwarp();
-      if (lane < nload) {  // nload <= 16 copies, one per lane
-        const uint32_t row = static_cast<uint32_t>(cur.lo + lane - cur.first) * bs * 128u;
-        const uint32_t dst = (is_v ? sV(st) : sK(st)) + dh * kHalf + row;
-        tma_load_3d(dst, map, full0 + 8 * st, dh * 64, kh, pb * bs, keep);
+      TableWindow win;
+      win.init(p.block_tables + static_cast<size_t>(w.s) * p.MB, w.p_max / bs + 1,
+               tile_blocks(w.j_lo, bs, w.kv_lo, w.p_max).lo, lane);
+      for (int j = 0; j < w.n; ++j, ++gt) {
+        const int st = gt % kRing;
+        bool ready = true;
+        if (lane == 0 && gt >= kRing) ready = wait_or_abort(empty0 + 8 * st, ((gt / kRing) - 1) & 1, abort);
+        if (!__shfl_sync(0xffffffffu, ready, 0)) {
+          ok = false;
+          break;
+        }
+        const TileBlocks cur = tile_blocks(w.j_lo + j, bs, w.kv_lo, w.p_max);
+        const int nload = cur.hi - cur.lo + 1;
+        int pb = win.get(cur.lo, nload, lane);
+        if (lane < nload && (pb < 0 || pb >= p.NB)) {
+          if (pi == 0) prefill_error(PA_DEVERR_TABLE);
+          pb = 0;
+        }
+        if (lane == 0) mbar_arrive_expect_tx(full0 + 8 * st, static_cast<uint32_t>(nload) * bs * 128u);
+        __syncwarp();
+        if (lane < nload) {  // nload <= 16 copies, one per lane
+          const uint32_t row = static_cast<uint32_t>(cur.lo + lane - cur.first) * bs * 128u;
+          const uint32_t dst = (is_v ? sV(st) : sK(st)) + dh * kHalf + row;
+          tma_load_3d(dst, map, full0 + 8 * st, dh * 64, w.kh, pb * bs, keep);
+        }
       }
+      ++uq;
     }
     if (lane == 0) {  // never leave with copies in flight
-      if (pi == 0) mbar_wait_bounded(q_full, 0);
-      for (int k = next - kRing < 0 ? 0 : next - kRing; k < next; ++k)
+      if (pi == 3 && uq > 0) mbar_wait_bounded(q_full, (uq - 1) & 1);
+      for (int k = gt - kRing < 0 ? 0 : gt - kRing; k < gt; ++k)
         mbar_wait_bounded(full0 + 8 * (k % kRing), (k / kRing) & 1);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------- MMA issuer --
-    // Polls without blocking; the value MMA goes first when both are ready, since the
-    // softmax warps wait on it and the next score MMA reuses its probabilities' columns.
+    // Polls without blocking.  Score MMAs run ahead through the unit list (the next
+    // unit's first scores overlap the current unit's last softmax); the value MMA goes
+    // first when both are ready, since the softmax warps wait on it and the next score
+    // MMA reuses its probabilities' columns.
     if (lane == 0) {
-      int s_next = 0, o_next = 0;
+      struct Side {
+        int k, u, uq, base, n, idx;
+      };
+      auto next_unit = [&](Side& sd) {  // advance to the next unit holding query rows
+        for (sd.u = unit_of(++sd.k); sd.u < p.units; sd.u = unit_of(++sd.k)) {
+          Unit w;
+          if (unit_at(p, sd.u, &w)) {
+            sd.base += sd.n;
+            sd.n = w.n;
+            sd.idx = 0;
+            ++sd.uq;
+            return;
+          }
+        }
+      };
+      Side S{-1, 0, -1, 0, 0, 0};
+      next_unit(S);
+      Side P = S;
+      bool q_ready = false;
       uint32_t idle = 0;
-      bool ok = wait_or_abort(q_full, 0, abort);
-      while (ok && o_next < n) {
+      while (P.u < p.units) {
         bool progressed = false;
-        if (o_next < s_next) {
-          const int st = o_next % kRing, b = o_next % 2;
-          if (mbar_test_wait(p_full0 + 8 * b, (o_next / 2) & 1) &&
-              mbar_test_wait(v_full0 + 8 * st, (o_next / kRing) & 1)) {
+        if (P.idx < P.n && P.base + P.idx < S.base + S.idx) {
+          const int t = P.base + P.idx;
+          const int st = t % kRing, b = t % 2;
+          if (mbar_test_wait(p_full0 + 8 * b, (t / 2) & 1) && mbar_test_wait(v_full0 + 8 * st, (t / kRing) & 1) &&
+              (P.idx > 0 || P.uq == 0 || mbar_test_wait(o_free, (P.uq - 1) & 1))) {
             tc_fence_after_sync();
 #pragma unroll
             for (int part = 0; part < (kSplit ? 2 : 1); ++part) {
@@ -307,20 +373,21 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
                 const int h = kk / 4;                    // softmax half owning these tokens
                 tc_mma_f16_ts(tmem + kColO + 128 * h, tmem + b * kKv + 64 * h + 32 * part + (kk % 4) * 8,
                               smem_desc(sV(st) + kk * 2048, kHalf, 1024, kSwizzle128B), kIdescO,
-                              o_next > 0 || part > 0 || (kk % 4) > 0);
+                              P.idx > 0 || part > 0 || (kk % 4) > 0);
               }
             }
             tc_commit(o_full0 + 8 * b);
             tc_commit(v_empty0 + 8 * st);
-            ++o_next;
+            if (++P.idx == P.n) next_unit(P);
             progressed = true;
           }
         }
-        if (s_next < n) {
-          const int st = s_next % kRing, b = s_next % 2;
-          // S(j) lands on P(j - 2): the value MMA that reads P(j - 2) must be issued first
-          // (MMAs of one thread run in order).
-          if (o_next >= s_next - 1 && mbar_test_wait(k_full0 + 8 * st, (s_next / kRing) & 1)) {
+        if (S.u < p.units) {
+          const int t = S.base + S.idx;
+          const int st = t % kRing, b = t % 2;
+          if (!q_ready) q_ready = mbar_test_wait(q_full, S.uq & 1);
+          // S(t) lands on P(t - 2): the value MMA that reads it must be issued first.
+          if (q_ready && t - 1 <= P.base + P.idx && mbar_test_wait(k_full0 + 8 * st, (t / kRing) & 1)) {
             tc_fence_after_sync();
 #pragma unroll
             for (int kk = 0; kk < kDim / 16; ++kk) {  // S[b] = Q . K^T, 16 dims per MMA
@@ -330,7 +397,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
             }
             tc_commit(s_full0 + 8 * b);
             tc_commit(k_empty0 + 8 * st);
-            ++s_next;
+            if (++S.idx == S.n) {
+              tc_commit(q_empty);  // the q rows may be replaced once these MMAs are done
+              q_ready = false;
+              next_unit(S);
+            }
             progressed = true;
           }
         }
@@ -351,157 +422,179 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     // Warps 2..9.  A warp may only touch the TMEM lane quarter (warp % 4); the two warps of
     // a quarter share its 32 query rows and split each tile's kv tokens: half h takes
     // tokens [64h, 64h + 64).  Each half runs its own online softmax (maximum, sum and
-    // output accumulator O_h), so the halves never wait for each other within the loop;
-    // they are combined once at the end.
+    // output accumulator O_h), so the halves never wait for each other within a unit;
+    // they combine at its end.  Both halves step through every unit and both exchange
+    // barriers even after a failed wait (then doing no other work), so neither can leave
+    // the other waiting at a barrier.
     const int q4 = warp & 3;
     const int half = (warp - 2) >> 2;
     const int r = 32 * q4 + lane;  // query row = TMEM lane
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q4) << 16;
     const uint32_t o_col = tmem + lane_addr + kColO + 128 * half;
+    const uint32_t pair_bar = 1 + q4;
     const int tl = r >> p.gq_shift, g = r & (p.GQ - 1);
-    const bool row_valid = tl < ntok;
-    const int pos = p_min + tl;
-    const int lo_row = p.window > 0 ? max(0, pos - p.window + 1) : 0;
-    float m_run = -FLT_MAX, l = 0.f;
     // Bounded wait for the value MMA of tile t, agreed by the whole warp.
     auto wait_pv = [&](int t) {
       return __all_sync(0xffffffffu, wait_or_abort(o_full0 + 8 * (t % 2), (t / 2) & 1, abort));
     };
+    int gt = 0;
     bool ok = true;
-    for (int j = 0; j < n && ok; ++j) {
-      const int b = j % 2, st = j % kRing;
-      if (!__all_sync(0xffffffffu, wait_or_abort(s_full0 + 8 * b, (j / 2) & 1, abort))) {
-        ok = false;
-        break;
-      }
-      const int kv0 = (j_lo + j) * kKv;
-      const int c0 = 64 * half;  // this warp's first column
-      const uint32_t s_col = tmem + lane_addr + b * kKv + c0;
-      float sc[64];
-      tc_fence_after_sync();
-      tmem_load64(s_col, sc);
-      // Interior tiles (every row attends every column) skip the mask.
-      const bool interior =
-          ntok == p.tq && kv0 + kKv - 1 <= p_min && (p.window <= 0 || kv0 >= p_max - p.window + 1);
-      if (!interior) {
-        const int c_lo = lo_row - kv0 - c0, c_hi = row_valid ? pos - kv0 - c0 : -1;
-#pragma unroll
-        for (int c = 0; c < 64; ++c) sc[c] = (c >= c_lo && c <= c_hi) ? sc[c] : -INFINITY;
-      }
-      float mx[8];  // eight independent chains instead of one 64-long one
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = sc[k];
-#pragma unroll
-      for (int c = 8; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], sc[c]);
-      const float mraw =
-          fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      const float mt = mraw * p.qscale;  // scores in base-2 units (qscale > 0 keeps the order)
-      float alpha = 1.f;
-      bool rescale = false;
-      if (mt > m_run + kRescaleThreshold) {  // move the reference maximum
-        alpha = ex2_ftz(m_run - mt);
-        rescale = l > 0.f;                   // O_h holds earlier contributions of this row
-        l *= alpha;
-        m_run = mt;
-      }
-      // O_h may be rescaled only after the previous value MMA.
-      if (__any_sync(0xffffffffu, rescale)) {
-        if (!wait_pv(j - 1)) {
+    for (int k = 0, u = unit_of(0); u < p.units; u = unit_of(++k)) {
+      Unit w;
+      if (!unit_at(p, u, &w)) continue;
+      const bool row_valid = tl < w.ntok;
+      const int pos = w.p_min + tl;
+      const int lo_row = p.window > 0 ? max(0, pos - p.window + 1) : 0;
+      float m_run = -FLT_MAX, l = 0.f;
+      for (int j = 0; j < w.n && ok; ++j) {
+        const int t = gt + j;
+        const int b = t % 2, st = t % kRing;
+        if (!__all_sync(0xffffffffu, wait_or_abort(s_full0 + 8 * b, (t / 2) & 1, abort))) {
           ok = false;
           break;
         }
+        const int kv0 = (w.j_lo + j) * kKv;
+        const int c0 = 64 * half;  // this warp's first column
+        const uint32_t s_col = tmem + lane_addr + b * kKv + c0;
+        float sc[64];
         tc_fence_after_sync();
-        const float a = rescale ? alpha : 1.f;
+        tmem_load64(s_col, sc);
+        // Interior tiles (every row attends every column) skip the mask.
+        const bool interior = w.ntok == p.tq && kv0 + kKv - 1 <= w.p_min &&
+                              (p.window <= 0 || kv0 >= w.p_max - p.window + 1);
+        if (!interior) {
+          const int c_lo = lo_row - kv0 - c0, c_hi = row_valid ? pos - kv0 - c0 : -1;
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          float o[32];
-          tmem_load32(o_col + 32 * c4, o);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] *= a;
-          tmem_store32(o_col + 32 * c4, o);
+          for (int c = 0; c < 64; ++c) sc[c] = (c >= c_lo && c <= c_hi) ? sc[c] : -INFINITY;
         }
-      }
-      // V rows of tokens outside the loaded blocks or past the context may hold anything
-      // (NaN); their weights are 0, so give the value MMA zeros there (kv row r; half 0
-      // clears its 64-dim lo half, half 1 the hi half).
-      const TileBlocks tb = tile_blocks(j_lo + j, bs, kv_lo, p_max);
-      const int clean_lo = tb.lo * bs - kv0, clean_hi = min(ctx, (tb.hi + 1) * bs) - kv0;
-      if (clean_lo > 0 || clean_hi < kKv) {
-        if (!__all_sync(0xffffffffu, wait_or_abort(v_full0 + 8 * st, (j / kRing) & 1, abort))) {
-          ok = false;
-          break;
+        float mx[8];  // eight independent chains instead of one 64-long one
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = sc[k];
+#pragma unroll
+        for (int c = 8; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], sc[c]);
+        const float mraw =
+            fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float mt = mraw * p.qscale;  // scores in base-2 units (qscale > 0 keeps the order)
+        float alpha = 1.f;
+        bool rescale = false;
+        if (mt > m_run + kRescaleThreshold) {  // move the reference maximum
+          alpha = ex2_ftz(m_run - mt);
+          rescale = l > 0.f;                   // O_h holds earlier contributions of this row
+          l *= alpha;
+          m_run = mt;
         }
-        if (r < clean_lo || r >= clean_hi) {
+        // O_h may be rescaled only after the previous value MMA.
+        if (__any_sync(0xffffffffu, rescale)) {
+          if (!wait_pv(t - 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const float a = rescale ? alpha : 1.f;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) st_shared_v4(sV(st) + half * kHalf + r * 128 + 16 * k, 0, 0, 0, 0);
-        }
-      }
-      // Probabilities of this half's 64 tokens, written over its own score columns as the
-      // A operand of the value MMA.  exp2(s * qscale - m) is one FFMA and one MUFU op; two
-      // weights are rounded and packed by one conversion.  The denominator sums the
-      // unrounded weights (fp16 rounding errors of the packed weights average out).
-      float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      const float neg_m = -m_run;
+          for (int c4 = 0; c4 < 4; ++c4) {
+            float o[32];
+            tmem_load32(o_col + 32 * c4, o);
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {  // two stores of 16 columns (32 tokens) each
-        uint32_t w_hi[16], w_lo[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int c = 32 * q + 2 * k;
-          const float x0 = ex2_ftz(fmaf(sc[c], p.qscale, neg_m));
-          const float x1 = ex2_ftz(fmaf(sc[c + 1], p.qscale, neg_m));
-          const Pair<IO> hi(x0, x1);
-          w_hi[k] = hi.bits;
-          if (kSplit) w_lo[k] = Pair<IO>(x0 - hi.lo_f(), x1 - hi.hi_f()).bits;
-          ls[k & 7] += x0 + x1;
-        }
-        tmem_store16_bits(s_col + 16 * q, w_hi);
-        if (kSplit) tmem_store16_bits(s_col + 32 + 16 * q, w_lo);
-      }
-      tmem_wait_store();
-      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-      fence_proxy_async_shared();  // zeroed V rows (if any) are read by the tensor core
-      tc_fence_before_sync();
-      mbar_arrive(p_full0 + 8 * b);
-    }
-    // Combine the halves: both must reach this barrier (neither returns early).  The S
-    // buffers are free once the last value MMA is done, so (m, l) travel through them.
-    const bool fin = ok && wait_pv(n - 1);
-    tc_fence_after_sync();
-    tmem_store1(tmem + lane_addr + 2 * half, m_run);
-    tmem_store1(tmem + lane_addr + 2 * half + 1, l);
-    tc_fence_before_sync();
-    named_barrier_sync(1 + q4, 64);
-    tc_fence_after_sync();
-    const float m_o = tmem_load1(tmem + lane_addr + 2 * (half ^ 1));
-    const float l_o = tmem_load1(tmem + lane_addr + 2 * (half ^ 1) + 1);
-    if (fin) {
-      const float m_all = fmaxf(m_run, m_o);
-      const float a_me = ex2_ftz(m_run - m_all), a_o = ex2_ftz(m_o - m_all);
-      const float l_all = l * a_me + l_o * a_o;
-      const float inv = row_valid ? 1.f / l_all : 0.f;
-      // this warp writes head dims [64 half, 64 half + 64): O_0 and O_1 there, weighted
-      const float w0 = (half == 0 ? a_me : a_o) * inv, w1 = (half == 0 ? a_o : a_me) * inv;
-      IO* orow = reinterpret_cast<IO*>(p.out) +
-                 (static_cast<size_t>(q_start + i0 + tl) * p.Hq + static_cast<size_t>(kh) * p.GQ + g) * kDim + 64 * half;
-#pragma unroll
-      for (int c4 = 0; c4 < 2; ++c4) {  // 32 columns at a time
-        float o0[32], o1[32];
-        tmem_load32(tmem + lane_addr + kColO + 64 * half + 32 * c4, o0);
-        tmem_load32(tmem + lane_addr + kColO + 128 + 64 * half + 32 * c4, o1);
-        if (row_valid) {
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = 8 * v + 2 * e;
-              w[e] = Pair<IO>(o0[c] * w0 + o1[c] * w1, o0[c + 1] * w0 + o1[c + 1] * w1).bits;
-            }
-            *reinterpret_cast<uint4*>(orow + 32 * c4 + 8 * v) = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int k = 0; k < 32; ++k) o[k] *= a;
+            tmem_store32(o_col + 32 * c4, o);
           }
         }
+        // V rows of tokens outside the loaded blocks or past the context may hold anything
+        // (NaN); their weights are 0, so give the value MMA zeros there (kv row r; half 0
+        // clears its 64-dim lo half, half 1 the hi half).
+        const TileBlocks tb = tile_blocks(w.j_lo + j, bs, w.kv_lo, w.p_max);
+        const int clean_lo = tb.lo * bs - kv0, clean_hi = min(w.ctx, (tb.hi + 1) * bs) - kv0;
+        if (clean_lo > 0 || clean_hi < kKv) {
+          if (!__all_sync(0xffffffffu, wait_or_abort(v_full0 + 8 * st, (t / kRing) & 1, abort))) {
+            ok = false;
+            break;
+          }
+          if (r < clean_lo || r >= clean_hi) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) st_shared_v4(sV(st) + half * kHalf + r * 128 + 16 * k, 0, 0, 0, 0);
+          }
+        }
+        // Probabilities of this half's 64 tokens, written over its own score columns as the
+        // A operand of the value MMA.  exp2(s * qscale - m) is one FFMA and one MUFU op; two
+        // weights are rounded and packed by one conversion.  The denominator sums the
+        // unrounded weights (fp16 rounding errors of the packed weights average out).
+        float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const float neg_m = -m_run;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {  // two stores of 16 columns (32 tokens) each
+          uint32_t w_hi[16], w_lo[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const int c = 32 * q + 2 * k;
+            const float x0 = ex2_ftz(fmaf(sc[c], p.qscale, neg_m));
+            const float x1 = ex2_ftz(fmaf(sc[c + 1], p.qscale, neg_m));
+            const Pair<IO> hi(x0, x1);
+            w_hi[k] = hi.bits;
+            if (kSplit) w_lo[k] = Pair<IO>(x0 - hi.lo_f(), x1 - hi.hi_f()).bits;
+            ls[k & 7] += x0 + x1;
+          }
+          tmem_store16_bits(s_col + 16 * q, w_hi);
+          if (kSplit) tmem_store16_bits(s_col + 32 + 16 * q, w_lo);
+        }
+        tmem_wait_store();
+        l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+        fence_proxy_async_shared();  // zeroed V rows (if any) are read by the tensor core
+        tc_fence_before_sync();
+        mbar_arrive(p_full0 + 8 * b);
       }
+      // ---- unit end: the halves combine (m, l) and write the rows ----
+      const bool fin = ok && wait_pv(gt + w.n - 1);
+      if (half == 1) {
+        sh.xch[0][r] = m_run;
+        sh.xch[1][r] = l;
+      }
+      named_barrier_sync(pair_bar, 64);
+      float w_me, w_other;  // weights of O_half and O_(1-half) in the output
+      if (half == 0) {
+        const float m1 = sh.xch[0][r], l1 = sh.xch[1][r];
+        const float m_all = fmaxf(m_run, m1);
+        const float a0 = ex2_ftz(m_run - m_all), a1 = ex2_ftz(m1 - m_all);
+        const float l_all = l * a0 + l1 * a1;
+        const float inv = row_valid && l_all > 0.f ? 1.f / l_all : 0.f;
+        w_me = a0 * inv;
+        w_other = a1 * inv;
+        sh.xch[0][r] = w_other;  // half 1's own weight
+        sh.xch[1][r] = w_me;     // half 1's weight for O_0
+      }
+      named_barrier_sync(pair_bar, 64);
+      if (half == 1) {
+        w_me = sh.xch[0][r];
+        w_other = sh.xch[1][r];
+      }
+      if (fin) {
+        tc_fence_after_sync();
+        const float w0 = half == 0 ? w_me : w_other, w1 = half == 0 ? w_other : w_me;
+        IO* orow = reinterpret_cast<IO*>(p.out) +
+                   (static_cast<size_t>(w.q_start + w.i0 + tl) * p.Hq + static_cast<size_t>(w.kh) * p.GQ + g) * kDim +
+                   64 * half;
+#pragma unroll
+        for (int c4 = 0; c4 < 2; ++c4) {  // this warp's 64 head dims, 32 at a time
+          float o0[32], o1[32];
+          tmem_load32(tmem + lane_addr + kColO + 64 * half + 32 * c4, o0);
+          tmem_load32(tmem + lane_addr + kColO + 128 + 64 * half + 32 * c4, o1);
+          if (row_valid) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint32_t wd[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int c = 8 * v + 2 * e;
+                wd[e] = Pair<IO>(o0[c] * w0 + o1[c] * w1, o0[c + 1] * w0 + o1[c + 1] * w1).bits;
+              }
+              *reinterpret_cast<uint4*>(orow + 32 * c4 + 8 * v) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+            }
+          }
+        }
+        tc_fence_before_sync();
+        mbar_arrive(o_free);  // O_0 and O_1 may now be overwritten by the next unit
+      }
+      gt += w.n;
     }
   }
 
@@ -603,6 +696,7 @@ extern "C" pa_status paged_attention_prefill(void* out, const void* q, const voi
   prm.NB = num_blocks;
   prm.window = window > 0 ? window : 0;
   prm.max_q_len = max_q_len;
+  prm.qtiles = (max_q_len + tq - 1) / tq;
   prm.qscale = scale * 1.4426950408889634f;
 
   const bool bf16 = dtype == PA_BF16;
@@ -615,8 +709,13 @@ extern "C" pa_status paged_attention_prefill(void* out, const void* q, const voi
     attr_err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(prefill)");
-  const dim3 grid(static_cast<unsigned>((max_q_len + tq - 1) / tq), static_cast<unsigned>(num_kv_heads),
-                  static_cast<unsigned>(num_seqs));
+  const long long units = static_cast<long long>(num_seqs) * num_kv_heads * prm.qtiles;
+  if (units > (1LL << 30)) return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: too many query tiles");
+  prm.units = static_cast<int>(units);
+  int dev = 0, sms = 0;
+  st = current_device(&dev, &sms);
+  if (st != PA_OK) return st;
+  const dim3 grid(static_cast<unsigned>(units < sms ? units : sms));  // persistent: one CTA per SM
   void* args[] = {&tmK, &tmV, &tmQ, &prm};
   cudaError_t err = launch_dependent(fn, grid, dim3(kThreads), smem, static_cast<cudaStream_t>(stream), args);
   if (err != cudaSuccess) return cuda_fail(err, "launching the prefill kernel");
