@@ -37,7 +37,9 @@ PRESET = "llama70b_fp16"
 CONTEXT_DESC = {"llama70b_fp16": "uniform [1, 2048]",
                 "chat_prefix_bf16": "2000 shared + lognormal(median 300, sigma 1) tail, 64 copy-on-write forks",
                 "sliding_window_fp16": "32768 each, window 4096",
-                "llama70b_gqa_fp16": "uniform [1, 2048], 64 query heads over 8 cached heads"}
+                "llama70b_gqa_fp16": "uniform [1, 2048], 64 query heads over 8 cached heads",
+                "llama70b_int8": "uniform [1, 2048], INT8 cache written by quantise-on-write",
+                "llama70b_fp8": "uniform [1, 2048], FP8 E4M3 cache written by quantise-on-write"}
 METRIC = "paged decode attention KV GB/s (% of B200 HBM peak) and tokens/s per layer"
 FALLBACK_HBM_GBS = 6650.0
 
@@ -174,11 +176,15 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------------
 # workload
 # ---------------------------------------------------------------------------------------
+EIGHT_BIT = {"llama70b_int8": torch.int8, "llama70b_fp8": torch.float8_e4m3fn}
+
+
 def build(seed: int, device, workload: str = PRESET, block_size=None):
     import paged_kv_cache_384_b200 as pa
     over = {} if block_size is None else {"block_size": block_size}
     big = workload == "sliding_window_fp16"          # 8.6 GB of cache: draw values on the GPU
-    w = synth.build_workload(workload, seed, pa.BlockManager, device=device if big else "cpu", **over)
+    preset = "llama70b_int8" if workload in EIGHT_BIT else workload
+    w = synth.build_workload(preset, seed, pa.BlockManager, device=device if big else "cpu", **over)
     ctx = w.context_lens.tolist()
     slots = pa.slot_mapping(w.block_tables, range(w.num_seqs), [c - 1 for c in ctx], w.block_size)
     host = dict(q=w.q.cpu(), k_new=w.k_new.cpu(), v_new=w.v_new.cpu(), slots=slots, block_tables=w.block_tables,
@@ -186,6 +192,24 @@ def build(seed: int, device, workload: str = PRESET, block_size=None):
     dev = {k: v.to(device) for k, v in host.items()}
     dev["k_cache"] = w.k_cache.to(device)
     dev["v_cache"] = w.v_cache.to(device)
+    dev["k_scale"] = dev["v_scale"] = None
+    if workload in EIGHT_BIT:
+        # The fp16 pool is quantised on the GPU by the library's own quantise-on-write
+        # kernel, every slot as one row (untimed setup); steps then write the newest rows
+        # through the same kernel.
+        src_k, src_v = dev["k_cache"], dev["v_cache"]
+        NB, bs, H, D = src_k.shape
+        code = EIGHT_BIT[workload]
+        dev["k_cache"] = torch.empty(NB, bs, H, D, dtype=code, device=device)
+        dev["v_cache"] = torch.empty_like(dev["k_cache"])
+        dev["k_scale"] = torch.empty(NB, bs, H, dtype=torch.float16, device=device)
+        dev["v_scale"] = torch.empty_like(dev["k_scale"])
+        all_slots = torch.arange(NB * bs, dtype=torch.int64, device=device)
+        pa.reshape_and_cache_quant(src_k.view(NB * bs, H, D), src_v.view(NB * bs, H, D), dev["k_cache"],
+                                   dev["v_cache"], dev["k_scale"], dev["v_scale"], all_slots)
+        torch.cuda.synchronize(device)
+        del src_k, src_v
+        w.cache_dtype = "int8" if code == torch.int8 else "fp8"
     dev["out"] = torch.empty_like(dev["q"])
     dev["ws"] = pa.alloc_workspace(w.num_seqs, w.num_heads, w.head_dim, device)
     dev["pairs"] = w.copy_pairs.to(device)
@@ -195,11 +219,16 @@ def build(seed: int, device, workload: str = PRESET, block_size=None):
 
 def step(pa, w, d, stream):
     """One pass of the hot path: append the newest rows, copy-on-write copies, decode."""
-    pa.reshape_and_cache(d["k_new"], d["v_new"], d["k_cache"], d["v_cache"], d["slots"], stream=stream)
+    if d["k_scale"] is not None:   # 8-bit cache: quantise-on-write
+        pa.reshape_and_cache_quant(d["k_new"], d["v_new"], d["k_cache"], d["v_cache"], d["k_scale"], d["v_scale"],
+                                   d["slots"], stream=stream)
+    else:
+        pa.reshape_and_cache(d["k_new"], d["v_new"], d["k_cache"], d["v_cache"], d["slots"], stream=stream)
     if d["pairs"].shape[0]:
         pa.copy_blocks(d["k_cache"], d["v_cache"], d["pairs"], stream=stream)
     pa.paged_attention_decode(d["out"], d["q"], d["k_cache"], d["v_cache"], d["block_tables"],
-                              d["context_lens"], w.scale, w.window, workspace=d["ws"], stream=stream)
+                              d["context_lens"], w.scale, w.window, d["k_scale"], d["v_scale"], workspace=d["ws"],
+                              stream=stream)
 
 
 class PackedInputs:
@@ -340,8 +369,6 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    if args.workload == "llama70b_int8":
-        raise SystemExit("the int8 workload needs a quantised cache; see --workload choices")
     w, host, d, kv_bytes = build(rank_seed(args.seed, rank), device, args.workload, args.block_size)
     stream = torch.cuda.current_stream(device)
     peak, peak_kind = measured_peak()
@@ -415,7 +442,7 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": {"fp16": "f16", "bf16": "bf16", "fp32": "f32", "int8": "i8"}[w.cache_dtype],
+        "vs_baseline": None, "dtype": {"fp16": "f16", "bf16": "bf16", "fp32": "f32", "int8": "i8", "fp8": "fp8_e4m3"}[w.cache_dtype],
         "data": "synthetic",
         "config": {"workload": args.workload, "num_seqs": w.num_seqs, "num_heads": w.num_heads, "head_dim": w.head_dim,
                    "block_size": w.block_size, "num_blocks": w.num_blocks, "window": w.window,
@@ -426,7 +453,8 @@ def run_ours(args):
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_kind,
-                     "kernel": "decode_partition_kernel", "partition_ms": round(part_avg, 4),
+                     "kernel": "decode_gqa_tc_kernel" if w.num_kv_heads * 4 <= w.num_heads else "decode_partition_kernel",
+                     "partition_ms": round(part_avg, 4),
                      "merge_ms": round(merge_avg, 4)},
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -657,7 +685,8 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=PRESET, choices=["llama70b_fp16", "chat_prefix_bf16", "sliding_window_fp16",
-                                                           "llama70b_gqa_fp16", "swap_llama70b_fp16", *PREFILL],
+                                                           "llama70b_gqa_fp16", "llama70b_int8", "llama70b_fp8", "swap_llama70b_fp16",
+                                                           *PREFILL],
                     help="secondary workloads are for study; the metric is quoted on the default")
     ap.add_argument("--block-size", type=int, default=None)
     args = ap.parse_args(argv)

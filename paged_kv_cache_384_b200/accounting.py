@@ -7,14 +7,14 @@
   PagedAttention memory design" (trdm.cn), section 一, flowchart; block-size-16 waste claim
   in "KV Cache memory optimisation and PagedAttention", section "vLLM调度器与PagedAttention协同工作").
 * Algorithmic bytes of one decode call: every attended token's K and V row for every head
-  is read exactly once (plus the fp16 scales of an INT8 cache).  This is the numerator of
+  is read exactly once (plus the fp16 scales of an INT8 or FP8 cache).  This is the numerator of
   the KV GB/s metric.
 """
 from __future__ import annotations
 
 from typing import Iterable
 
-ELEM_BYTES = {"fp32": 4, "fp16": 2, "bf16": 2, "int8": 1}
+ELEM_BYTES = {"fp32": 4, "fp16": 2, "bf16": 2, "int8": 1, "fp8": 1}
 
 
 def kv_bytes_per_token(layers: int, num_heads: int, head_dim: int, dtype_size: int) -> int:
@@ -41,10 +41,10 @@ def attended_tokens(context_len: int, window: int = 0) -> int:
 
 def decode_kv_bytes(context_lens: Iterable[int], num_heads: int, head_dim: int, cache_dtype: str,
                     window: int = 0) -> int:
-    """Algorithmic K+V bytes of one decode call over a batch (scales included for int8)."""
+    """Algorithmic K+V bytes of one decode call over a batch (scales included for 8-bit caches)."""
     e = ELEM_BYTES[cache_dtype]
     tokens = sum(attended_tokens(int(c), window) for c in context_lens)
     total = tokens * num_heads * head_dim * 2 * e
-    if cache_dtype == "int8":
+    if cache_dtype in ("int8", "fp8"):
         total += tokens * num_heads * 2 * 2  # one fp16 scale per (token, head) for K and for V
     return total
