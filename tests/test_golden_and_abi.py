@@ -143,3 +143,39 @@ def test_gqa_host_validation(L):
     assert call(6, 4) == 1              # query heads not a multiple of cached heads
     assert call(8, 0) == 1
     assert call(64, 8, 3, 3) == 1       # int8 queries are not a thing
+
+
+def test_prefill_host_validation(L):
+    P = ctypes.c_void_p
+    def call(T=40, mq=40, hq=8, hkv=2, D=128, bs=16, dt=1, ptr=16):
+        p = P(ptr) if ptr else None
+        return L.paged_attention_prefill(p, p, p, p, p, p, p, 1, T, mq, hq, hkv, D, bs, 64, 8, 0.1, 0, dt, None)
+    assert call(hq=6, hkv=4) == 1       # query heads not a multiple of cached heads
+    assert call(hq=12, hkv=4) == 2      # 3 query heads per cached head: unsupported
+    assert call(hq=64, hkv=2) == 2      # 32 per cached head: unsupported
+    assert call(D=64) == 2              # head_dim 128 only
+    assert call(bs=12) == 2             # block size must divide 128 in steps of 8
+    assert call(dt=0) == 2              # fp32 I/O is not a tensor-core type here
+    assert call(T=-1) == 1
+    assert call(ptr=0) == 1             # NULL pointers
+    assert call(ptr=24) == 1            # not 16-byte aligned
+    assert call(T=0) == 0               # nothing to do
+    assert call(mq=0) == 0
+    assert L.pa_last_error().decode()
+
+
+def test_swap_host_validation(L):
+    P = ctypes.c_void_p
+    def call(n=1, nsrc=4, ndst=4, bb=4096, scales=(None, None, None, None), sb=0, pairs=16):
+        return L.swap_blocks(P(16), P(16), P(16), P(16), P(pairs) if pairs else None, n, nsrc, ndst, bb,
+                             *[P(x) if x else None for x in scales], sb, None)
+    assert call(n=-1) == 1
+    assert call(nsrc=0) == 1
+    assert call(bb=0) == 1
+    assert call(scales=(16, 16, 16, None), sb=64) == 1   # all four scale pools or none
+    assert call(scales=(16, 16, 16, 16), sb=0) == 1
+    assert call(pairs=0) == 1                            # NULL pair array
+    assert call(pairs=20) == 1                           # pairs not 8-byte aligned
+    assert call(n=70000) == 2                            # more pairs than one launch takes
+    assert call(n=0) == 0                                # nothing to do
+
