@@ -101,23 +101,6 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
   return false;
 }
 
-// 2^x on the FMA pipe, for the share of a tile's weights that would otherwise queue on the
-// transcendental unit.  Range reduction x = n + f with n = round(x), f in [-1/2, 1/2]
-// (adding and subtracting 1.5 * 2^23 rounds to an integer that lands in the low mantissa
-// bits), a degree-4 polynomial for 2^f whose coefficients are a weighted least-squares
-// minimax fit of relative error on that interval (max relative error 2.7e-6, below
-// bf16's hi + lo weights), then n added to the exponent field.  Inputs below -125 give 0.
-__device__ __forceinline__ float ex2_poly(float x) {
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  float p = fmaf(0.009570098482072353f, f, 0.05591786280274391f);
-  p = fmaf(p, f, 0.240247443318367f);
-  p = fmaf(p, f, 0.6931217908859253f);
-  p = fmaf(p, f, 0.9999992847442627f);
-  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-  return x > -125.f ? r : 0.f;
-}
-
 // Two weights rounded to IO by one packed conversion, with their values back in fp32.
 template <typename IO> struct Pair;
 template <> struct Pair<__half> {
@@ -533,9 +516,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
           }
         }
         // Probabilities of this half's 64 tokens, written over its own score columns as the
-        // A operand of the value MMA.  exp2(s * qscale - m) is one FFMA and one MUFU op (or,
-        // for a quarter of the weights, the polynomial above); two weights are rounded and
-        // packed by one conversion.  The denominator sums the
+        // A operand of the value MMA.  exp2(s * qscale - m) is one FFMA and one MUFU op; two
+        // weights are rounded and packed by one conversion.  (Moving a quarter of them to a
+        // polynomial on the FMA pipe measured slower: the transcendental unit is not what
+        // limits this loop.)  The denominator sums the
         // unrounded weights (fp16 rounding errors of the packed weights average out).
         float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         const float neg_m = -m_run;
@@ -545,10 +529,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
             const int c = 32 * q + 2 * k;
-            // one pair in four goes to the FMA pipe, the rest to the transcendental unit
-            const float y0 = fmaf(sc[c], p.qscale, neg_m), y1 = fmaf(sc[c + 1], p.qscale, neg_m);
-            const float x0 = (k & 3) == 3 ? ex2_poly(y0) : ex2_ftz(y0);
-            const float x1 = (k & 3) == 3 ? ex2_poly(y1) : ex2_ftz(y1);
+            const float x0 = ex2_ftz(fmaf(sc[c], p.qscale, neg_m));
+            const float x1 = ex2_ftz(fmaf(sc[c + 1], p.qscale, neg_m));
             const Pair<IO> hi(x0, x1);
             w_hi[k] = hi.bits;
             if (kSplit) w_lo[k] = Pair<IO>(x0 - hi.lo_f(), x1 - hi.hi_f()).bits;
