@@ -13,7 +13,11 @@ __device__ __forceinline__ void decode_error(unsigned int bits) { atomicOr(&g_de
 
 constexpr int kMaxCtasPerSm = 4;    // persistent-grid CTAs per SM (upper bound)
 constexpr int kMaxHeadGroup = 8;    // heads per CTA (upper bound)
-constexpr int kMaxThreads = 32 * (kMaxHeadGroup + 1);
+constexpr int kMaxThreads = 32 * (kMaxHeadGroup + 1);  // CUDA-core kernel: TMA warp + head warps
+// Threads per CTA of any kernel that plans with plan_slice (the tensor-core kernel has 320);
+// PlanScratch holds one entry each.
+constexpr int kMaxPlanThreads = 320;
+static_assert(kMaxPlanThreads >= kMaxThreads, "plan scratch must cover the CUDA-core kernel");
 constexpr int kBarrierBytes = 128;  // mbarriers at the front of dynamic smem (<= 8 stages)
 
 struct DecodeParams {
@@ -117,7 +121,7 @@ __device__ __forceinline__ void store_floats(IO* dst, const float* src) {
 // the CTA must call it.  Returns count (0: nothing to do, or an impossible plan reported as
 // PA_DEVERR_TIMEOUT); *start is the cursor of tile t0.
 struct PlanScratch {
-  long long chunk[kMaxThreads];
+  long long chunk[kMaxPlanThreads];
   long long total;
   long long first_prefix;
   int first_seq;

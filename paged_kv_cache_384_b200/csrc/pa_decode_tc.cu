@@ -14,14 +14,13 @@
 // "vLLM source first look: PagedAttention memory design" (trdm.cn), section 三); the
 // grouped-query tile is this library's design.
 //
-// Roles (one CTA per SM, 9 warps):
+// Roles (one CTA per SM, 10 warps):
 //   warps 0,6-8 TMA producers, one per part of a tile (K or V, 64-dim half, 128-byte
 //               swizzle): each issues its part of every attended block into a 3-stage ring
 //               (warp 0 also the q rows of the head group); block-table entries are loaded
 //               by the lanes in parallel.
-//   warp 1      TMEM owner and MMA issuer (one lane): polls for ready work and issues the score
-//               MMA of the next landed tile or the value MMA of the oldest softmaxed tile,
-//               whichever is ready, so stages are released without waiting on later tiles.
+//   warp 1      TMEM owner and score-MMA issuer (one lane); warp 9 issues the value MMAs
+//               (one lane): the MMAs are small, so their issue is split over two warps.
 //   warps 2..5  softmax (thread = token row of S^T) and accumulation (thread = head dim row
 //               of O^T): online softmax in base 2, probabilities written as the B operand of
 //               the value MMA, V rows of unattended tokens zeroed, running output rescaled in
@@ -48,7 +47,8 @@ constexpr int kStageBytes = 4 * kHalf + 2 * kQHalf;  // K lo, K hi, V lo, V hi, 
 constexpr int kStages = 3;
 constexpr int kPBytes = kTokens * kHeadsN * 2;  // one probability operand, 128 tokens x 16 heads
 constexpr int kPBuffers = 4;                    // 2 tiles in flight x (hi, lo) parts
-constexpr int kThreads = 288;  // TMA warps 0 and 6..8, MMA warp 1, softmax warps 2..5
+constexpr int kThreads = 320;  // TMA warps 0 and 6..8, score-MMA warp 1, softmax warps 2..5, value-MMA warp 9
+static_assert(kThreads <= kMaxPlanThreads, "plan_slice keeps one scratch entry per thread");
 constexpr uint32_t kTmemCols = 64;              // S0 [0,16)  S1 [16,32)  O0 [32,48)  O1 [48,64)
 constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + kPBuffers * kPBytes;
 
@@ -56,6 +56,7 @@ struct TcShared {
   uint64_t full[kStages], empty[kStages];       // TMA ring
   uint64_t s_full[2], s_empty[2];               // score accumulators in TMEM
   uint64_t p_full[2], o_full[2];                // probabilities written / value MMA done
+  uint64_t mma_done;                            // both MMA warps' last MMAs finished
   uint32_t tmem_base;
   int abort;
   float red[2][4][kHeadsN];                     // per-tile maxima across the softmax warps (by tile parity)
@@ -133,6 +134,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       mbar_init(p_full0 + 8 * b, 128);
       mbar_init(o_full0 + 8 * b, 1);
     }
+    mbar_init(smem_u32(&sh.mma_done), 2);
     sh.abort = 0;
     fence_barrier_init();
   }
@@ -150,7 +152,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
   tc_fence_after_sync();
   const uint32_t tmem = sh.tmem_base;
 
-  if (warp == 0 || warp >= 6) {
+  if (warp == 0 || (warp >= 6 && warp <= 8)) {
     // ------------------------------------------------------------------ TMA producers --
     // Four warps, one per (K or V) x (64-dim half) part of a tile: a warp issues its copies
     // one after another, so four warps issue a tile four times as fast as one.  Warp 0
@@ -226,63 +228,50 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     if (lane == 0)  // never leave with copies in flight
       for (int k = issued - kStages < 0 ? 0 : issued - kStages; k < issued; ++k)
         wait_or_abort(full0 + 8 * (k % kStages), (k / kStages) & 1, abort);
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------- MMA issuer --
-    // One lane polls both kinds of work (non-blocking probes) and issues whichever is
-    // ready: the score MMA of the next tile whose K/V/q landed, or the value MMA of the
-    // oldest tile whose probabilities are written.  Neither waits behind the other, so a
-    // stage is released as soon as its value MMA is done.
+  } else if (warp == 1 || warp == 9) {
+    // ------------------------------------------------------------------ MMA issuers --
+    // The MMAs of a tile are small (N = 16), so issuing them costs more than running
+    // them: warp 1 issues the score MMAs and warp 9 the value MMAs, one lane each, so the
+    // two streams do not queue behind each other.  A stage is released by the value MMA
+    // that last reads it (its score MMA finished before the probabilities were written).
     if (lane == 0) {
-      int s_next = 0, o_next = 0;
-      uint32_t idle = 0;
-      while (o_next < n) {
-        bool progressed = false;
-        if (s_next < n) {
-          const int st = s_next % kStages, b = s_next % 2;
-          if (mbar_test_wait(full0 + 8 * st, (s_next / kStages) & 1) &&
-              (s_next < 2 || mbar_test_wait(s_empty0 + 8 * b, ((s_next / 2) - 1) & 1))) {
-            tc_fence_after_sync();
-            const uint32_t sb = stage(st);
+      if (warp == 1) {
+        for (int i = 0; i < n; ++i) {
+          const int st = i % kStages, b = i % 2;
+          if (!wait_or_abort(full0 + 8 * st, (i / kStages) & 1, abort)) break;
+          if (i >= 2 && !wait_or_abort(s_empty0 + 8 * b, ((i / 2) - 1) & 1, abort)) break;
+          tc_fence_after_sync();
+          const uint32_t sb = stage(st);
 #pragma unroll
-            for (int kk = 0; kk < kDim / 16; ++kk) {  // S^T[b] = K . Q^T, 16 dims per MMA
-              const uint32_t koff = (kk / 4) * kHalf + (kk % 4) * 32;  // 32 B steps inside a swizzled row
-              const uint32_t qoff = 4 * kHalf + (kk / 4) * kQHalf + (kk % 4) * 32;
-              tc_mma_f16(tmem + b * kHeadsN, smem_desc(sb + koff, 16, 1024, kSwizzle128B),
-                         smem_desc(sb + qoff, 16, 1024, kSwizzle128B), kIdescS, kk > 0);
-            }
-            tc_commit(s_full0 + 8 * b);
-            ++s_next;
-            progressed = true;
+          for (int kk = 0; kk < kDim / 16; ++kk) {  // S^T[b] = K . Q^T, 16 dims per MMA
+            const uint32_t koff = (kk / 4) * kHalf + (kk % 4) * 32;  // 32 B steps inside a swizzled row
+            const uint32_t qoff = 4 * kHalf + (kk / 4) * kQHalf + (kk % 4) * 32;
+            tc_mma_f16(tmem + b * kHeadsN, smem_desc(sb + koff, 16, 1024, kSwizzle128B),
+                       smem_desc(sb + qoff, 16, 1024, kSwizzle128B), kIdescS, kk > 0);
           }
+          tc_commit(s_full0 + 8 * b);
         }
-        if (o_next < s_next) {
-          const int b = o_next % 2;
-          if (mbar_test_wait(p_full0 + 8 * b, (o_next / 2) & 1)) {
-            tc_fence_after_sync();
-            const uint32_t sb = stage(o_next % kStages);
-            const uint32_t o_tmem = tmem + 2 * kHeadsN + b * kHeadsN;
+      } else {
+        for (int i = 0; i < n; ++i) {
+          const int b = i % 2;
+          if (!wait_or_abort(p_full0 + 8 * b, (i / 2) & 1, abort)) break;
+          tc_fence_after_sync();
+          const uint32_t sb = stage(i % kStages);
+          const uint32_t o_tmem = tmem + 2 * kHeadsN + b * kHeadsN;
 #pragma unroll
-            for (int part = 0; part < (kSplit ? 2 : 1); ++part) {
+          for (int part = 0; part < (kSplit ? 2 : 1); ++part) {
 #pragma unroll
-              for (int kk = 0; kk < kTokens / 16; ++kk) {  // O^T[b] = V^T . P^T, 16 tokens per MMA
-                tc_mma_f16(o_tmem, smem_desc(sb + 2 * kHalf + kk * 2048, kHalf, 1024, kSwizzle128B),
-                           smem_desc(pbuf(b, part) + kk * 512, kPBytes, 256, kSwizzle32B), kIdescO, part > 0 || kk > 0);
-              }
+            for (int kk = 0; kk < kTokens / 16; ++kk) {  // O^T[b] = V^T . P^T, 16 tokens per MMA
+              tc_mma_f16(o_tmem, smem_desc(sb + 2 * kHalf + kk * 2048, kHalf, 1024, kSwizzle128B),
+                         smem_desc(pbuf(b, part) + kk * 512, kPBytes, 256, kSwizzle32B), kIdescO, part > 0 || kk > 0);
             }
-            tc_commit(o_full0 + 8 * b);
-            tc_commit(empty0 + 8 * (o_next % kStages));
-            ++o_next;
-            progressed = true;
           }
-        }
-        if (progressed) {
-          idle = 0;
-        } else if (*abort || ++idle > 16 * kWaitLimit) {
-          if (!*abort) decode_error(PA_DEVERR_TIMEOUT);
-          *abort = 1;
-          break;
+          tc_commit(o_full0 + 8 * b);
+          tc_commit(empty0 + 8 * (i % kStages));
         }
       }
+      tc_commit(smem_u32(&sh.mma_done));  // this warp's MMAs have finished before TMEM is released
+      mbar_wait_bounded(smem_u32(&sh.mma_done), 0);
     }
     __syncwarp();
   } else {
