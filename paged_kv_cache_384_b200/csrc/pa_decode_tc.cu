@@ -19,8 +19,8 @@
 //               swizzle): each issues its part of every attended block into a 3-stage ring
 //               (warp 0 also the q rows of the head group); block-table entries are loaded
 //               by the lanes in parallel.
-//   warp 1      TMEM owner and score-MMA issuer (one lane); warp 9 issues the value MMAs
-//               (one lane): the MMAs are small, so their issue is split over two warps.
+//   warp 1      TMEM owner and MMA issuer (one lane); with up to 8 query heads per cached
+//               head warp 9 issues the value MMAs and warp 1 only the score MMAs.
 //   warps 2..5  softmax (thread = token row of S^T) and accumulation (thread = head dim row
 //               of O^T): online softmax in base 2, probabilities written as the B operand of
 //               the value MMA, V rows of unattended tokens zeroed, running output rescaled in
@@ -230,47 +230,84 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         wait_or_abort(full0 + 8 * (k % kStages), (k / kStages) & 1, abort);
   } else if (warp == 1 || warp == 9) {
     // ------------------------------------------------------------------ MMA issuers --
-    // The MMAs of a tile are small (N = 16), so issuing them costs more than running
-    // them: warp 1 issues the score MMAs and warp 9 the value MMAs, one lane each, so the
-    // two streams do not queue behind each other.  A stage is released by the value MMA
-    // that last reads it (its score MMA finished before the probabilities were written).
-    if (lane == 0) {
+    // Score MMAs: S^T[b] = K . Q^T, 16 dims per MMA.  Value MMAs: O^T[b] = V^T . P^T, 16
+    // tokens per MMA.  A stage is released by the value MMA that last reads it (its score
+    // MMA finished before the probabilities were written).
+    auto issue_scores = [&](int i) {
+      const int st = i % kStages, b = i % 2;
+      const uint32_t sb = stage(st);
+#pragma unroll
+      for (int kk = 0; kk < kDim / 16; ++kk) {
+        const uint32_t koff = (kk / 4) * kHalf + (kk % 4) * 32;  // 32 B steps inside a swizzled row
+        const uint32_t qoff = 4 * kHalf + (kk / 4) * kQHalf + (kk % 4) * 32;
+        tc_mma_f16(tmem + b * kHeadsN, smem_desc(sb + koff, 16, 1024, kSwizzle128B),
+                   smem_desc(sb + qoff, 16, 1024, kSwizzle128B), kIdescS, kk > 0);
+      }
+      tc_commit(s_full0 + 8 * b);
+    };
+    auto issue_values = [&](int i) {
+      const int b = i % 2;
+      const uint32_t sb = stage(i % kStages);
+      const uint32_t o_tmem = tmem + 2 * kHeadsN + b * kHeadsN;
+#pragma unroll
+      for (int part = 0; part < (kSplit ? 2 : 1); ++part) {
+#pragma unroll
+        for (int kk = 0; kk < kTokens / 16; ++kk) {
+          tc_mma_f16(o_tmem, smem_desc(sb + 2 * kHalf + kk * 2048, kHalf, 1024, kSwizzle128B),
+                     smem_desc(pbuf(b, part) + kk * 512, kPBytes, 256, kSwizzle32B), kIdescO, part > 0 || kk > 0);
+        }
+      }
+      tc_commit(o_full0 + 8 * b);
+      tc_commit(empty0 + 8 * (i % kStages));
+    };
+    // With up to 8 query heads per cached head the MMAs are small enough that issuing them
+    // is the cost, so warp 1 issues the score MMAs and warp 9 the value MMAs.  With 16 the
+    // softmax work per tile is larger and one lane of warp 1 polling for either kind of
+    // ready work measured faster (3.98 vs 3.08 TB/s at 4 cached heads); warp 9 then idles.
+    constexpr bool kTwoIssuers = NH <= 8;
+    if (lane == 0 && kTwoIssuers) {
       if (warp == 1) {
         for (int i = 0; i < n; ++i) {
-          const int st = i % kStages, b = i % 2;
-          if (!wait_or_abort(full0 + 8 * st, (i / kStages) & 1, abort)) break;
-          if (i >= 2 && !wait_or_abort(s_empty0 + 8 * b, ((i / 2) - 1) & 1, abort)) break;
+          if (!wait_or_abort(full0 + 8 * (i % kStages), (i / kStages) & 1, abort)) break;
+          if (i >= 2 && !wait_or_abort(s_empty0 + 8 * (i % 2), ((i / 2) - 1) & 1, abort)) break;
           tc_fence_after_sync();
-          const uint32_t sb = stage(st);
-#pragma unroll
-          for (int kk = 0; kk < kDim / 16; ++kk) {  // S^T[b] = K . Q^T, 16 dims per MMA
-            const uint32_t koff = (kk / 4) * kHalf + (kk % 4) * 32;  // 32 B steps inside a swizzled row
-            const uint32_t qoff = 4 * kHalf + (kk / 4) * kQHalf + (kk % 4) * 32;
-            tc_mma_f16(tmem + b * kHeadsN, smem_desc(sb + koff, 16, 1024, kSwizzle128B),
-                       smem_desc(sb + qoff, 16, 1024, kSwizzle128B), kIdescS, kk > 0);
-          }
-          tc_commit(s_full0 + 8 * b);
+          issue_scores(i);
         }
       } else {
         for (int i = 0; i < n; ++i) {
-          const int b = i % 2;
-          if (!wait_or_abort(p_full0 + 8 * b, (i / 2) & 1, abort)) break;
+          if (!wait_or_abort(p_full0 + 8 * (i % 2), (i / 2) & 1, abort)) break;
           tc_fence_after_sync();
-          const uint32_t sb = stage(i % kStages);
-          const uint32_t o_tmem = tmem + 2 * kHeadsN + b * kHeadsN;
-#pragma unroll
-          for (int part = 0; part < (kSplit ? 2 : 1); ++part) {
-#pragma unroll
-            for (int kk = 0; kk < kTokens / 16; ++kk) {  // O^T[b] = V^T . P^T, 16 tokens per MMA
-              tc_mma_f16(o_tmem, smem_desc(sb + 2 * kHalf + kk * 2048, kHalf, 1024, kSwizzle128B),
-                         smem_desc(pbuf(b, part) + kk * 512, kPBytes, 256, kSwizzle32B), kIdescO, part > 0 || kk > 0);
-            }
-          }
-          tc_commit(o_full0 + 8 * b);
-          tc_commit(empty0 + 8 * (i % kStages));
+          issue_values(i);
         }
       }
-      tc_commit(smem_u32(&sh.mma_done));  // this warp's MMAs have finished before TMEM is released
+    }
+    if (lane == 0 && !kTwoIssuers && warp == 1) {
+      int s_next = 0, o_next = 0;
+      uint32_t idle = 0;
+      while (o_next < n) {
+        bool progressed = false;
+        if (s_next < n && mbar_test_wait(full0 + 8 * (s_next % kStages), (s_next / kStages) & 1) &&
+            (s_next < 2 || mbar_test_wait(s_empty0 + 8 * (s_next % 2), ((s_next / 2) - 1) & 1))) {
+          tc_fence_after_sync();
+          issue_scores(s_next++);
+          progressed = true;
+        }
+        if (o_next < s_next && mbar_test_wait(p_full0 + 8 * (o_next % 2), (o_next / 2) & 1)) {
+          tc_fence_after_sync();
+          issue_values(o_next++);
+          progressed = true;
+        }
+        if (progressed) {
+          idle = 0;
+        } else if (*abort || ++idle > 16 * kWaitLimit) {
+          if (!*abort) decode_error(PA_DEVERR_TIMEOUT);
+          *abort = 1;
+          break;
+        }
+      }
+    }
+    if (lane == 0) {  // every MMA this warp issued has finished before TMEM is released
+      tc_commit(smem_u32(&sh.mma_done));
       mbar_wait_bounded(smem_u32(&sh.mma_done), 0);
     }
     __syncwarp();
