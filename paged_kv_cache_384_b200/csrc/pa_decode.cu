@@ -156,7 +156,12 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   const int v = lane % LPR;  // 16-byte vector within the row: dims [v*EV, v*EV + EV)
   Cursor c = start;
   bool seg_from_start = (c.j == 0);
+  // INT8 codes are widened and multiplied two at a time on packed fp32 pairs (fewer
+  // instructions per byte, which is what limits this path); q and the accumulator are then
+  // kept as pairs too.
+  constexpr bool kPairs = std::is_same<CT, int8_t>::value;
   float qf[EV], acc[EV];
+  uint64_t q2[EV / 2], acc2[EV / 2];
   float m = -FLT_MAX, l = 0.f;  // running max (base 2) and sum; -FLT_MAX keeps exp2 finite
   auto load_q = [&](const Cursor& cc) {
     const int h = cc.g * QW + w;
@@ -164,10 +169,15 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
     load_floats<IO, EV>(qrow, qf);
 #pragma unroll
     for (int e = 0; e < EV; ++e) qf[e] *= p.qscale;
+    if (kPairs)
+#pragma unroll
+      for (int j = 0; j < EV / 2; ++j) q2[j] = f2_pack(qf[2 * j], qf[2 * j + 1]);
   };
   load_q(c);
 #pragma unroll
   for (int e = 0; e < EV; ++e) acc[e] = 0.f;
+#pragma unroll
+  for (int j = 0; j < EV / 2; ++j) acc2[j] = 0;
 
   for (int it = 0; it < n; ++it) {
     const int st = it % NS;
@@ -190,10 +200,15 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
         const int t = pi * RPP + r;
         float part = 0.f;
         if (t < tt) {
-          float kf[EV];
-          Elem<CT>::to_float(ld_shared_v4(kt + ((t * HG + kw) * D + v * EV) * E), kf);
+          const uint4 kv = ld_shared_v4(kt + ((t * HG + kw) * D + v * EV) * E);
+          if constexpr (kPairs) {
+            part = Elem<CT>::dot(kv, q2);
+          } else {
+            float kf[EV];
+            Elem<CT>::to_float(kv, kf);
 #pragma unroll
-          for (int e = 0; e < EV; ++e) part = fmaf(qf[e], kf[e], part);
+            for (int e = 0; e < EV; ++e) part = fmaf(qf[e], kf[e], part);
+          }
         }
 #pragma unroll
         for (int off = LPR / 2; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
@@ -213,8 +228,14 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
     const float alpha = exp2f(m - m_new);
     m = m_new;
     l *= alpha;
+    if constexpr (kPairs) {
+      const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-    for (int e = 0; e < EV; ++e) acc[e] *= alpha;
+      for (int j = 0; j < EV / 2; ++j) acc2[j] = f2_fma(a2, acc2[j], 0);
+    } else {
+#pragma unroll
+      for (int e = 0; e < EV; ++e) acc[e] *= alpha;
+    }
 #pragma unroll
     for (int pi = 0; pi < MAXP; ++pi) {
       if (TT > 0 || pi * RPP < tt) {
@@ -222,12 +243,17 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
         if (sc[pi] != -INFINITY) {  // attended row (rows outside [lo, ctx) may hold garbage)
           const float pr = exp2f(sc[pi] - m);
           l += pr;
-          float vf[EV];
-          Elem<CT>::to_float(ld_shared_v4(vt + ((t * HG + kw) * D + v * EV) * E), vf);
+          const uint4 vv = ld_shared_v4(vt + ((t * HG + kw) * D + v * EV) * E);
           float pv = pr;
           if (kInt8) pv *= __half2float(__ushort_as_half(ld_shared_u16(kt + p.vs_off + (t * 8 + hs) * 2)));
+          if constexpr (kPairs) {
+            Elem<CT>::axpy(pv, vv, acc2);
+          } else {
+            float vf[EV];
+            Elem<CT>::to_float(vv, vf);
 #pragma unroll
-          for (int e = 0; e < EV; ++e) acc[e] = fmaf(pv, vf[e], acc[e]);
+            for (int e = 0; e < EV; ++e) acc[e] = fmaf(pv, vf[e], acc[e]);
+          }
         }
       }
     }
@@ -236,6 +262,9 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
 
     const bool seg_last = (c.j == c.sp.nb - 1);
     if (seg_last || it == n - 1) {
+      if constexpr (kPairs)
+#pragma unroll
+        for (int j = 0; j < EV / 2; ++j) f2_unpack(acc2[j], acc[2 * j], acc[2 * j + 1]);
       // Combine the RPP row groups of the warp.
       float lt = l;
 #pragma unroll
@@ -270,6 +299,8 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
       l = 0.f;
 #pragma unroll
       for (int e = 0; e < EV; ++e) acc[e] = 0.f;
+#pragma unroll
+      for (int j = 0; j < EV / 2; ++j) acc2[j] = 0;
     }
     if (it + 1 < n) {
       advance(c, p);

@@ -58,6 +58,32 @@ template <> struct Elem<__nv_bfloat16> {
   }
 };
 
+// Packed fp32 pairs (sm_100 `.f32x2` arithmetic: one instruction for two values, each
+// rounded exactly as the scalar instruction would).
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_pack_bits(uint32_t a, uint32_t b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 template <> struct Elem<int8_t> {
   static constexpr int kBytes = 1;
   static constexpr int kEV = 16;
@@ -76,6 +102,33 @@ template <> struct Elem<int8_t> {
         f[4 * i + b] = __uint_as_float(bits) - 8388736.0f;
       }
     }
+  }
+  // The same widening two codes at a time on packed pairs: codes 2j and 2j+1 of v.
+  static __device__ __forceinline__ uint64_t pair(const uint4& v, int j) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const uint32_t u = w[j >> 1] ^ 0x80808080u;
+    const int b = 2 * (j & 1);
+    return f2_add(f2_pack_bits(__byte_perm(u, 0x4B000000u, 0x7440u | b), __byte_perm(u, 0x4B000000u, 0x7440u | (b + 1))),
+                  f2_pack(-8388736.0f, -8388736.0f));
+  }
+  // sum_e q[e] * code[e] over the 16 codes of v; q2 holds q as 8 packed pairs.
+  static __device__ __forceinline__ float dot(const uint4& v, const uint64_t* q2) {
+    uint64_t a0 = 0, a1 = 0;  // two pair accumulators: four partial sums
+#pragma unroll
+    for (int j = 0; j < 8; j += 2) {
+      a0 = f2_fma(q2[j], pair(v, j), a0);
+      a1 = f2_fma(q2[j + 1], pair(v, j + 1), a1);
+    }
+    float x0, x1, x2, x3;
+    f2_unpack(a0, x0, x1);
+    f2_unpack(a1, x2, x3);
+    return (x0 + x1) + (x2 + x3);
+  }
+  // acc[e] += w * code[e] over the 16 codes of v; acc2 holds acc as 8 packed pairs.
+  static __device__ __forceinline__ void axpy(float w, const uint4& v, uint64_t* acc2) {
+    const uint64_t w2 = f2_pack(w, w);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc2[j] = f2_fma(w2, pair(v, j), acc2[j]);
   }
 };
 
