@@ -111,25 +111,6 @@ template <> struct Elem<int8_t> {
     return f2_add(f2_pack_bits(__byte_perm(u, 0x4B000000u, 0x7440u | b), __byte_perm(u, 0x4B000000u, 0x7440u | (b + 1))),
                   f2_pack(-8388736.0f, -8388736.0f));
   }
-  // sum_e q[e] * code[e] over the 16 codes of v; q2 holds q as 8 packed pairs.
-  static __device__ __forceinline__ float dot(const uint4& v, const uint64_t* q2) {
-    uint64_t a0 = 0, a1 = 0;  // two pair accumulators: four partial sums
-#pragma unroll
-    for (int j = 0; j < 8; j += 2) {
-      a0 = f2_fma(q2[j], pair(v, j), a0);
-      a1 = f2_fma(q2[j + 1], pair(v, j + 1), a1);
-    }
-    float x0, x1, x2, x3;
-    f2_unpack(a0, x0, x1);
-    f2_unpack(a1, x2, x3);
-    return (x0 + x1) + (x2 + x3);
-  }
-  // acc[e] += w * code[e] over the 16 codes of v; acc2 holds acc as 8 packed pairs.
-  static __device__ __forceinline__ void axpy(float w, const uint4& v, uint64_t* acc2) {
-    const uint64_t w2 = f2_pack(w, w);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc2[j] = f2_fma(w2, pair(v, j), acc2[j]);
-  }
 };
 
 // OCP FP8 E4M3 codes: the hardware converts pairs to fp16 exactly (every E4M3 value is an
@@ -152,6 +133,28 @@ template <> struct Elem<__nv_fp8_e4m3> {
     }
   }
 };
+
+// Dot product and axpy over the 16 8-bit codes of one 16-byte vector on packed fp32 pairs
+// (Elem<CT>::pair widens two codes).  q2 and acc2 hold 8 packed pairs each.
+template <typename CT>
+__device__ __forceinline__ float dot_pairs(const uint4& v, const uint64_t* q2) {
+  uint64_t a0 = 0, a1 = 0;  // two pair accumulators: four partial sums
+#pragma unroll
+  for (int j = 0; j < 8; j += 2) {
+    a0 = f2_fma(q2[j], Elem<CT>::pair(v, j), a0);
+    a1 = f2_fma(q2[j + 1], Elem<CT>::pair(v, j + 1), a1);
+  }
+  float x0, x1, x2, x3;
+  f2_unpack(a0, x0, x1);
+  f2_unpack(a1, x2, x3);
+  return (x0 + x1) + (x2 + x3);
+}
+template <typename CT>
+__device__ __forceinline__ void axpy_pairs(float w, const uint4& v, uint64_t* acc2) {
+  const uint64_t w2 = f2_pack(w, w);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc2[j] = f2_fma(w2, Elem<CT>::pair(v, j), acc2[j]);
+}
 
 template <typename T> __device__ __forceinline__ T float_to(float x);
 template <> __device__ __forceinline__ float float_to<float>(float x) { return x; }
