@@ -11,9 +11,9 @@
 // and block-table walk (the same page, section "PagedAttention注意力计算流程"); the causal
 // rule is the usual definition and the tiling below is this library's design.
 //
-// One CTA owns 128 query rows of one cached head: tq = 128 / GQ consecutive query tokens
-// times the GQ query heads that share the cached head (row = token * GQ + head).  Per
-// 128-token KV tile:
+// A persistent grid (one CTA per SM) works through units of 128 query rows of one cached
+// head: tq = 128 / GQ consecutive query tokens times the GQ query heads that share the
+// cached head (row = token * GQ + head).  Per 128-token KV tile of a unit:
 //
 //   S[128 rows x 128 kv]  = Q[128 x 128 d] . K^T          (K-major A and B in shared memory)
 //   O_h[128 rows x 128 d] += P[:, 64h..] . V[64h.., :]   (A = P in TMEM over S, MN-major V)
@@ -21,10 +21,10 @@
 // with fp32 accumulators in TMEM.  Keeping P in tensor memory leaves shared memory to the
 // q rows and 3-deep K and V rings.
 //
-// Roles (one CTA per SM, 10 warps):
-//   warp 0      TMA producer: the q rows once, then per tile the attended blocks' K and V
-//               (64-dim halves, 128-byte swizzle) into separate 3-deep K and V rings; block
-//               ids for the next tile are fetched while the current one is issued.
+// Roles (one CTA per SM, 11 warps):
+//   warps 0, 10 TMA producers: K into a 3-deep ring, V and each unit's q rows into another
+//               (64-dim halves, 128-byte swizzle, one copy per lane); block ids are fetched
+//               in prefetched windows.
 //   warp 1      TMEM owner and MMA issuer (one lane), polling: score MMA of the next tile
 //               whose K landed, value MMA of the tile whose probabilities are written.
 //   warps 2..9  softmax, two warps per query row (TMEM lane), each with its own half of
@@ -58,7 +58,7 @@ constexpr int kHalf = 128 * 128;          // one 64-element half of a 128-row op
 constexpr int kOpBytes = 2 * kHalf;       // a whole 128 x 128 operand (Q, K, V or P)
 constexpr int kRing = 3;                  // depth of the K ring and of the V ring
 constexpr int kSoftmaxThreads = 256;   // 8 warps: two per TMEM lane quarter, 64 columns each
-constexpr int kThreads = 160 + kSoftmaxThreads;  // + 4 producer warps and the MMA issuer
+constexpr int kThreads = 96 + kSoftmaxThreads;  // + K producer, MMA issuer, V producer
 constexpr uint32_t kTmemCols = 512;       // S0 [0,128)  S1 [128,256)  O_0 [256,384)  O_1 [384,512)
 // Each softmax half h owns the 64 score columns [64h, 64h+64) of an S buffer and writes its
 // probabilities over them: hi weights in the first 32 columns (two 16-bit weights per
@@ -207,7 +207,7 @@ struct TableWindow {
 };
 
 template <typename IO>
-__global__ void __launch_bounds__(kThreads, 1)  // 13 warps: 4 on one SM sub-partition, 128 registers
+__global__ void __launch_bounds__(kThreads, 1)  // 11 warps: at most 3 per SM sub-partition, 168 registers
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmQ, const PrefillParams p) {
   constexpr bool kSplit = std::is_same<IO, __nv_bfloat16>::value;
@@ -240,9 +240,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     mbar_init(q_empty, 1);
     mbar_init(o_free, kSoftmaxThreads);
     for (int st = 0; st < kRing; ++st) {
-      mbar_init(k_full0 + 8 * st, 2);  // one arrival per producer warp of the tensor
+      mbar_init(k_full0 + 8 * st, 1);
       mbar_init(k_empty0 + 8 * st, 1);
-      mbar_init(v_full0 + 8 * st, 2);
+      mbar_init(v_full0 + 8 * st, 1);
       mbar_init(v_empty0 + 8 * st, 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -262,16 +262,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 
   // Every role walks the same units in the same order; tile counters (ring slots and
   // barrier parities) and unit counters run on across units.
-  if (warp == 0 || warp >= 10) {
+  if (warp == 0 || warp == 10) {
     // ------------------------------------------------------------------ TMA producers --
-    // Four warps: (K, V) x (64-dim half).  A warp issues its copies one per lane, and a
-    // warp's copies go out one after another, so splitting them over four warps issues a
-    // tile four times as fast.  The V-hi warp also loads each unit's q rows once the last
-    // score MMA of the previous unit has read them.  Each warp walks the block table
-    // through its own prefetched window.
-    const int pi = warp == 0 ? 0 : warp - 9;  // 0: K lo, 1: V lo, 2: K hi, 3: V hi
-    const bool is_v = pi & 1;
-    const int dh = pi >> 1;                   // 64-dim half this warp copies
+    // Warp 0 loads K, warp 10 loads V and each unit's q rows (once the last score MMA of the
+    // previous unit has read them), each into its own ring, one copy (a 64-dim half of one
+    // block) per lane.  A warp's copies go out one after another, so two warps issue a tile
+    // twice as fast as one; four warps would be faster still, but 13 warps leave the
+    // softmax 128 registers instead of 168 and measured slower (579 vs 656 TFLOP/s).  Each
+    // warp walks the block table through its own prefetched window.
+    const bool is_v = warp == 10;
+    const int pi = is_v ? 3 : 0;
     const uint64_t keep = l2_policy_evict_last();    // K/V tiles are shared by the sequence's q tiles
     const uint64_t once = l2_policy_evict_first();   // q rows are read once
     const CUtensorMap* map = is_v ? &tmV : &tmK;
@@ -315,12 +315,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
           if (pi == 0) prefill_error(PA_DEVERR_TABLE);
           pb = 0;
         }
-        if (lane == 0) mbar_arrive_expect_tx(full0 + 8 * st, static_cast<uint32_t>(nload) * bs * 128u);
+        if (lane == 0) mbar_arrive_expect_tx(full0 + 8 * st, static_cast<uint32_t>(nload) * 2u * bs * 128u);
         __syncwarp();
-        if (lane < nload) {  // nload <= 16 copies, one per lane
-          const uint32_t row = static_cast<uint32_t>(cur.lo + lane - cur.first) * bs * 128u;
+        const int blk = __shfl_sync(0xffffffffu, pb, (lane >> 1) & 31);
+        if (lane < 2 * nload) {  // 2 * nload <= 32 copies, one per lane
+          const int dh = lane & 1;  // 64-dim half
+          const uint32_t row = static_cast<uint32_t>(cur.lo + (lane >> 1) - cur.first) * bs * 128u;
           const uint32_t dst = (is_v ? sV(st) : sK(st)) + dh * kHalf + row;
-          tma_load_3d(dst, map, full0 + 8 * st, dh * 64, w.kh, pb * bs, keep);
+          tma_load_3d(dst, map, full0 + 8 * st, dh * 64, w.kh, blk * bs, keep);
         }
       }
       ++uq;
