@@ -469,11 +469,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 #pragma unroll
           for (int c = 0; c < 64; ++c) sc[c] = (c >= c_lo && c <= c_hi) ? sc[c] : -INFINITY;
         }
-        float mx[8];  // eight independent chains instead of one 64-long one
+        float mx[8];  // eight independent chains of three-input maxima over columns k + 8i
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = sc[k];
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(sc[k], sc[8 + k]);
 #pragma unroll
-        for (int c = 8; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], sc[c]);
+        for (int c = 16; c < 64; c += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], sc[c + k], sc[c + 8 + k]);
         const float mraw =
             fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
         const float mt = mraw * p.qscale;  // scores in base-2 units (qscale > 0 keeps the order)
@@ -523,25 +525,30 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         // polynomial on the FMA pipe measured slower: the transcendental unit is not what
         // limits this loop.)  The denominator sums the
         // unrounded weights (fp16 rounding errors of the packed weights average out).
-        float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        const float neg_m = -m_run;
+        // The scale-and-subtract and the running sum work on packed fp32 pairs.
+        uint64_t ls2[4] = {0, 0, 0, 0};
+        const uint64_t q2 = f2_pack(p.qscale, p.qscale), nm2 = f2_pack(-m_run, -m_run);
 #pragma unroll
         for (int q = 0; q < 2; ++q) {  // two stores of 16 columns (32 tokens) each
           uint32_t w_hi[16], w_lo[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
             const int c = 32 * q + 2 * k;
-            const float x0 = ex2_ftz(fmaf(sc[c], p.qscale, neg_m));
-            const float x1 = ex2_ftz(fmaf(sc[c + 1], p.qscale, neg_m));
+            float y0, y1;
+            f2_unpack(f2_fma(f2_pack(sc[c], sc[c + 1]), q2, nm2), y0, y1);
+            const float x0 = ex2_ftz(y0), x1 = ex2_ftz(y1);
             const Pair<IO> hi(x0, x1);
             w_hi[k] = hi.bits;
             if (kSplit) w_lo[k] = Pair<IO>(x0 - hi.lo_f(), x1 - hi.hi_f()).bits;
-            ls[k & 7] += x0 + x1;
+            ls2[k & 3] = f2_add(ls2[k & 3], f2_pack(x0, x1));
           }
           tmem_store16_bits(s_col + 16 * q, w_hi);
           if (kSplit) tmem_store16_bits(s_col + 32 + 16 * q, w_lo);
         }
         tmem_wait_store();
+        float ls[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) f2_unpack(ls2[k], ls[2 * k], ls[2 * k + 1]);
         l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         fence_proxy_async_shared();  // zeroed V rows (if any) are read by the tensor core
         tc_fence_before_sync();
