@@ -178,3 +178,31 @@ def test_prefill_llama70b_prompt_batch_sampled(cuda_device):
         last = oracle.paged_prefill(rows[-k:].contiguous(), ks, vs, bt[s:s + 1], one, [n], scale)
         compare(out[s * n:s * n + k][:, heads], first, "fp16", TOL["fp16"])
         compare(out[(s + 1) * n - k:(s + 1) * n][:, heads], last, "fp16", TOL["fp16"])
+
+
+def test_chunked_prefill_workload_sampled(cuda_device):
+    """The chunked-prefill workload's shape: 8 sequences, 512-token chunks behind 1536 cached
+    tokens, 64 heads, bs 16, fp16.  The oracle checks the last 32 query rows of every chunk
+    on 4 heads (a suffix of a chunk is a problem of its own under the causal rule)."""
+    S, qn, cached, H, bs = 8, 512, 1536, 64, 16
+    ctx = qn + cached
+    g = torch.Generator().manual_seed(17)
+    nblk = ctx // bs
+    NB = S * nblk + 32
+    perm = torch.randperm(NB, generator=g)
+    bt = perm[: S * nblk].view(S, nblk).to(torch.int32).contiguous()
+    kc = torch.randn(NB, bs, H, 128, generator=g, dtype=torch.float16)
+    vc = torch.randn(NB, bs, H, 128, generator=g, dtype=torch.float16)
+    q = torch.randn(S * qn, H, 128, generator=g, dtype=torch.float16)
+    cu = torch.arange(0, S * qn + 1, qn, dtype=torch.int32)
+    cl = torch.full((S,), ctx, dtype=torch.int32)
+    scale = 1 / math.sqrt(128)
+    out = run_gpu(q, kc, vc, bt, cu, cl, scale).cpu()
+    assert_no_device_error()
+    heads = [1, 30, 47, 62]
+    ks, vs = kc[:, :, heads].contiguous(), vc[:, :, heads].contiguous()
+    k = 32
+    for s in range(0, S, 3):
+        rows = q[(s + 1) * qn - k:(s + 1) * qn][:, heads].contiguous()
+        ref = oracle.paged_prefill(rows, ks, vs, bt[s:s + 1], torch.tensor([0, k], dtype=torch.int32), [ctx], scale)
+        compare(out[(s + 1) * qn - k:(s + 1) * qn][:, heads], ref, "fp16", TOL["fp16"])
