@@ -47,8 +47,11 @@ constexpr int kStageBytes = 4 * kHalf + 2 * kQHalf;  // K lo, K hi, V lo, V hi, 
 constexpr int kStages = 3;
 constexpr int kPBytes = kTokens * kHeadsN * 2;  // one probability operand, 128 tokens x 16 heads
 constexpr int kPBuffers = 4;                    // 2 tiles in flight x (hi, lo) parts
-constexpr int kThreads = 320;  // TMA warps 0 and 6..8, score-MMA warp 1, softmax warps 2..5, value-MMA warp 9
-static_assert(kThreads <= kMaxPlanThreads, "plan_slice keeps one scratch entry per thread");
+// Threads of the kernel tracking NH query heads per row: TMA warps 0 and 6..8, MMA warps
+// 1 and 9, softmax warps 2..5 (and 10..13 when NH = 16: two warps per TMEM lane quarter,
+// 8 heads each).
+constexpr int threads_for(int nh) { return nh > 8 ? 448 : 320; }
+static_assert(threads_for(16) <= kMaxPlanThreads, "plan_slice keeps one scratch entry per thread");
 constexpr uint32_t kTmemCols = 64;              // S0 [0,16)  S1 [16,32)  O0 [32,48)  O1 [48,64)
 constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + kPBuffers * kPBytes;
 
@@ -86,12 +89,19 @@ __device__ __forceinline__ void store_p_row(uint32_t buf, int r, const uint32_t*
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + 16 * (sw ^ 1)), "r"(w[4]), "r"(w[5]), "r"(w[6]),
                "r"(w[7]) : "memory");
 }
+// Heads 8 * hh .. 8 * hh + 7 of row r only (the other 16-byte chunk belongs to another warp).
+__device__ __forceinline__ void store_p_half_row(uint32_t buf, int r, int hh, const uint32_t* w) {
+  const uint32_t sw = (r >> 2) & 1;
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(buf + r * 32 + 16 * (hh ^ sw)), "r"(w[0]), "r"(w[1]),
+               "r"(w[2]), "r"(w[3]) : "memory");
+}
 
-// IO: fp16 or bf16 cache and queries.  NH: query heads a thread tracks (8 or 16 >= GQ).
+// IO: fp16 or bf16 cache and queries.  NH: query heads of a row (8 or 16 >= GQ); a softmax
+// thread tracks 8 of them.
 // bf16 probabilities are split into hi + lo bf16 parts and the value MMA runs on both, so
 // the weights keep ~16 significant bits (one bf16 part alone keeps 8).
 template <typename IO, int NH>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_for(NH), 1)
 decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmQ, const DecodeParams p) {
   constexpr bool kSplit = std::is_same<IO, __nv_bfloat16>::value;
@@ -130,8 +140,8 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full0 + 8 * b, 1);
-      mbar_init(s_empty0 + 8 * b, 128);
-      mbar_init(p_full0 + 8 * b, 128);
+      mbar_init(s_empty0 + 8 * b, 128 * (NH / 8));
+      mbar_init(p_full0 + 8 * b, 128 * (NH / 8));
       mbar_init(o_full0 + 8 * b, 1);
     }
     mbar_init(smem_u32(&sh.mma_done), 2);
@@ -140,7 +150,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
   }
   // The q rows of a head group fill rows 0..GQ-1 of each stage's 16-row q block; rows
   // GQ..15 stay zero (padding of the MMA N dimension).
-  for (int i = threadIdx.x; i < kStages * 2 * kQHalf / 16; i += kThreads) {
+  for (int i = threadIdx.x; i < kStages * 2 * kQHalf / 16; i += threads_for(NH)) {
     const int st = i / (2 * kQHalf / 16), off = (i % (2 * kQHalf / 16)) * 16;
     uint8_t* ptr = smem_raw + (stage(st) - smem_u32(smem_raw)) + 4 * kHalf + off;
     *reinterpret_cast<uint4*>(ptr) = make_uint4(0, 0, 0, 0);
@@ -313,13 +323,17 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     __syncwarp();
   } else {
     // ------------------------------------------------- softmax + accumulation warps --
-    // (warps 2..5)
+    // (warps 2..5, and 10..13 for the heads 8..15 of a 16-head row)
+    constexpr int HPW = 8;                // query heads a thread tracks
+    constexpr int kSoftmax = 128 * (NH / 8);
     const int q4 = warp & 3;              // TMEM lane quarter this warp may access
+    const int hh = warp >= 10 ? 1 : 0;    // which 8 of the row's heads
+    const int h_base = 8 * hh;
     const int r = 32 * q4 + lane;         // token row (softmax) and head-dim row (accumulate)
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q4) << 16;
-    float m[NH], l[NH], acc[NH], alpha_prev[NH];
+    float m[HPW], l[HPW], acc[HPW], alpha_prev[HPW];
 #pragma unroll
-    for (int h = 0; h < NH; ++h) {
+    for (int h = 0; h < HPW; ++h) {
       m[h] = -FLT_MAX;
       l[h] = 0.f;
       acc[h] = 0.f;
@@ -329,11 +343,11 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     auto accumulate = [&](int t, const float* alpha) -> bool {
       if (!wait_or_abort(o_full0 + 8 * (t % 2), (t / 2) & 1, abort)) return false;
       tc_fence_after_sync();
-      float o[NH];
-      tmem_load<NH>(tmem + lane_addr + 2 * kHeadsN + (t % 2) * kHeadsN, o);
+      float o[HPW];
+      tmem_load<HPW>(tmem + lane_addr + 2 * kHeadsN + (t % 2) * kHeadsN + h_base, o);
       tc_fence_before_sync();
 #pragma unroll
-      for (int h = 0; h < NH; ++h) acc[h] = acc[h] * alpha[h] + o[h];
+      for (int h = 0; h < HPW; ++h) acc[h] = acc[h] * alpha[h] + o[h];
       return true;
     };
     Cursor c = start;
@@ -343,29 +357,30 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       const int b = i % 2, st = i % kStages;
       if (!wait_or_abort(s_full0 + 8 * b, (i / 2) & 1, abort)) break;
       tc_fence_after_sync();
-      float sc[NH];
-      tmem_load<NH>(tmem + lane_addr + b * kHeadsN, sc);
+      float sc[HPW];
+      tmem_load<HPW>(tmem + lane_addr + b * kHeadsN + h_base, sc);
       tc_fence_before_sync();
       mbar_arrive(s_empty0 + 8 * b);
 
       const int tok = (c.sp.first_t + c.j) * kTokens + r;
       const bool valid = tok >= c.sp.lo && tok < c.sp.ctx;
 #pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        sc[h] = (valid && h < GQ) ? sc[h] * p.qscale : -INFINITY;
+      for (int h = 0; h < HPW; ++h) {
+        sc[h] = (valid && h_base + h < GQ) ? sc[h] * p.qscale : -INFINITY;
         float x = sc[h];
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
-        if (lane == 0) sh.red[b][q4][h] = x;
+        if (lane == 0) sh.red[b][q4][h_base + h] = x;
       }
-      named_barrier_sync(1, 128);
-      float alpha[NH];
+      named_barrier_sync(1, kSoftmax);
+      float alpha[HPW];
       uint32_t w_hi[8], w_lo[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) w_hi[k] = w_lo[k] = 0;
 #pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        const float t = fmaxf(fmaxf(sh.red[b][0][h], sh.red[b][1][h]), fmaxf(sh.red[b][2][h], sh.red[b][3][h]));
+      for (int h = 0; h < HPW; ++h) {
+        const int hg = h_base + h;
+        const float t = fmaxf(fmaxf(sh.red[b][0][hg], sh.red[b][1][hg]), fmaxf(sh.red[b][2][hg], sh.red[b][3][hg]));
         const float m_new = fmaxf(m[h], t);
         alpha[h] = exp2f(m[h] - m_new);
         m[h] = m_new;
@@ -380,9 +395,14 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
           l[h] = l[h] * alpha[h] + static_cast<float>(hi);  // the rounded weight the MMA uses
         }
       }
-      store_p_row(pbuf(b, 0), r, w_hi);
-      if (kSplit) store_p_row(pbuf(b, 1), r, w_lo);
-      if (!valid) {  // unattended rows may hold anything (NaN): give the value MMA zeros
+      if (NH > 8) {  // this warp's 16-byte chunk of the 32-byte row
+        store_p_half_row(pbuf(b, 0), r, hh, w_hi);
+        if (kSplit) store_p_half_row(pbuf(b, 1), r, hh, w_lo);
+      } else {       // heads 8..15 of the padded row are zero
+        store_p_row(pbuf(b, 0), r, w_hi);
+        if (kSplit) store_p_row(pbuf(b, 1), r, w_lo);
+      }
+      if (!valid && hh == 0) {  // unattended rows may hold anything (NaN): give the value MMA zeros
         const uint32_t v0 = stage(st) + 2 * kHalf + r * 128;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
@@ -400,13 +420,13 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       if (!(seg_last || i == n - 1)) {
         pending = true;
 #pragma unroll
-        for (int h = 0; h < NH; ++h) alpha_prev[h] = alpha[h];
+        for (int h = 0; h < HPW; ++h) alpha_prev[h] = alpha[h];
       } else {
         if (!accumulate(i, alpha)) break;
         // Softmax denominators: every thread holds the sums of its own token rows.
-        float lt[NH];
+        float lt[HPW];
 #pragma unroll
-        for (int h = 0; h < NH; ++h) {
+        for (int h = 0; h < HPW; ++h) {
           float x = l[h];
 #pragma unroll
           for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
@@ -414,31 +434,35 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         }
         if (lane == 0)
 #pragma unroll
-          for (int h = 0; h < NH; ++h) sh.red_l[q4][h] = lt[h];
-        named_barrier_sync(1, 128);
+          for (int h = 0; h < HPW; ++h) sh.red_l[q4][h_base + h] = lt[h];
+        named_barrier_sync(1, kSoftmax);
 #pragma unroll
-        for (int h = 0; h < NH; ++h) lt[h] = sh.red_l[0][h] + sh.red_l[1][h] + sh.red_l[2][h] + sh.red_l[3][h];
-        named_barrier_sync(1, 128);  // sh.red_l is free again
-        const int h0 = c.g * GQ;
+        for (int h = 0; h < HPW; ++h) {
+          const int hg = h_base + h;
+          lt[h] = sh.red_l[0][hg] + sh.red_l[1][hg] + sh.red_l[2][hg] + sh.red_l[3][hg];
+        }
+        named_barrier_sync(1, kSoftmax);  // sh.red_l is free again
+        const int h0 = c.g * GQ + h_base;
         if (seg_from_start && seg_last) {
           IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(c.s) * p.Hq + h0) * kDim + r;
 #pragma unroll
-          for (int h = 0; h < NH; ++h)
-            if (h < GQ) orow[static_cast<size_t>(h) * kDim] = float_to<IO>(acc[h] / lt[h]);
+          for (int h = 0; h < HPW; ++h)
+            if (h_base + h < GQ) orow[static_cast<size_t>(h) * kDim] = float_to<IO>(acc[h] / lt[h]);
         } else {
           const long long slot = blockIdx.x + static_cast<long long>(c.s) * p.G + c.g;
 #pragma unroll
-          for (int h = 0; h < NH; ++h) {
-            if (h >= GQ) continue;
-            p.ws_acc[(slot * GQ + h) * kDim + r] = acc[h];
+          for (int h = 0; h < HPW; ++h) {
+            const int hg = h_base + h;
+            if (hg >= GQ) continue;
+            p.ws_acc[(slot * GQ + hg) * kDim + r] = acc[h];
             if (r == 0) {
-              p.ws_ml[(slot * GQ + h) * 2 + 0] = m[h];
-              p.ws_ml[(slot * GQ + h) * 2 + 1] = lt[h];
+              p.ws_ml[(slot * GQ + hg) * 2 + 0] = m[h];
+              p.ws_ml[(slot * GQ + hg) * 2 + 1] = lt[h];
             }
           }
         }
 #pragma unroll
-        for (int h = 0; h < NH; ++h) {
+        for (int h = 0; h < HPW; ++h) {
           m[h] = -FLT_MAX;
           l[h] = 0.f;
           acc[h] = 0.f;
@@ -504,7 +528,7 @@ pa_status tc_decode_launch(const CUtensorMap& tmK, const CUtensorMap& tmV, const
   CUtensorMap k = tmK, v = tmV, q = tmQ;
   DecodeParams p = prm;
   void* args[] = {&k, &v, &q, &p};
-  cudaError_t err = launch_dependent(fn, dim3(grid), dim3(kThreads), kSmemBytes, stream, args);
+  cudaError_t err = launch_dependent(fn, dim3(grid), dim3(small ? threads_for(8) : threads_for(16)), kSmemBytes, stream, args);
   if (err != cudaSuccess) return cuda_fail(err, "launching the tensor-core decode kernel");
   return PA_OK;
 }
