@@ -1,4 +1,4 @@
-"""paged_kv_cache_384_b200 -- paged decode attention for NVIDIA B200 (sm_100a).
+"""paged_kv_cache_384_b200 -- paged attention over a block-table KV cache on NVIDIA B200 (sm_100a).
 
 Thin Python binding over ``libpagedattn.so`` (C ABI in ``include/pagedattn.h``).  PyTorch
 only supplies device memory and the current CUDA stream; every step of the computation
@@ -7,14 +7,20 @@ dtypes and devices agree, and pass raw pointers.
 
     decode_workspace_bytes(num_seqs, num_heads, head_dim)
     paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, ...)
+        (grouped-query when the cache has fewer heads than q; tcgen05 kernel for 4-16 query
+        heads per cached head)
+    paged_attention_prefill(out, q, k_cache, v_cache, block_tables, cu_q_lens, context_lens,
+                            max_q_len, scale, window=0)
     reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, ...)
+    reshape_and_cache_quant(k, v, k_cache, v_cache, k_scale_cache, v_scale_cache, slot_mapping)
     copy_blocks(k_cache, v_cache, src_dst_pairs, ...)
+    swap_blocks(src_k, src_v, dst_k, dst_v, src_dst_pairs, ...)   (GPU <-> pinned host pools)
     BlockManager(num_blocks, block_size, free_order=None)
     slot_mapping(block_tables, seq_ids, positions, block_size)
     device_error(clear=True)
 
-Cache layout: [num_blocks, block_size, num_heads, head_dim]; INT8 scales [num_blocks,
-block_size, num_heads] fp16.
+Cache layout: [num_blocks, block_size, num_heads, head_dim]; INT8 / FP8 scales
+[num_blocks, block_size, num_heads] fp16.
 """
 from __future__ import annotations
 
