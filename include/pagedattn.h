@@ -236,7 +236,8 @@ pa_status reshape_and_cache(const void* k, const void* v, void* k_cache, void* v
  *   window) for window > 0, else 0.  q_len == 1 is decode.
  *
  *   out, q         [num_q_tokens, num_q_heads, 128] in dtype (PA_F16 or PA_BF16); the rows of
- *                  sequence s are cu_q_lens[s] .. cu_q_lens[s+1]-1
+ *                  sequence s are cu_q_lens[s] .. cu_q_lens[s+1]-1;
+ *                  num_q_tokens * num_q_heads < 2^31 (else PA_ERR_UNSUPPORTED)
  *   k_cache,       [num_blocks, block_size, num_kv_heads, 128] in dtype
  *   v_cache
  *   block_tables   [num_seqs, max_blocks_per_seq] int32

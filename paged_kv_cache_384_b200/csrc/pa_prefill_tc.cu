@@ -21,17 +21,20 @@
 // with fp32 accumulators in TMEM.  Keeping P in tensor memory leaves shared memory to the
 // q rows and 3-deep K and V rings.
 //
-// Roles (one CTA per SM, 11 warps):
-//   warps 0, 10 TMA producers: K into a 3-deep ring, V and each unit's q rows into another
-//               (64-dim halves, 128-byte swizzle, one copy per lane); block ids are fetched
-//               in prefetched windows.
-//   warp 1      TMEM owner and MMA issuer (one lane), polling: score MMA of the next tile
-//               whose K landed, value MMA of the tile whose probabilities are written.
-//   warps 2..9  softmax, two warps per query row (TMEM lane), each with its own half of
-//               every tile's kv tokens and its own accumulator O_h: scale, causal/window
-//               mask, online softmax in base 2 with a lazily moved reference maximum (O_h is
-//               rescaled only when the half's maximum grows by more than 2^8), probabilities
-//               into TMEM as the A operand; the halves are merged at the end.
+// Roles (one CTA per SM, 16 warps in four warpgroups; registers are moved with setmaxnreg
+// from the copy and MMA warpgroups, 64 each, to the softmax warpgroups, 192 each):
+//   warp 0       TMEM owner and MMA issuer (one lane), polling: score MMA of the next tile
+//                whose K landed, value MMA of the tile whose probabilities are written.
+//   warps 1..3   TMA producers: K (both 64-dim halves, warp 1) into a 3-deep ring, V and
+//                each unit's q rows (lo half warp 2, hi half warp 3) into another (128-byte
+//                swizzle, one copy per lane); block ids are fetched in prefetched windows.
+//                (warps 4..7 idle)
+//   warps 8..15  softmax, two warps per query row (TMEM lane), each with its own half of
+//                every tile's kv tokens and its own accumulator O_h: scale, causal/window
+//                mask, online softmax in base 2 with a lazily moved reference maximum (O_h
+//                is rescaled only when the half's maximum grows by more than 2^8),
+//                probabilities into TMEM as the A operand; the halves are merged when the
+//                unit's rows are written, which happens after the next unit's first tile.
 // bf16 probabilities are split into hi + lo bf16 parts (two value MMAs) so the weights keep
 // ~16 significant bits.  Every wait is bounded; one that gives up raises PA_DEVERR_TIMEOUT
 // and an abort flag that ends the others.
@@ -57,8 +60,14 @@ constexpr int kDim = 128;                 // head_dim
 constexpr int kHalf = 128 * 128;          // one 64-element half of a 128-row operand: 16 KiB
 constexpr int kOpBytes = 2 * kHalf;       // a whole 128 x 128 operand (Q, K, V or P)
 constexpr int kRing = 3;                  // depth of the K ring and of the V ring
-constexpr int kSoftmaxThreads = 256;   // 8 warps: two per TMEM lane quarter, 64 columns each
-constexpr int kThreads = 96 + kSoftmaxThreads;  // + K producer, MMA issuer, V producer
+constexpr int kSoftmaxThreads = 256;      // 8 warps: two per TMEM lane quarter, 64 columns each
+constexpr int kThreads = 256 + kSoftmaxThreads;  // + 4 copy warps, MMA warpgroup
+// Registers: the launch gives every thread 128 (65536 / 512); the copy and MMA warpgroups
+// hand back down to kRegsLow, the softmax warpgroups take kRegsHigh.  The split must add up
+// to the launch's 65536 exactly or less, else the increase waits for ever.
+constexpr int kRegsLaunch = 128, kRegsLow = 64, kRegsHigh = 192;
+static_assert(256 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split exceeds the launch's");
+static_assert(kRegsLow % 8 == 0 && kRegsHigh % 8 == 0, "setmaxnreg counts are multiples of 8");
 constexpr uint32_t kTmemCols = 512;       // S0 [0,128)  S1 [128,256)  O_0 [256,384)  O_1 [384,512)
 // Each softmax half h owns the 64 score columns [64h, 64h+64) of an S buffer and writes its
 // probabilities over them: hi weights in the first 32 columns (two 16-bit weights per
@@ -151,14 +160,14 @@ __device__ __forceinline__ int unit_of(int k) {  // k-th unit of this CTA
 struct Unit {
   int s, kh, q_start, i0, ntok, ctx, p_min, p_max, kv_lo, j_lo, n;
 };
-__device__ __forceinline__ bool unit_at(const PrefillParams& p, int u, Unit* w) {
+// Unit u from its sequence's bounds q_start, q_end (cu_q_lens) and ctx (context_lens);
+// false if the unit holds no query rows.
+__device__ __forceinline__ bool unit_at(const PrefillParams& p, int u, int q_start, int q_end, int ctx, Unit* w) {
   const int qt = p.qtiles - 1 - u % p.qtiles;
   const int g = u / p.qtiles;
   w->kh = g % p.Hkv;
   w->s = g / p.Hkv;
-  const int q_start = __ldg(p.cu_q + w->s);
-  const int q_len = __ldg(p.cu_q + w->s + 1) - q_start;
-  const int ctx = __ldg(p.context_lens + w->s);
+  const int q_len = q_end - q_start;
   if (q_start < 0 || q_len < 0 || q_start + q_len > p.T || q_len > ctx || ctx > p.MB * p.bs || q_len > p.max_q_len) {
     if (threadIdx.x == 0) prefill_error(PA_DEVERR_CONTEXT);
     return false;
@@ -175,6 +184,35 @@ __device__ __forceinline__ bool unit_at(const PrefillParams& p, int u, Unit* w) 
   w->n = w->p_max / kKv - w->j_lo + 1;  // KV tiles
   return true;
 }
+
+// Walks this CTA's units in order.  The sequence bounds of the next candidate are loaded
+// while the current unit is worked on, so moving on rarely waits for memory.
+struct UnitCursor {
+  int k, u, q0, q1, ctx;
+  __device__ __forceinline__ void fetch(const PrefillParams& p) {
+    u = unit_of(k);
+    if (u < p.units) {
+      const int s = u / p.qtiles / p.Hkv;
+      q0 = __ldg(p.cu_q + s);
+      q1 = __ldg(p.cu_q + s + 1);
+      ctx = __ldg(p.context_lens + s);
+    }
+  }
+  __device__ __forceinline__ void start(const PrefillParams& p) {
+    k = 0;
+    fetch(p);
+  }
+  // The next unit holding query rows; false once the list is done.
+  __device__ __forceinline__ bool next(const PrefillParams& p, Unit* w) {
+    while (u < p.units) {
+      const bool has = unit_at(p, u, q0, q1, ctx, w);
+      ++k;
+      fetch(p);
+      if (has) return true;
+    }
+    return false;
+  }
+};
 
 // Block-table entries of one sequence, 32 at a time, one per lane: the window in use and
 // the next one, whose load is in flight while the current one serves.
@@ -206,8 +244,33 @@ struct TableWindow {
   }
 };
 
+// Warps 0..7 (the copy and MMA warpgroups) hold the MMA warp and the copy warps.  A copy
+// warp's role is 4 * tensor + halves (tensor 0 = K, 1 = V; halves: bit 0 the lo 64-dim half,
+// bit 1 the hi half); -1 = none.  Every SM sub-partition (warp % 4) also runs two softmax
+// warps, and those measured ~0.45 us per tile slower when two busy warps (two copy warps,
+// or a copy warp and the MMA warp) shared their sub-partition; the softmax warps gate the
+// value MMA, so the busy warps sit on different sub-partitions: the MMA warp on 0, K (both
+// halves) on 1, V lo on 2, V hi on 3.  Warps 4..7 are idle.
+constexpr int kMmaWarp = 0;
+constexpr int kCopyWarpsK = 1, kCopyWarpsV = 2;  // copy warps per tensor
+__device__ __forceinline__ int copy_role(int warp) {
+  switch (warp) {
+    case 1: return 3;      // K, both halves
+    case 2: return 4 + 1;  // V, lo half
+    case 3: return 4 + 2;  // V, hi half
+    default: return -1;
+  }
+}
+
+template <int N> __device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N> __device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 template <typename IO>
-__global__ void __launch_bounds__(kThreads, 1)  // 11 warps: at most 3 per SM sub-partition, 168 registers
+__global__ void __launch_bounds__(kThreads, 1)  // 16 warps, 128 registers each at launch
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmQ, const PrefillParams p) {
   constexpr bool kSplit = std::is_same<IO, __nv_bfloat16>::value;
@@ -236,13 +299,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   volatile int* abort = &sh.abort;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    mbar_init(q_full, kCopyWarpsV);  // the V copy warps bring the q rows' halves
     mbar_init(q_empty, 1);
     mbar_init(o_free, kSoftmaxThreads);
     for (int st = 0; st < kRing; ++st) {
-      mbar_init(k_full0 + 8 * st, 1);
+      mbar_init(k_full0 + 8 * st, kCopyWarpsK);  // one arrival per copy warp of the tensor
       mbar_init(k_empty0 + 8 * st, 1);
-      mbar_init(v_full0 + 8 * st, 1);
+      mbar_init(v_full0 + 8 * st, kCopyWarpsV);
       mbar_init(v_empty0 + 8 * st, 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -254,182 +317,206 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     sh.abort = 0;
     fence_barrier_init();
   }
-  if (warp == 1) tmem_alloc(smem_u32(&sh.tmem_base), kTmemCols);
+  if (warp == kMmaWarp) tmem_alloc(smem_u32(&sh.tmem_base), kTmemCols);
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = sh.tmem_base;
+  // Each role ends with the CTA-wide barrier of its own (bar.sync 0 from every warp), after
+  // which the MMA warp releases TMEM.  setmaxnreg sits at the top of each role's branch.
+  auto end_barrier = [&]() {
+    tc_fence_before_sync();
+    __syncthreads();
+  };
 
   // Every role walks the same units in the same order; tile counters (ring slots and
   // barrier parities) and unit counters run on across units.
-  if (warp == 0 || warp == 10) {
-    // ------------------------------------------------------------------ TMA producers --
-    // Warp 0 loads K, warp 10 loads V and each unit's q rows (once the last score MMA of the
-    // previous unit has read them), each into its own ring, one copy (a 64-dim half of one
-    // block) per lane.  A warp's copies go out one after another, so two warps issue a tile
-    // twice as fast as one; four warps would be faster still, but 13 warps leave the
-    // softmax 128 registers instead of 168 and measured slower (579 vs 656 TFLOP/s).  Each
-    // warp walks the block table through its own prefetched window.
-    const bool is_v = warp == 10;
-    const int pi = is_v ? 3 : 0;
-    const uint64_t keep = l2_policy_evict_last();    // K/V tiles are shared by the sequence's q tiles
-    const uint64_t once = l2_policy_evict_first();   // q rows are read once
-    const CUtensorMap* map = is_v ? &tmV : &tmK;
-    if (lane == 0) {
-      prefetch_tensormap(map);
-      if (pi == 3) prefetch_tensormap(&tmQ);
-    }
-    const uint32_t full0 = is_v ? v_full0 : k_full0, empty0 = is_v ? v_empty0 : k_empty0;
-    int gt = 0, uq = 0;
-    bool ok = true;
-    for (int k = 0, u = unit_of(0); u < p.units && ok; u = unit_of(++k)) {
+  if (warp < 8) {
+    regs_decrease<kRegsLow>();
+    const int cr = copy_role(warp);
+    if (cr >= 0) {
+      // ------------------------------------------------------------------ TMA producers --
+      // The K warps load their 64-dim halves of K, the V warps those of V and of each unit's
+      // q rows (once the last score MMA of the previous unit has read them), each tensor
+      // into its own ring, one copy (a half of one block) per lane.  A warp's copies go out
+      // one after another (~60 ns each).  Each warp walks the block table through its own
+      // prefetched window.
+      const bool is_v = cr >= 4;
+      const int nh = (cr & 3) == 3 ? 2 : 1;    // halves this warp copies
+      const int h0 = (cr & 3) == 2 ? 1 : 0;    // its first half
+      const uint64_t keep = l2_policy_evict_last();    // K/V tiles are shared by the sequence's q tiles
+      const uint64_t once = l2_policy_evict_first();   // q rows are read once
+      const CUtensorMap* map = is_v ? &tmV : &tmK;
+      if (lane == 0) {
+        prefetch_tensormap(map);
+        if (is_v) prefetch_tensormap(&tmQ);
+      }
+      const uint32_t full0 = is_v ? v_full0 : k_full0, empty0 = is_v ? v_empty0 : k_empty0;
+      int gt = 0, uq = 0;
+      bool ok = true;
+      UnitCursor cur;
+      cur.start(p);
       Unit w;
-      if (!unit_at(p, u, &w)) continue;
-      if (pi == 3) {
-        if (lane == 0) {
-          ok = uq == 0 || wait_or_abort(q_empty, (uq - 1) & 1, abort);
-          if (ok) {
-            mbar_arrive_expect_tx(q_full, kOpBytes);
-            tma_load_3d(sQ, &tmQ, q_full, 0, w.kh * p.GQ, w.q_start + w.i0, once);
-            tma_load_3d(sQ + kHalf, &tmQ, q_full, 64, w.kh * p.GQ, w.q_start + w.i0, once);
+      while (ok && cur.next(p, &w)) {
+        if (is_v) {
+          if (lane == 0) {
+            ok = uq == 0 || wait_or_abort(q_empty, (uq - 1) & 1, abort);
+            if (ok) {
+              mbar_arrive_expect_tx(q_full, nh * kHalf);
+              for (int dh = h0; dh < h0 + nh; ++dh)
+                tma_load_3d(sQ + dh * kHalf, &tmQ, q_full, dh * 64, w.kh * p.GQ, w.q_start + w.i0, once);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+        }
+        TableWindow win;
+        win.init(p.block_tables + static_cast<size_t>(w.s) * p.MB, w.p_max / bs + 1,
+                 tile_blocks(w.j_lo, bs, w.kv_lo, w.p_max).lo, lane);
+        for (int j = 0; j < w.n; ++j, ++gt) {
+          const int st = gt % kRing;
+          bool ready = true;
+          if (lane == 0 && gt >= kRing) ready = wait_or_abort(empty0 + 8 * st, ((gt / kRing) - 1) & 1, abort);
+          if (!__shfl_sync(0xffffffffu, ready, 0)) {
+            ok = false;
+            break;
+          }
+          const TileBlocks tb = tile_blocks(w.j_lo + j, bs, w.kv_lo, w.p_max);
+          const int nload = tb.hi - tb.lo + 1;
+          int pb = win.get(tb.lo, nload, lane);
+          if (lane < nload && (pb < 0 || pb >= p.NB)) {
+            if (!is_v && h0 == 0) prefill_error(PA_DEVERR_TABLE);
+            pb = 0;
+          }
+          if (lane == 0) mbar_arrive_expect_tx(full0 + 8 * st, static_cast<uint32_t>(nh * nload) * bs * 128u);
+          __syncwarp();
+          const int bi = nh == 2 ? lane >> 1 : lane;  // block of this lane's copy
+          const int dh = nh == 2 ? lane & 1 : h0;     // and its 64-dim half
+          const int blk = __shfl_sync(0xffffffffu, pb, bi & 31);
+          if (lane < nh * nload) {  // nh * nload <= 32 copies, one per lane
+            const uint32_t row = static_cast<uint32_t>(tb.lo + bi - tb.first) * bs * 128u;
+            const uint32_t dst = (is_v ? sV(st) : sK(st)) + dh * kHalf + row;
+            tma_load_3d(dst, map, full0 + 8 * st, dh * 64, w.kh, blk * bs, keep);
           }
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
+        ++uq;
       }
-      TableWindow win;
-      win.init(p.block_tables + static_cast<size_t>(w.s) * p.MB, w.p_max / bs + 1,
-               tile_blocks(w.j_lo, bs, w.kv_lo, w.p_max).lo, lane);
-      for (int j = 0; j < w.n; ++j, ++gt) {
-        const int st = gt % kRing;
-        bool ready = true;
-        if (lane == 0 && gt >= kRing) ready = wait_or_abort(empty0 + 8 * st, ((gt / kRing) - 1) & 1, abort);
-        if (!__shfl_sync(0xffffffffu, ready, 0)) {
-          ok = false;
-          break;
-        }
-        const TileBlocks cur = tile_blocks(w.j_lo + j, bs, w.kv_lo, w.p_max);
-        const int nload = cur.hi - cur.lo + 1;
-        int pb = win.get(cur.lo, nload, lane);
-        if (lane < nload && (pb < 0 || pb >= p.NB)) {
-          if (pi == 0) prefill_error(PA_DEVERR_TABLE);
-          pb = 0;
-        }
-        if (lane == 0) mbar_arrive_expect_tx(full0 + 8 * st, static_cast<uint32_t>(nload) * 2u * bs * 128u);
-        __syncwarp();
-        const int blk = __shfl_sync(0xffffffffu, pb, (lane >> 1) & 31);
-        if (lane < 2 * nload) {  // 2 * nload <= 32 copies, one per lane
-          const int dh = lane & 1;  // 64-dim half
-          const uint32_t row = static_cast<uint32_t>(cur.lo + (lane >> 1) - cur.first) * bs * 128u;
-          const uint32_t dst = (is_v ? sV(st) : sK(st)) + dh * kHalf + row;
-          tma_load_3d(dst, map, full0 + 8 * st, dh * 64, w.kh, blk * bs, keep);
-        }
+      if (lane == 0) {  // never leave with copies in flight
+        if (is_v && uq > 0) mbar_wait_bounded(q_full, (uq - 1) & 1);
+        for (int k = gt - kRing < 0 ? 0 : gt - kRing; k < gt; ++k)
+          mbar_wait_bounded(full0 + 8 * (k % kRing), (k / kRing) & 1);
       }
-      ++uq;
-    }
-    if (lane == 0) {  // never leave with copies in flight
-      if (pi == 3 && uq > 0) mbar_wait_bounded(q_full, (uq - 1) & 1);
-      for (int k = gt - kRing < 0 ? 0 : gt - kRing; k < gt; ++k)
-        mbar_wait_bounded(full0 + 8 * (k % kRing), (k / kRing) & 1);
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------- MMA issuer --
-    // Polls without blocking.  Score MMAs run ahead through the unit list (the next
-    // unit's first scores overlap the current unit's last softmax); the value MMA goes
-    // first when both are ready, since the softmax warps wait on it and the next score
-    // MMA reuses its probabilities' columns.
-    if (lane == 0) {
-      struct Side {
-        int k, u, uq, base, n, idx;
-      };
-      auto next_unit = [&](Side& sd) {  // advance to the next unit holding query rows
-        for (sd.u = unit_of(++sd.k); sd.u < p.units; sd.u = unit_of(++sd.k)) {
+      __syncwarp();
+    } else if (warp == kMmaWarp) {
+      // ------------------------------------------------------------------- MMA issuer --
+      // Polls without blocking (a nap when idle measured slower).  Score MMAs run ahead through
+      // the unit list (the next unit's first scores overlap the current unit's last
+      // softmax); the value MMA goes first when both are ready, since the softmax warps wait
+      // on it and the next score MMA reuses its probabilities' columns.
+      if (lane == 0) {
+        struct Side {
+          UnitCursor cur;
+          bool live;
+          int uq, base, n, idx;
+        };
+        auto next_unit = [&](Side& sd) {  // advance to the next unit holding query rows
           Unit w;
-          if (unit_at(p, sd.u, &w)) {
+          sd.live = sd.cur.next(p, &w);
+          if (sd.live) {
             sd.base += sd.n;
             sd.n = w.n;
             sd.idx = 0;
             ++sd.uq;
-            return;
           }
-        }
-      };
-      Side S{-1, 0, -1, 0, 0, 0};
-      next_unit(S);
-      Side P = S;
-      bool q_ready = false;
-      uint32_t idle = 0;
-      while (P.u < p.units) {
-        bool progressed = false;
-        if (P.idx < P.n && P.base + P.idx < S.base + S.idx) {
-          const int t = P.base + P.idx;
-          const int st = t % kRing, b = t % 2;
-          if (mbar_test_wait(p_full0 + 8 * b, (t / 2) & 1) && mbar_test_wait(v_full0 + 8 * st, (t / kRing) & 1) &&
-              (P.idx > 0 || P.uq == 0 || mbar_test_wait(o_free, (P.uq - 1) & 1))) {
-            tc_fence_after_sync();
-#pragma unroll
-            for (int part = 0; part < (kSplit ? 2 : 1); ++part) {
-#pragma unroll
-              for (int kk = 0; kk < kKv / 16; ++kk) {  // O_h += P_h . V_h, 16 kv tokens per MMA
-                const int h = kk / 4;                    // softmax half owning these tokens
-                tc_mma_f16_ts(tmem + kColO + 128 * h, tmem + b * kKv + 64 * h + 32 * part + (kk % 4) * 8,
-                              smem_desc(sV(st) + kk * 2048, kHalf, 1024, kSwizzle128B), kIdescO,
-                              P.idx > 0 || part > 0 || (kk % 4) > 0);
+        };
+        Side S;
+        S.cur.start(p);
+        S.uq = -1;
+        S.base = S.n = S.idx = 0;
+        next_unit(S);
+        Side P = S;
+        bool q_ready = false;
+        uint32_t idle = 0;
+        while (P.live) {
+          bool progressed = false;
+          if (P.idx < P.n && P.base + P.idx < S.base + S.idx) {
+            const int t = P.base + P.idx;
+            const int st = t % kRing, b = t % 2;
+            if (mbar_test_wait(p_full0 + 8 * b, (t / 2) & 1) && mbar_test_wait(v_full0 + 8 * st, (t / kRing) & 1) &&
+                (P.idx > 0 || P.uq == 0 || mbar_test_wait(o_free, (P.uq - 1) & 1))) {
+              tc_fence_after_sync();
+  #pragma unroll
+              for (int part = 0; part < (kSplit ? 2 : 1); ++part) {
+  #pragma unroll
+                for (int kk = 0; kk < kKv / 16; ++kk) {  // O_h += P_h . V_h, 16 kv tokens per MMA
+                  const int h = kk / 4;                    // softmax half owning these tokens
+                  tc_mma_f16_ts(tmem + kColO + 128 * h, tmem + b * kKv + 64 * h + 32 * part + (kk % 4) * 8,
+                                smem_desc(sV(st) + kk * 2048, kHalf, 1024, kSwizzle128B), kIdescO,
+                                P.idx > 0 || part > 0 || (kk % 4) > 0);
+                }
               }
+              tc_commit(o_full0 + 8 * b);
+              tc_commit(v_empty0 + 8 * st);
+              if (++P.idx == P.n) next_unit(P);
+              progressed = true;
             }
-            tc_commit(o_full0 + 8 * b);
-            tc_commit(v_empty0 + 8 * st);
-            if (++P.idx == P.n) next_unit(P);
-            progressed = true;
+          }
+          if (S.live) {
+            const int t = S.base + S.idx;
+            const int st = t % kRing, b = t % 2;
+            if (!q_ready) q_ready = mbar_test_wait(q_full, S.uq & 1);
+            // S(t) lands on P(t - 2): the value MMA that reads it must be issued first.
+            if (q_ready && t - 1 <= P.base + P.idx && mbar_test_wait(k_full0 + 8 * st, (t / kRing) & 1)) {
+              tc_fence_after_sync();
+  #pragma unroll
+              for (int kk = 0; kk < kDim / 16; ++kk) {  // S[b] = Q . K^T, 16 dims per MMA
+                const uint32_t off = (kk / 4) * kHalf + (kk % 4) * 32;
+                tc_mma_f16(tmem + b * kKv, smem_desc(sQ + off, 16, 1024, kSwizzle128B),
+                           smem_desc(sK(st) + off, 16, 1024, kSwizzle128B), kIdescS, kk > 0);
+              }
+              tc_commit(s_full0 + 8 * b);
+              tc_commit(k_empty0 + 8 * st);
+              if (++S.idx == S.n) {
+                tc_commit(q_empty);  // the q rows may be replaced once these MMAs are done
+                q_ready = false;
+                next_unit(S);
+              }
+              progressed = true;
+            }
+          }
+          if (progressed) {
+            idle = 0;
+          } else if (*abort || ++idle > kWaitLimit) {
+            if (!*abort) prefill_error(PA_DEVERR_TIMEOUT);
+            *abort = 1;
+            break;
           }
         }
-        if (S.u < p.units) {
-          const int t = S.base + S.idx;
-          const int st = t % kRing, b = t % 2;
-          if (!q_ready) q_ready = mbar_test_wait(q_full, S.uq & 1);
-          // S(t) lands on P(t - 2): the value MMA that reads it must be issued first.
-          if (q_ready && t - 1 <= P.base + P.idx && mbar_test_wait(k_full0 + 8 * st, (t / kRing) & 1)) {
-            tc_fence_after_sync();
-#pragma unroll
-            for (int kk = 0; kk < kDim / 16; ++kk) {  // S[b] = Q . K^T, 16 dims per MMA
-              const uint32_t off = (kk / 4) * kHalf + (kk % 4) * 32;
-              tc_mma_f16(tmem + b * kKv, smem_desc(sQ + off, 16, 1024, kSwizzle128B),
-                         smem_desc(sK(st) + off, 16, 1024, kSwizzle128B), kIdescS, kk > 0);
-            }
-            tc_commit(s_full0 + 8 * b);
-            tc_commit(k_empty0 + 8 * st);
-            if (++S.idx == S.n) {
-              tc_commit(q_empty);  // the q rows may be replaced once these MMAs are done
-              q_ready = false;
-              next_unit(S);
-            }
-            progressed = true;
-          }
-        }
-        if (progressed) {
-          idle = 0;
-        } else if (*abort || ++idle > 16 * kWaitLimit) {
-          if (!*abort) prefill_error(PA_DEVERR_TIMEOUT);
-          *abort = 1;
-          break;
-        }
+        tc_commit(mma_done);  // every MMA issued above has finished before TMEM is released
+        mbar_wait_bounded(mma_done, 0);
       }
-      tc_commit(mma_done);  // every MMA issued above has finished before TMEM is released
-      mbar_wait_bounded(mma_done, 0);
+      __syncwarp();
     }
-    __syncwarp();
+    end_barrier();
+    if (warp == kMmaWarp) {
+      tc_fence_after_sync();
+      tmem_dealloc(tmem, kTmemCols);
+    }
   } else {
+    regs_increase<kRegsHigh>();
     // ------------------------------------------------------------- softmax warps --
-    // Warps 2..9.  A warp may only touch the TMEM lane quarter (warp % 4); the two warps of
+    // Warps 8..15.  A warp may only touch the TMEM lane quarter (warp % 4); the two warps of
     // a quarter share its 32 query rows and split each tile's kv tokens: half h takes
     // tokens [64h, 64h + 64).  Each half runs its own online softmax (maximum, sum and
     // output accumulator O_h), so the halves never wait for each other within a unit;
-    // they combine at its end.  Both halves step through every unit and both exchange
-    // barriers even after a failed wait (then doing no other work), so neither can leave
-    // the other waiting at a barrier.
+    // they combine when the unit is finished.  A unit is finished (its rows written out)
+    // after the probabilities of the next unit's first tile: that tile never touches O, its
+    // scores are ready early, and by then the unit's last value MMA is long done, so the
+    // softmax warps do not sit idle at unit boundaries.  Both halves finish every unit, with
+    // both exchange barriers, even after a failed wait (then doing no other work), so
+    // neither can leave the other waiting at a barrier.
     const int q4 = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int half = (warp - 8) >> 2;
     const int r = 32 * q4 + lane;  // query row = TMEM lane
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q4) << 16;
     const uint32_t o_col = tmem + lane_addr + kColO + 128 * half;
@@ -439,11 +526,68 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     auto wait_pv = [&](int t) {
       return __all_sync(0xffffffffu, wait_or_abort(o_full0 + 8 * (t % 2), (t / 2) & 1, abort));
     };
-    int gt = 0;
+    // The unit whose rows are still to be written (its last tile is gt - 1): this thread's
+    // maximum and sum, and its output row (token * Hq + head; -1: no query row here).
+    // pend_row == -2: none.
+    float pend_m = 0.f, pend_l = 0.f;
+    int pend_row = -2;
     bool ok = true;
-    for (int k = 0, u = unit_of(0); u < p.units; u = unit_of(++k)) {
-      Unit w;
-      if (!unit_at(p, u, &w)) continue;
+    int gt = 0;
+    auto finish = [&]() {
+      const bool fin = ok && wait_pv(gt - 1);
+      if (half == 1) {
+        sh.xch[0][r] = pend_m;
+        sh.xch[1][r] = pend_l;
+      }
+      named_barrier_sync(pair_bar, 64);
+      float w_me, w_other;  // weights of O_half and O_(1-half) in the output
+      if (half == 0) {
+        const float m1 = sh.xch[0][r], l1 = sh.xch[1][r];
+        const float m_all = fmaxf(pend_m, m1);
+        const float a0 = ex2_ftz(pend_m - m_all), a1 = ex2_ftz(m1 - m_all);
+        const float l_all = pend_l * a0 + l1 * a1;
+        const float inv = pend_row >= 0 && l_all > 0.f ? 1.f / l_all : 0.f;
+        w_me = a0 * inv;
+        w_other = a1 * inv;
+        sh.xch[0][r] = w_other;  // half 1's own weight
+        sh.xch[1][r] = w_me;     // half 1's weight for O_0
+      }
+      named_barrier_sync(pair_bar, 64);
+      if (half == 1) {
+        w_me = sh.xch[0][r];
+        w_other = sh.xch[1][r];
+      }
+      if (fin) {
+        tc_fence_after_sync();
+        const float w0 = half == 0 ? w_me : w_other, w1 = half == 0 ? w_other : w_me;
+        IO* orow = reinterpret_cast<IO*>(p.out) + static_cast<size_t>(pend_row) * kDim + 64 * half;
+#pragma unroll
+        for (int c4 = 0; c4 < 2; ++c4) {  // this warp's 64 head dims, 32 at a time
+          float o0[32], o1[32];
+          tmem_load32(tmem + lane_addr + kColO + 64 * half + 32 * c4, o0);
+          tmem_load32(tmem + lane_addr + kColO + 128 + 64 * half + 32 * c4, o1);
+          if (pend_row >= 0) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint32_t wd[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int c = 8 * v + 2 * e;
+                wd[e] = Pair<IO>(o0[c] * w0 + o1[c] * w1, o0[c + 1] * w0 + o1[c + 1] * w1).bits;
+              }
+              *reinterpret_cast<uint4*>(orow + 32 * c4 + 8 * v) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+            }
+          }
+        }
+        tc_fence_before_sync();
+        mbar_arrive(o_free);  // O_0 and O_1 may now be overwritten by the next unit
+      }
+      pend_row = -2;
+    };
+    UnitCursor cur;
+    cur.start(p);
+    Unit w;
+    while (cur.next(p, &w)) {
       const bool row_valid = tl < w.ntok;
       const int pos = w.p_min + tl;
       const int lo_row = p.window > 0 ? max(0, pos - p.window + 1) : 0;
@@ -553,67 +697,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         fence_proxy_async_shared();  // zeroed V rows (if any) are read by the tensor core
         tc_fence_before_sync();
         mbar_arrive(p_full0 + 8 * b);
+        if (pend_row != -2) finish();  // first tile of this unit done: finish the previous one
       }
-      // ---- unit end: the halves combine (m, l) and write the rows ----
-      const bool fin = ok && wait_pv(gt + w.n - 1);
-      if (half == 1) {
-        sh.xch[0][r] = m_run;
-        sh.xch[1][r] = l;
-      }
-      named_barrier_sync(pair_bar, 64);
-      float w_me, w_other;  // weights of O_half and O_(1-half) in the output
-      if (half == 0) {
-        const float m1 = sh.xch[0][r], l1 = sh.xch[1][r];
-        const float m_all = fmaxf(m_run, m1);
-        const float a0 = ex2_ftz(m_run - m_all), a1 = ex2_ftz(m1 - m_all);
-        const float l_all = l * a0 + l1 * a1;
-        const float inv = row_valid && l_all > 0.f ? 1.f / l_all : 0.f;
-        w_me = a0 * inv;
-        w_other = a1 * inv;
-        sh.xch[0][r] = w_other;  // half 1's own weight
-        sh.xch[1][r] = w_me;     // half 1's weight for O_0
-      }
-      named_barrier_sync(pair_bar, 64);
-      if (half == 1) {
-        w_me = sh.xch[0][r];
-        w_other = sh.xch[1][r];
-      }
-      if (fin) {
-        tc_fence_after_sync();
-        const float w0 = half == 0 ? w_me : w_other, w1 = half == 0 ? w_other : w_me;
-        IO* orow = reinterpret_cast<IO*>(p.out) +
-                   (static_cast<size_t>(w.q_start + w.i0 + tl) * p.Hq + static_cast<size_t>(w.kh) * p.GQ + g) * kDim +
-                   64 * half;
-#pragma unroll
-        for (int c4 = 0; c4 < 2; ++c4) {  // this warp's 64 head dims, 32 at a time
-          float o0[32], o1[32];
-          tmem_load32(tmem + lane_addr + kColO + 64 * half + 32 * c4, o0);
-          tmem_load32(tmem + lane_addr + kColO + 128 + 64 * half + 32 * c4, o1);
-          if (row_valid) {
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint32_t wd[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int c = 8 * v + 2 * e;
-                wd[e] = Pair<IO>(o0[c] * w0 + o1[c] * w1, o0[c + 1] * w0 + o1[c + 1] * w1).bits;
-              }
-              *reinterpret_cast<uint4*>(orow + 32 * c4 + 8 * v) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-            }
-          }
-        }
-        tc_fence_before_sync();
-        mbar_arrive(o_free);  // O_0 and O_1 may now be overwritten by the next unit
-      }
+      if (pend_row != -2) finish();  // the tile loop ended early (a failed wait)
+      pend_m = m_run;
+      pend_l = l;
+      pend_row = row_valid ? (w.q_start + w.i0 + tl) * p.Hq + w.kh * p.GQ + g : -1;
       gt += w.n;
     }
-  }
-
-  tc_fence_before_sync();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after_sync();
-    tmem_dealloc(tmem, kTmemCols);
+    if (pend_row != -2) finish();
+    end_barrier();
   }
 }
 
@@ -667,6 +760,8 @@ extern "C" pa_status paged_attention_prefill(void* out, const void* q, const voi
     return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: at most 65535 sequences and cached heads");
   if (static_cast<long long>(max_blocks_per_seq) * block_size > (1LL << 30))
     return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: max_blocks_per_seq * block_size too large");
+  if (static_cast<long long>(num_q_tokens) * num_q_heads >= (1LL << 31))
+    return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: num_q_tokens * num_q_heads must be below 2^31");
 
   EncodeTiledFn enc = nullptr;
   pa_status st = get_encoder(&enc);
@@ -715,11 +810,19 @@ extern "C" pa_status paged_attention_prefill(void* out, const void* q, const voi
                         : reinterpret_cast<const void*>(&prefill_tc_kernel<__half>);
   const size_t smem = kSmemBytes;
   static std::once_flag once[2];
+  static int launch_regs[2] = {0, 0};
   cudaError_t attr_err = cudaSuccess;
   std::call_once(once[bf16 ? 1 : 0], [&] {
     attr_err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    cudaFuncAttributes fa;
+    if (attr_err == cudaSuccess) attr_err = cudaFuncGetAttributes(&fa, fn);
+    if (attr_err == cudaSuccess) launch_regs[bf16 ? 1 : 0] = fa.numRegs;
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(prefill)");
+  // The warpgroups' register split (setmaxnreg) adds up to exactly what a 128-register
+  // launch provides; with any other allocation the kernel is not launched.
+  if (launch_regs[bf16 ? 1 : 0] != kRegsLaunch)
+    return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: kernel built with an unexpected register count");
   const long long units = static_cast<long long>(num_seqs) * num_kv_heads * prm.qtiles;
   if (units > (1LL << 30)) return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: too many query tiles");
   prm.units = static_cast<int>(units);
