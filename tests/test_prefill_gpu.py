@@ -206,3 +206,15 @@ def test_chunked_prefill_workload_sampled(cuda_device):
         rows = q[(s + 1) * qn - k:(s + 1) * qn][:, heads].contiguous()
         ref = oracle.paged_prefill(rows, ks, vs, bt[s:s + 1], torch.tensor([0, k], dtype=torch.int32), [ctx], scale)
         compare(out[(s + 1) * qn - k:(s + 1) * qn][:, heads], ref, "fp16", TOL["fp16"])
+
+
+@pytest.mark.parametrize("window", [0, 40])
+def test_prefill_many_short_units_per_cta(cuda_device, window):
+    """More units than SMs, most of them one KV tile: every CTA walks several units, so a
+    unit's rows are written while the next unit's first tile is in flight, and the q rows,
+    output accumulators and score buffers change hands across units many times."""
+    g = np.random.default_rng(19)
+    S = 420
+    ql = g.integers(1, 4, size=S).tolist()
+    ctx = [q + int(g.integers(0, 300)) for q in ql]
+    check(20 + window, ctx, ql, 4, 2, 16, "fp16", window)
