@@ -77,9 +77,9 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_traffic(kernel_source: str):
-    """ncu DRAM bytes per launch of the partition kernel, if captured for this exact source."""
-    path = os.path.join(ROOT, "profiles", "decode_partition_traffic.json")
+def kernel_traffic(kernel_source: str, record: str = "decode_partition_traffic.json", workload: str = None):
+    """ncu DRAM bytes per launch of a kernel, if captured for this exact source and workload."""
+    path = os.path.join(ROOT, "profiles", record)
     try:
         with open(path) as f:
             rec = json.load(f)
@@ -87,7 +87,7 @@ def kernel_traffic(kernel_source: str):
         return None
     with open(kernel_source, "rb") as f:
         sha = hashlib.sha256(f.read()).hexdigest()
-    if rec.get("source_sha256") != sha or rec.get("workload") != PRESET:
+    if rec.get("source_sha256") != sha or rec.get("workload") != (PRESET if workload is None else workload):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -664,7 +664,9 @@ def run_prefill(args):
                    "l2": "K/V and q per step larger than L2, no flush"},
         "tokens_per_s": round(T / sec, 1),
         "roofline": {"bound": "tensor", "achieved": round(flops / attn_sec / 1e12, 2), "peak": peak,
-                     "unit": "TFLOP/s", "frac": round(flops / attn_sec / 1e12 / peak, 4), "traffic": None,
+                     "unit": "TFLOP/s", "frac": round(flops / attn_sec / 1e12 / peak, 4),
+                     "traffic": kernel_traffic(os.path.join(ROOT, "paged_kv_cache_384_b200", "csrc", "pa_prefill_tc.cu"),
+                                               "prefill_tc_traffic.json", args.workload),
                      "peak_source": "measured (cuBLAS bf16 burst)", "kernel": "prefill_tc_kernel",
                      "kernel_ms": round(1e3 * attn_sec, 4)},
         "cpu_baseline": None,
