@@ -27,7 +27,6 @@ template <> struct Elem<float> {
     f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
     f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
   }
-  static __device__ __forceinline__ float from_float_store(float x) { return x; }
 };
 
 template <> struct Elem<__half> {
