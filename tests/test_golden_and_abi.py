@@ -161,6 +161,7 @@ def test_prefill_host_validation(L):
     assert call(ptr=24) == 1            # not 16-byte aligned
     assert call(T=0) == 0               # nothing to do
     assert call(mq=0) == 0
+    assert call(T=1 << 28) == 2         # T * Hq = 2^31: output row indices would overflow
     assert L.pa_last_error().decode()
 
 
