@@ -180,3 +180,25 @@ def test_swap_host_validation(L):
     assert call(n=70000) == 2                            # more pairs than one launch takes
     assert call(n=0) == 0                                # nothing to do
 
+
+
+def test_prefill_binding_refuses_before_any_launch():
+    """The Python binding only marshals: tensors that are not dense CUDA tensors of the right
+    shapes and dtypes are refused on the host (there is no CPU path to fall back to)."""
+    import torch
+    import paged_kv_cache_384_b200 as pa
+    T, Hq, Hkv, D, S, NB, bs = 8, 4, 2, 128, 2, 4, 16
+    q = torch.zeros(T, Hq, D, dtype=torch.float16)
+    kc = torch.zeros(NB, bs, Hkv, D, dtype=torch.float16)
+    bt = torch.zeros(S, 2, dtype=torch.int32)
+    cu = torch.tensor([0, 4, 8], dtype=torch.int32)
+    cl = torch.tensor([4, 4], dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        pa.paged_attention_prefill(torch.empty_like(q), q, kc, kc.clone(), bt, cu, cl, 4, 0.1)
+    with pytest.raises(ValueError, match="one dtype"):
+        pa.paged_attention_prefill(torch.empty_like(q, dtype=torch.bfloat16), q, kc, kc.clone(), bt, cu, cl, 4, 0.1)
+    with pytest.raises(ValueError, match="q's dtype"):
+        pa.paged_attention_prefill(torch.empty_like(q), q, kc.to(torch.bfloat16), kc.to(torch.bfloat16), bt, cu, cl,
+                                   4, 0.1)
+    with pytest.raises(ValueError, match="int32"):
+        pa.paged_attention_prefill(torch.empty_like(q), q, kc, kc.clone(), bt, cu.long(), cl, 4, 0.1)
