@@ -608,8 +608,7 @@ def run_prefill(args):
     out = torch.empty_like(q)
     scale = 1 / math.sqrt(D)
     stream = torch.cuda.current_stream(device)
-    attended = sum(p + 1 for p in range(cached, ctx))  # causal, no window: position p sees p + 1 tokens
-    flops = 4.0 * D * Hq * S * attended
+    flops = accounting.prefill_flops([ctx] * S, [qn] * S, Hq, D)  # causal: position p sees p + 1 tokens
 
     def attn():
         pa.paged_attention_prefill(out, q, kc, vc, bt, cu, cl, qn, scale, stream=stream)

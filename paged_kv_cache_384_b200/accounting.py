@@ -48,3 +48,15 @@ def decode_kv_bytes(context_lens: Iterable[int], num_heads: int, head_dim: int, 
     if cache_dtype in ("int8", "fp8"):
         total += tokens * num_heads * 2 * 2  # one fp16 scale per (token, head) for K and for V
     return total
+
+
+def prefill_flops(context_lens: Iterable[int], q_lens: Iterable[int], num_q_heads: int, head_dim: int,
+                  window: int = 0) -> float:
+    """Algorithmic FLOPs of one prefill call: query i of a sequence with ctx tokens and q_len
+    queries sits at position p = ctx - q_len + i and attends p + 1 tokens (at most ``window``),
+    each costing 4 * head_dim FLOPs (one multiply-add in QK^T and one in PV)."""
+    rows = 0
+    for ctx, ql in zip(context_lens, q_lens):
+        first = int(ctx) - int(ql)
+        rows += sum(attended_tokens(p + 1, window) for p in range(first, int(ctx)))
+    return 4.0 * head_dim * num_q_heads * rows

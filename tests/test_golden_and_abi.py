@@ -202,3 +202,20 @@ def test_prefill_binding_refuses_before_any_launch():
                                    4, 0.1)
     with pytest.raises(ValueError, match="int32"):
         pa.paged_attention_prefill(torch.empty_like(q), q, kc, kc.clone(), bt, cu.long(), cl, 4, 0.1)
+
+
+def test_prefill_flop_count():
+    """4 * head_dim FLOPs per (query row, attended token): a whole prompt of n tokens attends
+    n(n+1)/2 tokens per head; a chunk behind cached context attends the suffix of that sum;
+    a window caps every row; and the count equals a brute-force walk of the causal mask."""
+    D, H = 128, 3
+    assert accounting.prefill_flops([5], [5], H, D) == 4 * D * H * 15
+    assert accounting.prefill_flops([8], [3], H, D) == 4 * D * H * (6 + 7 + 8)
+    assert accounting.prefill_flops([8], [3], H, D, window=4) == 4 * D * H * 12
+    ctx, ql, window = [9, 4, 17], [4, 4, 1], 6
+    brute = 0
+    for c, q in zip(ctx, ql):
+        for i in range(q):
+            pos = c - q + i
+            brute += sum(1 for tok in range(c) if tok <= pos and pos - tok < window)
+    assert accounting.prefill_flops(ctx, ql, H, D, window) == 4 * D * H * brute
