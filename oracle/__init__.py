@@ -43,13 +43,13 @@ def _load():
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
             ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-            ctypes.c_int, ctypes.c_double, ctypes.c_int]
+            ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_int]
         lib.orc_paged_prefill.restype = ctypes.c_int
         lib.orc_paged_prefill.argtypes = [
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
             ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
             ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-            ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int]
+            ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_int]
         lib.orc_f16_to_f64.restype = ctypes.c_double
         lib.orc_f16_to_f64.argtypes = [ctypes.c_uint16]
         lib.orc_bf16_to_f64.restype = ctypes.c_double
@@ -106,13 +106,27 @@ def _u16(x):
     return np.ascontiguousarray(np.asarray(x, dtype=np.float16)).view(np.uint16)
 
 
+def available_cores() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _threads(threads):
+    return available_cores() if threads is None else max(1, int(threads))
+
+
 def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, window=0,
-                 k_scale=None, v_scale=None):
+                 k_scale=None, v_scale=None, threads=None):
     """Decode attention of one query token per sequence over a paged KV cache.
 
     q [S,Hq,D]; k_cache/v_cache [NB,bs,Hkv,D] with Hq a multiple of Hkv (grouped-query:
     query head h reads cached head h // (Hq // Hkv)); block_tables [S,MB] int; context_lens [S];
     k_scale/v_scale [NB,bs,H] fp16 for an int8 or fp8 (torch.float8_e4m3fn) cache.  Returns fp64 numpy [S,H,D].
+    ``threads``: worker threads sharing the independent (sequence, head) pairs (default: every
+    core this process may use); the result is bit-identical for any count.
     """
     lib = _load()
     qa, qd = _raw(q)
@@ -138,20 +152,21 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, window=
     st = lib.orc_paged_decode_gqa(
         out.ctypes.data, qa.ctypes.data, qd, ka.ctypes.data, va.ctypes.data, kd,
         ks.ctypes.data if ks is not None else None, vs.ctypes.data if vs is not None else None,
-        bt.ctypes.data, cl.ctypes.data, S, H, Hc, D, bs, MB, NB, float(scale), int(window))
+        bt.ctypes.data, cl.ctypes.data, S, H, Hc, D, bs, MB, NB, float(scale), int(window), _threads(threads))
     if st != 0:
         raise ValueError(f"oracle: {_STATUS.get(st, st)}")
     return out
 
 
 def paged_prefill(q, k_cache, v_cache, block_tables, cu_q, context_lens, scale, window=0,
-                  k_scale=None, v_scale=None):
+                  k_scale=None, v_scale=None, threads=None):
     """Causal attention of each sequence's newest q_len tokens over a paged KV cache.
 
     q [T,Hq,D] packs the sequences' query tokens (sequence s owns rows cu_q[s]..cu_q[s+1]-1);
     the chunk's own K/V are already in the cache, so query i of sequence s sits at position
     context_lens[s] - q_len + i and attends up to itself (the last ``window`` tokens if
-    window > 0).  Other arguments as for ``paged_decode``.  Returns fp64 numpy [T,Hq,D].
+    window > 0).  Other arguments as for ``paged_decode`` (threads share the independent
+    (sequence, cached head) pairs).  Returns fp64 numpy [T,Hq,D].
     """
     lib = _load()
     qa, qd = _raw(q)
@@ -181,7 +196,8 @@ def paged_prefill(q, k_cache, v_cache, block_tables, cu_q, context_lens, scale, 
     st = lib.orc_paged_prefill(
         out.ctypes.data, qa.ctypes.data, qd, ka.ctypes.data, va.ctypes.data, kd,
         ks.ctypes.data if ks is not None else None, vs.ctypes.data if vs is not None else None,
-        bt.ctypes.data, cu.ctypes.data, cl.ctypes.data, S, H, Hc, D, bs, MB, NB, float(scale), int(window))
+        bt.ctypes.data, cu.ctypes.data, cl.ctypes.data, S, H, Hc, D, bs, MB, NB, float(scale), int(window),
+        _threads(threads))
     if st != 0:
         raise ValueError(f"oracle: {_STATUS.get(st, st)}")
     return out

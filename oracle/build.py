@@ -1,7 +1,8 @@
 """Compile the fp64 oracle (``pa_oracle.c``) into ``liboracle.so`` with gcc.
 
 Test infrastructure only: the product library never links or loads the result.
-Plain ``-O2``, no fast-math, so ``exp`` and the fp64 arithmetic stay IEEE.
+Plain ``-O2``, no fast-math, so ``exp`` and the fp64 arithmetic stay IEEE; ``-pthread``
+for the worker threads that share out independent (sequence, head) items.
 """
 import os
 import subprocess
@@ -16,7 +17,7 @@ def build(force: bool = False) -> str:
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math", SRC, "-o", tmp, "-lm"]
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math", "-pthread", SRC, "-o", tmp, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
     return LIB

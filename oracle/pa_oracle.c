@@ -38,8 +38,13 @@
  *   4. m = max_i score_i;  p_i = exp(score_i - m) / sum_j exp(score_j - m).
  *   5. out[d] = sum_i p_i * Vc[i][d].
  *   ctx == 0 (nothing to attend): out = 0.
+ *
+ * The (sequence, head) pairs are independent, so a caller may spread them over threads;
+ * each pair is still computed by the same loops in the same order (see run_items).
  */
 #include <math.h>
+#include <pthread.h>
+#include <stdatomic.h>
 #include <stddef.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -103,6 +108,92 @@ static double load_value(const void* base, int dtype, size_t index) {
   }
 }
 
+
+/* ---------------------------------------------------------------------------------------
+ * Work items and threads.
+ *
+ * Every output row of the decode oracle depends on one (sequence, query head) pair only,
+ * and every output row of the prefill oracle on one (sequence, key/value head) pair, so
+ * these pairs are independent "items".  Each item is computed by exactly the same loops,
+ * in the same order, whether one thread runs every item or several threads share them;
+ * the result is therefore bit-identical for any thread count.  Threads take the next
+ * unclaimed item from a shared counter.  When items fail, the status returned is that of
+ * the lowest-numbered failing item, as a single thread walking the items in order would
+ * have stopped there first.
+ * ------------------------------------------------------------------------------------- */
+typedef struct {
+  double* Kc;    /* [max_ctx][D] gathered keys   */
+  double* Vc;    /* [max_ctx][D] gathered values */
+  double* score; /* [max_ctx]                    */
+  double* qv;    /* [D]                          */
+} scratch_t;
+
+typedef int (*item_fn)(const void* job, long item, scratch_t* buf);
+
+typedef struct {
+  const void* job;
+  item_fn fn;
+  long n_items;
+  int max_ctx, D;
+  atomic_long next;
+  pthread_mutex_t lock;
+  long bad_item; /* lowest failing item so far, or n_items */
+  int bad_status;
+} runner_t;
+
+static void* run_worker(void* arg) {
+  runner_t* r = (runner_t*)arg;
+  scratch_t b;
+  b.Kc = (double*)malloc(sizeof(double) * (size_t)r->max_ctx * r->D);
+  b.Vc = (double*)malloc(sizeof(double) * (size_t)r->max_ctx * r->D);
+  b.score = (double*)malloc(sizeof(double) * (size_t)r->max_ctx);
+  b.qv = (double*)malloc(sizeof(double) * (size_t)r->D);
+  if (!b.Kc || !b.Vc || !b.score || !b.qv) {
+    pthread_mutex_lock(&r->lock);
+    if (r->bad_item > 0) { r->bad_item = 0; r->bad_status = ORC_NO_MEMORY; }
+    pthread_mutex_unlock(&r->lock);
+  } else {
+    for (;;) {
+      long item = atomic_fetch_add(&r->next, 1);
+      if (item >= r->n_items) break;
+      int st = r->fn(r->job, item, &b);
+      if (st != ORC_OK) {
+        pthread_mutex_lock(&r->lock);
+        if (item < r->bad_item) { r->bad_item = item; r->bad_status = st; }
+        pthread_mutex_unlock(&r->lock);
+      }
+    }
+  }
+  free(b.Kc); free(b.Vc); free(b.score); free(b.qv);
+  return NULL;
+}
+
+/* Run items 0 .. n_items-1 of `job` on `threads` threads (the caller's thread is one). */
+static int run_items(const void* job, item_fn fn, long n_items, int max_ctx, int D, int threads) {
+  runner_t r;
+  r.job = job;
+  r.fn = fn;
+  r.n_items = n_items;
+  r.max_ctx = max_ctx;
+  r.D = D;
+  atomic_init(&r.next, 0);
+  pthread_mutex_init(&r.lock, NULL);
+  r.bad_item = n_items;
+  r.bad_status = ORC_OK;
+  if (threads < 1) threads = 1;
+  if (threads > n_items) threads = n_items > 0 ? (int)n_items : 1;
+  pthread_t* tid = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)threads);
+  int started = 0;
+  if (tid)
+    for (; started < threads - 1; ++started)
+      if (pthread_create(&tid[started], NULL, run_worker, &r) != 0) break;
+  run_worker(&r);
+  for (int i = 0; i < started; ++i) pthread_join(tid[i], NULL);
+  free(tid);
+  pthread_mutex_destroy(&r.lock);
+  return r.bad_status;
+}
+
 /*
  * Paged decode attention, one query token per sequence.  Grouped-query attention (not on
  * the pages; the usual definition): query head h reads key/value head h / (Hq / Hkv), so
@@ -116,88 +207,89 @@ static double load_value(const void* base, int dtype, size_t index) {
  *   v_scale
  *   block_tables [S, MB] int32; only entries of blocks that hold attended tokens are read
  *   context_lens [S] int32
+ *   threads      worker threads (>= 1); the result does not depend on it
  */
+typedef struct {
+  double* out;
+  const void *q, *k_cache, *v_cache;
+  int q_dtype, cache_dtype;
+  const uint16_t *k_scale, *v_scale;
+  const int32_t *block_tables, *context_lens;
+  int S, Hq, Hkv, D, bs, MB, NB, window;
+  double scale;
+} decode_job;
+
+/* One item: sequence s = item / Hq, query head h = item % Hq. */
+static int decode_item(const void* jp, long item, scratch_t* b) {
+  const decode_job* j = (const decode_job*)jp;
+  const int s = (int)(item / j->Hq), h = (int)(item % j->Hq);
+  const int D = j->D, bs = j->bs;
+  const int group = j->Hq / j->Hkv; /* query heads sharing one key/value head */
+  const int ctx = j->context_lens[s];
+  if (ctx < 0 || ctx > j->MB * bs) return ORC_BAD_CONTEXT;
+  int lo = 0;
+  if (j->window > 0 && ctx > j->window) lo = ctx - j->window;
+  const int n = ctx - lo;
+  double* o = j->out + ((size_t)s * j->Hq + h) * D;
+  if (n == 0) {
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    return ORC_OK;
+  }
+
+  /* step 2: gather through the block table */
+  for (int i = lo; i < ctx; ++i) {
+    int logical_block = i / bs;
+    int offset = i % bs;
+    int32_t pb = j->block_tables[(size_t)s * j->MB + logical_block];
+    if (pb < 0 || pb >= j->NB) return ORC_BAD_TABLE;
+    size_t row = ((size_t)pb * bs + offset) * j->Hkv + h / group; /* (pb*bs+off)*Hkv + kv head */
+    double ks = 1.0, vs = 1.0;
+    if (j->cache_dtype == ORC_I8 || j->cache_dtype == ORC_FP8) {
+      ks = orc_f16_to_f64(j->k_scale[row]);
+      vs = orc_f16_to_f64(j->v_scale[row]);
+    }
+    for (int d = 0; d < D; ++d) {
+      b->Kc[(size_t)(i - lo) * D + d] = load_value(j->k_cache, j->cache_dtype, row * D + d) * ks;
+      b->Vc[(size_t)(i - lo) * D + d] = load_value(j->v_cache, j->cache_dtype, row * D + d) * vs;
+    }
+  }
+
+  for (int d = 0; d < D; ++d) b->qv[d] = load_value(j->q, j->q_dtype, ((size_t)s * j->Hq + h) * D + d);
+
+  /* step 3: scaled dot products */
+  for (int i = 0; i < n; ++i) {
+    double dot = 0.0;
+    for (int d = 0; d < D; ++d) dot += b->qv[d] * b->Kc[(size_t)i * D + d];
+    b->score[i] = j->scale * dot;
+  }
+
+  /* step 4: textbook softmax */
+  double m = b->score[0];
+  for (int i = 1; i < n; ++i) if (b->score[i] > m) m = b->score[i];
+  double z = 0.0;
+  for (int i = 0; i < n; ++i) { b->score[i] = exp(b->score[i] - m); z += b->score[i]; }
+  for (int i = 0; i < n; ++i) b->score[i] /= z;
+
+  /* step 5: probability-weighted sum of the value rows */
+  for (int d = 0; d < D; ++d) {
+    double acc = 0.0;
+    for (int i = 0; i < n; ++i) acc += b->score[i] * b->Vc[(size_t)i * D + d];
+    o[d] = acc;
+  }
+  return ORC_OK;
+}
+
 int orc_paged_decode_gqa(double* out, const void* q, int q_dtype, const void* k_cache,
                          const void* v_cache, int cache_dtype, const uint16_t* k_scale,
                          const uint16_t* v_scale, const int32_t* block_tables,
                          const int32_t* context_lens, int S, int Hq, int Hkv, int D, int bs, int MB,
-                         int NB, double scale, int window) {
+                         int NB, double scale, int window, int threads) {
   if (S < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || D <= 0 || bs <= 0 || MB <= 0 || NB <= 0)
     return ORC_BAD_ARG;
-  const int group = Hq / Hkv; /* query heads sharing one key/value head */
   if ((cache_dtype == ORC_I8 || cache_dtype == ORC_FP8) && (!k_scale || !v_scale)) return ORC_BAD_ARG;
-
-  int max_ctx = MB * bs;
-  double* Kc = (double*)malloc(sizeof(double) * (size_t)max_ctx * D);
-  double* Vc = (double*)malloc(sizeof(double) * (size_t)max_ctx * D);
-  double* score = (double*)malloc(sizeof(double) * (size_t)max_ctx);
-  double* qv = (double*)malloc(sizeof(double) * (size_t)D);
-  if (!Kc || !Vc || !score || !qv) {
-    free(Kc); free(Vc); free(score); free(qv);
-    return ORC_NO_MEMORY;
-  }
-  int status = ORC_OK;
-
-  for (int s = 0; s < S && status == ORC_OK; ++s) {
-    int ctx = context_lens[s];
-    if (ctx < 0 || ctx > max_ctx) { status = ORC_BAD_CONTEXT; break; }
-    int lo = 0;
-    if (window > 0 && ctx > window) lo = ctx - window;
-    int n = ctx - lo;
-
-    for (int h = 0; h < Hq && status == ORC_OK; ++h) {
-      double* o = out + ((size_t)s * Hq + h) * D;
-      if (n == 0) {
-        for (int d = 0; d < D; ++d) o[d] = 0.0;
-        continue;
-      }
-
-      /* step 2: gather through the block table */
-      for (int i = lo; i < ctx; ++i) {
-        int logical_block = i / bs;
-        int offset = i % bs;
-        int32_t pb = block_tables[(size_t)s * MB + logical_block];
-        if (pb < 0 || pb >= NB) { status = ORC_BAD_TABLE; break; }
-        size_t row = ((size_t)pb * bs + offset) * Hkv + h / group; /* (pb*bs+off)*Hkv + kv head */
-        double ks = 1.0, vs = 1.0;
-        if (cache_dtype == ORC_I8 || cache_dtype == ORC_FP8) {
-          ks = orc_f16_to_f64(k_scale[row]);
-          vs = orc_f16_to_f64(v_scale[row]);
-        }
-        for (int d = 0; d < D; ++d) {
-          Kc[(size_t)(i - lo) * D + d] = load_value(k_cache, cache_dtype, row * D + d) * ks;
-          Vc[(size_t)(i - lo) * D + d] = load_value(v_cache, cache_dtype, row * D + d) * vs;
-        }
-      }
-      if (status != ORC_OK) break;
-
-      for (int d = 0; d < D; ++d) qv[d] = load_value(q, q_dtype, ((size_t)s * Hq + h) * D + d);
-
-      /* step 3: scaled dot products */
-      for (int i = 0; i < n; ++i) {
-        double dot = 0.0;
-        for (int d = 0; d < D; ++d) dot += qv[d] * Kc[(size_t)i * D + d];
-        score[i] = scale * dot;
-      }
-
-      /* step 4: textbook softmax */
-      double m = score[0];
-      for (int i = 1; i < n; ++i) if (score[i] > m) m = score[i];
-      double z = 0.0;
-      for (int i = 0; i < n; ++i) { score[i] = exp(score[i] - m); z += score[i]; }
-      for (int i = 0; i < n; ++i) score[i] /= z;
-
-      /* step 5: probability-weighted sum of the value rows */
-      for (int d = 0; d < D; ++d) {
-        double acc = 0.0;
-        for (int i = 0; i < n; ++i) acc += score[i] * Vc[(size_t)i * D + d];
-        o[d] = acc;
-      }
-    }
-  }
-
-  free(Kc); free(Vc); free(score); free(qv);
-  return status;
+  decode_job j = {out, q, k_cache, v_cache, q_dtype, cache_dtype, k_scale, v_scale,
+                  block_tables, context_lens, S, Hq, Hkv, D, bs, MB, NB, window, scale};
+  return run_items(&j, decode_item, (long)S * Hq, MB * bs, D, threads);
 }
 
 /* Multi-head decode: every query head has its own cached key/value head. */
@@ -207,7 +299,7 @@ int orc_paged_decode(double* out, const void* q, int q_dtype, const void* k_cach
                      const int32_t* context_lens, int S, int H, int D, int bs, int MB, int NB,
                      double scale, int window) {
   return orc_paged_decode_gqa(out, q, q_dtype, k_cache, v_cache, cache_dtype, k_scale, v_scale,
-                              block_tables, context_lens, S, H, H, D, bs, MB, NB, scale, window);
+                              block_tables, context_lens, S, H, H, D, bs, MB, NB, scale, window, 1);
 }
 
 /*
@@ -230,79 +322,83 @@ int orc_paged_decode(double* out, const void* q, int q_dtype, const void* k_cach
  *   cu_q         [S + 1] int32, cu_q[0] = 0, non-decreasing; q_len = cu_q[s+1] - cu_q[s]
  *   other arguments as for orc_paged_decode_gqa; q_len <= context_lens[s] is required.
  */
+typedef struct {
+  double* out;
+  const void *q, *k_cache, *v_cache;
+  int q_dtype, cache_dtype;
+  const uint16_t *k_scale, *v_scale;
+  const int32_t *block_tables, *cu_q, *context_lens;
+  int S, Hq, Hkv, D, bs, MB, NB, window;
+  double scale;
+} prefill_job;
+
+/* One item: sequence s = item / Hkv, key/value head kh = item % Hkv, with every query head
+ * that reads kh and every query token of s. */
+static int prefill_item(const void* jp, long item, scratch_t* b) {
+  const prefill_job* j = (const prefill_job*)jp;
+  const int s = (int)(item / j->Hkv), kh = (int)(item % j->Hkv);
+  const int D = j->D, bs = j->bs, Hq = j->Hq, Hkv = j->Hkv;
+  const int group = Hq / Hkv;
+  const int ctx = j->context_lens[s];
+  const int q_len = j->cu_q[s + 1] - j->cu_q[s];
+  if (ctx < 0 || ctx > j->MB * bs) return ORC_BAD_CONTEXT;
+  if (q_len < 0 || q_len > ctx) return ORC_BAD_ARG;
+  if (q_len == 0) return ORC_OK;
+
+  /* gather every cached token of this key/value head through the block table */
+  for (int i = 0; i < ctx; ++i) {
+    int32_t pb = j->block_tables[(size_t)s * j->MB + i / bs];
+    if (pb < 0 || pb >= j->NB) return ORC_BAD_TABLE;
+    size_t row = ((size_t)pb * bs + i % bs) * Hkv + kh;
+    double ks = 1.0, vs = 1.0;
+    if (j->cache_dtype == ORC_I8 || j->cache_dtype == ORC_FP8) {
+      ks = orc_f16_to_f64(j->k_scale[row]);
+      vs = orc_f16_to_f64(j->v_scale[row]);
+    }
+    for (int d = 0; d < D; ++d) {
+      b->Kc[(size_t)i * D + d] = load_value(j->k_cache, j->cache_dtype, row * D + d) * ks;
+      b->Vc[(size_t)i * D + d] = load_value(j->v_cache, j->cache_dtype, row * D + d) * vs;
+    }
+  }
+
+  for (int h = kh * group; h < (kh + 1) * group; ++h) {
+    for (int i = 0; i < q_len; ++i) {
+      const size_t t = (size_t)j->cu_q[s] + i;
+      const int p = ctx - q_len + i;
+      const int lo = (j->window > 0 && p + 1 > j->window) ? p + 1 - j->window : 0;
+      const int n = p + 1 - lo;
+      double* o = j->out + (t * Hq + h) * D;
+      for (int d = 0; d < D; ++d) b->qv[d] = load_value(j->q, j->q_dtype, (t * Hq + h) * D + d);
+      for (int k = 0; k < n; ++k) {
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += b->qv[d] * b->Kc[(size_t)(lo + k) * D + d];
+        b->score[k] = j->scale * dot;
+      }
+      double m = b->score[0];
+      for (int k = 1; k < n; ++k) if (b->score[k] > m) m = b->score[k];
+      double z = 0.0;
+      for (int k = 0; k < n; ++k) { b->score[k] = exp(b->score[k] - m); z += b->score[k]; }
+      for (int k = 0; k < n; ++k) b->score[k] /= z;
+      for (int d = 0; d < D; ++d) {
+        double acc = 0.0;
+        for (int k = 0; k < n; ++k) acc += b->score[k] * b->Vc[(size_t)(lo + k) * D + d];
+        o[d] = acc;
+      }
+    }
+  }
+  return ORC_OK;
+}
+
 int orc_paged_prefill(double* out, const void* q, int q_dtype, const void* k_cache,
                       const void* v_cache, int cache_dtype, const uint16_t* k_scale,
                       const uint16_t* v_scale, const int32_t* block_tables, const int32_t* cu_q,
                       const int32_t* context_lens, int S, int Hq, int Hkv, int D, int bs, int MB,
-                      int NB, double scale, int window) {
+                      int NB, double scale, int window, int threads) {
   if (S < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || D <= 0 || bs <= 0 || MB <= 0 || NB <= 0)
     return ORC_BAD_ARG;
   if ((cache_dtype == ORC_I8 || cache_dtype == ORC_FP8) && (!k_scale || !v_scale)) return ORC_BAD_ARG;
   if (S > 0 && cu_q[0] != 0) return ORC_BAD_ARG;
-  const int group = Hq / Hkv;
-  const int max_ctx = MB * bs;
-  double* Kc = (double*)malloc(sizeof(double) * (size_t)max_ctx * D);
-  double* Vc = (double*)malloc(sizeof(double) * (size_t)max_ctx * D);
-  double* score = (double*)malloc(sizeof(double) * (size_t)max_ctx);
-  double* qv = (double*)malloc(sizeof(double) * (size_t)D);
-  if (!Kc || !Vc || !score || !qv) {
-    free(Kc); free(Vc); free(score); free(qv);
-    return ORC_NO_MEMORY;
-  }
-  int status = ORC_OK;
-
-  for (int s = 0; s < S && status == ORC_OK; ++s) {
-    const int ctx = context_lens[s];
-    const int q_len = cu_q[s + 1] - cu_q[s];
-    if (ctx < 0 || ctx > max_ctx) { status = ORC_BAD_CONTEXT; break; }
-    if (q_len < 0 || q_len > ctx) { status = ORC_BAD_ARG; break; }
-    if (q_len == 0) continue;
-
-    for (int kh = 0; kh < Hkv && status == ORC_OK; ++kh) {
-      /* gather every cached token of this key/value head through the block table */
-      for (int i = 0; i < ctx; ++i) {
-        int32_t pb = block_tables[(size_t)s * MB + i / bs];
-        if (pb < 0 || pb >= NB) { status = ORC_BAD_TABLE; break; }
-        size_t row = ((size_t)pb * bs + i % bs) * Hkv + kh;
-        double ks = 1.0, vs = 1.0;
-        if (cache_dtype == ORC_I8 || cache_dtype == ORC_FP8) {
-          ks = orc_f16_to_f64(k_scale[row]);
-          vs = orc_f16_to_f64(v_scale[row]);
-        }
-        for (int d = 0; d < D; ++d) {
-          Kc[(size_t)i * D + d] = load_value(k_cache, cache_dtype, row * D + d) * ks;
-          Vc[(size_t)i * D + d] = load_value(v_cache, cache_dtype, row * D + d) * vs;
-        }
-      }
-      if (status != ORC_OK) break;
-
-      for (int h = kh * group; h < (kh + 1) * group; ++h) {
-        for (int i = 0; i < q_len; ++i) {
-          const size_t t = (size_t)cu_q[s] + i;
-          const int p = ctx - q_len + i;
-          const int lo = (window > 0 && p + 1 > window) ? p + 1 - window : 0;
-          const int n = p + 1 - lo;
-          double* o = out + (t * Hq + h) * D;
-          for (int d = 0; d < D; ++d) qv[d] = load_value(q, q_dtype, (t * Hq + h) * D + d);
-          for (int j = 0; j < n; ++j) {
-            double dot = 0.0;
-            for (int d = 0; d < D; ++d) dot += qv[d] * Kc[(size_t)(lo + j) * D + d];
-            score[j] = scale * dot;
-          }
-          double m = score[0];
-          for (int j = 1; j < n; ++j) if (score[j] > m) m = score[j];
-          double z = 0.0;
-          for (int j = 0; j < n; ++j) { score[j] = exp(score[j] - m); z += score[j]; }
-          for (int j = 0; j < n; ++j) score[j] /= z;
-          for (int d = 0; d < D; ++d) {
-            double acc = 0.0;
-            for (int j = 0; j < n; ++j) acc += score[j] * Vc[(size_t)(lo + j) * D + d];
-            o[d] = acc;
-          }
-        }
-      }
-    }
-  }
-  free(Kc); free(Vc); free(score); free(qv);
-  return status;
+  prefill_job j = {out, q, k_cache, v_cache, q_dtype, cache_dtype, k_scale, v_scale,
+                   block_tables, cu_q, context_lens, S, Hq, Hkv, D, bs, MB, NB, window, scale};
+  return run_items(&j, prefill_item, (long)S * Hkv, MB * bs, D, threads);
 }

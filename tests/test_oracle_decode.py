@@ -283,3 +283,32 @@ def test_gqa_dense_case_matches_library_attention():
     vt = torch.from_numpy(V[0]).double().permute(1, 0, 2)[None]
     ref = F.scaled_dot_product_attention(qt, kt, vt, scale=0.25, enable_gqa=True)[0, :, 0, :].numpy()
     np.testing.assert_allclose(out[0], ref, rtol=0, atol=1e-12)
+
+
+def test_threads_share_out_pairs_without_changing_a_bit():
+    """Several worker threads give the single-threaded result bit for bit, on a batch with
+    empty, windowed, grouped-query and 8-bit cases, and the same error status when an item
+    fails (the lowest failing (sequence, head) pair decides it)."""
+    rng = np.random.default_rng(21)
+    ctx = [0, 1, 17, 40, 3, 64, 33]
+    K = [rng.standard_normal((c, 2, 16)) for c in ctx]
+    V = [rng.standard_normal((c, 2, 16)) for c in ctx]
+    kc, vc, bt = _pack(K, V, ctx, 8, rng)
+    q = rng.standard_normal((len(ctx), 6, 16)).astype(np.float32)
+    kt, vt = _as_f32_tensor(kc), _as_f32_tensor(vc)
+    for window in (0, 9):
+        one = oracle.paged_decode(q, kt, vt, bt, ctx, 0.3, window, threads=1)
+        for n in (2, 5, 64):
+            many = oracle.paged_decode(q, kt, vt, bt, ctx, 0.3, window, threads=n)
+            assert np.array_equal(one.view(np.uint64), many.view(np.uint64))
+    bad = bt.copy()
+    bad[5, 2] = kc.shape[0] + 3             # sequence 5: an entry outside the pool
+    ctx_bad = list(ctx)
+    ctx_bad[6] = bt.shape[1] * 8 + 1        # sequence 6: a context beyond its table
+    for n in (1, 3, 16):
+        with pytest.raises(ValueError, match="block-table entry"):
+            oracle.paged_decode(q, kt, vt, bad, ctx_bad, 0.3, threads=n)
+    ctx_bad[2] = -1                          # now an earlier pair fails on its context
+    for n in (1, 3, 16):
+        with pytest.raises(ValueError, match="context length"):
+            oracle.paged_decode(q, kt, vt, bad, ctx_bad, 0.3, threads=n)

@@ -204,3 +204,27 @@ def test_rejects_more_queries_than_context():
     kc = torch.zeros(2, 4, 1, 8)
     with pytest.raises(ValueError):
         oracle.paged_prefill(torch.zeros(5, 1, 8), kc, kc, [[0, 1]], [0, 5], [4], 1.0)
+
+
+def test_threads_share_out_pairs_without_changing_a_bit():
+    """Worker threads give the single-threaded prefill result bit for bit."""
+    g = torch.Generator().manual_seed(31)
+    ctx, qlen, bs, Hq, Hkv, D = [9, 40, 1, 70], [9, 5, 1, 33], 8, 6, 3, 16
+    NB = sum(-(-c // bs) for c in ctx) + 2
+    perm = torch.randperm(NB, generator=g)
+    MB = max(-(-c // bs) for c in ctx)
+    bt = torch.full((len(ctx), MB), -1, dtype=torch.int32)
+    k = 0
+    for s, c in enumerate(ctx):
+        for lb in range(-(-c // bs)):
+            bt[s, lb] = int(perm[k])
+            k += 1
+    kc = torch.randn(NB, bs, Hkv, D, generator=g)
+    vc = torch.randn(NB, bs, Hkv, D, generator=g)
+    q = torch.randn(sum(qlen), Hq, D, generator=g)
+    cu = torch.tensor([0] + list(np.cumsum(qlen)), dtype=torch.int32)
+    for window in (0, 7):
+        one = oracle.paged_prefill(q, kc, vc, bt, cu, ctx, 0.25, window, threads=1)
+        for n in (2, 4, 32):
+            many = oracle.paged_prefill(q, kc, vc, bt, cu, ctx, 0.25, window, threads=n)
+            assert np.array_equal(one.view(np.uint64), many.view(np.uint64))
