@@ -17,6 +17,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import importlib.util
 import json
 import math
 import os
@@ -31,7 +32,19 @@ sys.path.insert(0, ROOT)
 import torch  # noqa: E402
 
 import synth  # noqa: E402
-from paged_kv_cache_384_b200 import accounting  # noqa: E402
+
+
+def _load_accounting():
+    """The package's byte / FLOP accounting (host arithmetic on sizes), loaded on its own so
+    that the reference arm never loads the CUDA library the package __init__ opens."""
+    spec = importlib.util.spec_from_file_location(
+        "pa_accounting", os.path.join(ROOT, "paged_kv_cache_384_b200", "accounting.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+accounting = _load_accounting()
 
 PRESET = "llama70b_fp16"
 CONTEXT_DESC = {"llama70b_fp16": "uniform [1, 2048]",
@@ -41,7 +54,9 @@ CONTEXT_DESC = {"llama70b_fp16": "uniform [1, 2048]",
                 "llama70b_int8": "uniform [1, 2048], INT8 cache written by quantise-on-write",
                 "llama70b_fp8": "uniform [1, 2048], FP8 E4M3 cache written by quantise-on-write"}
 METRIC = "paged decode attention KV GB/s (% of B200 HBM peak) and tokens/s per layer"
-FALLBACK_HBM_GBS = 6650.0
+FALLBACK_HBM_GBS = 6650.0      # copy bandwidth measured earlier on this GPU type
+FALLBACK_BF16_TFLOPS = 1590.0  # cuBLAS bf16 burst measured earlier on this GPU type
+NOMINAL_HBM_GBS = 8000.0       # the ~8 TB/s HBM3e figure quoted for B200 (7.7 TB/s in HGX systems)
 
 
 # ---------------------------------------------------------------------------------------
@@ -67,14 +82,25 @@ def whole_job_gbs(bytes_per_rank_step, steps: int, max_seconds: float) -> float:
     return sum(bytes_per_rank_step) * steps / max_seconds / 1e9
 
 
+def _peaks_file():
+    with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+        return json.load(f)
+
+
 def measured_peak():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    """HBM copy bandwidth (GB/s) of this GPU type and where it comes from."""
     try:
-        with open(path) as f:
-            p = json.load(f)
-        return float(p["hbm_gbs"]), "measured"
-    except (OSError, KeyError, ValueError):
+        return float(_peaks_file()["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError, TypeError):
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tensor_peak():
+    """Dense fp16/bf16 tensor throughput (TFLOP/s, burst) and where it comes from."""
+    try:
+        return float(_peaks_file()["bf16_tflops"]), "measured (cuBLAS bf16 burst)"
+    except (OSError, KeyError, ValueError, TypeError):
+        return FALLBACK_BF16_TFLOPS, "fallback (cuBLAS bf16 burst measured earlier on this GPU type)"
 
 
 def kernel_traffic(kernel_source: str, record: str = "decode_partition_traffic.json", workload: str = None):
@@ -311,48 +337,145 @@ def launches_per_step(d) -> int:
 # ---------------------------------------------------------------------------------------
 # arms
 # ---------------------------------------------------------------------------------------
-def cpu_oracle_rate(w, seqs, repeats=1):
-    """Time the fp64 oracle (single-threaded C) on the given sequences of the workload."""
-    import oracle  # the CPU-baseline leg is the one place the benchmark runs the oracle
+def cpu_oracle_rate(w, seqs, threads=1, repeats=1):
+    """Time the fp64 oracle (plain C, ``threads`` worker threads over the independent
+    (sequence, head) pairs) on the given sequences of the workload."""
+    import oracle  # the CPU-baseline legs are the one place the benchmark runs the oracle
     sel = list(seqs)
-    kv = accounting.decode_kv_bytes([int(w.context_lens[s]) for s in sel], w.num_heads, w.head_dim,
+    kv = accounting.decode_kv_bytes([int(w.context_lens[s]) for s in sel], w.num_kv_heads, w.head_dim,
                                     w.cache_dtype, w.window)
+    q, bt, cl = w.q[sel], w.block_tables[sel], w.context_lens[sel]
     t0 = time.perf_counter()
     for _ in range(repeats):
-        oracle.paged_decode(w.q[sel], w.k_cache, w.v_cache, w.block_tables[sel], w.context_lens[sel],
-                            w.scale, w.window)
+        oracle.paged_decode(q, w.k_cache, w.v_cache, bt, cl, w.scale, w.window, threads=threads)
     dt = (time.perf_counter() - t0) / repeats
     return kv / dt / 1e9, dt, kv
 
 
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
 def run_reference(args):
-    """The oracle as it stands on the host cores, same workload/metric; rank 0 only."""
+    """The oracle as it stands on the host cores, same workload/metric; rank 0 only.  The
+    batch is laid out by the oracle's own block manager, so nothing of the product library
+    is loaded.  A step is the whole 32-sequence batch on every core, unless one step would
+    make the run take more than about two minutes; then a strided sample of the sequences,
+    stated in ``config``."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    import paged_kv_cache_384_b200 as pa  # only for the block manager that lays out the batch
-    w = synth.build_workload(PRESET, args.seed, pa.BlockManager)
-    sample = list(range(0, w.num_seqs, 4))          # 8 of the 32 sequences per step
-    for _ in range(args.warmup):
-        cpu_oracle_rate(w, sample)
+    from oracle.block_manager import BlockManager as OracleBM
+    w = synth.build_workload(PRESET, args.seed, OracleBM)
+    cores = host_cores()
+    sel = list(range(w.num_seqs))
+    _, probe, _ = cpu_oracle_rate(w, sel, threads=cores)
+    stride = 1
+    while stride < w.num_seqs and probe / stride * (args.steps + args.warmup) > 120.0:
+        stride *= 2
+    sel = list(range(0, w.num_seqs, stride))
+    for _ in range(max(0, args.warmup - 1)):
+        cpu_oracle_rate(w, sel, threads=cores)
     times, kv = [], 0
     for _ in range(args.steps):
-        _, dt, kv = cpu_oracle_rate(w, sample)
+        _, dt, kv = cpu_oracle_rate(w, sel, threads=cores)
         times.append(dt)
     t = sum(times) / len(times)
     value = kv / t / 1e9
-    desc = f"sequences 0,4,...,28 (8 of 32) of the {PRESET} batch per step, fp64 C oracle"
+    if stride == 1:
+        desc = f"the whole {PRESET} batch (32 sequences) per step, fp64 C oracle on {cores} threads"
+    else:
+        desc = (f"sequences 0,{stride},...({len(sel)} of 32) of the {PRESET} batch per step, fp64 C oracle "
+                f"on {cores} threads")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * t, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": PRESET, "num_seqs": len(sample), "num_heads": w.num_heads, "head_dim": w.head_dim,
-                   "block_size": w.block_size, "context": "uniform [1, 2048]", "seed": args.seed},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "config": {"workload": PRESET, "num_seqs": len(sel), "num_heads": w.num_heads, "head_dim": w.head_dim,
+                   "block_size": w.block_size, "num_blocks": w.num_blocks, "window": w.window,
+                   "context": CONTEXT_DESC[PRESET], "seed": args.seed,
+                   "sample": "whole batch" if stride == 1 else f"every {stride}th sequence"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def timed_steps(pa, w, d, stream, steps) -> float:
+    """Seconds for ``steps`` steps, CUDA events on the launching stream."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step(pa, w, d, stream)
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / 1e3
+
+
+def decode_kernel_ms(pa, w, d, stream, steps):
+    """Average (attention kernel, merge kernel) ms per step, from the events the library
+    records around its own launches."""
+    pa.profile_enable(True)
+    pa.profile_read(reset=True)
+    for _ in range(steps):
+        step(pa, w, d, stream)
+    part_ms, merge_ms, calls = pa.profile_read(reset=True)
+    pa.profile_enable(False)
+    return part_ms / max(calls, 1), merge_ms / max(calls, 1)
+
+
+def decode_kernel_name(w) -> str:
+    return "decode_gqa_tc_kernel" if w.num_kv_heads * 4 <= w.num_heads else "decode_partition_kernel"
+
+
+# The other decode workloads of the method, measured after the metric's own workload in a
+# default run so that their numbers sit in the same record: the prefix-sharing chat batch,
+# the INT8 and FP8 caches, the 32k-token sliding window at block sizes 8 / 16 / 32, and the
+# grouped-query Llama-2-70B layer (64 query heads over 8 cached heads).
+SECONDARY = (("chat_prefix_bf16", None), ("llama70b_int8", None), ("llama70b_fp8", None),
+             ("sliding_window_fp16", 8), ("sliding_window_fp16", 16), ("sliding_window_fp16", 32),
+             ("llama70b_gqa_fp16", None))
+SECONDARY_STEPS = 100
+
+
+def measure_secondary(pa, name, bs, seed, device, stream, peak):
+    w, _host, d, kv = build(seed, device, name, bs)
+    for _ in range(5):
+        step(pa, w, d, stream)
+    torch.cuda.synchronize(device)
+    sec = timed_steps(pa, w, d, stream, SECONDARY_STEPS)
+    part, merge = decode_kernel_ms(pa, w, d, stream, SECONDARY_STEPS)
+    errs = pa.device_error(clear=True)
+    ms = 1e3 * sec / SECONDARY_STEPS
+    rec = {"workload": name, "block_size": w.block_size, "cache_dtype": w.cache_dtype, "steps": SECONDARY_STEPS,
+           "context": CONTEXT_DESC.get(name, ""), "kv_bytes_per_step": kv,
+           "ms_per_step": round(ms, 4), "kv_gbs": round(kv / sec * SECONDARY_STEPS / 1e9, 2),
+           "frac": round(kv / sec * SECONDARY_STEPS / 1e9 / peak, 4),
+           "frac_of_nominal": round(kv / sec * SECONDARY_STEPS / 1e9 / NOMINAL_HBM_GBS, 4),
+           "kernel": decode_kernel_name(w), "kernel_ms": round(part, 4), "merge_ms": round(merge, 4),
+           "kernel_gbs": round(kv / part / 1e6, 2), "kernel_frac": round(kv / part / 1e6 / peak, 4),
+           "tokens_per_s_per_layer": round(w.num_seqs / (ms / 1e3), 1), "device_errors": errs}
+    if name == "chat_prefix_bf16":
+        # The shared 2000-token prefix is read by all 256 sequences but held once, and it
+        # stays in L2: the logical bytes above exceed what HBM can deliver.  The roofline of
+        # this workload is the DRAM traffic the kernel causes (ncu byte counters, captured
+        # for this exact source) against the distinct rows it must read at least once.
+        unique = accounting.decode_unique_kv_bytes(w.block_tables.tolist(), w.context_lens.tolist(), w.block_size,
+                                                   w.num_kv_heads, w.head_dim, w.cache_dtype, w.window)
+        dram = kernel_traffic(os.path.join(ROOT, "paged_kv_cache_384_b200", "csrc", "pa_decode.cu"),
+                              "decode_partition_traffic_chat_prefix_bf16.json", name)
+        rec.update({"unique_kv_bytes": unique, "unique_gbs_kernel": round(unique / part / 1e6, 2),
+                    "dram_bytes_per_launch": dram,
+                    "dram_gbs_kernel": None if dram is None else round(dram / part / 1e6, 2),
+                    "dram_frac": None if dram is None else round(dram / part / 1e6 / peak, 4),
+                    "unique_over_dram": None if dram is None else round(unique / dram, 4)})
+    del w, d
+    torch.cuda.empty_cache()
+    return rec
 
 
 def run_ours(args):
@@ -410,15 +533,8 @@ def run_ours(args):
     device_errors = pa.device_error(clear=True)
     pa.device_error(clear=True)
 
-    # ---- roofline: the partition kernel alone (library events around it) ----
-    pa.profile_enable(True)
-    pa.profile_read(reset=True)
-    for _ in range(args.steps):
-        step(pa, w, d, stream)
-    part_ms, merge_ms, calls = pa.profile_read(reset=True)
-    pa.profile_enable(False)
-    part_avg = part_ms / max(calls, 1)
-    merge_avg = merge_ms / max(calls, 1)
+    # ---- roofline: the attention kernel alone (library events around it) ----
+    part_avg, merge_avg = decode_kernel_ms(pa, w, d, stream, args.steps)
     achieved = kv_bytes / (part_avg / 1e3) / 1e9
     traffic = kernel_traffic(os.path.join(ROOT, "paged_kv_cache_384_b200", "csrc", "pa_decode.cu"))
 
@@ -430,9 +546,27 @@ def run_ours(args):
     # ---- CPU baseline: the oracle on this batch, rank 0 at N = 1 only ----
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline and args.workload == PRESET:
-        rate, dt, _ = cpu_oracle_rate(w, range(w.num_seqs))
-        cpu = {"value": round(rate, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": f"the full {PRESET} batch (32 sequences) once, fp64 C oracle, {dt:.1f} s"}
+        cores = host_cores()
+        rate, dt, _ = cpu_oracle_rate(w, range(w.num_seqs), threads=cores, repeats=3)
+        rate1, dt1, _ = cpu_oracle_rate(w, range(w.num_seqs), threads=1)
+        cpu = {"value": round(rate, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": f"the full {PRESET} batch (32 sequences), fp64 C oracle, {cores} threads over the "
+                         f"(sequence, head) pairs, {dt:.2f} s per batch (mean of 3)",
+               "single_core": {"value": round(rate1, 4), "unit": "GB/s", "cores": 1, "seconds": round(dt1, 2)}}
+
+    launches = launches_per_step(d) * args.steps
+    cache_dtype, nseq, nheads, hd = w.cache_dtype, w.num_seqs, w.num_heads, w.head_dim
+    bsz, nblk, win, kernel_name = w.block_size, w.num_blocks, w.window, decode_kernel_name(w)
+    workloads = workloads_clocks = None
+    if world == 1 and args.workload == PRESET and not args.no_workloads:
+        del w, d, host   # free this batch before the next ones are built
+        torch.cuda.empty_cache()
+        workloads = []
+        with ClockSampler(smi_id) as wclocks:
+            wclocks.mark()
+            for name, bs in SECONDARY:
+                workloads.append(measure_secondary(pa, name, bs, rank_seed(args.seed, rank), device, stream, peak))
+        workloads_clocks = wclocks.summary()
 
     if dist is not None:
         dist.barrier(device_ids=[local])
@@ -442,25 +576,30 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": {"fp16": "f16", "bf16": "bf16", "fp32": "f32", "int8": "i8", "fp8": "fp8_e4m3"}[w.cache_dtype],
+        "vs_baseline": None, "dtype": {"fp16": "f16", "bf16": "bf16", "fp32": "f32", "int8": "i8", "fp8": "fp8_e4m3"}[cache_dtype],
         "data": "synthetic",
-        "config": {"workload": args.workload, "num_seqs": w.num_seqs, "num_heads": w.num_heads, "head_dim": w.head_dim,
-                   "block_size": w.block_size, "num_blocks": w.num_blocks, "window": w.window,
+        "config": {"workload": args.workload, "num_seqs": nseq, "num_heads": nheads, "head_dim": hd,
+                   "block_size": bsz, "num_blocks": nblk, "window": win,
                    "context": CONTEXT_DESC.get(args.workload, ""),
                    "kv_bytes_per_step_per_gpu": kv_bytes, "seed": args.seed,
                    "l2": "inputs larger than L2 (KV per step >> 126 MB), no flush", "parallelism": f"replicas x{world}"},
         "tokens_per_s_per_layer": round(tokens_per_s, 1),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "pct_of_nominal_hbm": round(100 * value / world / NOMINAL_HBM_GBS, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_kind,
-                     "kernel": "decode_gqa_tc_kernel" if w.num_kv_heads * 4 <= w.num_heads else "decode_partition_kernel",
+                     "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+                     "nominal_peak": NOMINAL_HBM_GBS,
+                     "kernel": kernel_name,
                      "partition_ms": round(part_avg, 4),
                      "merge_ms": round(merge_avg, 4)},
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step(d) * args.steps,
+        "gpu_launches": launches,
         "clocks": clocks.summary(),
         "device_errors": device_errors,
+        "workloads": workloads,
+        "workloads_clocks": workloads_clocks,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -635,8 +774,7 @@ def run_prefill(args):
         clocks.mark()
         sec = timed(step, args.steps)
         attn_sec = timed(attn, args.steps)
-    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
-    peak = float(peaks["bf16_tflops"])  # fp16 and bf16 run at the same tensor rate
+    peak, peak_kind = measured_tensor_peak()  # fp16 and bf16 run at the same tensor rate
     # end to end: q and the new K/V rows from pinned host memory, the output read back
     hq, hk, hv = q.cpu().pin_memory(), k_new.cpu().pin_memory(), v_new.cpu().pin_memory()
     hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -666,7 +804,7 @@ def run_prefill(args):
                      "unit": "TFLOP/s", "frac": round(flops / attn_sec / 1e12 / peak, 4),
                      "traffic": kernel_traffic(os.path.join(ROOT, "paged_kv_cache_384_b200", "csrc", "pa_prefill_tc.cu"),
                                                "prefill_tc_traffic.json", args.workload),
-                     "peak_source": "measured (cuBLAS bf16 burst)", "kernel": "prefill_tc_kernel",
+                     "peak_source": peak_kind, "kernel": "prefill_tc_kernel",
                      "kernel_ms": round(1e3 * attn_sec, 4)},
         "cpu_baseline": None,
         "e2e": {"value": round(flops / e2e_sec / 1e12, 2), "unit": "TFLOP/s",
@@ -685,6 +823,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other decode workloads that a default run measures after the metric's own")
     ap.add_argument("--workload", default=PRESET, choices=["llama70b_fp16", "chat_prefix_bf16", "sliding_window_fp16",
                                                            "llama70b_gqa_fp16", "llama70b_int8", "llama70b_fp8", "swap_llama70b_fp16",
                                                            *PREFILL],

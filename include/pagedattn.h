@@ -178,6 +178,12 @@ pa_status pa_decode_use_tensor_cores(int enable);
  *     PA_ERR_INVALID_ARG (nothing is launched).
  *   - The first call on a device looks up the array's device address (once per device,
  *     with that device current); make that first call before any stream capture.
+ *   - `stream` must belong to the current device: the address looked up and the size
+ *     check both refer to the current device.
+ *   - The address is kept for the life of the process.  Do not call this entry point
+ *     again on a device after cudaDeviceReset() of that device: the reset unloads the
+ *     library's device code together with the array, and the kept address then points
+ *     to nothing.
  *   - Every call on a device shares the one array: calls that may overlap on the GPU
  *     (different streams, no ordering between them) race and corrupt each other's
  *     results.  Calls ordered on one stream are fine.

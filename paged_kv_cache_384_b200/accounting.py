@@ -60,3 +60,27 @@ def prefill_flops(context_lens: Iterable[int], q_lens: Iterable[int], num_q_head
         first = int(ctx) - int(ql)
         rows += sum(attended_tokens(p + 1, window) for p in range(first, int(ctx)))
     return 4.0 * head_dim * num_q_heads * rows
+
+
+def decode_unique_kv_bytes(block_tables, context_lens: Iterable[int], block_size: int, num_heads: int,
+                           head_dim: int, cache_dtype: str, window: int = 0) -> int:
+    """Bytes of the distinct cache rows one decode call reads: rows shared by several
+    sequences (a common prompt prefix held once, "KV Cache optimisation strategies in
+    deployment" (yunthe.com), section "Prefix Cache复用共享前缀的KV Cache") count once.  This
+    is the least DRAM traffic the call can cause; ``decode_kv_bytes`` counts every
+    sequence's rows."""
+    e = ELEM_BYTES[cache_dtype]
+    rows = set()
+    for s, c in enumerate(context_lens):
+        c = int(c)
+        lo = c - attended_tokens(c, window)
+        table = block_tables[s]
+        for lb in range(lo // block_size, -(-c // block_size)):
+            first = max(lo, lb * block_size) - lb * block_size
+            last = min(c, (lb + 1) * block_size) - lb * block_size
+            pb = int(table[lb])
+            rows.update((pb, off) for off in range(first, last))
+    per_row = num_heads * head_dim * 2 * e
+    if cache_dtype in ("int8", "fp8"):
+        per_row += num_heads * 2 * 2
+    return len(rows) * per_row

@@ -18,3 +18,20 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+def pytest_terminal_summary(terminalreporter):
+    """How many outputs the GPU parity checks accepted as rounding-boundary cases (the
+    exact value within half an I/O ulp of the GPU's, yet more than the tolerance away from
+    the oracle rounded to the I/O dtype), per I/O dtype."""
+    parity = sys.modules.get("parity")
+    tally = getattr(parity, "BOUNDARY_TALLY", None)
+    if not tally:
+        return
+    per = {}
+    for io, n, total in tally:
+        a, b = per.get(io, (0, 0))
+        per[io] = (a + n, b + total)
+    terminalreporter.write_sep("-", "parity: rounding-boundary cases accepted")
+    for io, (n, total) in sorted(per.items()):
+        terminalreporter.write_line(f"{io}: {n} of {total} outputs compared")

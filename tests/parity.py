@@ -17,6 +17,10 @@ import oracle
 import paged_kv_cache_384_b200 as pa
 
 TOL = {"fp32": 2e-3, "fp16": 2e-3, "bf16": 2e-3, "int8": 1e-2}
+
+# (I/O dtype, rounding-boundary cases accepted, outputs compared) of every compare() call
+# in this process; the session summary (conftest.py) prints the totals.
+BOUNDARY_TALLY = []
 TORCH_DT = {"fp32": torch.float32, "fp16": torch.float16, "bf16": torch.bfloat16}
 
 
@@ -50,6 +54,7 @@ def compare(gpu: torch.Tensor, ref64: np.ndarray, io: str, tol: float, max_bound
         raise AssertionError(f"{int(hard.sum())} outputs off by > {tol}: max {err.max():.3e} at {idx.tolist()}; "
                              f"gpu {g[tuple(idx[0])]} oracle {ref64[tuple(idx[0])]}")
     assert boundary.sum() <= max(1, max_boundary_frac * g.size), f"{int(boundary.sum())} rounding-boundary cases"
+    BOUNDARY_TALLY.append((io, int(boundary.sum()), int(g.size)))
     return float(err.max(initial=0.0)), float(raw.max(initial=0.0)), int(boundary.sum())
 
 

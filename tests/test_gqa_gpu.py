@@ -2,7 +2,7 @@
 
 query head h reads cached head h // (Hq // Hkv).  Covers group sizes 1..8 on every cache
 dtype, block sizes 8/16/32, windows, NaN-poisoned unattended rows, and the real Llama-2-70B
-layer shape (64 query heads over 8 cached heads) at 256 sequences on sampled outputs.
+layer shape (64 query heads over 8 cached heads) at 256 sequences on every output.
 """
 import math
 
@@ -89,17 +89,15 @@ def test_window(cuda_device, window):
     _run(case, ref, io, TOL[io])
 
 
-def test_llama70b_gqa_layer_sampled(cuda_device):
-    """64 query heads over 8 cached heads, 256 sequences of U[1, 2048] tokens."""
+def test_llama70b_gqa_layer_full(cuda_device):
+    """64 query heads over 8 cached heads, 256 sequences of U[1, 2048] tokens: every output."""
     w = synth.build_workload("llama70b_gqa_fp16", 0, OracleBM)
     case = GpuCase(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale)
     out = case.decode()
     torch.cuda.synchronize()
     assert_no_device_error()
-    sample = torch.randperm(w.num_seqs, generator=torch.Generator().manual_seed(5))[:20].tolist()
-    sample += [int(torch.argmax(w.context_lens)), int(torch.argmin(w.context_lens))]
-    ref = oracle_decode(w.q[sample], w.k_cache, w.v_cache, w.block_tables[sample], w.context_lens[sample], w.scale)
-    compare(out[sample], ref, "fp16", TOL["fp16"])
+    ref = oracle_decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale)
+    compare(out, ref, "fp16", TOL["fp16"])
 
 
 def test_head_count_mismatch_is_rejected(cuda_device):
