@@ -155,12 +155,16 @@ pa_status paged_attention_decode_gqa(void* out, const void* q, const void* k_cac
 
 /*
  * Process-wide switch (default 1): let grouped-query decode run on the tensor cores when
- * the call qualifies -- fp16 or bf16 cache equal to io_dtype, head_dim 128, block_size a
- * multiple of 8 dividing 128, and 4..16 query heads per cached head.  Then each 128-token
- * tile of one cached head is two tcgen05 MMAs (scores K.q^T and the weighted sum
- * V^T.p^T, fp32 accumulators in tensor memory) instead of CUDA-core dot products.  0 forces
- * the CUDA-core kernel (same results within rounding).  Not thread-safe against concurrent
- * decode calls; set it once at start-up.
+ * the call qualifies -- fp16 or bf16 io_dtype with a cache of the same type (head_dim 64 or
+ * 128) or an INT8 / FP8 E4M3 cache (head_dim 128), block_size a multiple of 8 dividing 128, and 4..16 query heads
+ * per cached head, or more with a divisor in [4, 16] (multi-query attention: the query heads
+ * of a cached head are split into sub-groups of that size, each reading the cached head).  Then each 128-token tile of one cached head is two tcgen05 MMAs (scores
+ * K.q^T and the weighted sum V^T.p^T, fp32 accumulators in tensor memory) instead of
+ * CUDA-core dot products.  8-bit codes are first widened to io_dtype in shared memory
+ * (exact); the per-token K scale multiplies the score and the V scale the softmax weight,
+ * which the value MMA takes rounded to io_dtype.  0 forces the CUDA-core kernel (same
+ * results within the tolerances).  Not thread-safe against concurrent decode calls; set it
+ * once at start-up.
  */
 pa_status pa_decode_use_tensor_cores(int enable);
 
@@ -250,7 +254,7 @@ pa_status reshape_and_cache(const void* k, const void* v, void* k_cache, void* v
  *   cu_q_lens      [num_seqs + 1] int32 device array, cu_q_lens[0] = 0, non-decreasing
  *   context_lens   [num_seqs] int32 device array, q_len <= context_len <= max_blocks_per_seq*block_size
  *   max_q_len      an upper bound of every q_len (sizes the grid; a larger q_len is an error)
- *   num_q_heads    a multiple of num_kv_heads with 1, 2, 4, 8 or 16 query heads per cached head
+ *   num_q_heads    a multiple of num_kv_heads with a power of two up to 128 query heads per cached head
  *   block_size     8, 16, 32, 64 or 128
  * Tensor cores (tcgen05), fp32 accumulation; bf16 probabilities keep ~16 bits (hi + lo
  * parts).  A sequence whose q_len exceeds max_q_len or its context, whose rows run
@@ -264,6 +268,29 @@ pa_status paged_attention_prefill(void* out, const void* q, const void* k_cache,
                                   int max_q_len, int num_q_heads, int num_kv_heads, int head_dim,
                                   int block_size, int num_blocks, int max_blocks_per_seq,
                                   float scale, int window, pa_dtype dtype, void* stream);
+
+/*
+ * paged_attention_prefill over an 8-bit cache: INT8 or FP8 E4M3 codes with one fp16 scale
+ * per (token, cached head), as written by reshape_and_cache_quant.  Source: page B, section
+ * "量化压缩KV Cache的INT8与FP8方案" (8-bit KV caches), with the prefill reading above.
+ *
+ *   k_cache, v_cache  [num_blocks, block_size, num_kv_heads, 128] codes of cache_dtype
+ *   k_scale, v_scale  [num_blocks, block_size, num_kv_heads] fp16 (2-byte aligned)
+ *   io_dtype          PA_F16 or PA_BF16 (q and out)
+ *   cache_dtype       PA_I8 or PA_FP8_E4M3 (anything else: PA_ERR_INVALID_ARG)
+ * Other arguments, layouts and errors as paged_attention_prefill.  Each cached value
+ * code * scale enters the tensor-core products rounded once to io_dtype (relative error
+ * 2^-11 for fp16, 2^-8 for bf16); accumulation is fp32.
+ */
+pa_status paged_attention_prefill_quant(void* out, const void* q, const void* k_cache,
+                                        const void* v_cache, const void* k_scale,
+                                        const void* v_scale, const int32_t* block_tables,
+                                        const int32_t* cu_q_lens, const int32_t* context_lens,
+                                        int num_seqs, int num_q_tokens, int max_q_len,
+                                        int num_q_heads, int num_kv_heads, int head_dim,
+                                        int block_size, int num_blocks, int max_blocks_per_seq,
+                                        float scale, int window, pa_dtype io_dtype,
+                                        pa_dtype cache_dtype, void* stream);
 
 /*
  * Copy whole physical blocks for copy-on-write.  Source: page C, section 二,

@@ -136,18 +136,27 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
 # Cache maintenance
 # ---------------------------------------------------------------------------------------
 def paged_attention_prefill(out, q, k_cache, v_cache, block_tables, cu_q_lens, context_lens, max_q_len: int,
-                            scale: float, window: int = 0, stream=None):
+                            scale: float, window: int = 0, stream=None, k_scale=None, v_scale=None):
     """Causal attention of each sequence's newest q_len tokens over the paged cache.
 
     q/out [T, Hq, 128] (fp16 or bf16) pack the sequences' query rows (sequence s owns rows
     cu_q_lens[s]..cu_q_lens[s+1]-1, int32 [S+1] on the GPU); the chunk's K/V must already
     be in the cache, so query i of sequence s is at position context_lens[s] - q_len + i.
-    ``max_q_len`` bounds every q_len (host-known, sizes the grid).
+    ``max_q_len`` bounds every q_len (host-known, sizes the grid).  The caches hold q's
+    dtype, or int8 / float8_e4m3fn codes with fp16 k_scale / v_scale [NB, bs, Hkv].
     """
     if q.dim() != 3 or out.shape != q.shape or out.dtype != q.dtype:
         raise ValueError("q and out must be [T, Hq, D] of one dtype")
-    if k_cache.dim() != 4 or v_cache.shape != k_cache.shape or k_cache.dtype != q.dtype:
-        raise ValueError("caches must be [NB, bs, Hkv, D] in q's dtype")
+    eight_bit = k_cache.dtype in _SCALED
+    if k_cache.dim() != 4 or v_cache.shape != k_cache.shape or v_cache.dtype != k_cache.dtype or \
+            (k_cache.dtype != q.dtype and not eight_bit):
+        raise ValueError("caches must be [NB, bs, Hkv, D] in q's dtype, or int8 / float8_e4m3fn")
+    if eight_bit:
+        NB_, bs_, Hkv_ = k_cache.shape[:3]
+        if k_scale is None or v_scale is None or k_scale.dtype != torch.float16 or \
+                k_scale.shape != (NB_, bs_, Hkv_) or v_scale.shape != (NB_, bs_, Hkv_):
+            raise ValueError("an int8 / fp8 cache needs fp16 k_scale/v_scale of shape [NB, bs, Hkv]")
+        _dense("k_scale", k_scale), _dense("v_scale", v_scale)
     if cu_q_lens.dtype != torch.int32 or context_lens.dtype != torch.int32 or block_tables.dtype != torch.int32:
         raise ValueError("cu_q_lens, context_lens and block_tables must be int32")
     for name, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
@@ -158,6 +167,12 @@ def paged_attention_prefill(out, q, k_cache, v_cache, block_tables, cu_q_lens, c
     S = context_lens.shape[0]
     if cu_q_lens.shape[0] != S + 1:
         raise ValueError("cu_q_lens must have num_seqs + 1 entries")
+    if eight_bit:
+        _check(_L.paged_attention_prefill_quant(
+            _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+            _ptr(cu_q_lens), _ptr(context_lens), S, T, int(max_q_len), Hq, Hkv, D, bs, NB, block_tables.shape[1],
+            float(scale), int(window), _DTYPE[q.dtype], _DTYPE[k_cache.dtype], _stream(stream)))
+        return
     _check(_L.paged_attention_prefill(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                                       _ptr(cu_q_lens), _ptr(context_lens), S, T, int(max_q_len), Hq, Hkv, D, bs,
                                       NB, block_tables.shape[1], float(scale), int(window), _DTYPE[q.dtype],

@@ -40,7 +40,10 @@ namespace pa {
 //   IO: q/out type; CT: cache element type; D: head_dim; TT: rows per tile if fixed, 0 = runtime.
 // ---------------------------------------------------------------------------------------
 template <typename IO, typename CT, int D, int TT>
-__global__ void __launch_bounds__(kMaxThreads)
+// minBlocks = 1 states what the launch uses (shared memory allows 2 or 3 CTAs per SM); with
+// the bound left at its default ptxas capped several instantiations at 56 or 72 registers and
+// spilled.
+__global__ void __launch_bounds__(kMaxThreads, 1)
 decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ CUtensorMap tmKs, const __grid_constant__ CUtensorMap tmVs,
                         const DecodeParams p) {
@@ -156,29 +159,83 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   const int v = lane % LPR;  // 16-byte vector within the row: dims [v*EV, v*EV + EV)
   Cursor c = start;
   bool seg_from_start = (c.j == 0);
-  // INT8 codes are widened and multiplied two at a time on packed fp32 pairs (fewer
-  // instructions per byte, which is what limits this path; 69 -> 74 % of HBM); q and the
-  // accumulator are then kept as pairs too.  FP8 keeps the scalar path: its hardware
-  // convert already yields pairs, and packing them measured slower (78 -> 74 %).
-  constexpr bool kPairs = std::is_same<CT, int8_t>::value;
+  // INT8 weighted sums of V: code + 128 spliced under the exponent of 1024 is the f16 value
+  // 1152 + c, exactly, two codes per byte-permute; one f16 x f16 -> f32 FMA per code adds
+  // w * (1152 + c) with the weight w = p * v_scale rounded to f16, and the bias 1152 * sum(w)
+  // is removed once when the segment ends (the cancellation costs ~7 of fp32's 24 bits of the
+  // biased sum; typical error ~1e-5 of the output scale against the 1e-2 tolerance).
+  constexpr bool kBiasV = std::is_same<CT, int8_t>::value;
+  // INT8 scores are integer dot products: q is held as 24-bit fixed point per row (row
+  // maximum below 2^22 steps), split into a signed top byte and two unsigned bytes, and
+  // each byte plane is dotted with four codes per dp4a instruction into an exact int32 sum
+  // (16 dims per lane: |sum| < 2^19 per plane).  The only rounding is that of q to 2^-22 of
+  // its row maximum, finer than fp32's own rounding of most elements of the row.
+  constexpr bool kDp4a = std::is_same<CT, int8_t>::value;
+  // FP8 scores and weighted sums run on f16 x f16 -> f32 fused multiply-adds: pairs of E4M3
+  // codes convert exactly to f16 pairs, q is held in f16 after an exact power-of-two
+  // rescaling of its row (row maximum in [2^14, 2^15)), the softmax weight p * v_scale is
+  // rounded to f16 (relative 2^-11), and every product is exact in the fp32 accumulator.
+  constexpr bool kMixed = std::is_same<CT, __nv_fp8_e4m3>::value;
   float qf[EV], acc[EV];
-  uint64_t q2[EV / 2], acc2[EV / 2];
+  float wsum = 0.f;        // INT8: sum of the f16 weights, for the bias of the V sum
+  uint32_t qb[3][EV / 4];  // byte planes of the fixed-point q: [2] signed top, [1] and [0] unsigned
+  uint32_t qh2[EV / 2];    // f16 pairs of the rescaled q (FP8 cache)
+  float q_unit = 1.f;      // factor from the raw dot product to the base-2 score (before the K scale)
   float m = -FLT_MAX, l = 0.f;  // running max (base 2) and sum; -FLT_MAX keeps exp2 finite
   auto load_q = [&](const Cursor& cc) {
     const int h = cc.g * QW + w;
     const IO* qrow = reinterpret_cast<const IO*>(p.q) + (static_cast<size_t>(cc.s) * p.Hq + h) * D + v * EV;
     load_floats<IO, EV>(qrow, qf);
+    if constexpr (kMixed) {
+      float amax = 0.f;
 #pragma unroll
-    for (int e = 0; e < EV; ++e) qf[e] *= p.qscale;
-    if (kPairs)
+      for (int e = 0; e < EV; ++e) amax = fmaxf(amax, fabsf(qf[e]));
 #pragma unroll
-      for (int j = 0; j < EV / 2; ++j) q2[j] = f2_pack(qf[2 * j], qf[2 * j + 1]);
+      for (int off = LPR / 2; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      int ex = 0;
+      frexpf(amax, &ex);                          // amax < 2^ex
+      const int E = max(-100, min(100, 15 - ex));  // amax * 2^E < 2^15: finite in f16
+      const float up = ldexpf(1.f, E);
+      q_unit = p.qscale * ldexpf(1.f, -E);
+#pragma unroll
+      for (int j = 0; j < EV / 2; ++j) {
+        const __half2 h2 = __floats2half2_rn(qf[2 * j] * up, qf[2 * j + 1] * up);
+        qh2[j] = *reinterpret_cast<const uint32_t*>(&h2);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < EV; ++e) qf[e] *= p.qscale;
+    }
+    if constexpr (kDp4a) {
+      float amax = 0.f;
+#pragma unroll
+      for (int e = 0; e < EV; ++e) amax = fmaxf(amax, fabsf(qf[e]));
+#pragma unroll
+      for (int off = LPR / 2; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      int ex = 0;
+      frexpf(amax, &ex);                        // amax < 2^ex
+      const int E = max(-100, min(100, 22 - ex));  // amax * 2^E < 2^22
+      const float up = ldexpf(1.f, E);
+      q_unit = ldexpf(1.f, -E);
+#pragma unroll
+      for (int j = 0; j < EV / 4; ++j) {
+        uint32_t w2 = 0, w1 = 0, w0 = 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int qi = max(-(1 << 22) + 1, min((1 << 22) - 1, __float2int_rn(qf[4 * j + k] * up)));
+          w2 |= (static_cast<uint32_t>(qi >> 16) & 0xffu) << (8 * k);
+          w1 |= (static_cast<uint32_t>(qi >> 8) & 0xffu) << (8 * k);
+          w0 |= (static_cast<uint32_t>(qi) & 0xffu) << (8 * k);
+        }
+        qb[2][j] = w2;
+        qb[1][j] = w1;
+        qb[0][j] = w0;
+      }
+    }
   };
   load_q(c);
 #pragma unroll
   for (int e = 0; e < EV; ++e) acc[e] = 0.f;
-#pragma unroll
-  for (int j = 0; j < EV / 2; ++j) acc2[j] = 0;
 
   for (int it = 0; it < n; ++it) {
     const int st = it % NS;
@@ -202,8 +259,27 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
         float part = 0.f;
         if (t < tt) {
           const uint4 kv = ld_shared_v4(kt + ((t * HG + kw) * D + v * EV) * E);
-          if constexpr (kPairs) {
-            part = dot_pairs<CT>(kv, q2);
+          if constexpr (kDp4a) {
+            const uint32_t words[4] = {kv.x, kv.y, kv.z, kv.w};
+            int a2 = 0, a1 = 0, a0 = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              a2 = dp4a_ss(words[j], qb[2][j], a2);
+              a1 = dp4a_su(words[j], qb[1][j], a1);
+              a0 = dp4a_su(words[j], qb[0][j], a0);
+            }
+            part = fmaf(static_cast<float>(a2), 65536.f, fmaf(static_cast<float>(a1), 256.f, static_cast<float>(a0)));
+          } else if constexpr (kMixed) {
+            const uint32_t words[4] = {kv.x, kv.y, kv.z, kv.w};
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint32_t lo, hi;
+              e4m3x4_to_f16x2x2(words[j], lo, hi);
+              a0 = fma2_f16_f32(qh2[2 * j], lo, a0);
+              a1 = fma2_f16_f32(qh2[2 * j + 1], hi, a1);
+            }
+            part = a0 + a1;
           } else {
             float kf[EV];
             Elem<CT>::to_float(kv, kf);
@@ -215,7 +291,7 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
         for (int off = LPR / 2; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
         const int tok = tok0 + t;
         if (t < tt && tok >= c.sp.lo && tok < c.sp.ctx) {
-          if (kInt8) part *= __half2float(__ushort_as_half(ld_shared_u16(kt + p.ks_off + (t * 8 + hs) * 2)));
+          if (kInt8) part *= __half2float(__ushort_as_half(ld_shared_u16(kt + p.ks_off + (t * 8 + hs) * 2))) * q_unit;
           sc[pi] = part;
           tile_max = fmaxf(tile_max, part);
         }
@@ -229,14 +305,9 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
     const float alpha = exp2f(m - m_new);
     m = m_new;
     l *= alpha;
-    if constexpr (kPairs) {
-      const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-      for (int j = 0; j < EV / 2; ++j) acc2[j] = f2_fma(a2, acc2[j], 0);
-    } else {
-#pragma unroll
-      for (int e = 0; e < EV; ++e) acc[e] *= alpha;
-    }
+    for (int e = 0; e < EV; ++e) acc[e] *= alpha;
+    if (kBiasV) wsum *= alpha;
 #pragma unroll
     for (int pi = 0; pi < MAXP; ++pi) {
       if (TT > 0 || pi * RPP < tt) {
@@ -247,8 +318,28 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
           const uint4 vv = ld_shared_v4(vt + ((t * HG + kw) * D + v * EV) * E);
           float pv = pr;
           if (kInt8) pv *= __half2float(__ushort_as_half(ld_shared_u16(kt + p.vs_off + (t * 8 + hs) * 2)));
-          if constexpr (kPairs) {
-            axpy_pairs<CT>(pv, vv, acc2);
+          if constexpr (kBiasV) {
+            const __half2 w2 = __float2half2_rn(pv);
+            const uint32_t wb = *reinterpret_cast<const uint32_t*>(&w2);
+            wsum += __low2float(w2);
+            const uint32_t words[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t u = words[j] ^ 0x80808080u;
+              fma_f16x2_f32x2(wb, __byte_perm(u, 0x6464u, 0x4140u), acc[4 * j], acc[4 * j + 1]);
+              fma_f16x2_f32x2(wb, __byte_perm(u, 0x6464u, 0x4342u), acc[4 * j + 2], acc[4 * j + 3]);
+            }
+          } else if constexpr (kMixed) {
+            const uint32_t words[4] = {vv.x, vv.y, vv.z, vv.w};
+            const __half2 w2 = __float2half2_rn(pv);
+            const uint32_t wb = *reinterpret_cast<const uint32_t*>(&w2);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint32_t lo, hi;
+              e4m3x4_to_f16x2x2(words[j], lo, hi);
+              fma_f16x2_f32x2(wb, lo, acc[4 * j], acc[4 * j + 1]);
+              fma_f16x2_f32x2(wb, hi, acc[4 * j + 2], acc[4 * j + 3]);
+            }
           } else {
             float vf[EV];
             Elem<CT>::to_float(vv, vf);
@@ -263,9 +354,9 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
 
     const bool seg_last = (c.j == c.sp.nb - 1);
     if (seg_last || it == n - 1) {
-      if constexpr (kPairs)
+      if constexpr (kBiasV)
 #pragma unroll
-        for (int j = 0; j < EV / 2; ++j) f2_unpack(acc2[j], acc[2 * j], acc[2 * j + 1]);
+        for (int e = 0; e < EV; ++e) acc[e] = fmaf(-1152.f, wsum, acc[e]);
       // Combine the RPP row groups of the warp.
       float lt = l;
 #pragma unroll
@@ -298,10 +389,9 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
       }
       m = -FLT_MAX;
       l = 0.f;
+      wsum = 0.f;
 #pragma unroll
       for (int e = 0; e < EV; ++e) acc[e] = 0.f;
-#pragma unroll
-      for (int j = 0; j < EV / 2; ++j) acc2[j] = 0;
     }
     if (it + 1 < n) {
       advance(c, p);
@@ -314,8 +404,9 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
 }
 
 // ---------------------------------------------------------------------------------------
-// Merge kernel: one warp per (sequence, head) combines the partial states of a segment that
-// was split across CTAs:  M = max_k m_k,  out = sum_k 2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k.
+// Merge kernel: one warp per (sequence, head group) segment combines, head by head, the
+// partial states of a segment that was split across CTAs:
+//   M = max_k m_k,  out = sum_k 2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k.
 // Sequences with nothing to attend get zeros; segments held by one CTA were written by it.
 // Launched as a programmatic dependent of the partition kernel: the grid is resident while
 // the partition kernel runs and proceeds the moment its results are visible.
@@ -327,47 +418,53 @@ __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const De
   constexpr int DL = D / 32;  // dims per lane
   grid_dependency_wait();
   const int lane = threadIdx.x & 31;
+  // One warp per (sequence, head group) segment: a segment held by one CTA needs nothing, so
+  // most warps read the tile prefix once and leave; the heads of a split one are merged in turn.
   const long long item = static_cast<long long>(blockIdx.x) * kMergeWarps + (threadIdx.x >> 5);
-  if (item >= static_cast<long long>(p.S) * p.Hq) return;
-  const int s = static_cast<int>(item / p.Hq), h = static_cast<int>(item % p.Hq);
+  if (item >= static_cast<long long>(p.S) * p.G) return;
+  const int s = static_cast<int>(item / p.G), g = static_cast<int>(item % p.G);
   const long long per_group = p.ws_prefix[p.S];
   const long long pre = p.ws_prefix[s];
   const long long nb = p.ws_prefix[s + 1] - pre;
-  IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(s) * p.Hq + h) * D + lane * DL;
-  float o[DL];
+  if (nb == 0) {  // nothing to attend: zeros
+    for (int w = 0; w < p.QW; ++w) {
+      IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(s) * p.Hq + g * p.QW + w) * D + lane * DL;
 #pragma unroll
-  for (int e = 0; e < DL; ++e) o[e] = 0.f;
-  if (nb == 0) {
-#pragma unroll
-    for (int e = 0; e < DL; ++e) orow[e] = float_to<IO>(0.f);
+      for (int e = 0; e < DL; ++e) orow[e] = float_to<IO>(0.f);
+    }
     return;
   }
   const long long T = per_group * p.G;
-  const int g = h / p.QW, w = h % p.QW;
   const long long a = p.G * pre + g * nb;
   const int c0 = cta_of(a, T, p.num_ctas), c1 = cta_of(a + nb - 1, T, p.num_ctas);
   if (c0 == c1) return;
   const long long seg = static_cast<long long>(s) * p.G + g;
   const float2* ml = reinterpret_cast<const float2*>(p.ws_ml);
-  // Global max over the partials, 32 partials per round (one per lane).
-  float M = -FLT_MAX;
-  for (int k = c0 + lane; k <= c1; k += 32) M = fmaxf(M, ml[(k + seg) * p.QW + w].x);
+  for (int w = 0; w < p.QW; ++w) {
+    // Global max over the partials, 32 partials per round (one per lane).
+    float M = -FLT_MAX;
+    for (int k = c0 + lane; k <= c1; k += 32) M = fmaxf(M, ml[(k + seg) * p.QW + w].x);
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  float L = 0.f;
+    for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float o[DL];
+#pragma unroll
+    for (int e = 0; e < DL; ++e) o[e] = 0.f;
+    float L = 0.f;
 #pragma unroll 4
-  for (int k = c0; k <= c1; ++k) {
-    const long long row = (k + seg) * p.QW + w;
-    const float2 st = ml[row];
-    const float f = exp2f(st.x - M);
-    L = fmaf(f, st.y, L);
-    const float* src = p.ws_acc + row * D + lane * DL;
+    for (int k = c0; k <= c1; ++k) {
+      const long long row = (k + seg) * p.QW + w;
+      const float2 st = ml[row];
+      const float f = exp2f(st.x - M);
+      L = fmaf(f, st.y, L);
+      const float* src = p.ws_acc + row * D + lane * DL;
 #pragma unroll
-    for (int e = 0; e < DL; ++e) o[e] = fmaf(f, src[e], o[e]);
+      for (int e = 0; e < DL; ++e) o[e] = fmaf(f, src[e], o[e]);
+    }
+    const float inv = 1.f / L;
+    IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(s) * p.Hq + g * p.QW + w) * D + lane * DL;
+#pragma unroll
+    for (int e = 0; e < DL; ++e) orow[e] = float_to<IO>(o[e] * inv);
   }
-  const float inv = 1.f / L;
-#pragma unroll
-  for (int e = 0; e < DL; ++e) orow[e] = float_to<IO>(o[e] * inv);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -523,12 +620,14 @@ bool g_tensor_cores = true;  // pa_decode_use_tensor_cores()
 
 // Grouped-query decode on the tensor cores: one CTA per SM, 128-token tiles of one cached
 // head (pa_decode_tc.cu), then the shared merge kernel.
-pa_status decode_launch_tc(void* out, const void* q, const void* k_cache, const void* v_cache,
-                           const int32_t* block_tables, const int32_t* context_lens, int num_seqs, int num_q_heads,
-                           int num_kv_heads, int block_size, int num_blocks, int max_blocks_per_seq, float scale,
-                           int window, pa_dtype io_dtype, void* workspace, int sms, cudaStream_t s) {
-  const int head_dim = 128;
-  const int GQ = num_q_heads / num_kv_heads;
+pa_status decode_launch_tc(void* out, const void* q, const void* k_cache, const void* v_cache, const void* k_scale,
+                           const void* v_scale, const int32_t* block_tables, const int32_t* context_lens,
+                           int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                           int num_blocks, int max_blocks_per_seq, float scale, int window, pa_dtype io_dtype,
+                           pa_dtype cache_dtype, void* workspace, int sms, cudaStream_t s) {
+  const int SG = tc_decode_subgroup(num_q_heads / num_kv_heads);  // query heads per head group
+  const int NSUB = num_q_heads / num_kv_heads / SG;               // head groups per cached head
+  const int GQ = SG;
   const int C = sms;
   const long long rows = static_cast<long long>(C) * GQ + static_cast<long long>(num_seqs) * num_q_heads;
   const WsLayout lay = ws_layout(num_seqs, head_dim, rows);
@@ -537,20 +636,39 @@ pa_status decode_launch_tc(void* out, const void* q, const void* k_cache, const 
   pa_status st = get_encoder(&enc);
   if (st != PA_OK) return st;
   const CUtensorMapDataType ttype = io_dtype == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  CUtensorMap tmK, tmV, tmQ;
-  {
-    // [NB*bs rows][Hkv][128]: boxes of one block's rows x one head x 64 dims, 128-byte swizzle
-    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(num_kv_heads),
+  const bool eight_bit = cache_dtype != io_dtype;
+  CUtensorMap tmK, tmV, tmQ, tmKs, tmVs;
+  if (!eight_bit) {
+    // [NB*bs rows][Hkv][head_dim]: boxes of one block's rows x one head x 64 dims, 128-byte swizzle
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_kv_heads),
                                 static_cast<cuuint64_t>(num_blocks) * block_size};
-    const cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(num_kv_heads) * 256};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                                   static_cast<cuuint64_t>(num_kv_heads) * head_dim * 2};
     const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(block_size)};
     if ((st = encode(enc, &tmK, ttype, 3, k_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != PA_OK) return st;
     if ((st = encode(enc, &tmV, ttype, 3, v_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != PA_OK) return st;
+    tmKs = tmK;
+    tmVs = tmV;
+  } else {
+    // 8-bit codes [NB*bs rows][Hkv][128 B]: one block's rows x one head x all 128 dims,
+    // 128-byte swizzle; scales [NB*bs rows][Hkv] fp16: one block's rows x 8 heads (16 B)
+    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(num_kv_heads),
+                                static_cast<cuuint64_t>(num_blocks) * block_size};
+    const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(num_kv_heads) * 128};
+    const cuuint32_t box[3] = {128, 1, static_cast<cuuint32_t>(block_size)};
+    const CUtensorMapDataType ctype = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    if ((st = encode(enc, &tmK, ctype, 3, k_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != PA_OK) return st;
+    if ((st = encode(enc, &tmV, ctype, 3, v_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != PA_OK) return st;
+    const cuuint64_t sdims[2] = {static_cast<cuuint64_t>(num_kv_heads), static_cast<cuuint64_t>(num_blocks) * block_size};
+    const cuuint64_t sstrides[1] = {static_cast<cuuint64_t>(num_kv_heads) * 2};
+    const cuuint32_t sbox[2] = {8, static_cast<cuuint32_t>(block_size)};
+    if ((st = encode(enc, &tmKs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, k_scale, sdims, sstrides, sbox)) != PA_OK) return st;
+    if ((st = encode(enc, &tmVs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, v_scale, sdims, sstrides, sbox)) != PA_OK) return st;
   }
   {
-    // q as [S*Hq rows][128]: the GQ rows of one head group x 64 dims
-    const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(num_seqs) * num_q_heads};
-    const cuuint64_t strides[1] = {256};
+    // q as [S*Hq rows][head_dim]: the GQ rows of one head group x 64 dims
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_seqs) * num_q_heads};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * 2};
     const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(GQ)};
     if ((st = encode(enc, &tmQ, ttype, 2, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != PA_OK) return st;
   }
@@ -571,22 +689,24 @@ pa_status decode_launch_tc(void* out, const void* q, const void* k_cache, const 
   prm.tt = tc_decode_tile_tokens();
   prm.tpb = 1;
   prm.HG = 1;
-  prm.G = num_kv_heads;
+  prm.G = num_kv_heads * NSUB;
   prm.num_ctas = C;
   prm.nstage = 0;
   prm.Hq = num_q_heads;
   prm.GQ = GQ;
   prm.QW = GQ;
+  prm.sub = NSUB;
+  prm.dim = head_dim;
   prm.qscale = scale * 1.4426950408889634f;
 
   cudaEvent_t ev[3];
   profiling_next_events(ev);
   if (ev[0]) cudaEventRecord(ev[0], s);
-  if ((st = tc_decode_launch(tmK, tmV, tmQ, prm, io_dtype, C, s)) != PA_OK) return st;
+  if ((st = tc_decode_launch(tmK, tmV, tmQ, tmKs, tmVs, prm, io_dtype, cache_dtype, C, s)) != PA_OK) return st;
   if (ev[1]) cudaEventRecord(ev[1], s);
   {
     void* args[] = {&prm};
-    const long long items = static_cast<long long>(num_seqs) * num_q_heads;
+    const long long items = static_cast<long long>(num_seqs) * prm.G;  // one warp per segment
     const unsigned grid = static_cast<unsigned>((items + kMergeWarps - 1) / kMergeWarps);
     cudaError_t err = launch_dependent(select_merge(io_dtype, head_dim), dim3(grid), dim3(32 * kMergeWarps), 0, s, args);
     if (err != cudaSuccess) return cuda_fail(err, "launching the decode merge kernel");
@@ -612,7 +732,8 @@ pa_status decode_launch(void* out, const void* q, const void* k_cache, const voi
   if (GQ > kMaxHeadGroup && !use_tc)
     return fail(PA_ERR_UNSUPPORTED,
                 "%d query heads per cached head: up to %d on the CUDA-core kernel; more need the tensor-core "
-                "kernel (fp16/bf16 cache, head_dim 128, block_size a multiple of 8 dividing 128, up to 16)",
+                "kernel (fp16/bf16 io, head_dim 128, block_size a multiple of 8 dividing 128, and a group "
+                "of up to 16 or with a divisor in [4, 16])",
                 GQ, kMaxHeadGroup);
   if (head_dim != 64 && head_dim != 128) return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", head_dim);
   if (block_size < 1 || block_size > 32) return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 1..32)", block_size);
@@ -645,9 +766,9 @@ pa_status decode_launch(void* out, const void* q, const void* k_cache, const voi
   if (workspace_bytes < need)
     return fail(PA_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
   if (use_tc)
-    return decode_launch_tc(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_q_heads, num_heads,
-                            block_size, num_blocks, max_blocks_per_seq, scale, window, io_dtype, workspace, sms,
-                            static_cast<cudaStream_t>(stream));
+    return decode_launch_tc(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, num_seqs,
+                            num_q_heads, num_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, scale,
+                            window, io_dtype, cache_dtype, workspace, sms, static_cast<cudaStream_t>(stream));
 
   // Rows per tile: the largest divisor of block_size in [8, 16] (the whole block if none),
   // so 32-token blocks stream as two 16-row tiles and keep four heads per CTA.
@@ -733,6 +854,8 @@ pa_status decode_launch(void* out, const void* q, const void* k_cache, const voi
   prm.GQ = GQ;
   prm.QW = QW;
   prm.G = G;
+  prm.sub = 1;
+  prm.dim = head_dim;
   prm.num_ctas = C;
   prm.nstage = nstage;
   prm.qscale = scale * 1.4426950408889634f;  // log2(e): exp(x) = 2^(x log2 e)
@@ -755,7 +878,7 @@ pa_status decode_launch(void* out, const void* q, const void* k_cache, const voi
   if (ev[1]) cudaEventRecord(ev[1], s);
   {
     void* args[] = {&prm};
-    const long long items = static_cast<long long>(num_seqs) * num_q_heads;
+    const long long items = static_cast<long long>(num_seqs) * G;  // one warp per segment
     const unsigned grid = static_cast<unsigned>((items + kMergeWarps - 1) / kMergeWarps);
     cudaError_t err = launch_dependent(merge_fn, dim3(grid), dim3(32 * kMergeWarps), 0, s, args);
     if (err != cudaSuccess) return cuda_fail(err, "launching the decode merge kernel");

@@ -31,7 +31,10 @@ struct DecodeParams {
   int S, H, bs, MB, NB, window;
   int tt, tpb;           // rows per tile (a divisor of bs) and tiles per physical block
   int HG, G, num_ctas, nstage;   // cached heads per tile, head groups, grid size, ring depth
-  int Hq, GQ, QW;        // query heads, query heads per cached head, query heads per tile
+  int Hq, GQ, QW;        // query heads, query heads per cached head (per sub-group), query heads per tile
+  int sub;               // tensor-core kernel: head groups per cached head (1, or query sub-groups of
+                         // one cached head when it has more than 16 query heads)
+  int dim;               // head_dim (the tensor-core kernel takes 64 or 128 at run time)
   float qscale;          // softmax scale * log2(e): scores are kept in base 2
   uint32_t stage_bytes;  // bytes per pipeline stage
   uint32_t v_off, ks_off, vs_off;  // offsets of the V tile and the INT8 scale tiles in a stage
@@ -194,8 +197,12 @@ __device__ __forceinline__ long long plan_slice(const DecodeParams& p, PlanScrat
 namespace pa {
 // Tensor-core grouped-query decode (pa_decode_tc.cu).
 bool tc_decode_eligible(pa_dtype io, pa_dtype cache, int head_dim, int block_size, int group);
-size_t tc_decode_smem_bytes();
+// Query heads per head group of the tensor-core kernel: the group itself up to 16, else the
+// largest divisor of it in [4, 16] (0: none).
+int tc_decode_subgroup(int group);
 int tc_decode_tile_tokens();
+// tmKs / tmVs: fp16 scale maps of an 8-bit cache (ignored when cache == io).
 pa_status tc_decode_launch(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
-                           const DecodeParams& prm, pa_dtype io, int grid, cudaStream_t stream);
+                           const CUtensorMap& tmKs, const CUtensorMap& tmVs, const DecodeParams& prm, pa_dtype io,
+                           pa_dtype cache, int grid, cudaStream_t stream);
 }  // namespace pa

@@ -9,6 +9,10 @@
 //   O^T[128 d   x 16]  = V^T[128 d x 128 tok] . P^T[128 tok x 16 heads] (MN-major A and B)
 //
 // (query heads padded to N = 16; M = 128 puts one token, then one head dim, on each TMEM lane).
+// A cached head with more than 16 query heads (multi-query attention) is split into query
+// sub-groups of at most 16 that form head groups of their own and read the same cached
+// head; consecutive sub-groups are neighbouring segments of the tile stream, so their
+// copies of the same tiles mostly meet in L2.
 // The pages fix only the cache layout and the block-table walk ("KV Cache memory
 // optimisation and PagedAttention" (yunthe.com), section "PagedAttention注意力计算流程";
 // "vLLM source first look: PagedAttention memory design" (trdm.cn), section 三); the
@@ -23,13 +27,21 @@
 //               head warp 9 issues the value MMAs and warp 1 only the score MMAs.
 //   warps 2..5  softmax (thread = token row of S^T) and accumulation (thread = head dim row
 //               of O^T): online softmax in base 2, probabilities written as the B operand of
-//               the value MMA, V rows of unattended tokens zeroed, running output rescaled in
-//               registers.  Segment ends write the output or a partial (m, l, acc) exactly
+//               the value MMA, V rows of unattended tokens zeroed (by the widening TMA warps
+//               for an 8-bit cache), running output rescaled in registers.  Segment ends write the output or a partial (m, l, acc) exactly
 //               like the CUDA-core kernel, so the same merge kernel finishes split segments.
+// 8-bit caches (INT8 or FP8 E4M3 codes with one fp16 scale per token and head): the TMA
+// warps bring a tile's codes and scales, then widen every code in place (INT8 and E4M3
+// values are exact in fp16 and bf16): K to q's type, V to fp16, so the same MMAs run (the
+// value MMA in fp16); the softmax applies each token's K scale to its score row and folds
+// its V scale into the token's weight, rounded to fp16.  ("KV Cache optimisation strategies in deployment" (yunthe.com), section
+// "量化压缩KV Cache的INT8与FP8方案", for the 8-bit caches.)
 // Every wait is bounded; a wait that gives up sets an abort flag that ends all the others.
+#include <algorithm>
 #include <cfloat>
 #include <mutex>
 #include <type_traits>
+#include <vector>
 
 #include "pa_decode_shared.cuh"
 #include "pa_device.cuh"
@@ -39,24 +51,34 @@ namespace pa {
 namespace {
 
 constexpr int kTokens = 128;                    // tile rows (MMA M of the score product)
-constexpr int kDim = 128;                       // head_dim
+constexpr int kDim = 128;                       // head_dim (64: the hi halves stay unused)
 constexpr int kHeadsN = 16;                     // query heads per cached head, padded (MMA N)
 constexpr int kHalf = kTokens * 128;            // one 64-dim half of a tile: 128 rows x 128 B
 constexpr int kQHalf = kHeadsN * 128;           // one 64-dim half of the q rows: 16 rows x 128 B
-constexpr int kStageBytes = 4 * kHalf + 2 * kQHalf;  // K lo, K hi, V lo, V hi, Q lo, Q hi
+constexpr int kScaleBytes = kTokens * 16;       // fp16 scales of a tile for an 8-head column group
+// Stage: K lo, K hi, V lo, V hi, Q lo, Q hi (+ K scales, V scales for an 8-bit cache; the
+// codes land in K lo and V lo and are widened in place).
+constexpr int stage_bytes(bool quant) { return 4 * kHalf + 2 * kQHalf + (quant ? 2 * kScaleBytes : 0); }
 constexpr int kStages = 3;
 constexpr int kPBytes = kTokens * kHeadsN * 2;  // one probability operand, 128 tokens x 16 heads
-constexpr int kPBuffers = 4;                    // 2 tiles in flight x (hi, lo) parts
+constexpr int kConverters = 128;                // threads widening 8-bit codes (the four TMA warps)
 // Threads of the kernel tracking NH query heads per row: TMA warps 0 and 6..8, MMA warps
 // 1 and 9, softmax warps 2..5 (and 10..13 when NH = 16: two warps per TMEM lane quarter,
 // 8 heads each).
 constexpr int threads_for(int nh) { return nh > 8 ? 448 : 320; }
 static_assert(threads_for(16) <= kMaxPlanThreads, "plan_slice keeps one scratch entry per thread");
 constexpr uint32_t kTmemCols = 64;              // S0 [0,16)  S1 [16,32)  O0 [32,48)  O1 [48,64)
-constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + kPBuffers * kPBytes;
+// Probability operands: 2 tiles in flight x (hi, lo) parts for a bf16 cache, x 1 part otherwise.
+// The plan scratch shares their space (the plan is done before the first one is written).
+constexpr int p_parts(bool split) { return split ? 2 : 1; }
+constexpr size_t smem_bytes(bool quant, bool split) {
+  return 1024 + static_cast<size_t>(kStages) * stage_bytes(quant) + 2 * p_parts(split) * kPBytes;
+}
+static_assert(sizeof(PlanScratch) <= 2 * kPBytes, "plan scratch fits the probability buffers");
 
 struct TcShared {
   uint64_t full[kStages], empty[kStages];       // TMA ring
+  uint64_t conv[kStages];                       // 8-bit codes of a stage widened
   uint64_t s_full[2], s_empty[2];               // score accumulators in TMEM
   uint64_t p_full[2], o_full[2];                // probabilities written / value MMA done
   uint64_t mma_done;                            // both MMA warps' last MMAs finished
@@ -96,22 +118,68 @@ __device__ __forceinline__ void store_p_half_row(uint32_t buf, int r, int hh, co
                "r"(w[2]), "r"(w[3]) : "memory");
 }
 
-// IO: fp16 or bf16 cache and queries.  NH: query heads of a row (8 or 16 >= GQ); a softmax
-// thread tracks 8 of them.
+// Widen the 16 8-bit codes of one 16-byte chunk to 16 values of IO, exactly: out[0..3]
+// hold codes 0..7, out[4..7] codes 8..15, two per word, the lower code in the lower half.
+template <typename IO, typename CT>
+__device__ __forceinline__ void widen16(const uint4& in, uint32_t* out) {
+  const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if constexpr (std::is_same<CT, int8_t>::value && std::is_same<IO, __half>::value) {
+      // c + 128 spliced under the exponent of 1024 (0x6400 | b is the f16 value 1024 + b),
+      // minus 1152 in one f16x2 subtraction: exact for every code.
+      const uint32_t u = w[i] ^ 0x80808080u;
+      const uint32_t lo = __byte_perm(u, 0x6464u, 0x4140u), hi = __byte_perm(u, 0x6464u, 0x4342u);
+      const uint32_t bias = 0x64806480u;  // 1152, 1152
+      asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(out[2 * i]) : "r"(lo), "r"(bias));
+      asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(out[2 * i + 1]) : "r"(hi), "r"(bias));
+    } else if constexpr (std::is_same<CT, __nv_fp8_e4m3>::value && std::is_same<IO, __half>::value) {
+      e4m3x4_to_f16x2x2(w[i], out[2 * i], out[2 * i + 1]);
+    } else {
+      // bf16 operands: through fp32 (exact), then a pair conversion (exact: 8-bit values
+      // have at most 7 significant bits, and E4M3's exponents lie inside bf16's range).
+      float f[4];
+      if constexpr (std::is_same<CT, int8_t>::value) {
+        const uint32_t u = w[i] ^ 0x80808080u;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) f[b] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7440u | b)) - 8388736.0f;
+      } else {
+        uint32_t lo, hi;
+        e4m3x4_to_f16x2x2(w[i], lo, hi);
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+        f[0] = a.x, f[1] = a.y, f[2] = b.x, f[3] = b.y;
+      }
+      const __nv_bfloat162 p0 = __floats2bfloat162_rn(f[0], f[1]), p1 = __floats2bfloat162_rn(f[2], f[3]);
+      out[2 * i] = *reinterpret_cast<const uint32_t*>(&p0);
+      out[2 * i + 1] = *reinterpret_cast<const uint32_t*>(&p1);
+    }
+  }
+}
+
+// IO: fp16 or bf16 queries (and cache, unless CT is an 8-bit code type).  NH: query heads of
+// a row (8 or 16 >= GQ); a softmax thread tracks 8 of them.
 // bf16 probabilities are split into hi + lo bf16 parts and the value MMA runs on both, so
 // the weights keep ~16 significant bits (one bf16 part alone keeps 8).
-template <typename IO, int NH>
+template <typename IO, typename CT, int NH>
 __global__ void __launch_bounds__(threads_for(NH), 1)
 decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                     const __grid_constant__ CUtensorMap tmQ, const DecodeParams p) {
-  constexpr bool kSplit = std::is_same<IO, __nv_bfloat16>::value;
-  constexpr uint32_t kFmt = kSplit ? 1u : 0u;
+                     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKs,
+                     const __grid_constant__ CUtensorMap tmVs, const DecodeParams p) {
+  constexpr bool kQuant = !std::is_same<CT, IO>::value;  // 8-bit codes + per-token scales
+  // bf16 weights keep ~16 bits as hi + lo parts; with an 8-bit cache (tolerance 1e-2) one
+  // part is enough.
+  constexpr bool kSplit = std::is_same<IO, __nv_bfloat16>::value && !kQuant;
+  constexpr int kStageBytes = stage_bytes(kQuant);
+  constexpr int kParts = p_parts(kSplit);
+  constexpr uint32_t kFmt = std::is_same<IO, __nv_bfloat16>::value ? 1u : 0u;
   constexpr uint32_t kIdescS = mma_idesc_f16(kFmt, 0, 0, kTokens, kHeadsN);  // K-major A and B
-  constexpr uint32_t kIdescO = mma_idesc_f16(kFmt, 1, 1, kDim, kHeadsN);     // MN-major A and B
+  // The value MMA of an 8-bit cache runs in fp16 whatever q's type: V codes are exact in fp16
+  // and a weight p * v_scale keeps 11 significant bits there (8 in bf16).
+  constexpr uint32_t kIdescO = mma_idesc_f16(kQuant ? 0u : kFmt, 1, 1, kDim, kHeadsN);  // MN-major A and B
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ TcShared sh;
-  __shared__ PlanScratch plan;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int GQ = p.GQ;
@@ -119,16 +187,20 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
   grid_dependency_launch_next();
   grid_dependency_wait();
 
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;  // swizzle atoms are 1024-B aligned
+  const uint32_t pbase = base + kStages * kStageBytes;
+  auto stage = [&](int st) { return base + st * kStageBytes; };
+  auto pbuf = [&](int b, int part) { return pbase + (kParts * b + part) * kPBytes; };
+
   Cursor start;
   long long t0 = 0;
+  PlanScratch& plan = *reinterpret_cast<PlanScratch*>(smem_raw + (pbase - smem_u32(smem_raw)));
   const long long count = plan_slice(p, plan, &t0, &start);
   if (count == 0) return;
   const int n = static_cast<int>(count);
+  __syncthreads();  // every thread is done with the plan scratch before its space is reused
 
-  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;  // swizzle atoms are 1024-B aligned
-  auto stage = [&](int st) { return base + st * kStageBytes; };
-  auto pbuf = [&](int b, int part) { return base + kStages * kStageBytes + (2 * b + part) * kPBytes; };
-  const uint32_t full0 = smem_u32(&sh.full[0]), empty0 = smem_u32(&sh.empty[0]);
+  const uint32_t full0 = smem_u32(&sh.full[0]), empty0 = smem_u32(&sh.empty[0]), conv0 = smem_u32(&sh.conv[0]);
   const uint32_t s_full0 = smem_u32(&sh.s_full[0]), s_empty0 = smem_u32(&sh.s_empty[0]);
   const uint32_t p_full0 = smem_u32(&sh.p_full[0]), o_full0 = smem_u32(&sh.o_full[0]);
   volatile int* abort = &sh.abort;
@@ -137,6 +209,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     for (int st = 0; st < kStages; ++st) {
       mbar_init(full0 + 8 * st, 4);  // one arrival per TMA warp
       mbar_init(empty0 + 8 * st, 1);
+      mbar_init(conv0 + 8 * st, kConverters);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full0 + 8 * b, 1);
@@ -167,8 +240,11 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     // Four warps, one per (K or V) x (64-dim half) part of a tile: a warp issues its copies
     // one after another, so four warps issue a tile four times as fast as one.  Warp 0
     // also loads the q rows.  Every warp walks the same tile stream and block table.
+    // 8-bit cache: the parts are K codes (+ q rows), V codes, K scales and V scales, and the
+    // four warps then widen the codes of the tile issued kLag tiles earlier, thread = row.
     const int part = warp == 0 ? 0 : warp - 5;  // 0: K lo, 1: K hi, 2: V lo, 3: V hi
-    const CUtensorMap* map = part < 2 ? &tmK : &tmV;
+    const CUtensorMap* map = kQuant ? (part == 0 ? &tmK : part == 1 ? &tmV : part == 2 ? &tmKs : &tmVs)
+                                    : (part < 2 ? &tmK : &tmV);
     const uint64_t policy = l2_policy_evict_first();
     if (lane == 0) {
       prefetch_tensormap(map);
@@ -189,8 +265,58 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     int fst_seq = -1, fst_base = 0, fst = 0;     // first window of the sequence
     Cursor c = start;
     int issued = 0;
+    // Widening of 8-bit codes.  Thread r owns token row r of the tile: it reads the row's
+    // 128 codes (8 swizzled 16-byte chunks) into registers, then writes dims 0..63 over the
+    // same 128 bytes and dims 64..127 into the hi half, both in the 128-byte-swizzled
+    // layout the MMAs read.  V rows of unattended tokens become zeros (they may hold
+    // anything, and 0 * NaN would poison the weighted sum).  A stage is handed to the MMA
+    // issuer once all 128 rows are done.  kLag = 2 keeps a tile of copies in flight while one
+    // is widened; a stage's reuse waits for the value MMA of the tile three back, whose codes
+    // were widened in an earlier iteration, so the ring cannot stall on itself.
+    constexpr int kLag = 2;
+    Cursor cc = start;
+    int widened = 0;
+    const int wr = 32 * part + lane;  // row this thread widens
+    auto widen_tile = [&]() -> bool {
+      const int st = widened % kStages;
+      if (!wait_or_abort(full0 + 8 * st, (widened / kStages) & 1, abort)) return false;
+      const int tok = (cc.sp.first_t + cc.j) * kTokens + wr;
+      const bool valid = tok >= cc.sp.lo && tok < cc.sp.ctx;
+      const uint32_t sw = wr & 7;
+#pragma unroll
+      for (int kv = 0; kv < 2; ++kv) {  // K codes in K lo, V codes in V lo
+        const uint32_t row = stage(st) + kv * 2 * kHalf + wr * 128;
+        uint4 raw[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) raw[k] = ld_shared_v4(row + 16 * (k ^ sw));
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {  // codes 16k .. 16k + 15 -> 16-byte chunks 2k, 2k + 1
+          uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+          if (kv == 0)
+            widen16<IO, CT>(raw[k], o);       // K: the score MMA's type, q's
+          else if (valid)
+            widen16<__half, CT>(raw[k], o);   // V: fp16, like the weights of the value MMA
+          const uint32_t dst = row + (k >= 4 ? kHalf : 0);
+          const uint32_t m0 = (2 * k) & 7, m1 = (2 * k + 1) & 7;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16 * (m0 ^ sw)), "r"(o[0]), "r"(o[1]),
+                       "r"(o[2]), "r"(o[3]) : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16 * (m1 ^ sw)), "r"(o[4]), "r"(o[5]),
+                       "r"(o[6]), "r"(o[7]) : "memory");
+        }
+      }
+      fence_proxy_async_shared();  // the widened operands are read by the tensor cores
+      mbar_arrive(conv0 + 8 * st);
+      ++widened;
+      if (widened < n) advance(cc, p);
+      return true;
+    };
     for (; issued < n; ++issued) {
+      // Widen the tile issued kLag tiles ago first: its copies need no more than time, while
+      // the stage this tile needs may wait for the value MMA of the tile three back, which in
+      // turn waits for widened operands.
+      if (kQuant && issued - widened >= kLag && !widen_tile()) break;
       const int st = issued % kStages;
+      const int kh = c.g / p.sub;  // cached head of this head group
       const int tok0 = (c.sp.first_t + c.j) * kTokens;
       const int lb_first = tok0 / bs;
       const int lb_lo = max(lb_first, c.sp.lo / bs), lb_hi = min(lb_first + bpt - 1, (c.sp.ctx - 1) / bs);
@@ -218,23 +344,39 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         if (issued >= kStages) ok = wait_or_abort(empty0 + 8 * st, ((issued / kStages) - 1) & 1, abort);
         if (ok) {
           const uint32_t bar = full0 + 8 * st;
-          mbar_arrive_expect_tx(bar, (part == 0 ? 2u * GQ * 128u : 0u) + static_cast<uint32_t>(nload) * bs * 128u);
+          const uint32_t row_bytes = kQuant && part >= 2 ? 16u : 128u;  // a scale row: 8 heads x fp16
+          const uint32_t halves = p.dim / 64;  // 64-dim halves of q (and of K, V) to copy
+          const int nblk = (!kQuant && (part & 1) && halves == 1) ? 0 : nload;  // head_dim 64: no hi halves
+          mbar_arrive_expect_tx(bar, (part == 0 ? halves * GQ * 128u : 0u) + static_cast<uint32_t>(nblk) * bs * row_bytes);
           if (part == 0) {
             const uint32_t sb = stage(st);
             const int qrow = c.s * p.Hq + c.g * GQ;
             tma_load_2d(sb + 4 * kHalf, &tmQ, bar, 0, qrow, policy);
-            tma_load_2d(sb + 4 * kHalf + kQHalf, &tmQ, bar, 64, qrow, policy);
+            if (halves == 2) tma_load_2d(sb + 4 * kHalf + kQHalf, &tmQ, bar, 64, qrow, policy);
           }
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);  // also orders lane 0's expect_tx before any copy
       if (!ok) break;
-      if (lane < nload) {  // this warp's part of each attended block, one copy per lane
-        const uint32_t row = static_cast<uint32_t>(lb_lo + lane - lb_first) * bs * 128u;
-        tma_load_3d(stage(st) + part * kHalf + row, map, full0 + 8 * st, (part & 1) * 64, c.g, pb * bs, policy);
+      const bool copies = kQuant || !(part & 1) || p.dim == 128;  // head_dim 64: the hi-half warps only arrive
+      if (copies && lane < nload) {  // this warp's part of each attended block, one copy per lane
+        const uint32_t row0 = static_cast<uint32_t>(lb_lo + lane - lb_first) * bs;  // first row in the tile
+        if constexpr (kQuant) {
+          if (part < 2)
+            tma_load_3d(stage(st) + part * 2 * kHalf + row0 * 128u, map, full0 + 8 * st, 0, kh, pb * bs, policy);
+          else  // scale rows: x rounded down to a 16-byte boundary (8 heads)
+            tma_load_2d(stage(st) + 4 * kHalf + 2 * kQHalf + (part - 2) * kScaleBytes + row0 * 16u, map,
+                        full0 + 8 * st, kh & ~7, pb * bs, policy);
+        } else {
+          tma_load_3d(stage(st) + part * kHalf + row0 * 128u, map, full0 + 8 * st, (part & 1) * 64, kh, pb * bs,
+                      policy);
+        }
       }
       advance(c, p);
     }
+    if (kQuant && !*abort)
+      while (widened < issued)
+        if (!widen_tile()) break;
     if (lane == 0)  // never leave with copies in flight
       for (int k = issued - kStages < 0 ? 0 : issued - kStages; k < issued; ++k)
         wait_or_abort(full0 + 8 * (k % kStages), (k / kStages) & 1, abort);
@@ -248,6 +390,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       const uint32_t sb = stage(st);
 #pragma unroll
       for (int kk = 0; kk < kDim / 16; ++kk) {
+        if (kk * 16 >= p.dim) break;  // head_dim 64: the lo halves only
         const uint32_t koff = (kk / 4) * kHalf + (kk % 4) * 32;  // 32 B steps inside a swizzled row
         const uint32_t qoff = 4 * kHalf + (kk / 4) * kQHalf + (kk % 4) * 32;
         tc_mma_f16(tmem + b * kHeadsN, smem_desc(sb + koff, 16, 1024, kSwizzle128B),
@@ -260,7 +403,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       const uint32_t sb = stage(i % kStages);
       const uint32_t o_tmem = tmem + 2 * kHeadsN + b * kHeadsN;
 #pragma unroll
-      for (int part = 0; part < (kSplit ? 2 : 1); ++part) {
+      for (int part = 0; part < kParts; ++part) {
 #pragma unroll
         for (int kk = 0; kk < kTokens / 16; ++kk) {
           tc_mma_f16(o_tmem, smem_desc(sb + 2 * kHalf + kk * 2048, kHalf, 1024, kSwizzle128B),
@@ -275,10 +418,11 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     // softmax work per tile is larger and one lane of warp 1 polling for either kind of
     // ready work measured faster (3.98 vs 3.08 TB/s at 4 cached heads); warp 9 then idles.
     constexpr bool kTwoIssuers = NH <= 8;
+    const uint32_t ready0 = kQuant ? conv0 : full0;  // a stage's operands are complete
     if (lane == 0 && kTwoIssuers) {
       if (warp == 1) {
         for (int i = 0; i < n; ++i) {
-          if (!wait_or_abort(full0 + 8 * (i % kStages), (i / kStages) & 1, abort)) break;
+          if (!wait_or_abort(ready0 + 8 * (i % kStages), (i / kStages) & 1, abort)) break;
           if (i >= 2 && !wait_or_abort(s_empty0 + 8 * (i % 2), ((i / 2) - 1) & 1, abort)) break;
           tc_fence_after_sync();
           issue_scores(i);
@@ -296,7 +440,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       uint32_t idle = 0;
       while (o_next < n) {
         bool progressed = false;
-        if (s_next < n && mbar_test_wait(full0 + 8 * (s_next % kStages), (s_next / kStages) & 1) &&
+        if (s_next < n && mbar_test_wait(ready0 + 8 * (s_next % kStages), (s_next / kStages) & 1) &&
             (s_next < 2 || mbar_test_wait(s_empty0 + 8 * (s_next % 2), ((s_next / 2) - 1) & 1))) {
           tc_fence_after_sync();
           issue_scores(s_next++);
@@ -364,9 +508,16 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
 
       const int tok = (c.sp.first_t + c.j) * kTokens + r;
       const bool valid = tok >= c.sp.lo && tok < c.sp.ctx;
+      float kscale = 1.f, vscale = 1.f;  // this token's 8-bit scales
+      if (kQuant && valid) {
+        const uint32_t sa = stage(st) + 4 * kHalf + 2 * kQHalf + r * 16 + 2 * ((c.g / p.sub) & 7);
+        kscale = __half2float(__ushort_as_half(ld_shared_u16(sa)));
+        vscale = __half2float(__ushort_as_half(ld_shared_u16(sa + kScaleBytes)));
+      }
+      const float sfac = p.qscale * kscale;
 #pragma unroll
       for (int h = 0; h < HPW; ++h) {
-        sc[h] = (valid && h_base + h < GQ) ? sc[h] * p.qscale : -INFINITY;
+        sc[h] = (valid && h_base + h < GQ) ? sc[h] * sfac : -INFINITY;
         float x = sc[h];
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
@@ -385,6 +536,11 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         alpha[h] = exp2f(m[h] - m_new);
         m[h] = m_new;
         const float pr = sc[h] == -INFINITY ? 0.f : exp2f(sc[h] - m_new);
+        if constexpr (kQuant) {  // the value MMA multiplies V codes: fold the V scale into the weight
+          w_hi[h / 2] |= bits16(float_to<__half>(pr * vscale)) << (16 * (h & 1));
+          l[h] = l[h] * alpha[h] + pr;
+          continue;
+        }
         const IO hi = float_to<IO>(pr);
         w_hi[h / 2] |= bits16(hi) << (16 * (h & 1));
         if (kSplit) {
@@ -402,12 +558,15 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         store_p_row(pbuf(b, 0), r, w_hi);
         if (kSplit) store_p_row(pbuf(b, 1), r, w_lo);
       }
-      if (!valid && hh == 0) {  // unattended rows may hold anything (NaN): give the value MMA zeros
+      if (!kQuant && !valid && hh == 0) {  // unattended rows may hold anything (NaN): give the value MMA zeros
+        // Chunk k ^ (r & 7) at step k: neighbouring rows (128 B apart, the same banks)
+        // write different 16-byte chunks at each step, so a warp's stores do not conflict.
         const uint32_t v0 = stage(st) + 2 * kHalf + r * 128;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(v0 + 16 * k), "r"(0) : "memory");
-          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(v0 + kHalf + 16 * k), "r"(0) : "memory");
+          const uint32_t c = 16 * (k ^ (r & 7));
+          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(v0 + c), "r"(0) : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(v0 + kHalf + c), "r"(0) : "memory");
         }
       }
       fence_proxy_async_shared();
@@ -444,17 +603,18 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         named_barrier_sync(1, kSoftmax);  // sh.red_l is free again
         const int h0 = c.g * GQ + h_base;
         if (seg_from_start && seg_last) {
-          IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(c.s) * p.Hq + h0) * kDim + r;
+          IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(c.s) * p.Hq + h0) * p.dim + r;
+          if (r < p.dim)  // (head_dim 64: rows 64..127 of O^T come from the unused V hi half)
 #pragma unroll
-          for (int h = 0; h < HPW; ++h)
-            if (h_base + h < GQ) orow[static_cast<size_t>(h) * kDim] = float_to<IO>(acc[h] / lt[h]);
+            for (int h = 0; h < HPW; ++h)
+              if (h_base + h < GQ) orow[static_cast<size_t>(h) * p.dim] = float_to<IO>(acc[h] / lt[h]);
         } else {
           const long long slot = blockIdx.x + static_cast<long long>(c.s) * p.G + c.g;
 #pragma unroll
           for (int h = 0; h < HPW; ++h) {
             const int hg = h_base + h;
             if (hg >= GQ) continue;
-            p.ws_acc[(slot * GQ + hg) * kDim + r] = acc[h];
+            if (r < p.dim) p.ws_acc[(slot * GQ + hg) * p.dim + r] = acc[h];
             if (r == 0) {
               p.ws_ml[(slot * GQ + hg) * 2 + 0] = m[h];
               p.ws_ml[(slot * GQ + hg) * 2 + 1] = lt[h];
@@ -501,34 +661,59 @@ struct RegisterTc {
 
 }  // namespace
 
-bool tc_decode_eligible(pa_dtype io, pa_dtype cache, int head_dim, int block_size, int group) {
-  return (io == PA_F16 || io == PA_BF16) && cache == io && head_dim == kDim && block_size >= 8 &&
-         block_size <= kTokens && block_size % 8 == 0 && kTokens % block_size == 0 && group >= 4 &&
-         group <= kHeadsN;
+int tc_decode_subgroup(int group) {
+  if (group <= kHeadsN) return group;
+  for (int sg = kHeadsN; sg >= 4; --sg)
+    if (group % sg == 0) return sg;
+  return 0;
 }
 
-size_t tc_decode_smem_bytes() { return kSmemBytes; }
+bool tc_decode_eligible(pa_dtype io, pa_dtype cache, int head_dim, int block_size, int group) {
+  const bool eight_bit = cache == PA_I8 || cache == PA_FP8_E4M3;
+  return (io == PA_F16 || io == PA_BF16) && (cache == io || eight_bit) &&
+         (head_dim == kDim || (head_dim == 64 && !eight_bit)) && block_size >= 8 &&
+         block_size <= kTokens && block_size % 8 == 0 && kTokens % block_size == 0 && group >= 4 &&
+         tc_decode_subgroup(group) >= 4;
+}
 
 int tc_decode_tile_tokens() { return kTokens; }
 
+namespace {
+template <typename IO, typename CT, int NH>
+const void* tc_fn() {
+  return reinterpret_cast<const void*>(&decode_gqa_tc_kernel<IO, CT, NH>);
+}
+template <typename IO, int NH>
+const void* tc_fn_for_cache(pa_dtype cache) {
+  return cache == PA_I8 ? tc_fn<IO, int8_t, NH>() : cache == PA_FP8_E4M3 ? tc_fn<IO, __nv_fp8_e4m3, NH>()
+                                                                         : tc_fn<IO, IO, NH>();
+}
+}  // namespace
+
 pa_status tc_decode_launch(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
-                           const DecodeParams& prm, pa_dtype io, int grid, cudaStream_t stream) {
+                           const CUtensorMap& tmKs, const CUtensorMap& tmVs, const DecodeParams& prm, pa_dtype io,
+                           pa_dtype cache, int grid, cudaStream_t stream) {
   const bool small = prm.GQ <= 8;
-  const void* fn = io == PA_BF16
-                       ? (small ? reinterpret_cast<const void*>(&decode_gqa_tc_kernel<__nv_bfloat16, 8>)
-                                : reinterpret_cast<const void*>(&decode_gqa_tc_kernel<__nv_bfloat16, 16>))
-                       : (small ? reinterpret_cast<const void*>(&decode_gqa_tc_kernel<__half, 8>)
-                                : reinterpret_cast<const void*>(&decode_gqa_tc_kernel<__half, 16>));
-  static std::once_flag once[4];
-  cudaError_t attr_err = cudaSuccess;
-  std::call_once(once[(io == PA_BF16 ? 2 : 0) + (small ? 1 : 0)], [&] {
-    attr_err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
-  });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(tensor-core decode)");
-  CUtensorMap k = tmK, v = tmV, q = tmQ;
+  const bool quant = cache != io;
+  const void* fn = io == PA_BF16 ? (small ? tc_fn_for_cache<__nv_bfloat16, 8>(cache)
+                                          : tc_fn_for_cache<__nv_bfloat16, 16>(cache))
+                                 : (small ? tc_fn_for_cache<__half, 8>(cache) : tc_fn_for_cache<__half, 16>(cache));
+  const size_t smem = smem_bytes(quant, io == PA_BF16 && !quant);
+  // The dynamic shared-memory limit is a per-kernel attribute: set once per kernel.
+  static std::mutex m;
+  static std::vector<const void*> ready;
+  {
+    std::lock_guard<std::mutex> lock(m);
+    if (std::find(ready.begin(), ready.end(), fn) == ready.end()) {
+      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tensor-core decode)");
+      ready.push_back(fn);
+    }
+  }
+  CUtensorMap k = tmK, v = tmV, q = tmQ, ks = tmKs, vs = tmVs;
   DecodeParams p = prm;
-  void* args[] = {&k, &v, &q, &p};
-  cudaError_t err = launch_dependent(fn, dim3(grid), dim3(small ? threads_for(8) : threads_for(16)), kSmemBytes, stream, args);
+  void* args[] = {&k, &v, &q, &ks, &vs, &p};
+  cudaError_t err = launch_dependent(fn, dim3(grid), dim3(small ? threads_for(8) : threads_for(16)), smem, stream, args);
   if (err != cudaSuccess) return cuda_fail(err, "launching the tensor-core decode kernel");
   return PA_OK;
 }

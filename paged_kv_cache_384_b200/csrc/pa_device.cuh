@@ -109,14 +109,6 @@ template <> struct Elem<int8_t> {
       }
     }
   }
-  // The same widening two codes at a time on packed pairs: codes 2j and 2j+1 of v.
-  static __device__ __forceinline__ uint64_t pair(const uint4& v, int j) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    const uint32_t u = w[j >> 1] ^ 0x80808080u;
-    const int b = 2 * (j & 1);
-    return f2_add(f2_pack_bits(__byte_perm(u, 0x4B000000u, 0x7440u | b), __byte_perm(u, 0x4B000000u, 0x7440u | (b + 1))),
-                  f2_pack(-8388736.0f, -8388736.0f));
-  }
 };
 
 // OCP FP8 E4M3 codes: the hardware converts pairs to fp16 exactly (every E4M3 value is an
@@ -140,26 +132,43 @@ template <> struct Elem<__nv_fp8_e4m3> {
   }
 };
 
-// Dot product and axpy over the 16 8-bit codes of one 16-byte vector on packed fp32 pairs
-// (Elem<CT>::pair widens two codes).  q2 and acc2 hold 8 packed pairs each.
-template <typename CT>
-__device__ __forceinline__ float dot_pairs(const uint4& v, const uint64_t* q2) {
-  uint64_t a0 = 0, a1 = 0;  // two pair accumulators: four partial sums
-#pragma unroll
-  for (int j = 0; j < 8; j += 2) {
-    a0 = f2_fma(q2[j], Elem<CT>::pair(v, j), a0);
-    a1 = f2_fma(q2[j + 1], Elem<CT>::pair(v, j + 1), a1);
-  }
-  float x0, x1, x2, x3;
-  f2_unpack(a0, x0, x1);
-  f2_unpack(a1, x2, x3);
-  return (x0 + x1) + (x2 + x3);
+// Four-way byte dot products with a 32-bit accumulator: c + sum_k a.byte[k] * b.byte[k], the
+// bytes of `a` signed; those of `b` signed (ss) or unsigned (su).  Exact integer arithmetic.
+__device__ __forceinline__ int dp4a_ss(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
-template <typename CT>
-__device__ __forceinline__ void axpy_pairs(float w, const uint4& v, uint64_t* acc2) {
-  const uint64_t w2 = f2_pack(w, w);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) acc2[j] = f2_fma(w2, Elem<CT>::pair(v, j), acc2[j]);
+__device__ __forceinline__ int dp4a_su(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// Four E4M3 codes (bytes of w, lowest first) -> two f16 pairs, exactly (every E4M3 value is
+// an f16 value): lo = codes 0, 1 and hi = codes 2, 3, the lower code in the lower half.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+// c + a.lo * b.lo + a.hi * b.hi for f16 pairs a, b with f32 accumulation (sm_100 mixed-precision
+// fma: each f16 x f16 product is exact in fp32, one rounding per addition).
+__device__ __forceinline__ float fma2_f16_f32(uint32_t a, uint32_t b, float c) {
+  float d;
+  asm("{\n\t.reg .f16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+      "fma.rn.f32.f16 %0, a0, b0, %3;\n\tfma.rn.f32.f16 %0, a1, b1, %0;\n\t}"
+      : "=f"(d)
+      : "r"(a), "r"(b), "f"(c));
+  return d;
+}
+// c0 += a.lo * b.lo and c1 += a.hi * b.hi, f16 inputs, f32 accumulators.
+__device__ __forceinline__ void fma_f16x2_f32x2(uint32_t a, uint32_t b, float& c0, float& c1) {
+  asm("{\n\t.reg .f16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %2;\n\tmov.b32 {b0, b1}, %3;\n\t"
+      "fma.rn.f32.f16 %0, a0, b0, %0;\n\tfma.rn.f32.f16 %1, a1, b1, %1;\n\t}"
+      : "+f"(c0), "+f"(c1)
+      : "r"(a), "r"(b));
 }
 
 template <typename T> __device__ __forceinline__ T float_to(float x);

@@ -13,7 +13,8 @@
 //
 // A persistent grid (one CTA per SM) works through units of 128 query rows of one cached
 // head: tq = 128 / GQ consecutive query tokens times the GQ query heads that share the
-// cached head (row = token * GQ + head).  Per 128-token KV tile of a unit:
+// cached head (row = token * GQ + head; GQ a power of two up to 128, so multi-query
+// attention with up to 128 query heads per cached head fits one unit's rows).  Per 128-token KV tile of a unit:
 //
 //   S[128 rows x 128 kv]  = Q[128 x 128 d] . K^T          (K-major A and B in shared memory)
 //   O_h[128 rows x 128 d] += P[:, 64h..] . V[64h.., :]   (A = P in TMEM over S, MN-major V)
@@ -36,11 +37,21 @@
 //                probabilities into TMEM as the A operand; the halves are merged when the
 //                unit's rows are written, which happens after the next unit's first tile.
 // bf16 probabilities are split into hi + lo bf16 parts (two value MMAs) so the weights keep
-// ~16 significant bits.  Every wait is bounded; one that gives up raises PA_DEVERR_TIMEOUT
-// and an abort flag that ends the others.
+// ~16 significant bits.
+// 8-bit caches (INT8 or FP8 E4M3 codes with one fp16 scale per token and cached head, "KV
+// Cache optimisation strategies in deployment" (yunthe.com), section
+// "量化压缩KV Cache的INT8与FP8方案"): the copy warps bring each tile's codes (one 128-byte row
+// per token) into the lo half of its ring slot, and warps 4..7, one thread per kv row, turn
+// them in place into the 16-bit operand -- code times the row's scale, rounded once: K to
+// the I/O type (relative error 2^-11 for fp16, 2^-8 for bf16), V to fp16 (2^-11) -- with
+// zeros in rows no query attends; the MMA warp then sees an ordinary 16-bit tile, and the
+// value MMA runs in fp16 with fp16 weights whatever the I/O type (no hi + lo split).
+// Every wait is bounded; one that gives up raises PA_DEVERR_TIMEOUT and an abort flag that
+// ends the others.
 #include <cfloat>
 #include <mutex>
 #include <type_traits>
+#include <vector>
 
 #include "pa_device.cuh"
 #include "pa_host.h"
@@ -80,6 +91,8 @@ constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(1 + 2 * kRing) * kOpByt
 
 struct PrefillParams {
   void* out;
+  const uint16_t* k_scale;  // [NB*bs][Hkv] fp16 bits (8-bit cache only)
+  const uint16_t* v_scale;
   const int32_t* block_tables;
   const int32_t* cu_q;
   const int32_t* context_lens;
@@ -92,6 +105,7 @@ struct PrefillParams {
 struct PfShared {
   uint64_t q_full, q_empty, o_free;  // q rows landed / read by the last score MMA; O read out
   uint64_t k_full[kRing], k_empty[kRing], v_full[kRing], v_empty[kRing];
+  uint64_t k_conv[kRing], v_conv[kRing];  // 8-bit codes of a slot widened into the operand
   uint64_t s_full[2];
   uint64_t p_full[2], o_full[2];  // by tile parity: probabilities written / value MMA done
   uint64_t mma_done;
@@ -253,12 +267,61 @@ struct TableWindow {
 // halves) on 1, V lo on 2, V hi on 3.  Warps 4..7 are idle.
 constexpr int kMmaWarp = 0;
 constexpr int kCopyWarpsK = 1, kCopyWarpsV = 2;  // copy warps per tensor
+constexpr int kConvWarp0 = 4, kConvThreads = 128;  // warps 4..7 widen 8-bit codes, one kv row each
 __device__ __forceinline__ int copy_role(int warp) {
   switch (warp) {
     case 1: return 3;      // K, both halves
     case 2: return 4 + 1;  // V, lo half
     case 3: return 4 + 2;  // V, hi half
     default: return -1;
+  }
+}
+
+// 16 8-bit codes (one 16-byte chunk) times a scale, rounded to IO: out[0..3] hold codes 0..7,
+// out[4..7] codes 8..15, two per word, the lower code in the lower half.  fp16: the codes
+// widen exactly to f16 pairs, then one f16x2 multiply rounds each product once.  bf16: the
+// codes widen exactly to fp32, the product is rounded to fp32 and then to bf16.
+template <typename IO, typename CT>
+__device__ __forceinline__ void widen_scaled16(const uint4& in, float scale, uint32_t* out) {
+  const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+  if constexpr (std::is_same<IO, __half>::value) {
+    const __half2 s2 = __float2half2_rn(scale);  // the stored fp16 scale: exact
+    const uint32_t sb = *reinterpret_cast<const uint32_t*>(&s2);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t lo, hi;
+      if constexpr (std::is_same<CT, int8_t>::value) {
+        // c + 128 spliced under the exponent of 1024, minus 1152: exact f16 codes
+        const uint32_t u = w[i] ^ 0x80808080u;
+        const uint32_t bias = 0x64806480u;
+        asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(lo) : "r"(__byte_perm(u, 0x6464u, 0x4140u)), "r"(bias));
+        asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(__byte_perm(u, 0x6464u, 0x4342u)), "r"(bias));
+      } else {
+        e4m3x4_to_f16x2x2(w[i], lo, hi);
+      }
+      asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out[2 * i]) : "r"(lo), "r"(sb));
+      asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out[2 * i + 1]) : "r"(hi), "r"(sb));
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float f[4];
+      if constexpr (std::is_same<CT, int8_t>::value) {
+        const uint32_t u = w[i] ^ 0x80808080u;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) f[b] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7440u | b)) - 8388736.0f;
+      } else {
+        uint32_t lo, hi;
+        e4m3x4_to_f16x2x2(w[i], lo, hi);
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+        f[0] = a.x, f[1] = a.y, f[2] = b.x, f[3] = b.y;
+      }
+      const __nv_bfloat162 p0 = __floats2bfloat162_rn(f[0] * scale, f[1] * scale);
+      const __nv_bfloat162 p1 = __floats2bfloat162_rn(f[2] * scale, f[3] * scale);
+      out[2 * i] = *reinterpret_cast<const uint32_t*>(&p0);
+      out[2 * i + 1] = *reinterpret_cast<const uint32_t*>(&p1);
+    }
   }
 }
 
@@ -269,14 +332,18 @@ template <int N> __device__ __forceinline__ void regs_increase() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-template <typename IO>
+template <typename IO, typename CT>
 __global__ void __launch_bounds__(kThreads, 1)  // 16 warps, 128 registers each at launch
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmQ, const PrefillParams p) {
-  constexpr bool kSplit = std::is_same<IO, __nv_bfloat16>::value;
-  constexpr uint32_t kFmt = kSplit ? 1u : 0u;
+  constexpr bool kQuant = !std::is_same<CT, IO>::value;  // 8-bit codes + per-token scales
+  constexpr bool kSplit = std::is_same<IO, __nv_bfloat16>::value && !kQuant;
+  constexpr uint32_t kFmt = std::is_same<IO, __nv_bfloat16>::value ? 1u : 0u;
   constexpr uint32_t kIdescS = mma_idesc_f16(kFmt, 0, 0, kRows, kKv);  // K-major Q and K
-  constexpr uint32_t kIdescO = mma_idesc_f16(kFmt, 0, 1, kRows, kDim);  // K-major P, MN-major V
+  // With an 8-bit cache the value MMA runs in fp16 whatever q's type: V rows (code x scale)
+  // and the weights then keep 11 significant bits (8 in bf16).
+  using PW = typename std::conditional<kQuant, __half, IO>::type;  // probability / V operand type
+  constexpr uint32_t kIdescO = mma_idesc_f16(kQuant ? 0u : kFmt, 0, 1, kRows, kDim);  // K-major P, MN-major V
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ PfShared sh;
@@ -293,6 +360,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   const uint32_t q_full = smem_u32(&sh.q_full), q_empty = smem_u32(&sh.q_empty), o_free = smem_u32(&sh.o_free);
   const uint32_t k_full0 = smem_u32(&sh.k_full[0]), k_empty0 = smem_u32(&sh.k_empty[0]);
   const uint32_t v_full0 = smem_u32(&sh.v_full[0]), v_empty0 = smem_u32(&sh.v_empty[0]);
+  const uint32_t k_conv0 = smem_u32(&sh.k_conv[0]), v_conv0 = smem_u32(&sh.v_conv[0]);
+  // The MMA warp's operands are complete once the copies landed (16-bit cache) or once the
+  // codes were widened (8-bit cache).
+  const uint32_t k_ready0 = kQuant ? k_conv0 : k_full0, v_ready0 = kQuant ? v_conv0 : v_full0;
   const uint32_t s_full0 = smem_u32(&sh.s_full[0]);
   const uint32_t p_full0 = smem_u32(&sh.p_full[0]), o_full0 = smem_u32(&sh.o_full[0]);
   const uint32_t mma_done = smem_u32(&sh.mma_done);
@@ -307,6 +378,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       mbar_init(k_empty0 + 8 * st, 1);
       mbar_init(v_full0 + 8 * st, kCopyWarpsV);
       mbar_init(v_empty0 + 8 * st, 1);
+      mbar_init(k_conv0 + 8 * st, kConvThreads);
+      mbar_init(v_conv0 + 8 * st, kConvThreads);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full0 + 8 * b, 1);
@@ -388,15 +461,18 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
             if (!is_v && h0 == 0) prefill_error(PA_DEVERR_TABLE);
             pb = 0;
           }
-          if (lane == 0) mbar_arrive_expect_tx(full0 + 8 * st, static_cast<uint32_t>(nh * nload) * bs * 128u);
+          // 8-bit cache: one copy per block (a token's 128 codes are one 128-byte row) into
+          // the slot's lo half, by the K warp and the V lo warp; the V hi warp only arrives.
+          const int ncopy = kQuant ? (is_v && h0 == 1 ? 0 : 1) : nh;  // copies per block
+          if (lane == 0) mbar_arrive_expect_tx(full0 + 8 * st, static_cast<uint32_t>(ncopy * nload) * bs * 128u);
           __syncwarp();
-          const int bi = nh == 2 ? lane >> 1 : lane;  // block of this lane's copy
-          const int dh = nh == 2 ? lane & 1 : h0;     // and its 64-dim half
+          const int bi = ncopy == 2 ? lane >> 1 : lane;  // block of this lane's copy
+          const int dh = ncopy == 2 ? lane & 1 : (kQuant ? 0 : h0);  // and its 64-dim half
           const int blk = __shfl_sync(0xffffffffu, pb, bi & 31);
-          if (lane < nh * nload) {  // nh * nload <= 32 copies, one per lane
+          if (lane < ncopy * nload) {  // ncopy * nload <= 32 copies, one per lane
             const uint32_t row = static_cast<uint32_t>(tb.lo + bi - tb.first) * bs * 128u;
             const uint32_t dst = (is_v ? sV(st) : sK(st)) + dh * kHalf + row;
-            tma_load_3d(dst, map, full0 + 8 * st, dh * 64, w.kh, blk * bs, keep);
+            tma_load_3d(dst, map, full0 + 8 * st, kQuant ? 0 : dh * 64, w.kh, blk * bs, keep);
           }
         }
         ++uq;
@@ -442,7 +518,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
           if (P.idx < P.n && P.base + P.idx < S.base + S.idx) {
             const int t = P.base + P.idx;
             const int st = t % kRing, b = t % 2;
-            if (mbar_test_wait(p_full0 + 8 * b, (t / 2) & 1) && mbar_test_wait(v_full0 + 8 * st, (t / kRing) & 1) &&
+            if (mbar_test_wait(p_full0 + 8 * b, (t / 2) & 1) && mbar_test_wait(v_ready0 + 8 * st, (t / kRing) & 1) &&
                 (P.idx > 0 || P.uq == 0 || mbar_test_wait(o_free, (P.uq - 1) & 1))) {
               tc_fence_after_sync();
   #pragma unroll
@@ -466,7 +542,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
             const int st = t % kRing, b = t % 2;
             if (!q_ready) q_ready = mbar_test_wait(q_full, S.uq & 1);
             // S(t) lands on P(t - 2): the value MMA that reads it must be issued first.
-            if (q_ready && t - 1 <= P.base + P.idx && mbar_test_wait(k_full0 + 8 * st, (t / kRing) & 1)) {
+            if (q_ready && t - 1 <= P.base + P.idx && mbar_test_wait(k_ready0 + 8 * st, (t / kRing) & 1)) {
               tc_fence_after_sync();
   #pragma unroll
               for (int kk = 0; kk < kDim / 16; ++kk) {  // S[b] = Q . K^T, 16 dims per MMA
@@ -496,6 +572,91 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         mbar_wait_bounded(mma_done, 0);
       }
       __syncwarp();
+    } else if (kQuant && warp >= kConvWarp0) {
+      // --------------------------------------------------------------- 8-bit widening --
+      // Thread r owns kv row r of every tile.  It looks up its token's block and scales
+      // while the copies are in flight, then rewrites its row of the slot: dims 64..127
+      // into the hi half first, then dims 0..63 over the codes' own 128 bytes (both in the
+      // 128-byte-swizzled operand layout; chunk c of row r sits at c ^ (r & 7)).  Rows of
+      // tokens outside the loaded blocks or past the context become zeros (their codes may
+      // be anything, NaN included).
+      const int r = 32 * (warp - kConvWarp0) + lane;
+      const uint32_t sw = r & 7;
+      // Code chunk c (codes 16c .. 16c + 15) becomes operand chunks 2c and 2c + 1 of the lo
+      // half (c < 4) or, less 4, of the hi half.  The hi half goes first; the lo chunks are
+      // then made from c = 3 down to 0, so that every chunk written over the row was read
+      // already (chunks 2c and 2c + 1 >= c), and one code chunk is held at a time.
+      auto widen_chunk = [&](uint32_t row, int c, bool live, float sc, bool to_half) {
+        const uint4 raw = ld_shared_v4(row + 16 * (c ^ sw));
+        uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (live) {
+          if (to_half) widen_scaled16<__half, CT>(raw, sc, o);
+          else widen_scaled16<IO, CT>(raw, sc, o);
+        }
+        const uint32_t dst = row + (c >= 4 ? kHalf : 0);
+        const int m = 2 * (c & 3);
+        st_shared_v4(dst + 16 * (m ^ sw), o[0], o[1], o[2], o[3]);
+        st_shared_v4(dst + 16 * ((m + 1) ^ sw), o[4], o[5], o[6], o[7]);
+      };
+      auto widen_row = [&](uint32_t row, bool live, float sc, bool to_half) {
+#pragma unroll
+        for (int c = 4; c < 8; ++c) widen_chunk(row, c, live, sc, to_half);
+#pragma unroll
+        for (int c = 3; c >= 0; --c) widen_chunk(row, c, live, sc, to_half);
+        fence_proxy_async_shared();  // the operand is read by the tensor cores
+      };
+      // The tiles of this CTA in order, with this thread's row of each: whether it is live,
+      // and where its scales are.  The next tile's block-table entry and scales are loaded
+      // while the current one is widened, so the two dependent global loads stay off the
+      // critical path.
+      struct RowRef {
+        bool ok, live;
+        int kv, s, kh;
+        uint16_t ks, vs;  // fp16 bits of the scales (live rows)
+      };
+      UnitCursor cur;
+      cur.start(p);
+      Unit w;
+      int j = 0;
+      bool more = cur.next(p, &w);
+      auto take = [&](RowRef& t) {  // the next tile's row: table entry loaded, scales not yet
+        t.ok = more;
+        if (!more) return;
+        const int kv0 = (w.j_lo + j) * kKv;
+        const TileBlocks tb = tile_blocks(w.j_lo + j, bs, w.kv_lo, w.p_max);
+        t.live = r >= tb.lo * bs - kv0 && r < min(w.ctx, (tb.hi + 1) * bs) - kv0;
+        t.kv = kv0 + r;
+        t.s = w.s;
+        t.kh = w.kh;
+        t.ks = t.vs = 0;
+        if (++j == w.n) {
+          j = 0;
+          more = cur.next(p, &w);
+        }
+      };
+      auto scales = [&](RowRef& t) {
+        if (!t.ok || !t.live) return;
+        int pb = __ldg(p.block_tables + static_cast<size_t>(t.s) * p.MB + t.kv / bs);
+        if (pb < 0 || pb >= p.NB) pb = 0;  // reported by the K copy warp
+        const size_t srow = (static_cast<size_t>(pb) * bs + t.kv % bs) * p.Hkv + t.kh;
+        t.ks = __ldg(p.k_scale + srow);
+        t.vs = __ldg(p.v_scale + srow);
+      };
+      RowRef now, nxt;
+      take(now);
+      scales(now);
+      for (int gt = 0; now.ok; ++gt) {
+        take(nxt);
+        scales(nxt);  // in flight while this tile is widened
+        const int st = gt % kRing;
+        if (!__all_sync(0xffffffffu, wait_or_abort(k_full0 + 8 * st, (gt / kRing) & 1, abort))) break;
+        widen_row(sK(st) + r * 128, now.live, __half2float(__ushort_as_half(now.ks)), false);
+        mbar_arrive(k_conv0 + 8 * st);
+        if (!__all_sync(0xffffffffu, wait_or_abort(v_full0 + 8 * st, (gt / kRing) & 1, abort))) break;
+        widen_row(sV(st) + r * 128, now.live, __half2float(__ushort_as_half(now.vs)), true);
+        mbar_arrive(v_conv0 + 8 * st);
+        now = nxt;
+      }
     }
     end_barrier();
     if (warp == kMmaWarp) {
@@ -653,7 +814,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         // clears its 64-dim lo half, half 1 the hi half).
         const TileBlocks tb = tile_blocks(w.j_lo + j, bs, w.kv_lo, w.p_max);
         const int clean_lo = tb.lo * bs - kv0, clean_hi = min(w.ctx, (tb.hi + 1) * bs) - kv0;
-        if (clean_lo > 0 || clean_hi < kKv) {
+        if (!kQuant && (clean_lo > 0 || clean_hi < kKv)) {  // (8-bit: the widening warps wrote the zeros)
           if (!__all_sync(0xffffffffu, wait_or_abort(v_full0 + 8 * st, (t / kRing) & 1, abort))) {
             ok = false;
             break;
@@ -681,9 +842,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
             float y0, y1;
             f2_unpack(f2_fma(f2_pack(sc[c], sc[c + 1]), q2, nm2), y0, y1);
             const float x0 = ex2_ftz(y0), x1 = ex2_ftz(y1);
-            const Pair<IO> hi(x0, x1);
+            const Pair<PW> hi(x0, x1);
             w_hi[k] = hi.bits;
-            if (kSplit) w_lo[k] = Pair<IO>(x0 - hi.lo_f(), x1 - hi.hi_f()).bits;
+            if (kSplit) w_lo[k] = Pair<PW>(x0 - hi.lo_f(), x1 - hi.hi_f()).bits;
             ls2[k & 3] = f2_add(ls2[k & 3], f2_pack(x0, x1));
           }
           tmem_store16_bits(s_col + 16 * q, w_hi);
@@ -731,12 +892,20 @@ struct RegisterPrefill {
 
 using namespace pa;
 
-extern "C" pa_status paged_attention_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
-                                             const int32_t* block_tables, const int32_t* cu_q_lens,
-                                             const int32_t* context_lens, int num_seqs, int num_q_tokens,
-                                             int max_q_len, int num_q_heads, int num_kv_heads, int head_dim,
-                                             int block_size, int num_blocks, int max_blocks_per_seq, float scale,
-                                             int window, pa_dtype dtype, void* stream) {
+namespace {
+
+template <typename IO>
+const void* prefill_kernel_for(pa_dtype cache) {
+  return cache == PA_I8 ? reinterpret_cast<const void*>(&prefill_tc_kernel<IO, int8_t>)
+         : cache == PA_FP8_E4M3 ? reinterpret_cast<const void*>(&prefill_tc_kernel<IO, __nv_fp8_e4m3>)
+                                : reinterpret_cast<const void*>(&prefill_tc_kernel<IO, IO>);
+}
+
+pa_status prefill_launch(void* out, const void* q, const void* k_cache, const void* v_cache, const void* k_scale,
+                         const void* v_scale, const int32_t* block_tables, const int32_t* cu_q_lens,
+                         const int32_t* context_lens, int num_seqs, int num_q_tokens, int max_q_len, int num_q_heads,
+                         int num_kv_heads, int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                         float scale, int window, pa_dtype dtype, pa_dtype cache_dtype, void* stream) {
   if (num_seqs < 0 || num_q_tokens < 0 || max_q_len < 0)
     return fail(PA_ERR_INVALID_ARG, "paged_attention_prefill: negative size");
   if (num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0)
@@ -745,15 +914,21 @@ extern "C" pa_status paged_attention_prefill(void* out, const void* q, const voi
     return fail(PA_ERR_INVALID_ARG, "paged_attention_prefill: block_size, num_blocks and max_blocks_per_seq must be > 0");
   if (dtype != PA_F16 && dtype != PA_BF16)
     return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: dtype must be PA_F16 or PA_BF16");
+  const bool eight_bit = cache_dtype == PA_I8 || cache_dtype == PA_FP8_E4M3;
+  if (cache_dtype != dtype && !eight_bit)
+    return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: the cache must hold the I/O dtype, PA_I8 or PA_FP8_E4M3");
   if (head_dim != kDim) return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: head_dim must be 128");
   const int GQ = num_q_heads / num_kv_heads;
-  if (GQ > 16 || (GQ & (GQ - 1)) != 0)
-    return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: query heads per cached head must be 1, 2, 4, 8 or 16");
+  if (GQ > kRows || (GQ & (GQ - 1)) != 0)
+    return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: query heads per cached head must be a power of two up to 128");
   if (block_size % 8 != 0 || kKv % block_size != 0)
     return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: block_size must be 8, 16, 32, 64 or 128");
   if (num_seqs == 0 || num_q_tokens == 0 || max_q_len == 0) return PA_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !cu_q_lens || !context_lens)
     return fail(PA_ERR_INVALID_ARG, "paged_attention_prefill: NULL pointer");
+  if (eight_bit && (!k_scale || !v_scale || reinterpret_cast<uintptr_t>(k_scale) % 2 ||
+                    reinterpret_cast<uintptr_t>(v_scale) % 2))
+    return fail(PA_ERR_INVALID_ARG, "paged_attention_prefill: an 8-bit cache needs 2-byte aligned k_scale and v_scale");
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
     return fail(PA_ERR_INVALID_ARG, "paged_attention_prefill: out, q and the caches must be 16-byte aligned");
   if (num_seqs > 65535 || num_kv_heads > 65535)
@@ -770,13 +945,16 @@ extern "C" pa_status paged_attention_prefill(void* out, const void* q, const voi
   const int tq = kRows / GQ;
   CUtensorMap tmK, tmV, tmQ;
   {
-    // [NB*bs rows][Hkv][128]: boxes of one block's rows x one head x 64 dims, 128-byte swizzle
+    // [NB*bs rows][Hkv][128]: boxes of one block's rows x one head x 64 dims (16-bit cache)
+    // or all 128 one-byte codes (8-bit cache), 128-byte swizzle
+    const cuuint64_t e = eight_bit ? 1 : 2;
     const cuuint64_t dims[3] = {kDim, static_cast<cuuint64_t>(num_kv_heads),
                                 static_cast<cuuint64_t>(num_blocks) * block_size};
-    const cuuint64_t strides[2] = {kDim * 2, static_cast<cuuint64_t>(num_kv_heads) * kDim * 2};
-    const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(block_size)};
-    if ((st = encode(enc, &tmK, ttype, 3, k_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != PA_OK) return st;
-    if ((st = encode(enc, &tmV, ttype, 3, v_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != PA_OK) return st;
+    const cuuint64_t strides[2] = {kDim * e, static_cast<cuuint64_t>(num_kv_heads) * kDim * e};
+    const cuuint32_t box[3] = {eight_bit ? 128u : 64u, 1, static_cast<cuuint32_t>(block_size)};
+    const CUtensorMapDataType ctype = eight_bit ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : ttype;
+    if ((st = encode(enc, &tmK, ctype, 3, k_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != PA_OK) return st;
+    if ((st = encode(enc, &tmV, ctype, 3, v_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != PA_OK) return st;
   }
   {
     // q as [T][Hq][128]: tq tokens x the GQ heads of one cached head x 64 dims
@@ -787,6 +965,8 @@ extern "C" pa_status paged_attention_prefill(void* out, const void* q, const voi
   }
   PrefillParams prm = {};
   prm.out = out;
+  prm.k_scale = static_cast<const uint16_t*>(k_scale);
+  prm.v_scale = static_cast<const uint16_t*>(v_scale);
   prm.block_tables = block_tables;
   prm.cu_q = cu_q_lens;
   prm.context_lens = context_lens;
@@ -806,23 +986,30 @@ extern "C" pa_status paged_attention_prefill(void* out, const void* q, const voi
   prm.qscale = scale * 1.4426950408889634f;
 
   const bool bf16 = dtype == PA_BF16;
-  const void* fn = bf16 ? reinterpret_cast<const void*>(&prefill_tc_kernel<__nv_bfloat16>)
-                        : reinterpret_cast<const void*>(&prefill_tc_kernel<__half>);
+  const void* fn = bf16 ? prefill_kernel_for<__nv_bfloat16>(cache_dtype) : prefill_kernel_for<__half>(cache_dtype);
   const size_t smem = kSmemBytes;
-  static std::once_flag once[2];
-  static int launch_regs[2] = {0, 0};
-  cudaError_t attr_err = cudaSuccess;
-  std::call_once(once[bf16 ? 1 : 0], [&] {
-    attr_err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    cudaFuncAttributes fa;
-    if (attr_err == cudaSuccess) attr_err = cudaFuncGetAttributes(&fa, fn);
-    if (attr_err == cudaSuccess) launch_regs[bf16 ? 1 : 0] = fa.numRegs;
-  });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(prefill)");
-  // The warpgroups' register split (setmaxnreg) adds up to exactly what a 128-register
-  // launch provides; with any other allocation the kernel is not launched.
-  if (launch_regs[bf16 ? 1 : 0] != kRegsLaunch)
-    return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: kernel built with an unexpected register count");
+  // Once per kernel: the dynamic shared-memory limit, and the kernel's register count.  The
+  // warpgroups' register split (setmaxnreg) adds up to exactly what a 128-register launch
+  // provides; with any other allocation the kernel is not launched.
+  {
+    struct Entry { const void* fn; int regs; };
+    static std::mutex m;
+    static std::vector<Entry> seen;
+    std::lock_guard<std::mutex> lock(m);
+    int regs = -1;
+    for (const Entry& en : seen)
+      if (en.fn == fn) regs = en.regs;
+    if (regs < 0) {
+      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      cudaFuncAttributes fa;
+      if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, fn);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill)");
+      regs = fa.numRegs;
+      seen.push_back(Entry{fn, regs});
+    }
+    if (regs != kRegsLaunch)
+      return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: kernel built with an unexpected register count");
+  }
   const long long units = static_cast<long long>(num_seqs) * num_kv_heads * prm.qtiles;
   if (units > (1LL << 30)) return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: too many query tiles");
   prm.units = static_cast<int>(units);
@@ -834,4 +1021,32 @@ extern "C" pa_status paged_attention_prefill(void* out, const void* q, const voi
   cudaError_t err = launch_dependent(fn, grid, dim3(kThreads), smem, static_cast<cudaStream_t>(stream), args);
   if (err != cudaSuccess) return cuda_fail(err, "launching the prefill kernel");
   return PA_OK;
+}
+
+}  // namespace
+
+extern "C" pa_status paged_attention_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                             const int32_t* block_tables, const int32_t* cu_q_lens,
+                                             const int32_t* context_lens, int num_seqs, int num_q_tokens,
+                                             int max_q_len, int num_q_heads, int num_kv_heads, int head_dim,
+                                             int block_size, int num_blocks, int max_blocks_per_seq, float scale,
+                                             int window, pa_dtype dtype, void* stream) {
+  return prefill_launch(out, q, k_cache, v_cache, nullptr, nullptr, block_tables, cu_q_lens, context_lens, num_seqs,
+                        num_q_tokens, max_q_len, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                        max_blocks_per_seq, scale, window, dtype, dtype, stream);
+}
+
+extern "C" pa_status paged_attention_prefill_quant(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                                   const void* k_scale, const void* v_scale,
+                                                   const int32_t* block_tables, const int32_t* cu_q_lens,
+                                                   const int32_t* context_lens, int num_seqs, int num_q_tokens,
+                                                   int max_q_len, int num_q_heads, int num_kv_heads, int head_dim,
+                                                   int block_size, int num_blocks, int max_blocks_per_seq,
+                                                   float scale, int window, pa_dtype io_dtype, pa_dtype cache_dtype,
+                                                   void* stream) {
+  if (cache_dtype != PA_I8 && cache_dtype != PA_FP8_E4M3)
+    return fail(PA_ERR_INVALID_ARG, "paged_attention_prefill_quant: cache_dtype must be PA_I8 or PA_FP8_E4M3");
+  return prefill_launch(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, cu_q_lens, context_lens, num_seqs,
+                        num_q_tokens, max_q_len, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                        max_blocks_per_seq, scale, window, io_dtype, cache_dtype, stream);
 }

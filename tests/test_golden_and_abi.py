@@ -152,7 +152,8 @@ def test_prefill_host_validation(L):
         return L.paged_attention_prefill(p, p, p, p, p, p, p, 1, T, mq, hq, hkv, D, bs, 64, 8, 0.1, 0, dt, None)
     assert call(hq=6, hkv=4) == 1       # query heads not a multiple of cached heads
     assert call(hq=12, hkv=4) == 2      # 3 query heads per cached head: unsupported
-    assert call(hq=64, hkv=2) == 2      # 32 per cached head: unsupported
+    assert call(hq=48, hkv=2) == 2      # 24 per cached head: not a power of two
+    assert call(hq=512, hkv=2) == 2     # 256 per cached head: more than a unit's 128 rows
     assert call(D=64) == 2              # head_dim 128 only
     assert call(bs=12) == 2             # block size must divide 128 in steps of 8
     assert call(dt=0) == 2              # fp32 I/O is not a tensor-core type here
@@ -162,6 +163,21 @@ def test_prefill_host_validation(L):
     assert call(T=0) == 0               # nothing to do
     assert call(mq=0) == 0
     assert call(T=1 << 28) == 2         # T * Hq = 2^31: output row indices would overflow
+    assert L.pa_last_error().decode()
+
+
+def test_prefill_quant_host_validation(L):
+    P = ctypes.c_void_p
+    def call(cache=3, ks=16, vs=16, io=1):
+        p = P(16)
+        k = P(ks) if ks else None
+        v = P(vs) if vs else None
+        return L.paged_attention_prefill_quant(p, p, p, p, k, v, p, p, p, 1, 40, 40, 8, 2, 128, 16, 64, 8, 0.1, 0,
+                                               io, cache, None)
+    assert call(cache=1) == 1           # a 16-bit cache belongs to paged_attention_prefill
+    assert call(ks=0) == 1              # an 8-bit cache needs both scale pools
+    assert call(vs=17) == 1             # fp16 scales must be 2-byte aligned
+    assert call(io=0) == 2              # fp32 I/O is not a tensor-core type here
     assert L.pa_last_error().decode()
 
 

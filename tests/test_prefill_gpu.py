@@ -1,8 +1,8 @@
 """GPU paged prefill / chunked-prefill attention (tcgen05) through the C ABI against the
 fp64 oracle: whole prompts, chunks behind cached context and single tokens in one batch,
 fp16 and bf16, 1 to 16 query heads per cached head, every block size, sliding windows,
-several query and KV tiles with ragged tails, chunked = one-shot, empty sequences, and
-out-of-range inputs reported (not faulted).  Pool rows no sequence owns hold NaN, so a
+several query and KV tiles with ragged tails, chunked = one-shot, empty sequences,
+out-of-range inputs reported (not faulted), and INT8 / FP8 caches (tolerance 1e-2).  Pool rows no sequence owns hold NaN, so a
 read outside the attended tokens shows up as a non-finite output."""
 import math
 
@@ -12,7 +12,7 @@ import torch
 
 import oracle
 import paged_kv_cache_384_b200 as pa
-from parity import TOL, assert_no_device_error, compare
+from parity import TOL, assert_no_device_error, compare, quantize_cache, quantize_cache_fp8
 
 pytestmark = pytest.mark.gpu
 
@@ -203,3 +203,84 @@ def test_prefill_many_short_units_per_cta(cuda_device, window):
     ql = g.integers(1, 4, size=S).tolist()
     ctx = [q + int(g.integers(0, 300)) for q in ql]
     check(20 + window, ctx, ql, 4, 2, 16, "fp16", window)
+
+
+# ---------------------------------------------------------------------------------------
+# 8-bit caches: the fp16 pool of paged_case quantised by the oracle quantiser; rows no
+# sequence owns keep NaN scales (and FP8 NaN codes), so reading one shows up.
+# ---------------------------------------------------------------------------------------
+def quantised(kc, vc, dtype):
+    owned = ~torch.isnan(kc[..., 0].float())             # [NB, bs, Hkv]
+    quant = quantize_cache if dtype == "int8" else quantize_cache_fp8
+    k, ks = quant(torch.nan_to_num(kc.half()))
+    v, vs = quant(torch.nan_to_num(vc.half()))
+    ks[~owned] = float("nan")
+    vs[~owned] = float("nan")
+    if dtype == "fp8":
+        k.view(torch.uint8)[~owned] = 0x7F                # the E4M3 NaN code
+        v.view(torch.uint8)[~owned] = 0x7F
+    return k, v, ks, vs
+
+
+def check_8bit(seed, ctx, qlen, Hq, Hkv, bs, io, dtype, window=0):
+    q, kc, vc, bt, cu, cl = paged_case(seed, ctx, qlen, Hq, Hkv, bs, "fp16")
+    q = q.to(DT[io])
+    k, v, ks, vs = quantised(kc, vc, dtype)
+    scale = 1 / math.sqrt(128)
+    out = torch.empty_like(q, device="cuda")
+    pa.paged_attention_prefill(out, q.cuda(), k.cuda(), v.cuda(), bt.cuda(), cu.cuda(), cl.cuda(),
+                               int((cu[1:] - cu[:-1]).max()), scale, window, k_scale=ks.cuda(), v_scale=vs.cuda())
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    ref = oracle.paged_prefill(q, k, v, bt, cu, cl, scale, window, k_scale=ks, v_scale=vs)
+    return compare(out, ref, io, TOL["int8"])
+
+
+@pytest.mark.parametrize("io", ["fp16", "bf16"])
+@pytest.mark.parametrize("dtype", ["int8", "fp8"])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 2), (16, 2), (16, 1)])
+def test_prefill_eight_bit_caches_mixed_batch(cuda_device, io, dtype, Hq, Hkv):
+    check_8bit(31, [37, 300, 129, 16], [37, 90, 1, 16], Hq, Hkv, 16, io, dtype)
+
+
+@pytest.mark.parametrize("bs", [8, 32, 64, 128])
+@pytest.mark.parametrize("dtype", ["int8", "fp8"])
+def test_prefill_eight_bit_block_sizes(cuda_device, bs, dtype):
+    check_8bit(32, [130, 77, 256], [130, 40, 129], 4, 2, bs, "fp16", dtype)
+
+
+@pytest.mark.parametrize("window", [1, 100, 5000])
+def test_prefill_eight_bit_windows_and_many_tiles(cuda_device, window):
+    check_8bit(33, [1000, 260], [1000, 70], 8, 2, 16, "bf16", "int8", window)
+    check_8bit(34, [700], [500], 2, 2, 32, "fp16", "fp8", window)
+
+
+def test_prefill_llama70b_prompt_batch_int8_full(cuda_device):
+    """The prompt batch (4 x 2048 tokens, 64 heads, bs 16) over an INT8 cache: every output."""
+    S, n, H, bs = 4, 2048, 64, 16
+    g = torch.Generator().manual_seed(35)
+    NB = S * n // bs + 16
+    perm = torch.randperm(NB, generator=g)
+    bt = perm[: S * n // bs].view(S, n // bs).to(torch.int32).contiguous()
+    k, ks = quantize_cache(torch.randn(NB, bs, H, 128, generator=g, dtype=torch.float16))
+    v, vs = quantize_cache(torch.randn(NB, bs, H, 128, generator=g, dtype=torch.float16))
+    q = torch.randn(S * n, H, 128, generator=g, dtype=torch.float16)
+    cu = torch.arange(0, S * n + 1, n, dtype=torch.int32)
+    cl = torch.full((S,), n, dtype=torch.int32)
+    scale = 1 / math.sqrt(128)
+    out = torch.empty_like(q, device="cuda")
+    pa.paged_attention_prefill(out, q.cuda(), k.cuda(), v.cuda(), bt.cuda(), cu.cuda(), cl.cuda(), n, scale,
+                               k_scale=ks.cuda(), v_scale=vs.cuda())
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    ref = oracle.paged_prefill(q, k, v, bt, cu, cl, scale, k_scale=ks, v_scale=vs)
+    compare(out, ref, "fp16", TOL["int8"])
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(32, 1), (64, 2), (128, 1)])
+@pytest.mark.parametrize("io", ["fp16", "bf16"])
+def test_prefill_multi_query(cuda_device, Hq, Hkv, io):
+    """32 to 128 query heads per cached head: a unit's 128 rows are 4, 2 or 1 query tokens
+    times all the query heads of one cached head."""
+    check(41, [37, 300, 129, 16], [37, 90, 1, 16], Hq, Hkv, 16, io)
+    check(42, [400, 45], [400, 45], Hq, Hkv, 32, io, window=100)
