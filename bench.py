@@ -52,7 +52,11 @@ CONTEXT_DESC = {"llama70b_fp16": "uniform [1, 2048]",
                 "sliding_window_fp16": "32768 each, window 4096",
                 "llama70b_gqa_fp16": "uniform [1, 2048], 64 query heads over 8 cached heads",
                 "llama70b_int8": "uniform [1, 2048], INT8 cache written by quantise-on-write",
-                "llama70b_fp8": "uniform [1, 2048], FP8 E4M3 cache written by quantise-on-write"}
+                "llama70b_fp8": "uniform [1, 2048], FP8 E4M3 cache written by quantise-on-write",
+                "llama70b_gqa_int8": "uniform [1, 2048], 64 query heads over 8 cached heads, INT8 cache written by "
+                                     "quantise-on-write",
+                "llama70b_gqa_fp8": "uniform [1, 2048], 64 query heads over 8 cached heads, FP8 E4M3 cache written by "
+                                    "quantise-on-write"}
 METRIC = "paged decode attention KV GB/s (% of B200 HBM peak) and tokens/s per layer"
 FALLBACK_HBM_GBS = 6650.0      # copy bandwidth measured earlier on this GPU type
 FALLBACK_BF16_TFLOPS = 1590.0  # cuBLAS bf16 burst measured earlier on this GPU type
@@ -202,14 +206,17 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------------
 # workload
 # ---------------------------------------------------------------------------------------
-EIGHT_BIT = {"llama70b_int8": torch.int8, "llama70b_fp8": torch.float8_e4m3fn}
+# 8-bit workloads: (the fp16 batch their cache is quantised from, code dtype)
+EIGHT_BIT = {"llama70b_int8": ("llama70b_int8", torch.int8), "llama70b_fp8": ("llama70b_int8", torch.float8_e4m3fn),
+             "llama70b_gqa_int8": ("llama70b_gqa_fp16", torch.int8),
+             "llama70b_gqa_fp8": ("llama70b_gqa_fp16", torch.float8_e4m3fn)}
 
 
 def build(seed: int, device, workload: str = PRESET, block_size=None):
     import paged_kv_cache_384_b200 as pa
     over = {} if block_size is None else {"block_size": block_size}
     big = workload == "sliding_window_fp16"          # 8.6 GB of cache: draw values on the GPU
-    preset = "llama70b_int8" if workload in EIGHT_BIT else workload
+    preset = EIGHT_BIT[workload][0] if workload in EIGHT_BIT else workload
     w = synth.build_workload(preset, seed, pa.BlockManager, device=device if big else "cpu", **over)
     ctx = w.context_lens.tolist()
     slots = pa.slot_mapping(w.block_tables, range(w.num_seqs), [c - 1 for c in ctx], w.block_size)
@@ -225,7 +232,7 @@ def build(seed: int, device, workload: str = PRESET, block_size=None):
         # through the same kernel.
         src_k, src_v = dev["k_cache"], dev["v_cache"]
         NB, bs, H, D = src_k.shape
-        code = EIGHT_BIT[workload]
+        code = EIGHT_BIT[workload][1]
         dev["k_cache"] = torch.empty(NB, bs, H, D, dtype=code, device=device)
         dev["v_cache"] = torch.empty_like(dev["k_cache"])
         dev["k_scale"] = torch.empty(NB, bs, H, dtype=torch.float16, device=device)
@@ -435,10 +442,11 @@ def decode_kernel_name(w) -> str:
 # The other decode workloads of the method, measured after the metric's own workload in a
 # default run so that their numbers sit in the same record: the prefix-sharing chat batch,
 # the INT8 and FP8 caches, the 32k-token sliding window at block sizes 8 / 16 / 32, and the
-# grouped-query Llama-2-70B layer (64 query heads over 8 cached heads).
+# grouped-query Llama-2-70B layer (64 query heads over 8 cached heads) with fp16, INT8 and FP8
+# caches.
 SECONDARY = (("chat_prefix_bf16", None), ("llama70b_int8", None), ("llama70b_fp8", None),
              ("sliding_window_fp16", 8), ("sliding_window_fp16", 16), ("sliding_window_fp16", 32),
-             ("llama70b_gqa_fp16", None))
+             ("llama70b_gqa_fp16", None), ("llama70b_gqa_int8", None), ("llama70b_gqa_fp8", None))
 SECONDARY_STEPS = 100
 
 
@@ -713,7 +721,10 @@ PREFILL = {  # name: (prompts, prompt/chunk tokens, cached tokens before the chu
     "prefill_llama70b_fp16": (4, 2048, 0, 64, 64),
     "prefill_llama70b_gqa_fp16": (4, 2048, 0, 64, 8),
     "chunked_prefill_llama70b_fp16": (8, 512, 1536, 64, 64),
+    "prefill_llama70b_int8": (4, 2048, 0, 64, 64),
+    "prefill_llama70b_fp8": (4, 2048, 0, 64, 64),
 }
+PREFILL_CODES = {"prefill_llama70b_int8": torch.int8, "prefill_llama70b_fp8": torch.float8_e4m3fn}
 
 
 def run_prefill(args):
@@ -748,12 +759,27 @@ def run_prefill(args):
     scale = 1 / math.sqrt(D)
     stream = torch.cuda.current_stream(device)
     flops = accounting.prefill_flops([ctx] * S, [qn] * S, Hq, D)  # causal: position p sees p + 1 tokens
+    code = PREFILL_CODES.get(args.workload)
+    ks = vs = None
+    if code is not None:
+        # 8-bit cache: the fp16 pool quantised by the library's quantise-on-write (untimed
+        # setup); each step then quantises the new rows into it
+        ks = torch.empty(NB, bs, Hkv, dtype=torch.float16, device=device)
+        vs = torch.empty_like(ks)
+        kq, vq = torch.empty(kc.shape, dtype=code, device=device), torch.empty(vc.shape, dtype=code, device=device)
+        all_slots = torch.arange(NB * bs, dtype=torch.int64, device=device)
+        pa.reshape_and_cache_quant(kc.view(NB * bs, Hkv, D), vc.view(NB * bs, Hkv, D), kq, vq, ks, vs, all_slots)
+        torch.cuda.synchronize(device)
+        kc, vc = kq, vq
 
     def attn():
-        pa.paged_attention_prefill(out, q, kc, vc, bt, cu, cl, qn, scale, stream=stream)
+        pa.paged_attention_prefill(out, q, kc, vc, bt, cu, cl, qn, scale, stream=stream, k_scale=ks, v_scale=vs)
 
     def step():
-        pa.reshape_and_cache(k_new, v_new, kc, vc, slots, stream=stream)
+        if code is not None:
+            pa.reshape_and_cache_quant(k_new, v_new, kc, vc, ks, vs, slots, stream=stream)
+        else:
+            pa.reshape_and_cache(k_new, v_new, kc, vc, slots, stream=stream)
         attn()
 
     def timed(fn, reps):
@@ -796,6 +822,8 @@ def run_prefill(args):
         "warmup": args.warmup, "ms_per_step": round(1e3 * sec, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
         "config": {"workload": args.workload, "prompts": S, "new_tokens_per_seq": qn, "cached_before": cached,
+                   "cache": {None: "fp16", torch.int8: "int8 + fp16 scales",
+                             torch.float8_e4m3fn: "fp8 e4m3 + fp16 scales"}[code],
                    "num_q_heads": Hq, "num_kv_heads": Hkv, "head_dim": D, "block_size": bs, "seed": args.seed,
                    "step": "reshape_and_cache of the new K/V rows + paged_attention_prefill",
                    "l2": "K/V and q per step larger than L2, no flush"},
@@ -826,7 +854,8 @@ def main(argv=None):
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the other decode workloads that a default run measures after the metric's own")
     ap.add_argument("--workload", default=PRESET, choices=["llama70b_fp16", "chat_prefix_bf16", "sliding_window_fp16",
-                                                           "llama70b_gqa_fp16", "llama70b_int8", "llama70b_fp8", "swap_llama70b_fp16",
+                                                           "llama70b_gqa_fp16", "llama70b_int8", "llama70b_fp8",
+                                                           "llama70b_gqa_int8", "llama70b_gqa_fp8", "swap_llama70b_fp16",
                                                            *PREFILL],
                     help="secondary workloads are for study; the metric is quoted on the default")
     ap.add_argument("--block-size", type=int, default=None)
