@@ -39,11 +39,16 @@ namespace pa {
 // Partition kernel.
 //   IO: q/out type; CT: cache element type; D: head_dim; TT: rows per tile if fixed, 0 = runtime.
 // ---------------------------------------------------------------------------------------
+// CTAs per SM the register allocation is sized for: 8-bit caches (2 CTAs per SM by shared
+// memory) get the registers their widening needs without spilling; for 16-bit caches 3 keeps
+// the 72-register allocation that measured fastest (92 registers with 1 ran ~4 % slower).
+template <typename CT>
+constexpr int partition_min_blocks() {
+  return (std::is_same<CT, int8_t>::value || std::is_same<CT, __nv_fp8_e4m3>::value) ? 1 : 3;
+}
+
 template <typename IO, typename CT, int D, int TT>
-// minBlocks = 1 states what the launch uses (shared memory allows 2 or 3 CTAs per SM); with
-// the bound left at its default ptxas capped several instantiations at 56 or 72 registers and
-// spilled.
-__global__ void __launch_bounds__(kMaxThreads, 1)
+__global__ void __launch_bounds__(kMaxThreads, partition_min_blocks<CT>())
 decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ CUtensorMap tmKs, const __grid_constant__ CUtensorMap tmVs,
                         const DecodeParams p) {
@@ -404,9 +409,8 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
 }
 
 // ---------------------------------------------------------------------------------------
-// Merge kernel: one warp per (sequence, head group) segment combines, head by head, the
-// partial states of a segment that was split across CTAs:
-//   M = max_k m_k,  out = sum_k 2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k.
+// Merge kernel: one warp per (sequence, head) combines the partial states of a segment that
+// was split across CTAs:  M = max_k m_k,  out = sum_k 2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k.
 // Sequences with nothing to attend get zeros; segments held by one CTA were written by it.
 // Launched as a programmatic dependent of the partition kernel: the grid is resident while
 // the partition kernel runs and proceeds the moment its results are visible.
@@ -418,53 +422,47 @@ __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const De
   constexpr int DL = D / 32;  // dims per lane
   grid_dependency_wait();
   const int lane = threadIdx.x & 31;
-  // One warp per (sequence, head group) segment: a segment held by one CTA needs nothing, so
-  // most warps read the tile prefix once and leave; the heads of a split one are merged in turn.
   const long long item = static_cast<long long>(blockIdx.x) * kMergeWarps + (threadIdx.x >> 5);
-  if (item >= static_cast<long long>(p.S) * p.G) return;
-  const int s = static_cast<int>(item / p.G), g = static_cast<int>(item % p.G);
+  if (item >= static_cast<long long>(p.S) * p.Hq) return;
+  const int s = static_cast<int>(item / p.Hq), h = static_cast<int>(item % p.Hq);
   const long long per_group = p.ws_prefix[p.S];
   const long long pre = p.ws_prefix[s];
   const long long nb = p.ws_prefix[s + 1] - pre;
-  if (nb == 0) {  // nothing to attend: zeros
-    for (int w = 0; w < p.QW; ++w) {
-      IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(s) * p.Hq + g * p.QW + w) * D + lane * DL;
+  IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(s) * p.Hq + h) * D + lane * DL;
+  float o[DL];
 #pragma unroll
-      for (int e = 0; e < DL; ++e) orow[e] = float_to<IO>(0.f);
-    }
+  for (int e = 0; e < DL; ++e) o[e] = 0.f;
+  if (nb == 0) {
+#pragma unroll
+    for (int e = 0; e < DL; ++e) orow[e] = float_to<IO>(0.f);
     return;
   }
   const long long T = per_group * p.G;
+  const int g = h / p.QW, w = h % p.QW;
   const long long a = p.G * pre + g * nb;
   const int c0 = cta_of(a, T, p.num_ctas), c1 = cta_of(a + nb - 1, T, p.num_ctas);
   if (c0 == c1) return;
   const long long seg = static_cast<long long>(s) * p.G + g;
   const float2* ml = reinterpret_cast<const float2*>(p.ws_ml);
-  for (int w = 0; w < p.QW; ++w) {
-    // Global max over the partials, 32 partials per round (one per lane).
-    float M = -FLT_MAX;
-    for (int k = c0 + lane; k <= c1; k += 32) M = fmaxf(M, ml[(k + seg) * p.QW + w].x);
+  // Global max over the partials, 32 partials per round (one per lane).
+  float M = -FLT_MAX;
+  for (int k = c0 + lane; k <= c1; k += 32) M = fmaxf(M, ml[(k + seg) * p.QW + w].x);
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float o[DL];
-#pragma unroll
-    for (int e = 0; e < DL; ++e) o[e] = 0.f;
-    float L = 0.f;
+  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  float L = 0.f;
 #pragma unroll 4
-    for (int k = c0; k <= c1; ++k) {
-      const long long row = (k + seg) * p.QW + w;
-      const float2 st = ml[row];
-      const float f = exp2f(st.x - M);
-      L = fmaf(f, st.y, L);
-      const float* src = p.ws_acc + row * D + lane * DL;
+  for (int k = c0; k <= c1; ++k) {
+    const long long row = (k + seg) * p.QW + w;
+    const float2 st = ml[row];
+    const float f = exp2f(st.x - M);
+    L = fmaf(f, st.y, L);
+    const float* src = p.ws_acc + row * D + lane * DL;
 #pragma unroll
-      for (int e = 0; e < DL; ++e) o[e] = fmaf(f, src[e], o[e]);
-    }
-    const float inv = 1.f / L;
-    IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(s) * p.Hq + g * p.QW + w) * D + lane * DL;
-#pragma unroll
-    for (int e = 0; e < DL; ++e) orow[e] = float_to<IO>(o[e] * inv);
+    for (int e = 0; e < DL; ++e) o[e] = fmaf(f, src[e], o[e]);
   }
+  const float inv = 1.f / L;
+#pragma unroll
+  for (int e = 0; e < DL; ++e) orow[e] = float_to<IO>(o[e] * inv);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -706,7 +704,7 @@ pa_status decode_launch_tc(void* out, const void* q, const void* k_cache, const 
   if (ev[1]) cudaEventRecord(ev[1], s);
   {
     void* args[] = {&prm};
-    const long long items = static_cast<long long>(num_seqs) * prm.G;  // one warp per segment
+    const long long items = static_cast<long long>(num_seqs) * num_q_heads;
     const unsigned grid = static_cast<unsigned>((items + kMergeWarps - 1) / kMergeWarps);
     cudaError_t err = launch_dependent(select_merge(io_dtype, head_dim), dim3(grid), dim3(32 * kMergeWarps), 0, s, args);
     if (err != cudaSuccess) return cuda_fail(err, "launching the decode merge kernel");
@@ -878,7 +876,7 @@ pa_status decode_launch(void* out, const void* q, const void* k_cache, const voi
   if (ev[1]) cudaEventRecord(ev[1], s);
   {
     void* args[] = {&prm};
-    const long long items = static_cast<long long>(num_seqs) * G;  // one warp per segment
+    const long long items = static_cast<long long>(num_seqs) * num_q_heads;
     const unsigned grid = static_cast<unsigned>((items + kMergeWarps - 1) / kMergeWarps);
     cudaError_t err = launch_dependent(merge_fn, dim3(grid), dim3(32 * kMergeWarps), 0, s, args);
     if (err != cudaSuccess) return cuda_fail(err, "launching the decode merge kernel");

@@ -241,7 +241,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     // one after another, so four warps issue a tile four times as fast as one.  Warp 0
     // also loads the q rows.  Every warp walks the same tile stream and block table.
     // 8-bit cache: the parts are K codes (+ q rows), V codes, K scales and V scales, and the
-    // four warps then widen the codes of the tile issued kLag tiles earlier, thread = row.
+    // four warps also widen each landed tile's codes, thread = row.
     const int part = warp == 0 ? 0 : warp - 5;  // 0: K lo, 1: K hi, 2: V lo, 3: V hi
     const CUtensorMap* map = kQuant ? (part == 0 ? &tmK : part == 1 ? &tmV : part == 2 ? &tmKs : &tmVs)
                                     : (part < 2 ? &tmK : &tmV);
@@ -270,10 +270,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     // same 128 bytes and dims 64..127 into the hi half, both in the 128-byte-swizzled
     // layout the MMAs read.  V rows of unattended tokens become zeros (they may hold
     // anything, and 0 * NaN would poison the weighted sum).  A stage is handed to the MMA
-    // issuer once all 128 rows are done.  kLag = 2 keeps a tile of copies in flight while one
-    // is widened; a stage's reuse waits for the value MMA of the tile three back, whose codes
-    // were widened in an earlier iteration, so the ring cannot stall on itself.
-    constexpr int kLag = 2;
+    // issuer once all 128 rows are done.
     Cursor cc = start;
     int widened = 0;
     const int wr = 32 * part + lane;  // row this thread widens
@@ -310,11 +307,8 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       if (widened < n) advance(cc, p);
       return true;
     };
-    for (; issued < n; ++issued) {
-      // Widen the tile issued kLag tiles ago first: its copies need no more than time, while
-      // the stage this tile needs may wait for the value MMA of the tile three back, which in
-      // turn waits for widened operands.
-      if (kQuant && issued - widened >= kLag && !widen_tile()) break;
+    // Issue the copies of tile `issued` (waiting, bounded, for its stage to be free).
+    auto issue_next = [&]() -> bool {
       const int st = issued % kStages;
       const int kh = c.g / p.sub;  // cached head of this head group
       const int tok0 = (c.sp.first_t + c.j) * kTokens;
@@ -357,7 +351,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);  // also orders lane 0's expect_tx before any copy
-      if (!ok) break;
+      if (!ok) return false;
       const bool copies = kQuant || !(part & 1) || p.dim == 128;  // head_dim 64: the hi-half warps only arrive
       if (copies && lane < nload) {  // this warp's part of each attended block, one copy per lane
         const uint32_t row0 = static_cast<uint32_t>(lb_lo + lane - lb_first) * bs;  // first row in the tile
@@ -373,10 +367,50 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         }
       }
       advance(c, p);
+      ++issued;
+      return true;
+    };
+    if constexpr (!kQuant) {
+      while (issued < n)
+        if (!issue_next()) break;
+    } else {
+      // 8-bit cache: copies and widening interleave as each becomes possible -- the next
+      // tile's copies as soon as its stage is free, the widening of the oldest landed tile as
+      // soon as its codes have arrived -- so neither waits behind the other.  (Alternating
+      // them in a fixed order made every widening wait for the value MMA of an earlier tile.)
+      uint32_t idle = 0;
+      while (widened < n) {
+        bool progressed = false;
+        if (issued < n) {
+          int free_st = 1;
+          if (lane == 0 && issued >= kStages)
+            free_st = mbar_test_wait(empty0 + 8 * (issued % kStages), ((issued / kStages) - 1) & 1) ? 1 : 0;
+          if (__shfl_sync(0xffffffffu, free_st, 0)) {
+            if (!issue_next()) break;
+            progressed = true;
+          }
+        }
+        if (widened < issued) {
+          int landed = 0;
+          if (lane == 0) landed = mbar_test_wait(full0 + 8 * (widened % kStages), (widened / kStages) & 1) ? 1 : 0;
+          if (__shfl_sync(0xffffffffu, landed, 0)) {
+            if (!widen_tile()) break;
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          idle = 0;
+        } else {
+          if (*abort) break;
+          if (++idle > 16 * kWaitLimit) {
+            if (lane == 0) decode_error(PA_DEVERR_TIMEOUT);
+            *abort = 1;
+            break;
+          }
+          __nanosleep(32);
+        }
+      }
     }
-    if (kQuant && !*abort)
-      while (widened < issued)
-        if (!widen_tile()) break;
     if (lane == 0)  // never leave with copies in flight
       for (int k = issued - kStages < 0 ? 0 : issued - kStages; k < issued; ++k)
         wait_or_abort(full0 + 8 * (k % kStages), (k / kStages) & 1, abort);

@@ -3,11 +3,14 @@ seeded inputs and compare.
 
 Tolerances (fp32 accumulation on the GPU, fp64 in the oracle):
   * fp32 / fp16 / bf16 I/O: max |gpu - oracle| <= 2e-3, where the oracle is first rounded
-    to the I/O dtype (round to nearest even), because the GPU result is rounded too.  The
-    one exception allowed is a rounding-boundary case: the exact value lies so close to
-    the midpoint of two adjacent I/O values that the fp32 result rounded to the other one
-    (|gpu - oracle_fp64| <= half an I/O ulp + 1e-5 relative).  Such cases are counted and
-    must stay rare.  For bf16 one ulp at |o| >= 0.5 already exceeds 2e-3, hence the rule.
+    to the I/O dtype (round to nearest even), because the GPU result is rounded too.  An
+    output also passes when it lies within the tolerance of the exact fp64 value (the bar as
+    stated: max abs error against the oracle); with bf16 output and an 8-bit cache's 1e-2 a
+    result at |o| >= 2, where one bf16 ulp is 0.0156, can differ from the rounded oracle by
+    a whole ulp while within 1e-2 of the exact value.  The one other exception allowed is a
+    rounding-boundary case: the exact value lies so close to the midpoint of two adjacent
+    I/O values that the fp32 result rounded to the other one (|gpu - oracle_fp64| <= half an
+    I/O ulp + 1e-5 relative).  Both kinds are counted, and boundary cases must stay rare.
   * INT8 and FP8 caches: the same against the oracle on the dequantised values, with 1e-2.
 """
 import numpy as np
@@ -18,8 +21,9 @@ import paged_kv_cache_384_b200 as pa
 
 TOL = {"fp32": 2e-3, "fp16": 2e-3, "bf16": 2e-3, "int8": 1e-2}
 
-# (I/O dtype, rounding-boundary cases accepted, outputs compared) of every compare() call
-# in this process; the session summary (conftest.py) prints the totals.
+# (I/O dtype, rounding-boundary cases accepted, outputs compared, outputs accepted on their
+# distance to the exact value) of every compare() call in this process; the session summary
+# (conftest.py) prints the totals.
 BOUNDARY_TALLY = []
 TORCH_DT = {"fp32": torch.float32, "fp16": torch.float16, "bf16": torch.bfloat16}
 
@@ -46,7 +50,8 @@ def compare(gpu: torch.Tensor, ref64: np.ndarray, io: str, tol: float, max_bound
     r = round_io(ref64, io)
     err = np.abs(g - r)
     raw = np.abs(g - ref64)
-    over = err > tol
+    exact_ok = (err > tol) & (raw <= tol)   # within the tolerance of the exact value
+    over = (err > tol) & ~exact_ok
     boundary = over & (raw <= half_ulp(ref64, io) * (1 + 1e-6) + 1e-5 * np.abs(ref64))
     hard = over & ~boundary
     if hard.any():
@@ -54,7 +59,7 @@ def compare(gpu: torch.Tensor, ref64: np.ndarray, io: str, tol: float, max_bound
         raise AssertionError(f"{int(hard.sum())} outputs off by > {tol}: max {err.max():.3e} at {idx.tolist()}; "
                              f"gpu {g[tuple(idx[0])]} oracle {ref64[tuple(idx[0])]}")
     assert boundary.sum() <= max(1, max_boundary_frac * g.size), f"{int(boundary.sum())} rounding-boundary cases"
-    BOUNDARY_TALLY.append((io, int(boundary.sum()), int(g.size)))
+    BOUNDARY_TALLY.append((io, int(boundary.sum()), int(g.size), int(exact_ok.sum())))
     return float(err.max(initial=0.0)), float(raw.max(initial=0.0)), int(boundary.sum())
 
 
