@@ -170,11 +170,12 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   // is removed once when the segment ends (the cancellation costs ~7 of fp32's 24 bits of the
   // biased sum; typical error ~1e-5 of the output scale against the 1e-2 tolerance).
   constexpr bool kBiasV = std::is_same<CT, int8_t>::value;
-  // INT8 scores are integer dot products: q is held as 24-bit fixed point per row (row
-  // maximum below 2^22 steps), split into a signed top byte and two unsigned bytes, and
-  // each byte plane is dotted with four codes per dp4a instruction into an exact int32 sum
-  // (16 dims per lane: |sum| < 2^19 per plane).  The only rounding is that of q to 2^-22 of
-  // its row maximum, finer than fp32's own rounding of most elements of the row.
+  // INT8 scores are integer dot products: q is held as 16-bit fixed point per row (row
+  // maximum in [2^14, 2^15) steps), split into a signed high byte and an unsigned low byte;
+  // each byte plane is dotted with four codes per dp4a instruction and the two sums are
+  // combined as hi * 256 + lo, exactly, in int32 (|sum| < 2^27 for a lane's 16 dims, < 2^30
+  // after the reduction over the row's 8 lanes).  The one rounding is that of q, to 2^-15
+  // of its row maximum (finer than the f16 q of the FP8 path).
   constexpr bool kDp4a = std::is_same<CT, int8_t>::value;
   // FP8 scores and weighted sums run on f16 x f16 -> f32 fused multiply-adds: pairs of E4M3
   // codes convert exactly to f16 pairs, q is held in f16 after an exact power-of-two
@@ -183,7 +184,7 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   constexpr bool kMixed = std::is_same<CT, __nv_fp8_e4m3>::value;
   float qf[EV], acc[EV];
   float wsum = 0.f;        // INT8: sum of the f16 weights, for the bias of the V sum
-  uint32_t qb[3][EV / 4];  // byte planes of the fixed-point q: [2] signed top, [1] and [0] unsigned
+  uint32_t qb[2][EV / 4];  // byte planes of the fixed-point q: [1] signed high, [0] unsigned low
   uint32_t qh2[EV / 2];    // f16 pairs of the rescaled q (FP8 cache)
   float q_unit = 1.f;      // factor from the raw dot product to the base-2 score (before the K scale)
   float m = -FLT_MAX, l = 0.f;  // running max (base 2) and sum; -FLT_MAX keeps exp2 finite
@@ -218,21 +219,19 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
 #pragma unroll
       for (int off = LPR / 2; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
       int ex = 0;
-      frexpf(amax, &ex);                        // amax < 2^ex
-      const int E = max(-100, min(100, 22 - ex));  // amax * 2^E < 2^22
+      frexpf(amax, &ex);                           // amax < 2^ex
+      const int E = max(-100, min(100, 15 - ex));  // amax * 2^E < 2^15
       const float up = ldexpf(1.f, E);
       q_unit = ldexpf(1.f, -E);
 #pragma unroll
       for (int j = 0; j < EV / 4; ++j) {
-        uint32_t w2 = 0, w1 = 0, w0 = 0;
+        uint32_t w1 = 0, w0 = 0;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int qi = max(-(1 << 22) + 1, min((1 << 22) - 1, __float2int_rn(qf[4 * j + k] * up)));
-          w2 |= (static_cast<uint32_t>(qi >> 16) & 0xffu) << (8 * k);
+          const int qi = max(-32767, min(32767, __float2int_rn(qf[4 * j + k] * up)));
           w1 |= (static_cast<uint32_t>(qi >> 8) & 0xffu) << (8 * k);
           w0 |= (static_cast<uint32_t>(qi) & 0xffu) << (8 * k);
         }
-        qb[2][j] = w2;
         qb[1][j] = w1;
         qb[0][j] = w0;
       }
@@ -262,18 +261,18 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
       if (TT > 0 || pi * RPP < tt) {  // warp-uniform
         const int t = pi * RPP + r;
         float part = 0.f;
+        int ipart = 0;  // INT8: the exact integer dot product
         if (t < tt) {
           const uint4 kv = ld_shared_v4(kt + ((t * HG + kw) * D + v * EV) * E);
           if constexpr (kDp4a) {
             const uint32_t words[4] = {kv.x, kv.y, kv.z, kv.w};
-            int a2 = 0, a1 = 0, a0 = 0;
+            int a1 = 0, a0 = 0;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              a2 = dp4a_ss(words[j], qb[2][j], a2);
-              a1 = dp4a_su(words[j], qb[1][j], a1);
+              a1 = dp4a_ss(words[j], qb[1][j], a1);
               a0 = dp4a_su(words[j], qb[0][j], a0);
             }
-            part = fmaf(static_cast<float>(a2), 65536.f, fmaf(static_cast<float>(a1), 256.f, static_cast<float>(a0)));
+            ipart = a1 * 256 + a0;
           } else if constexpr (kMixed) {
             const uint32_t words[4] = {kv.x, kv.y, kv.z, kv.w};
             float a0 = 0.f, a1 = 0.f;
@@ -292,8 +291,14 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
             for (int e = 0; e < EV; ++e) part = fmaf(qf[e], kf[e], part);
           }
         }
+        if constexpr (kDp4a) {
 #pragma unroll
-        for (int off = LPR / 2; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+          for (int off = LPR / 2; off >= 1; off >>= 1) ipart += __shfl_xor_sync(0xffffffffu, ipart, off);
+          part = static_cast<float>(ipart);
+        } else {
+#pragma unroll
+          for (int off = LPR / 2; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+        }
         const int tok = tok0 + t;
         if (t < tt && tok >= c.sp.lo && tok < c.sp.ctx) {
           if (kInt8) part *= __half2float(__ushort_as_half(ld_shared_u16(kt + p.ks_off + (t * 8 + hs) * 2))) * q_unit;

@@ -265,12 +265,15 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     int fst_seq = -1, fst_base = 0, fst = 0;     // first window of the sequence
     Cursor c = start;
     int issued = 0;
-    // Widening of 8-bit codes.  Thread r owns token row r of the tile: it reads the row's
-    // 128 codes (8 swizzled 16-byte chunks) into registers, then writes dims 0..63 over the
-    // same 128 bytes and dims 64..127 into the hi half, both in the 128-byte-swizzled
-    // layout the MMAs read.  V rows of unattended tokens become zeros (they may hold
-    // anything, and 0 * NaN would poison the weighted sum).  A stage is handed to the MMA
-    // issuer once all 128 rows are done.
+    // Widening of 8-bit codes.  Thread r owns token row r of the tile: code chunk c (codes
+    // 16c .. 16c + 15, one swizzled 16-byte chunk) becomes operand chunks 2c and 2c + 1 of the
+    // lo half (c < 4) or, less 4, of the hi half, in the 128-byte-swizzled layout the MMAs
+    // read.  The hi half goes first; the lo half then overwrites the codes' own 128 bytes
+    // from c = 3 down to 0, so every chunk written there was read already, one code chunk at
+    // a time.  The loop is kept rolled: the fully unrolled form starved the warps of
+    // instructions.  V rows of unattended tokens become zeros (they may hold anything, and
+    // 0 * NaN would poison the weighted sum).  A stage is handed to the MMA issuer once all
+    // 128 rows are done.
     Cursor cc = start;
     int widened = 0;
     const int wr = 32 * part + lane;  // row this thread widens
@@ -280,26 +283,22 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       const int tok = (cc.sp.first_t + cc.j) * kTokens + wr;
       const bool valid = tok >= cc.sp.lo && tok < cc.sp.ctx;
       const uint32_t sw = wr & 7;
-#pragma unroll
-      for (int kv = 0; kv < 2; ++kv) {  // K codes in K lo, V codes in V lo
-        const uint32_t row = stage(st) + kv * 2 * kHalf + wr * 128;
-        uint4 raw[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) raw[k] = ld_shared_v4(row + 16 * (k ^ sw));
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {  // codes 16k .. 16k + 15 -> 16-byte chunks 2k, 2k + 1
-          uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-          if (kv == 0)
-            widen16<IO, CT>(raw[k], o);       // K: the score MMA's type, q's
-          else if (valid)
-            widen16<__half, CT>(raw[k], o);   // V: fp16, like the weights of the value MMA
-          const uint32_t dst = row + (k >= 4 ? kHalf : 0);
-          const uint32_t m0 = (2 * k) & 7, m1 = (2 * k + 1) & 7;
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16 * (m0 ^ sw)), "r"(o[0]), "r"(o[1]),
-                       "r"(o[2]), "r"(o[3]) : "memory");
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16 * (m1 ^ sw)), "r"(o[4]), "r"(o[5]),
-                       "r"(o[6]), "r"(o[7]) : "memory");
-        }
+#pragma unroll 1
+      for (int i = 0; i < 16; ++i) {  // K (i < 8), then V; chunks 4..7, then 3 down to 0
+        const int kv = i >> 3, k = (i & 7) < 4 ? 4 + (i & 3) : 3 - (i & 3);
+        const uint32_t row = stage(st) + kv * 2 * kHalf + wr * 128;  // K codes in K lo, V codes in V lo
+        const uint4 raw = ld_shared_v4(row + 16 * (k ^ sw));
+        uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (kv == 0)
+          widen16<IO, CT>(raw, o);       // K: the score MMA's type, q's
+        else if (valid)
+          widen16<__half, CT>(raw, o);   // V: fp16, like the weights of the value MMA
+        const uint32_t dst = row + (k >= 4 ? kHalf : 0);
+        const uint32_t m0 = (2 * k) & 7, m1 = (2 * k + 1) & 7;
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16 * (m0 ^ sw)), "r"(o[0]), "r"(o[1]),
+                     "r"(o[2]), "r"(o[3]) : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16 * (m1 ^ sw)), "r"(o[4]), "r"(o[5]),
+                     "r"(o[6]), "r"(o[7]) : "memory");
       }
       fence_proxy_async_shared();  // the widened operands are read by the tensor cores
       mbar_arrive(conv0 + 8 * st);

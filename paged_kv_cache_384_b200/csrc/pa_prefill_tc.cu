@@ -599,19 +599,19 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         st_shared_v4(dst + 16 * ((m + 1) ^ sw), o[4], o[5], o[6], o[7]);
       };
       auto widen_row = [&](uint32_t row, bool live, float sc, bool to_half) {
-#pragma unroll
-        for (int c = 4; c < 8; ++c) widen_chunk(row, c, live, sc, to_half);
-#pragma unroll
-        for (int c = 3; c >= 0; --c) widen_chunk(row, c, live, sc, to_half);
+        // rolled: the unrolled form starved the warps of instructions
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i) widen_chunk(row, i < 4 ? 4 + i : 7 - i, live, sc, to_half);
         fence_proxy_async_shared();  // the operand is read by the tensor cores
       };
       // The tiles of this CTA in order, with this thread's row of each: whether it is live,
-      // and where its scales are.  The next tile's block-table entry and scales are loaded
-      // while the current one is widened, so the two dependent global loads stay off the
-      // critical path.
+      // its block-table entry and its scales.  Loads run two tiles ahead: while a tile is
+      // widened, the block-table entry of the tile after next and the scales of the next tile
+      // (from the entry loaded one tile earlier) are in flight, so neither dependent global
+      // load sits on the critical path.
       struct RowRef {
         bool ok, live;
-        int kv, s, kh;
+        int kv, s, kh, pb;
         uint16_t ks, vs;  // fp16 bits of the scales (live rows)
       };
       UnitCursor cur;
@@ -629,6 +629,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         t.s = w.s;
         t.kh = w.kh;
         t.ks = t.vs = 0;
+        t.pb = t.live ? __ldg(p.block_tables + static_cast<size_t>(w.s) * p.MB + t.kv / bs) : 0;
         if (++j == w.n) {
           j = 0;
           more = cur.next(p, &w);
@@ -636,18 +637,18 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       };
       auto scales = [&](RowRef& t) {
         if (!t.ok || !t.live) return;
-        int pb = __ldg(p.block_tables + static_cast<size_t>(t.s) * p.MB + t.kv / bs);
-        if (pb < 0 || pb >= p.NB) pb = 0;  // reported by the K copy warp
+        const int pb = (t.pb < 0 || t.pb >= p.NB) ? 0 : t.pb;  // reported by the K copy warp
         const size_t srow = (static_cast<size_t>(pb) * bs + t.kv % bs) * p.Hkv + t.kh;
         t.ks = __ldg(p.k_scale + srow);
         t.vs = __ldg(p.v_scale + srow);
       };
-      RowRef now, nxt;
+      RowRef now, nxt, after;
       take(now);
       scales(now);
+      take(nxt);
       for (int gt = 0; now.ok; ++gt) {
-        take(nxt);
-        scales(nxt);  // in flight while this tile is widened
+        take(after);   // block-table entry of the tile after next: in flight
+        scales(nxt);   // scales of the next tile: in flight while this tile is widened
         const int st = gt % kRing;
         if (!__all_sync(0xffffffffu, wait_or_abort(k_full0 + 8 * st, (gt / kRing) & 1, abort))) break;
         widen_row(sK(st) + r * 128, now.live, __half2float(__ushort_as_half(now.ks)), false);
@@ -656,6 +657,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         widen_row(sV(st) + r * 128, now.live, __half2float(__ushort_as_half(now.vs)), true);
         mbar_arrive(v_conv0 + 8 * st);
         now = nxt;
+        nxt = after;
       }
     }
     end_barrier();
