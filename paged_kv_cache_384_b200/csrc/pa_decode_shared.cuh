@@ -14,9 +14,9 @@ __device__ __forceinline__ void decode_error(unsigned int bits) { atomicOr(&g_de
 constexpr int kMaxCtasPerSm = 4;    // persistent-grid CTAs per SM (upper bound)
 constexpr int kMaxHeadGroup = 8;    // heads per CTA (upper bound)
 constexpr int kMaxThreads = 32 * (kMaxHeadGroup + 1);  // CUDA-core kernel: TMA warp + head warps
-// Threads per CTA of any kernel that plans with plan_slice (the tensor-core kernel has up to 448);
+// Threads per CTA of any kernel that plans with plan_slice (the tensor-core kernel has up to 576);
 // PlanScratch holds one entry each.
-constexpr int kMaxPlanThreads = 448;
+constexpr int kMaxPlanThreads = 576;
 static_assert(kMaxPlanThreads >= kMaxThreads, "plan scratch must cover the CUDA-core kernel");
 constexpr int kBarrierBytes = 128;  // mbarriers at the front of dynamic smem (<= 8 stages)
 

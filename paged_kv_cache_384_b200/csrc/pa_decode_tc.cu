@@ -25,6 +25,8 @@
 //               by the lanes in parallel.
 //   warp 1      TMEM owner and MMA issuer (one lane); with up to 8 query heads per cached
 //               head warp 9 issues the value MMAs and warp 1 only the score MMAs.
+//   warps 10..13 (14..17 with 16 query heads per row), 8-bit caches only: widen each
+//               landed tile's codes in place to 16-bit operands, thread = token row.
 //   warps 2..5  softmax (thread = token row of S^T) and accumulation (thread = head dim row
 //               of O^T): online softmax in base 2, probabilities written as the B operand of
 //               the value MMA, V rows of unattended tokens zeroed (by the widening TMA warps
@@ -61,12 +63,14 @@ constexpr int kScaleBytes = kTokens * 16;       // fp16 scales of a tile for an 
 constexpr int stage_bytes(bool quant) { return 4 * kHalf + 2 * kQHalf + (quant ? 2 * kScaleBytes : 0); }
 constexpr int kStages = 3;
 constexpr int kPBytes = kTokens * kHeadsN * 2;  // one probability operand, 128 tokens x 16 heads
-constexpr int kConverters = 128;                // threads widening 8-bit codes (the four TMA warps)
 // Threads of the kernel tracking NH query heads per row: TMA warps 0 and 6..8, MMA warps
 // 1 and 9, softmax warps 2..5 (and 10..13 when NH = 16: two warps per TMEM lane quarter,
 // 8 heads each).
-constexpr int threads_for(int nh) { return nh > 8 ? 448 : 320; }
-static_assert(threads_for(16) <= kMaxPlanThreads, "plan_slice keeps one scratch entry per thread");
+constexpr int base_threads(int nh) { return nh > 8 ? 448 : 320; }
+// + four warps that widen the codes of an 8-bit cache (warps base_threads / 32 ..).
+constexpr int kConverters = 128;
+constexpr int threads_for(int nh, bool quant) { return base_threads(nh) + (quant ? kConverters : 0); }
+static_assert(threads_for(16, true) <= kMaxPlanThreads, "plan_slice keeps one scratch entry per thread");
 constexpr uint32_t kTmemCols = 64;              // S0 [0,16)  S1 [16,32)  O0 [32,48)  O1 [48,64)
 // Probability operands: 2 tiles in flight x (hi, lo) parts for a bf16 cache, x 1 part otherwise.
 // The plan scratch shares their space (the plan is done before the first one is written).
@@ -162,7 +166,7 @@ __device__ __forceinline__ void widen16(const uint4& in, uint32_t* out) {
 // bf16 probabilities are split into hi + lo bf16 parts and the value MMA runs on both, so
 // the weights keep ~16 significant bits (one bf16 part alone keeps 8).
 template <typename IO, typename CT, int NH>
-__global__ void __launch_bounds__(threads_for(NH), 1)
+__global__ void __launch_bounds__(threads_for(NH, !std::is_same<CT, IO>::value), 1)
 decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKs,
                      const __grid_constant__ CUtensorMap tmVs, const DecodeParams p) {
@@ -223,7 +227,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
   }
   // The q rows of a head group fill rows 0..GQ-1 of each stage's 16-row q block; rows
   // GQ..15 stay zero (padding of the MMA N dimension).
-  for (int i = threadIdx.x; i < kStages * 2 * kQHalf / 16; i += threads_for(NH)) {
+  for (int i = threadIdx.x; i < kStages * 2 * kQHalf / 16; i += blockDim.x) {
     const int st = i / (2 * kQHalf / 16), off = (i % (2 * kQHalf / 16)) * 16;
     uint8_t* ptr = smem_raw + (stage(st) - smem_u32(smem_raw)) + 4 * kHalf + off;
     *reinterpret_cast<uint4*>(ptr) = make_uint4(0, 0, 0, 0);
@@ -240,8 +244,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     // Four warps, one per (K or V) x (64-dim half) part of a tile: a warp issues its copies
     // one after another, so four warps issue a tile four times as fast as one.  Warp 0
     // also loads the q rows.  Every warp walks the same tile stream and block table.
-    // 8-bit cache: the parts are K codes (+ q rows), V codes, K scales and V scales, and the
-    // four warps also widen each landed tile's codes, thread = row.
+    // 8-bit cache: the parts are K codes (+ q rows), V codes, K scales and V scales.
     const int part = warp == 0 ? 0 : warp - 5;  // 0: K lo, 1: K hi, 2: V lo, 3: V hi
     const CUtensorMap* map = kQuant ? (part == 0 ? &tmK : part == 1 ? &tmV : part == 2 ? &tmKs : &tmVs)
                                     : (part < 2 ? &tmK : &tmV);
@@ -265,47 +268,6 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     int fst_seq = -1, fst_base = 0, fst = 0;     // first window of the sequence
     Cursor c = start;
     int issued = 0;
-    // Widening of 8-bit codes.  Thread r owns token row r of the tile: code chunk c (codes
-    // 16c .. 16c + 15, one swizzled 16-byte chunk) becomes operand chunks 2c and 2c + 1 of the
-    // lo half (c < 4) or, less 4, of the hi half, in the 128-byte-swizzled layout the MMAs
-    // read.  The hi half goes first; the lo half then overwrites the codes' own 128 bytes
-    // from c = 3 down to 0, so every chunk written there was read already, one code chunk at
-    // a time.  The loop is kept rolled: the fully unrolled form starved the warps of
-    // instructions.  V rows of unattended tokens become zeros (they may hold anything, and
-    // 0 * NaN would poison the weighted sum).  A stage is handed to the MMA issuer once all
-    // 128 rows are done.
-    Cursor cc = start;
-    int widened = 0;
-    const int wr = 32 * part + lane;  // row this thread widens
-    auto widen_tile = [&]() -> bool {
-      const int st = widened % kStages;
-      if (!wait_or_abort(full0 + 8 * st, (widened / kStages) & 1, abort)) return false;
-      const int tok = (cc.sp.first_t + cc.j) * kTokens + wr;
-      const bool valid = tok >= cc.sp.lo && tok < cc.sp.ctx;
-      const uint32_t sw = wr & 7;
-#pragma unroll 1
-      for (int i = 0; i < 16; ++i) {  // K (i < 8), then V; chunks 4..7, then 3 down to 0
-        const int kv = i >> 3, k = (i & 7) < 4 ? 4 + (i & 3) : 3 - (i & 3);
-        const uint32_t row = stage(st) + kv * 2 * kHalf + wr * 128;  // K codes in K lo, V codes in V lo
-        const uint4 raw = ld_shared_v4(row + 16 * (k ^ sw));
-        uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        if (kv == 0)
-          widen16<IO, CT>(raw, o);       // K: the score MMA's type, q's
-        else if (valid)
-          widen16<__half, CT>(raw, o);   // V: fp16, like the weights of the value MMA
-        const uint32_t dst = row + (k >= 4 ? kHalf : 0);
-        const uint32_t m0 = (2 * k) & 7, m1 = (2 * k + 1) & 7;
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16 * (m0 ^ sw)), "r"(o[0]), "r"(o[1]),
-                     "r"(o[2]), "r"(o[3]) : "memory");
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16 * (m1 ^ sw)), "r"(o[4]), "r"(o[5]),
-                     "r"(o[6]), "r"(o[7]) : "memory");
-      }
-      fence_proxy_async_shared();  // the widened operands are read by the tensor cores
-      mbar_arrive(conv0 + 8 * st);
-      ++widened;
-      if (widened < n) advance(cc, p);
-      return true;
-    };
     // Issue the copies of tile `issued` (waiting, bounded, for its stage to be free).
     auto issue_next = [&]() -> bool {
       const int st = issued % kStages;
@@ -369,47 +331,8 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       ++issued;
       return true;
     };
-    if constexpr (!kQuant) {
-      while (issued < n)
-        if (!issue_next()) break;
-    } else {
-      // 8-bit cache: copies and widening interleave as each becomes possible -- the next
-      // tile's copies as soon as its stage is free, the widening of the oldest landed tile as
-      // soon as its codes have arrived -- so neither waits behind the other.  (Alternating
-      // them in a fixed order made every widening wait for the value MMA of an earlier tile.)
-      uint32_t idle = 0;
-      while (widened < n) {
-        bool progressed = false;
-        if (issued < n) {
-          int free_st = 1;
-          if (lane == 0 && issued >= kStages)
-            free_st = mbar_test_wait(empty0 + 8 * (issued % kStages), ((issued / kStages) - 1) & 1) ? 1 : 0;
-          if (__shfl_sync(0xffffffffu, free_st, 0)) {
-            if (!issue_next()) break;
-            progressed = true;
-          }
-        }
-        if (widened < issued) {
-          int landed = 0;
-          if (lane == 0) landed = mbar_test_wait(full0 + 8 * (widened % kStages), (widened / kStages) & 1) ? 1 : 0;
-          if (__shfl_sync(0xffffffffu, landed, 0)) {
-            if (!widen_tile()) break;
-            progressed = true;
-          }
-        }
-        if (progressed) {
-          idle = 0;
-        } else {
-          if (*abort) break;
-          if (++idle > 16 * kWaitLimit) {
-            if (lane == 0) decode_error(PA_DEVERR_TIMEOUT);
-            *abort = 1;
-            break;
-          }
-          __nanosleep(32);
-        }
-      }
-    }
+    while (issued < n)
+      if (!issue_next()) break;
     if (lane == 0)  // never leave with copies in flight
       for (int k = issued - kStages < 0 ? 0 : issued - kStages; k < issued; ++k)
         wait_or_abort(full0 + 8 * (k % kStages), (k / kStages) & 1, abort);
@@ -498,6 +421,51 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       mbar_wait_bounded(smem_u32(&sh.mma_done), 0);
     }
     __syncwarp();
+  } else if (kQuant && warp >= base_threads(NH) / 32) {
+    // ------------------------------------------------------------- 8-bit widening --
+    // Four warps, thread = token row r of every tile.  Code chunk c (codes 16c .. 16c + 15,
+    // one swizzled 16-byte chunk) becomes operand chunks 2c and 2c + 1 of the lo half (c < 4)
+    // or, less 4, of the hi half, in the 128-byte-swizzled layout the MMAs read: K in q's
+    // type (the score MMA's), V in fp16 (the value MMA's).  The hi half is made first from
+    // chunks 4..7; then chunks 0..3, all four read before any store, become the lo half over
+    // the codes' own 128 bytes.  Four chunks at a time keep four independent chains in
+    // flight; the loop over the halves stays rolled (fully unrolled code starved the warps of
+    // instructions).  V rows of unattended tokens become zeros (they may hold anything, and
+    // 0 * NaN would poison the weighted sum).  A stage goes to the MMA issuer once all 128
+    // rows are done.
+    const int wr = 32 * (warp - base_threads(NH) / 32) + lane;
+    const uint32_t sw = wr & 7;
+    Cursor cc = start;
+    for (int i = 0; i < n; ++i) {
+      const int st = i % kStages;
+      if (!wait_or_abort(full0 + 8 * st, (i / kStages) & 1, abort)) break;
+      const int tok = (cc.sp.first_t + cc.j) * kTokens + wr;
+      const bool valid = tok >= cc.sp.lo && tok < cc.sp.ctx;
+#pragma unroll 1
+      for (int part = 0; part < 4; ++part) {  // (K, V) x (hi half, lo half)
+        const int kv = part >> 1, g = 1 - (part & 1);
+        const uint32_t row = stage(st) + kv * 2 * kHalf + wr * 128;  // K codes in K lo, V codes in V lo
+        uint4 raw[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) raw[k] = ld_shared_v4(row + 16 * ((4 * g + k) ^ sw));
+        const uint32_t dst = row + g * kHalf;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+          if (kv == 0)
+            widen16<IO, CT>(raw[k], o);
+          else if (valid)
+            widen16<__half, CT>(raw[k], o);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16 * ((2 * k) ^ sw)), "r"(o[0]),
+                       "r"(o[1]), "r"(o[2]), "r"(o[3]) : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16 * ((2 * k + 1) ^ sw)), "r"(o[4]),
+                       "r"(o[5]), "r"(o[6]), "r"(o[7]) : "memory");
+        }
+      }
+      fence_proxy_async_shared();  // the widened operands are read by the tensor cores
+      mbar_arrive(conv0 + 8 * st);
+      if (i + 1 < n) advance(cc, p);
+    }
   } else {
     // ------------------------------------------------- softmax + accumulation warps --
     // (warps 2..5, and 10..13 for the heads 8..15 of a 16-head row)
@@ -746,7 +714,8 @@ pa_status tc_decode_launch(const CUtensorMap& tmK, const CUtensorMap& tmV, const
   CUtensorMap k = tmK, v = tmV, q = tmQ, ks = tmKs, vs = tmVs;
   DecodeParams p = prm;
   void* args[] = {&k, &v, &q, &ks, &vs, &p};
-  cudaError_t err = launch_dependent(fn, dim3(grid), dim3(small ? threads_for(8) : threads_for(16)), smem, stream, args);
+  cudaError_t err =
+      launch_dependent(fn, dim3(grid), dim3(threads_for(small ? 8 : 16, quant)), smem, stream, args);
   if (err != cudaSuccess) return cuda_fail(err, "launching the tensor-core decode kernel");
   return PA_OK;
 }

@@ -583,25 +583,30 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       const int r = 32 * (warp - kConvWarp0) + lane;
       const uint32_t sw = r & 7;
       // Code chunk c (codes 16c .. 16c + 15) becomes operand chunks 2c and 2c + 1 of the lo
-      // half (c < 4) or, less 4, of the hi half.  The hi half goes first; the lo chunks are
-      // then made from c = 3 down to 0, so that every chunk written over the row was read
-      // already (chunks 2c and 2c + 1 >= c), and one code chunk is held at a time.
-      auto widen_chunk = [&](uint32_t row, int c, bool live, float sc, bool to_half) {
-        const uint4 raw = ld_shared_v4(row + 16 * (c ^ sw));
-        uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        if (live) {
-          if (to_half) widen_scaled16<__half, CT>(raw, sc, o);
-          else widen_scaled16<IO, CT>(raw, sc, o);
-        }
-        const uint32_t dst = row + (c >= 4 ? kHalf : 0);
-        const int m = 2 * (c & 3);
-        st_shared_v4(dst + 16 * (m ^ sw), o[0], o[1], o[2], o[3]);
-        st_shared_v4(dst + 16 * ((m + 1) ^ sw), o[4], o[5], o[6], o[7]);
-      };
+      // half (c < 4) or, less 4, of the hi half.  Two chunks at a time (two independent
+      // chains in flight within the 64 registers of this warpgroup), in the order (4, 5),
+      // (6, 7) -- the hi half -- then (3, 2), (1, 0), so every lo chunk written over the
+      // codes' own bytes was read already.  The loop stays rolled (fully unrolled code starved
+      // the warps of instructions).
       auto widen_row = [&](uint32_t row, bool live, float sc, bool to_half) {
-        // rolled: the unrolled form starved the warps of instructions
 #pragma unroll 1
-        for (int i = 0; i < 8; ++i) widen_chunk(row, i < 4 ? 4 + i : 7 - i, live, sc, to_half);
+        for (int i = 0; i < 4; ++i) {
+          const int c0 = i < 2 ? 4 + 2 * i : 7 - 2 * i, c1 = i < 2 ? c0 + 1 : c0 - 1;
+          const uint4 raw0 = ld_shared_v4(row + 16 * (c0 ^ sw)), raw1 = ld_shared_v4(row + 16 * (c1 ^ sw));
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int c = k ? c1 : c0;
+            uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            if (live) {
+              if (to_half) widen_scaled16<__half, CT>(k ? raw1 : raw0, sc, o);
+              else widen_scaled16<IO, CT>(k ? raw1 : raw0, sc, o);
+            }
+            const uint32_t dst = row + (c >= 4 ? kHalf : 0);
+            const int m = 2 * (c & 3);
+            st_shared_v4(dst + 16 * (m ^ sw), o[0], o[1], o[2], o[3]);
+            st_shared_v4(dst + 16 * ((m + 1) ^ sw), o[4], o[5], o[6], o[7]);
+          }
+        }
         fence_proxy_async_shared();  // the operand is read by the tensor cores
       };
       // The tiles of this CTA in order, with this thread's row of each: whether it is live,
