@@ -245,11 +245,12 @@ pa_status reshape_and_cache(const void* k, const void* v, void* k_cache, void* v
  *   sits at position p = ctx - q_len + i and attends tokens [lo, p], lo = max(0, p + 1 -
  *   window) for window > 0, else 0.  q_len == 1 is decode.
  *
- *   out, q         [num_q_tokens, num_q_heads, 128] in dtype (PA_F16 or PA_BF16); the rows of
- *                  sequence s are cu_q_lens[s] .. cu_q_lens[s+1]-1;
+ *   out, q         [num_q_tokens, num_q_heads, head_dim] in dtype (PA_F16 or PA_BF16); the
+ *                  rows of sequence s are cu_q_lens[s] .. cu_q_lens[s+1]-1;
  *                  num_q_tokens * num_q_heads < 2^31 (else PA_ERR_UNSUPPORTED)
- *   k_cache,       [num_blocks, block_size, num_kv_heads, 128] in dtype
+ *   k_cache,       [num_blocks, block_size, num_kv_heads, head_dim] in dtype
  *   v_cache
+ *   head_dim       128 or 64 (else PA_ERR_UNSUPPORTED)
  *   block_tables   [num_seqs, max_blocks_per_seq] int32
  *   cu_q_lens      [num_seqs + 1] int32 device array, cu_q_lens[0] = 0, non-decreasing
  *   context_lens   [num_seqs] int32 device array, q_len <= context_len <= max_blocks_per_seq*block_size
@@ -275,6 +276,7 @@ pa_status paged_attention_prefill(void* out, const void* q, const void* k_cache,
  * "量化压缩KV Cache的INT8与FP8方案" (8-bit KV caches), with the prefill reading above.
  *
  *   k_cache, v_cache  [num_blocks, block_size, num_kv_heads, 128] codes of cache_dtype
+ *                     (head_dim must be 128: another value is PA_ERR_UNSUPPORTED)
  *   k_scale, v_scale  [num_blocks, block_size, num_kv_heads] fp16 (2-byte aligned)
  *   io_dtype          PA_F16 or PA_BF16 (q and out)
  *   cache_dtype       PA_I8 or PA_FP8_E4M3 (anything else: PA_ERR_INVALID_ARG)

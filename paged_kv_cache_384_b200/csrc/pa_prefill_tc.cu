@@ -46,6 +46,9 @@
 // the I/O type (relative error 2^-11 for fp16, 2^-8 for bf16), V to fp16 (2^-11) -- with
 // zeros in rows no query attends; the MMA warp then sees an ordinary 16-bit tile, and the
 // value MMA runs in fp16 with fp16 weights whatever the I/O type (no hi + lo split).
+// head_dim 64 (16-bit caches): q, K and V use only the lo 64-dim halves of their slots, the
+// score MMAs take 4 K-steps instead of 8 and the value MMA has N = 64; each softmax warp
+// writes 32 of a row's 64 output dims.
 // Every wait is bounded; one that gives up raises PA_DEVERR_TIMEOUT and an abort flag that
 // ends the others.
 #include <cfloat>
@@ -67,7 +70,7 @@ namespace {
 
 constexpr int kRows = 128;                // query rows per CTA (MMA M)
 constexpr int kKv = 128;                  // kv tokens per tile
-constexpr int kDim = 128;                 // head_dim
+constexpr int kDim = 128;                 // largest head_dim (64 uses the lo halves only)
 constexpr int kHalf = 128 * 128;          // one 64-element half of a 128-row operand: 16 KiB
 constexpr int kOpBytes = 2 * kHalf;       // a whole 128 x 128 operand (Q, K, V or P)
 constexpr int kRing = 3;                  // depth of the K ring and of the V ring
@@ -97,6 +100,7 @@ struct PrefillParams {
   const int32_t* cu_q;
   const int32_t* context_lens;
   int S, T, Hq, Hkv, GQ, gq_shift, tq, bs, MB, NB, window, max_q_len;
+  int dim;       // head_dim: 128, or 64 (16-bit cache; the hi 64-dim halves stay unused)
   int qtiles;    // query tiles of the longest sequence: ceil(max_q_len / tq)
   int units;     // S * Hkv * qtiles work units, walked by a persistent grid
   float qscale;  // scale * log2(e)
@@ -344,6 +348,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   // and the weights then keep 11 significant bits (8 in bf16).
   using PW = typename std::conditional<kQuant, __half, IO>::type;  // probability / V operand type
   constexpr uint32_t kIdescO = mma_idesc_f16(kQuant ? 0u : kFmt, 0, 1, kRows, kDim);  // K-major P, MN-major V
+  constexpr uint32_t kIdescO64 = mma_idesc_f16(kQuant ? 0u : kFmt, 0, 1, kRows, 64);  // head_dim 64
+  const int nhalf = p.dim / 64;  // 64-dim halves of q, K, V and O in use (1 or 2)
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ PfShared sh;
@@ -435,8 +441,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
           if (lane == 0) {
             ok = uq == 0 || wait_or_abort(q_empty, (uq - 1) & 1, abort);
             if (ok) {
-              mbar_arrive_expect_tx(q_full, nh * kHalf);
-              for (int dh = h0; dh < h0 + nh; ++dh)
+              const int nq = max(0, min(h0 + nh, nhalf) - h0);  // halves of q this warp brings
+              mbar_arrive_expect_tx(q_full, nq * kHalf);
+              for (int dh = h0; dh < h0 + nq; ++dh)
                 tma_load_3d(sQ + dh * kHalf, &tmQ, q_full, dh * 64, w.kh * p.GQ, w.q_start + w.i0, once);
             }
           }
@@ -463,7 +470,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
           }
           // 8-bit cache: one copy per block (a token's 128 codes are one 128-byte row) into
           // the slot's lo half, by the K warp and the V lo warp; the V hi warp only arrives.
-          const int ncopy = kQuant ? (is_v && h0 == 1 ? 0 : 1) : nh;  // copies per block
+          // head_dim 64: the lo halves only.
+          const int ncopy = kQuant ? (is_v && h0 == 1 ? 0 : 1) : max(0, min(h0 + nh, nhalf) - h0);  // per block
           if (lane == 0) mbar_arrive_expect_tx(full0 + 8 * st, static_cast<uint32_t>(ncopy * nload) * bs * 128u);
           __syncwarp();
           const int bi = ncopy == 2 ? lane >> 1 : lane;  // block of this lane's copy
@@ -522,12 +530,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
                 (P.idx > 0 || P.uq == 0 || mbar_test_wait(o_free, (P.uq - 1) & 1))) {
               tc_fence_after_sync();
   #pragma unroll
+              const uint32_t idesc_o = nhalf == 2 ? kIdescO : kIdescO64;
+  #pragma unroll
               for (int part = 0; part < (kSplit ? 2 : 1); ++part) {
   #pragma unroll
                 for (int kk = 0; kk < kKv / 16; ++kk) {  // O_h += P_h . V_h, 16 kv tokens per MMA
                   const int h = kk / 4;                    // softmax half owning these tokens
                   tc_mma_f16_ts(tmem + kColO + 128 * h, tmem + b * kKv + 64 * h + 32 * part + (kk % 4) * 8,
-                                smem_desc(sV(st) + kk * 2048, kHalf, 1024, kSwizzle128B), kIdescO,
+                                smem_desc(sV(st) + kk * 2048, kHalf, 1024, kSwizzle128B), idesc_o,
                                 P.idx > 0 || part > 0 || (kk % 4) > 0);
                 }
               }
@@ -546,6 +556,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
               tc_fence_after_sync();
   #pragma unroll
               for (int kk = 0; kk < kDim / 16; ++kk) {  // S[b] = Q . K^T, 16 dims per MMA
+                if (kk >= 4 * nhalf) break;
                 const uint32_t off = (kk / 4) * kHalf + (kk % 4) * 32;
                 tc_mma_f16(tmem + b * kKv, smem_desc(sQ + off, 16, 1024, kSwizzle128B),
                            smem_desc(sK(st) + off, 16, 1024, kSwizzle128B), kIdescS, kk > 0);
@@ -728,12 +739,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       if (fin) {
         tc_fence_after_sync();
         const float w0 = half == 0 ? w_me : w_other, w1 = half == 0 ? w_other : w_me;
-        IO* orow = reinterpret_cast<IO*>(p.out) + static_cast<size_t>(pend_row) * kDim + 64 * half;
+        const int hd = 32 * nhalf;  // head dims this warp writes: 64, or 32 at head_dim 64
+        IO* orow = reinterpret_cast<IO*>(p.out) + static_cast<size_t>(pend_row) * p.dim + hd * half;
 #pragma unroll
-        for (int c4 = 0; c4 < 2; ++c4) {  // this warp's 64 head dims, 32 at a time
+        for (int c4 = 0; c4 < 2; ++c4) {  // this warp's head dims, 32 at a time
+          if (c4 >= nhalf) break;
           float o0[32], o1[32];
-          tmem_load32(tmem + lane_addr + kColO + 64 * half + 32 * c4, o0);
-          tmem_load32(tmem + lane_addr + kColO + 128 + 64 * half + 32 * c4, o1);
+          tmem_load32(tmem + lane_addr + kColO + hd * half + 32 * c4, o0);
+          tmem_load32(tmem + lane_addr + kColO + 128 + hd * half + 32 * c4, o1);
           if (pend_row >= 0) {
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -808,7 +821,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
           tc_fence_after_sync();
           const float a = rescale ? alpha : 1.f;
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
+          for (int c4 = 0; c4 < 4; ++c4) {  // the 64 * nhalf columns of O_h in use
+            if (c4 >= 2 * nhalf) break;
             float o[32];
             tmem_load32(o_col + 32 * c4, o);
 #pragma unroll
@@ -818,7 +832,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         }
         // V rows of tokens outside the loaded blocks or past the context may hold anything
         // (NaN); their weights are 0, so give the value MMA zeros there (kv row r; half 0
-        // clears its 64-dim lo half, half 1 the hi half).
+        // clears its 64-dim lo half, half 1 the hi half; at head_dim 64 the two halves clear
+        // four 16-byte chunks each of the lo half).
         const TileBlocks tb = tile_blocks(w.j_lo + j, bs, w.kv_lo, w.p_max);
         const int clean_lo = tb.lo * bs - kv0, clean_hi = min(w.ctx, (tb.hi + 1) * bs) - kv0;
         if (!kQuant && (clean_lo > 0 || clean_hi < kKv)) {  // (8-bit: the widening warps wrote the zeros)
@@ -827,8 +842,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
             break;
           }
           if (r < clean_lo || r >= clean_hi) {
+            const uint32_t zrow = nhalf == 2 ? sV(st) + half * kHalf + r * 128 : sV(st) + r * 128 + 64 * half;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) st_shared_v4(sV(st) + half * kHalf + r * 128 + 16 * k, 0, 0, 0, 0);
+            for (int k = 0; k < 8; ++k)
+              if (k < 4 * nhalf) st_shared_v4(zrow + 16 * k, 0, 0, 0, 0);
           }
         }
         // Probabilities of this half's 64 tokens, written over its own score columns as the
@@ -924,7 +941,8 @@ pa_status prefill_launch(void* out, const void* q, const void* k_cache, const vo
   const bool eight_bit = cache_dtype == PA_I8 || cache_dtype == PA_FP8_E4M3;
   if (cache_dtype != dtype && !eight_bit)
     return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: the cache must hold the I/O dtype, PA_I8 or PA_FP8_E4M3");
-  if (head_dim != kDim) return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: head_dim must be 128");
+  if (head_dim != kDim && (head_dim != 64 || eight_bit))
+    return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: head_dim must be 128 (or 64 with a 16-bit cache)");
   const int GQ = num_q_heads / num_kv_heads;
   if (GQ > kRows || (GQ & (GQ - 1)) != 0)
     return fail(PA_ERR_UNSUPPORTED, "paged_attention_prefill: query heads per cached head must be a power of two up to 128");
@@ -952,21 +970,22 @@ pa_status prefill_launch(void* out, const void* q, const void* k_cache, const vo
   const int tq = kRows / GQ;
   CUtensorMap tmK, tmV, tmQ;
   {
-    // [NB*bs rows][Hkv][128]: boxes of one block's rows x one head x 64 dims (16-bit cache)
-    // or all 128 one-byte codes (8-bit cache), 128-byte swizzle
-    const cuuint64_t e = eight_bit ? 1 : 2;
-    const cuuint64_t dims[3] = {kDim, static_cast<cuuint64_t>(num_kv_heads),
+    // [NB*bs rows][Hkv][head_dim]: boxes of one block's rows x one head x 64 dims (16-bit
+    // cache) or all 128 one-byte codes (8-bit cache), 128-byte swizzle
+    const cuuint64_t e = eight_bit ? 1 : 2, D = static_cast<cuuint64_t>(head_dim);
+    const cuuint64_t dims[3] = {D, static_cast<cuuint64_t>(num_kv_heads),
                                 static_cast<cuuint64_t>(num_blocks) * block_size};
-    const cuuint64_t strides[2] = {kDim * e, static_cast<cuuint64_t>(num_kv_heads) * kDim * e};
+    const cuuint64_t strides[2] = {D * e, static_cast<cuuint64_t>(num_kv_heads) * D * e};
     const cuuint32_t box[3] = {eight_bit ? 128u : 64u, 1, static_cast<cuuint32_t>(block_size)};
     const CUtensorMapDataType ctype = eight_bit ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : ttype;
     if ((st = encode(enc, &tmK, ctype, 3, k_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != PA_OK) return st;
     if ((st = encode(enc, &tmV, ctype, 3, v_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != PA_OK) return st;
   }
   {
-    // q as [T][Hq][128]: tq tokens x the GQ heads of one cached head x 64 dims
-    const cuuint64_t dims[3] = {kDim, static_cast<cuuint64_t>(num_q_heads), static_cast<cuuint64_t>(num_q_tokens)};
-    const cuuint64_t strides[2] = {kDim * 2, static_cast<cuuint64_t>(num_q_heads) * kDim * 2};
+    // q as [T][Hq][head_dim]: tq tokens x the GQ heads of one cached head x 64 dims
+    const cuuint64_t D = static_cast<cuuint64_t>(head_dim);
+    const cuuint64_t dims[3] = {D, static_cast<cuuint64_t>(num_q_heads), static_cast<cuuint64_t>(num_q_tokens)};
+    const cuuint64_t strides[2] = {D * 2, static_cast<cuuint64_t>(num_q_heads) * D * 2};
     const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(GQ), static_cast<cuuint32_t>(tq)};
     if ((st = encode(enc, &tmQ, ttype, 3, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != PA_OK) return st;
   }
@@ -989,6 +1008,7 @@ pa_status prefill_launch(void* out, const void* q, const void* k_cache, const vo
   prm.NB = num_blocks;
   prm.window = window > 0 ? window : 0;
   prm.max_q_len = max_q_len;
+  prm.dim = head_dim;
   prm.qtiles = (max_q_len + tq - 1) / tq;
   prm.qscale = scale * 1.4426950408889634f;
 

@@ -154,7 +154,8 @@ def test_prefill_host_validation(L):
     assert call(hq=12, hkv=4) == 2      # 3 query heads per cached head: unsupported
     assert call(hq=48, hkv=2) == 2      # 24 per cached head: not a power of two
     assert call(hq=512, hkv=2) == 2     # 256 per cached head: more than a unit's 128 rows
-    assert call(D=64) == 2              # head_dim 128 only
+    assert call(D=96) == 2              # head_dim 128 or 64 only
+    assert call(D=64, ptr=0) == 1       # head_dim 64 gets past the shape checks
     assert call(bs=12) == 2             # block size must divide 128 in steps of 8
     assert call(dt=0) == 2              # fp32 I/O is not a tensor-core type here
     assert call(T=-1) == 1
@@ -168,16 +169,17 @@ def test_prefill_host_validation(L):
 
 def test_prefill_quant_host_validation(L):
     P = ctypes.c_void_p
-    def call(cache=3, ks=16, vs=16, io=1):
+    def call(cache=3, ks=16, vs=16, io=1, D=128):
         p = P(16)
         k = P(ks) if ks else None
         v = P(vs) if vs else None
-        return L.paged_attention_prefill_quant(p, p, p, p, k, v, p, p, p, 1, 40, 40, 8, 2, 128, 16, 64, 8, 0.1, 0,
+        return L.paged_attention_prefill_quant(p, p, p, p, k, v, p, p, p, 1, 40, 40, 8, 2, D, 16, 64, 8, 0.1, 0,
                                                io, cache, None)
     assert call(cache=1) == 1           # a 16-bit cache belongs to paged_attention_prefill
     assert call(ks=0) == 1              # an 8-bit cache needs both scale pools
     assert call(vs=17) == 1             # fp16 scales must be 2-byte aligned
     assert call(io=0) == 2              # fp32 I/O is not a tensor-core type here
+    assert call(D=64) == 2              # 8-bit codes: head_dim 128 only
     assert L.pa_last_error().decode()
 
 

@@ -55,9 +55,9 @@ def run_gpu(q, kc, vc, bt, cu, ctx, scale, window=0, max_q_len=None):
     return out
 
 
-def check(seed, ctx, qlen, Hq, Hkv, bs, io, window=0):
-    q, kc, vc, bt, cu, cl = paged_case(seed, ctx, qlen, Hq, Hkv, bs, io)
-    scale = 1 / math.sqrt(128)
+def check(seed, ctx, qlen, Hq, Hkv, bs, io, window=0, D=128):
+    q, kc, vc, bt, cu, cl = paged_case(seed, ctx, qlen, Hq, Hkv, bs, io, D=D)
+    scale = 1 / math.sqrt(D)
     out = run_gpu(q, kc, vc, bt, cu, cl, scale, window)
     assert_no_device_error()
     ref = oracle.paged_prefill(q, kc, vc, bt, cu, cl, scale, window)
@@ -146,9 +146,14 @@ def test_prefill_host_validation(cuda_device):
     q, kc, vc, bt, cu, cl = paged_case(11, [20], [20], 6, 2, 16, "fp16")   # 3 heads per cached head
     with pytest.raises(pa.PagedAttnError):
         run_gpu(q, kc, vc, bt, cu, cl, 0.1)
-    q, kc, vc, bt, cu, cl = paged_case(12, [20], [20], 2, 2, 16, "fp16", D=64)
+    q, kc, vc, bt, cu, cl = paged_case(12, [20], [20], 2, 2, 16, "fp16", D=96)
     with pytest.raises(pa.PagedAttnError):
         run_gpu(q, kc, vc, bt, cu, cl, 0.1)
+    q, kc, vc, bt, cu, cl = paged_case(13, [20], [20], 2, 2, 16, "fp16", D=64)   # head_dim 64, 8-bit cache
+    k, v, ks, vs = quantised(kc, vc, "int8")
+    with pytest.raises(pa.PagedAttnError):
+        pa.paged_attention_prefill(torch.empty_like(q, device="cuda"), q.cuda(), k.cuda(), v.cuda(), bt.cuda(),
+                                   cu.cuda(), cl.cuda(), 20, 0.1, k_scale=ks.cuda(), v_scale=vs.cuda())
 
 
 def test_prefill_llama70b_prompt_batch_full(cuda_device):
@@ -284,3 +289,13 @@ def test_prefill_multi_query(cuda_device, Hq, Hkv, io):
     times all the query heads of one cached head."""
     check(41, [37, 300, 129, 16], [37, 90, 1, 16], Hq, Hkv, 16, io)
     check(42, [400, 45], [400, 45], Hq, Hkv, 32, io, window=100)
+
+
+@pytest.mark.parametrize("io", ["fp16", "bf16"])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 2), (32, 1)])
+def test_prefill_head_dim_64(cuda_device, io, Hq, Hkv):
+    """head_dim 64: the lo 64-dim halves of the operands, 4 score K-steps, a value MMA of
+    N = 64; mixed batch, several tiles, a window, and ragged tails."""
+    check(51, [37, 300, 129, 16], [37, 90, 1, 16], Hq, Hkv, 16, io, D=64)
+    check(52, [1000, 260], [1000, 70], Hq, Hkv, 32, io, window=100, D=64)
+    check(53, [130, 77], [130, 40], Hq, Hkv, 8, io, D=64)
