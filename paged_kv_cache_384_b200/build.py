@@ -19,7 +19,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libpagedattn.so")
-SOURCES = ["pa_host.cpp", "pa_decode.cu", "pa_decode_tc.cu", "pa_prefill_tc.cu", "pa_cache_ops.cu"]
+SOURCES = ["pa_host.cpp", "pa_decode.cu", "pa_decode_tc.cu", "pa_decode_tc8.cu", "pa_prefill_tc.cu", "pa_cache_ops.cu"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -14,9 +14,9 @@ __device__ __forceinline__ void decode_error(unsigned int bits) { atomicOr(&g_de
 constexpr int kMaxCtasPerSm = 4;    // persistent-grid CTAs per SM (upper bound)
 constexpr int kMaxHeadGroup = 8;    // heads per CTA (upper bound)
 constexpr int kMaxThreads = 32 * (kMaxHeadGroup + 1);  // CUDA-core kernel: TMA warp + head warps
-// Threads per CTA of any kernel that plans with plan_slice (the tensor-core kernel has up to 576);
+// Threads per CTA of any kernel that plans with plan_slice (the tensor-core kernels have up to 448);
 // PlanScratch holds one entry each.
-constexpr int kMaxPlanThreads = 576;
+constexpr int kMaxPlanThreads = 448;
 static_assert(kMaxPlanThreads >= kMaxThreads, "plan scratch must cover the CUDA-core kernel");
 constexpr int kBarrierBytes = 128;  // mbarriers at the front of dynamic smem (<= 8 stages)
 
@@ -124,7 +124,7 @@ __device__ __forceinline__ void store_floats(IO* dst, const float* src) {
 // the CTA must call it.  Returns count (0: nothing to do, or an impossible plan reported as
 // PA_DEVERR_TIMEOUT); *start is the cursor of tile t0.
 struct PlanScratch {
-  long long chunk[kMaxPlanThreads];
+  long long warp_sum[kMaxPlanThreads / 32];  // tiles counted by each warp, then their exclusive prefix
   long long total;
   long long first_prefix;
   int first_seq;
@@ -134,26 +134,37 @@ __device__ __forceinline__ long long plan_slice(const DecodeParams& p, PlanScrat
                                                 Cursor* start) {
   const int nthr = blockDim.x;
   const int G = p.G;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nwarps = (nthr + 31) >> 5;
   const int chunk = (p.S + nthr - 1) / nthr;
   const int s_lo = min(p.S, static_cast<int>(threadIdx.x) * chunk), s_hi = min(p.S, s_lo + chunk);
   long long mine = 0;
   for (int s = s_lo; s < s_hi; ++s) mine += seq_span(p, s, blockIdx.x == 0).nb;
-  sc.chunk[threadIdx.x] = mine;
+  // Exclusive prefix over the threads: a shuffle scan inside each warp, then over the warps'
+  // totals (a thread-serial scan measured ~6 us at 448 threads).
+  long long incl = mine;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const long long y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) sc.warp_sum[wid] = incl;
   if (threadIdx.x == 0) sc.first_seq = -1;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    long long run = 0;
-    for (int i = 0; i < nthr; ++i) {
-      const long long v = sc.chunk[i];
-      sc.chunk[i] = run;
-      run += v;
+  if (wid == 0) {
+    const long long v = lane < nwarps ? sc.warp_sum[lane] : 0;
+    long long w = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += y;
     }
-    sc.total = run;
+    if (lane < nwarps) sc.warp_sum[lane] = w - v;
+    if (lane == 31) sc.total = w;
   }
   __syncthreads();
   const long long per_group = sc.total;  // tiles of one head group over all sequences
   const long long T = per_group * G;
-  const long long my_prefix = sc.chunk[threadIdx.x];
+  const long long my_prefix = sc.warp_sum[wid] + incl - mine;
   if (blockIdx.x == 0) {  // publish the per-sequence prefix for the merge kernel
     long long r = my_prefix;
     for (int s = s_lo; s < s_hi; ++s) {
@@ -205,4 +216,8 @@ int tc_decode_tile_tokens();
 pa_status tc_decode_launch(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
                            const CUtensorMap& tmKs, const CUtensorMap& tmVs, const DecodeParams& prm, pa_dtype io,
                            pa_dtype cache, int grid, cudaStream_t stream);
+// 8-bit caches (pa_decode_tc8.cu): tmK / tmV map the codes, tmKs / tmVs the fp16 scales.
+pa_status tc8_decode_launch(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKs,
+                            const CUtensorMap& tmVs, const DecodeParams& prm, pa_dtype io, pa_dtype cache, int grid,
+                            cudaStream_t stream);
 }  // namespace pa

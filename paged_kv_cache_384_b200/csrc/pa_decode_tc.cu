@@ -25,19 +25,15 @@
 //               by the lanes in parallel.
 //   warp 1      TMEM owner and MMA issuer (one lane); with up to 8 query heads per cached
 //               head warp 9 issues the value MMAs and warp 1 only the score MMAs.
-//   warps 10..13 (14..17 with 16 query heads per row), 8-bit caches only: widen each
-//               landed tile's codes in place to 16-bit operands, thread = token row.
 //   warps 2..5  softmax (thread = token row of S^T) and accumulation (thread = head dim row
 //               of O^T): online softmax in base 2, probabilities written as the B operand of
-//               the value MMA, V rows of unattended tokens zeroed (by the widening TMA warps
-//               for an 8-bit cache), running output rescaled in registers.  Segment ends write the output or a partial (m, l, acc) exactly
-//               like the CUDA-core kernel, so the same merge kernel finishes split segments.
-// 8-bit caches (INT8 or FP8 E4M3 codes with one fp16 scale per token and head): the TMA
-// warps bring a tile's codes and scales, then widen every code in place (INT8 and E4M3
-// values are exact in fp16 and bf16): K to q's type, V to fp16, so the same MMAs run (the
-// value MMA in fp16); the softmax applies each token's K scale to its score row and folds
-// its V scale into the token's weight, rounded to fp16.  ("KV Cache optimisation strategies in deployment" (yunthe.com), section
-// "量化压缩KV Cache的INT8与FP8方案", for the 8-bit caches.)
+//               the value MMA, V rows of unattended tokens zeroed, running output rescaled
+//               in registers.  Segment ends write the output or a partial (m, l, acc)
+//               exactly like the CUDA-core kernel, so the same merge kernel finishes split
+//               segments.  (warps 10..13 too with 16 query heads per row: two warps per TMEM
+//               lane quarter, 8 heads each.)
+// 8-bit caches run on the kernel of pa_decode_tc8.cu, which feeds the codes to the tensor
+// cores as they are.
 // Every wait is bounded; a wait that gives up sets an abort flag that ends all the others.
 #include <algorithm>
 #include <cfloat>
@@ -57,32 +53,26 @@ constexpr int kDim = 128;                       // head_dim (64: the hi halves s
 constexpr int kHeadsN = 16;                     // query heads per cached head, padded (MMA N)
 constexpr int kHalf = kTokens * 128;            // one 64-dim half of a tile: 128 rows x 128 B
 constexpr int kQHalf = kHeadsN * 128;           // one 64-dim half of the q rows: 16 rows x 128 B
-constexpr int kScaleBytes = kTokens * 16;       // fp16 scales of a tile for an 8-head column group
-// Stage: K lo, K hi, V lo, V hi, Q lo, Q hi (+ K scales, V scales for an 8-bit cache; the
-// codes land in K lo and V lo and are widened in place).
-constexpr int stage_bytes(bool quant) { return 4 * kHalf + 2 * kQHalf + (quant ? 2 * kScaleBytes : 0); }
+// Stage: K lo, K hi, V lo, V hi, Q lo, Q hi.
+constexpr int kStageBytes = 4 * kHalf + 2 * kQHalf;
 constexpr int kStages = 3;
 constexpr int kPBytes = kTokens * kHeadsN * 2;  // one probability operand, 128 tokens x 16 heads
 // Threads of the kernel tracking NH query heads per row: TMA warps 0 and 6..8, MMA warps
 // 1 and 9, softmax warps 2..5 (and 10..13 when NH = 16: two warps per TMEM lane quarter,
 // 8 heads each).
 constexpr int base_threads(int nh) { return nh > 8 ? 448 : 320; }
-// + four warps that widen the codes of an 8-bit cache (warps base_threads / 32 ..).
-constexpr int kConverters = 128;
-constexpr int threads_for(int nh, bool quant) { return base_threads(nh) + (quant ? kConverters : 0); }
-static_assert(threads_for(16, true) <= kMaxPlanThreads, "plan_slice keeps one scratch entry per thread");
+static_assert(base_threads(16) <= kMaxPlanThreads, "plan_slice keeps one scratch entry per thread");
 constexpr uint32_t kTmemCols = 64;              // S0 [0,16)  S1 [16,32)  O0 [32,48)  O1 [48,64)
 // Probability operands: 2 tiles in flight x (hi, lo) parts for a bf16 cache, x 1 part otherwise.
 // The plan scratch shares their space (the plan is done before the first one is written).
 constexpr int p_parts(bool split) { return split ? 2 : 1; }
-constexpr size_t smem_bytes(bool quant, bool split) {
-  return 1024 + static_cast<size_t>(kStages) * stage_bytes(quant) + 2 * p_parts(split) * kPBytes;
+constexpr size_t smem_bytes(bool split) {
+  return 1024 + static_cast<size_t>(kStages) * kStageBytes + 2 * p_parts(split) * kPBytes;
 }
 static_assert(sizeof(PlanScratch) <= 2 * kPBytes, "plan scratch fits the probability buffers");
 
 struct TcShared {
   uint64_t full[kStages], empty[kStages];       // TMA ring
-  uint64_t conv[kStages];                       // 8-bit codes of a stage widened
   uint64_t s_full[2], s_empty[2];               // score accumulators in TMEM
   uint64_t p_full[2], o_full[2];                // probabilities written / value MMA done
   uint64_t mma_done;                            // both MMA warps' last MMAs finished
@@ -122,65 +112,19 @@ __device__ __forceinline__ void store_p_half_row(uint32_t buf, int r, int hh, co
                "r"(w[2]), "r"(w[3]) : "memory");
 }
 
-// Widen the 16 8-bit codes of one 16-byte chunk to 16 values of IO, exactly: out[0..3]
-// hold codes 0..7, out[4..7] codes 8..15, two per word, the lower code in the lower half.
-template <typename IO, typename CT>
-__device__ __forceinline__ void widen16(const uint4& in, uint32_t* out) {
-  const uint32_t w[4] = {in.x, in.y, in.z, in.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    if constexpr (std::is_same<CT, int8_t>::value && std::is_same<IO, __half>::value) {
-      // c + 128 spliced under the exponent of 1024 (0x6400 | b is the f16 value 1024 + b),
-      // minus 1152 in one f16x2 subtraction: exact for every code.
-      const uint32_t u = w[i] ^ 0x80808080u;
-      const uint32_t lo = __byte_perm(u, 0x6464u, 0x4140u), hi = __byte_perm(u, 0x6464u, 0x4342u);
-      const uint32_t bias = 0x64806480u;  // 1152, 1152
-      asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(out[2 * i]) : "r"(lo), "r"(bias));
-      asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(out[2 * i + 1]) : "r"(hi), "r"(bias));
-    } else if constexpr (std::is_same<CT, __nv_fp8_e4m3>::value && std::is_same<IO, __half>::value) {
-      e4m3x4_to_f16x2x2(w[i], out[2 * i], out[2 * i + 1]);
-    } else {
-      // bf16 operands: through fp32 (exact), then a pair conversion (exact: 8-bit values
-      // have at most 7 significant bits, and E4M3's exponents lie inside bf16's range).
-      float f[4];
-      if constexpr (std::is_same<CT, int8_t>::value) {
-        const uint32_t u = w[i] ^ 0x80808080u;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) f[b] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7440u | b)) - 8388736.0f;
-      } else {
-        uint32_t lo, hi;
-        e4m3x4_to_f16x2x2(w[i], lo, hi);
-        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo));
-        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hi));
-        f[0] = a.x, f[1] = a.y, f[2] = b.x, f[3] = b.y;
-      }
-      const __nv_bfloat162 p0 = __floats2bfloat162_rn(f[0], f[1]), p1 = __floats2bfloat162_rn(f[2], f[3]);
-      out[2 * i] = *reinterpret_cast<const uint32_t*>(&p0);
-      out[2 * i + 1] = *reinterpret_cast<const uint32_t*>(&p1);
-    }
-  }
-}
-
-// IO: fp16 or bf16 queries (and cache, unless CT is an 8-bit code type).  NH: query heads of
-// a row (8 or 16 >= GQ); a softmax thread tracks 8 of them.
-// bf16 probabilities are split into hi + lo bf16 parts and the value MMA runs on both, so
-// the weights keep ~16 significant bits (one bf16 part alone keeps 8).
-template <typename IO, typename CT, int NH>
-__global__ void __launch_bounds__(threads_for(NH, !std::is_same<CT, IO>::value), 1)
+// IO: fp16 or bf16 queries and cache.  NH: query heads of a row (8 or 16 >= GQ); a softmax
+// thread tracks 8 of them.  bf16 probabilities are split into hi + lo bf16 parts and the
+// value MMA runs on both, so the weights keep ~16 significant bits (one bf16 part alone
+// keeps 8).
+template <typename IO, int NH>
+__global__ void __launch_bounds__(base_threads(NH), 1)
 decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKs,
-                     const __grid_constant__ CUtensorMap tmVs, const DecodeParams p) {
-  constexpr bool kQuant = !std::is_same<CT, IO>::value;  // 8-bit codes + per-token scales
-  // bf16 weights keep ~16 bits as hi + lo parts; with an 8-bit cache (tolerance 1e-2) one
-  // part is enough.
-  constexpr bool kSplit = std::is_same<IO, __nv_bfloat16>::value && !kQuant;
-  constexpr int kStageBytes = stage_bytes(kQuant);
+                     const __grid_constant__ CUtensorMap tmQ, const DecodeParams p) {
+  constexpr bool kSplit = std::is_same<IO, __nv_bfloat16>::value;
   constexpr int kParts = p_parts(kSplit);
   constexpr uint32_t kFmt = std::is_same<IO, __nv_bfloat16>::value ? 1u : 0u;
   constexpr uint32_t kIdescS = mma_idesc_f16(kFmt, 0, 0, kTokens, kHeadsN);  // K-major A and B
-  // The value MMA of an 8-bit cache runs in fp16 whatever q's type: V codes are exact in fp16
-  // and a weight p * v_scale keeps 11 significant bits there (8 in bf16).
-  constexpr uint32_t kIdescO = mma_idesc_f16(kQuant ? 0u : kFmt, 1, 1, kDim, kHeadsN);  // MN-major A and B
+  constexpr uint32_t kIdescO = mma_idesc_f16(kFmt, 1, 1, kDim, kHeadsN);  // MN-major A and B
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ TcShared sh;
@@ -204,7 +148,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
   const int n = static_cast<int>(count);
   __syncthreads();  // every thread is done with the plan scratch before its space is reused
 
-  const uint32_t full0 = smem_u32(&sh.full[0]), empty0 = smem_u32(&sh.empty[0]), conv0 = smem_u32(&sh.conv[0]);
+  const uint32_t full0 = smem_u32(&sh.full[0]), empty0 = smem_u32(&sh.empty[0]);
   const uint32_t s_full0 = smem_u32(&sh.s_full[0]), s_empty0 = smem_u32(&sh.s_empty[0]);
   const uint32_t p_full0 = smem_u32(&sh.p_full[0]), o_full0 = smem_u32(&sh.o_full[0]);
   volatile int* abort = &sh.abort;
@@ -213,7 +157,6 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     for (int st = 0; st < kStages; ++st) {
       mbar_init(full0 + 8 * st, 4);  // one arrival per TMA warp
       mbar_init(empty0 + 8 * st, 1);
-      mbar_init(conv0 + 8 * st, kConverters);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full0 + 8 * b, 1);
@@ -244,10 +187,8 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     // Four warps, one per (K or V) x (64-dim half) part of a tile: a warp issues its copies
     // one after another, so four warps issue a tile four times as fast as one.  Warp 0
     // also loads the q rows.  Every warp walks the same tile stream and block table.
-    // 8-bit cache: the parts are K codes (+ q rows), V codes, K scales and V scales.
     const int part = warp == 0 ? 0 : warp - 5;  // 0: K lo, 1: K hi, 2: V lo, 3: V hi
-    const CUtensorMap* map = kQuant ? (part == 0 ? &tmK : part == 1 ? &tmV : part == 2 ? &tmKs : &tmVs)
-                                    : (part < 2 ? &tmK : &tmV);
+    const CUtensorMap* map = part < 2 ? &tmK : &tmV;
     const uint64_t policy = l2_policy_evict_first();
     if (lane == 0) {
       prefetch_tensormap(map);
@@ -299,10 +240,9 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         if (issued >= kStages) ok = wait_or_abort(empty0 + 8 * st, ((issued / kStages) - 1) & 1, abort);
         if (ok) {
           const uint32_t bar = full0 + 8 * st;
-          const uint32_t row_bytes = kQuant && part >= 2 ? 16u : 128u;  // a scale row: 8 heads x fp16
           const uint32_t halves = p.dim / 64;  // 64-dim halves of q (and of K, V) to copy
-          const int nblk = (!kQuant && (part & 1) && halves == 1) ? 0 : nload;  // head_dim 64: no hi halves
-          mbar_arrive_expect_tx(bar, (part == 0 ? halves * GQ * 128u : 0u) + static_cast<uint32_t>(nblk) * bs * row_bytes);
+          const int nblk = ((part & 1) && halves == 1) ? 0 : nload;  // head_dim 64: no hi halves
+          mbar_arrive_expect_tx(bar, (part == 0 ? halves * GQ * 128u : 0u) + static_cast<uint32_t>(nblk) * bs * 128u);
           if (part == 0) {
             const uint32_t sb = stage(st);
             const int qrow = c.s * p.Hq + c.g * GQ;
@@ -313,19 +253,10 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);  // also orders lane 0's expect_tx before any copy
       if (!ok) return false;
-      const bool copies = kQuant || !(part & 1) || p.dim == 128;  // head_dim 64: the hi-half warps only arrive
+      const bool copies = !(part & 1) || p.dim == 128;  // head_dim 64: the hi-half warps only arrive
       if (copies && lane < nload) {  // this warp's part of each attended block, one copy per lane
         const uint32_t row0 = static_cast<uint32_t>(lb_lo + lane - lb_first) * bs;  // first row in the tile
-        if constexpr (kQuant) {
-          if (part < 2)
-            tma_load_3d(stage(st) + part * 2 * kHalf + row0 * 128u, map, full0 + 8 * st, 0, kh, pb * bs, policy);
-          else  // scale rows: x rounded down to a 16-byte boundary (8 heads)
-            tma_load_2d(stage(st) + 4 * kHalf + 2 * kQHalf + (part - 2) * kScaleBytes + row0 * 16u, map,
-                        full0 + 8 * st, kh & ~7, pb * bs, policy);
-        } else {
-          tma_load_3d(stage(st) + part * kHalf + row0 * 128u, map, full0 + 8 * st, (part & 1) * 64, kh, pb * bs,
-                      policy);
-        }
+        tma_load_3d(stage(st) + part * kHalf + row0 * 128u, map, full0 + 8 * st, (part & 1) * 64, kh, pb * bs, policy);
       }
       advance(c, p);
       ++issued;
@@ -374,7 +305,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     // softmax work per tile is larger and one lane of warp 1 polling for either kind of
     // ready work measured faster (3.98 vs 3.08 TB/s at 4 cached heads); warp 9 then idles.
     constexpr bool kTwoIssuers = NH <= 8;
-    const uint32_t ready0 = kQuant ? conv0 : full0;  // a stage's operands are complete
+    const uint32_t ready0 = full0;  // a stage's operands are complete
     if (lane == 0 && kTwoIssuers) {
       if (warp == 1) {
         for (int i = 0; i < n; ++i) {
@@ -421,51 +352,6 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       mbar_wait_bounded(smem_u32(&sh.mma_done), 0);
     }
     __syncwarp();
-  } else if (kQuant && warp >= base_threads(NH) / 32) {
-    // ------------------------------------------------------------- 8-bit widening --
-    // Four warps, thread = token row r of every tile.  Code chunk c (codes 16c .. 16c + 15,
-    // one swizzled 16-byte chunk) becomes operand chunks 2c and 2c + 1 of the lo half (c < 4)
-    // or, less 4, of the hi half, in the 128-byte-swizzled layout the MMAs read: K in q's
-    // type (the score MMA's), V in fp16 (the value MMA's).  The hi half is made first from
-    // chunks 4..7; then chunks 0..3, all four read before any store, become the lo half over
-    // the codes' own 128 bytes.  Four chunks at a time keep four independent chains in
-    // flight; the loop over the halves stays rolled (fully unrolled code starved the warps of
-    // instructions).  V rows of unattended tokens become zeros (they may hold anything, and
-    // 0 * NaN would poison the weighted sum).  A stage goes to the MMA issuer once all 128
-    // rows are done.
-    const int wr = 32 * (warp - base_threads(NH) / 32) + lane;
-    const uint32_t sw = wr & 7;
-    Cursor cc = start;
-    for (int i = 0; i < n; ++i) {
-      const int st = i % kStages;
-      if (!wait_or_abort(full0 + 8 * st, (i / kStages) & 1, abort)) break;
-      const int tok = (cc.sp.first_t + cc.j) * kTokens + wr;
-      const bool valid = tok >= cc.sp.lo && tok < cc.sp.ctx;
-#pragma unroll 1
-      for (int part = 0; part < 4; ++part) {  // (K, V) x (hi half, lo half)
-        const int kv = part >> 1, g = 1 - (part & 1);
-        const uint32_t row = stage(st) + kv * 2 * kHalf + wr * 128;  // K codes in K lo, V codes in V lo
-        uint4 raw[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) raw[k] = ld_shared_v4(row + 16 * ((4 * g + k) ^ sw));
-        const uint32_t dst = row + g * kHalf;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-          if (kv == 0)
-            widen16<IO, CT>(raw[k], o);
-          else if (valid)
-            widen16<__half, CT>(raw[k], o);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16 * ((2 * k) ^ sw)), "r"(o[0]),
-                       "r"(o[1]), "r"(o[2]), "r"(o[3]) : "memory");
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16 * ((2 * k + 1) ^ sw)), "r"(o[4]),
-                       "r"(o[5]), "r"(o[6]), "r"(o[7]) : "memory");
-        }
-      }
-      fence_proxy_async_shared();  // the widened operands are read by the tensor cores
-      mbar_arrive(conv0 + 8 * st);
-      if (i + 1 < n) advance(cc, p);
-    }
   } else {
     // ------------------------------------------------- softmax + accumulation warps --
     // (warps 2..5, and 10..13 for the heads 8..15 of a 16-head row)
@@ -509,13 +395,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
 
       const int tok = (c.sp.first_t + c.j) * kTokens + r;
       const bool valid = tok >= c.sp.lo && tok < c.sp.ctx;
-      float kscale = 1.f, vscale = 1.f;  // this token's 8-bit scales
-      if (kQuant && valid) {
-        const uint32_t sa = stage(st) + 4 * kHalf + 2 * kQHalf + r * 16 + 2 * ((c.g / p.sub) & 7);
-        kscale = __half2float(__ushort_as_half(ld_shared_u16(sa)));
-        vscale = __half2float(__ushort_as_half(ld_shared_u16(sa + kScaleBytes)));
-      }
-      const float sfac = p.qscale * kscale;
+      const float sfac = p.qscale;
 #pragma unroll
       for (int h = 0; h < HPW; ++h) {
         sc[h] = (valid && h_base + h < GQ) ? sc[h] * sfac : -INFINITY;
@@ -537,11 +417,6 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         alpha[h] = exp2f(m[h] - m_new);
         m[h] = m_new;
         const float pr = sc[h] == -INFINITY ? 0.f : exp2f(sc[h] - m_new);
-        if constexpr (kQuant) {  // the value MMA multiplies V codes: fold the V scale into the weight
-          w_hi[h / 2] |= bits16(float_to<__half>(pr * vscale)) << (16 * (h & 1));
-          l[h] = l[h] * alpha[h] + pr;
-          continue;
-        }
         const IO hi = float_to<IO>(pr);
         w_hi[h / 2] |= bits16(hi) << (16 * (h & 1));
         if (kSplit) {
@@ -559,7 +434,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         store_p_row(pbuf(b, 0), r, w_hi);
         if (kSplit) store_p_row(pbuf(b, 1), r, w_lo);
       }
-      if (!kQuant && !valid && hh == 0) {  // unattended rows may hold anything (NaN): give the value MMA zeros
+      if (!valid && hh == 0) {  // unattended rows may hold anything (NaN): give the value MMA zeros
         // Chunk k ^ (r & 7) at step k: neighbouring rows (128 B apart, the same banks)
         // write different 16-byte chunks at each step, so a warp's stores do not conflict.
         const uint32_t v0 = stage(st) + 2 * kHalf + r * 128;
@@ -680,26 +555,20 @@ bool tc_decode_eligible(pa_dtype io, pa_dtype cache, int head_dim, int block_siz
 int tc_decode_tile_tokens() { return kTokens; }
 
 namespace {
-template <typename IO, typename CT, int NH>
-const void* tc_fn() {
-  return reinterpret_cast<const void*>(&decode_gqa_tc_kernel<IO, CT, NH>);
-}
 template <typename IO, int NH>
-const void* tc_fn_for_cache(pa_dtype cache) {
-  return cache == PA_I8 ? tc_fn<IO, int8_t, NH>() : cache == PA_FP8_E4M3 ? tc_fn<IO, __nv_fp8_e4m3, NH>()
-                                                                         : tc_fn<IO, IO, NH>();
+const void* tc_fn() {
+  return reinterpret_cast<const void*>(&decode_gqa_tc_kernel<IO, NH>);
 }
 }  // namespace
 
 pa_status tc_decode_launch(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
                            const CUtensorMap& tmKs, const CUtensorMap& tmVs, const DecodeParams& prm, pa_dtype io,
                            pa_dtype cache, int grid, cudaStream_t stream) {
+  if (cache != io) return tc8_decode_launch(tmK, tmV, tmKs, tmVs, prm, io, cache, grid, stream);
   const bool small = prm.GQ <= 8;
-  const bool quant = cache != io;
-  const void* fn = io == PA_BF16 ? (small ? tc_fn_for_cache<__nv_bfloat16, 8>(cache)
-                                          : tc_fn_for_cache<__nv_bfloat16, 16>(cache))
-                                 : (small ? tc_fn_for_cache<__half, 8>(cache) : tc_fn_for_cache<__half, 16>(cache));
-  const size_t smem = smem_bytes(quant, io == PA_BF16 && !quant);
+  const void* fn = io == PA_BF16 ? (small ? tc_fn<__nv_bfloat16, 8>() : tc_fn<__nv_bfloat16, 16>())
+                                 : (small ? tc_fn<__half, 8>() : tc_fn<__half, 16>());
+  const size_t smem = smem_bytes(io == PA_BF16);
   // The dynamic shared-memory limit is a per-kernel attribute: set once per kernel.
   static std::mutex m;
   static std::vector<const void*> ready;
@@ -711,11 +580,10 @@ pa_status tc_decode_launch(const CUtensorMap& tmK, const CUtensorMap& tmV, const
       ready.push_back(fn);
     }
   }
-  CUtensorMap k = tmK, v = tmV, q = tmQ, ks = tmKs, vs = tmVs;
+  CUtensorMap k = tmK, v = tmV, q = tmQ;
   DecodeParams p = prm;
-  void* args[] = {&k, &v, &q, &ks, &vs, &p};
-  cudaError_t err =
-      launch_dependent(fn, dim3(grid), dim3(threads_for(small ? 8 : 16, quant)), smem, stream, args);
+  void* args[] = {&k, &v, &q, &p};
+  cudaError_t err = launch_dependent(fn, dim3(grid), dim3(base_threads(small ? 8 : 16)), smem, stream, args);
   if (err != cudaSuccess) return cuda_fail(err, "launching the tensor-core decode kernel");
   return PA_OK;
 }
