@@ -182,12 +182,13 @@ template <> __device__ __forceinline__ void tmem_load_digits<8, 3>(uint32_t col,
   for (int i = 0; i < 24; ++i) out[i] = __uint_as_float(r[i]);
 }
 
-// Maxima over the 32 lanes of N values held by every lane (N = 4 or 8) in N + 4 - log2(N)
-// shuffles instead of 5 N: each of the first log2(N) steps hands half of the values still
-// held to the partner lane and keeps the other half, the last steps reduce the one value
-// left.  Returns the maximum of value *idx (the same for the 32 / N lanes of a group).
-template <int N>
-__device__ __forceinline__ float warp_max_transposed(float* v, int lane, int* idx) {
+// Maxima (kMax) or sums over the 32 lanes of N values held by every lane (N = 4 or 8) in
+// N + 4 - log2(N) shuffles instead of 5 N: each of the first log2(N) steps hands half of the
+// values still held to the partner lane and keeps the other half, the last steps reduce the
+// one value left.  Returns the result for value *idx (the same for the 32 / N lanes of a
+// group; lane & (32 / N - 1) == 0 is one lane of each group).
+template <int N, bool kMax>
+__device__ __forceinline__ float warp_reduce_transposed(float* v, int lane, int* idx) {
   int first = 0;
 #pragma unroll
   for (int w = N, m = 16; w > 1; w >>= 1, m >>= 1) {
@@ -196,12 +197,16 @@ __device__ __forceinline__ float warp_max_transposed(float* v, int lane, int* id
     for (int j = 0; j < w / 2; ++j) {
       const float keep = up ? v[w / 2 + j] : v[j];
       const float send = up ? v[j] : v[w / 2 + j];
-      v[j] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, m));
+      const float got = __shfl_xor_sync(0xffffffffu, send, m);
+      v[j] = kMax ? fmaxf(keep, got) : keep + got;
     }
     if (up) first += w / 2;
   }
 #pragma unroll
-  for (int m = 16 / N; m >= 1; m >>= 1) v[0] = fmaxf(v[0], __shfl_xor_sync(0xffffffffu, v[0], m));
+  for (int m = 16 / N; m >= 1; m >>= 1) {
+    const float got = __shfl_xor_sync(0xffffffffu, v[0], m);
+    v[0] = kMax ? fmaxf(v[0], got) : v[0] + got;
+  }
   *idx = first;
   return v[0];
 }
@@ -546,28 +551,35 @@ decode_gqa_tc8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
           out[h] = fmaf(d[2 * HPW + h], 1.f / 256.f, fmaf(d[HPW + h], 1.f / 16.f, d[h]));
       }
     };
+    // Every softmax thread runs every iteration and every named barrier, also after a wait
+    // gave up (ok false: the thread then skips its waits, stores and arrivals), so no thread
+    // is ever left at a barrier.  The TMEM loads run in every lane either way (the warp stays
+    // converged for them; the allocation is held until the end, and values read after a
+    // failed wait are never written out).
+    bool ok = true;
     // Fold the value product of tile t into the running output (thread = head dim r).
-    auto accumulate = [&](int t, const float* alpha, float unit) -> bool {
-      if (!wait_or_abort(o_full0 + 8 * (t % 2), (t / 2) & 1, abort)) return false;
+    auto accumulate = [&](int t, const float* alpha, float unit) {
+      ok = ok && wait_or_abort(o_full0 + 8 * (t % 2), (t / 2) & 1, abort);
+      __syncwarp();
       tc_fence_after_sync();
       float o[HPW];
       combine(tmem + lane_addr + 2 * NC + (t % 2) * NC + dcol, o);
       tc_fence_before_sync();
 #pragma unroll
       for (int h = 0; h < HPW; ++h) acc[h] = fmaf(acc[h], alpha[h], o[h] * unit);
-      return true;
     };
     Cursor c = start;
     bool seg_from_start = (c.j == 0);
     bool pending = false;  // the value product of the previous tile is not folded in yet
     for (int i = 0; i < n; ++i) {
       const int b = i % 2, st = i % kStages;
-      if (!wait_or_abort(s_full0 + 8 * b, (i / 2) & 1, abort)) break;
+      ok = ok && wait_or_abort(s_full0 + 8 * b, (i / 2) & 1, abort);
+      __syncwarp();
       tc_fence_after_sync();
       float sc[HPW];
       combine(tmem + lane_addr + b * NC + dcol, sc);
       tc_fence_before_sync();
-      mbar_arrive(s_empty0 + 8 * b);
+      if (ok) mbar_arrive(s_empty0 + 8 * b);
 
       const int tok = (c.sp.first_t + c.j) * kTokens + r;
       const bool valid = tok >= c.sp.lo && tok < c.sp.ctx;
@@ -593,7 +605,7 @@ decode_gqa_tc8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
           mv[h] = sc[h];
         }
         int hm;
-        const float x = warp_max_transposed<HPW>(mv, lane, &hm);
+        const float x = warp_reduce_transposed<HPW, true>(mv, lane, &hm);
         if ((lane & (32 / HPW - 1)) == 0) sh.red[b][q4][h_base + hm] = x;
       }
       {
@@ -647,25 +659,26 @@ decode_gqa_tc8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
           for (int k = 0; k < 3; ++k) dw[k][i] = d[k][0] | (d[k][1] << 16);
         }
       }
-      if constexpr (HPW == 8) {  // the whole block: bytes 0..15 in one chunk, 16..23 in the other
+      if (!ok) {
+      } else if constexpr (HPW == 8) {  // the whole block: bytes 0..15 in one chunk, 16..23 in the other
         st_shared_v4(c0, dw[0][0], dw[0][1], dw[1][0], dw[1][1]);
         if constexpr (!kInt) st_shared_v4(c1, dw[2][0], dw[2][1], 0, 0);
-      } else {                   // heads h0 .. h0 + 3 of the block: 4 bytes per digit
+      } else {                          // heads h0 .. h0 + 3 of the block: 4 bytes per digit
         const uint32_t h0 = h_base & 7;
         asm volatile("st.shared.b32 [%0], %1;" ::"r"(c0 + h0), "r"(dw[0][0]) : "memory");
         asm volatile("st.shared.b32 [%0], %1;" ::"r"(c0 + 8 + h0), "r"(dw[1][0]) : "memory");
         if constexpr (!kInt) asm volatile("st.shared.b32 [%0], %1;" ::"r"(c1 + h0), "r"(dw[kDigits - 1][0]) : "memory");
       }
-      if (!kInt && !valid && hh == 0) {  // an unattended row may hold NaN codes: give the value MMA zeros
+      if (ok && !kInt && !valid && hh == 0) {  // an unattended row may hold NaN codes: give the value MMA zeros
         const uint32_t v0 = stage(st) + kOffV + r * 128;
 #pragma unroll
         for (int k = 0; k < 8; ++k) st_shared_v4(v0 + 16 * (k ^ (r & 7)), 0, 0, 0, 0);
       }
       fence_proxy_async_shared();
-      mbar_arrive(p_full0 + 8 * b);
+      if (ok) mbar_arrive(p_full0 + 8 * b);
 
       // Overlap: the value MMA of tile i runs while the previous tile is folded in.
-      if (pending && !accumulate(i - 1, alpha_prev, unit_prev)) break;
+      if (pending) accumulate(i - 1, alpha_prev, unit_prev);
       pending = false;
       const bool seg_last = (c.j == c.sp.nb - 1);
       if (!(seg_last || i == n - 1)) {
@@ -674,19 +687,17 @@ decode_gqa_tc8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
 #pragma unroll
         for (int h = 0; h < HPW; ++h) alpha_prev[h] = alpha[h];
       } else {
-        if (!accumulate(i, alpha, unit)) break;
+        accumulate(i, alpha, unit);
         // Softmax denominators: every thread holds the sums of its own token rows.
         float lt[HPW];
+        {
+          float ls[HPW];
 #pragma unroll
-        for (int h = 0; h < HPW; ++h) {
-          float x = l[h];
-#pragma unroll
-          for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-          lt[h] = x;
+          for (int h = 0; h < HPW; ++h) ls[h] = l[h];
+          int hl;
+          const float x = warp_reduce_transposed<HPW, false>(ls, lane, &hl);
+          if ((lane & (32 / HPW - 1)) == 0) sh.red_l[q4][h_base + hl] = x;
         }
-        if (lane == 0)
-#pragma unroll
-          for (int h = 0; h < HPW; ++h) sh.red_l[q4][h_base + h] = lt[h];
         named_barrier_sync(1, kSoftmax);
 #pragma unroll
         for (int h = 0; h < HPW; ++h) {
@@ -695,7 +706,8 @@ decode_gqa_tc8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         }
         named_barrier_sync(1, kSoftmax);  // sh.red_l is free again
         const int h0 = c.g * GQ + h_base;
-        if (seg_from_start && seg_last) {
+        if (!ok) {
+        } else if (seg_from_start && seg_last) {
           IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(c.s) * p.Hq + h0) * kDim + r;
 #pragma unroll
           for (int h = 0; h < HPW; ++h)
