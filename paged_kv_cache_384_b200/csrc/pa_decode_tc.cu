@@ -80,6 +80,7 @@ struct TcShared {
   int abort;
   float red[2][4][kHeadsN];                     // per-tile maxima across the softmax warps (by tile parity)
   float red_l[4][kHeadsN];                      // softmax denominators at segment ends
+  int stop[2];                                  // abort flag as seen before a tile's exchange barrier
 };
 
 __device__ __forceinline__ uint32_t bits16(__half x) { return __half_as_ushort(x); }
@@ -370,41 +371,50 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       acc[h] = 0.f;
       alpha_prev[h] = 1.f;
     }
+    // No softmax thread leaves the loop on its own: a wait that gives up only stops the
+    // thread's arrivals, and all of them leave together after a tile's exchange barrier once
+    // the abort flag, as one thread saw it before that barrier, is set.  So no thread is ever
+    // left at a named barrier.  (The TMEM loads run in every lane either way: the allocation
+    // is held until the end, and values read after a failed wait are never written out.)
     // Fold the value product of tile t into the running output (thread = head dim r).
-    auto accumulate = [&](int t, const float* alpha) -> bool {
-      if (!wait_or_abort(o_full0 + 8 * (t % 2), (t / 2) & 1, abort)) return false;
+    auto accumulate = [&](int t, const float* alpha) {
+      wait_or_abort(o_full0 + 8 * (t % 2), (t / 2) & 1, abort);
       tc_fence_after_sync();
       float o[HPW];
       tmem_load<HPW>(tmem + lane_addr + 2 * kHeadsN + (t % 2) * kHeadsN + h_base, o);
       tc_fence_before_sync();
 #pragma unroll
       for (int h = 0; h < HPW; ++h) acc[h] = acc[h] * alpha[h] + o[h];
-      return true;
     };
     Cursor c = start;
     bool seg_from_start = (c.j == 0);
     bool pending = false;  // the value product of the previous tile is not folded in yet
     for (int i = 0; i < n; ++i) {
       const int b = i % 2, st = i % kStages;
-      if (!wait_or_abort(s_full0 + 8 * b, (i / 2) & 1, abort)) break;
+      const bool got = wait_or_abort(s_full0 + 8 * b, (i / 2) & 1, abort);
       tc_fence_after_sync();
       float sc[HPW];
       tmem_load<HPW>(tmem + lane_addr + b * kHeadsN + h_base, sc);
       tc_fence_before_sync();
-      mbar_arrive(s_empty0 + 8 * b);
+      if (got) mbar_arrive(s_empty0 + 8 * b);
 
       const int tok = (c.sp.first_t + c.j) * kTokens + r;
       const bool valid = tok >= c.sp.lo && tok < c.sp.ctx;
       const float sfac = p.qscale;
+      {
+        float mv[HPW];
 #pragma unroll
-      for (int h = 0; h < HPW; ++h) {
-        sc[h] = (valid && h_base + h < GQ) ? sc[h] * sfac : -INFINITY;
-        float x = sc[h];
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
-        if (lane == 0) sh.red[b][q4][h_base + h] = x;
+        for (int h = 0; h < HPW; ++h) {
+          sc[h] = (valid && h_base + h < GQ) ? sc[h] * sfac : -INFINITY;
+          mv[h] = sc[h];
+        }
+        int hm;
+        const float x = warp_reduce_transposed<HPW, true>(mv, lane, &hm);
+        if ((lane & (32 / HPW - 1)) == 0) sh.red[b][q4][h_base + hm] = x;
       }
+      if (threadIdx.x == 64) sh.stop[b] = *abort;  // the first softmax thread
       named_barrier_sync(1, kSoftmax);
+      if (sh.stop[b]) break;  // every softmax thread, at the same tile
       float alpha[HPW];
       uint32_t w_hi[8], w_lo[8];
 #pragma unroll
@@ -414,9 +424,9 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         const int hg = h_base + h;
         const float t = fmaxf(fmaxf(sh.red[b][0][hg], sh.red[b][1][hg]), fmaxf(sh.red[b][2][hg], sh.red[b][3][hg]));
         const float m_new = fmaxf(m[h], t);
-        alpha[h] = exp2f(m[h] - m_new);
+        alpha[h] = ex2_ftz(m[h] - m_new);
         m[h] = m_new;
-        const float pr = sc[h] == -INFINITY ? 0.f : exp2f(sc[h] - m_new);
+        const float pr = sc[h] == -INFINITY ? 0.f : ex2_ftz(sc[h] - m_new);
         const IO hi = float_to<IO>(pr);
         w_hi[h / 2] |= bits16(hi) << (16 * (h & 1));
         if (kSplit) {
@@ -449,7 +459,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       mbar_arrive(p_full0 + 8 * b);
 
       // Overlap: the value MMA of tile i runs while the previous tile is folded in.
-      if (pending && !accumulate(i - 1, alpha_prev)) break;
+      if (pending) accumulate(i - 1, alpha_prev);
       pending = false;
       const bool seg_last = (c.j == c.sp.nb - 1);
       if (!(seg_last || i == n - 1)) {
@@ -457,7 +467,7 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
 #pragma unroll
         for (int h = 0; h < HPW; ++h) alpha_prev[h] = alpha[h];
       } else {
-        if (!accumulate(i, alpha)) break;
+        accumulate(i, alpha);
         // Softmax denominators: every thread holds the sums of its own token rows.
         float lt[HPW];
 #pragma unroll

@@ -87,6 +87,7 @@ struct Tc8Shared {
   int abort;
   float red[2][4][kHeadsN + 1];                  // per-tile maxima across the softmax warps (+ v_max)
   float red_l[4][kHeadsN];                       // softmax denominators at segment ends
+  int stop[2];                                   // abort flag as seen before a tile's exchange barrier
 };
 
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort) {
@@ -180,35 +181,6 @@ template <> __device__ __forceinline__ void tmem_load_digits<8, 3>(uint32_t col,
       : "memory");
 #pragma unroll
   for (int i = 0; i < 24; ++i) out[i] = __uint_as_float(r[i]);
-}
-
-// Maxima (kMax) or sums over the 32 lanes of N values held by every lane (N = 4 or 8) in
-// N + 4 - log2(N) shuffles instead of 5 N: each of the first log2(N) steps hands half of the
-// values still held to the partner lane and keeps the other half, the last steps reduce the
-// one value left.  Returns the result for value *idx (the same for the 32 / N lanes of a
-// group; lane & (32 / N - 1) == 0 is one lane of each group).
-template <int N, bool kMax>
-__device__ __forceinline__ float warp_reduce_transposed(float* v, int lane, int* idx) {
-  int first = 0;
-#pragma unroll
-  for (int w = N, m = 16; w > 1; w >>= 1, m >>= 1) {
-    const bool up = (lane & m) != 0;
-#pragma unroll
-    for (int j = 0; j < w / 2; ++j) {
-      const float keep = up ? v[w / 2 + j] : v[j];
-      const float send = up ? v[j] : v[w / 2 + j];
-      const float got = __shfl_xor_sync(0xffffffffu, send, m);
-      v[j] = kMax ? fmaxf(keep, got) : keep + got;
-    }
-    if (up) first += w / 2;
-  }
-#pragma unroll
-  for (int m = 16 / N; m >= 1; m >>= 1) {
-    const float got = __shfl_xor_sync(0xffffffffu, v[0], m);
-    v[0] = kMax ? fmaxf(v[0], got) : v[0] + got;
-  }
-  *idx = first;
-  return v[0];
 }
 
 // IO: fp16 or bf16 queries and output; CT: int8_t or __nv_fp8_e4m3 codes; NH: query heads of
@@ -551,16 +523,14 @@ decode_gqa_tc8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
           out[h] = fmaf(d[2 * HPW + h], 1.f / 256.f, fmaf(d[HPW + h], 1.f / 16.f, d[h]));
       }
     };
-    // Every softmax thread runs every iteration and every named barrier, also after a wait
-    // gave up (ok false: the thread then skips its waits, stores and arrivals), so no thread
-    // is ever left at a barrier.  The TMEM loads run in every lane either way (the warp stays
-    // converged for them; the allocation is held until the end, and values read after a
-    // failed wait are never written out).
-    bool ok = true;
+    // No softmax thread leaves the loop on its own: a wait that gives up only stops the
+    // thread's arrivals, and all of them leave together after a tile's exchange barrier once
+    // the abort flag, as one thread saw it before that barrier, is set.  So no thread is ever
+    // left at a named barrier.  (The TMEM loads run in every lane either way: the allocation
+    // is held until the end, and values read after a failed wait are never written out.)
     // Fold the value product of tile t into the running output (thread = head dim r).
     auto accumulate = [&](int t, const float* alpha, float unit) {
-      ok = ok && wait_or_abort(o_full0 + 8 * (t % 2), (t / 2) & 1, abort);
-      __syncwarp();
+      wait_or_abort(o_full0 + 8 * (t % 2), (t / 2) & 1, abort);
       tc_fence_after_sync();
       float o[HPW];
       combine(tmem + lane_addr + 2 * NC + (t % 2) * NC + dcol, o);
@@ -573,13 +543,12 @@ decode_gqa_tc8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     bool pending = false;  // the value product of the previous tile is not folded in yet
     for (int i = 0; i < n; ++i) {
       const int b = i % 2, st = i % kStages;
-      ok = ok && wait_or_abort(s_full0 + 8 * b, (i / 2) & 1, abort);
-      __syncwarp();
+      const bool got = wait_or_abort(s_full0 + 8 * b, (i / 2) & 1, abort);
       tc_fence_after_sync();
       float sc[HPW];
       combine(tmem + lane_addr + b * NC + dcol, sc);
       tc_fence_before_sync();
-      if (ok) mbar_arrive(s_empty0 + 8 * b);
+      if (got) mbar_arrive(s_empty0 + 8 * b);
 
       const int tok = (c.sp.first_t + c.j) * kTokens + r;
       const bool valid = tok >= c.sp.lo && tok < c.sp.ctx;
@@ -614,7 +583,9 @@ decode_gqa_tc8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         for (int off = 16; off >= 1; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
         if (lane == 0 && hh == 0) sh.red[b][q4][kHeadsN] = x;
       }
+      if (threadIdx.x == 64) sh.stop[b] = *abort;  // the first softmax thread
       named_barrier_sync(1, kSoftmax);
+      if (sh.stop[b]) break;  // every softmax thread, at the same tile
       const float vmax = fmaxf(fmaxf(sh.red[b][0][kHeadsN], sh.red[b][1][kHeadsN]),
                                fmaxf(sh.red[b][2][kHeadsN], sh.red[b][3][kHeadsN]));
       const float vrel = vmax > 0.f ? vscale / vmax : 0.f;  // in [0, 1]
@@ -659,8 +630,7 @@ decode_gqa_tc8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
           for (int k = 0; k < 3; ++k) dw[k][i] = d[k][0] | (d[k][1] << 16);
         }
       }
-      if (!ok) {
-      } else if constexpr (HPW == 8) {  // the whole block: bytes 0..15 in one chunk, 16..23 in the other
+      if constexpr (HPW == 8) {  // the whole block: bytes 0..15 in one chunk, 16..23 in the other
         st_shared_v4(c0, dw[0][0], dw[0][1], dw[1][0], dw[1][1]);
         if constexpr (!kInt) st_shared_v4(c1, dw[2][0], dw[2][1], 0, 0);
       } else {                          // heads h0 .. h0 + 3 of the block: 4 bytes per digit
@@ -669,13 +639,13 @@ decode_gqa_tc8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         asm volatile("st.shared.b32 [%0], %1;" ::"r"(c0 + 8 + h0), "r"(dw[1][0]) : "memory");
         if constexpr (!kInt) asm volatile("st.shared.b32 [%0], %1;" ::"r"(c1 + h0), "r"(dw[kDigits - 1][0]) : "memory");
       }
-      if (ok && !kInt && !valid && hh == 0) {  // an unattended row may hold NaN codes: give the value MMA zeros
+      if (!kInt && !valid && hh == 0) {  // an unattended row may hold NaN codes: give the value MMA zeros
         const uint32_t v0 = stage(st) + kOffV + r * 128;
 #pragma unroll
         for (int k = 0; k < 8; ++k) st_shared_v4(v0 + 16 * (k ^ (r & 7)), 0, 0, 0, 0);
       }
       fence_proxy_async_shared();
-      if (ok) mbar_arrive(p_full0 + 8 * b);
+      mbar_arrive(p_full0 + 8 * b);
 
       // Overlap: the value MMA of tile i runs while the previous tile is folded in.
       if (pending) accumulate(i - 1, alpha_prev, unit_prev);
@@ -706,8 +676,7 @@ decode_gqa_tc8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         }
         named_barrier_sync(1, kSoftmax);  // sh.red_l is free again
         const int h0 = c.g * GQ + h_base;
-        if (!ok) {
-        } else if (seg_from_start && seg_last) {
+        if (seg_from_start && seg_last) {
           IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(c.s) * p.Hq + h0) * kDim + r;
 #pragma unroll
           for (int h = 0; h < HPW; ++h)

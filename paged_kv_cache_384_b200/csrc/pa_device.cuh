@@ -548,6 +548,35 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t c) {
   return h;
 }
 
+// Maxima (kMax) or sums over the 32 lanes of N values held by every lane (N = 4 or 8) in
+// N + 4 - log2(N) shuffles instead of 5 N: each of the first log2(N) steps hands half of the
+// values still held to the partner lane and keeps the other half, the last steps reduce the
+// one value left.  Returns the result for value *idx (the same for the 32 / N lanes of a
+// group; lane & (32 / N - 1) == 0 is one lane of each group).
+template <int N, bool kMax>
+__device__ __forceinline__ float warp_reduce_transposed(float* v, int lane, int* idx) {
+  int first = 0;
+#pragma unroll
+  for (int w = N, m = 16; w > 1; w >>= 1, m >>= 1) {
+    const bool up = (lane & m) != 0;
+#pragma unroll
+    for (int j = 0; j < w / 2; ++j) {
+      const float keep = up ? v[w / 2 + j] : v[j];
+      const float send = up ? v[j] : v[w / 2 + j];
+      const float got = __shfl_xor_sync(0xffffffffu, send, m);
+      v[j] = kMax ? fmaxf(keep, got) : keep + got;
+    }
+    if (up) first += w / 2;
+  }
+#pragma unroll
+  for (int m = 16 / N; m >= 1; m >>= 1) {
+    const float got = __shfl_xor_sync(0xffffffffu, v[0], m);
+    v[0] = kMax ? fmaxf(v[0], got) : v[0] + got;
+  }
+  *idx = first;
+  return v[0];
+}
+
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
