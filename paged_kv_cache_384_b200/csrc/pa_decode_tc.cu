@@ -18,20 +18,20 @@
 // "vLLM source first look: PagedAttention memory design" (trdm.cn), section 三); the
 // grouped-query tile is this library's design.
 //
-// Roles (one CTA per SM, 10 warps):
+// Roles (one CTA per SM, 14 warps):
 //   warps 0,6-8 TMA producers, one per part of a tile (K or V, 64-dim half, 128-byte
 //               swizzle): each issues its part of every attended block into a 3-stage ring
 //               (warp 0 also the q rows of the head group); block-table entries are loaded
 //               by the lanes in parallel.
 //   warp 1      TMEM owner and MMA issuer (one lane); with up to 8 query heads per cached
 //               head warp 9 issues the value MMAs and warp 1 only the score MMAs.
-//   warps 2..5  softmax (thread = token row of S^T) and accumulation (thread = head dim row
-//               of O^T): online softmax in base 2, probabilities written as the B operand of
-//               the value MMA, V rows of unattended tokens zeroed, running output rescaled
-//               in registers.  Segment ends write the output or a partial (m, l, acc)
-//               exactly like the CUDA-core kernel, so the same merge kernel finishes split
-//               segments.  (warps 10..13 too with 16 query heads per row: two warps per TMEM
-//               lane quarter, 8 heads each.)
+//   warps 2..5, 10..13  softmax (thread = token row of S^T) and accumulation (thread = head
+//               dim row of O^T), two warps per TMEM lane quarter, each with half of the
+//               row's query heads: online softmax in base 2, probabilities written as the B
+//               operand of the value MMA, V rows of unattended tokens zeroed, running output
+//               rescaled in registers.  Segment ends write the output or a partial (m, l,
+//               acc) exactly like the CUDA-core kernel, so the same merge kernel finishes
+//               split segments.
 // 8-bit caches run on the kernel of pa_decode_tc8.cu, which feeds the codes to the tensor
 // cores as they are.
 // Every wait is bounded; a wait that gives up sets an abort flag that ends all the others.
@@ -60,7 +60,7 @@ constexpr int kPBytes = kTokens * kHeadsN * 2;  // one probability operand, 128 
 // Threads of the kernel tracking NH query heads per row: TMA warps 0 and 6..8, MMA warps
 // 1 and 9, softmax warps 2..5 (and 10..13 when NH = 16: two warps per TMEM lane quarter,
 // 8 heads each).
-constexpr int base_threads(int nh) { return nh > 8 ? 448 : 320; }
+constexpr int base_threads(int) { return 448; }
 static_assert(base_threads(16) <= kMaxPlanThreads, "plan_slice keeps one scratch entry per thread");
 constexpr uint32_t kTmemCols = 64;              // S0 [0,16)  S1 [16,32)  O0 [32,48)  O1 [48,64)
 // Probability operands: 2 tiles in flight x (hi, lo) parts for a bf16 cache, x 1 part otherwise.
@@ -96,15 +96,13 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
   return false;
 }
 
-// Row r of a probability operand P^T (MN-major, 32-byte swizzle): 16 heads = 32 B, the two
+// Rows of a probability operand P^T (MN-major, 32-byte swizzle): 16 heads = 32 B, the two
 // 16-byte chunks trade places on rows 4..7 of every 8.
-__device__ __forceinline__ void store_p_row(uint32_t buf, int r, const uint32_t* w) {
-  const uint32_t row = buf + r * 32;
+// Heads 4 * hh .. 4 * hh + 3 of row r only (8 bytes of the first 16-byte chunk).
+__device__ __forceinline__ void store_p_quarter_row(uint32_t buf, int r, int hh, const uint32_t* w) {
   const uint32_t sw = (r >> 2) & 1;
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + 16 * sw), "r"(w[0]), "r"(w[1]), "r"(w[2]),
-               "r"(w[3]) : "memory");
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + 16 * (sw ^ 1)), "r"(w[4]), "r"(w[5]), "r"(w[6]),
-               "r"(w[7]) : "memory");
+  asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(buf + r * 32 + 16 * sw + 8 * hh), "r"(w[0]), "r"(w[1])
+               : "memory");
 }
 // Heads 8 * hh .. 8 * hh + 7 of row r only (the other 16-byte chunk belongs to another warp).
 __device__ __forceinline__ void store_p_half_row(uint32_t buf, int r, int hh, const uint32_t* w) {
@@ -114,7 +112,7 @@ __device__ __forceinline__ void store_p_half_row(uint32_t buf, int r, int hh, co
 }
 
 // IO: fp16 or bf16 queries and cache.  NH: query heads of a row (8 or 16 >= GQ); a softmax
-// thread tracks 8 of them.  bf16 probabilities are split into hi + lo bf16 parts and the
+// thread tracks NH / 2 of them.  bf16 probabilities are split into hi + lo bf16 parts and the
 // value MMA runs on both, so the weights keep ~16 significant bits (one bf16 part alone
 // keeps 8).
 template <typename IO, int NH>
@@ -161,13 +159,19 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full0 + 8 * b, 1);
-      mbar_init(s_empty0 + 8 * b, 128 * (NH / 8));
-      mbar_init(p_full0 + 8 * b, 128 * (NH / 8));
+      mbar_init(s_empty0 + 8 * b, 256);  // every softmax thread
+      mbar_init(p_full0 + 8 * b, 256);
       mbar_init(o_full0 + 8 * b, 1);
     }
     mbar_init(smem_u32(&sh.mma_done), 2);
     sh.abort = 0;
     fence_barrier_init();
+  }
+  // The probability operands start as zeros (they held the plan scratch): with up to 8 query
+  // heads per row the padding heads 8..15 are never written again.
+  for (int i = threadIdx.x; i < 2 * kParts * kPBytes / 16; i += blockDim.x) {
+    uint8_t* ptr = smem_raw + (pbase - smem_u32(smem_raw)) + 16 * i;
+    *reinterpret_cast<uint4*>(ptr) = make_uint4(0, 0, 0, 0);
   }
   // The q rows of a head group fill rows 0..GQ-1 of each stage's 16-row q block; rows
   // GQ..15 stay zero (padding of the MMA N dimension).
@@ -355,12 +359,12 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     __syncwarp();
   } else {
     // ------------------------------------------------- softmax + accumulation warps --
-    // (warps 2..5, and 10..13 for the heads 8..15 of a 16-head row)
-    constexpr int HPW = 8;                // query heads a thread tracks
-    constexpr int kSoftmax = 128 * (NH / 8);
+    // Warps 2..5 and 10..13: two per TMEM lane quarter, each with half of the row's heads.
+    constexpr int HPW = NH / 2;           // query heads a thread tracks
+    constexpr int kSoftmax = 256;
     const int q4 = warp & 3;              // TMEM lane quarter this warp may access
-    const int hh = warp >= 10 ? 1 : 0;    // which 8 of the row's heads
-    const int h_base = 8 * hh;
+    const int hh = warp >= 10 ? 1 : 0;    // which half of the row's heads
+    const int h_base = HPW * hh;
     const int r = 32 * q4 + lane;         // token row (softmax) and head-dim row (accumulate)
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q4) << 16;
     float m[HPW], l[HPW], acc[HPW], alpha_prev[HPW];
@@ -440,9 +444,9 @@ decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       if (NH > 8) {  // this warp's 16-byte chunk of the 32-byte row
         store_p_half_row(pbuf(b, 0), r, hh, w_hi);
         if (kSplit) store_p_half_row(pbuf(b, 1), r, hh, w_lo);
-      } else {       // heads 8..15 of the padded row are zero
-        store_p_row(pbuf(b, 0), r, w_hi);
-        if (kSplit) store_p_row(pbuf(b, 1), r, w_lo);
+      } else {       // heads 4 hh .. 4 hh + 3: 8 bytes of the first chunk (heads 8..15 stay zero)
+        store_p_quarter_row(pbuf(b, 0), r, hh, w_hi);
+        if (kSplit) store_p_quarter_row(pbuf(b, 1), r, hh, w_lo);
       }
       if (!valid && hh == 0) {  // unattended rows may hold anything (NaN): give the value MMA zeros
         // Chunk k ^ (r & 7) at step k: neighbouring rows (128 B apart, the same banks)

@@ -407,7 +407,21 @@ __device__ __forceinline__ void tmem_load16(uint32_t taddr, float* v) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 4 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_load4(uint32_t taddr, float* v) {
+  uint32_t r[4];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 template <int N> __device__ __forceinline__ void tmem_load(uint32_t taddr, float* v);
+template <> __device__ __forceinline__ void tmem_load<4>(uint32_t taddr, float* v) { tmem_load4(taddr, v); }
 template <> __device__ __forceinline__ void tmem_load<8>(uint32_t taddr, float* v) { tmem_load8(taddr, v); }
 template <> __device__ __forceinline__ void tmem_load<16>(uint32_t taddr, float* v) { tmem_load16(taddr, v); }
 
