@@ -430,9 +430,11 @@ __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const De
   const long long item = static_cast<long long>(blockIdx.x) * kMergeWarps + (threadIdx.x >> 5);
   if (item >= static_cast<long long>(p.S) * p.Hq) return;
   const int s = static_cast<int>(item / p.Hq), h = static_cast<int>(item % p.Hq);
+  // The plan's unit stream (tiles plus seg_units per segment; see plan_slice).
   const long long per_group = p.ws_prefix[p.S];
   const long long pre = p.ws_prefix[s];
-  const long long nb = p.ws_prefix[s + 1] - pre;
+  const long long su = p.ws_prefix[s + 1] - pre;  // units of one head group of this sequence
+  const long long nb = su > 0 ? su - p.seg_units : 0;
   IO* orow = reinterpret_cast<IO*>(p.out) + (static_cast<size_t>(s) * p.Hq + h) * D + lane * DL;
   float o[DL];
 #pragma unroll
@@ -442,10 +444,10 @@ __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const De
     for (int e = 0; e < DL; ++e) orow[e] = float_to<IO>(0.f);
     return;
   }
-  const long long T = per_group * p.G;
+  const long long U = per_group * p.G;
   const int g = h / p.QW, w = h % p.QW;
-  const long long a = p.G * pre + g * nb;
-  const int c0 = cta_of(a, T, p.num_ctas), c1 = cta_of(a + nb - 1, T, p.num_ctas);
+  const long long a = p.G * pre + g * su + p.seg_units;  // unit of the segment's first tile
+  const int c0 = cta_of(a, U, p.num_ctas), c1 = cta_of(a + nb - 1, U, p.num_ctas);
   if (c0 == c1) return;
   const long long seg = static_cast<long long>(s) * p.G + g;
   const float2* ml = reinterpret_cast<const float2*>(p.ws_ml);
@@ -700,6 +702,10 @@ pa_status decode_launch_tc(void* out, const void* q, const void* k_cache, const 
   prm.QW = GQ;
   prm.sub = NSUB;
   prm.dim = head_dim;
+  // A segment's end (denominators, output or partial written, the pipeline refilled) costs
+  // about one tile on the tensor-core kernels: CTAs whose shares hold many short segments
+  // finished last when the stream was split by tiles alone.
+  prm.seg_units = 1;
   prm.qscale = scale * 1.4426950408889634f;
 
   cudaEvent_t ev[3];

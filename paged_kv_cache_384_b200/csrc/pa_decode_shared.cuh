@@ -35,6 +35,8 @@ struct DecodeParams {
   int sub;               // tensor-core kernel: head groups per cached head (1, or query sub-groups of
                          // one cached head when it has more than 16 query heads)
   int dim;               // head_dim (the tensor-core kernel takes 64 or 128 at run time)
+  int seg_units;         // cost of a segment's end, in tiles: the stream is split into equal
+                         // shares of (tiles + seg_units per segment) among the CTAs
   float qscale;          // softmax scale * log2(e): scores are kept in base 2
   uint32_t stage_bytes;  // bytes per pipeline stage
   uint32_t v_off, ks_off, vs_off;  // offsets of the V tile and the INT8 scale tiles in a stage
@@ -118,88 +120,122 @@ __device__ __forceinline__ void store_floats(IO* dst, const float* src) {
 }
 
 
-// Device-side plan shared by the partition kernels: count every sequence's tiles, prefix-sum
-// them over the CTA (CTA 0 also publishes the prefix for the merge kernel), and locate this
-// CTA's slice [t0, t0 + count) of the (sequence, head group, tile) stream.  Every thread of
-// the CTA must call it.  Returns count (0: nothing to do, or an impossible plan reported as
-// PA_DEVERR_TIMEOUT); *start is the cursor of tile t0.
+// Device-side plan shared by the partition kernels.  The (sequence, head group, tile) stream
+// is split into equal shares of cost units: each tile is one unit and each segment (one
+// head group of one sequence) adds p.seg_units more before its first tile (the work at a
+// segment's end, which made CTAs with many short segments finish last).  Tile j of segment
+// (s, g) sits at unit G * U(s) + g * (nb + w) + w + j, where U(s) counts the units of the
+// sequences before s for one head group and w = p.seg_units; CTA c takes the tiles whose
+// units fall in its share.  Every thread of the CTA must call plan_slice: it counts every
+// sequence's tiles, prefix-sums the units over the CTA (CTA 0 also publishes U for the
+// merge kernel) and locates this CTA's first and one-past-last tile.  Returns the number of
+// tiles (0: nothing to do, or an impossible plan reported as PA_DEVERR_TIMEOUT); *start is
+// the cursor of the first.
 struct PlanScratch {
-  long long warp_sum[kMaxPlanThreads / 32];  // tiles counted by each warp, then their exclusive prefix
-  long long total;
-  long long first_prefix;
-  int first_seq;
+  long long warp_sum[kMaxPlanThreads / 32][2];  // units and tiles of each warp, then their exclusive prefixes
+  long long total_units, total_tiles;
+  long long tile_at[2];                         // stream index of the first tile at or after u0, u1
+  int first_seq, first_g, first_j;
 };
+
+// Units of one head group's segment of a sequence with nb tiles.
+__device__ __forceinline__ long long seg_units_of(int nb, int w) { return nb > 0 ? nb + w : 0; }
+
+// Units -> CTA (the inverse of the equal split of the units).
+__device__ __forceinline__ int cta_of_unit(long long u, long long U, int C) { return cta_of(u, U, C); }
 
 __device__ __forceinline__ long long plan_slice(const DecodeParams& p, PlanScratch& sc, long long* t0_out,
                                                 Cursor* start) {
-  const int nthr = blockDim.x;
-  const int G = p.G;
+  const int nthr = blockDim.x;  // a multiple of 32
+  const int G = p.G, w = p.seg_units;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nwarps = (nthr + 31) >> 5;
   const int chunk = (p.S + nthr - 1) / nthr;
   const int s_lo = min(p.S, static_cast<int>(threadIdx.x) * chunk), s_hi = min(p.S, s_lo + chunk);
-  long long mine = 0;
-  for (int s = s_lo; s < s_hi; ++s) mine += seq_span(p, s, blockIdx.x == 0).nb;
-  // Exclusive prefix over the threads: a shuffle scan inside each warp, then over the warps'
+  long long mine_t = 0, mine_u = 0;
+  for (int s = s_lo; s < s_hi; ++s) {
+    const int nb = seq_span(p, s, blockIdx.x == 0).nb;
+    mine_t += nb;
+    mine_u += seg_units_of(nb, w);
+  }
+  // Exclusive prefixes over the threads: shuffle scans inside each warp, then over the warps'
   // totals (a thread-serial scan measured ~6 us at 448 threads).
-  long long incl = mine;
+  long long inc_t = mine_t, inc_u = mine_u;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
-    const long long y = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += y;
+    const long long yt = __shfl_up_sync(0xffffffffu, inc_t, off);
+    const long long yu = __shfl_up_sync(0xffffffffu, inc_u, off);
+    if (lane >= off) inc_t += yt, inc_u += yu;
   }
-  if (lane == 31) sc.warp_sum[wid] = incl;
+  if (lane == 31) sc.warp_sum[wid][0] = inc_u, sc.warp_sum[wid][1] = inc_t;
   if (threadIdx.x == 0) sc.first_seq = -1;
   __syncthreads();
   if (wid == 0) {
-    const long long v = lane < nwarps ? sc.warp_sum[lane] : 0;
-    long long w = v;
+    const long long vu = lane < nwarps ? sc.warp_sum[lane][0] : 0, vt = lane < nwarps ? sc.warp_sum[lane][1] : 0;
+    long long au = vu, at = vt;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-      const long long y = __shfl_up_sync(0xffffffffu, w, off);
-      if (lane >= off) w += y;
+      const long long yu = __shfl_up_sync(0xffffffffu, au, off);
+      const long long yt = __shfl_up_sync(0xffffffffu, at, off);
+      if (lane >= off) au += yu, at += yt;
     }
-    if (lane < nwarps) sc.warp_sum[lane] = w - v;
-    if (lane == 31) sc.total = w;
+    if (lane < nwarps) sc.warp_sum[lane][0] = au - vu, sc.warp_sum[lane][1] = at - vt;
+    if (lane == 31) sc.total_units = au, sc.total_tiles = at;
   }
   __syncthreads();
-  const long long per_group = sc.total;  // tiles of one head group over all sequences
-  const long long T = per_group * G;
-  const long long my_prefix = sc.warp_sum[wid] + incl - mine;
-  if (blockIdx.x == 0) {  // publish the per-sequence prefix for the merge kernel
-    long long r = my_prefix;
+  const long long per_group = sc.total_units;  // units of one head group over all sequences
+  const long long U = per_group * G, T = sc.total_tiles * G;
+  const long long pre_u = sc.warp_sum[wid][0] + inc_u - mine_u, pre_t = sc.warp_sum[wid][1] + inc_t - mine_t;
+  if (blockIdx.x == 0) {  // publish the per-sequence unit prefix for the merge kernel
+    long long r = pre_u;
     for (int s = s_lo; s < s_hi; ++s) {
       p.ws_prefix[s] = r;
-      r += seq_span(p, s, false).nb;
+      r += seg_units_of(seq_span(p, s, false).nb, w);
     }
     if (threadIdx.x == 0) p.ws_prefix[p.S] = per_group;
   }
-  long long t0, count;
-  cta_slice(T, p.num_ctas, blockIdx.x, &t0, &count);
-  if (count == 0) return 0;  // uniform across the CTA
-  // Sequence holding t0: sequence s starts at tile G * prefix(s).
-  if (t0 >= G * my_prefix && t0 < G * (my_prefix + mine)) {
-    long long r = my_prefix;
-    for (int s = s_lo; s < s_hi; ++s) {
-      const int nb = seq_span(p, s, false).nb;
-      if (t0 < G * (r + nb)) {
-        sc.first_seq = s;
-        sc.first_prefix = r;
-        break;
+  long long u0, ucount;
+  cta_slice(U, p.num_ctas, blockIdx.x, &u0, &ucount);
+  if (ucount == 0) return 0;  // uniform across the CTA
+  // The first tile at or after unit u0 and after u0 + ucount: located by the thread whose
+  // sequences hold that unit (an end at U has no owner: T).
+  if (threadIdx.x == 0 && u0 + ucount >= U) sc.tile_at[1] = T;
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const long long u = e == 0 ? u0 : u0 + ucount;
+    if (u < U && u >= G * pre_u && u < G * (pre_u + mine_u)) {
+      long long ru = pre_u, rt = pre_t;
+      for (int s = s_lo; s < s_hi; ++s) {
+        const int nb = seq_span(p, s, false).nb;
+        const long long su = seg_units_of(nb, w);
+        if (u < G * (ru + su)) {
+          const long long rem = u - G * ru;
+          const int g = static_cast<int>(rem / su);
+          const int j = static_cast<int>(max(0ll, rem % su - w));
+          sc.tile_at[e] = G * rt + static_cast<long long>(g) * nb + j;
+          if (e == 0) {
+            sc.first_seq = s;
+            sc.first_g = g;
+            sc.first_j = j;
+          }
+          break;
+        }
+        ru += su;
+        rt += nb;
       }
-      r += nb;
     }
   }
   __syncthreads();
-  if (sc.first_seq < 0) {  // cannot happen when count > 0; never index with it
+  if (sc.first_seq < 0) {  // cannot happen when ucount > 0; never index with it
     if (threadIdx.x == 0) decode_error(PA_DEVERR_TIMEOUT);
     return 0;
   }
+  const long long count = sc.tile_at[1] - sc.tile_at[0];
+  if (count <= 0) return 0;  // a share of segment-end units only
   start->s = sc.first_seq;
   start->sp = seq_span(p, start->s, false);
-  const long long rem = t0 - G * sc.first_prefix;
-  start->g = static_cast<int>(rem / start->sp.nb);
-  start->j = static_cast<int>(rem % start->sp.nb);
-  *t0_out = t0;
+  start->g = sc.first_g;
+  start->j = sc.first_j;
+  *t0_out = sc.tile_at[0];
   return count;
 }
 
