@@ -842,7 +842,7 @@ pa_status decode_launch(void* out, const void* q, const void* k_cache, const voi
     tmVs = tmV;
   }
 
-  DecodeParams prm;
+  DecodeParams prm = {};
   prm.out = out;
   prm.q = q;
   prm.block_tables = block_tables;
@@ -865,6 +865,7 @@ pa_status decode_launch(void* out, const void* q, const void* k_cache, const voi
   prm.G = G;
   prm.sub = 1;
   prm.dim = head_dim;
+  prm.seg_units = 0;  // the stream is split by tiles alone
   prm.num_ctas = C;
   prm.nstage = nstage;
   prm.qscale = scale * 1.4426950408889634f;  // log2(e): exp(x) = 2^(x log2 e)
