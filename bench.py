@@ -107,6 +107,22 @@ def measured_tensor_peak():
         return FALLBACK_BF16_TFLOPS, "fallback (cuBLAS bf16 burst measured earlier on this GPU type)"
 
 
+def source_digest(kernel_source: str) -> str:
+    """SHA-256 over a kernel's source file followed by the device headers beside it that the
+    kernels include (pa_device.cuh, pa_decode_shared.cuh), so a record goes stale when any of
+    them changes."""
+    h = hashlib.sha256()
+    with open(kernel_source, "rb") as f:
+        h.update(f.read())
+    here = os.path.dirname(kernel_source)
+    for name in ("pa_device.cuh", "pa_decode_shared.cuh"):
+        path = os.path.join(here, name)
+        if os.path.exists(path):
+            with open(path, "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()
+
+
 def kernel_traffic(kernel_source: str, record: str = "decode_partition_traffic.json", workload: str = None):
     """ncu DRAM bytes per launch of a kernel, if captured for this exact source and workload."""
     path = os.path.join(ROOT, "profiles", record)
@@ -115,8 +131,7 @@ def kernel_traffic(kernel_source: str, record: str = "decode_partition_traffic.j
             rec = json.load(f)
     except (OSError, ValueError):
         return None
-    with open(kernel_source, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()
+    sha = source_digest(kernel_source)
     if rec.get("source_sha256") != sha or rec.get("workload") != (PRESET if workload is None else workload):
         return None
     return rec.get("dram_bytes_per_launch")
@@ -436,7 +451,9 @@ def decode_kernel_ms(pa, w, d, stream, steps):
 
 
 def decode_kernel_name(w) -> str:
-    return "decode_gqa_tc_kernel" if w.num_kv_heads * 4 <= w.num_heads else "decode_partition_kernel"
+    if w.num_kv_heads * 4 > w.num_heads:
+        return "decode_partition_kernel"
+    return "decode_gqa_tc8_kernel" if w.cache_dtype in ("int8", "fp8") else "decode_gqa_tc_kernel"
 
 
 # The other decode workloads of the method, measured after the metric's own workload in a
