@@ -8,7 +8,7 @@ import os
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-RECORDS = ["decode_partition_traffic.json", "prefill_tc_traffic.json"]
+RECORDS = ["decode_partition_traffic.json", "decode_partition_traffic_chat_prefix_bf16.json", "prefill_tc_traffic.json"]
 
 
 def load_bench():
