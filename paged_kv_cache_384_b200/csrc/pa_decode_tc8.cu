@@ -267,7 +267,9 @@ decode_gqa_tc8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     // ------------------------------------------------------------------ TMA producers --
     const int part = warp == 0 ? 0 : warp - 5;  // 0: K codes, 1: V codes, 2: K scales, 3: V scales
     const CUtensorMap* map = part == 0 ? &tmK : part == 1 ? &tmV : part == 2 ? &tmKs : &tmVs;
-    const uint64_t policy = l2_policy_evict_first();
+    // Codes are read once (evict first); a scale row holds 8 cached heads and serves the
+    // tiles of all 8, which follow one another in the stream (evict last).
+    const uint64_t policy = part < 2 ? l2_policy_evict_first() : l2_policy_evict_last();
     if (lane == 0) prefetch_tensormap(map);
     const int bs = p.bs;
     const int bpt = kTokens / bs;  // blocks per tile
