@@ -529,7 +529,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
             if (mbar_test_wait(p_full0 + 8 * b, (t / 2) & 1) && mbar_test_wait(v_ready0 + 8 * st, (t / kRing) & 1) &&
                 (P.idx > 0 || P.uq == 0 || mbar_test_wait(o_free, (P.uq - 1) & 1))) {
               tc_fence_after_sync();
-  #pragma unroll
               const uint32_t idesc_o = nhalf == 2 ? kIdescO : kIdescO64;
   #pragma unroll
               for (int part = 0; part < (kSplit ? 2 : 1); ++part) {
