@@ -623,8 +623,9 @@ namespace {
 
 bool g_tensor_cores = true;  // pa_decode_use_tensor_cores()
 
-// Grouped-query decode on the tensor cores: one CTA per SM, 128-token tiles of one cached
-// head (pa_decode_tc.cu), then the shared merge kernel.
+// Grouped-query decode on the tensor cores: one CTA per SM (two for 8-bit caches with up to
+// 8 query heads per cached head), 128-token tiles of one cached head (pa_decode_tc.cu,
+// pa_decode_tc8.cu), then the shared merge kernel.
 pa_status decode_launch_tc(void* out, const void* q, const void* k_cache, const void* v_cache, const void* k_scale,
                            const void* v_scale, const int32_t* block_tables, const int32_t* context_lens,
                            int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
@@ -633,7 +634,8 @@ pa_status decode_launch_tc(void* out, const void* q, const void* k_cache, const 
   const int SG = tc_decode_subgroup(num_q_heads / num_kv_heads);  // query heads per head group
   const int NSUB = num_q_heads / num_kv_heads / SG;               // head groups per cached head
   const int GQ = SG;
-  const int C = sms;
+  const bool eight_bit = cache_dtype != io_dtype;  // INT8 or FP8 codes with per-token scales
+  const int C = sms * (eight_bit ? tc8_ctas_per_sm(GQ) : 1);
   const long long rows = static_cast<long long>(C) * GQ + static_cast<long long>(num_seqs) * num_q_heads;
   const WsLayout lay = ws_layout(num_seqs, head_dim, rows);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -641,7 +643,6 @@ pa_status decode_launch_tc(void* out, const void* q, const void* k_cache, const 
   pa_status st = get_encoder(&enc);
   if (st != PA_OK) return st;
   const CUtensorMapDataType ttype = io_dtype == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const bool eight_bit = cache_dtype != io_dtype;
   CUtensorMap tmK, tmV, tmQ, tmKs, tmVs;
   if (!eight_bit) {
     // [NB*bs rows][Hkv][head_dim]: boxes of one block's rows x one head x 64 dims, 128-byte swizzle

@@ -256,4 +256,6 @@ pa_status tc_decode_launch(const CUtensorMap& tmK, const CUtensorMap& tmV, const
 pa_status tc8_decode_launch(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKs,
                             const CUtensorMap& tmVs, const DecodeParams& prm, pa_dtype io, pa_dtype cache, int grid,
                             cudaStream_t stream);
+// CTAs per SM of the 8-bit kernel for a head group of `group` query heads (1 or 2).
+int tc8_ctas_per_sm(int group);
 }  // namespace pa

@@ -67,7 +67,11 @@ constexpr int q_digit_bytes(int nh) { return (nh / 8) * kNBlock * kDim; }  // q 
 constexpr int stage_bytes(int nh) {
   return (2 * kCodeBytes + q_digit_bytes(nh) + 2 * kScaleBytes + kUnitBytes + 1023) / 1024 * 1024;
 }
-constexpr int stages_for(int nh) { return nh > 8 ? 4 : 5; }
+// Up to 8 query heads per cached head two CTAs share an SM (72 registers a thread): each
+// CTA's per-tile softmax chain is latency-bound, and a second chain per SM runs in its gaps.
+// Two stages each then fit the SM's shared memory.
+constexpr int ctas_per_sm(int nh) { return nh > 8 ? 1 : 2; }
+constexpr int stages_for(int nh) { return nh > 8 ? 4 : 2; }
 constexpr int p_bytes(int nh) { return kTokens * kNBlock * (nh / 8); }  // one weight-digit operand W^T
 constexpr size_t smem_bytes(int nh) {
   return 1024 + static_cast<size_t>(stages_for(nh)) * stage_bytes(nh) + 2 * p_bytes(nh);
@@ -186,7 +190,7 @@ template <> __device__ __forceinline__ void tmem_load_digits<8, 3>(uint32_t col,
 // IO: fp16 or bf16 queries and output; CT: int8_t or __nv_fp8_e4m3 codes; NH: query heads of
 // a row (8 or 16 >= GQ); a softmax thread tracks NH / 2 of them.
 template <typename IO, typename CT, int NH>
-__global__ void __launch_bounds__(base_threads(NH), 1)
+__global__ void __launch_bounds__(base_threads(NH), ctas_per_sm(NH))
 decode_gqa_tc8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmKs, const __grid_constant__ CUtensorMap tmVs,
                       const DecodeParams p) {
@@ -728,6 +732,8 @@ const void* tc8_fn_for(pa_dtype cache) {
 }
 
 }  // namespace
+
+int tc8_ctas_per_sm(int group) { return ctas_per_sm(group <= 8 ? 8 : 16); }
 
 pa_status tc8_decode_launch(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKs,
                             const CUtensorMap& tmVs, const DecodeParams& prm, pa_dtype io, pa_dtype cache, int grid,
