@@ -140,10 +140,12 @@ def test_tensor_core_path_windows_and_long_contexts(cuda_device):
 @pytest.mark.parametrize("gq", [4, 8, 16])
 @pytest.mark.parametrize("bs", [8, 16, 32])
 def test_tensor_core_path_eight_bit_caches(cuda_device, io, dtype, gq, bs):
-    """INT8 / FP8 caches with 4..16 query heads per cached head run on tcgen05: the codes are
-    widened to fp16 / bf16 in shared memory, the per-token K scale multiplies the score row
-    and the V scale the weight.  Unattended rows carry NaN scales.  Parity at 1e-2 against the
-    oracle on the dequantised values, and against the CUDA-core kernel where it applies."""
+    """INT8 / FP8 caches with 4..16 query heads per cached head run on tcgen05 with the codes
+    as the MMA operands (q and the weights as 8-bit digits), the per-token K scale applied to
+    the score row and the V scale folded into the weight; up to 8 query heads per cached head
+    two CTAs share an SM.  Unattended rows carry NaN scales.  Contexts of 0 and 1 token, and a
+    batch with fewer work units than CTAs.  Parity at 1e-2 against the oracle on the
+    dequantised values, and against the CUDA-core kernel where it applies."""
     ctx = [0, 1, 127, 128, 129, 300, 2048, 5, 700]
     case, ref, ioname = _case(gq * 10 + bs, 8 * gq, 8, 128, bs, ctx, dtype, io_name=io)
     _run(case, ref, ioname, TOL["int8"])
