@@ -27,9 +27,9 @@
 // into the weights relative to the tile's largest V scale v_max, and O is scaled back by
 // v_max / 65535 (INT8) or v_max / 256 (FP8) when it is folded into the running output.
 //
-// Roles (one CTA per SM, 14 warps):
-//   warps 0,6-8 TMA producers (K codes, V codes, K scales, V scales), each into a 4- or
-//               5-stage ring; their 128 lanes also hold the head group's q digits (loaded
+// Roles (14 warps; two CTAs per SM with up to 8 query heads per cached head, one with 16):
+//   warps 0,6-8 TMA producers (K codes, V codes, K scales, V scales), each into a 2-stage
+//               (two CTAs per SM) or 4-stage ring; their 128 lanes also hold the head group's q digits (loaded
 //               and split once per segment, the next segment's q rows prefetched) and store
 //               them into each stage with the copies.
 //   warp 1      TMEM owner and MMA issuer; with up to 8 query heads per cached head warp 9
