@@ -160,10 +160,11 @@ pa_status paged_attention_decode_gqa(void* out, const void* q, const void* k_cac
  * per cached head, or more with a divisor in [4, 16] (multi-query attention: the query heads
  * of a cached head are split into sub-groups of that size, each reading the cached head).  Then each 128-token tile of one cached head is two tcgen05 MMAs (scores
  * K.q^T and the weighted sum V^T.p^T, fp32 accumulators in tensor memory) instead of
- * CUDA-core dot products.  8-bit codes are first widened to io_dtype in shared memory
- * (exact); the per-token K scale multiplies the score and the V scale the softmax weight,
- * which the value MMA takes rounded to io_dtype.  0 forces the CUDA-core kernel (same
- * results within the tolerances).  Not thread-safe against concurrent decode calls; set it
+ * CUDA-core dot products.  8-bit codes are the MMA operands as stored (INT8: integer MMAs,
+ * FP8: E4M3 MMAs); q and the softmax weights enter as 8-bit digits (INT8: the two bytes of
+ * a 16-bit fixed-point value; FP8: three E4M3 digits, ~12 significant bits), the per-token
+ * K scale multiplies the score and the V scale is folded into the weight.  0 forces the
+ * CUDA-core kernel (same results within the tolerances).  Not thread-safe against concurrent decode calls; set it
  * once at start-up.
  */
 pa_status pa_decode_use_tensor_cores(int enable);
